@@ -1,0 +1,331 @@
+/*
+ * AVQ-Attention oracle: a plain, slow float64 CPU implementation of the
+ * forward pass of "AVQ-Attention: Adaptive Vector-Quantized Attention".
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library.  It shares no
+ * code with the CUDA path.
+ *
+ * Stage 1 follows Algorithm 1 (VQ Precompute kernel, Sec. 4.2) and Stage 2
+ * follows Algorithm 2 (Flash AVQ-Attention kernel, Sec. 4.3), step by step,
+ * in the order and notation of the paper, with no blocking or reordering
+ * beyond the per-query-block structure the algorithm itself defines.
+ *
+ * Readings taken where the paper leaves a step open:
+ *   - Logits are scaled by `scale` (1/sqrt(d) in every workload); the paper's
+ *     Eq. 1 omits the factor "for clarity" (Sec. 3.1).  Distances use raw keys.
+ *   - Parent ties go to the lowest index (argmin, Alg. 1 step 7).  A child is
+ *     taken only if strictly closer than the running best child (Alg. 1
+ *     step 14) and strictly closer than the parent (Alg. 1 step 16).
+ *   - Top-P ties go to the lower parent index; the selection is listed in
+ *     descending importance (Alg. 2 step 9).
+ *   - Importance uses the parents-only denominator (Alg. 2 step 8 precedes
+ *     step 9; Eq. 7).
+ *   - A partial last query block (N not a multiple of the block) is a block
+ *     with fewer rows that selects independently.
+ *
+ * Layouts (all row-major, contiguous):
+ *   K, V, Q, O   [BH][N][d]            BH = B*H, head h = bh % H
+ *   parents      [H][M0][d]
+ *   children     [H][M0][C][d]         child (m,c) is codeword M0 + m*C + c
+ *   assign       [BH][N]               final code in [0, M0*(1+C))
+ *   vsum         [BH][Mt][d]           Mt = M0*(1+C)  (value sums, Eq. 3)
+ *   counts       [BH][Mt]              key counts n_a (Eq. 3)
+ *   sel          [BH][nblk][P]         nblk = ceil(N/block)
+ *   importance   [BH][nblk][M0]
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double sqdist(const double* a, const double* b, int d) {
+  double s = 0.0;
+  for (int t = 0; t < d; ++t) {
+    double diff = a[t] - b[t];
+    s += diff * diff;
+  }
+  return s;
+}
+
+static double dot(const double* a, const double* b, int d) {
+  double s = 0.0;
+  for (int t = 0; t < d; ++t) s += a[t] * b[t];
+  return s;
+}
+
+/*
+ * Algorithm 1, steps 3-16, for one key: nearest parent (steps 5-7), then the
+ * nearest of that parent's C children (steps 9-15), reassigned only if the
+ * child is strictly closer than the cached parent distance (step 16).
+ * Returns the final code.  The decision distances are written for the
+ * near-tie rule used by the tests:
+ *   dec[0] = best parent distance, dec[1] = second-best parent distance,
+ *   dec[2] = best child distance (INFINITY if C == 0),
+ *   dec[3] = second-best child distance (INFINITY if C < 2).
+ */
+static int32_t assign_one(const double* k, const double* par_h, const double* ch_h,
+                          int d, int M0, int C, double* dec) {
+  /* steps 5-7: d = ||k - c_p||^2 over the M0 parents, a = argmin, d_best = min */
+  int a = 0;
+  double d_best = INFINITY, d_second = INFINITY;
+  for (int m = 0; m < M0; ++m) {
+    double dm = sqdist(k, par_h + (size_t)m * d, d);
+    if (dm < d_best) {
+      d_second = d_best;
+      d_best = dm;
+      a = m;
+    } else if (dm < d_second) {
+      d_second = dm;
+    }
+  }
+  /* steps 9-15: c0 = M0 + a*C, d_child = inf, c* = c0, scan the C children */
+  int32_t c0 = M0 + a * C;
+  double d_child = INFINITY, d_child2 = INFINITY;
+  int32_t c_star = c0;
+  for (int c = 0; c < C; ++c) {
+    const double* cc = ch_h + ((size_t)a * C + c) * d;
+    double dc = sqdist(k, cc, d);
+    if (dc < d_child) { /* step 14: where d_c < d_child */
+      d_child2 = d_child;
+      d_child = dc;
+      c_star = c0 + c;
+    } else if (dc < d_child2) {
+      d_child2 = dc;
+    }
+  }
+  if (dec) {
+    dec[0] = d_best;
+    dec[1] = d_second;
+    dec[2] = d_child;
+    dec[3] = d_child2;
+  }
+  /* step 16: where d_child < d_best the key moves to child c* */
+  if (C > 0 && d_child < d_best) return c_star;
+  return a;
+}
+
+/*
+ * Algorithm 1 (VQ Precompute).  Step 1 zeroes the statistics; every key then
+ * adds its value and a count of one to its parent (step 8) and, if it moved,
+ * also to its child (step 16).  Parents thus hold their whole cluster and
+ * children only the keys that are closer to them than to the parent.
+ * `dec` (nullable) receives 4 decision distances per key, see assign_one.
+ */
+void avq_oracle_quantize(int BH, int H, int N, int d, int M0, int C,
+                         const double* K, const double* V,
+                         const double* parents, const double* children,
+                         int32_t* assign, double* vsum, int64_t* counts,
+                         double* dec) {
+  const int Mt = M0 * (1 + C);
+#pragma omp parallel for schedule(dynamic)
+  for (int bh = 0; bh < BH; ++bh) {
+    const int h = bh % H;
+    const double* par_h = parents + (size_t)h * M0 * d;
+    const double* ch_h = children + (size_t)h * M0 * C * d;
+    double* vs = vsum + (size_t)bh * Mt * d;
+    int64_t* ns = counts + (size_t)bh * Mt;
+    /* step 1: initialise V-bar = 0, n = 0 */
+    memset(vs, 0, sizeof(double) * (size_t)Mt * d);
+    memset(ns, 0, sizeof(int64_t) * (size_t)Mt);
+    for (int j = 0; j < N; ++j) {
+      const double* k = K + ((size_t)bh * N + j) * d;
+      const double* v = V + ((size_t)bh * N + j) * d;
+      double* dj = dec ? dec + ((size_t)bh * N + j) * 4 : NULL;
+      int32_t code = assign_one(k, par_h, ch_h, d, M0, C, dj);
+      int32_t a = code < M0 ? code : (code - M0) / C;
+      /* step 8: V-bar[a] += v; n[a] += 1 */
+      for (int t = 0; t < d; ++t) vs[(size_t)a * d + t] += v[t];
+      ns[a] += 1;
+      /* step 16: masked add to the child */
+      if (code >= M0) {
+        for (int t = 0; t < d; ++t) vs[(size_t)code * d + t] += v[t];
+        ns[code] += 1;
+      }
+      assign[(size_t)bh * N + j] = code;
+    }
+  }
+}
+
+/*
+ * The aggregation of Algorithm 1 (steps 1, 8 and 16) for given final codes:
+ * used to check statistics against assignments made elsewhere.
+ */
+void avq_oracle_aggregate(int BH, int N, int d, int M0, int C,
+                          const int32_t* assign, const double* V,
+                          double* vsum, int64_t* counts) {
+  const int Mt = M0 * (1 + C);
+  for (int bh = 0; bh < BH; ++bh) {
+    double* vs = vsum + (size_t)bh * Mt * d;
+    int64_t* ns = counts + (size_t)bh * Mt;
+    memset(vs, 0, sizeof(double) * (size_t)Mt * d);
+    memset(ns, 0, sizeof(int64_t) * (size_t)Mt);
+    for (int j = 0; j < N; ++j) {
+      int32_t code = assign[(size_t)bh * N + j];
+      int32_t a = code < M0 ? code : (code - M0) / C;
+      const double* v = V + ((size_t)bh * N + j) * d;
+      for (int t = 0; t < d; ++t) vs[(size_t)a * d + t] += v[t];
+      ns[a] += 1;
+      if (code >= M0) {
+        for (int t = 0; t < d; ++t) vs[(size_t)code * d + t] += v[t];
+        ns[code] += 1;
+      }
+    }
+  }
+}
+
+/*
+ * Top-P of the importance vector w[0..M0): the P largest entries in
+ * descending order, ties to the lower index (Alg. 2 step 9).
+ */
+static void top_p(const double* w, int M0, int P, int32_t* out) {
+  char* taken = (char*)calloc((size_t)M0, 1);
+  for (int r = 0; r < P; ++r) {
+    int best = -1;
+    for (int j = 0; j < M0; ++j) {
+      if (taken[j]) continue;
+      if (best < 0 || w[j] > w[best]) best = j; /* strict: equal keeps lower index */
+    }
+    taken[best] = 1;
+    out[r] = best;
+  }
+  free(taken);
+}
+
+/*
+ * Algorithm 2 (Flash AVQ-Attention) for one query block I = [i0, i1) of one
+ * head.  Steps 2-8: coarse pass over the M0 parents with the masked running
+ * max (Eq. 18), count-weighted denominator (Eq. 6) and importance (Eq. 7).
+ * Step 9: top-P.  Steps 10-19: for each selected parent, child logits, online
+ * max merge, parent logit recovered as the mean of the child logits (Eq. 8),
+ * correcting attention dA = exp(S_ic) - exp(S_ip) (Eq. 9) masked for empty
+ * children, and the accumulator update.  Step 20: Y = x / z.
+ */
+static void attend_block(int d, int M0, int C, int P, double scale,
+                         const double* Q, int i0, int i1,
+                         const double* par_h, const double* ch_h,
+                         const double* vs, const double* ns,
+                         const int32_t* sel_in, double* O, int32_t* sel_out,
+                         double* imp_out) {
+  const int nI = i1 - i0;
+  double* s = (double*)malloc(sizeof(double) * (size_t)nI * M0);
+  double* A = (double*)malloc(sizeof(double) * (size_t)nI * M0);
+  double* m = (double*)malloc(sizeof(double) * (size_t)nI);
+  double* x = (double*)malloc(sizeof(double) * (size_t)nI * d);
+  double* z = (double*)malloc(sizeof(double) * (size_t)nI);
+  double* w = (double*)malloc(sizeof(double) * (size_t)M0);
+  int32_t* S = (int32_t*)malloc(sizeof(int32_t) * (size_t)(P > 0 ? P : 1));
+  double* sc = (double*)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1));
+
+  for (int r = 0; r < nI; ++r) {
+    const double* q = Q + (size_t)(i0 + r) * d;
+    /* step 4: s = q c^T over the parents */
+    for (int j = 0; j < M0; ++j) s[(size_t)r * M0 + j] = scale * dot(q, par_h + (size_t)j * d, d);
+    /* step 5: m = max over j with n_j > 0 */
+    m[r] = -INFINITY;
+    for (int j = 0; j < M0; ++j)
+      if (ns[j] > 0 && s[(size_t)r * M0 + j] > m[r]) m[r] = s[(size_t)r * M0 + j];
+    /* step 6: A = exp(s - m), A_j = 0 where n_j = 0 */
+    for (int j = 0; j < M0; ++j)
+      A[(size_t)r * M0 + j] = ns[j] > 0 ? exp(s[(size_t)r * M0 + j] - m[r]) : 0.0;
+    /* step 7: x = A v-bar, z = sum_j A_j n_j */
+    for (int t = 0; t < d; ++t) x[(size_t)r * d + t] = 0.0;
+    z[r] = 0.0;
+    for (int j = 0; j < M0; ++j) {
+      double a = A[(size_t)r * M0 + j];
+      for (int t = 0; t < d; ++t) x[(size_t)r * d + t] += a * vs[(size_t)j * d + t];
+      z[r] += a * ns[j];
+    }
+  }
+  /* step 8: w_j = sum_i A_ij n_j / z_i  (Eq. 7) */
+  for (int j = 0; j < M0; ++j) {
+    w[j] = 0.0;
+    for (int r = 0; r < nI; ++r) w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];
+  }
+  if (imp_out) memcpy(imp_out, w, sizeof(double) * (size_t)M0);
+  /* step 9: S = top-P(w), or the caller's selection */
+  if (P > 0) {
+    if (sel_in) memcpy(S, sel_in, sizeof(int32_t) * (size_t)P);
+    else top_p(w, M0, P, S);
+    if (sel_out) memcpy(sel_out, S, sizeof(int32_t) * (size_t)P);
+  }
+  /* steps 10-19: child refinement (no-op when C == 0) */
+  if (C > 0) {
+    for (int r = 0; r < nI; ++r) {
+      const double* q = Q + (size_t)(i0 + r) * d;
+      for (int k = 0; k < P; ++k) {
+        int p = S[k];
+        const double* ch_p = ch_h + (size_t)p * C * d;
+        const double* vc = vs + (size_t)(M0 + p * C) * d;
+        const double* nc = ns + (M0 + p * C);
+        /* step 12: s_c = q c_c^T */
+        for (int c = 0; c < C; ++c) sc[c] = scale * dot(q, ch_p + (size_t)c * d, d);
+        /* step 13: m' = max(m, max over c with n_c > 0 of s_c) */
+        double mp = m[r];
+        for (int c = 0; c < C; ++c)
+          if (nc[c] > 0 && sc[c] > mp) mp = sc[c];
+        /* step 14: rescale the accumulators to m' */
+        double f = exp(m[r] - mp);
+        for (int t = 0; t < d; ++t) x[(size_t)r * d + t] *= f;
+        z[r] *= f;
+        m[r] = mp;
+        /* step 15: s_p = (1/C) sum_c s_c   (Eq. 8) */
+        double sp = 0.0;
+        for (int c = 0; c < C; ++c) sp += sc[c];
+        sp /= C;
+        /* steps 16-18: dA = exp(s_c - m) - exp(s_p - m), zero where n_c = 0 */
+        double Ap = exp(sp - m[r]);
+        for (int c = 0; c < C; ++c) {
+          double dA = nc[c] > 0 ? exp(sc[c] - m[r]) - Ap : 0.0;
+          for (int t = 0; t < d; ++t) x[(size_t)r * d + t] += dA * vc[(size_t)c * d + t];
+          z[r] += dA * nc[c];
+        }
+      }
+    }
+  }
+  /* step 20: Y = x / z */
+  for (int r = 0; r < nI; ++r)
+    for (int t = 0; t < d; ++t) O[(size_t)(i0 + r) * d + t] = x[(size_t)r * d + t] / z[r];
+
+  free(s); free(A); free(m); free(x); free(z); free(w); free(S); free(sc);
+}
+
+/*
+ * Algorithm 2 over every (bh, query block), or over the listed ones only
+ * (`blocks` holds nlist pairs (bh, block index); nullable = all).  `counts`
+ * are passed as doubles.  `sel_in` (nullable) overrides the top-P selection:
+ * [BH][nblk][P].  O rows of unlisted blocks are left untouched.
+ */
+void avq_oracle_attention(int BH, int H, int N, int d, int M0, int C, int P, int block,
+                          double scale, const double* Q,
+                          const double* parents, const double* children,
+                          const double* vsum, const double* counts,
+                          const int32_t* sel_in, const int32_t* blocks, int nlist,
+                          double* O, int32_t* sel_out, double* imp_out) {
+  const int Mt = M0 * (1 + C);
+  const int nblk = (N + block - 1) / block;
+  const int total = blocks ? nlist : BH * nblk;
+#pragma omp parallel for schedule(dynamic)
+  for (int u = 0; u < total; ++u) {
+    int bh = blocks ? blocks[2 * u] : u / nblk;
+    int b = blocks ? blocks[2 * u + 1] : u % nblk;
+    int h = bh % H;
+    int i0 = b * block;
+    int i1 = i0 + block < N ? i0 + block : N;
+    size_t sb = (size_t)bh * nblk + b;
+    attend_block(d, M0, C, P, scale, Q + (size_t)bh * N * d, i0, i1,
+                 parents + (size_t)h * M0 * d, children + (size_t)h * M0 * C * d,
+                 vsum + (size_t)bh * Mt * d, counts + (size_t)bh * Mt,
+                 sel_in ? sel_in + sb * P : NULL, O + (size_t)bh * N * d,
+                 sel_out ? sel_out + sb * P : NULL, imp_out ? imp_out + sb * M0 : NULL);
+  }
+}
+
+int avq_oracle_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

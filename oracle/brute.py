@@ -1,0 +1,155 @@
+"""Independent closed forms that pin the oracle (test infrastructure only).
+
+Written separately from `avq_oracle.c` and vectorised with numpy, so that a
+mistake in the step-by-step oracle shows up as a disagreement here.
+
+- `assign_brute`: nearest parent, then nearest child of that parent, moved
+  only when strictly closer (Sec. 4.2; Alg. 1), by full distance tables.
+- `aggregate_brute`: value sums and counts of Eq. 3 for a two-level tree.
+- `representative_attention`: the identity behind the correcting attention
+  (Sec. C, Eqs. 15-17): AVQ output equals exact softmax attention over keys
+  that are each replaced by a representative -- the child when the key moved
+  to a child whose parent is selected for the query's block, else the parent.
+- `flat_vq_attention`: VQ attention over a fixed codebook (Eq. 4).
+- `exact_attention`: softmax attention (Eq. 1), logits scaled by `scale`.
+- `importance_brute`: Eq. 7 written as a block sum of the flat-VQ softmax
+  mass of each parent, n_j exp(s_ij) / sum_l n_l exp(s_il).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(a):
+    if hasattr(a, "detach"):
+        import torch
+
+        a = a.detach().to("cpu").to(torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def assign_brute(K, parents, children):
+    """Final codes [B,H,N] from full distance tables."""
+    K, parents, children = _f64(K), _f64(parents), _f64(children)
+    B, H, N, d = K.shape
+    M0 = parents.shape[1]
+    C = children.shape[2]
+    codes = np.empty((B, H, N), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            k = K[b, h]
+            dp = ((k[:, None, :] - parents[h][None, :, :]) ** 2).sum(-1)  # [N, M0]
+            a = dp.argmin(axis=1)  # first minimum
+            best = dp[np.arange(N), a]
+            if C == 0:
+                codes[b, h] = a
+                continue
+            ch = children[h][a]  # [N, C, d]
+            dc = ((k[:, None, :] - ch) ** 2).sum(-1)  # [N, C]
+            c = dc.argmin(axis=1)
+            move = dc[np.arange(N), c] < best
+            codes[b, h] = np.where(move, M0 + a * C + c, a)
+    return codes
+
+
+def aggregate_brute(codes, V, M0, C):
+    """V-bar [B,H,Mt,d] and n [B,H,Mt]: every key counts for its parent, and
+    for its child when it moved to one."""
+    V = _f64(V)
+    codes = np.asarray(codes)
+    B, H, N, d = V.shape
+    Mt = M0 * (1 + C)
+    vs = np.zeros((B, H, Mt, d))
+    ns = np.zeros((B, H, Mt), dtype=np.int64)
+    parent = np.where(codes < M0, codes, (codes - M0) // max(C, 1))
+    for b in range(B):
+        for h in range(H):
+            np.add.at(vs[b, h], parent[b, h], V[b, h])
+            np.add.at(ns[b, h], parent[b, h], 1)
+            mv = codes[b, h] >= M0
+            np.add.at(vs[b, h], codes[b, h][mv], V[b, h][mv])
+            np.add.at(ns[b, h], codes[b, h][mv], 1)
+    return vs, ns
+
+
+def _softmax_rows(logits):
+    mx = logits.max(axis=-1, keepdims=True)
+    e = np.exp(logits - mx)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def representative_attention(Q, K_codes, V, parents, children, sel, block, scale):
+    """Exact softmax attention over representative keys (Sec. C identity)."""
+    Q, V, parents, children = _f64(Q), _f64(V), _f64(parents), _f64(children)
+    codes = np.asarray(K_codes)
+    B, H, N, d = Q.shape
+    M0 = parents.shape[1]
+    C = children.shape[2]
+    sel = np.asarray(sel)
+    Y = np.empty_like(Q)
+    nblk = (N + block - 1) // block
+    for b in range(B):
+        for h in range(H):
+            c = codes[b, h]
+            par = np.where(c < M0, c, (c - M0) // max(C, 1))
+            parent_vec = parents[h][par]  # [N, d]
+            if C > 0:
+                flat_children = children[h].reshape(M0 * C, d)
+                child_vec = flat_children[np.clip(c - M0, 0, M0 * C - 1)]
+            for blk in range(nblk):
+                i0, i1 = blk * block, min(N, (blk + 1) * block)
+                rep = parent_vec.copy()
+                if C > 0 and sel.shape[-1] > 0:
+                    chosen = np.zeros(M0, dtype=bool)
+                    chosen[sel[b, h, blk]] = True
+                    use_child = (c >= M0) & chosen[par]
+                    rep[use_child] = child_vec[use_child]
+                logits = scale * Q[b, h, i0:i1] @ rep.T  # [nI, N]
+                Y[b, h, i0:i1] = _softmax_rows(logits) @ V[b, h]
+    return Y
+
+
+def flat_vq_attention(Q, codebook, vsum, counts, scale):
+    """Eq. 4: sum_a exp(q c_a) V-bar_a / sum_a exp(q c_a) n_a over one codebook
+    per head (codebook [H,M,d], vsum [B,H,M,d], counts [B,H,M])."""
+    Q, codebook, vsum, counts = _f64(Q), _f64(codebook), _f64(vsum), _f64(counts)
+    B, H, N, d = Q.shape
+    Y = np.empty_like(Q)
+    for b in range(B):
+        for h in range(H):
+            s = scale * Q[b, h] @ codebook[h].T  # [N, M]
+            live = counts[b, h] > 0
+            s = np.where(live[None, :], s, -np.inf)
+            mx = s.max(axis=1, keepdims=True)
+            e = np.where(live[None, :], np.exp(s - mx), 0.0)
+            Y[b, h] = (e @ vsum[b, h]) / (e @ counts[b, h])[:, None]
+    return Y
+
+
+def exact_attention(Q, K, V, scale):
+    """Eq. 1 with scaled logits."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    B, H, N, d = Q.shape
+    Y = np.empty_like(Q)
+    for b in range(B):
+        for h in range(H):
+            Y[b, h] = _softmax_rows(scale * Q[b, h] @ K[b, h].T) @ V[b, h]
+    return Y
+
+
+def importance_brute(Q, parents, counts, block, scale):
+    """w_j(I) = sum_{i in I} n_j exp(s_ij) / sum_l n_l exp(s_il)  [B,H,nblk,M0]."""
+    Q, parents, counts = _f64(Q), _f64(parents), _f64(counts)
+    B, H, N, d = Q.shape
+    M0 = parents.shape[1]
+    nblk = (N + block - 1) // block
+    W = np.zeros((B, H, nblk, M0))
+    for b in range(B):
+        for h in range(H):
+            n = counts[b, h][:M0]
+            with np.errstate(divide="ignore"):
+                logn = np.where(n > 0, np.log(np.where(n > 0, n, 1.0)), -np.inf)
+            mass = _softmax_rows(scale * Q[b, h] @ parents[h].T + logn[None, :])  # [N, M0]
+            for blk in range(nblk):
+                W[b, h, blk] = mass[blk * block:(blk + 1) * block].sum(axis=0)
+    return W

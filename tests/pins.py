@@ -1,0 +1,358 @@
+"""Pins of the oracle: checks against what the paper and the mathematics fix.
+
+Each `pin_*` takes an `oracle.Oracle` and raises AssertionError on a
+mismatch.  They are run against the real oracle (test_oracle_pins.py) and
+against deliberately broken copies of it (test_oracle_mutations.py), to show
+that a plausible mistake anywhere in the oracle fails at least one of them.
+References are to "AVQ-Attention: Adaptive Vector-Quantized Attention".
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+from adaptive_vector_quantized_b200 import synth
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.max(np.abs(a - b)) / max(1e-300, np.max(np.abs(b))))
+
+
+# small seeded cases (sizes that finish in well under a second) --------------
+def case_tiny():
+    return synth.make_inputs(synth.get_config("tiny"), 11)
+
+
+def case_regions():
+    cfg = dict(dtype="bf16", B=1, H=2, N=1024, d=64, M0=16, C=8, P=4, block=128,
+               keys="regions", side=32, key_sigma=0.1, noise=0.1, order="hilbert",
+               sigma_c=0.3)
+    return synth.make_inputs(cfg, 12)
+
+
+def case_wide():
+    cfg = dict(dtype="bf16", B=1, H=1, N=300, d=128, M0=32, C=8, P=8, block=64,
+               keys="tree", key_sigma=0.1, sigma_c=0.3)
+    return synth.make_inputs(cfg, 13)
+
+
+CASES = (case_tiny, case_regions, case_wide)
+
+
+def _run(orc, inp, P=None, block=None, sel=None):
+    P = inp["P"] if P is None else P
+    block = inp["block"] if block is None else block
+    assign, vsum, counts, dec = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+    O, s, imp = orc.attention(inp["Q"], inp["parents"], inp["children"], vsum, counts,
+                              P, block, inp["scale"], sel=sel)
+    return assign, vsum, counts, O, s, imp
+
+
+# ---------------------------------------------------------------------------
+def pin_hand_worked(orc):
+    """Hand-derived d=2 example (Alg. 1, Alg. 2, Eqs. 7-9, Eq. 18)."""
+    g = json.load(open(os.path.join(GOLDEN, "hand_worked_d2.json")))
+    par = np.array(g["parents"])[None]
+    ch = np.array(g["children"])[None]
+    K = np.array(g["keys"])[None, None]
+    V = np.array(g["values"])[None, None]
+    Q = np.array(g["queries"])[None, None]
+    env = {"v0": V[0, 0, 0], "v1": V[0, 0, 1], "v2": V[0, 0, 2], "exp": math.exp}
+    ev = lambda s: np.asarray(eval(s, {"__builtins__": {}}, env), dtype=np.float64)  # noqa: E731
+    exp = g["expected"]
+    assign, vsum, counts, _ = orc.quantize(K, V, par, ch)
+    assert assign[0, 0].tolist() == exp["codes"], assign
+    assert counts[0, 0].tolist() == exp["counts"], counts
+    for row, expr in exp["vsum"].items():
+        assert _rel(vsum[0, 0, int(row)], ev(expr) + 0.0) < 1e-15 or np.all(ev(expr) == vsum[0, 0, int(row)])
+    O, sel, imp = orc.attention(Q, par, ch, vsum, counts, 1, 1, g["scale"])
+    for i, expr in enumerate(exp["Y_P1"]):
+        assert _rel(O[0, 0, i], ev(expr)) < 1e-13, (i, O[0, 0, i], ev(expr))
+    assert sel[0, 0].tolist() == exp["sel_P1_block1"]
+    O3, sel3, imp3 = orc.attention(Q, par, ch, vsum, counts, 1, 3, g["scale"])
+    for j, expr in enumerate(exp["importance_block3"]):
+        assert abs(imp3[0, 0, 0, j] - float(ev(expr))) < 1e-13
+    assert _rel(O3[0, 0], O[0, 0]) < 1e-13
+    O0, _, _ = orc.attention(Q, par, ch, vsum, counts, 0, 1, g["scale"])
+    for i, expr in enumerate(exp["Y_P0"]):
+        assert _rel(O0[0, 0, i], ev(expr)) < 1e-13, (i, O0[0, 0, i], ev(expr))
+
+
+def pin_assign_brute(orc):
+    """Alg. 1 codes equal a vectorised full-distance-table assignment."""
+    for mk in CASES:
+        inp = mk()
+        assign, _, _, _ = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+        ref = brute.assign_brute(inp["K"], inp["parents"], inp["children"])
+        assert (assign == ref).all(), (mk.__name__, int((assign != ref).sum()))
+
+
+def pin_aggregate(orc):
+    """Eq. 3 statistics of the two-level tree, plus their invariants."""
+    for mk in CASES:
+        inp = mk()
+        M0, C, N = inp["M0"], inp["C"], inp["N"]
+        assign, vsum, counts, _ = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+        vs_ref, ns_ref = brute.aggregate_brute(assign, inp["V"], M0, C)
+        assert (counts == ns_ref).all()
+        assert _rel(vsum, vs_ref) < 1e-12
+        V = brute._f64(inp["V"])
+        # every key counts once at the parent level: sum_p n_p = N, sum_p Vbar_p = sum_j V_j
+        assert (counts[..., :M0].sum(-1) == N).all()
+        assert _rel(vsum[..., :M0, :].sum(-2), V.sum(-2)) < 1e-10
+        # children hold a subset of their parent's keys (Eq. 15: n_stay >= 0)
+        if C > 0:
+            ch_counts = counts[..., M0:].reshape(*counts.shape[:-1], M0, C).sum(-1)
+            assert (ch_counts <= counts[..., :M0]).all()
+            moved = assign >= M0
+            assert (counts[..., M0:].sum(-1) == moved.sum(-1)).all()
+
+
+def pin_representative(orc):
+    """Sec. C identity: AVQ output equals exact softmax attention over the
+    representative keys, for several P including P = M0."""
+    for mk in CASES:
+        inp = mk()
+        for P in sorted({1, inp["P"], inp["M0"]}):
+            assign, vsum, counts, O, sel, _ = _run(orc, inp, P=P)
+            Y = brute.representative_attention(inp["Q"], assign, inp["V"], inp["parents"],
+                                               inp["children"], sel, inp["block"], inp["scale"])
+            assert _rel(O, Y) < 1e-10, (mk.__name__, P, _rel(O, Y))
+
+
+def pin_rescale_exercised(orc):
+    """The representative check above covers the online-max merge (Alg. 2
+    steps 13-14) only if some selected non-empty child logit exceeds the
+    parent max; make sure the regions case has such rows."""
+    inp = case_regions()
+    assign, vsum, counts, O, sel, _ = _run(orc, inp)
+    Q = brute._f64(inp["Q"])
+    par = brute._f64(inp["parents"])
+    ch = brute._f64(inp["children"])
+    M0, C, blk = inp["M0"], inp["C"], inp["block"]
+    found = 0
+    for h in range(inp["H"]):
+        s = inp["scale"] * Q[0, h] @ par[h].T
+        live = counts[0, h, :M0] > 0
+        m = np.where(live[None], s, -np.inf).max(1)
+        for b in range(sel.shape[2]):
+            for p in sel[0, h, b]:
+                sc = inp["scale"] * Q[0, h, b * blk:(b + 1) * blk] @ ch[h, p].T
+                nz = counts[0, h, M0 + p * C: M0 + (p + 1) * C] > 0
+                found += int((np.where(nz[None], sc, -np.inf) > m[b * blk:(b + 1) * blk, None]).any())
+    assert found > 0
+    Y = brute.representative_attention(inp["Q"], assign, inp["V"], inp["parents"],
+                                       inp["children"], sel, blk, inp["scale"])
+    assert _rel(O, Y) < 1e-10
+
+
+def pin_flat_p0(orc):
+    """P = 0 is fixed-codebook VQ attention over the parents (Eq. 4); C = 0
+    (a flat codebook) is the same for any P."""
+    inp = case_regions()
+    assign, vsum, counts, O, _, _ = _run(orc, inp, P=0)
+    M0 = inp["M0"]
+    Y = brute.flat_vq_attention(inp["Q"], inp["parents"], vsum[..., :M0, :], counts[..., :M0],
+                                inp["scale"])
+    assert _rel(O, Y) < 1e-10
+    cfg = dict(dtype="bf16", B=1, H=1, N=700, d=64, M0=48, C=0, P=5, block=64,
+               keys="tree", key_sigma=0.1)
+    flat = synth.make_inputs(cfg, 21)
+    assign, vsum, counts, O, _, _ = _run(orc, flat)
+    assert (assign < 48).all()
+    Y = brute.flat_vq_attention(flat["Q"], flat["parents"], vsum, counts, flat["scale"])
+    assert _rel(O, Y) < 1e-10
+
+
+def _exact_codebook_case(rng, on_children: bool):
+    H, M0, C, d, N = 1, 12, 4, 8, 240
+    par, ch = synth.make_codebook(rng, H, M0, C, d, sigma_c=0.1)
+    par = par / 64.0
+    ch = ch / 64.0
+    if on_children:
+        p = rng.integers(0, M0, N)
+        c = rng.integers(0, C, N)
+        K = ch[0][p, c]
+    else:
+        K = par[0][rng.integers(0, M0, N)]
+    Q = rng.standard_normal((1, H, N, d))
+    V = rng.standard_normal((1, H, N, d))
+    return Q, K[None, None], V, par, ch
+
+
+def pin_exact_codebook(orc):
+    """A codebook holding every distinct key reproduces exact attention (Eq. 1):
+    keys on the parents give exact attention for any P; keys on the children
+    give it for P = M0."""
+    rng = np.random.default_rng(31)
+    Q, K, V, par, ch = _exact_codebook_case(rng, on_children=False)
+    Y = brute.exact_attention(Q, K, V, 0.5)
+    for P in (0, 3, 12):
+        assign, vsum, counts, _ = orc.quantize(K, V, par, ch)
+        assert (assign < 12).all()
+        O, _, _ = orc.attention(Q, par, ch, vsum, counts, P, 32, 0.5)
+        assert _rel(O, Y) < 1e-10, (P, _rel(O, Y))
+    Q, K, V, par, ch = _exact_codebook_case(rng, on_children=True)
+    assign, vsum, counts, _ = orc.quantize(K, V, par, ch)
+    assert (assign >= 12).all()
+    O, _, _ = orc.attention(Q, par, ch, vsum, counts, 12, 32, 0.5)
+    assert _rel(O, brute.exact_attention(Q, K, V, 0.5)) < 1e-10
+
+
+def pin_importance(orc):
+    """Eq. 7 equals the block sum of each parent's flat-VQ softmax mass, and
+    sums to the block size."""
+    for mk in CASES:
+        inp = mk()
+        assign, vsum, counts, O, sel, imp = _run(orc, inp)
+        W = brute.importance_brute(inp["Q"], inp["parents"], counts, inp["block"], inp["scale"])
+        assert _rel(imp, W) < 1e-12
+        N, blk = inp["N"], inp["block"]
+        sizes = np.array([min(blk, N - b * blk) for b in range(imp.shape[2])], dtype=np.float64)
+        assert np.allclose(imp.sum(-1), sizes[None, None, :], rtol=1e-12)
+
+
+def _topp_ref(w, P):
+    order = np.lexsort((np.arange(w.shape[-1]), -w))  # descending, ties to lower index
+    return order[:P]
+
+
+def pin_topp(orc):
+    """Top-P: the P largest importances, descending, ties to the lower index."""
+    for mk in CASES:
+        inp = mk()
+        _, _, _, _, sel, imp = _run(orc, inp)
+        for idx in np.ndindex(*sel.shape[:3]):
+            assert sel[idx].tolist() == _topp_ref(imp[idx], inp["P"]).tolist()
+    # exact ties: zero queries make every logit 0; equal counts make every w equal
+    M0, C, d = 8, 2, 4
+    rng = np.random.default_rng(41)
+    par, ch = synth.make_codebook(rng, 1, M0, C, d)
+    par, ch = par / 64.0, ch / 64.0
+    K = np.repeat(par[0], 4, axis=0)[None, None]
+    V = rng.standard_normal(K.shape)
+    Q = np.zeros_like(K)
+    assign, vsum, counts, _ = orc.quantize(K, V, par, ch)
+    _, sel, imp = orc.attention(Q, par, ch, vsum, counts, 3, 32, 1.0)
+    assert np.all(imp[0, 0, 0] == imp[0, 0, 0, 0])
+    assert sel[0, 0, 0].tolist() == [0, 1, 2]
+
+
+def pin_relabel(orc):
+    """Relabelling parents (with their child runs) permutes the selection and
+    leaves the output unchanged."""
+    inp = case_tiny()
+    M0, C = inp["M0"], inp["C"]
+    assign, vsum, counts, O, sel, imp = _run(orc, inp)
+    perm = np.random.default_rng(51).permutation(M0)
+    inv = np.argsort(perm)
+    par2 = inp["parents"][:, perm]
+    ch2 = inp["children"][:, perm]
+    assign2, vsum2, counts2, O2, sel2, imp2 = _run(orc, dict(inp, parents=par2, children=ch2))
+    assert _rel(O2, O) < 1e-12
+    for idx in np.ndindex(*sel.shape[:3]):
+        w = np.sort(imp[idx])[::-1]
+        if abs(w[inp["P"] - 1] - w[inp["P"]]) <= 1e-9 * w[inp["P"] - 1]:
+            continue
+        assert sorted(perm[sel2[idx]].tolist()) == sorted(sel[idx].tolist())
+    par_code = np.where(assign < M0, assign, (assign - M0) // C)
+    par_code2 = np.where(assign2 < M0, assign2, (assign2 - M0) // C)
+    assert (perm[par_code2] == par_code).all()
+    assert (counts2[..., :M0] == counts[..., :M0][..., perm]).all()
+    assert (inv[perm] == np.arange(M0)).all()
+
+
+def pin_key_permutation(orc):
+    """Counts and sums do not depend on the order of the keys; codes move with them."""
+    inp = case_regions()
+    assign, vsum, counts, _ = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+    perm = np.random.default_rng(61).permutation(inp["N"])
+    assign2, vsum2, counts2, _ = orc.quantize(inp["K"][:, :, perm], inp["V"][:, :, perm],
+                                              inp["parents"], inp["children"])
+    assert (assign2 == assign[:, :, perm]).all()
+    assert (counts2 == counts).all()
+    assert _rel(vsum2, vsum) < 1e-12
+
+
+def pin_keys_on_codewords(orc):
+    """A key placed exactly on a codeword is assigned to it."""
+    inp = case_tiny()
+    M0, C = inp["M0"], inp["C"]
+    par = brute._f64(inp["parents"])
+    ch = brute._f64(inp["children"])
+    codes = np.arange(M0 * (1 + C))
+    K = np.concatenate([par[0], ch[0].reshape(M0 * C, -1)])[None, None]
+    V = np.zeros_like(K)
+    assign, _, _, _ = orc.quantize(K, V, par, ch)
+    assert (assign[0, 0] == codes).all()
+
+
+def pin_strict_ties(orc):
+    """Ties: equal parents -> lower index (argmin); a child must be strictly
+    closer than the best child so far (first child wins, Alg. 1 step 14) and
+    strictly closer than the parent (step 16)."""
+    par = np.array([[[0.0, 0.0], [10.0, 10.0]]])
+    ch = np.array([[[[1, 1], [1, -1], [-1, 1], [-1, -1]],
+                    [[11, 11], [11, 9], [9, 11], [9, 9]]]], dtype=np.float64)
+    K = np.array([[1.0, 0.0],    # parent 0 at 1, children 0 and 1 at 1: stays
+                  [1.2, 0.0],    # children 0 and 1 tie at 1.04 < 1.44: child 0 -> code 2
+                  [5.0, 5.0],    # both parents at 50: lower index; children of 0 at 32 -> code 2
+                  [0.0, 0.0],    # on parent 0
+                  [-1.2, 0.0]])  # children 2 and 3 tie: child 2 -> code 4
+    K = K[None, None]
+    V = np.ones_like(K)
+    assign, _, _, _ = orc.quantize(K, V, par, ch)
+    assert assign[0, 0].tolist() == [0, 2, 2, 0, 4], assign
+
+
+def pin_masking(orc):
+    """Eq. 18 and Sec. D: an empty child or parent with a huge logit neither
+    sets the running max nor produces inf*0; the output is still the
+    representative-key attention."""
+    par = np.array([[[0.0, 0.0], [-60.0, 0.0], [50.0, 0.0]]])
+    ch = np.array([[[[30.0, 0.0], [-30.0, 0.0]],
+                    [[-61.0, 0.0], [-59.0, 0.0]],
+                    [[49.0, 0.0], [51.0, 0.0]]]])
+    rng = np.random.default_rng(71)
+    stay = np.stack([rng.uniform(-0.5, 0.5, 6), rng.uniform(-0.5, 0.5, 6)], 1)
+    moved = np.array([[-29.9, 0.0], [-29.95, 0.1]])
+    far = np.array([[-60.0, 0.2], [-60.1, 0.0]])
+    K = np.concatenate([stay, moved, far])[None, None]
+    N = K.shape[2]
+    V = rng.standard_normal((1, 1, N, 2))
+    Q = np.tile(np.array([40.0, 0.0]), (N, 1))[None, None]
+    assign, vsum, counts, _ = orc.quantize(K, V, par, ch)
+    assert counts[0, 0, 2] == 0 and counts[0, 0, 3] == 0, counts  # parent 2 and child (0,0) empty
+    assert counts[0, 0, 4] == 2
+    O, sel, _ = orc.attention(Q, par, ch, vsum, counts, 1, N, 1.0)
+    assert sel[0, 0, 0].tolist() == [0]
+    assert np.isfinite(O).all()
+    Y = brute.representative_attention(Q, assign, V, par, ch, sel, N, 1.0)
+    assert _rel(O, Y) < 1e-12
+
+
+def pin_counting(orc):
+    """Codebook size and per-block code count of the paper's configurations."""
+    g = json.load(open(os.path.join(GOLDEN, "counting.json")))
+    for row in g["mtotal"]:
+        assert synth.m_total(row["M0"], row["C"]) == row["Mtotal"]
+    for row in g["codes_per_query"]:
+        assert row["M0"] + row["P"] * row["C"] == row["codes"]
+    # the oracle's statistics are laid out over the same M0*(1+C) codes
+    inp = case_tiny()
+    _, vsum, counts, _ = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+    assert counts.shape[-1] == synth.m_total(inp["M0"], inp["C"])
+
+
+ALL_PINS = [pin_hand_worked, pin_assign_brute, pin_aggregate, pin_representative,
+            pin_rescale_exercised, pin_flat_p0, pin_exact_codebook, pin_importance, pin_topp,
+            pin_relabel, pin_key_permutation, pin_keys_on_codewords, pin_strict_ties,
+            pin_masking, pin_counting]

@@ -1,0 +1,58 @@
+"""Plant plausible mistakes in a copy of the oracle and check the pins catch
+each one (CPU only).  The mistakes are planted in a temporary copy of the C
+source; the committed oracle is never modified."""
+import os
+import tempfile
+
+import pytest
+
+import oracle
+from tests import pins
+
+# (name, exact text in avq_oracle.c, replacement)
+MUTANTS = [
+    ("child-not-strict-vs-parent", "if (C > 0 && d_child < d_best) return c_star;",
+     "if (C > 0 && d_child <= d_best) return c_star;"),
+    ("child-tie-to-last", "if (dc < d_child) { /* step 14", "if (dc <= d_child) { /* step 14"),
+    ("parent-tie-to-last", "if (dm < d_best) {", "if (dm <= d_best) {"),
+    ("child-count-dropped", "ns[code] += 1;\n      }\n      assign", "\n      }\n      assign"),
+    ("child-index-transposed", "ch_h + ((size_t)a * C + c) * d", "ch_h + ((size_t)c * M0 + a) * d"),
+    ("dA-sign", "exp(sc[c] - m[r]) - Ap", "Ap - exp(sc[c] - m[r])"),
+    ("no-rescale", "double f = exp(m[r] - mp);", "double f = 1.0;"),
+    ("max-includes-empty-child", "if (nc[c] > 0 && sc[c] > mp) mp = sc[c];", "if (sc[c] > mp) mp = sc[c];"),
+    ("dA-not-masked", "double dA = nc[c] > 0 ? exp(sc[c] - m[r]) - Ap : 0.0;",
+     "double dA = exp(sc[c] - m[r]) - Ap;"),
+    ("A-not-masked", "ns[j] > 0 ? exp(s[(size_t)r * M0 + j] - m[r]) : 0.0;",
+     "exp(s[(size_t)r * M0 + j] - m[r]);"),
+    ("importance-no-denominator", "w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];",
+     "w[j] += A[(size_t)r * M0 + j] * ns[j];"),
+    ("importance-no-count", "w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];",
+     "w[j] += A[(size_t)r * M0 + j] / z[r];"),
+    ("topp-tie-to-higher", "if (best < 0 || w[j] > w[best]) best = j;",
+     "if (best < 0 || w[j] >= w[best]) best = j;"),
+    ("child-logit-unscaled", "sc[c] = scale * dot(q, ch_p + (size_t)c * d, d);",
+     "sc[c] = dot(q, ch_p + (size_t)c * d, d);"),
+    ("parent-mean-wrong-divisor", "sp /= C;", "sp /= (C + 1);"),
+    ("z-missing-count", "z[r] += a * ns[j];", "z[r] += a;"),
+    ("child-z-missing-count", "z[r] += dA * nc[c];", "z[r] += dA;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, old, new):
+    src = open(oracle.SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique or missing: {name}"
+    with tempfile.TemporaryDirectory() as tmp:
+        msrc = os.path.join(tmp, "mutant.c")
+        with open(msrc, "w") as f:
+            f.write(src.replace(old, new))
+        lib = oracle.build(src=msrc, out=os.path.join(tmp, "libmutant.so"), force=True)
+        orc = oracle.Oracle(lib)
+        caught = []
+        for pin in pins.ALL_PINS:
+            try:
+                with __import__("numpy").errstate(all="ignore"):
+                    pin(orc)
+            except (AssertionError, ValueError, IndexError, FloatingPointError) as e:  # noqa: PERF203
+                caught.append((pin.__name__, type(e).__name__))
+        assert caught, f"no pin caught mutant {name}"
