@@ -1,1 +1,252 @@
-"""B200-native AVQ-Attention forward (placeholder; binding added with the library)."""
+"""B200-native forward pass of AVQ-Attention (Adaptive Vector-Quantized Attention).
+
+Thin Python binding over the C ABI of ``libavq.so`` (declared in
+``include/avq.h``).  The functions keep the C names and only marshal
+arguments: they check tensor dtypes/shapes/devices, allocate outputs with
+torch when the caller passes none, and hand raw device pointers and the
+current CUDA stream to the library.  Every step of the computation runs in
+the library's CUDA kernels; there is no CPU or PyTorch fallback -- if the
+library is missing the import of the first call raises.
+
+Stage 1, ``avq_quantize``: full-tree key quantisation and aggregation
+("AVQ-Attention: Adaptive Vector-Quantized Attention", Sec. 4.2, Algorithm 1).
+Stage 2, ``avq_attention``: count-weighted attention over the parents with
+top-P child refinement per query block (Sec. 4.3, Algorithm 2).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libavq.so")
+
+AVQ_OK, AVQ_ERR_INVALID_ARG, AVQ_ERR_UNSUPPORTED, AVQ_ERR_CUDA = 0, 1, 2, 3
+AVQ_ERR_DEVICE, AVQ_ERR_TIMEOUT, AVQ_ERR_WORKSPACE = 4, 5, 6
+AVQ_F32, AVQ_BF16 = 0, 1
+AVQ_PATH_AUTO, AVQ_PATH_SIMT, AVQ_PATH_TC = 0, 1, 2
+
+
+class AVQError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{status_string(status)}: {msg}")
+        self.status = status
+
+
+class avq_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("d", ctypes.c_int), ("M0", ctypes.c_int), ("C", ctypes.c_int)]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+_vp = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libavq.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        with _lib_lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise ImportError(
+                        f"{LIB_PATH} is missing: build it with "
+                        "`python -m adaptive_vector_quantized_b200.build`")
+                L = ctypes.CDLL(LIB_PATH)
+                P = ctypes.POINTER
+                L.avq_quantize.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
+                                           _vp, ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+                L.avq_attention.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                            _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+                L.avq_permute.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, _vp]
+                L.avq_hilbert_order.argtypes = [ctypes.c_int, _vp]
+                L.avq_workspace_size.argtypes = [P(avq_dims), ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_int]
+                L.avq_workspace_size.restype = ctypes.c_size_t
+                L.avq_check_device.argtypes = [_vp]
+                L.avq_set_path.argtypes = [ctypes.c_int]
+                L.avq_set_path.restype = ctypes.c_int
+                for name in ("avq_status_string", "avq_last_error", "avq_last_kernels"):
+                    getattr(L, name).restype = ctypes.c_char_p
+                L.avq_status_string.argtypes = [ctypes.c_int]
+                L.avq_version.restype = ctypes.c_int
+                for name in ("avq_quantize", "avq_attention", "avq_permute", "avq_hilbert_order",
+                             "avq_check_device"):
+                    getattr(L, name).restype = ctypes.c_int
+                _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().avq_status_string(int(status)).decode()
+
+
+def last_error() -> str:
+    return lib().avq_last_error().decode()
+
+
+def last_kernels() -> str:
+    return lib().avq_last_kernels().decode()
+
+
+def avq_set_path(path: int) -> int:
+    old = lib().avq_set_path(int(path))
+    if old < 0:
+        raise ValueError(f"unknown path {path}")
+    return old
+
+
+def _check(status: int):
+    if status != AVQ_OK:
+        raise AVQError(status, last_error())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return AVQ_F32
+    if t.dtype == torch.bfloat16:
+        return AVQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return _vp(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _vp(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dims(Q_like: torch.Tensor, parents: torch.Tensor, children) -> avq_dims:
+    B, H, N, d = Q_like.shape
+    Hp, M0, dp = parents.shape
+    C = 0 if children is None else children.shape[2]
+    if Hp != H or dp != d:
+        raise ValueError("parents must be [H, M0, d]")
+    if children is not None and tuple(children.shape) != (H, M0, C, d):
+        raise ValueError("children must be [H, M0, C, d]")
+    return avq_dims(B, H, N, d, M0, C)
+
+
+def avq_workspace_size(dims: avq_dims, dtype: int, deterministic=False, two_pass=False,
+                       P: int = 0, block: int = 128) -> int:
+    return int(lib().avq_workspace_size(ctypes.byref(dims), int(dtype), int(bool(deterministic)),
+                                        int(bool(two_pass)), int(P), int(block)))
+
+
+def workspace(dims: avq_dims, dtype: int, device, deterministic=False, two_pass=False, P=0,
+              block=128):
+    """A device byte tensor of the size the library asks for (None when 0)."""
+    n = avq_workspace_size(dims, dtype, deterministic, two_pass, P, block)
+    if n == 0:
+        return None
+    return torch.empty(n + 256, dtype=torch.uint8, device=device)
+
+
+def _ws_ptr(ws):
+    if ws is None:
+        return None, 0
+    p = ws.data_ptr()
+    off = (-p) % 256
+    return _vp(p + off), ws.numel() - off
+
+
+def avq_quantize(K, V, parents, children, assign=None, vsum=None, counts=None,
+                 deterministic=False, ws=None, stream=None):
+    """Stage 1.  K, V [B,H,N,d]; parents [H,M0,d]; children [H,M0,C,d] (or None
+    for C = 0).  Returns (assign [B,H,N] int32, vsum [B,H,Mt,d] fp32,
+    counts [B,H,Mt] int32)."""
+    dims = _dims(K, parents, children)
+    dt = _dtype_code(K)
+    B, H, N, d = K.shape
+    Mt = dims.M0 * (1 + dims.C)
+    dev = K.device
+    if assign is None:
+        assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    if vsum is None:
+        vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
+    if counts is None:
+        counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
+    if deterministic and ws is None:
+        ws = workspace(dims, dt, dev, deterministic=True)
+    wp, wn = _ws_ptr(ws)
+    _check(lib().avq_quantize(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
+                              _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
+                              int(bool(deterministic)), wp, wn, _stream(stream)))
+    return assign, vsum, counts
+
+
+def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, scale=None,
+                  two_pass=False, O=None, sel=None, importance=False, ws=None, stream=None):
+    """Stage 2.  Returns (O [B,H,N,d], sel [B,H,nblk,P] int32, importance
+    [B,H,nblk,M0] fp32 or None).  `importance=True` asks for the importance
+    output; a tensor is written in place."""
+    dims = _dims(Q, parents, children)
+    dt = _dtype_code(Q)
+    B, H, N, d = Q.shape
+    nblk = (N + block - 1) // block
+    dev = Q.device
+    if scale is None:
+        scale = d ** -0.5
+    if O is None:
+        O = torch.empty_like(Q)
+    if sel is None:
+        sel = torch.empty((B, H, nblk, max(P, 0)), dtype=torch.int32, device=dev)
+    imp = None
+    if isinstance(importance, torch.Tensor):
+        imp = importance
+    elif importance:
+        imp = torch.empty((B, H, nblk, dims.M0), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(dims, dt, dev, two_pass=two_pass, P=P, block=block)
+    wp, wn = _ws_ptr(ws)
+    _check(lib().avq_attention(ctypes.byref(dims), dt, _ptr(Q), _ptr(parents), _ptr(children),
+                               _ptr(vsum), _ptr(counts), int(P), int(block), float(scale),
+                               int(bool(two_pass)), _ptr(O), _ptr(sel) if P > 0 else None,
+                               _ptr(imp), wp, wn, _stream(stream)))
+    return O, sel, imp
+
+
+def avq_permute(X, idx, inverse=False, Y=None, stream=None):
+    """Gather (inverse=False: Y[b,i] = X[b,idx[i]]) or scatter back along dim -2
+    of a [..., rows, cols] tensor; idx is an int32 CUDA tensor."""
+    rows = X.shape[-2]
+    batch = X.numel() // (rows * X.shape[-1])
+    row_bytes = X.shape[-1] * X.element_size()
+    if Y is None:
+        Y = torch.empty_like(X)
+    if idx.dtype != torch.int32:
+        raise TypeError("idx must be int32")
+    _check(lib().avq_permute(_ptr(X), _ptr(idx), _ptr(Y), int(batch), int(rows), int(row_bytes),
+                             int(bool(inverse)), _stream(stream)))
+    return Y
+
+
+def avq_hilbert_order(side: int) -> torch.Tensor:
+    """Raster index of the t-th cell along a Hilbert curve (host tensor, int32)."""
+    out = torch.empty(side * side, dtype=torch.int32)
+    _check(lib().avq_hilbert_order(int(side), _vp(out.data_ptr())))
+    return out
+
+
+def avq_check_device(stream=None):
+    """Synchronise the stream and raise if a kernel recorded a device-side error."""
+    _check(lib().avq_check_device(_stream(stream)))
+
+
+def avq_version() -> int:
+    return int(lib().avq_version())

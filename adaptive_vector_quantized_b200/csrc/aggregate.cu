@@ -1,0 +1,387 @@
+// Stage 1, aggregation ("AVQ-Attention: Adaptive Vector-Quantized Attention",
+// Sec. 4.2, Algorithm 1 steps 1, 8 and 16; Eq. 3).
+//
+// Given every key's final code, each key adds its value and a count of one to
+// its parent, and to its child when it moved to one.  Parents therefore hold
+// their whole cluster, children only the keys closer to them than to the
+// parent.
+//
+// Atomics variant: one CTA per chunk of keys of one head.  Warps walk
+// contiguous key ranges with lanes over the head dimension, merge runs of equal
+// codes in registers and flush each run with shared-memory atomics into
+// per-CTA partials [Mt][d]; the CTA then adds its non-empty rows to global
+// memory with vector reductions.  When the partials do not fit in shared
+// memory, runs are flushed straight to global memory.
+//
+// Deterministic variant: keys are stably sorted by (parent, child) with a
+// counting sort over fixed 1024-key chunks, each segment is summed in key
+// order by one warp, and parent totals are formed as stay + children in a
+// fixed order.  Nothing depends on the grid or the GPU's size.
+#include "common.cuh"
+#include "internal.h"
+
+namespace avq {
+
+namespace {
+
+constexpr int kAggThreads = 512;
+constexpr int kAggBatch = 16;  // keys whose loads are in flight per warp
+
+template <int E>
+__device__ __forceinline__ void flush_run(float* part, int* cnt, int code, const float* acc, int n,
+                                          int lane, int D) {
+  float* row = part + (size_t)code * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) atomicAdd(row + e, acc[e]);
+  if (lane == 0) atomicAdd(cnt + code, n);
+}
+
+template <typename T, int D, bool SMEM>
+__global__ void __launch_bounds__(kAggThreads) aggregate_kernel(
+    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
+    int32_t* __restrict__ counts, int N, int M0, int C, int chunk) {
+  extern __shared__ __align__(16) float sm[];
+  constexpr int E = D / 32;
+  const int bh = blockIdx.y;
+  const int Mt = M0 * (1 + C);
+  float* gvs = vsum + (size_t)bh * Mt * D;
+  int* gcnt = counts + (size_t)bh * Mt;
+  float* part = SMEM ? sm : gvs;
+  int* cnt = SMEM ? reinterpret_cast<int*>(sm + (size_t)Mt * D) : gcnt;
+  if (SMEM) {
+    float4* s4 = reinterpret_cast<float4*>(sm);
+    for (int i = threadIdx.x; i < Mt * D / 4; i += blockDim.x) s4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = threadIdx.x; i < Mt; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int k0 = blockIdx.x * chunk;
+  const int k1 = min(N, k0 + chunk);
+  const int per = (k1 - k0 + nw - 1) / nw;
+  const int j0 = k0 + warp * per;
+  const int j1 = min(k1, j0 + per);
+  const int32_t* asg = assign + (size_t)bh * N;
+  const T* vb = V + (size_t)bh * N * D + lane * E;
+
+  float accP[E], accC[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
+  int curP = -1, curC = -1, nP = 0, nC = 0;
+  for (int jb = j0; jb < j1; jb += kAggBatch) {
+    int code[kAggBatch];
+    float v[kAggBatch][E];
+#pragma unroll
+    for (int u = 0; u < kAggBatch; ++u) {
+      const int j = jb + u;
+      if (j < j1) {
+        code[u] = __ldg(asg + j);
+        loadE<E>(vb + (size_t)j * D, v[u]);
+      } else {
+        code[u] = -1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAggBatch; ++u) {
+      const int c = code[u];
+      if (c < 0) break;
+      const int p = c < M0 ? c : (c - M0) / C;
+      if (p != curP) {
+        if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
+        curP = p;
+        nP = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) accP[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) accP[e] += v[u][e];
+      ++nP;
+      if (c >= M0) {
+        if (c != curC) {
+          if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
+          curC = c;
+          nC = 0;
+#pragma unroll
+          for (int e = 0; e < E; ++e) accC[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) accC[e] += v[u][e];
+        ++nC;
+      }
+    }
+  }
+  if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
+  if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
+  if (SMEM) {
+    __syncthreads();
+    const float4* s4 = reinterpret_cast<const float4*>(sm);
+    for (int i = threadIdx.x; i < Mt * D / 4; i += blockDim.x) {
+      const int row = i / (D / 4);
+      if (cnt[row] > 0) {
+        const float4 a = s4[i];
+        red_add_v4(gvs + (size_t)4 * i, a.x, a.y, a.z, a.w);
+      }
+    }
+    for (int r = threadIdx.x; r < Mt; r += blockDim.x)
+      if (cnt[r] > 0) atomicAdd(gcnt + r, cnt[r]);
+  }
+}
+
+// ---- deterministic variant ------------------------------------------------
+constexpr int kDetChunk = 1024;  // keys per sort chunk (fixed: independent of the GPU)
+constexpr int kDetWarps = 4;     // chunks per CTA
+
+__device__ __forceinline__ int sort_bin(int code, int M0, int C) {
+  // parent*(C+1) + 0 for keys that stay at the parent, + 1 + c for child c
+  if (code < M0) return code * (C + 1);
+  const int r = code - M0;
+  const int p = r / C;
+  return p * (C + 1) + 1 + (r - p * C);
+}
+
+// hist[bh][bin][chunk]: keys of `chunk` that fall in `bin`.
+__global__ void __launch_bounds__(kDetWarps * 32) det_hist_kernel(const int32_t* __restrict__ assign,
+                                                                  int* __restrict__ hist, int N,
+                                                                  int M0, int C, int nch) {
+  extern __shared__ int hs[];  // [kDetWarps][Mt]
+  const int Mt = M0 * (1 + C);
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* h = hs + warp * Mt;
+  for (int i = lane; i < Mt; i += 32) h[i] = 0;
+  __syncwarp();
+  const int ch = blockIdx.x * kDetWarps + warp;
+  if (ch < nch) {
+    const int j0 = ch * kDetChunk, j1 = min(N, j0 + kDetChunk);
+    for (int j = j0 + lane; j < j1; j += 32) atomicAdd(h + sort_bin(assign[(size_t)bh * N + j], M0, C), 1);
+    __syncwarp();
+    int* out = hist + (size_t)bh * Mt * nch;
+    for (int b = lane; b < Mt; b += 32) out[(size_t)b * nch + ch] = h[b];
+  }
+}
+
+// In place exclusive scan of hist[bh][*] (bin-major, then chunk): one CTA per head.
+__global__ void __launch_bounds__(1024) det_scan_kernel(int* __restrict__ hist, int total) {
+  __shared__ int part[1024];
+  int* h = hist + (size_t)blockIdx.x * total;
+  const int per = (total + blockDim.x - 1) / blockDim.x;
+  const int s0 = threadIdx.x * per, s1 = min(total, s0 + per);
+  int sum = 0;
+  for (int i = s0; i < s1; ++i) sum += h[i];
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {  // Hillis-Steele inclusive scan
+    const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int run = threadIdx.x ? part[threadIdx.x - 1] : 0;
+  for (int i = s0; i < s1; ++i) {
+    const int c = h[i];
+    h[i] = run;
+    run += c;
+  }
+}
+
+// Stable scatter of key indices into sorted order (one warp per chunk).
+__global__ void __launch_bounds__(kDetWarps * 32) det_scatter_kernel(
+    const int32_t* __restrict__ assign, const int* __restrict__ offs, int* __restrict__ order,
+    int N, int M0, int C, int nch) {
+  extern __shared__ int cs[];  // [kDetWarps][Mt] running positions
+  const int Mt = M0 * (1 + C);
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ch = blockIdx.x * kDetWarps + warp;
+  if (ch >= nch) return;
+  int* pos = cs + warp * Mt;
+  const int* o = offs + (size_t)bh * Mt * nch;
+  for (int b = lane; b < Mt; b += 32) pos[b] = o[(size_t)b * nch + ch];
+  __syncwarp();
+  const int j0 = ch * kDetChunk, j1 = min(N, j0 + kDetChunk);
+  int* ord = order + (size_t)bh * N;
+  for (int jb = j0; jb < j1; jb += 32) {
+    const int j = jb + lane;
+    const bool ok = j < j1;
+    const int bin = ok ? sort_bin(assign[(size_t)bh * N + j], M0, C) : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int base = ok ? pos[bin] : 0;
+    __syncwarp();
+    if (ok) {
+      ord[base + rank] = j;
+      if (rank == 0) pos[bin] = base + __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+// One warp per (bh, bin): sum of the segment's value rows in sorted (= key) order.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) det_segsum_kernel(const T* __restrict__ V,
+                                                         const int* __restrict__ offs,
+                                                         const int* __restrict__ order,
+                                                         float* __restrict__ seg, int N, int Mt,
+                                                         int nch) {
+  constexpr int E = D / 32;
+  const int bh = blockIdx.y;
+  const int bin = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (bin >= Mt) return;
+  const int* o = offs + (size_t)bh * Mt * nch;
+  const int start = o[(size_t)bin * nch];
+  const int end = bin + 1 < Mt ? o[(size_t)(bin + 1) * nch] : N;
+  const int* ord = order + (size_t)bh * N;
+  const T* vb = V + (size_t)bh * N * D + lane * E;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int i = start; i < end; i += 8) {
+    float v[8][E];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (i + u < end) loadE<E>(vb + (size_t)__ldg(ord + i + u) * D, v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (i + u < end) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] += v[u][e];
+      }
+    }
+  }
+  float* out = seg + ((size_t)bh * Mt + bin) * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) out[e] = acc[e];
+}
+
+// vsum/counts from the segment sums: child (p,c) = segment (p, 1+c); parent p =
+// stay segment + children segments in child order.
+__global__ void det_combine_kernel(const float* __restrict__ seg, const int* __restrict__ offs,
+                                   float* __restrict__ vsum, int32_t* __restrict__ counts, int N,
+                                   int M0, int C, int D, int nch) {
+  const int bh = blockIdx.y;
+  const int Mt = M0 * (1 + C);
+  const int p = blockIdx.x;
+  const int* o = offs + (size_t)bh * Mt * nch;
+  const float* sg = seg + (size_t)bh * Mt * D;
+  float* vs = vsum + (size_t)bh * Mt * D;
+  int32_t* ns = counts + (size_t)bh * Mt;
+  for (int t = threadIdx.x; t < D; t += blockDim.x) {
+    const int b0 = p * (C + 1);
+    float tot = sg[(size_t)b0 * D + t];
+    for (int c = 0; c < C; ++c) {
+      const float v = sg[(size_t)(b0 + 1 + c) * D + t];
+      tot += v;
+      vs[(size_t)(M0 + p * C + c) * D + t] = v;
+    }
+    vs[(size_t)p * D + t] = tot;
+  }
+  if (threadIdx.x == 0) {
+    auto seg_len = [&](int bin) {
+      const int s = o[(size_t)bin * nch];
+      const int e = bin + 1 < Mt ? o[(size_t)(bin + 1) * nch] : N;
+      return e - s;
+    };
+    const int b0 = p * (C + 1);
+    int tot = seg_len(b0);
+    for (int c = 0; c < C; ++c) {
+      const int n = seg_len(b0 + 1 + c);
+      ns[M0 + p * C + c] = n;
+      tot += n;
+    }
+    ns[p] = tot;
+  }
+}
+
+size_t agg_smem_bytes(const Shape& s) { return (size_t)s.Mt() * (s.d + 1) * sizeof(float); }
+
+}  // namespace
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t aggregate_det_workspace(const Shape& s) {
+  const size_t nch = (s.N + kDetChunk - 1) / kDetChunk;
+  const size_t hist = align256((size_t)s.BH() * s.Mt() * nch * sizeof(int));
+  const size_t order = align256((size_t)s.BH() * s.N * sizeof(int));
+  const size_t seg = align256((size_t)s.BH() * s.Mt() * s.d * sizeof(float));
+  return hist + order + seg;
+}
+
+cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
+                             float* vsum, int32_t* counts, cudaStream_t st, LaunchLog& log) {
+  cudaError_t e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * s.Mt() * s.d * sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  const size_t smem = agg_smem_bytes(s);
+  const bool use_smem = smem <= 200 * 1024;
+  // about one resident CTA per SM in total; chunks are whole warps' worth of keys
+  const int sms = num_sms();
+  int per_head = sms >= s.BH() ? sms / s.BH() : 1;  // a single wave where possible
+  if (!use_smem) per_head *= 4;
+  int chunk = (s.N + per_head - 1) / per_head;
+  chunk = ((chunk + 511) / 512) * 512;
+  if (chunk < 512) chunk = 512;
+  dim3 grid((s.N + chunk - 1) / chunk, s.BH());
+#define AVQ_AGG(T, D, SM)                                                                      \
+  do {                                                                                         \
+    auto kern = aggregate_kernel<T, D, SM>;                                                    \
+    if (SM) {                                                                                  \
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);  \
+      if (e != cudaSuccess) return e;                                                          \
+    }                                                                                          \
+    kern<<<grid, kAggThreads, SM ? smem : 0, st>>>((const T*)V, assign, vsum, counts, s.N,     \
+                                                   s.M0, s.C, chunk);                          \
+  } while (0)
+#define AVQ_AGG_D(T, SM) \
+  if (s.d == 64) AVQ_AGG(T, 64, SM); else AVQ_AGG(T, 128, SM)
+  if (dt == AVQ_F32) {
+    if (use_smem) AVQ_AGG_D(float, true); else AVQ_AGG_D(float, false);
+  } else {
+    if (use_smem) AVQ_AGG_D(bf16, true); else AVQ_AGG_D(bf16, false);
+  }
+#undef AVQ_AGG_D
+#undef AVQ_AGG
+  log.add(use_smem ? "aggregate_smem" : "aggregate_global");
+  return cudaGetLastError();
+}
+
+cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
+                                 const int32_t* assign, float* vsum, int32_t* counts, void* ws,
+                                 cudaStream_t st, LaunchLog& log) {
+  const int nch = (s.N + kDetChunk - 1) / kDetChunk;
+  const int Mt = s.Mt();
+  char* w = static_cast<char*>(ws);
+  int* hist = reinterpret_cast<int*>(w);
+  w += align256((size_t)s.BH() * Mt * nch * sizeof(int));
+  int* order = reinterpret_cast<int*>(w);
+  w += align256((size_t)s.BH() * s.N * sizeof(int));
+  float* seg = reinterpret_cast<float*>(w);
+
+  const size_t hsmem = (size_t)kDetWarps * Mt * sizeof(int);
+  cudaError_t e;
+  if (hsmem > 48 * 1024) {
+    e = cudaFuncSetAttribute(det_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(det_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 g1((nch + kDetWarps - 1) / kDetWarps, s.BH());
+  det_hist_kernel<<<g1, kDetWarps * 32, hsmem, st>>>(assign, hist, s.N, s.M0, s.C, nch);
+  det_scan_kernel<<<s.BH(), 1024, 0, st>>>(hist, Mt * nch);
+  det_scatter_kernel<<<g1, kDetWarps * 32, hsmem, st>>>(assign, hist, order, s.N, s.M0, s.C, nch);
+  dim3 g4((Mt + 7) / 8, s.BH());
+  if (dt == AVQ_F32) {
+    if (s.d == 64) det_segsum_kernel<float, 64><<<g4, 256, 0, st>>>((const float*)V, hist, order, seg, s.N, Mt, nch);
+    else det_segsum_kernel<float, 128><<<g4, 256, 0, st>>>((const float*)V, hist, order, seg, s.N, Mt, nch);
+  } else {
+    if (s.d == 64) det_segsum_kernel<bf16, 64><<<g4, 256, 0, st>>>((const bf16*)V, hist, order, seg, s.N, Mt, nch);
+    else det_segsum_kernel<bf16, 128><<<g4, 256, 0, st>>>((const bf16*)V, hist, order, seg, s.N, Mt, nch);
+  }
+  det_combine_kernel<<<dim3(s.M0, s.BH()), 128, 0, st>>>(seg, hist, vsum, counts, s.N, s.M0, s.C,
+                                                         s.d, nch);
+  log.add("det_hist det_scan det_scatter det_segsum det_combine");
+  return cudaGetLastError();
+}
+
+}  // namespace avq

@@ -1,0 +1,282 @@
+// C ABI of libavq.so: host-side validation and dispatch.  Every check runs on
+// the host before anything is enqueued; a failed check launches nothing.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace avq {
+
+// One error word per device (module-scope device memory, created with the
+// module; no allocation by the library).
+__device__ unsigned int g_avq_error_word;
+
+namespace {
+thread_local char t_error[512];
+thread_local char t_kernels[512];
+thread_local int t_path = AVQ_PATH_AUTO;
+
+avq_status fail(avq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_error, sizeof(t_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+avq_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(AVQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned int* g_err_ptr[kMaxDevices];
+int g_sms[kMaxDevices];
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  return dev;
+}
+
+avq_status check_dims(const avq_dims* d, avq_dtype dt) {
+  if (d == nullptr) return fail(AVQ_ERR_INVALID_ARG, "dims is NULL");
+  if (dt != AVQ_F32 && dt != AVQ_BF16) return fail(AVQ_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (d->B < 1 || d->H < 1 || d->N < 1)
+    return fail(AVQ_ERR_INVALID_ARG, "B, H and N must be >= 1 (got %d, %d, %d)", d->B, d->H, d->N);
+  if (d->d != 64 && d->d != 128) return fail(AVQ_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d->d);
+  if (d->M0 < 1 || d->M0 > 256) return fail(AVQ_ERR_UNSUPPORTED, "M0 must be in [1, 256] (got %d)", d->M0);
+  if (d->C < 0 || d->C > 8) return fail(AVQ_ERR_UNSUPPORTED, "C must be in [0, 8] (got %d)", d->C);
+  const long long rows = (long long)d->B * d->H * d->N;
+  if (rows > (1ll << 31) - 1 || (long long)d->B * d->H > 65535 * 64)
+    return fail(AVQ_ERR_UNSUPPORTED, "B*H*N = %lld exceeds the supported range", rows);
+  return AVQ_OK;
+}
+
+Shape to_shape(const avq_dims* d) { return Shape{d->B, d->H, d->N, d->d, d->M0, d->C}; }
+
+avq_status check_ws(size_t need, void* ws, size_t ws_bytes) {
+  if (need == 0) return AVQ_OK;
+  if (ws == nullptr || ws_bytes < need)
+    return fail(AVQ_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need,
+                ws_bytes, ws);
+  if (!aligned(ws, 256)) return fail(AVQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return AVQ_OK;
+}
+
+#define AVQ_REQUIRE_PTR(p, name)                                                        \
+  do {                                                                                  \
+    if ((p) == nullptr) return fail(AVQ_ERR_INVALID_ARG, "%s is NULL", name);           \
+    if (!aligned((p), 16)) return fail(AVQ_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+}  // namespace
+
+void LaunchLog::add(const char* name) {
+  const int n = (int)strlen(name);
+  if (len + n + 2 >= (int)sizeof(text)) return;
+  if (len) text[len++] = ' ';
+  memcpy(text + len, name, n);
+  len += n;
+  text[len] = 0;
+}
+
+unsigned int* error_word() {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_avq_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+int num_sms() {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sms[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    g_sms[dev] = v;
+  }
+  return g_sms[dev];
+}
+
+}  // namespace avq
+
+using namespace avq;
+
+extern "C" {
+
+const char* avq_status_string(avq_status s) {
+  switch (s) {
+    case AVQ_OK: return "AVQ_OK";
+    case AVQ_ERR_INVALID_ARG: return "AVQ_ERR_INVALID_ARG";
+    case AVQ_ERR_UNSUPPORTED: return "AVQ_ERR_UNSUPPORTED";
+    case AVQ_ERR_CUDA: return "AVQ_ERR_CUDA";
+    case AVQ_ERR_DEVICE: return "AVQ_ERR_DEVICE";
+    case AVQ_ERR_TIMEOUT: return "AVQ_ERR_TIMEOUT";
+    case AVQ_ERR_WORKSPACE: return "AVQ_ERR_WORKSPACE";
+  }
+  return "AVQ_ERR_UNKNOWN";
+}
+
+const char* avq_last_error(void) { return t_error; }
+const char* avq_last_kernels(void) { return t_kernels; }
+int avq_version(void) { return 100; }
+
+int avq_set_path(int path) {
+  if (path != AVQ_PATH_AUTO && path != AVQ_PATH_SIMT && path != AVQ_PATH_TC) return -1;
+  const int old = t_path;
+  t_path = path;
+  return old;
+}
+
+size_t avq_workspace_size(const avq_dims* dims, avq_dtype dtype, int deterministic, int two_pass,
+                          int P, int block) {
+  if (dims == nullptr) return 0;
+  const Shape s = to_shape(dims);
+  size_t need = 0;
+  if (deterministic) need = aggregate_det_workspace(s);
+  if (attention_tc_supported(s, dtype, P, block, two_pass)) {
+    const size_t a = attention_tc_workspace(s, P, block, two_pass);
+    if (a > need) need = a;
+  }
+  return need;
+}
+
+avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, const void* V,
+                        const void* parents, const void* children, int32_t* assign, float* vsum,
+                        int32_t* counts, int deterministic, void* ws, size_t ws_bytes,
+                        avq_stream_t stream) {
+  t_error[0] = 0;
+  avq_status st = check_dims(dims, dtype);
+  if (st != AVQ_OK) return st;
+  const Shape s = to_shape(dims);
+  AVQ_REQUIRE_PTR(K, "K");
+  AVQ_REQUIRE_PTR(V, "V");
+  AVQ_REQUIRE_PTR(parents, "parents");
+  if (s.C > 0) AVQ_REQUIRE_PTR(children, "children");
+  AVQ_REQUIRE_PTR(assign, "assign");
+  AVQ_REQUIRE_PTR(vsum, "vsum");
+  AVQ_REQUIRE_PTR(counts, "counts");
+  if (deterministic) {
+    st = check_ws(aggregate_det_workspace(s), ws, ws_bytes);
+    if (st != AVQ_OK) return st;
+  }
+  const bool tc_ok = assign_tc_supported(s, dtype);
+  if (t_path == AVQ_PATH_TC && !tc_ok)
+    return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core assignment kernel for this shape/dtype");
+  const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  LaunchLog log{};
+  cudaError_t e;
+  if (use_tc) {
+    unsigned int* err = error_word();
+    if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+    e = launch_assign_tc(s, K, parents, children, assign, err, cs, log);
+  } else {
+    e = launch_assign_simt(s, dtype, K, parents, children, assign, cs, log);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
+  if (deterministic)
+    e = launch_aggregate_det(s, dtype, V, assign, vsum, counts, ws, cs, log);
+  else
+    e = launch_aggregate(s, dtype, V, assign, vsum, counts, cs, log);
+  if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}
+
+avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, const void* parents,
+                         const void* children, const float* vsum, const int32_t* counts, int P,
+                         int block, float scale, int two_pass, void* O, int32_t* sel,
+                         float* importance, void* ws, size_t ws_bytes, avq_stream_t stream) {
+  t_error[0] = 0;
+  avq_status st = check_dims(dims, dtype);
+  if (st != AVQ_OK) return st;
+  const Shape s = to_shape(dims);
+  if (P < 0 || P > s.M0) return fail(AVQ_ERR_INVALID_ARG, "P must be in [0, M0] (got %d)", P);
+  if (block != 64 && block != 128)
+    return fail(AVQ_ERR_UNSUPPORTED, "block must be 64 or 128 (got %d)", block);
+  if (!(scale > 0.f) || !isfinite(scale))
+    return fail(AVQ_ERR_INVALID_ARG, "scale must be finite and > 0");
+  AVQ_REQUIRE_PTR(Q, "Q");
+  AVQ_REQUIRE_PTR(parents, "parents");
+  if (s.C > 0) AVQ_REQUIRE_PTR(children, "children");
+  AVQ_REQUIRE_PTR(vsum, "vsum");
+  AVQ_REQUIRE_PTR(counts, "counts");
+  AVQ_REQUIRE_PTR(O, "O");
+  if (P > 0) AVQ_REQUIRE_PTR(sel, "sel");
+  if (importance != nullptr && !aligned(importance, 16))
+    return fail(AVQ_ERR_INVALID_ARG, "importance is not 16-byte aligned");
+  const bool tc_ok = attention_tc_supported(s, dtype, P, block, two_pass);
+  if (t_path == AVQ_PATH_TC && !tc_ok)
+    return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core attention kernel for this shape/dtype");
+  const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  LaunchLog log{};
+  cudaError_t e;
+  if (use_tc) {
+    st = check_ws(attention_tc_workspace(s, P, block, two_pass), ws, ws_bytes);
+    if (st != AVQ_OK) return st;
+    unsigned int* err = error_word();
+    if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+    e = launch_attention_tc(s, Q, parents, children, vsum, counts, P, block, scale, two_pass, O,
+                            sel, importance, ws, err, cs, log);
+  } else {
+    e = launch_attention_simt(s, dtype, Q, parents, children, vsum, counts, P, block, scale, O,
+                              sel, importance, cs, log);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}
+
+avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
+                       int row_bytes, int inverse, avq_stream_t stream) {
+  t_error[0] = 0;
+  if (batch < 1 || rows < 1) return fail(AVQ_ERR_INVALID_ARG, "batch and rows must be >= 1");
+  if (row_bytes < 16 || row_bytes % 16 != 0)
+    return fail(AVQ_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16");
+  AVQ_REQUIRE_PTR(X, "X");
+  AVQ_REQUIRE_PTR(Y, "Y");
+  if (idx == nullptr) return fail(AVQ_ERR_INVALID_ARG, "idx is NULL");
+  if (!aligned(idx, 4)) return fail(AVQ_ERR_INVALID_ARG, "idx is not 4-byte aligned");
+  const size_t bytes = (size_t)batch * rows * row_bytes;
+  const char* x = static_cast<const char*>(X);
+  const char* y = static_cast<const char*>(Y);
+  if (x < y + bytes && y < x + bytes) return fail(AVQ_ERR_INVALID_ARG, "X and Y overlap");
+  LaunchLog log{};
+  cudaError_t e = launch_permute(X, idx, Y, batch, rows, row_bytes, inverse,
+                                 reinterpret_cast<cudaStream_t>(stream), log);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}
+
+avq_status avq_check_device(avq_stream_t stream) {
+  t_error[0] = 0;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_avq_error_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (word == 0) return AVQ_OK;
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbol(g_avq_error_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  if (word & kErrTimeout) return fail(AVQ_ERR_TIMEOUT, "a bounded device wait ran out (word 0x%x)", word);
+  return fail(AVQ_ERR_DEVICE, "device error word 0x%x", word);
+}
+
+}  // extern "C"

@@ -1,0 +1,94 @@
+// Device helpers shared by the AVQ kernels: element loads/stores for the two
+// supported element types and small warp utilities.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace avq {
+
+typedef __nv_bfloat16 bf16;
+
+// Error bits recorded in the per-device error word.
+enum : unsigned int {
+  kErrTimeout = 1u,   // a bounded wait ran out
+  kErrBounds = 2u,    // a debug bounds check refused an access
+  kErrInternal = 4u,  // an impossible state (e.g. a TMEM allocation failure)
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 8 consecutive elements -> fp32 (p must be 16-byte aligned).
+__device__ __forceinline__ void load8(const float* p, float* o) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void load8(const bf16* p, float* o) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  o[0] = bf16_lo(u.x); o[1] = bf16_hi(u.x);
+  o[2] = bf16_lo(u.y); o[3] = bf16_hi(u.y);
+  o[4] = bf16_lo(u.z); o[5] = bf16_hi(u.z);
+  o[6] = bf16_lo(u.w); o[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return l | (h << 16);
+}
+
+// 8 fp32 -> 8 consecutive elements (16-byte aligned destination).
+__device__ __forceinline__ void store8(float* p, const float* v) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(bf16* p, const float* v) {
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]);
+  u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]);
+  u.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// E consecutive elements (E in {2, 4}) -> fp32, naturally aligned.
+template <int E>
+__device__ __forceinline__ void loadE(const float* p, float* o) {
+  if constexpr (E == 2) {
+    const float2 a = __ldg(reinterpret_cast<const float2*>(p));
+    o[0] = a.x; o[1] = a.y;
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  }
+}
+template <int E>
+__device__ __forceinline__ void loadE(const bf16* p, float* o) {
+  if constexpr (E == 2) {
+    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+    o[0] = bf16_lo(u); o[1] = bf16_hi(u);
+  } else {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    o[0] = bf16_lo(u.x); o[1] = bf16_hi(u.x);
+    o[2] = bf16_lo(u.y); o[3] = bf16_hi(u.y);
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Vector reduction into global memory (sm_90+): four fp32 adds in one op.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+}  // namespace avq

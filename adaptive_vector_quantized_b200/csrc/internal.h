@@ -1,0 +1,71 @@
+// Host-side launch interface between the C ABI (avq_api.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/avq.h"
+
+namespace avq {
+
+struct Shape {
+  int B, H, N, d, M0, C;
+  int BH() const { return B * H; }
+  int Mt() const { return M0 * (1 + C); }
+};
+
+// Every launcher returns cudaSuccess or the launch error, and appends the
+// names of the kernels it enqueued to `names` (space separated).
+struct LaunchLog {
+  char text[512];
+  int len;
+  void add(const char* name);
+};
+
+// ---- stage 1 ------------------------------------------------------------
+// Algorithm 1 steps 3-16 (assignment only): writes assign[BH][N].
+cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
+                               const void* children, int32_t* assign, cudaStream_t st,
+                               LaunchLog& log);
+// Algorithm 1 steps 1, 8, 16 (aggregation for given codes), atomics variant.
+// vsum/counts are zeroed inside.
+cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
+                             float* vsum, int32_t* counts, cudaStream_t st, LaunchLog& log);
+// Deterministic aggregation (fixed-order sums, independent of the grid).
+size_t aggregate_det_workspace(const Shape& s);
+cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
+                                 const int32_t* assign, float* vsum, int32_t* counts, void* ws,
+                                 cudaStream_t st, LaunchLog& log);
+
+// tcgen05 assignment kernel (bf16, d in {64,128}, M0 a multiple of 16 up to 256).
+bool assign_tc_supported(const Shape& s, avq_dtype dt);
+cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
+                             const void* children, int32_t* assign, unsigned int* err,
+                             cudaStream_t st, LaunchLog& log);
+
+// ---- stage 2 ------------------------------------------------------------
+cudaError_t launch_attention_simt(const Shape& s, avq_dtype dt, const void* Q, const void* parents,
+                                  const void* children, const float* vsum, const int32_t* counts,
+                                  int P, int block, float scale, void* O, int32_t* sel,
+                                  float* importance, cudaStream_t st, LaunchLog& log);
+
+bool attention_tc_supported(const Shape& s, avq_dtype dt, int P, int block, int two_pass);
+size_t attention_tc_workspace(const Shape& s, int P, int block, int two_pass);
+cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* parents,
+                                const void* children, const float* vsum, const int32_t* counts,
+                                int P, int block, float scale, int two_pass, void* O,
+                                int32_t* sel, float* importance, void* ws, unsigned int* err,
+                                cudaStream_t st, LaunchLog& log);
+
+// ---- token permutation ----------------------------------------------------
+cudaError_t launch_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
+                           int row_bytes, int inverse, cudaStream_t st, LaunchLog& log);
+
+// Device address of the current device's error word.
+unsigned int* error_word();
+
+int num_sms();
+
+}  // namespace avq

@@ -1,0 +1,393 @@
+#!/usr/bin/env python3
+"""Throughput of the AVQ-Attention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long] [--impl avq|reference]
+
+One step = stage 1 (avq_quantize: full-tree key quantisation + aggregation)
+and stage 2 (avq_attention: parent attention, top-P per query block, child
+refinement) over one batch of the workload, inputs already resident in HBM.
+Metric: queries/s = B*H*N per step / step time, whole job over all ranks
+(weak scaling: every rank runs its own independent batch; there is no
+collective on the data path).  Rank 0 prints one JSON line.
+
+`--impl reference` times the float64 CPU oracle instead, on a bounded sample
+of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "AVQ fwd queries/s at N=64K,M0=64,C=8,P=16,d=64; % of HBM/TC roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="long")
+    ap.add_argument("--impl", default="avq", choices=["avq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=None)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def algorithmic(cfg):
+    """Bytes and tensor FLOPs the method must move/compute per step, per stage.
+
+    Stage 1 reads K and V once, the codebook once per head and writes the
+    assignments and the statistics; stage 2 reads Q, the codebook and the
+    statistics and writes O and the selections.  FLOPs count the score
+    contractions and the value products (2 per multiply-add)."""
+    B, H, N, d, M0, C, P, blk = (cfg[k] for k in ("B", "H", "N", "d", "M0", "C", "P", "block"))
+    s = 2 if cfg["dtype"] == "bf16" else 4
+    BH = B * H
+    Mt = M0 * (1 + C)
+    nblk = -(-N // blk)
+    stats = BH * Mt * (4 * d + 4)
+    code = H * Mt * d * s
+    s1_bytes = 2 * BH * N * d * s + code + stats + 4 * BH * N
+    s1_flops = 2 * BH * N * (M0 + C) * d
+    s2_bytes = BH * N * d * (s + s) + stats + code + 4 * BH * nblk * P
+    s2_flops = 4 * BH * N * (M0 + P * C) * d
+    return dict(s1_bytes=s1_bytes, s1_flops=s1_flops, s2_bytes=s2_bytes, s2_flops=s2_flops)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for k, nm in enumerate(names):
+                if r[5 + k].strip().lower() == "active":
+                    reasons.add(nm)
+        sm.sort()
+        return dict(sm_mhz=sm[len(sm) // 2] if sm else None, sm_max_mhz=max(smax) if smax else None,
+                    reasons=sorted(reasons), samples=len(rows))
+
+
+def src_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(kernel_file, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of that kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rows = json.load(open(p))
+    except ValueError:
+        return None
+    src = os.path.join(ROOT, "adaptive_vector_quantized_b200", "csrc", kernel_file)
+    for r in rows:
+        if r.get("file") == kernel_file and r.get("workload") == workload and \
+                os.path.exists(src) and r.get("source_sha") == src_sha(src):
+            return r.get("bytes_per_launch")
+    return None
+
+
+def max_over_ranks(ms, device, world):
+    """The slowest rank's time: every rank contributes, every rank gets the max."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base, rank):
+    """Each rank runs its own independent batch (weak scaling)."""
+    return base + 17 * rank
+
+
+# ---------------------------------------------------------------------------
+def cpu_oracle_sample(inp, heads, steps=1):
+    """Time the float64 oracle (Alg. 1 + Alg. 2) on `heads` heads of the
+    workload: every key and every query of those heads."""
+    import oracle
+
+    orc = oracle.default()
+    Kh = inp["K"][:1, :heads]
+    Vh = inp["V"][:1, :heads]
+    Qh = inp["Q"][:1, :heads]
+    par = inp["parents"][:heads]
+    ch = inp["children"][:heads]
+    K64, V64, Q64 = (oracle._f64(t) for t in (Kh, Vh, Qh))
+    p64, c64 = oracle._f64(par), oracle._f64(ch)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        a, vs, n, _ = orc.quantize(K64, V64, p64, c64)
+        orc.attention(Q64, p64, c64, vs, n, inp["P"], inp["block"], inp["scale"])
+        times.append(time.perf_counter() - t0)
+    return heads * inp["N"], times, orc.num_threads()
+
+
+def run_reference(args, cfg, inp):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle  # noqa: F401  (the reference arm is the oracle)
+
+    heads = 1
+    queries, times, cores = cpu_oracle_sample(inp, heads, steps=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    t = sum(timed)
+    value = queries * len(timed) / t
+    sample = f"{heads} head(s) x N={inp['N']}: all keys quantised and all queries attended per step"
+    line = dict(metric=METRIC, value=value, unit="queries/s", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * t / len(timed), higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+                config=workload_config(args.config, cfg),
+                cpu_baseline=dict(value=value, unit="queries/s", cores=cores, kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit="queries/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(name, cfg):
+    keys = ("B", "H", "N", "d", "M0", "C", "P", "block")
+    out = {"workload": name}
+    out.update({k: cfg[k] for k in keys})
+    out["order"] = cfg.get("order", "natural")
+    out["two_pass"] = bool(cfg.get("two_pass", False))
+    return out
+
+
+# ---------------------------------------------------------------------------
+def run_avq(args, cfg, inp):
+    import torch
+    import torch.distributed as dist
+
+    import adaptive_vector_quantized_b200 as avq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+    P, block = cfg["P"], cfg["block"]
+    two_pass = bool(cfg.get("two_pass", False))
+    Q, K, V = (inp[k].to(dev) for k in ("Q", "K", "V"))
+    par = inp["parents"].to(dev)
+    ch = inp["children"].to(dev) if cfg["C"] > 0 else None
+    stream = torch.cuda.current_stream(dev)
+    dims = avq.avq_dims(B, H, N, d, cfg["M0"], cfg["C"])
+    dt = avq.AVQ_BF16 if cfg["dtype"] == "bf16" else avq.AVQ_F32
+    ws = avq.workspace(dims, dt, dev, two_pass=two_pass, P=P, block=block)
+    Mt = cfg["M0"] * (1 + cfg["C"])
+    nblk = -(-N // block)
+    assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
+    counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    sel = torch.empty((B, H, nblk, max(P, 1)), dtype=torch.int32, device=dev)
+
+    def step():
+        avq.avq_quantize(K, V, par, ch, assign, vsum, counts, stream=stream)
+        k1 = avq.last_kernels()
+        avq.avq_attention(Q, par, ch, vsum, counts, P, block, cfg["scale"], two_pass, O, sel,
+                          ws=ws, stream=stream)
+        return k1, avq.last_kernels()
+
+    for _ in range(args.warmup):
+        k1, k2 = step()
+    avq.avq_check_device(stream)
+    kernels_per_step = len(k1.split()) + len(k2.split())
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            avq.avq_quantize(K, V, par, ch, assign, vsum, counts, stream=stream)
+            ev[s][1].record(stream)
+            avq.avq_attention(Q, par, ch, vsum, counts, P, block, cfg["scale"], two_pass, O, sel,
+                              ws=ws, stream=stream)
+            ev[s][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    avq.avq_check_device(stream)
+    ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
+    t_s1 = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    t_s2 = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    ms_step = ms / args.steps
+    queries = B * H * N * world
+    value = queries / (ms_step * 1e-3)
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (inp[k].pin_memory() for k in ("Q", "K", "V"))
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        hsel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
+
+        def e2e_step():
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            step()
+            hO.copy_(O, non_blocking=True)
+            hsel.copy_(sel, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 10))
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(a0.elapsed_time(a1), dev, world)
+        h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV))
+        d2h = hO.numel() * hO.element_size() + hsel.numel() * hsel.element_size()
+        e2e = dict(value=queries / (ems / n_e2e * 1e-3), unit="queries/s", h2d_bytes_per_step=h2d,
+                   d2h_bytes_per_step=d2h, steps=n_e2e)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    alg = algorithmic(cfg)
+    s1_gbs = alg["s1_bytes"] / (t_s1 * 1e-3) / 1e9
+    s2_gbs = alg["s2_bytes"] / (t_s2 * 1e-3) / 1e9
+    s2_tfs = alg["s2_flops"] / (t_s2 * 1e-3) / 1e12
+    t_roof = (max(alg["s1_bytes"] / (peaks["hbm"] * 1e9), alg["s1_flops"] / (peaks["bf16"] * 1e12))
+              + max(alg["s2_bytes"] / (peaks["hbm"] * 1e9), alg["s2_flops"] / (peaks["bf16"] * 1e12)))
+    # dominant stage (larger share of the step) for the roofline object
+    if t_s2 >= t_s1:
+        dom, dom_bytes, dom_t, dom_file = "attention", alg["s2_bytes"], t_s2, "attention_tc.cu"
+    else:
+        dom, dom_bytes, dom_t, dom_file = "quantize", alg["s1_bytes"], t_s1, "assign_tc.cu"
+    achieved = dom_bytes / (dom_t * 1e-3) / 1e9
+    roofline = dict(bound="hbm", achieved=achieved, peak=peaks["hbm"], unit="GB/s",
+                    frac=achieved / peaks["hbm"], traffic=traffic_for(dom_file, args.config),
+                    kernel=dom, peak_source=peaks["source"],
+                    step_roofline_us=t_roof * 1e6, step_frac=t_roof * 1e3 / ms_step)
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:  # rank 0 at N=1 only
+        heads = min(cfg["H"], max(1, os.cpu_count() or 1))
+        q, times, cores = cpu_oracle_sample(inp, heads, steps=1)
+        cpu = dict(value=q / times[0], unit="queries/s", cores=cores, kind="oracle",
+                   sample=f"{heads} head(s) x N={N} of the same workload, b=0: all keys quantised "
+                          f"and all queries attended, float64, OpenMP")
+    line = dict(metric=METRIC, value=value, unit="queries/s", n_gpus=world, steps=args.steps,
+                warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype=cfg["dtype"], data="synthetic",
+                config=dict(workload_config(args.config, cfg),
+                            l2="inputs larger than L2 (Q, K, V 134 MB each per step); no flush"
+                            if cfg["N"] * cfg["H"] * cfg["B"] * cfg["d"] * 2 > 126e6 else
+                            "inputs smaller than L2; no flush"),
+                roofline=roofline, cpu_baseline=cpu, e2e=e2e,
+                gpu_launches=kernels_per_step * args.steps,
+                clocks=clk.summary(),
+                stages=dict(quantize_us=t_s1 * 1e3, attention_us=t_s2 * 1e3,
+                            quantize_gbs=s1_gbs, attention_gbs=s2_gbs, attention_tflops=s2_tfs,
+                            quantize_kernels=k1, attention_kernels=k2))
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from adaptive_vector_quantized_b200 import synth
+
+    cfg = synth.get_config(args.config) if args.config in synth.CONFIGS else None
+    if cfg is None:
+        raise SystemExit(f"unknown config {args.config}")
+    rank = int(os.environ.get("RANK", "0"))
+    seed = rank_seed(args.seed if args.seed is not None else synth.CONFIG_SEEDS.get(args.config, 1000), rank)
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = synth.make_inputs(dict(cfg, B=1, H=1), seed)
+        run_reference(args, cfg, inp)
+        return
+    inp = synth.make_inputs(cfg, seed)
+    run_avq(args, cfg, inp)
+
+
+if __name__ == "__main__":
+    main()

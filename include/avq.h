@@ -1,0 +1,181 @@
+/*
+ * avq.h -- C ABI of libavq.so, a B200-native (sm_100a) forward pass of
+ * AVQ-Attention ("AVQ-Attention: Adaptive Vector-Quantized Attention").
+ *
+ * Two stages, as in the paper's inference pipeline (Sec. 4.3 "Summary",
+ * Fig. 4): avq_quantize builds the statistics of the full codebook tree
+ * (Sec. 4.2, Algorithm 1); avq_attention attends over the parents with
+ * count-weighted online softmax, picks the top-P parents per query block and
+ * replaces their contribution with their children's (Sec. 4.3, Algorithm 2).
+ *
+ * Conventions shared by every call
+ *   - Ownership: the caller allocates and owns every buffer, host or device.
+ *     The library allocates no memory and keeps no state across calls except
+ *     thread-local settings (avq_set_path) and diagnostics (avq_last_error,
+ *     avq_last_kernels) and one device-side error word per GPU.
+ *   - Execution: device calls are enqueued on `stream` (NULL = legacy default
+ *     stream) and return without synchronising.  Results are valid once the
+ *     stream has completed the call.
+ *   - Errors: arguments are validated on the host before anything is launched;
+ *     a failed check returns AVQ_ERR_INVALID_ARG, AVQ_ERR_UNSUPPORTED or
+ *     AVQ_ERR_WORKSPACE, launches nothing and leaves every output untouched.
+ *     AVQ_ERR_CUDA means a launch was rejected by the CUDA runtime.  Faults
+ *     detected inside kernels (a bounded wait that ran out) are recorded in
+ *     the device error word and reported by avq_check_device.
+ *   - Layouts are dense row-major.  BH = B*H; tensor [B,H,N,d] puts head
+ *     (b,h) at offset (b*H+h)*N*d.  Device pointers must be 16-byte aligned.
+ *   - Codebook: one per head, shared by the batch (Algorithm 1 input
+ *     C in R^{H x Mtotal x D}).  Mt = M0*(1+C).  Codeword a < M0 is parent a;
+ *     codeword M0 + m*C + c is child c of parent m (Algorithm 1, comment on
+ *     step 9).  Each parent must equal the mean of its children (Sec. 4.1,
+ *     Eq. 5); the attention recovers parent logits from that (Eq. 8).
+ */
+#ifndef AVQ_H
+#define AVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* A CUDA stream (cudaStream_t).  NULL selects the legacy default stream. */
+typedef struct CUstream_st* avq_stream_t;
+
+typedef enum {
+  AVQ_OK = 0,
+  AVQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape    */
+  AVQ_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement  */
+  AVQ_ERR_CUDA = 3,        /* the CUDA runtime rejected a launch or copy    */
+  AVQ_ERR_DEVICE = 4,      /* a kernel recorded an error in the error word  */
+  AVQ_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out            */
+  AVQ_ERR_WORKSPACE = 6    /* workspace missing or smaller than required    */
+} avq_status;
+
+/* Element type of Q, K, V, O and of the codebook.  Arithmetic is fp32 in
+ * both cases (fp32 accumulation of bf16 products on the tensor cores). */
+typedef enum { AVQ_F32 = 0, AVQ_BF16 = 1 } avq_dtype;
+
+/* Problem shape of one attention layer.  Supported: B, H >= 1; N >= 1;
+ * d in {64, 128}; 1 <= M0 <= 256; 0 <= C <= 8. */
+typedef struct {
+  int B, H, N, d, M0, C;
+} avq_dims;
+
+/* Kernel family selection (thread-local; default AVQ_PATH_AUTO).
+ * AUTO picks the tensor-core kernels where they apply, SIMT otherwise.
+ * SIMT forces the general CUDA-core kernels.  TC forces the tcgen05
+ * kernels and makes calls they do not cover return AVQ_ERR_UNSUPPORTED. */
+typedef enum { AVQ_PATH_AUTO = 0, AVQ_PATH_SIMT = 1, AVQ_PATH_TC = 2 } avq_path;
+
+/*
+ * avq_quantize -- full-tree key quantisation and aggregation
+ * (Sec. 4.2 "Vector Quantization for (A)VQ-Attention", Algorithm 1, Eq. 3).
+ *
+ * Every key K[b,h,j] goes to its nearest parent a (squared Euclidean
+ * distance, ties to the lower index); it moves to the nearest child c* of a
+ * (ties to the first child) only if that child is strictly closer than a.
+ * Outputs (device, written in full; the call zeroes them first):
+ *   assign [B,H,N]    int32  final code: a, or M0 + a*C + c* if moved
+ *   vsum   [B,H,Mt,d] fp32   value sums V-bar (Eq. 3): a parent sums its whole
+ *                            cluster, a child only the keys that moved to it
+ *   counts [B,H,Mt]   int32  key counts n with the same membership
+ * Inputs (device): K, V [B,H,N,d]; parents [H,M0,d]; children [H,M0,C,d]
+ * (may be NULL when C == 0), all of `dtype`.
+ * deterministic != 0 makes vsum bitwise reproducible from run to run and
+ * independent of the GPU's size (fixed-order reduction; needs workspace).
+ * Workspace: `ws` (device, 256-byte aligned) of at least
+ * avq_workspace_size(...) bytes; may be NULL when that size is 0.
+ */
+avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype,
+                        const void* K, const void* V,
+                        const void* parents, const void* children,
+                        int32_t* assign, float* vsum, int32_t* counts,
+                        int deterministic, void* ws, size_t ws_bytes,
+                        avq_stream_t stream);
+
+/*
+ * avq_attention -- adaptive attention with per-query-block refinement
+ * (Sec. 4.3 "Computing (A)VQ-Attention with Flash Attention", Algorithm 2;
+ * Eqs. 6-9; masked running max of Sec. D, Eq. 18).
+ *
+ * For each head and each block I of `block` consecutive queries (the last
+ * block may be shorter): logits S = scale * Q C^T over the M0 parents; running
+ * max over non-empty parents; A = exp(S - m), zero for empty parents;
+ * x = A V-bar, z = A n (Eq. 6); importance w_j(I) = sum_i A_ij n_j / z_i
+ * (Eq. 7); the P parents of largest w (descending, ties to the lower index)
+ * are refined: child logits S_c, parent logit recovered as their mean (Eq. 8),
+ * dA = exp(S_c) - exp(S_p) (Eq. 9), zero for empty children, added to x and z;
+ * O = x / z.  With C == 0 or P == 0 no refinement happens (flat VQ attention,
+ * Eq. 4).
+ * Inputs (device): Q [B,H,N,d] of `dtype`; parents, children as for
+ * avq_quantize; vsum, counts as produced by avq_quantize.
+ * P in [0, M0]; block in {64, 128}; scale > 0 (1/sqrt(d) for standard
+ * attention; the paper omits it for clarity, Sec. 3.1).
+ * two_pass != 0 selects the exact two-pass denominator: a first pass over
+ * parent tiles finds the row max and z, a second recomputes the logits for
+ * x and the importance.  Results equal the single-pass ones; it serves parent
+ * codebooks too large to hold on chip.
+ * Outputs (device): O [B,H,N,d] of `dtype`; sel [B,H,nblk,P] int32, the
+ * selected parents in descending importance (nblk = ceil(N/block)), may be
+ * NULL when P == 0; importance [B,H,nblk,M0] fp32 or NULL.
+ * Workspace as for avq_quantize.
+ */
+avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q,
+                         const void* parents, const void* children,
+                         const float* vsum, const int32_t* counts,
+                         int P, int block, float scale, int two_pass,
+                         void* O, int32_t* sel, float* importance,
+                         void* ws, size_t ws_bytes, avq_stream_t stream);
+
+/*
+ * avq_permute -- token reordering gather/scatter (Sec. 4.2 and Fig. 3:
+ * tokens reordered along a space-filling curve so that query tiles are
+ * spatially compact).
+ * X, Y [batch, rows, row_bytes] (device); idx [rows] int32 (device), a
+ * permutation of 0..rows-1 shared by every batch entry.
+ * inverse == 0: Y[b, i] = X[b, idx[i]]  (gather into curve order)
+ * inverse != 0: Y[b, idx[i]] = X[b, i]  (scatter back)
+ * row_bytes must be a positive multiple of 16; X and Y must not overlap.
+ * idx is not checked for being a permutation on the device.
+ */
+avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
+                       int row_bytes, int inverse, avq_stream_t stream);
+
+/*
+ * avq_hilbert_order -- host helper: idx[t] = raster index (y*side + x) of the
+ * t-th cell of a Hilbert curve over a side x side grid, side a power of two
+ * (the power-of-two case of the generalised Hilbert curve of Sec. 4.2).
+ * idx is host memory of side*side int32.
+ */
+avq_status avq_hilbert_order(int side, int32_t* idx);
+
+/* Bytes of device workspace that avq_quantize and avq_attention need for
+ * these arguments (the larger of the two).  0 means none. */
+size_t avq_workspace_size(const avq_dims* dims, avq_dtype dtype, int deterministic,
+                          int two_pass, int P, int block);
+
+/* Synchronises `stream`, reads and clears the current device's error word.
+ * Returns AVQ_OK, AVQ_ERR_TIMEOUT, AVQ_ERR_DEVICE or AVQ_ERR_CUDA. */
+avq_status avq_check_device(avq_stream_t stream);
+
+/* Thread-local kernel family selection; returns the previous setting, or -1
+ * for a value outside avq_path. */
+int avq_set_path(int path);
+
+const char* avq_status_string(avq_status status);
+/* Thread-local text of the last failure on this thread ("" if none). */
+const char* avq_last_error(void);
+/* Thread-local, space-separated names of the kernels the last successful
+ * call on this thread enqueued. */
+const char* avq_last_kernels(void);
+/* Library version, major*10000 + minor*100 + patch. */
+int avq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AVQ_H */

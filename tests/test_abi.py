@@ -1,0 +1,106 @@
+"""The C-ABI library loads, exports what include/avq.h declares, and rejects
+bad arguments on the host before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import adaptive_vector_quantized_b200 as avq
+from adaptive_vector_quantized_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "avq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(avq_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "avq_quantize" in names and "avq_attention" in names and "avq_permute" in names
+    L = avq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", avq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(avq_\w+)$", out, flags=re.M))
+    assert set(names) <= exported, set(names) - exported
+
+
+def test_status_strings_and_version():
+    assert avq.status_string(0) == "AVQ_OK"
+    assert avq.status_string(6) == "AVQ_ERR_WORKSPACE"
+    assert avq.status_string(99) == "AVQ_ERR_UNKNOWN"
+    assert avq.avq_version() >= 100
+
+
+def test_set_path():
+    old = avq.avq_set_path(avq.AVQ_PATH_SIMT)
+    assert old == avq.AVQ_PATH_AUTO
+    assert avq.avq_set_path(avq.AVQ_PATH_AUTO) == avq.AVQ_PATH_SIMT
+    with pytest.raises(ValueError):
+        avq.avq_set_path(7)
+
+
+def _q(dims, K=0x1000, V=0x2000, par=0x3000, ch=0x4000, a=0x5000, vs=0x6000, n=0x7000,
+       dt=avq.AVQ_BF16, det=0, ws=None, wsb=0):
+    L = avq.lib()
+    d = None if dims is None else ctypes.byref(dims)
+    return L.avq_quantize(d, dt, K, V, par, ch, a, vs, n, det, ws, wsb, None)
+
+
+def _a(dims, P=4, block=128, scale=0.125, Q=0x1000, par=0x3000, ch=0x4000, vs=0x6000, n=0x7000,
+       O=0x8000, sel=0x9000, imp=None, dt=avq.AVQ_BF16):
+    L = avq.lib()
+    return L.avq_attention(ctypes.byref(dims), dt, Q, par, ch, vs, n, P, block, scale, 0, O, sel,
+                           imp, None, 0, None)
+
+
+def test_host_validation_rejects_before_launch():
+    ok = avq.avq_dims(1, 2, 1024, 64, 16, 4)
+    E = avq
+    assert _q(None) == E.AVQ_ERR_INVALID_ARG
+    assert _q(ok, dt=5) == E.AVQ_ERR_INVALID_ARG
+    assert _q(avq.avq_dims(1, 2, 0, 64, 16, 4)) == E.AVQ_ERR_INVALID_ARG
+    assert _q(avq.avq_dims(1, 2, 64, 96, 16, 4)) == E.AVQ_ERR_UNSUPPORTED
+    assert _q(avq.avq_dims(1, 2, 64, 64, 300, 4)) == E.AVQ_ERR_UNSUPPORTED
+    assert _q(avq.avq_dims(1, 2, 64, 64, 16, 9)) == E.AVQ_ERR_UNSUPPORTED
+    assert _q(ok, K=None) == E.AVQ_ERR_INVALID_ARG
+    assert "K is NULL" in avq.last_error()
+    assert _q(ok, V=0x2004) == E.AVQ_ERR_INVALID_ARG
+    assert "16-byte" in avq.last_error()
+    assert _q(ok, ch=None) == E.AVQ_ERR_INVALID_ARG
+    assert _q(ok, det=1) == E.AVQ_ERR_WORKSPACE
+    assert _q(ok, det=1, ws=0x10010, wsb=1 << 30) == E.AVQ_ERR_INVALID_ARG  # not 256-aligned
+    assert _a(ok, P=17) == E.AVQ_ERR_INVALID_ARG
+    assert _a(ok, P=-1) == E.AVQ_ERR_INVALID_ARG
+    assert _a(ok, block=32) == E.AVQ_ERR_UNSUPPORTED
+    assert _a(ok, scale=0.0) == E.AVQ_ERR_INVALID_ARG
+    assert _a(ok, scale=float("inf")) == E.AVQ_ERR_INVALID_ARG
+    assert _a(ok, sel=None) == E.AVQ_ERR_INVALID_ARG
+    assert _a(ok, O=None) == E.AVQ_ERR_INVALID_ARG
+    assert _a(ok, imp=0x123) == E.AVQ_ERR_INVALID_ARG
+    L = avq.lib()
+    assert L.avq_permute(0x1000, 0x2000, 0x3000, 1, 10, 24, 0, None) == E.AVQ_ERR_INVALID_ARG
+    assert L.avq_permute(0x1000, 0x2000, 0x1040, 1, 10, 16, 0, None) == E.AVQ_ERR_INVALID_ARG  # overlap
+    assert L.avq_permute(0x1000, None, 0x90000, 1, 10, 16, 0, None) == E.AVQ_ERR_INVALID_ARG
+
+
+def test_workspace_sizes():
+    d = avq.avq_dims(1, 16, 65536, 64, 64, 8)
+    assert avq.avq_workspace_size(d, avq.AVQ_BF16, deterministic=True) > 0
+    assert avq.avq_workspace_size(None if False else d, avq.AVQ_F32, deterministic=False) >= 0
+
+
+def test_hilbert_order_matches_textbook_curve():
+    for side in (1, 2, 8, 64, 256):
+        got = avq.avq_hilbert_order(side).numpy()
+        assert np.array_equal(got, synth.hilbert_cells(side))
+    with pytest.raises(avq.AVQError):
+        avq.avq_hilbert_order(12)

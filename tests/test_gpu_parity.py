@@ -1,0 +1,173 @@
+"""CUDA path against the float64 oracle, through the C ABI (needs a B200).
+
+Sizes are chosen so that the oracle finishes in seconds while still spanning
+several tiles and a ragged tail; the full-size workloads are checked on
+sampled query blocks plus full assignment/statistics checks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import adaptive_vector_quantized_b200 as avq
+import oracle
+from adaptive_vector_quantized_b200 import synth
+from tests import gpu_helpers as gh
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"simt": avq.AVQ_PATH_SIMT, "auto": avq.AVQ_PATH_AUTO}
+
+
+def _cfg(**kw):
+    base = dict(dtype="bf16", B=1, H=2, N=2048, d=64, M0=64, C=8, P=16, block=128,
+                keys="tree", key_sigma=0.1, sigma_c=0.3, two_pass=False)
+    base.update(kw)
+    return base
+
+
+CASES = {
+    "tiny": (synth.get_config("tiny"), 1000),
+    "vit_h3": (synth.get_config("vit", B=1, H=3), 1001),
+    "vit_full": (synth.get_config("vit"), 1001),
+    "largecb_small": (synth.get_config("largecb", H=2, N=2048), 1003),
+    "ragged_1000_b64": (_cfg(N=1000, block=64, M0=32, P=8), 7),
+    "ragged_1000_b128": (_cfg(N=1000, block=128, M0=32, P=8), 8),
+    "ragged_d128": (_cfg(N=777, d=128, M0=48, C=4, P=5), 9),
+    "n1": (_cfg(N=1, M0=16, P=4), 10),
+    "n65": (_cfg(N=65, M0=16, P=4, block=64), 11),
+    "m0_1": (_cfg(N=512, M0=1, P=1), 12),
+    "c1": (_cfg(N=512, M0=16, C=1, P=4), 13),
+    "p_eq_m0": (_cfg(N=1024, M0=16, P=16), 14),
+    "p0": (_cfg(N=1024, M0=16, P=0), 15),
+    "flat192": (synth.sweep_config(0, 4096, flat192=True), 1004),
+    "f32_d128": (_cfg(dtype="f32", N=1500, d=128, M0=24, C=4, P=6, block=64), 16),
+    "sweep_p4_random": (synth.sweep_config(4, 4096, "random"), 1004),
+    "sweep_p64_hilbert": (synth.sweep_config(64, 4096, "hilbert"), 1004),
+}
+
+
+@pytest.fixture(scope="module")
+def inputs():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cfg, seed = CASES[name]
+            cache[name] = synth.make_inputs(cfg, seed)
+        return cache[name]
+
+    return get
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("case", list(CASES))
+def test_forward_parity(inputs, case, path):
+    inp = inputs(case)
+    res = gh.gpu_forward(inp, path=PATHS[path])
+    diag = gh.check_forward(inp, res)
+    print(case, path, res["kernels"], diag)
+
+
+@pytest.mark.parametrize("P,block", [(0, 128), (1, 64), (8, 128), (64, 64)])
+def test_vit_p_and_block_variants(inputs, P, block):
+    inp = inputs("vit_h3")
+    for path in PATHS.values():
+        res = gh.gpu_forward(inp, P=P, block=block, path=path)
+        gh.check_forward(inp, res, P=P, block=block)
+
+
+def test_two_pass_equals_single_pass(inputs):
+    inp = inputs("largecb_small")
+    a = gh.gpu_forward(inp, two_pass=True)
+    b = gh.gpu_forward(inp, two_pass=False)
+    gh.check_forward(inp, a)
+    gh.check_forward(inp, b)
+    assert np.array_equal(a["assign"], b["assign"])
+
+
+def _sample_blocks(inp, n, seed):
+    rng = np.random.default_rng(seed)
+    nblk = (inp["N"] + inp["block"] - 1) // inp["block"]
+    BH = inp["B"] * inp["H"]
+    pick = rng.choice(BH * nblk, size=min(n, BH * nblk), replace=False)
+    blocks = [(int(u // nblk), int(u % nblk)) for u in pick]
+    blocks.append((BH - 1, nblk - 1))  # always include the last block
+    return blocks
+
+
+@pytest.mark.parametrize("name", ["long", "largecb"])
+def test_full_size_sampled(name):
+    cfg = synth.get_config(name)
+    inp = synth.make_inputs(cfg, synth.CONFIG_SEEDS[name])
+    res = gh.gpu_forward(inp)
+    diag = gh.check_forward(inp, res, blocks=_sample_blocks(inp, 48, 5))
+    # invariants that hold at any size
+    N, M0 = inp["N"], inp["M0"]
+    assert (res["counts"][..., :M0].sum(-1) == N).all()
+    moved = (res["assign"] >= M0).sum(-1)
+    assert (res["counts"][..., M0:].sum(-1) == moved).all()
+    imp_sums = res["imp"].sum(-1)
+    sizes = np.minimum(inp["block"], N - np.arange(imp_sums.shape[-1]) * inp["block"])
+    assert np.allclose(imp_sums, sizes[None, None, :], rtol=1e-4)
+    print(name, res["kernels"], diag)
+
+
+def test_deterministic_mode(inputs):
+    inp = inputs("vit_h3")
+    dev = gh.to_dev(inp)
+    a = gh.gpu_forward(inp, deterministic=True, dev=dev)
+    b = gh.gpu_forward(inp, deterministic=True, dev=dev)
+    c = gh.gpu_forward(inp, deterministic=False, dev=dev)
+    assert np.array_equal(a["vsum"].view(np.uint32), b["vsum"].view(np.uint32))
+    assert np.array_equal(a["counts"], c["counts"])
+    assert np.array_equal(a["O"].view(torch.int16).numpy(), b["O"].view(torch.int16).numpy())
+    gh.check_forward(inp, a)
+    assert "det_" in a["kernels"]
+
+
+def test_deterministic_matches_fixed_order_sum(inputs):
+    """The deterministic value sums are the plain sequential fp32 sums of each
+    (parent, child) segment in key order, and parents add stay + children."""
+    inp = inputs("tiny")
+    a = gh.gpu_forward(inp, deterministic=True)
+    V = inp["V"].numpy().astype(np.float32)
+    codes = a["assign"][0, 0]
+    M0, C = inp["M0"], inp["C"]
+    seg = {}
+    for j, code in enumerate(codes):
+        key = int(code)
+        acc = seg.get(key, np.zeros(V.shape[-1], dtype=np.float32))
+        seg[key] = np.float32(acc + V[0, 0, j])
+    for p in range(M0):
+        tot = seg.get(p, np.zeros(V.shape[-1], dtype=np.float32))
+        for c in range(C):
+            ch = seg.get(M0 + p * C + c, np.zeros(V.shape[-1], dtype=np.float32))
+            assert np.array_equal(a["vsum"][0, 0, M0 + p * C + c], ch)
+            tot = np.float32(tot + ch)
+        assert np.array_equal(a["vsum"][0, 0, p], tot)
+
+
+def test_permute_roundtrip_and_definition():
+    torch.manual_seed(0)
+    for rows, cols, dt in [(4096, 64, torch.bfloat16), (1000, 8, torch.float32), (7, 128, torch.bfloat16)]:
+        X = torch.randn(3, rows, cols).to(dt).cuda()
+        perm = torch.randperm(rows, dtype=torch.int64)
+        idx = perm.to(torch.int32).cuda()
+        Y = avq.avq_permute(X, idx)
+        Z = avq.avq_permute(Y, idx, inverse=True)
+        torch.cuda.synchronize()
+        Xc = X.cpu().numpy() if dt == torch.float32 else X.cpu().view(torch.int16).numpy()
+        Yc = Y.cpu().numpy() if dt == torch.float32 else Y.cpu().view(torch.int16).numpy()
+        Zc = Z.cpu().numpy() if dt == torch.float32 else Z.cpu().view(torch.int16).numpy()
+        assert np.array_equal(Yc, Xc[:, perm.numpy()])  # Y[b, i] = X[b, idx[i]]
+        assert np.array_equal(Zc, Xc)
+    side = 64
+    order = avq.avq_hilbert_order(side).cuda()
+    X = torch.arange(side * side * 8, dtype=torch.float32).reshape(1, side * side, 8).cuda()
+    Y = avq.avq_permute(X, order)
+    assert torch.equal(Y.cpu()[0, :, 0] / 8, order.cpu().float())
+
+
+def test_device_error_word_clean():
+    avq.avq_check_device()
