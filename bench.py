@@ -253,7 +253,7 @@ def run_avq(args, cfg, inp):
     def step():
         avq.avq_quantize(K, V, par, ch, assign, vsum, counts, stream=stream)
         k1 = avq.last_kernels()
-        avq.avq_attention(Q, par, ch, vsum, counts, P, block, cfg["scale"], two_pass, O, sel,
+        avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
                           ws=ws, stream=stream)
         return k1, avq.last_kernels()
 
@@ -274,7 +274,7 @@ def run_avq(args, cfg, inp):
             ev[s][0].record(stream)
             avq.avq_quantize(K, V, par, ch, assign, vsum, counts, stream=stream)
             ev[s][1].record(stream)
-            avq.avq_attention(Q, par, ch, vsum, counts, P, block, cfg["scale"], two_pass, O, sel,
+            avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
                               ws=ws, stream=stream)
             ev[s][2].record(stream)
         t1.record(stream)
