@@ -1,11 +1,591 @@
-// placeholder: tensor-core attention kernel (added next)
+// Stage 2 on the tcgen05 tensor cores ("AVQ-Attention: Adaptive
+// Vector-Quantized Attention", Sec. 4.3, Algorithm 2; Eqs. 6-9; Sec. D).
+//
+// One CTA per (head, block of 128 queries), 4 warps; thread i owns query row
+// i, which is TMEM lane i of every accumulator.  Per block:
+//   Q tile    TMA (128B swizzle) -> shared memory, stays for both logit MMAs
+//   parents   S = Q C_p^T on tcgen05 into TMEM; each thread loads its row,
+//             takes the masked max (Eq. 18), A = 2^(t - m) with t the scaled
+//             log2-domain logit, z = sum A n; the importance column sums
+//             (Eq. 7) are warp butterfly reduce-scatters in fp32; A goes to
+//             shared memory as bf16 and x = A Vbar_p accumulates in TMEM.
+//             If the parents do not fit one tile (or two_pass is set) the
+//             parent tiles are swept twice: running max and z first, then A,
+//             x and the importance with the exact denominator.
+//   top-P     ranks of the M0 importances (descending, ties to the lower
+//             index), all 128 threads.
+//   children  the selected parents' children (C = 8: one swizzle atom each)
+//             are bulk-copied from a prepared bf16 image; S_c = Q C_c^T on
+//             tcgen05; per row the parent logit is the mean of its 8 child
+//             logits (Eq. 8); dA = 2^(t_c - m) - 2^(t_p - m), zero for empty
+//             children (Eq. 9); x += dA Vbar_c on tcgen05; z += dA n_c.
+//             The reference max stays the parents' max unless a child logit
+//             exceeds it by more than 2^24, in which case x (TMEM) and z are
+//             rescaled first; the result is the same as the online merge of
+//             Algorithm 2 steps 13-14 because the max cancels in x / z.
+//   output    O = x / z, bf16, staged in shared memory and stored by TMA.
+// The codewords and the value sums are first converted by a small kernel
+// into bf16 images of 1024-byte swizzled atoms (8 codes x 64 dims), so that
+// every operand tile is one or more contiguous bulk copies.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tc_util.cuh"
+
 namespace avq {
-bool attention_tc_supported(const Shape&, avq_dtype, int, int, int) { return false; }
-size_t attention_tc_workspace(const Shape&, int, int, int) { return 0; }
-cudaError_t launch_attention_tc(const Shape&, const void*, const void*, const void*, const float*,
-                                const int32_t*, int, int, float, int, void*, int32_t*, float*,
-                                void*, unsigned int*, cudaStream_t, LaunchLog&) {
-  return cudaErrorNotSupported;
+
+namespace {
+
+constexpr int kRows = 128;          // queries per block (MMA M)
+constexpr int kTile = 128;          // parent codes per tile / child codes per chunk
+constexpr int kChunkParents = kTile / 8;
+constexpr float kRescaleLog2 = 24.f;
+
+struct AttnArgs {
+  const bf16* cw;   // [H][Mt/8][KH][8][64] swizzled codeword atoms
+  const bf16* vb;   // [BH][Mt/8][NH][8][64] swizzled value-sum atoms
+  const int32_t* counts;  // [BH][Mt]
+  int32_t* sel;     // [BH][nblk][P] or null
+  float* importance;  // [BH][nblk][M0] or null
+  unsigned int* err;
+  int H, N, M0, C, P, nblk, two_pass;
+  float scale_log2;  // scale * log2(e)
+};
+
+// shared memory plan (bytes); every operand region 1024-aligned
+template <int D>
+struct Smem {
+  static constexpr int KH = D / 64;
+  static constexpr int kQ = 0;                              // Q tile / O staging
+  static constexpr int kCW = kQ + kRows * D * 2;            // codeword tile
+  static constexpr int kVB = kCW + kTile * D * 2;           // value-sum tile
+  static constexpr int kPR = kVB + kTile * D * 2;           // probabilities [2][128][64]
+  static constexpr int kNF = kPR + kRows * kTile * 2;       // counts of the tile (float)
+  static constexpr int kW = kNF + kTile * 4;                // importance [256]
+  static constexpr int kWP = kW + 256 * 4;                  // per-warp partial sums [4][kTile]
+  static constexpr int kSEL = kWP + 4 * kTile * 4;          // selected parents [256]
+  static constexpr int kBAR = kSEL + 256 * 4;               // 3 mbarriers
+  static constexpr int kMISC = kBAR + 32;                   // tmem base, abort flag
+  static constexpr int kTotal = kMISC + 32;
+};
+
+__device__ __forceinline__ void fail(unsigned int* err, int* abort_flag) {
+  atomicOr(err, kErrTimeout);
+  *abort_flag = 1;
 }
+
+// Butterfly reduce-scatter of 32 per-lane values: lane L returns the warp sum
+// of element L.
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const bool hi = (lane & s) != 0;
+      const float send = hi ? v[i] : v[i + s];
+      const float keep = hi ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                           const __grid_constant__ CUtensorMap omap,
+                                                           const AttnArgs a) {
+  using S = Smem<D>;
+  constexpr int KH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = sm + S::kQ;
+  uint8_t* sCW = sm + S::kCW;
+  uint8_t* sVB = sm + S::kVB;
+  uint8_t* sPR = sm + S::kPR;
+  float* sNF = reinterpret_cast<float*>(sm + S::kNF);
+  float* sW = reinterpret_cast<float*>(sm + S::kW);
+  float* sWP = reinterpret_cast<float*>(sm + S::kWP);
+  int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
+  uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + S::kBAR);
+  uint64_t* bar_cp = bar_q + 1;
+  uint64_t* bar_mma = bar_q + 2;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S::kMISC);
+  int* sAbort = reinterpret_cast<int*>(sm + S::kMISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int blk = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
+  const int row0 = blk * kRows;
+  const bool valid = row0 + tid < a.N;
+  const int M0 = a.M0, Mt = M0 * (1 + a.C);
+  const int groups = Mt / 8;
+  const bf16* cw_h = a.cw + (size_t)h * groups * KH * 512;
+  const bf16* vb_bh = a.vb + (size_t)bh * groups * KH * 512;
+  const int32_t* cnt = a.counts + (size_t)bh * Mt;
+
+  if (tid == 0) {
+    tc::mbar_init(bar_q, 1);
+    tc::mbar_init(bar_cp, 1);
+    tc::mbar_init(bar_mma, 1);
+    tc::fence_mbar_init();
+    *sAbort = 0;
+    tc::prefetch_tensormap(&qmap);
+    tc::prefetch_tensormap(&omap);
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(sTmem, 256);
+    tc::tmem_relinquish();
+  }
+  for (int j = tid; j < M0; j += 128) sW[j] = 0.f;
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t tS = tmem;          // logits, up to 128 columns
+  const uint32_t tX = tmem + 128;    // output accumulator, D columns
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+  uint32_t ph_cp = 0, ph_mma = 0;
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh) tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, row0, bh, bar_q);
+  }
+
+  const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
+  const uint32_t sQa = tc::smem_u32(sQ), sCWa = tc::smem_u32(sCW), sVBa = tc::smem_u32(sVB),
+                 sPRa = tc::smem_u32(sPR);
+  // issue S = Q * CW^T (n codes) -- one thread
+  auto issue_logits = [&](int n) {
+    const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+      const uint64_t ad = tc::sdesc_sw128(sQa + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16, 1024);
+      const uint64_t bd = tc::sdesc_sw128(sCWa + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+      tc::mma_bf16(tS, ad, bd, idesc, k > 0);
+    }
+    tc::mma_commit(bar_mma);
+  };
+  // issue x += PR * VB (n codes) -- one thread
+  auto issue_values = [&](int n, bool acc) {
+#pragma unroll 1
+    for (int k = 0; k < n / 16; ++k) {
+      const uint64_t ad = tc::sdesc_sw128(sPRa + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16, 1024);
+      const uint64_t bd = tc::sdesc_sw128(sVBa + k * 2 * (KH * 1024), 1024, KH * 1024);
+      tc::mma_bf16(tX, ad, bd, idesc_x, (acc || k > 0) ? 1u : 0u);
+    }
+    tc::mma_commit(bar_mma);
+  };
+  auto wait_mma = [&]() {
+    if (!tc::mbar_wait(bar_mma, ph_mma)) fail(a.err, sAbort);
+    ph_mma ^= 1;
+    tc::tc_fence_after();
+  };
+  auto wait_cp = [&]() {
+    if (!tc::mbar_wait(bar_cp, ph_cp)) fail(a.err, sAbort);
+    ph_cp ^= 1;
+  };
+
+  const float NEG_INF = __int_as_float(0xff800000);
+  float m = NEG_INF, z = 0.f;
+  const int nT = (M0 + kTile - 1) / kTile;
+  const int sweeps = (a.two_pass || nT > 1) ? 2 : 1;
+  bool x_started = false;
+  bool q_ready = false;
+
+  for (int sweep = 0; sweep < sweeps; ++sweep) {
+    const bool last = sweep == sweeps - 1;
+    for (int t = 0; t < nT; ++t) {
+      const int c0 = t * kTile;
+      const int n = min(kTile, M0 - c0);
+      // bring the codeword tile (and its value sums on the last sweep)
+      if (tid == 0) {
+        const uint32_t cwb = (uint32_t)n * D * 2;
+        tc::mbar_arrive_expect_tx(bar_cp, last ? 2 * cwb : cwb);
+        tc::bulk_g2s(sCW, cw_h + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
+        if (last) tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
+      }
+      for (int j = tid; j < n; j += 128) sNF[j] = (float)__ldg(cnt + c0 + j);
+      if (!q_ready) {
+        if (!tc::mbar_wait(bar_q, 0)) fail(a.err, sAbort);
+        q_ready = true;
+      }
+      wait_cp();
+      __syncthreads();
+      if (*sAbort) goto done;
+      if (tid == 0) {
+        tc::tc_fence_after();
+        issue_logits(n);
+      }
+      wait_mma();
+      // pass over the row's logits in groups of 32 columns
+      {
+        float tmax = NEG_INF;
+        if (sweeps == 1 || !last) {
+          for (int g = 0; g < n; g += 16) {
+            uint32_t r[16];
+            tc::tmem_ld16(tS + lane_off + g, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float tv = __uint_as_float(r[e]) * a.scale_log2;
+              if (sNF[g + e] > 0.f) tmax = fmaxf(tmax, tv);
+            }
+          }
+          if (!last) {  // first sweep: online max and denominator
+            const float mn = fmaxf(m, tmax);
+            if (mn != NEG_INF) {
+              float zt = 0.f;
+              for (int g = 0; g < n; g += 16) {
+                uint32_t r[16];
+                tc::tmem_ld16(tS + lane_off + g, r);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const float nf = sNF[g + e];
+                  const float tv = __uint_as_float(r[e]) * a.scale_log2;
+                  zt += nf > 0.f ? nf * tc::ex2(tv - mn) : 0.f;
+                }
+              }
+              z = z * tc::ex2(m - mn) + zt;
+              m = mn;
+            }
+          } else {  // single sweep: the tile holds every parent
+            m = tmax;
+            z = 0.f;
+            for (int g = 0; g < n; g += 16) {
+              uint32_t r[16];
+              tc::tmem_ld16(tS + lane_off + g, r);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float nf = sNF[g + e];
+                const float tv = __uint_as_float(r[e]) * a.scale_log2;
+                z += nf > 0.f ? nf * tc::ex2(tv - m) : 0.f;
+              }
+            }
+          }
+        }
+        if (last) {
+          // A = 2^(t - m) (masked), bf16 -> probabilities, importance sums
+          const float rz = valid ? 1.f / z : 0.f;
+          for (int g = 0; g < n; g += 32) {
+            float v[32];
+            uint32_t r[32];
+            tc::tmem_ld16(tS + lane_off + g, r);
+            tc::tmem_ld16(tS + lane_off + g + 16, r + 16);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float tv = __uint_as_float(r[e]) * a.scale_log2;
+              v[e] = (g + e < n && sNF[g + e] > 0.f) ? tc::ex2(tv - m) : 0.f;
+            }
+            // probabilities (row tid, codes g..g+31) as four 16-byte chunks
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = g + q * 8;
+              uint4 u;
+              u.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              u.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              u.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              u.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              *reinterpret_cast<uint4*>(sPR + (col >> 6) * (kRows * 128) + tc::sw128_offset(tid, col & 63)) = u;
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= rz;
+            sWP[warp * kTile + g + lane] = reduce_scatter32(v, lane);
+          }
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      if (last) {
+        for (int j = tid; j < n; j += 128)
+          sW[c0 + j] += sNF[j] * (sWP[j] + sWP[kTile + j] + sWP[2 * kTile + j] + sWP[3 * kTile + j]);
+        if (tid == 0) {
+          tc::tc_fence_after();
+          issue_values(n, x_started);
+        }
+        x_started = true;
+        wait_mma();
+      }
+      __syncthreads();
+      if (*sAbort) goto done;
+    }
+  }
+
+  // ---- top-P over the importance (descending, ties to the lower index) ----
+  {
+    const int P = a.P;
+    for (int j = tid; j < M0; j += 128) {
+      const float wj = sW[j];
+      int rank = 0;
+      for (int l = 0; l < M0; ++l) {
+        const float wl = sW[l];
+        rank += (wl > wj) || (wl == wj && l < j);
+      }
+      if (rank < P) sSEL[rank] = j;
+      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + j] = wj;
+    }
+    __syncthreads();
+    if (a.sel)
+      for (int r = tid; r < P; r += 128) a.sel[((size_t)bh * a.nblk + blk) * P + r] = sSEL[r];
+  }
+
+  // ---- child refinement in chunks of 16 selected parents ----
+  if (a.C > 0 && a.P > 0) {
+    float mref = m;
+    const int nch = (a.P + kChunkParents - 1) / kChunkParents;
+    for (int q = 0; q < nch; ++q) {
+      // an odd number of parents is padded with a copy of the last one (masked
+      // as empty) so that the MMA N stays a multiple of 16
+      const int np = min(kChunkParents, a.P - q * kChunkParents);
+      const int slots = (np + 1) & ~1;
+      const int n = slots * 8;
+      if (tid == 0) {
+        tc::mbar_arrive_expect_tx(bar_cp, 2u * slots * KH * 1024);
+        for (int r = 0; r < slots; ++r) {
+          const int p = sSEL[q * kChunkParents + min(r, np - 1)];
+          const size_t g = (size_t)(M0 / 8 + p) * KH * 512;
+          tc::bulk_g2s(sCW + r * KH * 1024, cw_h + g, KH * 1024, bar_cp);
+          tc::bulk_g2s(sVB + r * KH * 1024, vb_bh + g, KH * 1024, bar_cp);
+        }
+      }
+      for (int j = tid; j < n; j += 128) {
+        const int r = j >> 3;
+        sNF[j] = r < np ? (float)__ldg(cnt + M0 + sSEL[q * kChunkParents + r] * 8 + (j & 7)) : 0.f;
+      }
+      wait_cp();
+      __syncthreads();
+      if (*sAbort) goto done;
+      if (tid == 0) {
+        tc::tc_fence_after();
+        issue_logits(n);
+      }
+      wait_mma();
+      // row max over the non-empty children of the chunk
+      float cmax = NEG_INF;
+      for (int g = 0; g < n; g += 16) {
+        uint32_t r[16];
+        tc::tmem_ld16(tS + lane_off + g, r);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float tv = __uint_as_float(r[e]) * a.scale_log2;
+          if (sNF[g + e] > 0.f) cmax = fmaxf(cmax, tv);
+        }
+      }
+      // rare: a child logit far above the reference max -> rescale x and z
+      const bool need = cmax > mref + kRescaleLog2;
+      if (__any_sync(0xffffffffu, need)) {
+        const float f = need ? tc::ex2(mref - cmax) : 1.f;
+        for (int g = 0; g < D; g += 16) {
+          uint32_t r[16];
+          tc::tmem_ld16(tX + lane_off + g, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+          tc::tmem_st16(tX + lane_off + g, r);
+        }
+        tc::tmem_wait_st();
+        z *= f;
+        if (need) mref = cmax;
+      }
+      // dA = 2^(t_c - m) - 2^(t_p - m), t_p = mean of the parent's child logits
+      for (int g = 0; g < n; g += 16) {
+        uint32_t r[16];
+        tc::tmem_ld16(tS + lane_off + g, r);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          float tc8[8];
+          float tp = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            tc8[e] = __uint_as_float(r[s * 8 + e]) * a.scale_log2;
+            tp += tc8[e];
+          }
+          tp *= 0.125f;
+          const float ap = tc::ex2(tp - mref);
+          float da[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float nf = sNF[g + s * 8 + e];
+            da[e] = nf > 0.f ? tc::ex2(tc8[e] - mref) - ap : 0.f;
+            z = fmaf(da[e], nf, z);
+          }
+          const int col = g + s * 8;
+          uint4 u;
+          u.x = pack_bf16x2(da[0], da[1]);
+          u.y = pack_bf16x2(da[2], da[3]);
+          u.z = pack_bf16x2(da[4], da[5]);
+          u.w = pack_bf16x2(da[6], da[7]);
+          *reinterpret_cast<uint4*>(sPR + (col >> 6) * (kRows * 128) + tc::sw128_offset(tid, col & 63)) = u;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc::tc_fence_after();
+        issue_values(n, true);
+      }
+      wait_mma();
+      __syncthreads();
+      if (*sAbort) goto done;
+    }
+  }
+
+  // ---- O = x / z -> bf16 -> shared (Q region) -> TMA store ----
+  {
+    const float iz = 1.f / z;
+    for (int g = 0; g < D; g += 16) {
+      uint32_t r[16];
+      tc::tmem_ld16(tX + lane_off + g, r);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int col = g + s * 8;
+        uint4 u;
+        u.x = pack_bf16x2(__uint_as_float(r[s * 8 + 0]) * iz, __uint_as_float(r[s * 8 + 1]) * iz);
+        u.y = pack_bf16x2(__uint_as_float(r[s * 8 + 2]) * iz, __uint_as_float(r[s * 8 + 3]) * iz);
+        u.z = pack_bf16x2(__uint_as_float(r[s * 8 + 4]) * iz, __uint_as_float(r[s * 8 + 5]) * iz);
+        u.w = pack_bf16x2(__uint_as_float(r[s * 8 + 6]) * iz, __uint_as_float(r[s * 8 + 7]) * iz);
+        *reinterpret_cast<uint4*>(sQ + (col >> 6) * (kRows * 128) + tc::sw128_offset(tid, col & 63)) = u;
+      }
+    }
+    tc::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+      for (int kh = 0; kh < KH; ++kh) tc::tma_store_3d(&omap, sQ + kh * kRows * 128, kh * 64, row0, bh);
+      tc::bulk_commit_group();
+      tc::bulk_wait_group_read0();
+    }
+  }
+
+done:
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
+  (void)valid;
+}
+
+// Codewords and value sums -> bf16 images of swizzled atoms.  Code a of a head
+// (parents first, then child c of parent p at M0 + p*C + c) lands in atom
+// a/8, row a%8; for d = 128 each atom group holds two 64-column halves.
+template <int D>
+__global__ void __launch_bounds__(256) attention_prep_kernel(const bf16* __restrict__ parents,
+                                                             const bf16* __restrict__ children,
+                                                             const float* __restrict__ vsum,
+                                                             bf16* __restrict__ cw, bf16* __restrict__ vb,
+                                                             int H, int BH, int M0, int C) {
+  constexpr int KH = D / 64;
+  const int Mt = M0 * (1 + C);
+  const int chunks_per_code = D / 8;
+  const long long n_cw = (long long)H * Mt * chunks_per_code;
+  const long long n_vb = (long long)BH * Mt * chunks_per_code;
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < n_cw + n_vb;
+       g += (long long)gridDim.x * blockDim.x) {
+    const bool is_cw = g < n_cw;
+    const long long u = is_cw ? g : g - n_cw;
+    const int chunk = (int)(u % chunks_per_code);
+    const long long hc = u / chunks_per_code;
+    const int code = (int)(hc % Mt);
+    const long long head = hc / Mt;  // h for codewords, bh for value sums
+    float v[8];
+    if (is_cw) {
+      const bf16* src = code < M0 ? parents + ((size_t)head * M0 + code) * D
+                                  : children + ((size_t)head * M0 * C + (code - M0)) * D;
+      load8(src + chunk * 8, v);
+    } else {
+      load8(vsum + ((size_t)head * Mt + code) * D + chunk * 8, v);
+    }
+    const int kh = chunk >> 3, c = chunk & 7, r = code & 7;
+    bf16* dst = (is_cw ? cw : vb) + (((size_t)head * (Mt / 8) + (code >> 3)) * KH + kh) * 512 + r * 64 +
+                ((c ^ r) * 8);
+    store8(dst, v);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+bool attention_tc_supported(const Shape& s, avq_dtype dt, int P, int block, int /*two_pass*/) {
+  if (dt != AVQ_BF16 || block != 128) return false;
+  if (s.d != 64 && s.d != 128) return false;
+  if (s.M0 % 16 != 0 || s.M0 > 256) return false;
+  if (s.C != 0 && s.C != 8) return false;
+  (void)P;
+  return true;
+}
+
+size_t attention_tc_workspace(const Shape& s, int, int, int) {
+  return align256((size_t)s.H * s.Mt() * s.d * 2) + align256((size_t)s.BH() * s.Mt() * s.d * 2);
+}
+
+cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* parents,
+                                const void* children, const float* vsum, const int32_t* counts,
+                                int P, int block, float scale, int two_pass, void* O,
+                                int32_t* sel, float* importance, void* ws, unsigned int* err,
+                                cudaStream_t st, LaunchLog& log) {
+  (void)block;
+  bf16* cw = static_cast<bf16*>(ws);
+  bf16* vb = reinterpret_cast<bf16*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
+  const long long work = (long long)(s.H + s.BH()) * s.Mt() * (s.d / 8);
+  const int pblocks = (int)std::min<long long>((work + 255) / 256, (long long)num_sms() * 8);
+  if (s.d == 64)
+    attention_prep_kernel<64><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, vsum,
+                                                       cw, vb, s.H, s.BH(), s.M0, s.C);
+  else
+    attention_prep_kernel<128><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, vsum,
+                                                        cw, vb, s.H, s.BH(), s.M0, s.C);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  log.add("attention_prep");
+
+  CUtensorMap qmap, omap;
+  e = make_tmap_3d_bf16(&qmap, Q, s.d, s.N, s.BH(), 64, kRows);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_3d_bf16(&omap, O, s.d, s.N, s.BH(), 64, kRows);
+  if (e != cudaSuccess) return e;
+
+  AttnArgs a;
+  a.cw = cw;
+  a.vb = vb;
+  a.counts = counts;
+  a.sel = sel;
+  a.importance = importance;
+  a.err = err;
+  a.H = s.H;
+  a.N = s.N;
+  a.M0 = s.M0;
+  a.C = s.C;
+  a.P = P;
+  a.nblk = (s.N + kRows - 1) / kRows;
+  a.two_pass = two_pass;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid(a.nblk, s.BH());
+  if (s.d == 64) {
+    const int smem = Smem<64>::kTotal + 1024;
+    e = cudaFuncSetAttribute(attention_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attention_tc_kernel<64><<<grid, 128, smem, st>>>(qmap, omap, a);
+  } else {
+    const int smem = Smem<128>::kTotal + 1024;
+    e = cudaFuncSetAttribute(attention_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attention_tc_kernel<128><<<grid, 128, smem, st>>>(qmap, omap, a);
+  }
+  log.add("attention_tc");
+  return cudaGetLastError();
+}
+
 }  // namespace avq

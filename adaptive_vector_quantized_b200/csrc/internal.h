@@ -2,6 +2,7 @@
 // translation units.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -62,6 +63,11 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
 // ---- token permutation ----------------------------------------------------
 cudaError_t launch_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
                            int row_bytes, int inverse, cudaStream_t st, LaunchLog& log);
+
+// 3-D tiled TMA map over a bf16 tensor [batch][rows][inner] (inner contiguous),
+// box {box_inner, box_rows, 1}, 128-byte swizzle, zero fill out of bounds.
+cudaError_t make_tmap_3d_bf16(CUtensorMap* map, const void* base, int inner, int rows, int batch,
+                              int box_inner, int box_rows);
 
 // Device address of the current device's error word.
 unsigned int* error_word();

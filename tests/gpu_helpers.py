@@ -17,8 +17,10 @@ def to_dev(inp):
 
 
 def gpu_forward(inp, P=None, block=None, two_pass=None, path=avq.AVQ_PATH_AUTO,
-                deterministic=False, dev=None):
-    """Both stages on the GPU; returns CPU copies and the kernels launched."""
+                deterministic=False, dev=None, apath=None, scale=None):
+    """Both stages on the GPU; returns CPU copies and the kernels launched.
+    `path` selects the kernel family of both stages, `apath` overrides it for
+    the attention stage."""
     P = inp["P"] if P is None else P
     block = inp["block"] if block is None else block
     two_pass = inp.get("two_pass", False) if two_pass is None else two_pass
@@ -29,8 +31,10 @@ def gpu_forward(inp, P=None, block=None, two_pass=None, path=avq.AVQ_PATH_AUTO,
         assign, vsum, counts = avq.avq_quantize(d["K"], d["V"], d["parents"], ch,
                                                 deterministic=deterministic)
         k1 = avq.last_kernels()
+        avq.avq_set_path(path if apath is None else apath)
         O, sel, imp = avq.avq_attention(d["Q"], d["parents"], ch, vsum, counts, P, block,
-                                        scale=inp["scale"], two_pass=two_pass, importance=True)
+                                        scale=inp["scale"] if scale is None else scale,
+                                        two_pass=two_pass, importance=True)
         k2 = avq.last_kernels()
         avq.avq_check_device()
     finally:

@@ -69,6 +69,50 @@ def test_forward_parity(inputs, case, path):
     print(case, path, res["kernels"], diag)
 
 
+def _forward_tc_attention(inp, **kw):
+    try:
+        return gh.gpu_forward(inp, apath=avq.AVQ_PATH_TC, **kw)
+    except avq.AVQError as e:
+        if e.status == avq.AVQ_ERR_UNSUPPORTED:
+            pytest.skip("no tensor-core attention kernel for this case")
+        raise
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_forward_parity_tc_attention(inputs, case):
+    inp = inputs(case)
+    res = _forward_tc_attention(inp)
+    assert "attention_tc" in res["kernels"]
+    diag = gh.check_forward(inp, res)
+    print(case, "tc-attention", res["kernels"], diag)
+
+
+def test_tc_attention_rescale_path():
+    """Non-empty children whose logits exceed the parents' max by far more than
+    the reference-max margin: the TMEM rescale branch must reproduce the oracle."""
+    H, M0, C, d, N = 1, 16, 8, 64, 512
+    rng = np.random.default_rng(5)
+    par = np.zeros((H, M0, d), dtype=np.float32)
+    par[0, :, 1:] = np.rint(rng.standard_normal((M0, d - 1)) * 8) / 8
+    off = np.zeros((C, d), dtype=np.float32)
+    off[:, 0] = [4, -4, 3, -3, 2, -2, 1, -1]
+    ch = par[:, :, None, :] + off[None, None]
+    assert np.array_equal(ch.mean(2), par)
+    pick_p = rng.integers(0, M0, N)
+    pick_c = rng.integers(0, 2, N) * 2  # children 0 or 2: far along +e0
+    K = ch[0][pick_p, pick_c][None, None]
+    Q = np.zeros((1, H, N, d), dtype=np.float32)
+    Q[..., 0] = 16.0
+    Q[..., 1:] = np.rint(rng.standard_normal((N, d - 1)) * 4) / 16
+    V = rng.standard_normal((1, H, N, d)).astype(np.float32)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)  # noqa: E731
+    inp = dict(Q=t(Q), K=t(K), V=t(V), parents=t(par), children=t(ch), B=1, H=H, N=N, d=d,
+               M0=M0, C=C, P=4, block=128, scale=1.0, dtype="bf16", two_pass=False)
+    res = _forward_tc_attention(inp)
+    diag = gh.check_forward(inp, res)
+    print("rescale", res["kernels"], diag)
+
+
 @pytest.mark.parametrize("P,block", [(0, 128), (1, 64), (8, 128), (64, 64)])
 def test_vit_p_and_block_variants(inputs, P, block):
     inp = inputs("vit_h3")
