@@ -181,8 +181,8 @@ def avq_quantize(K, V, parents, children, assign=None, vsum=None, counts=None,
         vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
     if counts is None:
         counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
-    if deterministic and ws is None:
-        ws = workspace(dims, dt, dev, deterministic=True)
+    if ws is None:
+        ws = workspace(dims, dt, dev, deterministic=deterministic)
     wp, wn = _ws_ptr(ws)
     _check(lib().avq_quantize(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
                               _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),

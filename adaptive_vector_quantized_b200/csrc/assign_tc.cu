@@ -1,9 +1,355 @@
-// placeholder: tensor-core assignment kernel (added next)
+// Stage 1 assignment on the tcgen05 tensor cores ("AVQ-Attention: Adaptive
+// Vector-Quantized Attention", Sec. 4.2, Algorithm 1 steps 3-16).
+//
+// Persistent CTAs walk contiguous ranges of 128-key tiles.  Per tile:
+//   K tile      TMA (128B swizzle) into a two-slot ring, the next tile in
+//               flight while the current one is processed
+//   parents     D = K P^T on tcgen05 into TMEM (M = 128 keys, N = M0);
+//               thread r owns key r = TMEM lane r and takes the first
+//               minimum of |p|^2 - 2 k.p over the parents (|k|^2 is the same
+//               for every codeword of a key and is dropped)
+//   children    the C = 8 children of the chosen parent, read from a bf16
+//               image in shared memory (or L2 when it does not fit), dot
+//               products with bf16 x bf16 -> fp32 fused multiply-adds
+//               (exact products, fp32 accumulation); the key moves to the
+//               first strictly smallest child only if it is strictly closer
+//               than the parent
+//   output      assign[key] = parent, or M0 + parent*C + child
+// Codewords are first converted into the swizzled-atom image shared with
+// the attention kernel (8 codes x 64 dims per 1024-byte atom) plus their
+// squared norms in fp32.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tc_util.cuh"
+
 namespace avq {
-bool assign_tc_supported(const Shape&, avq_dtype) { return false; }
-cudaError_t launch_assign_tc(const Shape&, const void*, const void*, const void*, int32_t*,
-                             unsigned int*, cudaStream_t, LaunchLog&) {
-  return cudaErrorNotSupported;
+
+namespace {
+
+constexpr int kKeys = 128;
+
+struct AssignArgs {
+  const bf16* cw;      // [H][Mt/8][KH][8][64] swizzled codeword atoms
+  const float* norms;  // [H][Mt] squared norms
+  int32_t* assign;     // [BH][N]
+  unsigned int* err;
+  int H, N, M0, C, nblk, ntiles, tiles_per_cta;
+};
+
+// bf16 pair x bf16 pair accumulated into fp32 (two exact products, two roundings).
+__device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 t, a0, b0, %3;\n\t"
+      "fma.rn.f32.bf16 %0, a1, b1, t;\n\t}"
+      : "=f"(d)
+      : "r"(a), "r"(b), "f"(c));
+  return d;
 }
+
+template <int D, bool CH_SMEM>
+struct AssignSmem {
+  static constexpr int KH = D / 64;
+  // parents image | children image (optional) | K ring [2] | norms | barriers
+  __host__ __device__ static size_t parents_bytes(int M0) { return (size_t)M0 * D * 2; }
+  __host__ __device__ static size_t children_bytes(int M0, int C) { return CH_SMEM ? (size_t)M0 * C * D * 2 : 0; }
+  __host__ __device__ static size_t ring_off(int M0, int C) { return parents_bytes(M0) + children_bytes(M0, C); }
+  __host__ __device__ static size_t norms_off(int M0, int C) { return ring_off(M0, C) + 2 * kKeys * D * 2; }
+  __host__ __device__ static size_t bar_off(int M0, int C) {
+    return (norms_off(M0, C) + (size_t)M0 * (1 + C) * 4 + 15) & ~(size_t)15;
+  }
+  __host__ __device__ static size_t total(int M0, int C) { return bar_off(M0, C) + 64; }
+};
+
+template <int D, bool CH_SMEM>
+__global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                        const AssignArgs a) {
+  using S = AssignSmem<D, CH_SMEM>;
+  constexpr int KH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int M0 = a.M0, C = a.C, Mt = M0 * (1 + C);
+  uint8_t* sPar = sm;
+  uint8_t* sCh = sm + S::parents_bytes(M0);
+  uint8_t* sRing = sm + S::ring_off(M0, C);
+  float* sNorm = reinterpret_cast<float*>(sm + S::norms_off(M0, C));
+  uint64_t* bar_k = reinterpret_cast<uint64_t*>(sm + S::bar_off(M0, C));  // [2]
+  uint64_t* bar_cb = bar_k + 2;
+  uint64_t* bar_mma = bar_k + 3;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar_k + 4);
+  int* sAbort = reinterpret_cast<int*>(bar_k + 4) + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int t0 = blockIdx.x * a.tiles_per_cta;
+  const int t1 = min(a.ntiles, t0 + a.tiles_per_cta);
+  if (t0 >= t1) return;
+  const uint32_t ncols = M0 <= 32 ? 32 : M0 <= 64 ? 64 : M0 <= 128 ? 128 : 256;
+
+  if (tid == 0) {
+    tc::mbar_init(&bar_k[0], 1);
+    tc::mbar_init(&bar_k[1], 1);
+    tc::mbar_init(bar_cb, 1);
+    tc::mbar_init(bar_mma, 1);
+    tc::fence_mbar_init();
+    *sAbort = 0;
+    tc::prefetch_tensormap(&kmap);
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(sTmem, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+  auto issue_k = [&](int t, int slot) {
+    const int bh = t / a.nblk, blk = t % a.nblk;
+    tc::mbar_arrive_expect_tx(&bar_k[slot], kKeys * D * 2);
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh)
+      tc::tma_load_3d(sRing + slot * (kKeys * D * 2) + kh * (kKeys * 128), &kmap, kh * 64, blk * kKeys, bh,
+                      &bar_k[slot]);
+  };
+  if (tid == 0) {
+    issue_k(t0, 0);
+    if (t0 + 1 < t1) issue_k(t0 + 1, 1);
+  }
+
+  const uint32_t idesc = tc::idesc_bf16(kKeys, M0, 0, 0);
+  const uint32_t sParA = tc::smem_u32(sPar);
+  uint32_t ph_cb = 0, ph_mma = 0;
+  int cur_h = -1;
+  const float INF = __int_as_float(0x7f800000);
+
+  for (int t = t0; t < t1; ++t) {
+    const int it = t - t0, slot = it & 1;
+    const uint32_t ph_k = (it >> 1) & 1;
+    const int bh = t / a.nblk, blk = t % a.nblk, h = bh % a.H;
+    if (h != cur_h) {  // (re)load the head's codebook image and norms
+      if (tid == 0) {
+        const size_t bytes = S::parents_bytes(M0) + S::children_bytes(M0, C);
+        tc::mbar_arrive_expect_tx(bar_cb, (uint32_t)bytes);
+        const bf16* src = a.cw + (size_t)h * Mt * D;
+        // parents and (optionally) children are contiguous in the image
+        size_t off = 0;
+        while (off < bytes) {
+          const uint32_t part = (uint32_t)std::min<size_t>(bytes - off, 65536);
+          tc::bulk_g2s(sPar + off, reinterpret_cast<const uint8_t*>(src) + off, part, bar_cb);
+          off += part;
+        }
+      }
+      for (int j = tid; j < Mt; j += 128) sNorm[j] = __ldg(a.norms + (size_t)h * Mt + j);
+      if (!tc::mbar_wait(bar_cb, ph_cb)) {
+        atomicOr(a.err, kErrTimeout);
+        *sAbort = 1;
+      }
+      ph_cb ^= 1;
+      cur_h = h;
+      __syncthreads();
+    }
+    if (!tc::mbar_wait(&bar_k[slot], ph_k)) {
+      atomicOr(a.err, kErrTimeout);
+      *sAbort = 1;
+    }
+    __syncthreads();
+    if (*sAbort) break;
+    const uint8_t* sK = sRing + slot * (kKeys * D * 2);
+    if (tid == 0) {
+      tc::tc_fence_after();
+      const uint32_t sKa = tc::smem_u32(sK);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint64_t ad = tc::sdesc_sw128(sKa + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::sdesc_sw128(sParA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+        tc::mma_bf16(tmem, ad, bd, idesc, k > 0);
+      }
+      tc::mma_commit(bar_mma);
+    }
+    if (!tc::mbar_wait(bar_mma, ph_mma)) atomicOr(a.err, kErrTimeout);
+    ph_mma ^= 1;
+    tc::tc_fence_after();
+
+    // nearest parent: first minimum of |p|^2 - 2 k.p
+    float best = INF;
+    int par = 0;
+    for (int g = 0; g < M0; g += 16) {
+      uint32_t r[16];
+      tc::tmem_ld16(tmem + lane_off + g, r);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float dm = fmaf(-2.f, __uint_as_float(r[e]), sNorm[g + e]);
+        if (dm < best) {
+          best = dm;
+          par = g + e;
+        }
+      }
+    }
+    int code = par;
+    if (C > 0) {
+      // key row in registers, 16-byte chunks in rotated order
+      const int rot = tid & 7;
+      uint4 kq[KH][8];
+#pragma unroll
+      for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int lc = (s + rot) & 7;
+          kq[kh][s] = *reinterpret_cast<const uint4*>(sK + kh * (kKeys * 128) + tid * 128 + ((lc ^ rot) << 4));
+        }
+      float dchild = INF;
+      int cstar = 0;
+      const uint8_t* atom = CH_SMEM ? sCh + (size_t)par * (KH * 1024)
+                                    : reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + par * 8) * D);
+      for (int c = 0; c < C; ++c) {
+        float acc = 0.f;
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const int lc = (s + rot) & 7;
+            const uint8_t* p = atom + kh * 1024 + c * 128 + ((lc ^ c) << 4);
+            const uint4 cv = CH_SMEM ? *reinterpret_cast<const uint4*>(p)
+                                     : __ldg(reinterpret_cast<const uint4*>(p));
+            acc = fma_bf16x2(kq[kh][s].x, cv.x, acc);
+            acc = fma_bf16x2(kq[kh][s].y, cv.y, acc);
+            acc = fma_bf16x2(kq[kh][s].z, cv.z, acc);
+            acc = fma_bf16x2(kq[kh][s].w, cv.w, acc);
+          }
+        const float dc = fmaf(-2.f, acc, sNorm[M0 + par * C + c]);
+        if (dc < dchild) {
+          dchild = dc;
+          cstar = c;
+        }
+      }
+      if (dchild < best) code = M0 + par * C + cstar;
+    }
+    const int row = blk * kKeys + tid;
+    if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
+
+    tc::tc_fence_before();
+    __syncthreads();  // K slot and TMEM free
+    if (tid == 0 && t + 2 < t1) issue_k(t + 2, slot);
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, ncols);
+  }
+}
+
+// Codewords -> swizzled-atom image (code a in atom a/8, row a%8) and fp32
+// squared norms.  Children of parent p are codes M0 + p*C + c.
+template <int D>
+__global__ void __launch_bounds__(256) codebook_prep_kernel(const bf16* __restrict__ parents,
+                                                            const bf16* __restrict__ children,
+                                                            bf16* __restrict__ cw,
+                                                            float* __restrict__ norms, int H, int M0,
+                                                            int C) {
+  constexpr int KH = D / 64;
+  const int Mt = M0 * (1 + C);
+  const long long total = (long long)H * Mt;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int code = (int)(u % Mt);
+    const long long h = u / Mt;
+    const bf16* src = code < M0 ? parents + ((size_t)h * M0 + code) * D
+                                : children + ((size_t)h * M0 * C + (code - M0)) * D;
+    float nrm = 0.f;
+    const int r = code & 7;
+#pragma unroll
+    for (int chunk = 0; chunk < D / 8; ++chunk) {
+      float v[8];
+      load8(src + chunk * 8, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) nrm = fmaf(v[e], v[e], nrm);
+      const int kh = chunk >> 3, c = chunk & 7;
+      store8(cw + (((size_t)h * (Mt / 8) + (code >> 3)) * KH + kh) * 512 + r * 64 + ((c ^ r) * 8), v);
+    }
+    norms[u] = nrm;
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+template <int D, bool CH>
+cudaError_t launch_impl(const Shape& s, const CUtensorMap& kmap, AssignArgs a, cudaStream_t st) {
+  using S = AssignSmem<D, CH>;
+  const size_t smem = S::total(s.M0, s.C) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<D, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int per_sm = smem <= 110 * 1024 ? 2 : 1;
+  const int ctas = std::min(a.ntiles, num_sms() * per_sm);
+  a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
+  const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+  assign_tc_kernel<D, CH><<<grid, 128, smem, st>>>(kmap, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool assign_tc_supported(const Shape& s, avq_dtype dt) {
+  if (dt != AVQ_BF16) return false;
+  if (s.d != 64 && s.d != 128) return false;
+  if (s.M0 % 16 != 0 || s.M0 > 256) return false;
+  if (s.C != 0 && s.C != 8) return false;
+  return true;
+}
+
+size_t assign_tc_workspace(const Shape& s) {
+  return align256((size_t)s.H * s.Mt() * s.d * 2) + align256((size_t)s.H * s.Mt() * 4);
+}
+
+cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents, const void* children,
+                             int32_t* assign, void* ws, unsigned int* err, cudaStream_t st, LaunchLog& log) {
+  bf16* cw = static_cast<bf16*>(ws);
+  float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
+  const long long work = (long long)s.H * s.Mt();
+  const int pblocks = (int)std::max<long long>(1, std::min<long long>((work + 255) / 256, num_sms() * 4));
+  if (s.d == 64)
+    codebook_prep_kernel<64><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
+                                                      s.H, s.M0, s.C);
+  else
+    codebook_prep_kernel<128><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
+                                                       s.H, s.M0, s.C);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  log.add("codebook_prep");
+
+  CUtensorMap kmap;
+  e = make_tmap_3d_bf16(&kmap, K, s.d, s.N, s.BH(), 64, kKeys);
+  if (e != cudaSuccess) return e;
+  AssignArgs a;
+  a.cw = cw;
+  a.norms = norms;
+  a.assign = assign;
+  a.err = err;
+  a.H = s.H;
+  a.N = s.N;
+  a.M0 = s.M0;
+  a.C = s.C;
+  a.nblk = (s.N + kKeys - 1) / kKeys;
+  a.ntiles = a.nblk * s.BH();
+  a.tiles_per_cta = 1;
+  const size_t ch_bytes = (size_t)s.M0 * s.C * s.d * 2;
+  const bool ch_smem = ch_bytes <= 96 * 1024;
+  if (s.d == 64)
+    e = ch_smem ? launch_impl<64, true>(s, kmap, a, st) : launch_impl<64, false>(s, kmap, a, st);
+  else
+    e = ch_smem ? launch_impl<128, true>(s, kmap, a, st) : launch_impl<128, false>(s, kmap, a, st);
+  log.add(ch_smem ? "assign_tc" : "assign_tc_l2children");
+  return e;
+}
+
 }  // namespace avq

@@ -180,7 +180,8 @@ size_t avq_workspace_size(const avq_dims* dims, avq_dtype dtype, int determinist
   if (dims == nullptr) return 0;
   const Shape s = to_shape(dims);
   size_t need = 0;
-  if (deterministic) need = aggregate_det_workspace(s);
+  if (assign_tc_supported(s, dtype)) need += (assign_tc_workspace(s) + 255) & ~(size_t)255;
+  if (deterministic) need += aggregate_det_workspace(s);
   if (attention_tc_supported(s, dtype, P, block, two_pass)) {
     const size_t a = attention_tc_workspace(s, P, block, two_pass);
     if (a > need) need = a;
@@ -203,27 +204,31 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
   AVQ_REQUIRE_PTR(assign, "assign");
   AVQ_REQUIRE_PTR(vsum, "vsum");
   AVQ_REQUIRE_PTR(counts, "counts");
-  if (deterministic) {
-    st = check_ws(aggregate_det_workspace(s), ws, ws_bytes);
-    if (st != AVQ_OK) return st;
-  }
   const bool tc_ok = assign_tc_supported(s, dtype);
   if (t_path == AVQ_PATH_TC && !tc_ok)
     return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core assignment kernel for this shape/dtype");
   const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
+  // workspace: [tensor-core codebook image | deterministic reduction scratch]
+  const size_t ws_tc = use_tc ? (assign_tc_workspace(s) + 255) & ~(size_t)255 : 0;
+  const size_t ws_det = deterministic ? aggregate_det_workspace(s) : 0;
+  if (ws_tc + ws_det > 0) {
+    st = check_ws(ws_tc + ws_det, ws, ws_bytes);
+    if (st != AVQ_OK) return st;
+  }
+  void* ws_det_ptr = ws_det ? static_cast<char*>(ws) + ws_tc : nullptr;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   LaunchLog log{};
   cudaError_t e;
   if (use_tc) {
     unsigned int* err = error_word();
     if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
-    e = launch_assign_tc(s, K, parents, children, assign, err, cs, log);
+    e = launch_assign_tc(s, K, parents, children, assign, ws, err, cs, log);
   } else {
     e = launch_assign_simt(s, dtype, K, parents, children, assign, cs, log);
   }
   if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
   if (deterministic)
-    e = launch_aggregate_det(s, dtype, V, assign, vsum, counts, ws, cs, log);
+    e = launch_aggregate_det(s, dtype, V, assign, vsum, counts, ws_det_ptr, cs, log);
   else
     e = launch_aggregate(s, dtype, V, assign, vsum, counts, cs, log);
   if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");

@@ -40,10 +40,12 @@ cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
                                  const int32_t* assign, float* vsum, int32_t* counts, void* ws,
                                  cudaStream_t st, LaunchLog& log);
 
-// tcgen05 assignment kernel (bf16, d in {64,128}, M0 a multiple of 16 up to 256).
+// tcgen05 assignment kernel (bf16, d in {64,128}, M0 a multiple of 16 up to 256,
+// C in {0, 8}); needs assign_tc_workspace(s) bytes of workspace.
 bool assign_tc_supported(const Shape& s, avq_dtype dt);
+size_t assign_tc_workspace(const Shape& s);
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
-                             const void* children, int32_t* assign, unsigned int* err,
+                             const void* children, int32_t* assign, void* ws, unsigned int* err,
                              cudaStream_t st, LaunchLog& log);
 
 // ---- stage 2 ------------------------------------------------------------

@@ -251,36 +251,43 @@ def run_avq(args, cfg, inp):
     sel = torch.empty((B, H, nblk, max(P, 1)), dtype=torch.int32, device=dev)
 
     def step():
-        avq.avq_quantize(K, V, par, ch, assign, vsum, counts, stream=stream)
+        avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
         k1 = avq.last_kernels()
         avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
                           ws=ws, stream=stream)
         return k1, avq.last_kernels()
 
-    for _ in range(args.warmup):
-        k1, k2 = step()
-    avq.avq_check_device(stream)
-    kernels_per_step = len(k1.split()) + len(k2.split())
-
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
+        wall0 = time.time()
+        for _ in range(args.warmup):
+            k1, k2 = step()
+        avq.avq_check_device(stream)
+        kernels_per_step = len(k1.split()) + len(k2.split())
+        # untimed soak so that the clock sampler sees the GPU under this load
+        soak = 0
+        while time.time() - wall0 < 1.0:
+            step()
+            soak += 1
+            if soak % 32 == 0:
+                torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
         t0.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
-            avq.avq_quantize(K, V, par, ch, assign, vsum, counts, stream=stream)
+            avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
             ev[s][1].record(stream)
             avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
                               ws=ws, stream=stream)
             ev[s][2].record(stream)
         t1.record(stream)
         torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+        if world > 1:
+            dist.barrier()
     avq.avq_check_device(stream)
     ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
     t_s1 = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
@@ -363,7 +370,8 @@ def run_avq(args, cfg, inp):
                             "inputs smaller than L2; no flush"),
                 roofline=roofline, cpu_baseline=cpu, e2e=e2e,
                 gpu_launches=kernels_per_step * args.steps,
-                clocks=clk.summary(),
+                clocks=dict(clk.summary() or {}, window=f"sampled every 200 ms over warmup, "
+                            f"{soak} untimed soak steps and the timed steps"),
                 stages=dict(quantize_us=t_s1 * 1e3, attention_us=t_s2 * 1e3,
                             quantize_gbs=s1_gbs, attention_gbs=s2_gbs, attention_tflops=s2_tfs,
                             quantize_kernels=k1, attention_kernels=k2))

@@ -79,6 +79,21 @@ def _forward_tc_attention(inp, **kw):
 
 
 @pytest.mark.parametrize("case", list(CASES))
+def test_forward_parity_tc_both(inputs, case):
+    """Both stages forced onto the tcgen05 kernels."""
+    inp = inputs(case)
+    try:
+        res = gh.gpu_forward(inp, path=avq.AVQ_PATH_TC)
+    except avq.AVQError as e:
+        if e.status == avq.AVQ_ERR_UNSUPPORTED:
+            pytest.skip("no tensor-core kernel for this case")
+        raise
+    assert "assign_tc" in res["kernels"] and "attention_tc" in res["kernels"]
+    diag = gh.check_forward(inp, res)
+    print(case, "tc-both", res["kernels"], diag)
+
+
+@pytest.mark.parametrize("case", list(CASES))
 def test_forward_parity_tc_attention(inputs, case):
     inp = inputs(case)
     res = _forward_tc_attention(inp)
