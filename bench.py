@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=None)
+    ap.add_argument("--profile", action="store_true",
+                    help="for profiler runs: no clock soak, no end-to-end leg, no CPU baseline")
     return ap.parse_args()
 
 
@@ -268,7 +270,7 @@ def run_avq(args, cfg, inp):
         kernels_per_step = len(k1.split()) + len(k2.split())
         # untimed soak so that the clock sampler sees the GPU under this load
         soak = 0
-        while time.time() - wall0 < 1.0:
+        while not args.profile and time.time() - wall0 < 1.0:
             step()
             soak += 1
             if soak % 32 == 0:
@@ -298,7 +300,7 @@ def run_avq(args, cfg, inp):
 
     # end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.profile:
         hQ, hK, hV = (inp[k].pin_memory() for k in ("Q", "K", "V"))
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
         hsel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
@@ -355,7 +357,7 @@ def run_avq(args, cfg, inp):
                     step_roofline_us=t_roof * 1e6, step_frac=t_roof * 1e3 / ms_step)
 
     cpu = None
-    if not args.no_cpu_baseline and world == 1:  # rank 0 at N=1 only
+    if not args.no_cpu_baseline and not args.profile and world == 1:  # rank 0 at N=1 only
         heads = min(cfg["H"], max(1, os.cpu_count() or 1))
         q, times, cores = cpu_oracle_sample(inp, heads, steps=1)
         cpu = dict(value=q / times[0], unit="queries/s", cores=cores, kind="oracle",
