@@ -19,6 +19,7 @@
 // fixed order.  Nothing depends on the grid or the GPU's size.
 #include "common.cuh"
 #include "internal.h"
+#include "tc_util.cuh"
 
 namespace avq {
 
@@ -124,6 +125,138 @@ __global__ void __launch_bounds__(kAggThreads) aggregate_kernel(
     for (int r = threadIdx.x; r < Mt; r += blockDim.x)
       if (cnt[r] > 0) atomicAdd(gcnt + r, cnt[r]);
   }
+}
+
+// Ring variant: one CTA per chunk of keys of one head, 16 warps.  Value rows
+// stream through a two-slot shared-memory ring filled by 1-D bulk copies
+// (the next tile is in flight while the current one is consumed); each warp
+// takes 16 consecutive keys of a tile with lanes over the head dimension,
+// merges runs of equal codes in registers and flushes a run into the
+// per-CTA partials with shared-memory atomics only when the code changes.
+// Codes are prefetched one tile ahead into registers (lane u holds key u).
+constexpr int kRingThreads = 512;
+constexpr int kRingWarps = kRingThreads / 32;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kRingThreads) aggregate_ring_kernel(
+    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
+    int32_t* __restrict__ counts, int N, int M0, int C, int chunk, int tile, unsigned int* err) {
+  extern __shared__ __align__(128) uint8_t smraw[];
+  constexpr int E = D / 32;
+  constexpr int RB = D * (int)sizeof(T);  // bytes per value row
+  const int bh = blockIdx.y;
+  const int Mt = M0 * (1 + C);
+  float* part = reinterpret_cast<float*>(smraw);
+  int* cnt = reinterpret_cast<int*>(part + (size_t)Mt * D);
+  uint8_t* ring = reinterpret_cast<uint8_t*>(((uintptr_t)(cnt + Mt) + 127) & ~(uintptr_t)127);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + 2 * (size_t)tile * RB);  // [2]
+  int* sAbort = reinterpret_cast<int*>(full + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k0 = blockIdx.x * chunk;
+  const int k1 = min(N, k0 + chunk);
+  if (k0 >= k1) return;
+  const int ntile = (k1 - k0 + tile - 1) / tile;
+  const T* vb = V + (size_t)bh * N * D;
+  const int32_t* asg = assign + (size_t)bh * N;
+
+  {
+    float4* s4 = reinterpret_cast<float4*>(part);
+    for (int i = tid; i < Mt * D / 4; i += blockDim.x) s4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = tid; i < Mt; i += blockDim.x) cnt[i] = 0;
+  }
+  if (tid == 0) {
+    tc::mbar_init(&full[0], 1);
+    tc::mbar_init(&full[1], 1);
+    tc::fence_mbar_init();
+    *sAbort = 0;
+  }
+  __syncthreads();
+  auto issue = [&](int t) {
+    const int j0 = k0 + t * tile;
+    const int nk = min(tile, k1 - j0);
+    const int slot = t & 1;
+    tc::mbar_arrive_expect_tx(&full[slot], (uint32_t)nk * RB);
+    tc::bulk_g2s(ring + (size_t)slot * tile * RB, vb + (size_t)j0 * D, (uint32_t)nk * RB, &full[slot]);
+  };
+  if (tid == 0) {
+    issue(0);
+    if (ntile > 1) issue(1);
+  }
+  const int per_warp = tile / kRingWarps;  // 16 keys
+  auto load_codes = [&](int t) {
+    const int j = k0 + t * tile + warp * per_warp + lane;
+    return (lane < per_warp && t < ntile && j < k1) ? __ldg(asg + j) : -1;
+  };
+  int codes = load_codes(0);
+  float accP[E], accC[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
+  int curP = -1, curC = -1, nP = 0, nC = 0;
+  for (int t = 0; t < ntile; ++t) {
+    const int slot = t & 1;
+    const int next = load_codes(t + 1);
+    if (!tc::mbar_wait(&full[slot], (t >> 1) & 1)) *sAbort = 1;
+    const uint8_t* rows = ring + (size_t)slot * tile * RB + (size_t)warp * per_warp * RB + lane * E * sizeof(T);
+    for (int u = 0; u < per_warp; ++u) {
+      const int c = __shfl_sync(0xffffffffu, codes, u);
+      if (c < 0) break;
+      float v[E];
+      if constexpr (sizeof(T) == 2) {
+        if constexpr (E == 2) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + (size_t)u * RB);
+          v[0] = bf16_lo(w); v[1] = bf16_hi(w);
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(rows + (size_t)u * RB);
+          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = reinterpret_cast<const float*>(rows + (size_t)u * RB)[e];
+      }
+      const int p = c < M0 ? c : (c - M0) / C;
+      if (p != curP) {
+        if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
+        curP = p;
+        nP = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) accP[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) accP[e] += v[e];
+      ++nP;
+      if (c >= M0) {
+        if (c != curC) {
+          if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
+          curC = c;
+          nC = 0;
+#pragma unroll
+          for (int e = 0; e < E; ++e) accC[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) accC[e] += v[e];
+        ++nC;
+      }
+    }
+    codes = next;
+    __syncthreads();  // slot consumed by every warp
+    if (tid == 0 && t + 2 < ntile) issue(t + 2);
+  }
+  if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
+  if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
+  __syncthreads();
+  float* gvs = vsum + (size_t)bh * Mt * D;
+  int* gcnt = counts + (size_t)bh * Mt;
+  const float4* s4 = reinterpret_cast<const float4*>(part);
+  for (int i = tid; i < Mt * D / 4; i += blockDim.x) {
+    const int row = i / (D / 4);
+    if (cnt[row] > 0) {
+      const float4 a4 = s4[i];
+      red_add_v4(gvs + (size_t)4 * i, a4.x, a4.y, a4.z, a4.w);
+    }
+  }
+  for (int r = tid; r < Mt; r += blockDim.x)
+    if (cnt[r] > 0) atomicAdd(gcnt + r, cnt[r]);
+  if (tid == 0 && *sAbort) atomicOr(err, kErrTimeout);
 }
 
 // ---- deterministic variant ------------------------------------------------
@@ -308,41 +441,59 @@ size_t aggregate_det_workspace(const Shape& s) {
 }
 
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
-                             float* vsum, int32_t* counts, cudaStream_t st, LaunchLog& log) {
+                             float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
+                             LaunchLog& log) {
   cudaError_t e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * s.Mt() * s.d * sizeof(float), st);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
-  const size_t smem = agg_smem_bytes(s);
-  const bool use_smem = smem <= 200 * 1024;
-  // about one resident CTA per SM in total; chunks are whole warps' worth of keys
   const int sms = num_sms();
-  int per_head = sms >= s.BH() ? sms / s.BH() : 1;  // a single wave where possible
-  if (!use_smem) per_head *= 4;
+  const size_t part = agg_smem_bytes(s);
+  const size_t row_bytes = (size_t)s.d * (dt == AVQ_F32 ? 4 : 2);
+  // ring variant: partials + two value tiles of `tile` keys (+ alignment, barriers)
+  int tile = 256;
+  while (tile >= kRingWarps && part + 128 + 2 * tile * row_bytes + 64 > 220 * 1024) tile /= 2;
+  if (tile >= kRingWarps && err != nullptr) {
+    const size_t smem = part + 128 + 2 * tile * row_bytes + 64;
+    int per_head = sms >= s.BH() ? sms / s.BH() : 1;
+    int chunk = (s.N + per_head - 1) / per_head;
+    chunk = ((chunk + tile - 1) / tile) * tile;
+    dim3 grid((s.N + chunk - 1) / chunk, s.BH());
+#define AVQ_RING(T, D)                                                                             \
+  do {                                                                                             \
+    auto kern = aggregate_ring_kernel<T, D>;                                                       \
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);        \
+    if (e != cudaSuccess) return e;                                                                \
+    kern<<<grid, kRingThreads, smem, st>>>((const T*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk, \
+                                           tile, err);                                             \
+  } while (0)
+    if (dt == AVQ_F32) {
+      if (s.d == 64) AVQ_RING(float, 64); else AVQ_RING(float, 128);
+    } else {
+      if (s.d == 64) AVQ_RING(bf16, 64); else AVQ_RING(bf16, 128);
+    }
+#undef AVQ_RING
+    log.add("aggregate_ring");
+    return cudaGetLastError();
+  }
+  // partials too large for shared memory: runs flushed straight to global memory
+  int per_head = (sms >= s.BH() ? sms / s.BH() : 1) * 4;
   int chunk = (s.N + per_head - 1) / per_head;
   chunk = ((chunk + 511) / 512) * 512;
   if (chunk < 512) chunk = 512;
   dim3 grid((s.N + chunk - 1) / chunk, s.BH());
-#define AVQ_AGG(T, D, SM)                                                                      \
-  do {                                                                                         \
-    auto kern = aggregate_kernel<T, D, SM>;                                                    \
-    if (SM) {                                                                                  \
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);  \
-      if (e != cudaSuccess) return e;                                                          \
-    }                                                                                          \
-    kern<<<grid, kAggThreads, SM ? smem : 0, st>>>((const T*)V, assign, vsum, counts, s.N,     \
-                                                   s.M0, s.C, chunk);                          \
-  } while (0)
-#define AVQ_AGG_D(T, SM) \
-  if (s.d == 64) AVQ_AGG(T, 64, SM); else AVQ_AGG(T, 128, SM)
   if (dt == AVQ_F32) {
-    if (use_smem) AVQ_AGG_D(float, true); else AVQ_AGG_D(float, false);
+    if (s.d == 64)
+      aggregate_kernel<float, 64, false><<<grid, kAggThreads, 0, st>>>((const float*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
+    else
+      aggregate_kernel<float, 128, false><<<grid, kAggThreads, 0, st>>>((const float*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
   } else {
-    if (use_smem) AVQ_AGG_D(bf16, true); else AVQ_AGG_D(bf16, false);
+    if (s.d == 64)
+      aggregate_kernel<bf16, 64, false><<<grid, kAggThreads, 0, st>>>((const bf16*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
+    else
+      aggregate_kernel<bf16, 128, false><<<grid, kAggThreads, 0, st>>>((const bf16*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
   }
-#undef AVQ_AGG_D
-#undef AVQ_AGG
-  log.add(use_smem ? "aggregate_smem" : "aggregate_global");
+  log.add("aggregate_global");
   return cudaGetLastError();
 }
 

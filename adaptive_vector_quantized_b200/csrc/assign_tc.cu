@@ -177,24 +177,45 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     ph_mma ^= 1;
     tc::tc_fence_after();
 
-    // nearest parent: first minimum of |p|^2 - 2 k.p
+    // nearest parent: first minimum of |p|^2 - 2 k.p; four independent running
+    // minima over interleaved 16-column groups, merged in index order
     float best = INF;
     int par = 0;
-    for (int g = 0; g < M0; g += 16) {
-      uint32_t r[16];
-      tc::tmem_ld16(tmem + lane_off + g, r);
-      tc::tmem_wait_ld();
+    for (int g0 = 0; g0 < M0; g0 += 64) {
+      uint32_t r[64];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float dm = fmaf(-2.f, __uint_as_float(r[e]), sNorm[g + e]);
-        if (dm < best) {
-          best = dm;
-          par = g + e;
-        }
+      for (int q = 0; q < 4; ++q)
+        if (g0 + q * 16 < M0) tc::tmem_ld16(tmem + lane_off + g0 + q * 16, r + q * 16);
+      tc::tmem_wait_ld();
+      float bq[4];
+      int iq[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        bq[q] = INF;
+        iq[q] = 0;
       }
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int m = g0 + q * 16 + e;
+          if (m < M0) {
+            const float dm = fmaf(-2.f, __uint_as_float(r[q * 16 + e]), sNorm[m]);
+            if (dm < bq[q]) {
+              bq[q] = dm;
+              iq[q] = m;
+            }
+          }
+        }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (bq[q] < best) {
+          best = bq[q];
+          par = iq[q];
+        }
     }
     int code = par;
-    if (C > 0) {
+    if (C > 0) {  // C == 8 on this path
       // key row in registers, 16-byte chunks in rotated order
       const int rot = tid & 7;
       uint4 kq[KH][8];
@@ -205,32 +226,39 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
           const int lc = (s + rot) & 7;
           kq[kh][s] = *reinterpret_cast<const uint4*>(sK + kh * (kKeys * 128) + tid * 128 + ((lc ^ rot) << 4));
         }
-      float dchild = INF;
-      int cstar = 0;
       const uint8_t* atom = CH_SMEM ? sCh + (size_t)par * (KH * 1024)
                                     : reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + par * 8) * D);
-      for (int c = 0; c < C; ++c) {
-        float acc = 0.f;
+      // eight independent dot products (one per child)
+      float acc[8];
 #pragma unroll
-        for (int kh = 0; kh < KH; ++kh)
+      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const int lc = (s + rot) & 7;
+      for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int lc = (s + rot) & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
             const uint8_t* p = atom + kh * 1024 + c * 128 + ((lc ^ c) << 4);
             const uint4 cv = CH_SMEM ? *reinterpret_cast<const uint4*>(p)
                                      : __ldg(reinterpret_cast<const uint4*>(p));
-            acc = fma_bf16x2(kq[kh][s].x, cv.x, acc);
-            acc = fma_bf16x2(kq[kh][s].y, cv.y, acc);
-            acc = fma_bf16x2(kq[kh][s].z, cv.z, acc);
-            acc = fma_bf16x2(kq[kh][s].w, cv.w, acc);
+            acc[c] = fma_bf16x2(kq[kh][s].x, cv.x, acc[c]);
+            acc[c] = fma_bf16x2(kq[kh][s].y, cv.y, acc[c]);
+            acc[c] = fma_bf16x2(kq[kh][s].z, cv.z, acc[c]);
+            acc[c] = fma_bf16x2(kq[kh][s].w, cv.w, acc[c]);
           }
-        const float dc = fmaf(-2.f, acc, sNorm[M0 + par * C + c]);
+        }
+      float dchild = INF;
+      int cstar = 0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float dc = fmaf(-2.f, acc[c], sNorm[M0 + par * 8 + c]);
         if (dc < dchild) {
           dchild = dc;
           cstar = c;
         }
       }
-      if (dchild < best) code = M0 + par * C + cstar;
+      if (dchild < best) code = M0 + par * 8 + cstar;
     }
     const int row = blk * kKeys + tid;
     if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;

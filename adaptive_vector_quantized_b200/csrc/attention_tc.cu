@@ -40,7 +40,7 @@ namespace avq {
 namespace {
 
 constexpr int kRows = 128;          // queries per block (MMA M)
-constexpr int kTile = 128;          // parent codes per tile / child codes per chunk
+constexpr int kTile = 64;           // parent codes per tile / child codes per chunk
 constexpr int kChunkParents = kTile / 8;
 constexpr float kRescaleLog2 = 24.f;
 
@@ -58,18 +58,19 @@ struct AttnArgs {
 // shared memory plan (bytes); every operand region 1024-aligned
 template <int D>
 struct Smem {
-  static constexpr int KH = D / 64;
   static constexpr int kQ = 0;                              // Q tile / O staging
-  static constexpr int kCW = kQ + kRows * D * 2;            // codeword tile
-  static constexpr int kVB = kCW + kTile * D * 2;           // value-sum tile
-  static constexpr int kPR = kVB + kTile * D * 2;           // probabilities [2][128][64]
+  static constexpr int kCW = kQ + kRows * D * 2;            // codeword tile (64 codes)
+  static constexpr int kVB = kCW + kTile * D * 2;           // value-sum tile (64 codes)
+  static constexpr int kPR = kVB + kTile * D * 2;           // probabilities [128][64] bf16
   static constexpr int kNF = kPR + kRows * kTile * 2;       // counts of the tile (float)
-  static constexpr int kW = kNF + kTile * 4;                // importance [256]
+  static constexpr int kBI = kNF + kTile * 4;               // mask bias of the tile (0 / -inf)
+  static constexpr int kW = kBI + kTile * 4;                // importance [256]
   static constexpr int kWP = kW + 256 * 4;                  // per-warp partial sums [4][kTile]
   static constexpr int kSEL = kWP + 4 * kTile * 4;          // selected parents [256]
   static constexpr int kBAR = kSEL + 256 * 4;               // 3 mbarriers
   static constexpr int kMISC = kBAR + 32;                   // tmem base, abort flag
   static constexpr int kTotal = kMISC + 32;
+  static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
 };
 
 __device__ __forceinline__ void fail(unsigned int* err, int* abort_flag) {
@@ -79,7 +80,7 @@ __device__ __forceinline__ void fail(unsigned int* err, int* abort_flag) {
 
 // Butterfly reduce-scatter of 32 per-lane values: lane L returns the warp sum
 // of element L.
-__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+__device__ __forceinline__ float reduce_scatter32(float* v, int lane) {
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) {
 #pragma unroll
@@ -93,8 +94,26 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
   return v[0];
 }
 
+__device__ __forceinline__ void store_chunk8(uint8_t* tile, int row, int col, const float* v) {
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]);
+  u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]);
+  u.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(tile + (col >> 6) * (kRows * 128) + tc::sw128_offset(row, col & 63)) = u;
+}
+
+// 64 TMEM columns of this thread's row -> registers.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
+  tc::tmem_ld16(taddr, r);
+  tc::tmem_ld16(taddr + 16, r + 16);
+  tc::tmem_ld16(taddr + 32, r + 32);
+  tc::tmem_ld16(taddr + 48, r + 48);
+  tc::tmem_wait_ld();
+}
+
 template <int D>
-__global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+__global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                                                            const __grid_constant__ CUtensorMap omap,
                                                            const AttnArgs a) {
   using S = Smem<D>;
@@ -106,6 +125,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
   uint8_t* sVB = sm + S::kVB;
   uint8_t* sPR = sm + S::kPR;
   float* sNF = reinterpret_cast<float*>(sm + S::kNF);
+  float* sBI = reinterpret_cast<float*>(sm + S::kBI);
   float* sW = reinterpret_cast<float*>(sm + S::kW);
   float* sWP = reinterpret_cast<float*>(sm + S::kWP);
   int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
@@ -124,6 +144,8 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
   const bf16* cw_h = a.cw + (size_t)h * groups * KH * 512;
   const bf16* vb_bh = a.vb + (size_t)bh * groups * KH * 512;
   const int32_t* cnt = a.counts + (size_t)bh * Mt;
+  const float NEG_INF = __int_as_float(0xff800000);
+  const float sl2 = a.scale_log2;
 
   if (tid == 0) {
     tc::mbar_init(bar_q, 1);
@@ -135,7 +157,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
     tc::prefetch_tensormap(&omap);
   }
   if (warp == 0) {
-    tc::tmem_alloc(sTmem, 256);
+    tc::tmem_alloc(sTmem, S::kTmemCols);
     tc::tmem_relinquish();
   }
   for (int j = tid; j < M0; j += 128) sW[j] = 0.f;
@@ -143,8 +165,8 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *sTmem;
-  const uint32_t tS = tmem;          // logits, up to 128 columns
-  const uint32_t tX = tmem + 128;    // output accumulator, D columns
+  const uint32_t tS = tmem;          // logits, 64 columns
+  const uint32_t tX = tmem + kTile;  // output accumulator, D columns
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
   uint32_t ph_cp = 0, ph_mma = 0;
@@ -157,7 +179,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
   const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
   const uint32_t sQa = tc::smem_u32(sQ), sCWa = tc::smem_u32(sCW), sVBa = tc::smem_u32(sVB),
                  sPRa = tc::smem_u32(sPR);
-  // issue S = Q * CW^T (n codes) -- one thread
+  // S = Q * CW^T over n codes (n a multiple of 16, <= 64) -- one thread
   auto issue_logits = [&](int n) {
     const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
 #pragma unroll
@@ -168,11 +190,10 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
     }
     tc::mma_commit(bar_mma);
   };
-  // issue x += PR * VB (n codes) -- one thread
+  // x += PR * VB over n codes -- one thread
   auto issue_values = [&](int n, bool acc) {
-#pragma unroll 1
     for (int k = 0; k < n / 16; ++k) {
-      const uint64_t ad = tc::sdesc_sw128(sPRa + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16, 1024);
+      const uint64_t ad = tc::sdesc_sw128(sPRa + (k & 3) * 32, 16, 1024);
       const uint64_t bd = tc::sdesc_sw128(sVBa + k * 2 * (KH * 1024), 1024, KH * 1024);
       tc::mma_bf16(tX, ad, bd, idesc_x, (acc || k > 0) ? 1u : 0u);
     }
@@ -188,26 +209,30 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
     ph_cp ^= 1;
   };
 
-  const float NEG_INF = __int_as_float(0xff800000);
   float m = NEG_INF, z = 0.f;
   const int nT = (M0 + kTile - 1) / kTile;
   const int sweeps = (a.two_pass || nT > 1) ? 2 : 1;
   bool x_started = false;
   bool q_ready = false;
 
+  // ---- parents: one sweep (all parents in one tile) or two (running max and
+  //      denominator first, then probabilities, values and importance) ----
   for (int sweep = 0; sweep < sweeps; ++sweep) {
     const bool last = sweep == sweeps - 1;
     for (int t = 0; t < nT; ++t) {
       const int c0 = t * kTile;
       const int n = min(kTile, M0 - c0);
-      // bring the codeword tile (and its value sums on the last sweep)
       if (tid == 0) {
         const uint32_t cwb = (uint32_t)n * D * 2;
         tc::mbar_arrive_expect_tx(bar_cp, last ? 2 * cwb : cwb);
         tc::bulk_g2s(sCW, cw_h + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
         if (last) tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
       }
-      for (int j = tid; j < n; j += 128) sNF[j] = (float)__ldg(cnt + c0 + j);
+      for (int j = tid; j < kTile; j += 128) {
+        const float nf = j < n ? (float)__ldg(cnt + c0 + j) : 0.f;
+        sNF[j] = nf;
+        sBI[j] = nf > 0.f ? 0.f : NEG_INF;
+      }
       if (!q_ready) {
         if (!tc::mbar_wait(bar_q, 0)) fail(a.err, sAbort);
         q_ready = true;
@@ -220,91 +245,61 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
         issue_logits(n);
       }
       wait_mma();
-      // pass over the row's logits in groups of 32 columns
       {
+        uint32_t r[64];
+        tmem_ld64(tS + lane_off, r);
+        // t = scaled log2 logit, -inf for empty codes (and columns >= n)
         float tmax = NEG_INF;
-        if (sweeps == 1 || !last) {
-          for (int g = 0; g < n; g += 16) {
-            uint32_t r[16];
-            tc::tmem_ld16(tS + lane_off + g, r);
-            tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float tv = __uint_as_float(r[e]) * a.scale_log2;
-              if (sNF[g + e] > 0.f) tmax = fmaxf(tmax, tv);
-            }
-          }
-          if (!last) {  // first sweep: online max and denominator
-            const float mn = fmaxf(m, tmax);
-            if (mn != NEG_INF) {
-              float zt = 0.f;
-              for (int g = 0; g < n; g += 16) {
-                uint32_t r[16];
-                tc::tmem_ld16(tS + lane_off + g, r);
-                tc::tmem_wait_ld();
+        for (int e = 0; e < 64; ++e) {
+          // select, not add: TMEM columns past the tile may hold stale bits
+          const float tv = sBI[e] == 0.f ? __uint_as_float(r[e]) * sl2 : NEG_INF;
+          r[e] = __float_as_uint(tv);
+          tmax = fmaxf(tmax, tv);
+        }
+        if (!last || sweeps == 1) {
+          const float mn = fmaxf(m, tmax);
+          if (mn != NEG_INF) {
+            float zt = 0.f;
+            if (sweeps == 1) {
+              // single sweep: keep A = 2^(t - m) in place
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const float nf = sNF[g + e];
-                  const float tv = __uint_as_float(r[e]) * a.scale_log2;
-                  zt += nf > 0.f ? nf * tc::ex2(tv - mn) : 0.f;
-                }
+              for (int e = 0; e < 64; ++e) {
+                const float av = tc::ex2(__uint_as_float(r[e]) - mn);
+                r[e] = __float_as_uint(av);
+                zt = fmaf(av, sNF[e], zt);
               }
-              z = z * tc::ex2(m - mn) + zt;
-              m = mn;
-            }
-          } else {  // single sweep: the tile holds every parent
-            m = tmax;
-            z = 0.f;
-            for (int g = 0; g < n; g += 16) {
-              uint32_t r[16];
-              tc::tmem_ld16(tS + lane_off + g, r);
-              tc::tmem_wait_ld();
+            } else {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float nf = sNF[g + e];
-                const float tv = __uint_as_float(r[e]) * a.scale_log2;
-                z += nf > 0.f ? nf * tc::ex2(tv - m) : 0.f;
-              }
+              for (int e = 0; e < 64; ++e) zt = fmaf(tc::ex2(__uint_as_float(r[e]) - mn), sNF[e], zt);
             }
+            z = z * tc::ex2(m - mn) + zt;
+            m = mn;
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) r[e] = __float_as_uint(tc::ex2(__uint_as_float(r[e]) - m));
         }
         if (last) {
-          // A = 2^(t - m) (masked), bf16 -> probabilities, importance sums
+          // probabilities as bf16, importance column sums of A / z in fp32
           const float rz = valid ? 1.f / z : 0.f;
-          for (int g = 0; g < n; g += 32) {
-            float v[32];
-            uint32_t r[32];
-            tc::tmem_ld16(tS + lane_off + g, r);
-            tc::tmem_ld16(tS + lane_off + g + 16, r + 16);
-            tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float tv = __uint_as_float(r[e]) * a.scale_log2;
-              v[e] = (g + e < n && sNF[g + e] > 0.f) ? tc::ex2(tv - m) : 0.f;
-            }
-            // probabilities (row tid, codes g..g+31) as four 16-byte chunks
+          for (int q = 0; q < 8; ++q) store_chunk8(sPR, tid, q * 8, reinterpret_cast<const float*>(r) + q * 8);
+          float v[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int col = g + q * 8;
-              uint4 u;
-              u.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-              u.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-              u.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-              u.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-              *reinterpret_cast<uint4*>(sPR + (col >> 6) * (kRows * 128) + tc::sw128_offset(tid, col & 63)) = u;
-            }
+          for (int hgrp = 0; hgrp < 2; ++hgrp) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= rz;
-            sWP[warp * kTile + g + lane] = reduce_scatter32(v, lane);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[hgrp * 32 + e]) * rz;
+            sWP[warp * kTile + hgrp * 32 + lane] = reduce_scatter32(v, lane);
           }
         }
       }
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      __syncthreads();
       if (last) {
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
         for (int j = tid; j < n; j += 128)
-          sW[c0 + j] += sNF[j] * (sWP[j] + sWP[kTile + j] + sWP[2 * kTile + j] + sWP[3 * kTile + j]);
+          sW[c0 + j] += sNF[j] * ((sWP[j] + sWP[kTile + j]) + (sWP[2 * kTile + j] + sWP[3 * kTile + j]));
         if (tid == 0) {
           tc::tc_fence_after();
           issue_values(n, x_started);
@@ -312,6 +307,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
         x_started = true;
         wait_mma();
       }
+      tc::tc_fence_before();
       __syncthreads();
       if (*sAbort) goto done;
     }
@@ -335,7 +331,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
       for (int r = tid; r < P; r += 128) a.sel[((size_t)bh * a.nblk + blk) * P + r] = sSEL[r];
   }
 
-  // ---- child refinement in chunks of 16 selected parents ----
+  // ---- child refinement in chunks of 8 selected parents ----
   if (a.C > 0 && a.P > 0) {
     float mref = m;
     const int nch = (a.P + kChunkParents - 1) / kChunkParents;
@@ -354,7 +350,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
           tc::bulk_g2s(sVB + r * KH * 1024, vb_bh + g, KH * 1024, bar_cp);
         }
       }
-      for (int j = tid; j < n; j += 128) {
+      for (int j = tid; j < kTile; j += 128) {
         const int r = j >> 3;
         sNF[j] = r < np ? (float)__ldg(cnt + M0 + sSEL[q * kChunkParents + r] * 8 + (j & 7)) : 0.f;
       }
@@ -366,65 +362,47 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
         issue_logits(n);
       }
       wait_mma();
-      // row max over the non-empty children of the chunk
+      uint32_t r[64];
+      tmem_ld64(tS + lane_off, r);
+      // scaled logits and the row max over non-empty children
       float cmax = NEG_INF;
-      for (int g = 0; g < n; g += 16) {
-        uint32_t r[16];
-        tc::tmem_ld16(tS + lane_off + g, r);
-        tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float tv = __uint_as_float(r[e]) * a.scale_log2;
-          if (sNF[g + e] > 0.f) cmax = fmaxf(cmax, tv);
-        }
+      for (int e = 0; e < 64; ++e) {
+        const float tv = __uint_as_float(r[e]) * sl2;
+        r[e] = __float_as_uint(tv);
+        if (sNF[e] > 0.f) cmax = fmaxf(cmax, tv);
       }
       // rare: a child logit far above the reference max -> rescale x and z
       const bool need = cmax > mref + kRescaleLog2;
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? tc::ex2(mref - cmax) : 1.f;
         for (int g = 0; g < D; g += 16) {
-          uint32_t r[16];
-          tc::tmem_ld16(tX + lane_off + g, r);
+          uint32_t xr[16];
+          tc::tmem_ld16(tX + lane_off + g, xr);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-          tc::tmem_st16(tX + lane_off + g, r);
+          for (int e = 0; e < 16; ++e) xr[e] = __float_as_uint(__uint_as_float(xr[e]) * f);
+          tc::tmem_st16(tX + lane_off + g, xr);
         }
         tc::tmem_wait_st();
         z *= f;
         if (need) mref = cmax;
       }
-      // dA = 2^(t_c - m) - 2^(t_p - m), t_p = mean of the parent's child logits
-      for (int g = 0; g < n; g += 16) {
-        uint32_t r[16];
-        tc::tmem_ld16(tS + lane_off + g, r);
-        tc::tmem_wait_ld();
+      // dA = 2^(t_c - m) - 2^(t_p - m), t_p = mean of the parent's child logits (Eq. 8)
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          float tc8[8];
-          float tp = 0.f;
+      for (int sl = 0; sl < 8; ++sl) {
+        float tp = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            tc8[e] = __uint_as_float(r[s * 8 + e]) * a.scale_log2;
-            tp += tc8[e];
-          }
-          tp *= 0.125f;
-          const float ap = tc::ex2(tp - mref);
-          float da[8];
+        for (int e = 0; e < 8; ++e) tp += __uint_as_float(r[sl * 8 + e]);
+        const float ap = tc::ex2(tp * 0.125f - mref);
+        float da[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float nf = sNF[g + s * 8 + e];
-            da[e] = nf > 0.f ? tc::ex2(tc8[e] - mref) - ap : 0.f;
-            z = fmaf(da[e], nf, z);
-          }
-          const int col = g + s * 8;
-          uint4 u;
-          u.x = pack_bf16x2(da[0], da[1]);
-          u.y = pack_bf16x2(da[2], da[3]);
-          u.z = pack_bf16x2(da[4], da[5]);
-          u.w = pack_bf16x2(da[6], da[7]);
-          *reinterpret_cast<uint4*>(sPR + (col >> 6) * (kRows * 128) + tc::sw128_offset(tid, col & 63)) = u;
+        for (int e = 0; e < 8; ++e) {
+          const float nf = sNF[sl * 8 + e];
+          da[e] = nf > 0.f ? tc::ex2(__uint_as_float(r[sl * 8 + e]) - mref) - ap : 0.f;
+          z = fmaf(da[e], nf, z);
         }
+        store_chunk8(sPR, tid, sl * 8, da);
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
@@ -434,6 +412,7 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
         issue_values(n, true);
       }
       wait_mma();
+      tc::tc_fence_before();
       __syncthreads();
       if (*sAbort) goto done;
     }
@@ -443,19 +422,14 @@ __global__ void __launch_bounds__(128) attention_tc_kernel(const __grid_constant
   {
     const float iz = 1.f / z;
     for (int g = 0; g < D; g += 16) {
-      uint32_t r[16];
-      tc::tmem_ld16(tX + lane_off + g, r);
+      uint32_t xr[16];
+      tc::tmem_ld16(tX + lane_off + g, xr);
       tc::tmem_wait_ld();
+      float v[16];
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const int col = g + s * 8;
-        uint4 u;
-        u.x = pack_bf16x2(__uint_as_float(r[s * 8 + 0]) * iz, __uint_as_float(r[s * 8 + 1]) * iz);
-        u.y = pack_bf16x2(__uint_as_float(r[s * 8 + 2]) * iz, __uint_as_float(r[s * 8 + 3]) * iz);
-        u.z = pack_bf16x2(__uint_as_float(r[s * 8 + 4]) * iz, __uint_as_float(r[s * 8 + 5]) * iz);
-        u.w = pack_bf16x2(__uint_as_float(r[s * 8 + 6]) * iz, __uint_as_float(r[s * 8 + 7]) * iz);
-        *reinterpret_cast<uint4*>(sQ + (col >> 6) * (kRows * 128) + tc::sw128_offset(tid, col & 63)) = u;
-      }
+      for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(xr[e]) * iz;
+      store_chunk8(sQ, tid, g, v);
+      store_chunk8(sQ, tid, g + 8, v + 8);
     }
     tc::fence_proxy_async_smem();
     __syncthreads();
@@ -472,9 +446,8 @@ done:
   __syncthreads();
   if (warp == 0) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, S::kTmemCols);
   }
-  (void)valid;
 }
 
 // Codewords and value sums -> bf16 images of swizzled atoms.  Code a of a head

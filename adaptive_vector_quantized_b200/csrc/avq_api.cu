@@ -219,9 +219,9 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   LaunchLog log{};
   cudaError_t e;
+  unsigned int* err = error_word();
+  if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
   if (use_tc) {
-    unsigned int* err = error_word();
-    if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
     e = launch_assign_tc(s, K, parents, children, assign, ws, err, cs, log);
   } else {
     e = launch_assign_simt(s, dtype, K, parents, children, assign, cs, log);
@@ -230,7 +230,7 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
   if (deterministic)
     e = launch_aggregate_det(s, dtype, V, assign, vsum, counts, ws_det_ptr, cs, log);
   else
-    e = launch_aggregate(s, dtype, V, assign, vsum, counts, cs, log);
+    e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log);
   if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
   snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
   return AVQ_OK;

@@ -33,7 +33,8 @@ cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, cons
 // Algorithm 1 steps 1, 8, 16 (aggregation for given codes), atomics variant.
 // vsum/counts are zeroed inside.
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
-                             float* vsum, int32_t* counts, cudaStream_t st, LaunchLog& log);
+                             float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
+                             LaunchLog& log);
 // Deterministic aggregation (fixed-order sums, independent of the grid).
 size_t aggregate_det_workspace(const Shape& s);
 cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
