@@ -127,20 +127,23 @@ __global__ void __launch_bounds__(kAggThreads) aggregate_kernel(
   }
 }
 
-// Ring variant: one CTA per chunk of keys of one head, 16 warps.  Value rows
+// Ring variant: one CTA per chunk of keys of one head, 8 warps.  Value rows
 // stream through a two-slot shared-memory ring filled by 1-D bulk copies
-// (the next tile is in flight while the current one is consumed); each warp
-// takes 16 consecutive keys of a tile with lanes over the head dimension,
-// merges runs of equal codes in registers and flushes a run into the
-// per-CTA partials with shared-memory atomics only when the code changes.
-// Codes are prefetched one tile ahead into registers (lane u holds key u).
-constexpr int kRingThreads = 512;
+// (the next tile is in flight while the current one is consumed).  In each
+// 256-key tile warp w takes keys 32w..32w+31: lane u holds key u's code and
+// parent, ballots mark where runs of equal codes start, and lanes then walk
+// the keys over the head dimension, adding values in registers and flushing
+// a run into the per-CTA partials (shared-memory atomics) only where a run
+// ends.  Each warp counts itself out of a slot; the last one to leave refills
+// it, so warps never wait for each other.
+constexpr int kRingThreads = 256;
 constexpr int kRingWarps = kRingThreads / 32;
+constexpr int kRingTile = kRingWarps * 32;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kRingThreads) aggregate_ring_kernel(
     const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
-    int32_t* __restrict__ counts, int N, int M0, int C, int chunk, int tile, unsigned int* err) {
+    int32_t* __restrict__ counts, int N, int M0, int C, int chunk, int log2C, unsigned int* err) {
   extern __shared__ __align__(128) uint8_t smraw[];
   constexpr int E = D / 32;
   constexpr int RB = D * (int)sizeof(T);  // bytes per value row
@@ -149,13 +152,14 @@ __global__ void __launch_bounds__(kRingThreads) aggregate_ring_kernel(
   float* part = reinterpret_cast<float*>(smraw);
   int* cnt = reinterpret_cast<int*>(part + (size_t)Mt * D);
   uint8_t* ring = reinterpret_cast<uint8_t*>(((uintptr_t)(cnt + Mt) + 127) & ~(uintptr_t)127);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + 2 * (size_t)tile * RB);  // [2]
-  int* sAbort = reinterpret_cast<int*>(full + 2);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + 2 * (size_t)kRingTile * RB);  // [2]
+  int* leave = reinterpret_cast<int*>(full + 2);                                   // [2]
+  int* sAbort = leave + 2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k0 = blockIdx.x * chunk;
   const int k1 = min(N, k0 + chunk);
   if (k0 >= k1) return;
-  const int ntile = (k1 - k0 + tile - 1) / tile;
+  const int ntile = (k1 - k0 + kRingTile - 1) / kRingTile;
   const T* vb = V + (size_t)bh * N * D;
   const int32_t* asg = assign + (size_t)bh * N;
 
@@ -168,38 +172,45 @@ __global__ void __launch_bounds__(kRingThreads) aggregate_ring_kernel(
     tc::mbar_init(&full[0], 1);
     tc::mbar_init(&full[1], 1);
     tc::fence_mbar_init();
+    leave[0] = leave[1] = 0;
     *sAbort = 0;
   }
   __syncthreads();
   auto issue = [&](int t) {
-    const int j0 = k0 + t * tile;
-    const int nk = min(tile, k1 - j0);
+    const int j0 = k0 + t * kRingTile;
+    const int nk = min(kRingTile, k1 - j0);
     const int slot = t & 1;
     tc::mbar_arrive_expect_tx(&full[slot], (uint32_t)nk * RB);
-    tc::bulk_g2s(ring + (size_t)slot * tile * RB, vb + (size_t)j0 * D, (uint32_t)nk * RB, &full[slot]);
+    tc::bulk_g2s(ring + (size_t)slot * kRingTile * RB, vb + (size_t)j0 * D, (uint32_t)nk * RB, &full[slot]);
   };
   if (tid == 0) {
     issue(0);
     if (ntile > 1) issue(1);
   }
-  const int per_warp = tile / kRingWarps;  // 16 keys
-  auto load_codes = [&](int t) {
-    const int j = k0 + t * tile + warp * per_warp + lane;
-    return (lane < per_warp && t < ntile && j < k1) ? __ldg(asg + j) : -1;
+  auto load_code = [&](int t) {
+    const int j = k0 + t * kRingTile + warp * 32 + lane;
+    return (t < ntile && j < k1) ? __ldg(asg + j) : -1;
   };
-  int codes = load_codes(0);
+  int code = load_code(0);
   float accP[E], accC[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
   int curP = -1, curC = -1, nP = 0, nC = 0;
   for (int t = 0; t < ntile; ++t) {
     const int slot = t & 1;
-    const int next = load_codes(t + 1);
+    const int next = load_code(t + 1);
+    // per-lane parent code and run starts (uniform bit masks)
+    const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / C);
+    const int prevc = __shfl_up_sync(0xffffffffu, code, 1);
+    const int prevp = __shfl_up_sync(0xffffffffu, par, 1);
+    const unsigned live = __ballot_sync(0xffffffffu, code >= 0);
+    const unsigned newP = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 || prevp != par));
+    const unsigned isC = __ballot_sync(0xffffffffu, code >= M0);
+    const unsigned newC = __ballot_sync(0xffffffffu, code >= M0 && (lane == 0 || prevc != code));
     if (!tc::mbar_wait(&full[slot], (t >> 1) & 1)) *sAbort = 1;
-    const uint8_t* rows = ring + (size_t)slot * tile * RB + (size_t)warp * per_warp * RB + lane * E * sizeof(T);
-    for (int u = 0; u < per_warp; ++u) {
-      const int c = __shfl_sync(0xffffffffu, codes, u);
-      if (c < 0) break;
+    const uint8_t* rows = ring + (size_t)slot * kRingTile * RB + (size_t)warp * 32 * RB + lane * E * sizeof(T);
+    const int nlive = __popc(live);
+    for (int u = 0; u < nlive; ++u) {
       float v[E];
       if constexpr (sizeof(T) == 2) {
         if constexpr (E == 2) {
@@ -213,33 +224,45 @@ __global__ void __launch_bounds__(kRingThreads) aggregate_ring_kernel(
 #pragma unroll
         for (int e = 0; e < E; ++e) v[e] = reinterpret_cast<const float*>(rows + (size_t)u * RB)[e];
       }
-      const int p = c < M0 ? c : (c - M0) / C;
-      if (p != curP) {
-        if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
-        curP = p;
-        nP = 0;
+      const unsigned bit = 1u << u;
+      if (newP & bit) {
+        const int p = __shfl_sync(0xffffffffu, par, u);
+        if (p != curP) {
+          if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
+          curP = p;
+          nP = 0;
 #pragma unroll
-        for (int e = 0; e < E; ++e) accP[e] = 0.f;
+          for (int e = 0; e < E; ++e) accP[e] = 0.f;
+        }
       }
 #pragma unroll
       for (int e = 0; e < E; ++e) accP[e] += v[e];
       ++nP;
-      if (c >= M0) {
-        if (c != curC) {
-          if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
-          curC = c;
-          nC = 0;
+      if (isC & bit) {
+        if (newC & bit) {
+          const int c = __shfl_sync(0xffffffffu, code, u);
+          if (c != curC) {
+            if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
+            curC = c;
+            nC = 0;
 #pragma unroll
-          for (int e = 0; e < E; ++e) accC[e] = 0.f;
+            for (int e = 0; e < E; ++e) accC[e] = 0.f;
+          }
         }
 #pragma unroll
         for (int e = 0; e < E; ++e) accC[e] += v[e];
         ++nC;
       }
     }
-    codes = next;
-    __syncthreads();  // slot consumed by every warp
-    if (tid == 0 && t + 2 < ntile) issue(t + 2);
+    code = next;
+    __syncwarp();
+    if (lane == 0 && atomicAdd(&leave[slot], 1) == kRingWarps - 1) {
+      leave[slot] = 0;  // every warp has read this slot: refill it
+      if (t + 2 < ntile) {
+        tc::fence_proxy_async_smem();
+        issue(t + 2);
+      }
+    }
   }
   if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
   if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
@@ -451,13 +474,14 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   const size_t part = agg_smem_bytes(s);
   const size_t row_bytes = (size_t)s.d * (dt == AVQ_F32 ? 4 : 2);
   // ring variant: partials + two value tiles of `tile` keys (+ alignment, barriers)
-  int tile = 256;
-  while (tile >= kRingWarps && part + 128 + 2 * tile * row_bytes + 64 > 220 * 1024) tile /= 2;
-  if (tile >= kRingWarps && err != nullptr) {
-    const size_t smem = part + 128 + 2 * tile * row_bytes + 64;
+  const size_t smem = part + 128 + 2 * (size_t)kRingTile * row_bytes + 64;
+  if (smem <= 220 * 1024 && err != nullptr) {
     int per_head = sms >= s.BH() ? sms / s.BH() : 1;
     int chunk = (s.N + per_head - 1) / per_head;
-    chunk = ((chunk + tile - 1) / tile) * tile;
+    chunk = ((chunk + kRingTile - 1) / kRingTile) * kRingTile;
+    int log2C = -1;
+    for (int b = 0; b <= 3; ++b)
+      if (s.C == (1 << b)) log2C = b;
     dim3 grid((s.N + chunk - 1) / chunk, s.BH());
 #define AVQ_RING(T, D)                                                                             \
   do {                                                                                             \
@@ -465,7 +489,7 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);        \
     if (e != cudaSuccess) return e;                                                                \
     kern<<<grid, kRingThreads, smem, st>>>((const T*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk, \
-                                           tile, err);                                             \
+                                           log2C, err);                                            \
   } while (0)
     if (dt == AVQ_F32) {
       if (s.d == 64) AVQ_RING(float, 64); else AVQ_RING(float, 128);

@@ -8,12 +8,18 @@
 //               thread r owns key r = TMEM lane r and takes the first
 //               minimum of |p|^2 - 2 k.p over the parents (|k|^2 is the same
 //               for every codeword of a key and is dropped)
-//   children    the C = 8 children of the chosen parent, read from a bf16
-//               image in shared memory (or L2 when it does not fit), dot
-//               products with bf16 x bf16 -> fp32 fused multiply-adds
-//               (exact products, fp32 accumulation); the key moves to the
-//               first strictly smallest child only if it is strictly closer
-//               than the parent
+//   children    the C = 8 children of every parent are in shared memory as
+//               one swizzled atom each, so the children of two adjacent
+//               parents form an N = 16 operand tile: one MMA per parent pair
+//               that some key of the tile chose gives every key of the tile
+//               its dot products with those 16 children (TMEM, in rounds of
+//               16 pairs); each thread then loads the 8 columns of its own
+//               parent (one TMEM load per distinct pair in its warp).  When
+//               the children do not fit in shared memory they are read from
+//               L2 and the dot products are bf16 x bf16 -> fp32 fused
+//               multiply-adds on the CUDA cores.  Either way the key moves
+//               to the first strictly smallest child only if it is strictly
+//               closer than the parent
 //   output      assign[key] = parent, or M0 + parent*C + child
 // Codewords are first converted into the swizzled-atom image shared with
 // the attention kernel (8 codes x 64 dims per 1024-byte atom) plus their
@@ -56,14 +62,15 @@ __device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
 template <int D, bool CH_SMEM>
 struct AssignSmem {
   static constexpr int KH = D / 64;
-  // parents image | children image (optional) | K ring [2] | norms | barriers
+  // parents image | children image (optional) | K ring [2] | norms | pair bits | barriers
   __host__ __device__ static size_t parents_bytes(int M0) { return (size_t)M0 * D * 2; }
   __host__ __device__ static size_t children_bytes(int M0, int C) { return CH_SMEM ? (size_t)M0 * C * D * 2 : 0; }
   __host__ __device__ static size_t ring_off(int M0, int C) { return parents_bytes(M0) + children_bytes(M0, C); }
   __host__ __device__ static size_t norms_off(int M0, int C) { return ring_off(M0, C) + 2 * kKeys * D * 2; }
-  __host__ __device__ static size_t bar_off(int M0, int C) {
+  __host__ __device__ static size_t pairs_off(int M0, int C) {
     return (norms_off(M0, C) + (size_t)M0 * (1 + C) * 4 + 15) & ~(size_t)15;
   }
+  __host__ __device__ static size_t bar_off(int M0, int C) { return pairs_off(M0, C) + 16; }
   __host__ __device__ static size_t total(int M0, int C) { return bar_off(M0, C) + 64; }
 };
 
@@ -79,6 +86,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
   uint8_t* sCh = sm + S::parents_bytes(M0);
   uint8_t* sRing = sm + S::ring_off(M0, C);
   float* sNorm = reinterpret_cast<float*>(sm + S::norms_off(M0, C));
+  uint32_t* sPairs = reinterpret_cast<uint32_t*>(sm + S::pairs_off(M0, C));  // 128-bit set of parent pairs
   uint64_t* bar_k = reinterpret_cast<uint64_t*>(sm + S::bar_off(M0, C));  // [2]
   uint64_t* bar_cb = bar_k + 2;
   uint64_t* bar_mma = bar_k + 3;
@@ -89,7 +97,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
   const int t0 = blockIdx.x * a.tiles_per_cta;
   const int t1 = min(a.ntiles, t0 + a.tiles_per_cta);
   if (t0 >= t1) return;
-  const uint32_t ncols = M0 <= 32 ? 32 : M0 <= 64 ? 64 : M0 <= 128 ? 128 : 256;
+  const uint32_t ncols = CH_SMEM ? 256u : (M0 <= 32 ? 32u : M0 <= 64 ? 64u : M0 <= 128 ? 128u : 256u);
 
   if (tid == 0) {
     tc::mbar_init(&bar_k[0], 1);
@@ -98,6 +106,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     tc::mbar_init(bar_mma, 1);
     tc::fence_mbar_init();
     *sAbort = 0;
+    sPairs[0] = sPairs[1] = sPairs[2] = sPairs[3] = 0;
     tc::prefetch_tensormap(&kmap);
   }
   if (warp == 0) {
@@ -215,7 +224,85 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         }
     }
     int code = par;
-    if (C > 0) {  // C == 8 on this path
+    if constexpr (CH_SMEM) {
+      if (C > 0) {  // C == 8 on this path
+        const int pair = par >> 1;
+        atomicOr(&sPairs[pair >> 5], 1u << (pair & 31));
+        tc::tc_fence_before();
+        __syncthreads();  // pair set complete, parents' logits read
+        uint32_t bits[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) bits[w] = sPairs[w];
+        int npairs = 0, slot = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          if (w < (pair >> 5)) slot += __popc(bits[w]);
+          npairs += __popc(bits[w]);
+        }
+        slot += __popc(bits[pair >> 5] & ((1u << (pair & 31)) - 1u));
+        const uint32_t idesc16 = tc::idesc_bf16(kKeys, 16, 0, 0);
+        const uint32_t sKa = tc::smem_u32(sK), sCha = tc::smem_u32(sCh);
+        float vals[8];
+        for (int round = 0; round * 16 < npairs; ++round) {
+          if (tid == 0) {
+            tc::tc_fence_after();
+            int idx = 0;
+            for (int w = 0; w < 4; ++w) {
+              uint32_t b = bits[w];
+              while (b) {
+                const int q = w * 32 + __ffs(b) - 1;
+                b &= b - 1;
+                if (idx >= round * 16 && idx < round * 16 + 16) {
+                  const uint32_t col = (uint32_t)(idx - round * 16) * 16;
+#pragma unroll
+                  for (int k = 0; k < D / 16; ++k) {
+                    const uint64_t ad = tc::sdesc_sw128(sKa + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024);
+                    const uint64_t bd = tc::sdesc_sw128(sCha + (2 * q) * (KH * 1024) + (k >> 2) * 1024 + (k & 3) * 32,
+                                                        16, KH * 1024);
+                    tc::mma_bf16(tmem + col, ad, bd, idesc16, k > 0);
+                  }
+                }
+                ++idx;
+              }
+            }
+            tc::mma_commit(bar_mma);
+          }
+          if (!tc::mbar_wait(bar_mma, ph_mma)) atomicOr(a.err, kErrTimeout);
+          ph_mma ^= 1;
+          tc::tc_fence_after();
+          // one TMEM load per distinct pair slot among this warp's keys
+          const int my = (slot >= round * 16 && slot < round * 16 + 16) ? slot - round * 16 : -1;
+          unsigned pending = __ballot_sync(0xffffffffu, my >= 0);
+          while (pending) {
+            const int leader = __ffs(pending) - 1;
+            const int sl = __shfl_sync(0xffffffffu, my, leader);
+            uint32_t r[16];
+            tc::tmem_ld16(tmem + lane_off + sl * 16, r);
+            tc::tmem_wait_ld();
+            if (my == sl) {
+              const int half = (par & 1) * 8;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) vals[c] = __uint_as_float(half ? r[8 + c] : r[c]);
+            }
+            pending &= ~__ballot_sync(0xffffffffu, my == sl);
+          }
+          tc::tc_fence_before();
+          __syncthreads();  // TMEM columns free for the next round
+        }
+        float dchild = INF;
+        int cstar = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float dc = fmaf(-2.f, vals[c], sNorm[M0 + par * 8 + c]);
+          if (dc < dchild) {
+            dchild = dc;
+            cstar = c;
+          }
+        }
+        if (dchild < best) code = M0 + par * 8 + cstar;
+        if (tid < 4) sPairs[tid] = 0;  // for the next tile (read by everyone above)
+      }
+    } else if (C > 0) {  // C == 8; children from L2, dot products on the CUDA cores
       // key row in registers, 16-byte chunks in rotated order
       const int rot = tid & 7;
       uint4 kq[KH][8];
@@ -226,33 +313,23 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
           const int lc = (s + rot) & 7;
           kq[kh][s] = *reinterpret_cast<const uint4*>(sK + kh * (kKeys * 128) + tid * 128 + ((lc ^ rot) << 4));
         }
-      const uint8_t* atom = CH_SMEM ? sCh + (size_t)par * (KH * 1024)
-                                    : reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + par * 8) * D);
-      // eight independent dot products (one per child)
-      float acc[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-#pragma unroll
-      for (int kh = 0; kh < KH; ++kh)
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int lc = (s + rot) & 7;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint8_t* p = atom + kh * 1024 + c * 128 + ((lc ^ c) << 4);
-            const uint4 cv = CH_SMEM ? *reinterpret_cast<const uint4*>(p)
-                                     : __ldg(reinterpret_cast<const uint4*>(p));
-            acc[c] = fma_bf16x2(kq[kh][s].x, cv.x, acc[c]);
-            acc[c] = fma_bf16x2(kq[kh][s].y, cv.y, acc[c]);
-            acc[c] = fma_bf16x2(kq[kh][s].z, cv.z, acc[c]);
-            acc[c] = fma_bf16x2(kq[kh][s].w, cv.w, acc[c]);
-          }
-        }
+      const uint8_t* atom = reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + par * 8) * D);
       float dchild = INF;
       int cstar = 0;
-#pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float dc = fmaf(-2.f, acc[c], sNorm[M0 + par * 8 + c]);
+        float acc = 0.f;
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const int lc = (s + rot) & 7;
+            const uint4 cv = __ldg(reinterpret_cast<const uint4*>(atom + kh * 1024 + c * 128 + ((lc ^ c) << 4)));
+            acc = fma_bf16x2(kq[kh][s].x, cv.x, acc);
+            acc = fma_bf16x2(kq[kh][s].y, cv.y, acc);
+            acc = fma_bf16x2(kq[kh][s].z, cv.z, acc);
+            acc = fma_bf16x2(kq[kh][s].w, cv.w, acc);
+          }
+        const float dc = fmaf(-2.f, acc, sNorm[M0 + par * 8 + c]);
         if (dc < dchild) {
           dchild = dc;
           cstar = c;
