@@ -127,159 +127,105 @@ __global__ void __launch_bounds__(kAggThreads) aggregate_kernel(
   }
 }
 
-// Ring variant: one CTA per chunk of keys of one head, 8 warps.  Value rows
-// stream through a two-slot shared-memory ring filled by 1-D bulk copies
-// (the next tile is in flight while the current one is consumed).  In each
-// 256-key tile warp w takes keys 32w..32w+31: lane u holds key u's code and
-// parent, ballots mark where runs of equal codes start, and lanes then walk
-// the keys over the head dimension, adding values in registers and flushing
-// a run into the per-CTA partials (shared-memory atomics) only where a run
-// ends.  Each warp counts itself out of a slot; the last one to leave refills
-// it, so warps never wait for each other.
-constexpr int kRingThreads = 256;
-constexpr int kRingWarps = kRingThreads / 32;
-constexpr int kRingTile = kRingWarps * 32;
+// Streaming variant (the default): every warp owns a contiguous range of
+// keys of one head (so runs of equal codes stay long), lanes cover the head
+// dimension, value rows are loaded straight from global memory sixteen keys
+// ahead, codes one 32-key group ahead.  Per 32-key group, warp ballots mark
+// where runs start, so the per-key work is a bit test and two adds.  A run
+// is flushed with one vector reduction per lane into the global statistics
+// (L2-resident) and one count reduction; there are no shared-memory atomics
+// and no per-CTA partials.
+constexpr int kStreamThreads = 256;
+constexpr int kStreamBatch = 16;
+
+template <int E>
+__device__ __forceinline__ void flush_global(float* vsum, int32_t* counts, int code, const float* acc,
+                                             int n, int lane, int D) {
+  float* row = vsum + (size_t)code * D + lane * E;
+  if constexpr (E == 2) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(row), "f"(acc[0]), "f"(acc[1]) : "memory");
+  } else {
+    red_add_v4(row, acc[0], acc[1], acc[2], acc[3]);
+  }
+  if (lane == 0) atomicAdd(counts + code, n);
+}
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kRingThreads) aggregate_ring_kernel(
+__global__ void __launch_bounds__(kStreamThreads, 3) aggregate_stream_kernel(
     const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
-    int32_t* __restrict__ counts, int N, int M0, int C, int chunk, int log2C, unsigned int* err) {
-  extern __shared__ __align__(128) uint8_t smraw[];
+    int32_t* __restrict__ counts, int BH, int N, int M0, int C, int keys_per_warp, int log2C) {
   constexpr int E = D / 32;
-  constexpr int RB = D * (int)sizeof(T);  // bytes per value row
-  const int bh = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (kStreamThreads / 32) + (threadIdx.x >> 5);
+  const int warps_per_head = (N + keys_per_warp - 1) / keys_per_warp;
+  const int bh = gw / warps_per_head;
+  const int j0 = (gw % warps_per_head) * keys_per_warp;
+  const int j1 = min(N, j0 + keys_per_warp);
+  if (bh >= BH || j0 >= j1) return;
   const int Mt = M0 * (1 + C);
-  float* part = reinterpret_cast<float*>(smraw);
-  int* cnt = reinterpret_cast<int*>(part + (size_t)Mt * D);
-  uint8_t* ring = reinterpret_cast<uint8_t*>(((uintptr_t)(cnt + Mt) + 127) & ~(uintptr_t)127);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + 2 * (size_t)kRingTile * RB);  // [2]
-  int* leave = reinterpret_cast<int*>(full + 2);                                   // [2]
-  int* sAbort = leave + 2;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int k0 = blockIdx.x * chunk;
-  const int k1 = min(N, k0 + chunk);
-  if (k0 >= k1) return;
-  const int ntile = (k1 - k0 + kRingTile - 1) / kRingTile;
-  const T* vb = V + (size_t)bh * N * D;
+  float* vs = vsum + (size_t)bh * Mt * D;
+  int32_t* ns = counts + (size_t)bh * Mt;
+  const T* vb = V + (size_t)bh * N * D + lane * E;
   const int32_t* asg = assign + (size_t)bh * N;
 
-  {
-    float4* s4 = reinterpret_cast<float4*>(part);
-    for (int i = tid; i < Mt * D / 4; i += blockDim.x) s4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = tid; i < Mt; i += blockDim.x) cnt[i] = 0;
-  }
-  if (tid == 0) {
-    tc::mbar_init(&full[0], 1);
-    tc::mbar_init(&full[1], 1);
-    tc::fence_mbar_init();
-    leave[0] = leave[1] = 0;
-    *sAbort = 0;
-  }
-  __syncthreads();
-  auto issue = [&](int t) {
-    const int j0 = k0 + t * kRingTile;
-    const int nk = min(kRingTile, k1 - j0);
-    const int slot = t & 1;
-    tc::mbar_arrive_expect_tx(&full[slot], (uint32_t)nk * RB);
-    tc::bulk_g2s(ring + (size_t)slot * kRingTile * RB, vb + (size_t)j0 * D, (uint32_t)nk * RB, &full[slot]);
-  };
-  if (tid == 0) {
-    issue(0);
-    if (ntile > 1) issue(1);
-  }
-  auto load_code = [&](int t) {
-    const int j = k0 + t * kRingTile + warp * 32 + lane;
-    return (t < ntile && j < k1) ? __ldg(asg + j) : -1;
-  };
-  int code = load_code(0);
   float accP[E], accC[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
   int curP = -1, curC = -1, nP = 0, nC = 0;
-  for (int t = 0; t < ntile; ++t) {
-    const int slot = t & 1;
-    const int next = load_code(t + 1);
-    // per-lane parent code and run starts (uniform bit masks)
-    const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / C);
+  int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
+  for (int g = j0; g < j1; g += 32) {
+    const int code = code_next;
+    code_next = g + 32 + lane < j1 ? __ldg(asg + g + 32 + lane) : -1;
+    const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / max(C, 1));
     const int prevc = __shfl_up_sync(0xffffffffu, code, 1);
     const int prevp = __shfl_up_sync(0xffffffffu, par, 1);
     const unsigned live = __ballot_sync(0xffffffffu, code >= 0);
-    const unsigned newP = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 || prevp != par));
+    // run starts relative to the previous key of this group (lane 0 compares with the carry)
+    const unsigned newP = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? par != curP : prevp != par));
     const unsigned isC = __ballot_sync(0xffffffffu, code >= M0);
-    const unsigned newC = __ballot_sync(0xffffffffu, code >= M0 && (lane == 0 || prevc != code));
-    if (!tc::mbar_wait(&full[slot], (t >> 1) & 1)) *sAbort = 1;
-    const uint8_t* rows = ring + (size_t)slot * kRingTile * RB + (size_t)warp * 32 * RB + lane * E * sizeof(T);
+    const unsigned newC = __ballot_sync(0xffffffffu, code >= M0 && (lane == 0 ? code != curC : prevc != code));
     const int nlive = __popc(live);
-    for (int u = 0; u < nlive; ++u) {
-      float v[E];
-      if constexpr (sizeof(T) == 2) {
-        if constexpr (E == 2) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + (size_t)u * RB);
-          v[0] = bf16_lo(w); v[1] = bf16_hi(w);
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(rows + (size_t)u * RB);
-          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
-        }
-      } else {
+    for (int u0 = 0; u0 < nlive; u0 += kStreamBatch) {
+      float v[kStreamBatch][E];
 #pragma unroll
-        for (int e = 0; e < E; ++e) v[e] = reinterpret_cast<const float*>(rows + (size_t)u * RB)[e];
-      }
-      const unsigned bit = 1u << u;
-      if (newP & bit) {
-        const int p = __shfl_sync(0xffffffffu, par, u);
-        if (p != curP) {
-          if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
-          curP = p;
+      for (int b = 0; b < kStreamBatch; ++b)
+        if (u0 + b < nlive) loadE<E>(vb + (size_t)(g + u0 + b) * D, v[b]);
+#pragma unroll
+      for (int b = 0; b < kStreamBatch; ++b) {
+        const int u = u0 + b;
+        if (u >= nlive) break;
+        const unsigned bit = 1u << u;
+        if (newP & bit) {
+          if (curP >= 0) flush_global<E>(vs, ns, curP, accP, nP, lane, D);
+          curP = __shfl_sync(0xffffffffu, par, u);
           nP = 0;
 #pragma unroll
           for (int e = 0; e < E; ++e) accP[e] = 0.f;
         }
-      }
 #pragma unroll
-      for (int e = 0; e < E; ++e) accP[e] += v[e];
-      ++nP;
-      if (isC & bit) {
-        if (newC & bit) {
-          const int c = __shfl_sync(0xffffffffu, code, u);
-          if (c != curC) {
-            if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
-            curC = c;
-            nC = 0;
+        for (int e = 0; e < E; ++e) accP[e] += v[b][e];
+        ++nP;
+        if (isC & bit) {
+          if (newC & bit) {
+            // the previous key may have stayed at a parent: compare with the open run
+            const int c = __shfl_sync(0xffffffffu, code, u);
+            if (c != curC) {
+              if (curC >= 0) flush_global<E>(vs, ns, curC, accC, nC, lane, D);
+              curC = c;
+              nC = 0;
 #pragma unroll
-            for (int e = 0; e < E; ++e) accC[e] = 0.f;
+              for (int e = 0; e < E; ++e) accC[e] = 0.f;
+            }
           }
-        }
 #pragma unroll
-        for (int e = 0; e < E; ++e) accC[e] += v[e];
-        ++nC;
-      }
-    }
-    code = next;
-    __syncwarp();
-    if (lane == 0 && atomicAdd(&leave[slot], 1) == kRingWarps - 1) {
-      leave[slot] = 0;  // every warp has read this slot: refill it
-      if (t + 2 < ntile) {
-        tc::fence_proxy_async_smem();
-        issue(t + 2);
+          for (int e = 0; e < E; ++e) accC[e] += v[b][e];
+          ++nC;
+        }
       }
     }
   }
-  if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
-  if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
-  __syncthreads();
-  float* gvs = vsum + (size_t)bh * Mt * D;
-  int* gcnt = counts + (size_t)bh * Mt;
-  const float4* s4 = reinterpret_cast<const float4*>(part);
-  for (int i = tid; i < Mt * D / 4; i += blockDim.x) {
-    const int row = i / (D / 4);
-    if (cnt[row] > 0) {
-      const float4 a4 = s4[i];
-      red_add_v4(gvs + (size_t)4 * i, a4.x, a4.y, a4.z, a4.w);
-    }
-  }
-  for (int r = tid; r < Mt; r += blockDim.x)
-    if (cnt[r] > 0) atomicAdd(gcnt + r, cnt[r]);
-  if (tid == 0 && *sAbort) atomicOr(err, kErrTimeout);
+  if (curP >= 0) flush_global<E>(vs, ns, curP, accP, nP, lane, D);
+  if (curC >= 0) flush_global<E>(vs, ns, curC, accC, nC, lane, D);
 }
 
 // ---- deterministic variant ------------------------------------------------
@@ -471,33 +417,30 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const int sms = num_sms();
-  const size_t part = agg_smem_bytes(s);
-  const size_t row_bytes = (size_t)s.d * (dt == AVQ_F32 ? 4 : 2);
-  // ring variant: partials + two value tiles of `tile` keys (+ alignment, barriers)
-  const size_t smem = part + 128 + 2 * (size_t)kRingTile * row_bytes + 64;
-  if (smem <= 220 * 1024 && err != nullptr) {
-    int per_head = sms >= s.BH() ? sms / s.BH() : 1;
-    int chunk = (s.N + per_head - 1) / per_head;
-    chunk = ((chunk + kRingTile - 1) / kRingTile) * kRingTile;
+  {
     int log2C = -1;
     for (int b = 0; b <= 3; ++b)
       if (s.C == (1 << b)) log2C = b;
-    dim3 grid((s.N + chunk - 1) / chunk, s.BH());
-#define AVQ_RING(T, D)                                                                             \
-  do {                                                                                             \
-    auto kern = aggregate_ring_kernel<T, D>;                                                       \
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);        \
-    if (e != cudaSuccess) return e;                                                                \
-    kern<<<grid, kRingThreads, smem, st>>>((const T*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk, \
-                                           log2C, err);                                            \
-  } while (0)
+    // about 24 warps per SM in total (3 CTAs), each a contiguous multiple of 32 keys
+    const long long total_keys = (long long)s.BH() * s.N;
+    const long long want_warps = (long long)sms * 24;
+    int kpw = (int)((total_keys + want_warps - 1) / want_warps);
+    kpw = ((kpw + 31) / 32) * 32;
+    if (kpw < 64) kpw = 64;
+    const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
+    const int wpb = kStreamThreads / 32;
+    const unsigned blocks = (unsigned)((warps + wpb - 1) / wpb);
+#define AVQ_STREAM(T, D)                                                                             \
+  aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, counts, \
+                                                                   s.BH(), s.N, s.M0, s.C, kpw, log2C)
     if (dt == AVQ_F32) {
-      if (s.d == 64) AVQ_RING(float, 64); else AVQ_RING(float, 128);
+      if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
     } else {
-      if (s.d == 64) AVQ_RING(bf16, 64); else AVQ_RING(bf16, 128);
+      if (s.d == 64) AVQ_STREAM(bf16, 64); else AVQ_STREAM(bf16, 128);
     }
-#undef AVQ_RING
-    log.add("aggregate_ring");
+#undef AVQ_STREAM
+    log.add("aggregate_stream");
+    (void)err;
     return cudaGetLastError();
   }
   // partials too large for shared memory: runs flushed straight to global memory

@@ -6,7 +6,7 @@
 // continuous.
 #include <stdint.h>
 
-#include "../../include/avq.h"
+#include "avq.h"
 
 namespace {
 

@@ -7,7 +7,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/avq.h"
+#include "avq.h"
 
 namespace avq {
 
