@@ -1,22 +1,20 @@
 // Stage 1, aggregation ("AVQ-Attention: Adaptive Vector-Quantized Attention",
 // Sec. 4.2, Algorithm 1 steps 1, 8 and 16; Eq. 3).
 //
-// Given every key's final code, each key adds its value and a count of one to
-// its parent, and to its child when it moved to one.  Parents therefore hold
-// their whole cluster, children only the keys closer to them than to the
-// parent.
+// Given every key's final code, each key adds its value to its parent, and to
+// its child when it moved to one.  Parents therefore hold their whole
+// cluster, children only the keys closer to them than to the parent.  (The
+// key counts n of Eq. 3 are produced by the assignment kernels.)
 //
-// Atomics variant: one CTA per chunk of keys of one head.  Warps walk
-// contiguous key ranges with lanes over the head dimension, merge runs of equal
-// codes in registers and flush each run with shared-memory atomics into
-// per-CTA partials [Mt][d]; the CTA then adds its non-empty rows to global
-// memory with vector reductions.  When the partials do not fit in shared
-// memory, runs are flushed straight to global memory.
+// Streaming variant: runs of equal codes are summed in registers and added to
+// the statistics with global vector reductions; see aggregate_stream_kernel.
 //
 // Deterministic variant: keys are stably sorted by (parent, child) with a
 // counting sort over fixed 1024-key chunks, each segment is summed in key
 // order by one warp, and parent totals are formed as stay + children in a
 // fixed order.  Nothing depends on the grid or the GPU's size.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_util.cuh"
@@ -25,207 +23,138 @@ namespace avq {
 
 namespace {
 
-constexpr int kAggThreads = 512;
-constexpr int kAggBatch = 16;  // keys whose loads are in flight per warp
-
-template <int E>
-__device__ __forceinline__ void flush_run(float* part, int* cnt, int code, const float* acc, int n,
-                                          int lane, int D) {
-  float* row = part + (size_t)code * D + lane * E;
-#pragma unroll
-  for (int e = 0; e < E; ++e) atomicAdd(row + e, acc[e]);
-  if (lane == 0) atomicAdd(cnt + code, n);
-}
-
-template <typename T, int D, bool SMEM>
-__global__ void __launch_bounds__(kAggThreads) aggregate_kernel(
-    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
-    int32_t* __restrict__ counts, int N, int M0, int C, int chunk) {
-  extern __shared__ __align__(16) float sm[];
-  constexpr int E = D / 32;
-  const int bh = blockIdx.y;
-  const int Mt = M0 * (1 + C);
-  float* gvs = vsum + (size_t)bh * Mt * D;
-  int* gcnt = counts + (size_t)bh * Mt;
-  float* part = SMEM ? sm : gvs;
-  int* cnt = SMEM ? reinterpret_cast<int*>(sm + (size_t)Mt * D) : gcnt;
-  if (SMEM) {
-    float4* s4 = reinterpret_cast<float4*>(sm);
-    for (int i = threadIdx.x; i < Mt * D / 4; i += blockDim.x) s4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = threadIdx.x; i < Mt; i += blockDim.x) cnt[i] = 0;
-    __syncthreads();
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int k0 = blockIdx.x * chunk;
-  const int k1 = min(N, k0 + chunk);
-  const int per = (k1 - k0 + nw - 1) / nw;
-  const int j0 = k0 + warp * per;
-  const int j1 = min(k1, j0 + per);
-  const int32_t* asg = assign + (size_t)bh * N;
-  const T* vb = V + (size_t)bh * N * D + lane * E;
-
-  float accP[E], accC[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
-  int curP = -1, curC = -1, nP = 0, nC = 0;
-  for (int jb = j0; jb < j1; jb += kAggBatch) {
-    int code[kAggBatch];
-    float v[kAggBatch][E];
-#pragma unroll
-    for (int u = 0; u < kAggBatch; ++u) {
-      const int j = jb + u;
-      if (j < j1) {
-        code[u] = __ldg(asg + j);
-        loadE<E>(vb + (size_t)j * D, v[u]);
-      } else {
-        code[u] = -1;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kAggBatch; ++u) {
-      const int c = code[u];
-      if (c < 0) break;
-      const int p = c < M0 ? c : (c - M0) / C;
-      if (p != curP) {
-        if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
-        curP = p;
-        nP = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) accP[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < E; ++e) accP[e] += v[u][e];
-      ++nP;
-      if (c >= M0) {
-        if (c != curC) {
-          if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
-          curC = c;
-          nC = 0;
-#pragma unroll
-          for (int e = 0; e < E; ++e) accC[e] = 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) accC[e] += v[u][e];
-        ++nC;
-      }
-    }
-  }
-  if (curP >= 0) flush_run<E>(part, cnt, curP, accP, nP, lane, D);
-  if (curC >= 0) flush_run<E>(part, cnt, curC, accC, nC, lane, D);
-  if (SMEM) {
-    __syncthreads();
-    const float4* s4 = reinterpret_cast<const float4*>(sm);
-    for (int i = threadIdx.x; i < Mt * D / 4; i += blockDim.x) {
-      const int row = i / (D / 4);
-      if (cnt[row] > 0) {
-        const float4 a = s4[i];
-        red_add_v4(gvs + (size_t)4 * i, a.x, a.y, a.z, a.w);
-      }
-    }
-    for (int r = threadIdx.x; r < Mt; r += blockDim.x)
-      if (cnt[r] > 0) atomicAdd(gcnt + r, cnt[r]);
-  }
-}
-
 // Streaming variant (the default): every warp owns a contiguous range of
-// keys of one head (so runs of equal codes stay long), lanes cover the head
-// dimension, value rows are loaded straight from global memory sixteen keys
-// ahead, codes one 32-key group ahead.  Per 32-key group, warp ballots mark
-// where runs start, so the per-key work is a bit test and two adds.  A run
-// is flushed with one vector reduction per lane into the global statistics
-// (L2-resident) and one count reduction; there are no shared-memory atomics
-// and no per-CTA partials.
-constexpr int kStreamThreads = 256;
-constexpr int kStreamBatch = 16;
+// keys of one head (so runs of equal codes stay long) and streams it through
+// its own four-slot shared-memory ring: lane 0 issues 1-D bulk copies of the
+// next 32 value rows and 32 codes, so each warp runs on its own and about
+// 128 KB are in flight per SM.  Per 32-key group, warp ballots mark where
+// runs start; the per-key work is a bit test and two adds with lanes over the
+// head dimension.  A finished run is added to the global value sums (L2
+// resident) with one vector reduction per lane.  Counts are not touched here:
+// the assignment kernels produce them.
+constexpr int kStreamWarps = 8;
+constexpr int kStreamThreads = kStreamWarps * 32;
+constexpr int kStreamSlots = 4;
+constexpr int kStreamGroup = 32;  // keys per slot
 
 template <int E>
-__device__ __forceinline__ void flush_global(float* vsum, int32_t* counts, int code, const float* acc,
-                                             int n, int lane, int D) {
+__device__ __forceinline__ void flush_sum(float* vsum, int code, const float* acc, int lane, int D) {
   float* row = vsum + (size_t)code * D + lane * E;
   if constexpr (E == 2) {
     asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(row), "f"(acc[0]), "f"(acc[1]) : "memory");
   } else {
     red_add_v4(row, acc[0], acc[1], acc[2], acc[3]);
   }
-  if (lane == 0) atomicAdd(counts + code, n);
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kStreamThreads, 3) aggregate_stream_kernel(
-    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
-    int32_t* __restrict__ counts, int BH, int N, int M0, int C, int keys_per_warp, int log2C) {
+__global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
+    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum, int BH, int N,
+    int M0, int C, int keys_per_warp, int log2C, unsigned int* err) {
   constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * (kStreamThreads / 32) + (threadIdx.x >> 5);
+  constexpr int RB = D * (int)sizeof(T);
+  constexpr int SLOT = kStreamGroup * RB + kStreamGroup * 4;  // values then codes
+  extern __shared__ __align__(128) uint8_t smraw[];
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  uint8_t* ring = smraw + (size_t)wl * kStreamSlots * SLOT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStreamWarps * kStreamSlots * SLOT) +
+                   wl * kStreamSlots;
+  const int gw = blockIdx.x * kStreamWarps + wl;
   const int warps_per_head = (N + keys_per_warp - 1) / keys_per_warp;
   const int bh = gw / warps_per_head;
   const int j0 = (gw % warps_per_head) * keys_per_warp;
   const int j1 = min(N, j0 + keys_per_warp);
-  if (bh >= BH || j0 >= j1) return;
+  if (bh >= BH || j0 >= j1) return;  // whole warp leaves; no block-wide barrier follows
   const int Mt = M0 * (1 + C);
   float* vs = vsum + (size_t)bh * Mt * D;
-  int32_t* ns = counts + (size_t)bh * Mt;
-  const T* vb = V + (size_t)bh * N * D + lane * E;
+  const T* vb = V + (size_t)bh * N * D;
   const int32_t* asg = assign + (size_t)bh * N;
+  const int ngroups = (j1 - j0 + kStreamGroup - 1) / kStreamGroup;
+
+  if (lane == 0) {
+    for (int q = 0; q < kStreamSlots; ++q) tc::mbar_init(&full[q], 1);
+    tc::fence_mbar_init();
+  }
+  __syncwarp();
+  auto issue = [&](int g) {
+    const int slot = g % kStreamSlots;
+    const int k = j0 + g * kStreamGroup;
+    const int nk = min(kStreamGroup, j1 - k);
+    const uint32_t vbytes = (uint32_t)nk * RB;
+    // codes go in whole 16-byte pieces; a ragged tail (N % 4 != 0) is read directly
+    const uint32_t cbytes = (uint32_t)(nk & ~3) * 4;
+    tc::mbar_arrive_expect_tx(&full[slot], vbytes + cbytes);
+    uint8_t* dst = ring + (size_t)slot * SLOT;
+    tc::bulk_g2s(dst, vb + (size_t)k * D, vbytes, &full[slot]);
+    if (cbytes) tc::bulk_g2s(dst + kStreamGroup * RB, asg + k, cbytes, &full[slot]);
+  };
+  if (lane == 0)
+    for (int g = 0; g < kStreamSlots && g < ngroups; ++g) issue(g);
 
   float accP[E], accC[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
-  int curP = -1, curC = -1, nP = 0, nC = 0;
-  int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
-  for (int g = j0; g < j1; g += 32) {
-    const int code = code_next;
-    code_next = g + 32 + lane < j1 ? __ldg(asg + g + 32 + lane) : -1;
+  int curP = -1, curC = -1;
+  bool timed_out = false;
+  for (int g = 0; g < ngroups; ++g) {
+    const int slot = g % kStreamSlots;
+    if (!tc::mbar_wait(&full[slot], (g / kStreamSlots) & 1)) timed_out = true;
+    const uint8_t* sl = ring + (size_t)slot * SLOT;
+    const int nk = min(kStreamGroup, j1 - (j0 + g * kStreamGroup));
+    const int code = lane < (nk & ~3) ? reinterpret_cast<const int*>(sl + kStreamGroup * RB)[lane]
+                     : lane < nk ? __ldg(asg + j0 + g * kStreamGroup + lane) : -1;
     const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / max(C, 1));
     const int prevc = __shfl_up_sync(0xffffffffu, code, 1);
     const int prevp = __shfl_up_sync(0xffffffffu, par, 1);
-    const unsigned live = __ballot_sync(0xffffffffu, code >= 0);
-    // run starts relative to the previous key of this group (lane 0 compares with the carry)
     const unsigned newP = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? par != curP : prevp != par));
     const unsigned isC = __ballot_sync(0xffffffffu, code >= M0);
     const unsigned newC = __ballot_sync(0xffffffffu, code >= M0 && (lane == 0 ? code != curC : prevc != code));
-    const int nlive = __popc(live);
-    for (int u0 = 0; u0 < nlive; u0 += kStreamBatch) {
-      float v[kStreamBatch][E];
-#pragma unroll
-      for (int b = 0; b < kStreamBatch; ++b)
-        if (u0 + b < nlive) loadE<E>(vb + (size_t)(g + u0 + b) * D, v[b]);
-#pragma unroll
-      for (int b = 0; b < kStreamBatch; ++b) {
-        const int u = u0 + b;
-        if (u >= nlive) break;
-        const unsigned bit = 1u << u;
-        if (newP & bit) {
-          if (curP >= 0) flush_global<E>(vs, ns, curP, accP, nP, lane, D);
-          curP = __shfl_sync(0xffffffffu, par, u);
-          nP = 0;
-#pragma unroll
-          for (int e = 0; e < E; ++e) accP[e] = 0.f;
+    const uint8_t* rows = sl + lane * E * sizeof(T);
+#pragma unroll 4
+    for (int u = 0; u < nk; ++u) {
+      float v[E];
+      if constexpr (sizeof(T) == 2) {
+        if constexpr (E == 2) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + (size_t)u * RB);
+          v[0] = bf16_lo(w); v[1] = bf16_hi(w);
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(rows + (size_t)u * RB);
+          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
         }
+      } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) accP[e] += v[b][e];
-        ++nP;
-        if (isC & bit) {
-          if (newC & bit) {
-            // the previous key may have stayed at a parent: compare with the open run
-            const int c = __shfl_sync(0xffffffffu, code, u);
-            if (c != curC) {
-              if (curC >= 0) flush_global<E>(vs, ns, curC, accC, nC, lane, D);
-              curC = c;
-              nC = 0;
+        for (int e = 0; e < E; ++e) v[e] = reinterpret_cast<const float*>(rows + (size_t)u * RB)[e];
+      }
+      const unsigned bit = 1u << u;
+      if (newP & bit) {
+        if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
+        curP = __shfl_sync(0xffffffffu, par, u);
 #pragma unroll
-              for (int e = 0; e < E; ++e) accC[e] = 0.f;
-            }
+        for (int e = 0; e < E; ++e) accP[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) accP[e] += v[e];
+      if (isC & bit) {
+        if (newC & bit) {
+          // the previous key may have stayed at a parent: compare with the open run
+          const int c = __shfl_sync(0xffffffffu, code, u);
+          if (c != curC) {
+            if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
+            curC = c;
+#pragma unroll
+            for (int e = 0; e < E; ++e) accC[e] = 0.f;
           }
-#pragma unroll
-          for (int e = 0; e < E; ++e) accC[e] += v[b][e];
-          ++nC;
         }
+#pragma unroll
+        for (int e = 0; e < E; ++e) accC[e] += v[e];
       }
     }
+    __syncwarp();  // the slot has been read by every lane
+    if (lane == 0 && g + kStreamSlots < ngroups) issue(g + kStreamSlots);
   }
-  if (curP >= 0) flush_global<E>(vs, ns, curP, accP, nP, lane, D);
-  if (curC >= 0) flush_global<E>(vs, ns, curC, accC, nC, lane, D);
+  if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
+  if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
+  if (timed_out && lane == 0) atomicOr(err, kErrTimeout);
 }
 
 // ---- deterministic variant ------------------------------------------------
@@ -395,8 +324,6 @@ __global__ void det_combine_kernel(const float* __restrict__ seg, const int* __r
   }
 }
 
-size_t agg_smem_bytes(const Shape& s) { return (size_t)s.Mt() * (s.d + 1) * sizeof(float); }
-
 }  // namespace
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -414,25 +341,32 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
                              LaunchLog& log) {
   cudaError_t e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * s.Mt() * s.d * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), st);
-  if (e != cudaSuccess) return e;
+  (void)counts;
   const int sms = num_sms();
   {
     int log2C = -1;
     for (int b = 0; b <= 3; ++b)
       if (s.C == (1 << b)) log2C = b;
-    // about 24 warps per SM in total (3 CTAs), each a contiguous multiple of 32 keys
+    const size_t row_bytes = (size_t)s.d * (dt == AVQ_F32 ? 4 : 2);
+    const size_t slot = kStreamGroup * row_bytes + kStreamGroup * 4;
+    const size_t smem = (size_t)kStreamWarps * kStreamSlots * slot + kStreamWarps * kStreamSlots * 8;
+    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (220 * 1024) / smem));
+    // about per_sm CTAs per SM in total, each warp a contiguous multiple of 32 keys
     const long long total_keys = (long long)s.BH() * s.N;
-    const long long want_warps = (long long)sms * 24;
+    const long long want_warps = (long long)sms * per_sm * kStreamWarps;
     int kpw = (int)((total_keys + want_warps - 1) / want_warps);
     kpw = ((kpw + 31) / 32) * 32;
     if (kpw < 64) kpw = 64;
     const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
-    const int wpb = kStreamThreads / 32;
-    const unsigned blocks = (unsigned)((warps + wpb - 1) / wpb);
-#define AVQ_STREAM(T, D)                                                                             \
-  aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, counts, \
-                                                                   s.BH(), s.N, s.M0, s.C, kpw, log2C)
+    const unsigned blocks = (unsigned)((warps + kStreamWarps - 1) / kStreamWarps);
+#define AVQ_STREAM(T, D)                                                                              \
+  do {                                                                                                \
+    auto kern = aggregate_stream_kernel<T, D>;                                                        \
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
+    if (e != cudaSuccess) return e;                                                                   \
+    kern<<<blocks, kStreamThreads, smem, st>>>((const T*)V, assign, vsum, s.BH(), s.N, s.M0, s.C, kpw, \
+                                               log2C, err);                                           \
+  } while (0)
     if (dt == AVQ_F32) {
       if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
     } else {
@@ -440,28 +374,8 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
     }
 #undef AVQ_STREAM
     log.add("aggregate_stream");
-    (void)err;
     return cudaGetLastError();
   }
-  // partials too large for shared memory: runs flushed straight to global memory
-  int per_head = (sms >= s.BH() ? sms / s.BH() : 1) * 4;
-  int chunk = (s.N + per_head - 1) / per_head;
-  chunk = ((chunk + 511) / 512) * 512;
-  if (chunk < 512) chunk = 512;
-  dim3 grid((s.N + chunk - 1) / chunk, s.BH());
-  if (dt == AVQ_F32) {
-    if (s.d == 64)
-      aggregate_kernel<float, 64, false><<<grid, kAggThreads, 0, st>>>((const float*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
-    else
-      aggregate_kernel<float, 128, false><<<grid, kAggThreads, 0, st>>>((const float*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
-  } else {
-    if (s.d == 64)
-      aggregate_kernel<bf16, 64, false><<<grid, kAggThreads, 0, st>>>((const bf16*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
-    else
-      aggregate_kernel<bf16, 128, false><<<grid, kAggThreads, 0, st>>>((const bf16*)V, assign, vsum, counts, s.N, s.M0, s.C, chunk);
-  }
-  log.add("aggregate_global");
-  return cudaGetLastError();
 }
 
 cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,

@@ -31,12 +31,14 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) assign_simt_kernel(const T* __restrict__ K,
                                                           const T* __restrict__ parents,
                                                           const T* __restrict__ children,
-                                                          int32_t* __restrict__ assign, int H,
+                                                          int32_t* __restrict__ assign,
+                                                          int32_t* __restrict__ counts, int H,
                                                           int N, int M0, int C) {
   const int bh = blockIdx.y;
   const int h = bh % H;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= N) return;
+  const int j0 = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool valid = j0 < N;
+  const int j = valid ? j0 : N - 1;  // out-of-range lanes recompute the last key, store nothing
   float k[D];
   const T* kp = K + ((size_t)bh * N + j) * D;
 #pragma unroll
@@ -68,17 +70,19 @@ __global__ void __launch_bounds__(128) assign_simt_kernel(const T* __restrict__ 
     }
     if (dchild < best) code = M0 + a * C + cstar;
   }
-  assign[(size_t)bh * N + j] = code;
+  if (valid) assign[(size_t)bh * N + j] = code;
+  count_codes(counts + (size_t)bh * M0 * (1 + C), code, valid, M0, C);
 }
 
 cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
-                               const void* children, int32_t* assign, cudaStream_t st,
-                               LaunchLog& log) {
+                               const void* children, int32_t* assign, int32_t* counts,
+                               cudaStream_t st, LaunchLog& log) {
   dim3 grid((s.N + 127) / 128, s.BH());
   dim3 block(128);
 #define AVQ_LAUNCH(T, D)                                                                       \
   assign_simt_kernel<T, D><<<grid, block, 0, st>>>((const T*)K, (const T*)parents,            \
-                                                   (const T*)children, assign, s.H, s.N, s.M0, \
+                                                   (const T*)children, assign, counts, s.H,   \
+                                                   s.N, s.M0,                                  \
                                                    s.C)
   if (dt == AVQ_F32) {
     if (s.d == 64) AVQ_LAUNCH(float, 64); else AVQ_LAUNCH(float, 128);

@@ -42,6 +42,7 @@ struct AssignArgs {
   const bf16* cw;      // [H][Mt/8][KH][8][64] swizzled codeword atoms
   const float* norms;  // [H][Mt] squared norms
   int32_t* assign;     // [BH][N]
+  int32_t* counts;     // [BH][Mt], accumulated (zeroed by the caller)
   unsigned int* err;
   int H, N, M0, C, nblk, ntiles, tiles_per_cta;
 };
@@ -339,6 +340,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     }
     const int row = blk * kKeys + tid;
     if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
+    count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
 
     tc::tc_fence_before();
     __syncthreads();  // K slot and TMEM free
@@ -417,7 +419,8 @@ size_t assign_tc_workspace(const Shape& s) {
 }
 
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents, const void* children,
-                             int32_t* assign, void* ws, unsigned int* err, cudaStream_t st, LaunchLog& log) {
+                             int32_t* assign, int32_t* counts, void* ws, unsigned int* err, cudaStream_t st,
+                             LaunchLog& log) {
   bf16* cw = static_cast<bf16*>(ws);
   float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
   const long long work = (long long)s.H * s.Mt();
@@ -439,6 +442,7 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
   a.cw = cw;
   a.norms = norms;
   a.assign = assign;
+  a.counts = counts;
   a.err = err;
   a.H = s.H;
   a.N = s.N;

@@ -221,10 +221,12 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
   cudaError_t e;
   unsigned int* err = error_word();
   if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+  e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "zero counts");
   if (use_tc) {
-    e = launch_assign_tc(s, K, parents, children, assign, ws, err, cs, log);
+    e = launch_assign_tc(s, K, parents, children, assign, counts, ws, err, cs, log);
   } else {
-    e = launch_assign_simt(s, dtype, K, parents, children, assign, cs, log);
+    e = launch_assign_simt(s, dtype, K, parents, children, assign, counts, cs, log);
   }
   if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
   if (deterministic)

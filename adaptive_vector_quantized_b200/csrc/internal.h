@@ -26,12 +26,13 @@ struct LaunchLog {
 };
 
 // ---- stage 1 ------------------------------------------------------------
-// Algorithm 1 steps 3-16 (assignment only): writes assign[BH][N].
+// Algorithm 1 steps 3-16 (assignment): writes assign[BH][N] and adds the key
+// counts (Eq. 3) into counts[BH][Mt], which the caller zeroes first.
 cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
-                               const void* children, int32_t* assign, cudaStream_t st,
-                               LaunchLog& log);
-// Algorithm 1 steps 1, 8, 16 (aggregation for given codes), atomics variant.
-// vsum/counts are zeroed inside.
+                               const void* children, int32_t* assign, int32_t* counts,
+                               cudaStream_t st, LaunchLog& log);
+// Algorithm 1 steps 1, 8, 16 (value sums for given codes), streaming variant.
+// vsum is zeroed inside; counts are left to the assignment kernels.
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
                              LaunchLog& log);
@@ -46,8 +47,8 @@ cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
 bool assign_tc_supported(const Shape& s, avq_dtype dt);
 size_t assign_tc_workspace(const Shape& s);
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
-                             const void* children, int32_t* assign, void* ws, unsigned int* err,
-                             cudaStream_t st, LaunchLog& log);
+                             const void* children, int32_t* assign, int32_t* counts, void* ws,
+                             unsigned int* err, cudaStream_t st, LaunchLog& log);
 
 // ---- stage 2 ------------------------------------------------------------
 cudaError_t launch_attention_simt(const Shape& s, avq_dtype dt, const void* Q, const void* parents,
