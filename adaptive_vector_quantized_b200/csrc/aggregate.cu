@@ -24,17 +24,20 @@ namespace avq {
 namespace {
 
 // Streaming variant (the default): every warp owns a contiguous range of
-// keys of one head (so runs of equal codes stay long) and streams it through
-// its own four-slot shared-memory ring: lane 0 issues 1-D bulk copies of the
-// next 32 value rows and 32 codes, so each warp runs on its own and about
-// 128 KB are in flight per SM.  Per 32-key group, warp ballots mark where
+// keys of one head (so runs of equal codes stay long) and streams its value
+// rows through its own shared-memory ring of up to four 32-row slots: lane 0
+// issues 1-D bulk copies of the next groups (row offsets are multiples of
+// 128 bytes, so every copy is 16-byte aligned), each warp runs on its own and
+// about 128 KB are in flight per SM.  Codes are read with plain coalesced
+// loads one group ahead (a head's codes start at bh*N*4 bytes, which need not
+// be 16-byte aligned).  Per 32-key group, warp ballots mark where
 // runs start; the per-key work is a bit test and two adds with lanes over the
 // head dimension.  A finished run is added to the global value sums (L2
 // resident) with one vector reduction per lane.  Counts are not touched here:
 // the assignment kernels produce them.
 constexpr int kStreamWarps = 8;
 constexpr int kStreamThreads = kStreamWarps * 32;
-constexpr int kStreamSlots = 4;
+constexpr int kStreamMaxSlots = 4;
 constexpr int kStreamGroup = 32;  // keys per slot
 
 template <int E>
@@ -50,15 +53,14 @@ __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* ac
 template <typename T, int D>
 __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum, int BH, int N,
-    int M0, int C, int keys_per_warp, int log2C, unsigned int* err) {
+    int M0, int C, int keys_per_warp, int log2C, int nslots, unsigned int* err) {
   constexpr int E = D / 32;
   constexpr int RB = D * (int)sizeof(T);
-  constexpr int SLOT = kStreamGroup * RB + kStreamGroup * 4;  // values then codes
+  constexpr int SLOT = kStreamGroup * RB;
   extern __shared__ __align__(128) uint8_t smraw[];
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  uint8_t* ring = smraw + (size_t)wl * kStreamSlots * SLOT;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStreamWarps * kStreamSlots * SLOT) +
-                   wl * kStreamSlots;
+  uint8_t* ring = smraw + (size_t)wl * nslots * SLOT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStreamWarps * nslots * SLOT) + wl * nslots;
   const int gw = blockIdx.x * kStreamWarps + wl;
   const int warps_per_head = (N + keys_per_warp - 1) / keys_per_warp;
   const int bh = gw / warps_per_head;
@@ -72,24 +74,21 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   const int ngroups = (j1 - j0 + kStreamGroup - 1) / kStreamGroup;
 
   if (lane == 0) {
-    for (int q = 0; q < kStreamSlots; ++q) tc::mbar_init(&full[q], 1);
+    for (int q = 0; q < nslots; ++q) tc::mbar_init(&full[q], 1);
     tc::fence_mbar_init();
   }
   __syncwarp();
   auto issue = [&](int g) {
-    const int slot = g % kStreamSlots;
+    const int slot = g % nslots;
     const int k = j0 + g * kStreamGroup;
     const int nk = min(kStreamGroup, j1 - k);
-    const uint32_t vbytes = (uint32_t)nk * RB;
-    // codes go in whole 16-byte pieces; a ragged tail (N % 4 != 0) is read directly
-    const uint32_t cbytes = (uint32_t)(nk & ~3) * 4;
-    tc::mbar_arrive_expect_tx(&full[slot], vbytes + cbytes);
-    uint8_t* dst = ring + (size_t)slot * SLOT;
-    tc::bulk_g2s(dst, vb + (size_t)k * D, vbytes, &full[slot]);
-    if (cbytes) tc::bulk_g2s(dst + kStreamGroup * RB, asg + k, cbytes, &full[slot]);
+    const uint32_t vbytes = (uint32_t)nk * RB;  // k*RB and bh*N*RB are multiples of 128
+    tc::mbar_arrive_expect_tx(&full[slot], vbytes);
+    tc::bulk_g2s(ring + (size_t)slot * SLOT, vb + (size_t)k * D, vbytes, &full[slot]);
   };
   if (lane == 0)
-    for (int g = 0; g < kStreamSlots && g < ngroups; ++g) issue(g);
+    for (int g = 0; g < nslots && g < ngroups; ++g) issue(g);
+  int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
 
   float accP[E], accC[E];
 #pragma unroll
@@ -97,12 +96,15 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   int curP = -1, curC = -1;
   bool timed_out = false;
   for (int g = 0; g < ngroups; ++g) {
-    const int slot = g % kStreamSlots;
-    if (!tc::mbar_wait(&full[slot], (g / kStreamSlots) & 1)) timed_out = true;
-    const uint8_t* sl = ring + (size_t)slot * SLOT;
+    const int slot = g % nslots;
     const int nk = min(kStreamGroup, j1 - (j0 + g * kStreamGroup));
-    const int code = lane < (nk & ~3) ? reinterpret_cast<const int*>(sl + kStreamGroup * RB)[lane]
-                     : lane < nk ? __ldg(asg + j0 + g * kStreamGroup + lane) : -1;
+    const int code = code_next;
+    {
+      const int jn = j0 + (g + 1) * kStreamGroup + lane;
+      code_next = jn < j1 ? __ldg(asg + jn) : -1;
+    }
+    if (!tc::mbar_wait(&full[slot], (g / nslots) & 1)) timed_out = true;
+    const uint8_t* sl = ring + (size_t)slot * SLOT;
     const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / max(C, 1));
     const int prevc = __shfl_up_sync(0xffffffffu, code, 1);
     const int prevp = __shfl_up_sync(0xffffffffu, par, 1);
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
       }
     }
     __syncwarp();  // the slot has been read by every lane
-    if (lane == 0 && g + kStreamSlots < ngroups) issue(g + kStreamSlots);
+    if (lane == 0 && g + nslots < ngroups) issue(g + nslots);
   }
   if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
   if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
@@ -348,8 +350,10 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
     for (int b = 0; b <= 3; ++b)
       if (s.C == (1 << b)) log2C = b;
     const size_t row_bytes = (size_t)s.d * (dt == AVQ_F32 ? 4 : 2);
-    const size_t slot = kStreamGroup * row_bytes + kStreamGroup * 4;
-    const size_t smem = (size_t)kStreamWarps * kStreamSlots * slot + kStreamWarps * kStreamSlots * 8;
+    const size_t slot = kStreamGroup * row_bytes;  // 4 KB (bf16, d=64) .. 16 KB (fp32, d=128)
+    const int nslots = (int)std::max<size_t>(
+        1, std::min<size_t>(kStreamMaxSlots, (200 * 1024) / (kStreamWarps * (slot + 8))));
+    const size_t smem = (size_t)kStreamWarps * nslots * (slot + 8);
     const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (220 * 1024) / smem));
     // about per_sm CTAs per SM in total, each warp a contiguous multiple of 32 keys
     const long long total_keys = (long long)s.BH() * s.N;
@@ -365,7 +369,7 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
     if (e != cudaSuccess) return e;                                                                   \
     kern<<<blocks, kStreamThreads, smem, st>>>((const T*)V, assign, vsum, s.BH(), s.N, s.M0, s.C, kpw, \
-                                               log2C, err);                                           \
+                                               log2C, nslots, err);                                   \
   } while (0)
     if (dt == AVQ_F32) {
       if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
