@@ -24,21 +24,15 @@ namespace avq {
 namespace {
 
 // Streaming variant (the default): every warp owns a contiguous range of
-// keys of one head (so runs of equal codes stay long) and streams its value
-// rows through its own shared-memory ring of up to four 32-row slots: lane 0
-// issues 1-D bulk copies of the next groups (row offsets are multiples of
-// 128 bytes, so every copy is 16-byte aligned), each warp runs on its own and
-// about 128 KB are in flight per SM.  Codes are read with plain coalesced
-// loads one group ahead (a head's codes start at bh*N*4 bytes, which need not
-// be 16-byte aligned).  Per 32-key group, warp ballots mark where
-// runs start; the per-key work is a bit test and two adds with lanes over the
-// head dimension.  A finished run is added to the global value sums (L2
-// resident) with one vector reduction per lane.  Counts are not touched here:
-// the assignment kernels produce them.
-constexpr int kStreamWarps = 8;
-constexpr int kStreamThreads = kStreamWarps * 32;
-constexpr int kStreamMaxSlots = 4;
-constexpr int kStreamGroup = 32;  // keys per slot
+// keys of one head (so runs of equal codes stay long), lanes cover the head
+// dimension, value rows are loaded straight from global memory in batches of
+// eight keys, codes one 32-key group ahead.  Per 32-key group, warp ballots
+// mark where runs start, so the per-key work is a bit test and two adds.  A
+// finished run is added to the global value sums (L2 resident) with one
+// vector reduction per lane; there are no shared-memory atomics and no
+// per-CTA partials.  Counts are produced by the assignment kernels.
+constexpr int kStreamThreads = 256;
+constexpr int kStreamBatch = 8;
 
 template <int E>
 __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* acc, int lane, int D) {
@@ -53,110 +47,74 @@ __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* ac
 template <typename T, int D>
 __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum, int BH, int N,
-    int M0, int C, int keys_per_warp, int log2C, int nslots, unsigned int* err) {
+    int M0, int C, int keys_per_warp, int log2C) {
   constexpr int E = D / 32;
-  constexpr int RB = D * (int)sizeof(T);
-  constexpr int SLOT = kStreamGroup * RB;
-  extern __shared__ __align__(128) uint8_t smraw[];
-  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  uint8_t* ring = smraw + (size_t)wl * nslots * SLOT;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStreamWarps * nslots * SLOT) + wl * nslots;
-  const int gw = blockIdx.x * kStreamWarps + wl;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (kStreamThreads / 32) + (threadIdx.x >> 5);
   const int warps_per_head = (N + keys_per_warp - 1) / keys_per_warp;
   const int bh = gw / warps_per_head;
   const int j0 = (gw % warps_per_head) * keys_per_warp;
   const int j1 = min(N, j0 + keys_per_warp);
-  if (bh >= BH || j0 >= j1) return;  // whole warp leaves; no block-wide barrier follows
+  if (bh >= BH || j0 >= j1) return;
   const int Mt = M0 * (1 + C);
   float* vs = vsum + (size_t)bh * Mt * D;
-  const T* vb = V + (size_t)bh * N * D;
+  const T* vb = V + (size_t)bh * N * D + lane * E;
   const int32_t* asg = assign + (size_t)bh * N;
-  const int ngroups = (j1 - j0 + kStreamGroup - 1) / kStreamGroup;
-
-  if (lane == 0) {
-    for (int q = 0; q < nslots; ++q) tc::mbar_init(&full[q], 1);
-    tc::fence_mbar_init();
-  }
-  __syncwarp();
-  auto issue = [&](int g) {
-    const int slot = g % nslots;
-    const int k = j0 + g * kStreamGroup;
-    const int nk = min(kStreamGroup, j1 - k);
-    const uint32_t vbytes = (uint32_t)nk * RB;  // k*RB and bh*N*RB are multiples of 128
-    tc::mbar_arrive_expect_tx(&full[slot], vbytes);
-    tc::bulk_g2s(ring + (size_t)slot * SLOT, vb + (size_t)k * D, vbytes, &full[slot]);
-  };
-  if (lane == 0)
-    for (int g = 0; g < nslots && g < ngroups; ++g) issue(g);
-  int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
 
   float accP[E], accC[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
   int curP = -1, curC = -1;
-  bool timed_out = false;
-  for (int g = 0; g < ngroups; ++g) {
-    const int slot = g % nslots;
-    const int nk = min(kStreamGroup, j1 - (j0 + g * kStreamGroup));
+  int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
+  for (int g = j0; g < j1; g += 32) {
     const int code = code_next;
-    {
-      const int jn = j0 + (g + 1) * kStreamGroup + lane;
-      code_next = jn < j1 ? __ldg(asg + jn) : -1;
-    }
-    if (!tc::mbar_wait(&full[slot], (g / nslots) & 1)) timed_out = true;
-    const uint8_t* sl = ring + (size_t)slot * SLOT;
+    code_next = g + 32 + lane < j1 ? __ldg(asg + g + 32 + lane) : -1;
     const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / max(C, 1));
     const int prevc = __shfl_up_sync(0xffffffffu, code, 1);
     const int prevp = __shfl_up_sync(0xffffffffu, par, 1);
+    const unsigned live = __ballot_sync(0xffffffffu, code >= 0);
+    // run starts relative to the previous key (lane 0 compares with the open run)
     const unsigned newP = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? par != curP : prevp != par));
     const unsigned isC = __ballot_sync(0xffffffffu, code >= M0);
     const unsigned newC = __ballot_sync(0xffffffffu, code >= M0 && (lane == 0 ? code != curC : prevc != code));
-    const uint8_t* rows = sl + lane * E * sizeof(T);
-#pragma unroll 4
-    for (int u = 0; u < nk; ++u) {
-      float v[E];
-      if constexpr (sizeof(T) == 2) {
-        if constexpr (E == 2) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + (size_t)u * RB);
-          v[0] = bf16_lo(w); v[1] = bf16_hi(w);
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(rows + (size_t)u * RB);
-          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    const int nlive = __popc(live);
+    for (int u0 = 0; u0 < nlive; u0 += kStreamBatch) {
+      float v[kStreamBatch][E];
+#pragma unroll
+      for (int b = 0; b < kStreamBatch; ++b)
+        if (u0 + b < nlive) loadE<E>(vb + (size_t)(g + u0 + b) * D, v[b]);
+#pragma unroll
+      for (int b = 0; b < kStreamBatch; ++b) {
+        const int u = u0 + b;
+        if (u >= nlive) break;
+        const unsigned bit = 1u << u;
+        if (newP & bit) {
+          if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
+          curP = __shfl_sync(0xffffffffu, par, u);
+#pragma unroll
+          for (int e = 0; e < E; ++e) accP[e] = 0.f;
         }
-      } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) v[e] = reinterpret_cast<const float*>(rows + (size_t)u * RB)[e];
-      }
-      const unsigned bit = 1u << u;
-      if (newP & bit) {
-        if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
-        curP = __shfl_sync(0xffffffffu, par, u);
+        for (int e = 0; e < E; ++e) accP[e] += v[b][e];
+        if (isC & bit) {
+          if (newC & bit) {
+            // the previous key may have stayed at a parent: compare with the open run
+            const int c = __shfl_sync(0xffffffffu, code, u);
+            if (c != curC) {
+              if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
+              curC = c;
 #pragma unroll
-        for (int e = 0; e < E; ++e) accP[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < E; ++e) accP[e] += v[e];
-      if (isC & bit) {
-        if (newC & bit) {
-          // the previous key may have stayed at a parent: compare with the open run
-          const int c = __shfl_sync(0xffffffffu, code, u);
-          if (c != curC) {
-            if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
-            curC = c;
-#pragma unroll
-            for (int e = 0; e < E; ++e) accC[e] = 0.f;
+              for (int e = 0; e < E; ++e) accC[e] = 0.f;
+            }
           }
-        }
 #pragma unroll
-        for (int e = 0; e < E; ++e) accC[e] += v[e];
+          for (int e = 0; e < E; ++e) accC[e] += v[b][e];
+        }
       }
     }
-    __syncwarp();  // the slot has been read by every lane
-    if (lane == 0 && g + nslots < ngroups) issue(g + nslots);
   }
   if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
   if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
-  if (timed_out && lane == 0) atomicOr(err, kErrTimeout);
 }
 
 // ---- deterministic variant ------------------------------------------------
@@ -345,41 +303,29 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   if (e != cudaSuccess) return e;
   (void)counts;
   const int sms = num_sms();
-  {
-    int log2C = -1;
-    for (int b = 0; b <= 3; ++b)
-      if (s.C == (1 << b)) log2C = b;
-    const size_t row_bytes = (size_t)s.d * (dt == AVQ_F32 ? 4 : 2);
-    const size_t slot = kStreamGroup * row_bytes;  // 4 KB (bf16, d=64) .. 16 KB (fp32, d=128)
-    const int nslots = (int)std::max<size_t>(
-        1, std::min<size_t>(kStreamMaxSlots, (200 * 1024) / (kStreamWarps * (slot + 8))));
-    const size_t smem = (size_t)kStreamWarps * nslots * (slot + 8);
-    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (220 * 1024) / smem));
-    // about per_sm CTAs per SM in total, each warp a contiguous multiple of 32 keys
-    const long long total_keys = (long long)s.BH() * s.N;
-    const long long want_warps = (long long)sms * per_sm * kStreamWarps;
-    int kpw = (int)((total_keys + want_warps - 1) / want_warps);
-    kpw = ((kpw + 31) / 32) * 32;
-    if (kpw < 64) kpw = 64;
-    const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
-    const unsigned blocks = (unsigned)((warps + kStreamWarps - 1) / kStreamWarps);
-#define AVQ_STREAM(T, D)                                                                              \
-  do {                                                                                                \
-    auto kern = aggregate_stream_kernel<T, D>;                                                        \
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
-    if (e != cudaSuccess) return e;                                                                   \
-    kern<<<blocks, kStreamThreads, smem, st>>>((const T*)V, assign, vsum, s.BH(), s.N, s.M0, s.C, kpw, \
-                                               log2C, nslots, err);                                   \
-  } while (0)
-    if (dt == AVQ_F32) {
-      if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
-    } else {
-      if (s.d == 64) AVQ_STREAM(bf16, 64); else AVQ_STREAM(bf16, 128);
-    }
-#undef AVQ_STREAM
-    log.add("aggregate_stream");
-    return cudaGetLastError();
+  int log2C = -1;
+  for (int b = 0; b <= 3; ++b)
+    if (s.C == (1 << b)) log2C = b;
+  // grid sized for about 32 resident warps per SM, each a contiguous multiple of 32 keys
+  const long long total_keys = (long long)s.BH() * s.N;
+  const long long want_warps = (long long)sms * 32;
+  int kpw = (int)((total_keys + want_warps - 1) / want_warps);
+  kpw = ((kpw + 31) / 32) * 32;
+  if (kpw < 64) kpw = 64;
+  const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
+  const unsigned blocks = (unsigned)((warps + (kStreamThreads / 32) - 1) / (kStreamThreads / 32));
+#define AVQ_STREAM(T, D)                                                                            \
+  aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, s.BH(), \
+                                                                   s.N, s.M0, s.C, kpw, log2C)
+  if (dt == AVQ_F32) {
+    if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
+  } else {
+    if (s.d == 64) AVQ_STREAM(bf16, 64); else AVQ_STREAM(bf16, 128);
   }
+#undef AVQ_STREAM
+  log.add("aggregate_stream");
+  (void)err;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,

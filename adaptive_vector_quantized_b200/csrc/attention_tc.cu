@@ -67,7 +67,8 @@ struct Smem {
   static constexpr int kW = kBI + kTile * 4;                // importance [256]
   static constexpr int kWP = kW + 256 * 4;                  // per-warp partial sums [4][kTile]
   static constexpr int kSEL = kWP + 4 * kTile * 4;          // selected parents [256]
-  static constexpr int kBAR = kSEL + 256 * 4;               // 3 mbarriers
+  static constexpr int kRK = kSEL + 256 * 4;                // partial ranks [2][128]
+  static constexpr int kBAR = kRK + 256 * 4;                // 4 mbarriers
   static constexpr int kMISC = kBAR + 32;                   // tmem base, abort flag
   static constexpr int kTotal = kMISC + 32;
   static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
@@ -130,8 +131,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   float* sWP = reinterpret_cast<float*>(sm + S::kWP);
   int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
   uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + S::kBAR);
-  uint64_t* bar_cp = bar_q + 1;
+  uint64_t* bar_cp = bar_q + 1;   // codeword tiles
   uint64_t* bar_mma = bar_q + 2;
+  uint64_t* bar_vb = bar_q + 3;   // value-sum tiles (waited on only before the value MMA)
+  int* sRK = reinterpret_cast<int*>(sm + S::kRK);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S::kMISC);
   int* sAbort = reinterpret_cast<int*>(sm + S::kMISC + 4);
 
@@ -151,6 +154,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
     tc::mbar_init(bar_q, 1);
     tc::mbar_init(bar_cp, 1);
     tc::mbar_init(bar_mma, 1);
+    tc::mbar_init(bar_vb, 1);
     tc::fence_mbar_init();
     *sAbort = 0;
     tc::prefetch_tensormap(&qmap);
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   const uint32_t tX = tmem + kTile;  // output accumulator, D columns
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-  uint32_t ph_cp = 0, ph_mma = 0;
+  uint32_t ph_cp = 0, ph_mma = 0, ph_vb = 0;
   if (tid == 0) {
     tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
 #pragma unroll
@@ -208,6 +212,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
     if (!tc::mbar_wait(bar_cp, ph_cp)) fail(a.err, sAbort);
     ph_cp ^= 1;
   };
+  auto wait_vb = [&]() {
+    if (!tc::mbar_wait(bar_vb, ph_vb)) fail(a.err, sAbort);
+    ph_vb ^= 1;
+  };
 
   float m = NEG_INF, z = 0.f;
   const int nT = (M0 + kTile - 1) / kTile;
@@ -224,15 +232,26 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       const int n = min(kTile, M0 - c0);
       if (tid == 0) {
         const uint32_t cwb = (uint32_t)n * D * 2;
-        tc::mbar_arrive_expect_tx(bar_cp, last ? 2 * cwb : cwb);
+        tc::mbar_arrive_expect_tx(bar_cp, cwb);
         tc::bulk_g2s(sCW, cw_h + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
-        if (last) tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
+        if (last) {
+          tc::mbar_arrive_expect_tx(bar_vb, cwb);
+          tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, cwb, bar_vb);
+        }
+      }
+      // a partial tile: zero the unused codeword rows so that the logits MMA can
+      // always run over 64 columns with finite results
+      for (int i = tid; i < (kTile - n) * KH * 8; i += 128) {
+        const int row = n + i / (KH * 8), rest = i % (KH * 8);
+        *reinterpret_cast<uint4*>(sCW + (row >> 3) * (KH * 1024) + (rest >> 3) * 1024 + (row & 7) * 128 +
+                                  (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
       }
       for (int j = tid; j < kTile; j += 128) {
         const float nf = j < n ? (float)__ldg(cnt + c0 + j) : 0.f;
         sNF[j] = nf;
         sBI[j] = nf > 0.f ? 0.f : NEG_INF;
       }
+      tc::fence_proxy_async_smem();
       if (!q_ready) {
         if (!tc::mbar_wait(bar_q, 0)) fail(a.err, sAbort);
         q_ready = true;
@@ -242,38 +261,44 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       if (*sAbort) goto done;
       if (tid == 0) {
         tc::tc_fence_after();
-        issue_logits(n);
+        issue_logits(kTile);
       }
       wait_mma();
       {
         uint32_t r[64];
         tmem_ld64(tS + lane_off, r);
-        // t = scaled log2 logit, -inf for empty codes (and columns >= n)
-        float tmax = NEG_INF;
+        const float4* bi4 = reinterpret_cast<const float4*>(sBI);
+        const float4* nf4 = reinterpret_cast<const float4*>(sNF);
+        // t = scaled log2 logit; the bias is 0 for non-empty codes, -inf for empty
+        // codes and unused columns (Eq. 18: those never set the max)
+        float tm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          // select, not add: TMEM columns past the tile may hold stale bits
-          const float tv = sBI[e] == 0.f ? __uint_as_float(r[e]) * sl2 : NEG_INF;
-          r[e] = __float_as_uint(tv);
-          tmax = fmaxf(tmax, tv);
+        for (int e = 0; e < 64; e += 4) {
+          const float4 b = bi4[e >> 2];
+          const float t0 = fmaf(__uint_as_float(r[e]), sl2, b.x), t1 = fmaf(__uint_as_float(r[e + 1]), sl2, b.y);
+          const float t2 = fmaf(__uint_as_float(r[e + 2]), sl2, b.z), t3 = fmaf(__uint_as_float(r[e + 3]), sl2, b.w);
+          r[e] = __float_as_uint(t0); r[e + 1] = __float_as_uint(t1);
+          r[e + 2] = __float_as_uint(t2); r[e + 3] = __float_as_uint(t3);
+          tm[0] = fmaxf(tm[0], t0); tm[1] = fmaxf(tm[1], t1); tm[2] = fmaxf(tm[2], t2); tm[3] = fmaxf(tm[3], t3);
         }
+        const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
         if (!last || sweeps == 1) {
           const float mn = fmaxf(m, tmax);
           if (mn != NEG_INF) {
-            float zt = 0.f;
-            if (sweeps == 1) {
-              // single sweep: keep A = 2^(t - m) in place
+            float zp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int e = 0; e < 64; ++e) {
-                const float av = tc::ex2(__uint_as_float(r[e]) - mn);
-                r[e] = __float_as_uint(av);
-                zt = fmaf(av, sNF[e], zt);
+            for (int e = 0; e < 64; e += 4) {
+              const float4 nf = nf4[e >> 2];
+              const float a0 = tc::ex2(__uint_as_float(r[e]) - mn), a1 = tc::ex2(__uint_as_float(r[e + 1]) - mn);
+              const float a2 = tc::ex2(__uint_as_float(r[e + 2]) - mn), a3 = tc::ex2(__uint_as_float(r[e + 3]) - mn);
+              zp[0] = fmaf(a0, nf.x, zp[0]); zp[1] = fmaf(a1, nf.y, zp[1]);
+              zp[2] = fmaf(a2, nf.z, zp[2]); zp[3] = fmaf(a3, nf.w, zp[3]);
+              if (sweeps == 1) {  // single sweep: keep A = 2^(t - m) in place
+                r[e] = __float_as_uint(a0); r[e + 1] = __float_as_uint(a1);
+                r[e + 2] = __float_as_uint(a2); r[e + 3] = __float_as_uint(a3);
               }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 64; ++e) zt = fmaf(tc::ex2(__uint_as_float(r[e]) - mn), sNF[e], zt);
             }
-            z = z * tc::ex2(m - mn) + zt;
+            z = z * tc::ex2(m - mn) + ((zp[0] + zp[1]) + (zp[2] + zp[3]));
             m = mn;
           }
         } else {
@@ -297,6 +322,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       if (last) {
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
+        wait_vb();
         __syncthreads();
         for (int j = tid; j < n; j += 128)
           sW[c0 + j] += sNF[j] * ((sWP[j] + sWP[kTile + j]) + (sWP[2 * kTile + j] + sWP[3 * kTile + j]));
@@ -314,17 +340,39 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   }
 
   // ---- top-P over the importance (descending, ties to the lower index) ----
+  // rank_j = #{l : w_l > w_j or (w_l == w_j and l < j)}; for M0 <= 64 two
+  // threads share each j, each counting over half of the l range
   {
     const int P = a.P;
-    for (int j = tid; j < M0; j += 128) {
-      const float wj = sW[j];
-      int rank = 0;
-      for (int l = 0; l < M0; ++l) {
-        const float wl = sW[l];
-        rank += (wl > wj) || (wl == wj && l < j);
+    if (M0 <= 64) {
+      const int j = tid % M0, half = tid / M0;
+      if (tid < 2 * M0) {
+        const float wj = sW[j];
+        const int l0 = half * (M0 >> 1), l1 = half ? M0 : (M0 >> 1);
+        int rank = 0;
+        for (int l = l0; l < l1; ++l) {
+          const float wl = sW[l];
+          rank += (wl > wj) || (wl == wj && l < j);
+        }
+        sRK[half * 128 + j] = rank;
       }
-      if (rank < P) sSEL[rank] = j;
-      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + j] = wj;
+      __syncthreads();
+      if (tid < M0) {
+        const int rank = sRK[tid] + sRK[128 + tid];
+        if (rank < P) sSEL[rank] = tid;
+        if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = sW[tid];
+      }
+    } else {
+      for (int j = tid; j < M0; j += 128) {
+        const float wj = sW[j];
+        int rank = 0;
+        for (int l = 0; l < M0; ++l) {
+          const float wl = sW[l];
+          rank += (wl > wj) || (wl == wj && l < j);
+        }
+        if (rank < P) sSEL[rank] = j;
+        if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + j] = wj;
+      }
     }
     __syncthreads();
     if (a.sel)
@@ -342,12 +390,17 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       const int slots = (np + 1) & ~1;
       const int n = slots * 8;
       if (tid == 0) {
-        tc::mbar_arrive_expect_tx(bar_cp, 2u * slots * KH * 1024);
+        tc::mbar_arrive_expect_tx(bar_cp, 1u * slots * KH * 1024);
+        tc::mbar_arrive_expect_tx(bar_vb, 1u * slots * KH * 1024);
         for (int r = 0; r < slots; ++r) {
           const int p = sSEL[q * kChunkParents + min(r, np - 1)];
           const size_t g = (size_t)(M0 / 8 + p) * KH * 512;
           tc::bulk_g2s(sCW + r * KH * 1024, cw_h + g, KH * 1024, bar_cp);
-          tc::bulk_g2s(sVB + r * KH * 1024, vb_bh + g, KH * 1024, bar_cp);
+        }
+        for (int r = 0; r < slots; ++r) {
+          const int p = sSEL[q * kChunkParents + min(r, np - 1)];
+          const size_t g = (size_t)(M0 / 8 + p) * KH * 512;
+          tc::bulk_g2s(sVB + r * KH * 1024, vb_bh + g, KH * 1024, bar_vb);
         }
       }
       for (int j = tid; j < kTile; j += 128) {
@@ -364,14 +417,18 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       wait_mma();
       uint32_t r[64];
       tmem_ld64(tS + lane_off, r);
-      // scaled logits and the row max over non-empty children
-      float cmax = NEG_INF;
+      const float4* nf4 = reinterpret_cast<const float4*>(sNF);
+      // row max of the raw logits over non-empty children (the scale is positive)
+      float cm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const float tv = __uint_as_float(r[e]) * sl2;
-        r[e] = __float_as_uint(tv);
-        if (sNF[e] > 0.f) cmax = fmaxf(cmax, tv);
+      for (int e = 0; e < 64; e += 4) {
+        const float4 nf = nf4[e >> 2];
+        cm[0] = fmaxf(cm[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
+        cm[1] = fmaxf(cm[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
+        cm[2] = fmaxf(cm[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
+        cm[3] = fmaxf(cm[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
       }
+      const float cmax = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) * sl2;
       // rare: a child logit far above the reference max -> rescale x and z
       const bool need = cmax > mref + kRescaleLog2;
       if (__any_sync(0xffffffffu, need)) {
@@ -388,24 +445,30 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
         z *= f;
         if (need) mref = cmax;
       }
-      // dA = 2^(t_c - m) - 2^(t_p - m), t_p = mean of the parent's child logits (Eq. 8)
+      // dA = 2^(t_c - m) - 2^(t_p - m) with t = scale*log2(e)*S and the parent
+      // logit t_p the mean of its children's logits (Eq. 8); zero for empty children
+      const float nm = -mref, sl8 = sl2 * 0.125f;
+      float zp[2] = {0.f, 0.f};
 #pragma unroll
       for (int sl = 0; sl < 8; ++sl) {
-        float tp = 0.f;
+        float ssum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) tp += __uint_as_float(r[sl * 8 + e]);
-        const float ap = tc::ex2(tp * 0.125f - mref);
+        for (int e = 0; e < 8; ++e) ssum += __uint_as_float(r[sl * 8 + e]);
+        const float ap = tc::ex2(fmaf(ssum, sl8, nm));
+        const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
+        const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
         float da[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float nf = sNF[sl * 8 + e];
-          da[e] = nf > 0.f ? tc::ex2(__uint_as_float(r[sl * 8 + e]) - mref) - ap : 0.f;
-          z = fmaf(da[e], nf, z);
+          da[e] = nfv[e] > 0.f ? tc::ex2(fmaf(__uint_as_float(r[sl * 8 + e]), sl2, nm)) - ap : 0.f;
+          zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
         }
         store_chunk8(sPR, tid, sl * 8, da);
       }
+      z += zp[0] + zp[1];
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
+      wait_vb();
       __syncthreads();
       if (tid == 0) {
         tc::tc_fence_after();
