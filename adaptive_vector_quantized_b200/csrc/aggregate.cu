@@ -1,5 +1,5 @@
 // Stage 1, aggregation ("AVQ-Attention: Adaptive Vector-Quantized Attention",
-// Sec. 4.2, Algorithm 1 steps 1, 8 and 16; Eq. 3).
+// Sec. 4.2, the aggregation of Algorithm 1; Eq. 3).
 //
 // Given every key's final code, each key adds its value to its parent, and to
 // its child when it moved to one.  Parents therefore hold their whole

@@ -1,5 +1,5 @@
 // Stage 1, assignment on CUDA cores ("AVQ-Attention: Adaptive
-// Vector-Quantized Attention", Sec. 4.2, Algorithm 1 steps 3-16).
+// Vector-Quantized Attention", Sec. 4.2, Algorithm 1: parent and child assignment).
 //
 // One thread per key.  The key is held in registers as fp32; the parent and
 // child codewords are read with warp-uniform addresses (broadcast loads).
@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(128) assign_simt_kernel(const T* __restrict__ 
 #pragma unroll
   for (int t = 0; t < D; t += 8) load8(kp + t, k + t);
 
-  // steps 5-7: nearest parent, first minimum
+  // nearest parent, first minimum
   const T* par = parents + (size_t)h * M0 * D;
   float best = __int_as_float(0x7f800000);
   int a = 0;
@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(128) assign_simt_kernel(const T* __restrict__ 
     }
   }
   int code = a;
-  // steps 9-16: nearest child of a, moved only when strictly closer than a
+  // nearest child of a, moved only when strictly closer than a
   if (C > 0) {
     const T* ch = children + ((size_t)h * M0 + a) * C * D;
     float dchild = __int_as_float(0x7f800000);

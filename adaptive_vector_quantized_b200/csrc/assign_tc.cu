@@ -1,5 +1,5 @@
 // Stage 1 assignment on the tcgen05 tensor cores ("AVQ-Attention: Adaptive
-// Vector-Quantized Attention", Sec. 4.2, Algorithm 1 steps 3-16).
+// Vector-Quantized Attention", Sec. 4.2, Algorithm 1: parent and child assignment).
 //
 // Persistent CTAs walk contiguous ranges of 128-key tiles.  Per tile:
 //   K tile      TMA (128B swizzle) into a two-slot ring, the next tile in

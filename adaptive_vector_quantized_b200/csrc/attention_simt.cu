@@ -9,7 +9,7 @@
 // denominator), which is the exact two-pass denominator and equals the
 // single-pass result.  Importance column sums use warp shuffles plus one
 // shared atomic per warp; top-P ranks every parent in one warp (descending,
-// ties to the lower index); the refinement follows Algorithm 2 steps 10-19
+// ties to the lower index); the refinement follows Algorithm 2
 // with the online max merge per selected parent.
 #include "common.cuh"
 #include "internal.h"
@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
   const T* par = parents + (size_t)h * M0 * D;
   const float* vs = vsum + (size_t)bh * Mt * D;
 
-  // Sweep 1 (Alg. 2 steps 4-7, denominator only): running max over non-empty
+  // Sweep 1 (denominator only): running max over non-empty
   // parents (Eq. 18) and z = sum_j exp(s_j - m) n_j.
   float m = __int_as_float(0xff800000), z = 0.f;
   for (int j = 0; j < M0; ++j) {
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
       }
     }
   }
-  // Sweep 2 (steps 6-8): A = exp(s - m) masked, x = A V-bar, importance (Eq. 7).
+  // Sweep 2: A = exp(s - m) masked, x = A V-bar, importance (Eq. 7).
   float x[D];
 #pragma unroll
   for (int t = 0; t < D; ++t) x[t] = 0.f;
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
   }
   __syncthreads();
 
-  // Step 9: top-P (descending, ties to the lower index) in one warp.
+  // Top-P (descending, ties to the lower index) in one warp.
   const int nsel = C > 0 ? P : 0;
   if (tid < 32) {
     for (int j = lane; j < M0; j += 32) {
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
   }
   __syncthreads();
 
-  // Steps 10-19: child refinement of the selected parents.
+  // Child refinement of the selected parents.
   for (int r = 0; r < nsel; ++r) {
     const int p = ssel[r];
     const T* cc = children + ((size_t)h * M0 + p) * C * D;
@@ -136,11 +136,11 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
       if (c < C) {
         sc[c] = scale * dot_row<T, D>(qr, cc + (size_t)c * D);
         sp += sc[c];
-        if (nf[M0 + p * C + c] > 0.f && sc[c] > mp) mp = sc[c];  // step 13
+        if (nf[M0 + p * C + c] > 0.f && sc[c] > mp) mp = sc[c];  // online max
       }
     }
-    sp = sp / (float)C;  // step 15, Eq. 8
-    const float f = expf(m - mp);  // step 14
+    sp = sp / (float)C;  // Eq. 8
+    const float f = expf(m - mp);  // rescale
     z *= f;
 #pragma unroll
     for (int t = 0; t < D; ++t) x[t] *= f;
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
     for (int c = 0; c < 8; ++c) {
       if (c < C) {
         const float nc = nf[M0 + p * C + c];
-        if (nc > 0.f) {  // steps 16-18, dA zeroed for empty children
+        if (nc > 0.f) {  // Eq. 9, dA zeroed for empty children
           const float da = expf(sc[c] - m) - ap;
           const float* vc = vs + (size_t)(M0 + p * C + c) * D;
 #pragma unroll
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
       }
     }
   }
-  // Step 20: Y = x / z.
+  // Y = x / z.
   if (valid) {
     const float iz = 1.f / z;
     T* o = O + ((size_t)bh * N + i) * D;

@@ -22,7 +22,7 @@
 //             The reference max stays the parents' max unless a child logit
 //             exceeds it by more than 2^24, in which case x (TMEM) and z are
 //             rescaled first; the result is the same as the online merge of
-//             Algorithm 2 steps 13-14 because the max cancels in x / z.
+//             Algorithm 2 because the max cancels in x / z.
 //   output    O = x / z, bf16, staged in shared memory and stored by TMA.
 // The codewords and the value sums are first converted by a small kernel
 // into bf16 images of 1024-byte swizzled atoms (8 codes x 64 dims), so that

@@ -26,12 +26,12 @@ struct LaunchLog {
 };
 
 // ---- stage 1 ------------------------------------------------------------
-// Algorithm 1 steps 3-16 (assignment): writes assign[BH][N] and adds the key
+// Algorithm 1, assignment: writes assign[BH][N] and adds the key
 // counts (Eq. 3) into counts[BH][Mt], which the caller zeroes first.
 cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
                                const void* children, int32_t* assign, int32_t* counts,
                                cudaStream_t st, LaunchLog& log);
-// Algorithm 1 steps 1, 8, 16 (value sums for given codes), streaming variant.
+// Algorithm 1, value sums for given codes, streaming variant.
 // vsum is zeroed inside; counts are left to the assignment kernels.
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,

@@ -26,8 +26,8 @@
  *     (b,h) at offset (b*H+h)*N*d.  Device pointers must be 16-byte aligned.
  *   - Codebook: one per head, shared by the batch (Algorithm 1 input
  *     C in R^{H x Mtotal x D}).  Mt = M0*(1+C).  Codeword a < M0 is parent a;
- *     codeword M0 + m*C + c is child c of parent m (Algorithm 1, comment on
- *     step 9).  Each parent must equal the mean of its children (Sec. 4.1,
+ *     codeword M0 + m*C + c is child c of parent m (Algorithm 1's first-child
+ *     index).  Each parent must equal the mean of its children (Sec. 4.1,
  *     Eq. 5); the attention recovers parent logits from that (Eq. 8).
  */
 #ifndef AVQ_H

@@ -97,7 +97,7 @@ class Oracle:
         return assign, vsum, counts, dec
 
     def aggregate(self, assign, V, M0: int, C: int):
-        """Statistics (Alg. 1 steps 1, 8, 16) for given final codes."""
+        """Statistics (the aggregation of Algorithm 1) for given final codes."""
         V = _f64(V)
         B, H, N, d = V.shape
         assign = np.ascontiguousarray(np.asarray(assign), dtype=np.int32)

@@ -14,13 +14,14 @@
  * Readings taken where the paper leaves a step open:
  *   - Logits are scaled by `scale` (1/sqrt(d) in every workload); the paper's
  *     Eq. 1 omits the factor "for clarity" (Sec. 3.1).  Distances use raw keys.
- *   - Parent ties go to the lowest index (argmin, Alg. 1 step 7).  A child is
- *     taken only if strictly closer than the running best child (Alg. 1
- *     step 14) and strictly closer than the parent (Alg. 1 step 16).
+ *   - Parent ties go to the lowest index (argmin in Algorithm 1).  A child is
+ *     taken only if strictly closer than the running best child and the key
+ *     moves only if that child is strictly closer than the parent (the two
+ *     strict comparisons of Algorithm 1).
  *   - Top-P ties go to the lower parent index; the selection is listed in
- *     descending importance (Alg. 2 step 9).
- *   - Importance uses the parents-only denominator (Alg. 2 step 8 precedes
- *     step 9; Eq. 7).
+ *     descending importance (the top-P of Algorithm 2).
+ *   - Importance uses the parents-only denominator (Algorithm 2 computes it
+ *     before the selection and the refinement; Eq. 7).
  *   - A partial last query block (N not a multiple of the block) is a block
  *     with fewer rows that selects independently.
  *
@@ -55,9 +56,9 @@ static double dot(const double* a, const double* b, int d) {
 }
 
 /*
- * Algorithm 1, steps 3-16, for one key: nearest parent (steps 5-7), then the
- * nearest of that parent's C children (steps 9-15), reassigned only if the
- * child is strictly closer than the cached parent distance (step 16).
+ * Algorithm 1 for one key: nearest parent, then the nearest of that parent's
+ * C children, reassigned only if the child is strictly closer than the cached
+ * parent distance.
  * Returns the final code.  The decision distances are written for the
  * near-tie rule used by the tests:
  *   dec[0] = best parent distance, dec[1] = second-best parent distance,
@@ -66,7 +67,7 @@ static double dot(const double* a, const double* b, int d) {
  */
 static int32_t assign_one(const double* k, const double* par_h, const double* ch_h,
                           int d, int M0, int C, double* dec) {
-  /* steps 5-7: d = ||k - c_p||^2 over the M0 parents, a = argmin, d_best = min */
+  /* d = ||k - c_p||^2 over the M0 parents, a = argmin, d_best = min */
   int a = 0;
   double d_best = INFINITY, d_second = INFINITY;
   for (int m = 0; m < M0; ++m) {
@@ -79,14 +80,14 @@ static int32_t assign_one(const double* k, const double* par_h, const double* ch
       d_second = dm;
     }
   }
-  /* steps 9-15: c0 = M0 + a*C, d_child = inf, c* = c0, scan the C children */
+  /* c0 = M0 + a*C, d_child = inf, c* = c0, scan the C children of a */
   int32_t c0 = M0 + a * C;
   double d_child = INFINITY, d_child2 = INFINITY;
   int32_t c_star = c0;
   for (int c = 0; c < C; ++c) {
     const double* cc = ch_h + ((size_t)a * C + c) * d;
     double dc = sqdist(k, cc, d);
-    if (dc < d_child) { /* step 14: where d_c < d_child */
+    if (dc < d_child) { /* where d_c < d_child: strict */
       d_child2 = d_child;
       d_child = dc;
       c_star = c0 + c;
@@ -100,15 +101,15 @@ static int32_t assign_one(const double* k, const double* par_h, const double* ch
     dec[2] = d_child;
     dec[3] = d_child2;
   }
-  /* step 16: where d_child < d_best the key moves to child c* */
+  /* where d_child < d_best (strict) the key moves to child c* */
   if (C > 0 && d_child < d_best) return c_star;
   return a;
 }
 
 /*
- * Algorithm 1 (VQ Precompute).  Step 1 zeroes the statistics; every key then
- * adds its value and a count of one to its parent (step 8) and, if it moved,
- * also to its child (step 16).  Parents thus hold their whole cluster and
+ * Algorithm 1 (VQ Precompute).  The statistics start at zero; every key then
+ * adds its value and a count of one to its parent and, if it moved, also to
+ * its child (the masked add).  Parents thus hold their whole cluster and
  * children only the keys that are closer to them than to the parent.
  * `dec` (nullable) receives 4 decision distances per key, see assign_one.
  */
@@ -125,7 +126,7 @@ void avq_oracle_quantize(int BH, int H, int N, int d, int M0, int C,
     const double* ch_h = children + (size_t)h * M0 * C * d;
     double* vs = vsum + (size_t)bh * Mt * d;
     int64_t* ns = counts + (size_t)bh * Mt;
-    /* step 1: initialise V-bar = 0, n = 0 */
+    /* initialise V-bar = 0, n = 0 */
     memset(vs, 0, sizeof(double) * (size_t)Mt * d);
     memset(ns, 0, sizeof(int64_t) * (size_t)Mt);
     for (int j = 0; j < N; ++j) {
@@ -134,10 +135,10 @@ void avq_oracle_quantize(int BH, int H, int N, int d, int M0, int C,
       double* dj = dec ? dec + ((size_t)bh * N + j) * 4 : NULL;
       int32_t code = assign_one(k, par_h, ch_h, d, M0, C, dj);
       int32_t a = code < M0 ? code : (code - M0) / C;
-      /* step 8: V-bar[a] += v; n[a] += 1 */
+      /* V-bar[a] += v; n[a] += 1 */
       for (int t = 0; t < d; ++t) vs[(size_t)a * d + t] += v[t];
       ns[a] += 1;
-      /* step 16: masked add to the child */
+      /* masked add to the child */
       if (code >= M0) {
         for (int t = 0; t < d; ++t) vs[(size_t)code * d + t] += v[t];
         ns[code] += 1;
@@ -148,7 +149,7 @@ void avq_oracle_quantize(int BH, int H, int N, int d, int M0, int C,
 }
 
 /*
- * The aggregation of Algorithm 1 (steps 1, 8 and 16) for given final codes:
+ * The aggregation of Algorithm 1 for given final codes:
  * used to check statistics against assignments made elsewhere.
  */
 void avq_oracle_aggregate(int BH, int N, int d, int M0, int C,
@@ -176,7 +177,7 @@ void avq_oracle_aggregate(int BH, int N, int d, int M0, int C,
 
 /*
  * Top-P of the importance vector w[0..M0): the P largest entries in
- * descending order, ties to the lower index (Alg. 2 step 9).
+ * descending order, ties to the lower index (the top-P of Algorithm 2).
  */
 static void top_p(const double* w, int M0, int P, int32_t* out) {
   char* taken = (char*)calloc((size_t)M0, 1);
@@ -194,12 +195,12 @@ static void top_p(const double* w, int M0, int P, int32_t* out) {
 
 /*
  * Algorithm 2 (Flash AVQ-Attention) for one query block I = [i0, i1) of one
- * head.  Steps 2-8: coarse pass over the M0 parents with the masked running
+ * head.  Coarse pass over the M0 parents with the masked running
  * max (Eq. 18), count-weighted denominator (Eq. 6) and importance (Eq. 7).
- * Step 9: top-P.  Steps 10-19: for each selected parent, child logits, online
+ * Top-P.  Then, for each selected parent: child logits, online
  * max merge, parent logit recovered as the mean of the child logits (Eq. 8),
  * correcting attention dA = exp(S_ic) - exp(S_ip) (Eq. 9) masked for empty
- * children, and the accumulator update.  Step 20: Y = x / z.
+ * children, and the accumulator update.  Finally Y = x / z.
  */
 static void attend_block(int d, int M0, int C, int P, double scale,
                          const double* Q, int i0, int i1,
@@ -219,16 +220,16 @@ static void attend_block(int d, int M0, int C, int P, double scale,
 
   for (int r = 0; r < nI; ++r) {
     const double* q = Q + (size_t)(i0 + r) * d;
-    /* step 4: s = q c^T over the parents */
+    /* s = q c^T over the parents */
     for (int j = 0; j < M0; ++j) s[(size_t)r * M0 + j] = scale * dot(q, par_h + (size_t)j * d, d);
-    /* step 5: m = max over j with n_j > 0 */
+    /* m = max over j with n_j > 0 (Eq. 18) */
     m[r] = -INFINITY;
     for (int j = 0; j < M0; ++j)
       if (ns[j] > 0 && s[(size_t)r * M0 + j] > m[r]) m[r] = s[(size_t)r * M0 + j];
-    /* step 6: A = exp(s - m), A_j = 0 where n_j = 0 */
+    /* A = exp(s - m), A_j = 0 where n_j = 0 */
     for (int j = 0; j < M0; ++j)
       A[(size_t)r * M0 + j] = ns[j] > 0 ? exp(s[(size_t)r * M0 + j] - m[r]) : 0.0;
-    /* step 7: x = A v-bar, z = sum_j A_j n_j */
+    /* x = A v-bar, z = sum_j A_j n_j  (Eq. 6) */
     for (int t = 0; t < d; ++t) x[(size_t)r * d + t] = 0.0;
     z[r] = 0.0;
     for (int j = 0; j < M0; ++j) {
@@ -237,19 +238,19 @@ static void attend_block(int d, int M0, int C, int P, double scale,
       z[r] += a * ns[j];
     }
   }
-  /* step 8: w_j = sum_i A_ij n_j / z_i  (Eq. 7) */
+  /* w_j = sum_i A_ij n_j / z_i  (Eq. 7) */
   for (int j = 0; j < M0; ++j) {
     w[j] = 0.0;
     for (int r = 0; r < nI; ++r) w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];
   }
   if (imp_out) memcpy(imp_out, w, sizeof(double) * (size_t)M0);
-  /* step 9: S = top-P(w), or the caller's selection */
+  /* S = top-P(w), or the caller's selection */
   if (P > 0) {
     if (sel_in) memcpy(S, sel_in, sizeof(int32_t) * (size_t)P);
     else top_p(w, M0, P, S);
     if (sel_out) memcpy(sel_out, S, sizeof(int32_t) * (size_t)P);
   }
-  /* steps 10-19: child refinement (no-op when C == 0) */
+  /* child refinement (no-op when C == 0) */
   if (C > 0) {
     for (int r = 0; r < nI; ++r) {
       const double* q = Q + (size_t)(i0 + r) * d;
@@ -258,22 +259,22 @@ static void attend_block(int d, int M0, int C, int P, double scale,
         const double* ch_p = ch_h + (size_t)p * C * d;
         const double* vc = vs + (size_t)(M0 + p * C) * d;
         const double* nc = ns + (M0 + p * C);
-        /* step 12: s_c = q c_c^T */
+        /* s_c = q c_c^T */
         for (int c = 0; c < C; ++c) sc[c] = scale * dot(q, ch_p + (size_t)c * d, d);
-        /* step 13: m' = max(m, max over c with n_c > 0 of s_c) */
+        /* m' = max(m, max over c with n_c > 0 of s_c) */
         double mp = m[r];
         for (int c = 0; c < C; ++c)
           if (nc[c] > 0 && sc[c] > mp) mp = sc[c];
-        /* step 14: rescale the accumulators to m' */
+        /* rescale the accumulators to m' */
         double f = exp(m[r] - mp);
         for (int t = 0; t < d; ++t) x[(size_t)r * d + t] *= f;
         z[r] *= f;
         m[r] = mp;
-        /* step 15: s_p = (1/C) sum_c s_c   (Eq. 8) */
+        /* s_p = (1/C) sum_c s_c   (Eq. 8) */
         double sp = 0.0;
         for (int c = 0; c < C; ++c) sp += sc[c];
         sp /= C;
-        /* steps 16-18: dA = exp(s_c - m) - exp(s_p - m), zero where n_c = 0 */
+        /* dA = exp(s_c - m) - exp(s_p - m), zero where n_c = 0  (Eq. 9) */
         double Ap = exp(sp - m[r]);
         for (int c = 0; c < C; ++c) {
           double dA = nc[c] > 0 ? exp(sc[c] - m[r]) - Ap : 0.0;
@@ -283,7 +284,7 @@ static void attend_block(int d, int M0, int C, int P, double scale,
       }
     }
   }
-  /* step 20: Y = x / z */
+  /* Y = x / z */
   for (int r = 0; r < nI; ++r)
     for (int t = 0; t < d; ++t) O[(size_t)(i0 + r) * d + t] = x[(size_t)r * d + t] / z[r];
 

@@ -129,8 +129,8 @@ def pin_representative(orc):
 
 
 def pin_rescale_exercised(orc):
-    """The representative check above covers the online-max merge (Alg. 2
-    steps 13-14) only if some selected non-empty child logit exceeds the
+    """The representative check above covers the online-max merge of
+    Algorithm 2 only if some selected non-empty child logit exceeds the
     parent max; make sure the regions case has such rows."""
     inp = case_regions()
     assign, vsum, counts, O, sel, _ = _run(orc, inp)
@@ -297,8 +297,8 @@ def pin_keys_on_codewords(orc):
 
 def pin_strict_ties(orc):
     """Ties: equal parents -> lower index (argmin); a child must be strictly
-    closer than the best child so far (first child wins, Alg. 1 step 14) and
-    strictly closer than the parent (step 16)."""
+    closer than the best child so far (first child wins) and strictly closer
+    than the parent (the two strict comparisons of Algorithm 1)."""
     par = np.array([[[0.0, 0.0], [10.0, 10.0]]])
     ch = np.array([[[[1, 1], [1, -1], [-1, 1], [-1, -1]],
                     [[11, 11], [11, 9], [9, 11], [9, 9]]]], dtype=np.float64)

@@ -13,7 +13,7 @@ from tests import pins
 MUTANTS = [
     ("child-not-strict-vs-parent", "if (C > 0 && d_child < d_best) return c_star;",
      "if (C > 0 && d_child <= d_best) return c_star;"),
-    ("child-tie-to-last", "if (dc < d_child) { /* step 14", "if (dc <= d_child) { /* step 14"),
+    ("child-tie-to-last", "if (dc < d_child) { /* where", "if (dc <= d_child) { /* where"),
     ("parent-tie-to-last", "if (dm < d_best) {", "if (dm <= d_best) {"),
     ("child-count-dropped", "ns[code] += 1;\n      }\n      assign", "\n      }\n      assign"),
     ("child-index-transposed", "ch_h + ((size_t)a * C + c) * d", "ch_h + ((size_t)c * M0 + a) * d"),
