@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
                 P = ctypes.POINTER
                 L.avq_quantize.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _vp, ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+                L.avq_quantize_noalloc.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp,
+                                                   _vp, _vp, _vp, _vp]
                 L.avq_attention.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                             _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -76,8 +78,8 @@ def lib() -> ctypes.CDLL:
                     getattr(L, name).restype = ctypes.c_char_p
                 L.avq_status_string.argtypes = [ctypes.c_int]
                 L.avq_version.restype = ctypes.c_int
-                for name in ("avq_quantize", "avq_attention", "avq_permute", "avq_hilbert_order",
-                             "avq_check_device"):
+                for name in ("avq_quantize", "avq_quantize_noalloc", "avq_attention", "avq_permute",
+                             "avq_hilbert_order", "avq_check_device"):
                     getattr(L, name).restype = ctypes.c_int
                 _lib = L
     return _lib
@@ -187,6 +189,28 @@ def avq_quantize(K, V, parents, children, assign=None, vsum=None, counts=None,
     _check(lib().avq_quantize(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
                               _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
                               int(bool(deterministic)), wp, wn, _stream(stream)))
+    return assign, vsum, counts
+
+
+def avq_quantize_noalloc(K, V, parents, children, assign=None, vsum=None, counts=None, stream=None):
+    """Stage 1 through the library's static scratch instead of a workspace
+    (no device memory is allocated by the call; pass `assign`, `vsum` and
+    `counts` to keep this wrapper from allocating the outputs).  Calls whose
+    executions may overlap on one device race on that scratch."""
+    dims = _dims(K, parents, children)
+    dt = _dtype_code(K)
+    B, H, N, d = K.shape
+    Mt = dims.M0 * (1 + dims.C)
+    dev = K.device
+    if assign is None:
+        assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    if vsum is None:
+        vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
+    if counts is None:
+        counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
+    _check(lib().avq_quantize_noalloc(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
+                                      _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
+                                      _stream(stream)))
     return assign, vsum, counts
 
 

@@ -321,3 +321,84 @@ avq_status avq_check_device(avq_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// avq_quantize_noalloc: stage 1 for callers that cannot hand the library a
+// workspace.  The tensor-core assignment needs a bf16 image of the codebook
+// and its squared norms; here they live in a fixed module-scope device array
+// instead of caller memory, so the call allocates nothing.
+namespace avq {
+
+__device__ __align__(256) unsigned char g_avq_noalloc_scratch[AVQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+
+// Resolves the scratch array's address on the current device, once per
+// device (the first call on a device does this set-up).
+avq_status noalloc_scratch(void** out) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_avq_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(AVQ_ERR_CUDA, "cannot resolve the static scratch on device %d: %s", dev,
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return AVQ_OK;
+}
+}  // namespace
+}  // namespace avq
+
+extern "C" avq_status avq_quantize_noalloc(const avq_dims* dims, avq_dtype dtype, const void* K,
+                                           const void* V, const void* parents, const void* children,
+                                           int32_t* assign, float* vsum, int32_t* counts,
+                                           avq_stream_t stream) {
+  t_error[0] = 0;
+  avq_status st = check_dims(dims, dtype);
+  if (st != AVQ_OK) return st;
+  const Shape s = to_shape(dims);
+  AVQ_REQUIRE_PTR(K, "K");
+  AVQ_REQUIRE_PTR(V, "V");
+  AVQ_REQUIRE_PTR(parents, "parents");
+  if (s.C > 0) AVQ_REQUIRE_PTR(children, "children");
+  AVQ_REQUIRE_PTR(assign, "assign");
+  AVQ_REQUIRE_PTR(vsum, "vsum");
+  AVQ_REQUIRE_PTR(counts, "counts");
+  const bool tc_ok = assign_tc_supported(s, dtype);
+  if (t_path == AVQ_PATH_TC && !tc_ok)
+    return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core assignment kernel for this shape/dtype");
+  const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
+  void* scratch = nullptr;
+  if (use_tc) {
+    const size_t need = assign_tc_workspace(s);
+    if (need > AVQ_NOALLOC_SCRATCH_BYTES)
+      return fail(AVQ_ERR_WORKSPACE,
+                  "the codebook image needs %zu bytes but the static scratch holds %zu; "
+                  "call avq_quantize with a workspace instead",
+                  need, (size_t)AVQ_NOALLOC_SCRATCH_BYTES);
+    st = noalloc_scratch(&scratch);
+    if (st != AVQ_OK) return st;
+  }
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  LaunchLog log{};
+  unsigned int* err = error_word();
+  if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+  // The assignment kernels add into counts, so counts must start at zero.
+  // The scratch needs no clearing: the codebook image is rewritten in full
+  // by every call before the assignment reads it.
+  cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "zero counts");
+  if (use_tc)
+    e = launch_assign_tc(s, K, parents, children, assign, counts, scratch, err, cs, log);
+  else
+    e = launch_assign_simt(s, dtype, K, parents, children, assign, counts, cs, log);
+  if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
+  e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log);
+  if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}

@@ -12,7 +12,8 @@
  *   - Ownership: the caller allocates and owns every buffer, host or device.
  *     The library allocates no memory and keeps no state across calls except
  *     thread-local settings (avq_set_path) and diagnostics (avq_last_error,
- *     avq_last_kernels) and one device-side error word per GPU.
+ *     avq_last_kernels), one device-side error word per GPU and the static
+ *     scratch array of avq_quantize_noalloc.
  *   - Execution: device calls are enqueued on `stream` (NULL = legacy default
  *     stream) and return without synchronising.  Results are valid once the
  *     stream has completed the call.
@@ -95,6 +96,44 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype,
                         int32_t* assign, float* vsum, int32_t* counts,
                         int deterministic, void* ws, size_t ws_bytes,
                         avq_stream_t stream);
+
+/*
+ * avq_quantize_noalloc -- avq_quantize without a caller workspace.  This call
+ * is an engineering addition of this library; the paper has no counterpart.
+ *
+ * For callers that cannot hand over device memory for a workspace: a runtime
+ * whose device memory is reserved up front by its own pool and that must not
+ * allocate while it serves requests, or a plain C caller that wants a single
+ * call with no buffer to size, allocate and keep alive.  Nothing is
+ * allocated: the tensor-core codebook image lives in a fixed device array of
+ * AVQ_NOALLOC_SCRATCH_BYTES inside the library, one per GPU.
+ *
+ * Arguments, outputs and results are those of avq_quantize with
+ * deterministic = 0 (the fixed-order reduction needs scratch that grows with
+ * N, so it is not offered here).  counts is zeroed by the call, as in
+ * avq_quantize; the static scratch needs no clearing.
+ *
+ * Limit: the tensor-core path needs H*Mt*d*2 bytes (rounded up to 256) plus
+ * H*Mt*4 bytes (rounded up to 256) of scratch; above AVQ_NOALLOC_SCRATCH_BYTES
+ * the call returns AVQ_ERR_WORKSPACE and launches nothing.  Shapes or dtypes
+ * without a tensor-core kernel (and AVQ_PATH_SIMT) use the CUDA-core
+ * assignment, which needs no scratch.
+ *
+ * Set-up: the first call on each device, with that device current, resolves
+ * the scratch array's device address; make that first call before any stream
+ * capture.
+ *
+ * Races: every call on one device shares the one scratch array.  Calls
+ * ordered on one stream are safe; two calls whose executions may overlap
+ * (different streams without ordering between them, or different host threads
+ * on one device) overwrite each other's codebook image and give wrong results.
+ */
+#define AVQ_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+avq_status avq_quantize_noalloc(const avq_dims* dims, avq_dtype dtype,
+                                const void* K, const void* V,
+                                const void* parents, const void* children,
+                                int32_t* assign, float* vsum, int32_t* counts,
+                                avq_stream_t stream);
 
 /*
  * avq_attention -- adaptive attention with per-query-block refinement

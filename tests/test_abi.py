@@ -104,3 +104,24 @@ def test_hilbert_order_matches_textbook_curve():
         assert np.array_equal(got, synth.hilbert_cells(side))
     with pytest.raises(avq.AVQError):
         avq.avq_hilbert_order(12)
+
+
+def test_noalloc_quantize_host_checks():
+    """The no-alloc stage-1 entry rejects, before any launch, a codebook whose
+    tensor-core image exceeds its static scratch, and bad pointers."""
+    L = avq.lib()
+    big = avq.avq_dims(1, 64, 1024, 128, 256, 8)  # 64 * 2304 * 128 * 2 bytes > 8 MiB
+    st = L.avq_quantize_noalloc(ctypes.byref(big), avq.AVQ_BF16, 0x1000, 0x2000, 0x3000, 0x4000,
+                                0x5000, 0x6000, 0x7000, None)
+    assert st == 6, avq.last_error()
+    assert "static scratch" in avq.last_error()
+    ok = avq.avq_dims(1, 16, 1024, 64, 64, 8)
+    st = L.avq_quantize_noalloc(ctypes.byref(ok), avq.AVQ_BF16, None, 0x2000, 0x3000, 0x4000,
+                                0x5000, 0x6000, 0x7000, None)
+    assert st == 1 and "K is NULL" in avq.last_error()
+    st = L.avq_quantize_noalloc(ctypes.byref(ok), avq.AVQ_BF16, 0x1008, 0x2000, 0x3000, 0x4000,
+                                0x5000, 0x6000, 0x7000, None)
+    assert st == 1 and "aligned" in avq.last_error()
+    st = L.avq_quantize_noalloc(None, avq.AVQ_BF16, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000,
+                                0x6000, 0x7000, None)
+    assert st == 1
