@@ -355,6 +355,406 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Warpgroup-pipelined variant for M0 <= 64 with the children in shared memory.
+// One CTA per SM holds the head's codebook image once; each of its NWG
+// warpgroups walks its own interleaved sequence of 128-key tiles with its own
+// two-slot K ring, barriers and 128 TMEM columns, so that the tensor-core
+// latency of one warpgroup's tile hides behind the other warpgroups' work.
+// Children of a tile: the child atoms of the parents that some key chose are
+// gathered (in index order, up to 8 per round) into a contiguous staging
+// operand, so one MMA chain of N = 8 x (atoms, rounded up to even) gives every
+// key its dot products with all those children.
+// Scores: T = k.c - |c|^2 / 2 orders the codewords of a key like the squared
+// distance |k|^2 - 2 T, reversed.  For the parents the -|p|^2 / 2 term is
+// folded into the MMA as one more K step: A holds 1, 1, 1 in its first three
+// columns, B the bf16 triple (hi, mid, lo) whose sum is -|p|^2 / 2 to within
+// 2^-24 of it, so TMEM receives T directly.
+constexpr int kStageAtoms = 8;
+
+template <int D>
+struct WgSmem {
+  static constexpr int KH = D / 64;
+  static constexpr size_t kTile = (size_t)kKeys * D * 2;
+  static constexpr size_t kStage = (size_t)kStageAtoms * KH * 1024;
+  static constexpr size_t kWg = 2 * kTile + kStage;
+  static constexpr size_t kOnes = (size_t)kKeys * 128;  // A operand of the norm step
+  static constexpr size_t kBnorm = 64 * 128;            // B operand of the norm step
+  __host__ __device__ static size_t cb_bytes(int M0, int C) { return (size_t)M0 * (1 + C) * D * 2; }
+  __host__ __device__ static size_t ones_off(int M0, int C) { return (cb_bytes(M0, C) + 1023) & ~(size_t)1023; }
+  __host__ __device__ static size_t bnorm_off(int M0, int C) { return ones_off(M0, C) + kOnes; }
+  __host__ __device__ static size_t wg_off(int M0, int C) { return bnorm_off(M0, C) + kBnorm; }
+  __host__ __device__ static size_t norms_off(int M0, int C, int nwg) { return wg_off(M0, C) + nwg * kWg; }
+  __host__ __device__ static size_t misc_off(int M0, int C, int nwg) {
+    return (norms_off(M0, C, nwg) + (size_t)M0 * (1 + C) * 4 + 15) & ~(size_t)15;
+  }
+  // barriers: cb + 4 per warpgroup; masks: 4 words per warpgroup; tmem base, abort
+  __host__ __device__ static size_t total(int M0, int C, int nwg) {
+    return misc_off(M0, C, nwg) + 8 * (1 + 4 * nwg) + 16 * nwg + 16;
+  }
+};
+
+__device__ __forceinline__ void wg_bar(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+// Named-barrier sync of one warpgroup that also ORs a flag over its threads.
+__device__ __forceinline__ bool wg_bar_or(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
+}
+// Position of the n-th (0-based) set bit of a 32-bit word (binary search
+// with population counts; the word has more than n set bits).
+__device__ __forceinline__ int nth_set(uint32_t m, int n) {
+  int pos = 0;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const int c = __popc(m & ((1u << w) - 1u));
+    if (n >= c) {
+      n -= c;
+      m >>= w;
+      pos += w;
+    }
+  }
+  return pos;
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
+}
+
+// bf16 bits of x, round to nearest even.
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+template <int D, int M0>
+__global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                           const AssignArgs a) {
+  using S = WgSmem<D>;
+  constexpr int KH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nwg = blockDim.x >> 7;
+  const int C = a.C, Mt = M0 * (1 + C);
+  const int tid = threadIdx.x, g = tid >> 7, wt = tid & 127, wwarp = wt >> 5;
+  uint8_t* sPar = sm;
+  const uint8_t* sCh = sm + (size_t)M0 * D * 2;
+  uint8_t* sRing = sm + S::wg_off(M0, C) + (size_t)g * S::kWg;
+  uint8_t* sStage = sRing + 2 * S::kTile;
+  uint8_t* sOnes = sm + S::ones_off(M0, C);
+  uint8_t* sBn = sm + S::bnorm_off(M0, C);
+  float* sNorm = reinterpret_cast<float*>(sm + S::norms_off(M0, C, nwg));  // -|c|^2 / 2
+  uint64_t* bar_cb = reinterpret_cast<uint64_t*>(sm + S::misc_off(M0, C, nwg));
+  uint64_t* bar_k = bar_cb + 1 + 4 * g;  // [2]
+  uint64_t* bar_p = bar_k + 2;           // parent MMA done
+  uint64_t* bar_c = bar_k + 3;           // child MMA done
+  uint32_t* sMaskAll = reinterpret_cast<uint32_t*>(bar_cb + 1 + 4 * nwg);
+  uint32_t* sMask = sMaskAll + 4 * g;  // [tile parity][2 words]
+  uint32_t* sTmem = sMaskAll + 4 * nwg;
+  int* sAbort = reinterpret_cast<int*>(sTmem + 1);
+
+  const int t0 = blockIdx.x * a.tiles_per_cta;
+  const int t1 = min(a.ntiles, t0 + a.tiles_per_cta);
+  if (t0 >= t1) return;
+  const uint32_t ncols = nwg == 1 ? 128u : nwg == 2 ? 256u : 512u;
+
+  if (tid == 0) {
+    tc::mbar_init(bar_cb, 1);
+    for (int w = 0; w < 4 * nwg; ++w) tc::mbar_init(bar_cb + 1 + w, 1);
+    tc::fence_mbar_init();
+    for (int w = 0; w < 4 * nwg; ++w) sMaskAll[w] = 0;
+    *sAbort = 0;
+    tc::prefetch_tensormap(&kmap);
+  }
+  // staging starts zeroed: padding atoms feed columns nobody reads, but stay finite
+  for (int i = wt; i < (int)(S::kStage / 16); i += 128)
+    reinterpret_cast<uint4*>(sStage)[i] = make_uint4(0, 0, 0, 0);
+  // A of the norm step: row r = (1, 1, 1, 0, ...) in logical 16-byte chunk 0
+  for (int i = tid; i < (int)(S::kOnes / 16); i += blockDim.x) {
+    const int r = i >> 3, pos = i & 7;
+    reinterpret_cast<uint4*>(sOnes)[i] =
+        pos == (r & 7) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0, 0, 0, 0);
+  }
+  tc::fence_proxy_async_smem();
+  if (tid < 32) {
+    tc::tmem_alloc(sTmem, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_g = *sTmem + (uint32_t)g * 128u;
+  const uint32_t lane_off = (uint32_t)(wwarp * 32) << 16;
+  const int barid = 1 + g;
+
+  auto issue_k = [&](int t, int slot) {
+    const int bh = t / a.nblk, blk = t % a.nblk;
+    tc::mbar_arrive_expect_tx(&bar_k[slot], (uint32_t)S::kTile);
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh)
+      tc::tma_load_3d(sRing + slot * S::kTile + kh * (kKeys * 128), &kmap, kh * 64, blk * kKeys, bh,
+                      &bar_k[slot]);
+  };
+
+  const uint32_t idescP = tc::idesc_bf16(kKeys, M0, 0, 0);
+  const uint32_t sParA = tc::smem_u32(sPar), sStA = tc::smem_u32(sStage);
+  const uint32_t sOnesA = tc::smem_u32(sOnes), sBnA = tc::smem_u32(sBn);
+  uint32_t ph_cb = 0, ph_p = 0, ph_c = 0;
+  int cur_h = -1, it = 0;
+  bool aborted = false, kerr = false;
+  // parent scores of the K tile in `kslot` into TMEM half `kslot` (norm step last)
+  auto issue_parents = [&](int kslot) {
+    const uint32_t sKa = tc::smem_u32(sRing + kslot * S::kTile);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+      const uint64_t ad = tc::sdesc_sw128(sKa + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024);
+      const uint64_t bd = tc::sdesc_sw128(sParA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+      tc::mma_bf16(tmem_g + (uint32_t)kslot * 64u, ad, bd, idescP, k > 0);
+    }
+    tc::mma_bf16(tmem_g + (uint32_t)kslot * 64u, tc::sdesc_sw128(sOnesA, 16, 1024),
+                 tc::sdesc_sw128(sBnA, 16, 1024), idescP, 1);
+    tc::mma_commit(bar_p);
+  };
+
+  for (int s0 = t0; s0 < t1;) {
+    const int bh = s0 / a.nblk;
+    const int s1 = min(t1, (bh + 1) * a.nblk);
+    const int h = bh % a.H;
+    if (h != cur_h) {  // (re)load the head's codebook image and norms, CTA-wide
+      if (tid == 0) {
+        const size_t bytes = S::cb_bytes(M0, C);
+        tc::mbar_arrive_expect_tx(bar_cb, (uint32_t)bytes);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cw + (size_t)h * Mt * D);
+        for (size_t off = 0; off < bytes;) {
+          const uint32_t part = (uint32_t)std::min<size_t>(bytes - off, 65536);
+          tc::bulk_g2s(sPar + off, src + off, part, bar_cb);
+          off += part;
+        }
+      }
+      for (int j = tid; j < Mt; j += blockDim.x) sNorm[j] = -0.5f * __ldg(a.norms + (size_t)h * Mt + j);
+      for (int i = tid; i < 64 * 8; i += blockDim.x) {  // B of the norm step
+        const int m = i >> 3, pos = i & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (m < M0 && pos == (m & 7)) {
+          const float n = -0.5f * __ldg(a.norms + (size_t)h * Mt + m);
+          const uint32_t hi = bf16_bits(n);
+          const float r1 = n - __uint_as_float(hi << 16);
+          const uint32_t mid = bf16_bits(r1);
+          const uint32_t lo = bf16_bits(r1 - __uint_as_float(mid << 16));
+          v = make_uint4(hi | (mid << 16), lo, 0u, 0u);
+        }
+        reinterpret_cast<uint4*>(sBn)[i] = v;
+      }
+      tc::fence_proxy_async_smem();
+      if (!tc::mbar_wait(bar_cb, ph_cb)) {
+        atomicOr(a.err, kErrTimeout);
+        *sAbort = 1;
+      }
+      ph_cb ^= 1;
+      cur_h = h;
+      __syncthreads();
+      if (*sAbort) break;
+    }
+    const int first = s0 + g;
+    // prologue: K of the first two tiles, parent MMA of the first
+    if (wt == 0 && first < s1) {
+      issue_k(first, it & 1);
+      if (first + nwg < s1) issue_k(first + nwg, (it + 1) & 1);
+      if (tc::mbar_wait(&bar_k[it & 1], (it >> 1) & 1)) {
+        tc::tc_fence_after();
+        issue_parents(it & 1);
+      } else {
+        kerr = true;
+      }
+    }
+    for (int t = first; t < s1; t += nwg, ++it) {
+      const int slot = it & 1;
+      const uint32_t tP = tmem_g + (uint32_t)slot * 64u;  // parent, then child scores of this tile
+      bool bad = false;
+      if (wt == 0) bad = kerr || !tc::mbar_wait(bar_p, ph_p);
+      ph_p ^= 1;
+      tc::tc_fence_before();
+      if (wg_bar_or(barid, bad)) {  // parent scores of tile t in TMEM
+        if (wt == 0) atomicOr(a.err, kErrTimeout);
+        aborted = true;
+        break;
+      }
+      tc::tc_fence_after();
+      // next tile's parent MMA into the other half (its scores there were read
+      // before the barrier above), so that it overlaps this tile's epilogue
+      auto next_parents = [&]() {
+        if (wt == 0 && t + nwg < s1) {
+          if (tc::mbar_wait(&bar_k[slot ^ 1], ((it + 1) >> 1) & 1)) {
+            tc::tc_fence_after();
+            issue_parents(slot ^ 1);
+          } else {
+            kerr = true;
+          }
+        }
+      };
+      if (C == 0) {
+        next_parents();
+        if (wt == 0 && t + 2 * nwg < s1) issue_k(t + 2 * nwg, slot);  // K slot read by nothing else
+      }
+
+      // nearest parent = first maximum of T over the M0 parents: eight running
+      // maxima over contiguous groups of M0/8 columns, merged in index order
+      float best;
+      int par;
+      {
+        constexpr int G = M0 / 8;
+        uint32_t r[M0];
+#pragma unroll
+        for (int q = 0; q < M0 / 16; ++q) tc::tmem_ld16(tP + lane_off + q * 16, r + q * 16);
+        tc::tmem_wait_ld();
+        float bv[8];
+        int bi[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          bv[q] = __uint_as_float(r[q * G]);
+          bi[q] = q * G;
+        }
+#pragma unroll
+        for (int e = 1; e < G; ++e)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float v = __uint_as_float(r[q * G + e]);
+            if (v > bv[q]) {
+              bv[q] = v;
+              bi[q] = q * G + e;
+            }
+          }
+#pragma unroll
+        for (int w = 1; w < 8; w *= 2)
+#pragma unroll
+          for (int q = 0; q < 8; q += 2 * w)
+            if (bv[q + w] > bv[q]) {
+              bv[q] = bv[q + w];
+              bi[q] = bi[q + w];
+            }
+        best = bv[0];
+        par = bi[0];
+      }
+      int code = par;
+      if (C > 0) {  // C == 8 on this path
+        uint32_t* mk = sMask + slot * 2;
+        const uint32_t lo = __reduce_or_sync(0xffffffffu, par < 32 ? 1u << par : 0u);
+        const uint32_t hi = __reduce_or_sync(0xffffffffu, par >= 32 ? 1u << (par - 32) : 0u);
+        if ((wt & 31) == 0) {
+          if (lo) atomicOr(mk, lo);
+          if (hi) atomicOr(mk + 1, hi);
+        }
+        tc::tc_fence_before();
+        wg_bar(barid);  // parent set complete, parent scores read
+        if (wt == 0) {  // the other parity's set, for the next tile
+          sMask[(slot ^ 1) * 2] = 0;
+          sMask[(slot ^ 1) * 2 + 1] = 0;
+        }
+        next_parents();
+        const uint32_t m_lo = mk[0], m_hi = mk[1];
+        const int n_lo = __popc(m_lo), np = n_lo + __popc(m_hi);
+        const int myslot = par < 32 ? __popc(m_lo & ((1u << par) - 1u))
+                                    : n_lo + __popc(m_hi & ((1u << (par - 32)) - 1u));
+        float vals[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) vals[c] = 0.f;
+        for (int r0 = 0; r0 < np; r0 += kStageAtoms) {
+          const int nr = min(kStageAtoms, np - r0);
+          const int nat = (nr + 1) & ~1;
+          {  // 16 threads per atom, KH * 4 chunks of 16 bytes each
+            const int j = wt >> 4;
+            if (j < nr) {
+              const int n = r0 + j;
+              const int p = n < n_lo ? nth_set(m_lo, n) : 32 + nth_set(m_hi, n - n_lo);
+              const uint4* src = reinterpret_cast<const uint4*>(sCh + (size_t)p * (KH * 1024));
+              uint4* dst = reinterpret_cast<uint4*>(sStage + (size_t)j * (KH * 1024));
+              uint4 v[KH * 4];
+#pragma unroll
+              for (int u = 0; u < KH * 4; ++u) v[u] = src[(wt & 15) + 16 * u];
+#pragma unroll
+              for (int u = 0; u < KH * 4; ++u) dst[(wt & 15) + 16 * u] = v[u];
+            }
+          }
+          tc::fence_proxy_async_smem();
+          wg_bar(barid);  // staging written
+          if (wt == 0) {
+            tc::tc_fence_after();
+            const uint32_t idescC = tc::idesc_bf16(kKeys, 8 * nat, 0, 0);
+            const uint32_t sKa = tc::smem_u32(sRing + slot * S::kTile);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t ad = tc::sdesc_sw128(sKa + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024);
+              const uint64_t bd = tc::sdesc_sw128(sStA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+              tc::mma_bf16(tP, ad, bd, idescC, k > 0);
+            }
+            tc::mma_commit(bar_c);
+            if (!tc::mbar_wait(bar_c, ph_c)) atomicOr(a.err, kErrTimeout);
+            // last round: the K slot is read by nothing else now
+            if (r0 + kStageAtoms >= np && t + 2 * nwg < s1) issue_k(t + 2 * nwg, slot);
+          }
+          ph_c ^= 1;
+          wg_bar(barid);  // child scores in TMEM
+          tc::tc_fence_after();
+          // one TMEM load per distinct staging slot among this warp's keys
+          const int my = (myslot >= r0 && myslot < r0 + kStageAtoms) ? myslot - r0 : -1;
+          unsigned pending = __ballot_sync(0xffffffffu, my >= 0);
+          while (pending) {
+            const int sl = __shfl_sync(0xffffffffu, my, __ffs(pending) - 1);
+            uint32_t rr[8];
+            tmem_ld8(tP + lane_off + sl * 8, rr);
+            tc::tmem_wait_ld();
+            if (my == sl) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) vals[c] = __uint_as_float(rr[c]);
+            }
+            pending &= ~__ballot_sync(0xffffffffu, my == sl);
+          }
+          if (r0 + kStageAtoms < np) {
+            tc::tc_fence_before();
+            wg_bar(barid);  // staging and child columns free for the next round
+          }
+        }
+        float tchild = vals[0] + sNorm[M0 + par * 8];
+        int cstar = 0;
+#pragma unroll
+        for (int c = 1; c < 8; ++c) {
+          const float tc = vals[c] + sNorm[M0 + par * 8 + c];
+          if (tc > tchild) {
+            tchild = tc;
+            cstar = c;
+          }
+        }
+        if (tchild > best) code = M0 + par * 8 + cstar;
+      }
+      const int row = (t - bh * a.nblk) * kKeys + wt;
+      if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
+      count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
+    }
+    if (aborted) *sAbort = 1;
+    tc::tc_fence_before();
+    __syncthreads();  // every warpgroup done with this head's image
+    if (*sAbort) break;
+    s0 = s1;
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(*sTmem, ncols);
+  }
+}
+
 // Codewords -> swizzled-atom image (code a in atom a/8, row a%8) and fp32
 // squared norms.  Children of parent p are codes M0 + p*C + c.
 template <int D>
@@ -402,6 +802,39 @@ cudaError_t launch_impl(const Shape& s, const CUtensorMap& kmap, AssignArgs a, c
   const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
   assign_tc_kernel<D, CH><<<grid, 128, smem, st>>>(kmap, a);
   return cudaGetLastError();
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// Warpgroups per CTA for the pipelined kernel (0: the image does not fit).
+template <int D>
+int wg_count(const Shape& s) {
+  for (int nwg = 3; nwg >= 1; --nwg)
+    if (WgSmem<D>::total(s.M0, s.C, nwg) + 1024 <= kMaxSmem) return nwg;
+  return 0;
+}
+
+template <int D, int M0>
+cudaError_t launch_wg_m(const Shape& s, const CUtensorMap& kmap, AssignArgs a, int nwg, cudaStream_t st) {
+  const size_t smem = WgSmem<D>::total(s.M0, s.C, nwg) + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(assign_wg_kernel<D, M0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int ctas = std::min(a.ntiles, num_sms());
+  a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
+  const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+  assign_wg_kernel<D, M0><<<grid, 128 * nwg, smem, st>>>(kmap, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_wg(const Shape& s, const CUtensorMap& kmap, AssignArgs a, int nwg, cudaStream_t st) {
+  switch (s.M0) {
+    case 16: return launch_wg_m<D, 16>(s, kmap, a, nwg, st);
+    case 32: return launch_wg_m<D, 32>(s, kmap, a, nwg, st);
+    case 48: return launch_wg_m<D, 48>(s, kmap, a, nwg, st);
+    default: return launch_wg_m<D, 64>(s, kmap, a, nwg, st);
+  }
 }
 
 }  // namespace
@@ -452,6 +885,14 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
   a.ntiles = a.nblk * s.BH();
   a.tiles_per_cta = 1;
   const size_t ch_bytes = (size_t)s.M0 * s.C * s.d * 2;
+  if (s.M0 <= 64) {  // warpgroup-pipelined kernel when the whole image fits
+    const int nwg = s.d == 64 ? wg_count<64>(s) : wg_count<128>(s);
+    if (nwg > 0) {
+      e = s.d == 64 ? launch_wg<64>(s, kmap, a, nwg, st) : launch_wg<128>(s, kmap, a, nwg, st);
+      log.add("assign_tc_wg");
+      return e;
+    }
+  }
   const bool ch_smem = ch_bytes <= 96 * 1024;
   if (s.d == 64)
     e = ch_smem ? launch_impl<64, true>(s, kmap, a, st) : launch_impl<64, false>(s, kmap, a, st);
