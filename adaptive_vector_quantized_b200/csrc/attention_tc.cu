@@ -513,6 +513,407 @@ done:
   }
 }
 
+// ---------------------------------------------------------------------------
+// Fast path for one parent tile (M0 in {16, 32, 48, 64}, single sweep).
+// Same algorithm and data layout as the general kernel above; what changes is
+// work skipped because it cannot change the result, and earlier copies:
+//   - the parent masks (Eq. 18) are applied only when the block has an empty
+//     parent (a block-uniform test);
+//   - children: the rescale test uses the unmasked child maximum, so in the
+//     common case every 2^(t - m) is at most 2^24 and dA of an empty child is
+//     finite; its value sum and count are exactly zero, so it adds nothing to
+//     x or z and needs no mask.  Only if the unmasked maximum exceeds the
+//     reference by more than 2^24 are the masks applied (and x, z rescaled if
+//     the masked maximum does too).  A padding slot (odd number of parents in
+//     a chunk) gets a zero value atom for the same reason;
+//   - the codewords of chunk q + 1 are copied as soon as the logit MMA of
+//     chunk q has read its own, the value sums as soon as its value MMA has;
+//   - the value MMAs are not waited for until their operands are reused.
+template <int D>
+struct FastSmem {
+  static constexpr int kAtomBytes = 1024 * (D / 64);       // one 8-code atom group
+  static constexpr int kQ = 0;                             // Q tile / O staging
+  static constexpr int kCW = kQ + kRows * D * 2;           // codewords: parents, then chunks
+  static constexpr int kVB = kCW + 8 * kAtomBytes;         // value sums: parents, then chunks
+  static constexpr int kPR = kVB + 8 * kAtomBytes;         // probabilities / dA [128][64] bf16
+  static constexpr int kNF = kPR + kRows * 64 * 2;         // counts [2][64]: parents, current chunk
+  static constexpr int kW = kNF + 2 * 64 * 4;              // importance [64]
+  static constexpr int kWP = kW + 64 * 4;                  // per-warp partial sums [4][64]
+  static constexpr int kSEL = kWP + 4 * 64 * 4;            // selected parents [64]
+  static constexpr int kRK = kSEL + 64 * 4;                // partial ranks [2][64]
+  static constexpr int kBAR = kRK + 2 * 64 * 4;            // 6 mbarriers
+  static constexpr int kMISC = kBAR + 64;                  // tmem base, abort flag
+  static constexpr int kTotal = kMISC + 32;
+  static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
+};
+
+template <int D, int M0>
+__global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap, const AttnArgs a) {
+  using S = FastSmem<D>;
+  constexpr int KH = D / 64;
+  constexpr int AB = S::kAtomBytes;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = sm + S::kQ;
+  uint8_t* sCW = sm + S::kCW;
+  uint8_t* sVB = sm + S::kVB;
+  uint8_t* sPR = sm + S::kPR;
+  float* sNF = reinterpret_cast<float*>(sm + S::kNF);  // [0..63] parents, [64..127] current chunk
+  float* sW = reinterpret_cast<float*>(sm + S::kW);
+  float* sWP = reinterpret_cast<float*>(sm + S::kWP);
+  int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
+  int* sRK = reinterpret_cast<int*>(sm + S::kRK);
+  uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + S::kBAR);
+  uint64_t* bar_cw = bar_q + 1;   // codeword copies (parents, then one per chunk)
+  uint64_t* bar_vb = bar_q + 2;   // value-sum copies (parents, then one per chunk)
+  uint64_t* bar_mma = bar_q + 3;  // logit MMAs
+  uint64_t* bar_x = bar_q + 4;    // value MMAs
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S::kMISC);
+  int* sAbort = reinterpret_cast<int*>(sm + S::kMISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int blk = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
+  const int row0 = blk * kRows;
+  const bool valid = row0 + tid < a.N;
+  const int C = a.C, Mt = M0 * (1 + C), P = a.P;
+  const bf16* cw_h = a.cw + (size_t)h * (Mt / 8) * KH * 512;
+  const bf16* vb_bh = a.vb + (size_t)bh * (Mt / 8) * KH * 512;
+  const int32_t* cnt = a.counts + (size_t)bh * Mt;
+  const float NEG_INF = __int_as_float(0xff800000);
+  const float sl2 = a.scale_log2;
+
+  if (tid == 0) {
+    for (int i = 0; i < 5; ++i) tc::mbar_init(bar_q + i, 1);
+    tc::fence_mbar_init();
+    *sAbort = 0;
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(sTmem, S::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();  // barriers initialised before anyone waits on them
+  tc::tc_fence_after();
+  if (tid == 0) {
+    tc::prefetch_tensormap(&qmap);
+    tc::prefetch_tensormap(&omap);
+    tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh) tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, row0, bh, bar_q);
+    tc::mbar_arrive_expect_tx(bar_cw, M0 * D * 2);
+    tc::bulk_g2s(sCW, cw_h, M0 * D * 2, bar_cw);
+    tc::mbar_arrive_expect_tx(bar_vb, M0 * D * 2);
+    tc::bulk_g2s(sVB, vb_bh, M0 * D * 2, bar_vb);
+  }
+  float nfj = 0.f;
+  if (tid < M0) {
+    nfj = (float)__ldg(cnt + tid);
+    sNF[tid] = nfj;
+  }
+  if (!(tc::mbar_wait(bar_q, 0) && tc::mbar_wait(bar_cw, 0))) fail(a.err, sAbort);
+  tc::tc_fence_before();
+  const bool any_empty = __syncthreads_or(tid < M0 && !(nfj > 0.f)) != 0;
+  tc::tc_fence_after();
+  if (*sAbort) goto done;
+  {
+    const uint32_t tmem = *sTmem;
+    const uint32_t tS = tmem;          // logits
+    const uint32_t tX = tmem + kTile;  // output accumulator, D columns
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t sQa = tc::smem_u32(sQ), sCWa = tc::smem_u32(sCW), sVBa = tc::smem_u32(sVB),
+                   sPRa = tc::smem_u32(sPR);
+    const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
+    uint32_t ph_cw = 1, ph_vb = 0, ph_mma = 0, ph_x = 0;  // the parents' codeword phase is consumed
+
+    auto issue_logits = [&](int n) {  // S = Q * CW^T over n codes
+      const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint64_t ad = tc::sdesc_sw128(sQa + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::sdesc_sw128(sCWa + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+        tc::mma_bf16(tS, ad, bd, idesc, k > 0);
+      }
+      tc::mma_commit(bar_mma);
+    };
+    auto issue_values = [&](int n, bool acc) {  // x (+)= PR * VB over n codes
+      for (int k = 0; k < n / 16; ++k) {
+        const uint64_t ad = tc::sdesc_sw128(sPRa + (k & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::sdesc_sw128(sVBa + k * 2 * AB, 1024, KH * 1024);
+        tc::mma_bf16(tX, ad, bd, idesc_x, (acc || k > 0) ? 1u : 0u);
+      }
+      tc::mma_commit(bar_x);
+    };
+    auto wait_bar = [&](uint64_t* bar, uint32_t& ph) {
+      if (!tc::mbar_wait(bar, ph)) fail(a.err, sAbort);
+      ph ^= 1;
+    };
+    // child codewords / value sums of chunk q into the staging buffer (thread 0)
+    auto chunk_np = [&](int q) { return min(kChunkParents, P - q * kChunkParents); };
+    auto copy_cw = [&](int q) {
+      const int np = chunk_np(q), slots = (np + 1) & ~1;
+      tc::mbar_arrive_expect_tx(bar_cw, (uint32_t)slots * AB);
+      for (int rr = 0; rr < slots; ++rr) {
+        const int p = sSEL[q * kChunkParents + min(rr, np - 1)];
+        tc::bulk_g2s(sCW + rr * AB, cw_h + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_cw);
+      }
+    };
+    auto copy_vb = [&](int q) {
+      const int np = chunk_np(q);
+      tc::mbar_arrive_expect_tx(bar_vb, (uint32_t)np * AB);
+      for (int rr = 0; rr < np; ++rr) {
+        const int p = sSEL[q * kChunkParents + rr];
+        tc::bulk_g2s(sVB + rr * AB, vb_bh + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_vb);
+      }
+    };
+
+    // ---- parents: logits, masked max, A = 2^(t - m), z, importance ----
+    if (tid == 0) {
+      tc::tc_fence_after();
+      issue_logits(M0);
+    }
+    wait_bar(bar_mma, ph_mma);
+    tc::tc_fence_after();
+    float m, z;
+    {
+      uint32_t r[M0];
+#pragma unroll
+      for (int q = 0; q < M0 / 16; ++q) tc::tmem_ld16(tS + lane_off + q * 16, r + q * 16);
+      tc::tmem_wait_ld();
+      const float4* nf4 = reinterpret_cast<const float4*>(sNF);
+      float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+      if (!any_empty) {
+#pragma unroll
+        for (int e = 0; e < M0; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(r[e]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < M0; e += 4) {
+          const float4 nf = nf4[e >> 2];
+          mx[0] = fmaxf(mx[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
+          mx[1] = fmaxf(mx[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
+          mx[2] = fmaxf(mx[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
+          mx[3] = fmaxf(mx[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
+        }
+      }
+      m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      const float nm = -m;
+      float zp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < M0; e += 4) {
+        const float4 nf = nf4[e >> 2];
+        float a0 = tc::ex2(fmaf(__uint_as_float(r[e]), sl2, nm));
+        float a1 = tc::ex2(fmaf(__uint_as_float(r[e + 1]), sl2, nm));
+        float a2 = tc::ex2(fmaf(__uint_as_float(r[e + 2]), sl2, nm));
+        float a3 = tc::ex2(fmaf(__uint_as_float(r[e + 3]), sl2, nm));
+        if (any_empty) {
+          a0 = nf.x > 0.f ? a0 : 0.f;
+          a1 = nf.y > 0.f ? a1 : 0.f;
+          a2 = nf.z > 0.f ? a2 : 0.f;
+          a3 = nf.w > 0.f ? a3 : 0.f;
+        }
+        zp[0] = fmaf(a0, nf.x, zp[0]);
+        zp[1] = fmaf(a1, nf.y, zp[1]);
+        zp[2] = fmaf(a2, nf.z, zp[2]);
+        zp[3] = fmaf(a3, nf.w, zp[3]);
+        r[e] = __float_as_uint(a0);
+        r[e + 1] = __float_as_uint(a1);
+        r[e + 2] = __float_as_uint(a2);
+        r[e + 3] = __float_as_uint(a3);
+      }
+      z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+#pragma unroll
+      for (int c = 0; c < M0 / 8; ++c) store_chunk8(sPR, tid, c * 8, reinterpret_cast<const float*>(r) + c * 8);
+      // importance column sums of A / z (Eq. 7), fp32
+      const float rz = valid ? 1.f / z : 0.f;
+#pragma unroll
+      for (int g = 0; g < (M0 + 31) / 32; ++g) {
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = (g * 32 + e < M0) ? __uint_as_float(r[(g * 32 + e) % M0]) * rz : 0.f;
+        sWP[warp * 64 + g * 32 + lane] = reduce_scatter32(v, lane);
+      }
+    }
+    tc::fence_proxy_async_smem();
+    wait_bar(bar_vb, ph_vb);
+    tc::tc_fence_before();
+    __syncthreads();
+    if (*sAbort) goto done;
+    if (tid < M0) sW[tid] = nfj * ((sWP[tid] + sWP[64 + tid]) + (sWP[128 + tid] + sWP[192 + tid]));
+    if (tid == 0) {
+      tc::tc_fence_after();
+      issue_values(M0, false);
+    }
+    __syncthreads();
+
+    // ---- top-P over the importance (descending, ties to the lower index) ----
+    {
+      const int j = tid % M0, half = tid / M0;
+      if (tid < 2 * M0) {
+        const float wj = sW[j];
+        const int l0 = half * (M0 >> 1), l1 = half ? M0 : (M0 >> 1);
+        int rank = 0;
+        for (int l = l0; l < l1; ++l) {
+          const float wl = sW[l];
+          rank += (wl > wj) || (wl == wj && l < j);
+        }
+        sRK[half * 64 + j] = rank;
+      }
+      __syncthreads();
+      if (tid < M0) {
+        const int rank = sRK[tid] + sRK[64 + tid];
+        if (rank < P) sSEL[rank] = tid;
+        if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = sW[tid];
+      }
+      __syncthreads();
+      if (a.sel)
+        for (int rr = tid; rr < P; rr += 128) a.sel[((size_t)bh * a.nblk + blk) * P + rr] = sSEL[rr];
+    }
+    // every thread waits for the parents' value MMA (its operands are reused next)
+    wait_bar(bar_x, ph_x);
+    const int nch = (C > 0 && P > 0) ? (P + kChunkParents - 1) / kChunkParents : 0;
+    if (tid == 0 && nch > 0) {
+      copy_cw(0);
+      copy_vb(0);
+    }
+
+    // ---- child refinement in chunks of 8 selected parents ----
+    float mref = m;
+    float* nfc = sNF + 64;
+    for (int q = 0; q < nch; ++q) {
+      const int np = chunk_np(q);
+      const int slots = (np + 1) & ~1;
+      const int n = slots * 8;
+      wait_bar(bar_cw, ph_cw);
+      if (tid < 64) {
+        const int rr = tid >> 3;
+        nfc[tid] = rr < np ? (float)__ldg(cnt + M0 + sSEL[q * kChunkParents + rr] * 8 + (tid & 7)) : 0.f;
+      }
+      tc::tc_fence_before();
+      __syncthreads();
+      if (*sAbort) goto done;
+      if (tid == 0) {
+        tc::tc_fence_after();
+        issue_logits(n);
+      }
+      wait_bar(bar_mma, ph_mma);
+      tc::tc_fence_after();
+      if (tid == 0 && q + 1 < nch) copy_cw(q + 1);  // the logit MMA has read this chunk's codewords
+      uint32_t r[64];
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        if (g * 16 < n) tc::tmem_ld16(tS + lane_off + g * 16, r + g * 16);
+      tc::tmem_wait_ld();
+      const float4* nf4 = reinterpret_cast<const float4*>(nfc);
+      float cm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        if (e < n) cm[e & 3] = fmaxf(cm[e & 3], __uint_as_float(r[e]));
+      const float cmax_any = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) * sl2;
+      if (q > 0) wait_bar(bar_x, ph_x);  // previous chunk's value MMA: PR, VB and x are free
+      const bool masked = __syncthreads_or(cmax_any > mref + kRescaleLog2) != 0;  // block-uniform, rare
+      if (tid == 0 && q > 0) copy_vb(q);
+      if (masked) {
+        // masked maximum over non-empty children; rescale x and z if it is far above
+        float cmm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+          if (e < n) {
+            const float4 nf = nf4[e >> 2];
+            cmm[0] = fmaxf(cmm[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
+            cmm[1] = fmaxf(cmm[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
+            cmm[2] = fmaxf(cmm[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
+            cmm[3] = fmaxf(cmm[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
+          }
+        }
+        const float cmax = fmaxf(fmaxf(cmm[0], cmm[1]), fmaxf(cmm[2], cmm[3])) * sl2;
+        const bool need = cmax > mref + kRescaleLog2;
+        if (__syncthreads_or(need)) {
+          tc::tc_fence_after();
+          const float f = need ? tc::ex2(mref - cmax) : 1.f;
+          for (int g = 0; g < D; g += 16) {
+            uint32_t xr[16];
+            tc::tmem_ld16(tX + lane_off + g, xr);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xr[e] = __float_as_uint(__uint_as_float(xr[e]) * f);
+            tc::tmem_st16(tX + lane_off + g, xr);
+          }
+          tc::tmem_wait_st();
+          z *= f;
+          if (need) mref = cmax;
+        }
+      }
+      // dA = 2^(t_c - m) - 2^(t_p - m), t_p the mean of the 8 child logits (Eq. 8)
+      const float nm = -mref, sl8 = sl2 * 0.125f;
+      float zp[2] = {0.f, 0.f};
+#pragma unroll
+      for (int sl = 0; sl < 8; ++sl) {
+        if (sl < slots) {
+          float ssum = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ssum += __uint_as_float(r[sl * 8 + e]);
+          const float ap = tc::ex2(fmaf(ssum, sl8, nm));
+          const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
+          const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+          float da[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            da[e] = tc::ex2(fmaf(__uint_as_float(r[sl * 8 + e]), sl2, nm)) - ap;
+            if (masked && !(nfv[e] > 0.f)) da[e] = 0.f;
+            zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
+          }
+          store_chunk8(sPR, tid, sl * 8, da);
+        }
+      }
+      z += zp[0] + zp[1];
+      if (np & 1)  // padding slot: zero value sums, so it adds nothing
+        for (int i = tid; i < AB / 16; i += 128)
+          reinterpret_cast<uint4*>(sVB + np * AB)[i] = make_uint4(0, 0, 0, 0);
+      tc::fence_proxy_async_smem();
+      wait_bar(bar_vb, ph_vb);
+      tc::tc_fence_before();
+      __syncthreads();
+      if (*sAbort) goto done;
+      if (tid == 0) {
+        tc::tc_fence_after();
+        issue_values(n, true);
+      }
+    }
+    if (nch > 0) wait_bar(bar_x, ph_x);  // the last value MMA
+    tc::tc_fence_after();
+
+    // ---- O = x / z -> bf16 -> shared (Q region) -> TMA store ----
+    {
+      const float iz = 1.f / z;
+      for (int g = 0; g < D; g += 16) {
+        uint32_t xr[16];
+        tc::tmem_ld16(tX + lane_off + g, xr);
+        tc::tmem_wait_ld();
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(xr[e]) * iz;
+        store_chunk8(sQ, tid, g, v);
+        store_chunk8(sQ, tid, g + 8, v + 8);
+      }
+      tc::fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh) tc::tma_store_3d(&omap, sQ + kh * kRows * 128, kh * 64, row0, bh);
+        tc::bulk_commit_group();
+        tc::bulk_wait_group_read0();
+      }
+    }
+  }
+done:
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(*sTmem, S::kTmemCols);
+  }
+}
+
 // Codewords and value sums -> bf16 images of swizzled atoms.  Code a of a head
 // (parents first, then child c of parent p at M0 + p*C + c) lands in atom
 // a/8, row a%8; for d = 128 each atom group holds two 64-column halves.
@@ -551,6 +952,28 @@ __global__ void __launch_bounds__(256) attention_prep_kernel(const bf16* __restr
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+template <int D, int M0>
+cudaError_t launch_fast_m(dim3 grid, const CUtensorMap& qmap, const CUtensorMap& omap, const AttnArgs& a,
+                          cudaStream_t st) {
+  const int smem = FastSmem<D>::kTotal + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(attention_fast_kernel<D, M0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attention_fast_kernel<D, M0><<<grid, 128, smem, st>>>(qmap, omap, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_fast(int M0, dim3 grid, const CUtensorMap& qmap, const CUtensorMap& omap, const AttnArgs& a,
+                        cudaStream_t st) {
+  switch (M0) {
+    case 16: return launch_fast_m<D, 16>(grid, qmap, omap, a, st);
+    case 32: return launch_fast_m<D, 32>(grid, qmap, omap, a, st);
+    case 48: return launch_fast_m<D, 48>(grid, qmap, omap, a, st);
+    default: return launch_fast_m<D, 64>(grid, qmap, omap, a, st);
+  }
+}
 
 }  // namespace
 
@@ -609,6 +1032,11 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
   a.two_pass = two_pass;
   a.scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(a.nblk, s.BH());
+  if (!two_pass && s.M0 <= 64) {  // one parent tile: the fast kernel
+    e = s.d == 64 ? launch_fast<64>(s.M0, grid, qmap, omap, a, st) : launch_fast<128>(s.M0, grid, qmap, omap, a, st);
+    log.add("attention_tc_fast");
+    return e;
+  }
   if (s.d == 64) {
     const int smem = Smem<64>::kTotal + 1024;
     e = cudaFuncSetAttribute(attention_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

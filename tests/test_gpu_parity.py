@@ -128,6 +128,25 @@ def test_tc_attention_rescale_path():
     print("rescale", res["kernels"], diag)
 
 
+@pytest.mark.parametrize("P", [3, 13, 24, 40, 64])
+def test_tc_attention_chunking(inputs, P):
+    """Tensor-core attention with P not a multiple of 8 (a padded child slot)
+    and with more than two chunks of 8 parents (staging buffers reused)."""
+    inp = inputs("vit_h3")
+    res = _forward_tc_attention(inp, P=P)
+    assert "attention_tc" in res["kernels"]
+    gh.check_forward(inp, res, P=P)
+
+
+def test_tc_m0_48(inputs):
+    """M0 = 48: a parent count that is not a power of two on both tensor-core stages."""
+    cfg = _cfg(N=1000, M0=48, P=7)
+    inp = synth.make_inputs(cfg, 18)
+    res = gh.gpu_forward(inp, path=avq.AVQ_PATH_TC)
+    assert "assign_tc" in res["kernels"] and "attention_tc" in res["kernels"]
+    gh.check_forward(inp, res)
+
+
 @pytest.mark.parametrize("P,block", [(0, 128), (1, 64), (8, 128), (64, 64)])
 def test_vit_p_and_block_variants(inputs, P, block):
     inp = inputs("vit_h3")
