@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     nfj = (float)__ldg(cnt + tid);
     sNF[tid] = nfj;
   }
-  if (!(tc::mbar_wait(bar_q, 0) && tc::mbar_wait(bar_cw, 0))) fail(a.err, sAbort);
+  if (tid == 0 && !(tc::mbar_wait(bar_q, 0) && tc::mbar_wait(bar_cw, 0))) fail(a.err, sAbort);
   tc::tc_fence_before();
   const bool any_empty = __syncthreads_or(tid < M0 && !(nfj > 0.f)) != 0;
   tc::tc_fence_after();
@@ -644,8 +644,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       }
       tc::mma_commit(bar_x);
     };
+    // Waits are taken by thread 0 alone; the others meet it at the CTA barrier
+    // that follows every wait, so no warp spins on the issue slots.
     auto wait_bar = [&](uint64_t* bar, uint32_t& ph) {
-      if (!tc::mbar_wait(bar, ph)) fail(a.err, sAbort);
+      if (tid == 0 && !tc::mbar_wait(bar, ph)) fail(a.err, sAbort);
       ph ^= 1;
     };
     // child codewords / value sums of chunk q into the staging buffer (thread 0)
@@ -673,6 +675,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       issue_logits(M0);
     }
     wait_bar(bar_mma, ph_mma);
+    __syncthreads();
     tc::tc_fence_after();
     float m, z;
     {
@@ -768,7 +771,8 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       if (a.sel)
         for (int rr = tid; rr < P; rr += 128) a.sel[((size_t)bh * a.nblk + blk) * P + rr] = sSEL[rr];
     }
-    // every thread waits for the parents' value MMA (its operands are reused next)
+    // the parents' value MMA must be done before its operands are reused; the
+    // CTA barrier after the first child copies orders everyone behind this
     wait_bar(bar_x, ph_x);
     const int nch = (C > 0 && P > 0) ? (P + kChunkParents - 1) / kChunkParents : 0;
     if (tid == 0 && nch > 0) {
@@ -796,8 +800,9 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         issue_logits(n);
       }
       wait_bar(bar_mma, ph_mma);
-      tc::tc_fence_after();
       if (tid == 0 && q + 1 < nch) copy_cw(q + 1);  // the logit MMA has read this chunk's codewords
+      __syncthreads();
+      tc::tc_fence_after();
       uint32_t r[64];
 #pragma unroll
       for (int g = 0; g < 4; ++g)
@@ -880,6 +885,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       }
     }
     if (nch > 0) wait_bar(bar_x, ph_x);  // the last value MMA
+    __syncthreads();
     tc::tc_fence_after();
 
     // ---- O = x / z -> bf16 -> shared (Q region) -> TMA store ----
