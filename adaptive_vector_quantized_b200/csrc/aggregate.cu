@@ -23,16 +23,52 @@ namespace avq {
 
 namespace {
 
-// Streaming variant (the default): every warp owns a contiguous range of
-// keys of one head (so runs of equal codes stay long), lanes cover the head
-// dimension, value rows are loaded straight from global memory in batches of
-// eight keys, codes one 32-key group ahead.  Per 32-key group, warp ballots
-// mark where runs start, so the per-key work is a bit test and two adds.  A
-// finished run is added to the global value sums (L2 resident) with one
-// vector reduction per lane; there are no shared-memory atomics and no
-// per-CTA partials.  Counts are produced by the assignment kernels.
+// Streaming variant (the default), in two steps.  First every key's value is
+// added to its final code only (the child if it moved, else the parent):
+// every warp owns a contiguous range of keys of one head (so runs of equal
+// codes stay long), lanes cover the head dimension, a warp ballot per 32-key
+// group marks where runs start, the group's value rows are loaded up front
+// (one coalesced row per key) and the keys are walked in a fully unrolled
+// loop whose per-key work is a bit test and the adds.  A finished run is
+// added to the global value sums (L2 resident) with one vector reduction per
+// lane.  Then each parent adds its children's sums to its own, which makes
+// it the sum over its whole cluster (Eq. 3).  Counts are produced by the
+// assignment kernels.
 constexpr int kStreamThreads = 256;
-constexpr int kStreamBatch = 8;
+
+// One lane's E consecutive elements of a value row, as loaded.
+template <typename T, int E>
+struct Frag;
+template <>
+struct Frag<bf16, 2> {
+  using R = uint32_t;
+  static constexpr int kBatch = 32;
+  __device__ __forceinline__ static R load(const bf16* p) { return __ldg(reinterpret_cast<const unsigned*>(p)); }
+  __device__ __forceinline__ static void unpack(R r, float* o) { o[0] = bf16_lo(r); o[1] = bf16_hi(r); }
+};
+template <>
+struct Frag<bf16, 4> {
+  using R = uint2;
+  static constexpr int kBatch = 32;
+  __device__ __forceinline__ static R load(const bf16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
+  __device__ __forceinline__ static void unpack(R r, float* o) {
+    o[0] = bf16_lo(r.x); o[1] = bf16_hi(r.x); o[2] = bf16_lo(r.y); o[3] = bf16_hi(r.y);
+  }
+};
+template <>
+struct Frag<float, 2> {
+  using R = float2;
+  static constexpr int kBatch = 32;
+  __device__ __forceinline__ static R load(const float* p) { return __ldg(reinterpret_cast<const float2*>(p)); }
+  __device__ __forceinline__ static void unpack(R r, float* o) { o[0] = r.x; o[1] = r.y; }
+};
+template <>
+struct Frag<float, 4> {
+  using R = float4;
+  static constexpr int kBatch = 16;
+  __device__ __forceinline__ static R load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+  __device__ __forceinline__ static void unpack(R r, float* o) { o[0] = r.x; o[1] = r.y; o[2] = r.z; o[3] = r.w; }
+};
 
 template <int E>
 __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* acc, int lane, int D) {
@@ -47,8 +83,10 @@ __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* ac
 template <typename T, int D>
 __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum, int BH, int N,
-    int M0, int C, int keys_per_warp, int log2C) {
+    int M0, int C, int keys_per_warp) {
   constexpr int E = D / 32;
+  using F = Frag<T, E>;
+  constexpr int B = F::kBatch;  // keys loaded at once (32 / B batches per group)
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kStreamThreads / 32) + (threadIdx.x >> 5);
   const int warps_per_head = (N + keys_per_warp - 1) / keys_per_warp;
@@ -61,60 +99,61 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   const T* vb = V + (size_t)bh * N * D + lane * E;
   const int32_t* asg = assign + (size_t)bh * N;
 
-  float accP[E], accC[E];
+  float acc[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) accP[e] = accC[e] = 0.f;
-  int curP = -1, curC = -1;
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  int cur = -1;
   int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
   for (int g = j0; g < j1; g += 32) {
     const int code = code_next;
     code_next = g + 32 + lane < j1 ? __ldg(asg + g + 32 + lane) : -1;
-    const int par = code < M0 ? code : (log2C >= 0 ? (code - M0) >> log2C : (code - M0) / max(C, 1));
     const int prevc = __shfl_up_sync(0xffffffffu, code, 1);
-    const int prevp = __shfl_up_sync(0xffffffffu, par, 1);
-    const unsigned live = __ballot_sync(0xffffffffu, code >= 0);
+    const int nlive = __popc(__ballot_sync(0xffffffffu, code >= 0));
     // run starts relative to the previous key (lane 0 compares with the open run)
-    const unsigned newP = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? par != curP : prevp != par));
-    const unsigned isC = __ballot_sync(0xffffffffu, code >= M0);
-    const unsigned newC = __ballot_sync(0xffffffffu, code >= M0 && (lane == 0 ? code != curC : prevc != code));
-    const int nlive = __popc(live);
-    for (int u0 = 0; u0 < nlive; u0 += kStreamBatch) {
-      float v[kStreamBatch][E];
+    const unsigned newR = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? code != cur : prevc != code));
 #pragma unroll
-      for (int b = 0; b < kStreamBatch; ++b)
-        if (u0 + b < nlive) loadE<E>(vb + (size_t)(g + u0 + b) * D, v[b]);
+    for (int b0 = 0; b0 < 32; b0 += B) {
+      typename F::R raw[B];
 #pragma unroll
-      for (int b = 0; b < kStreamBatch; ++b) {
-        const int u = u0 + b;
-        if (u >= nlive) break;
-        const unsigned bit = 1u << u;
-        if (newP & bit) {
-          if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
-          curP = __shfl_sync(0xffffffffu, par, u);
+      for (int b = 0; b < B; ++b)
+        if (b0 + b < nlive) raw[b] = F::load(vb + (size_t)(g + b0 + b) * D);
 #pragma unroll
-          for (int e = 0; e < E; ++e) accP[e] = 0.f;
-        }
+      for (int b = 0; b < B; ++b) {
+        const int u = b0 + b;
+        if (u < nlive) {
+          float v[E];
+          F::unpack(raw[b], v);
+          if ((newR >> u) & 1u) {
+            if (cur >= 0) flush_sum<E>(vs, cur, acc, lane, D);
+            cur = __shfl_sync(0xffffffffu, code, u);
 #pragma unroll
-        for (int e = 0; e < E; ++e) accP[e] += v[b][e];
-        if (isC & bit) {
-          if (newC & bit) {
-            // the previous key may have stayed at a parent: compare with the open run
-            const int c = __shfl_sync(0xffffffffu, code, u);
-            if (c != curC) {
-              if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
-              curC = c;
-#pragma unroll
-              for (int e = 0; e < E; ++e) accC[e] = 0.f;
-            }
+            for (int e = 0; e < E; ++e) acc[e] = 0.f;
           }
 #pragma unroll
-          for (int e = 0; e < E; ++e) accC[e] += v[b][e];
+          for (int e = 0; e < E; ++e) acc[e] += v[e];
         }
       }
     }
   }
-  if (curP >= 0) flush_sum<E>(vs, curP, accP, lane, D);
-  if (curC >= 0) flush_sum<E>(vs, curC, accC, lane, D);
+  if (cur >= 0) flush_sum<E>(vs, cur, acc, lane, D);
+}
+
+// Parents hold their whole cluster: add the children's sums (keys that moved)
+// to the parent's own (keys that stayed), children in index order.
+__global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restrict__ vsum, int BH, int M0, int C,
+                                                               int D) {
+  const int Mt = M0 * (1 + C);
+  const long long total = (long long)BH * M0 * D;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(u % D);
+    const long long bp = u / D;
+    const int p = (int)(bp % M0);
+    float* vs = vsum + (bp / M0) * (long long)Mt * D;
+    float s = vs[(size_t)p * D + t];
+    for (int c = 0; c < C; ++c) s += vs[(size_t)(M0 + p * C + c) * D + t];
+    vs[(size_t)p * D + t] = s;
+  }
 }
 
 // ---- deterministic variant ------------------------------------------------
@@ -303,9 +342,6 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   if (e != cudaSuccess) return e;
   (void)counts;
   const int sms = num_sms();
-  int log2C = -1;
-  for (int b = 0; b <= 3; ++b)
-    if (s.C == (1 << b)) log2C = b;
   // grid sized for about 32 resident warps per SM, each a contiguous multiple of 32 keys
   const long long total_keys = (long long)s.BH() * s.N;
   const long long want_warps = (long long)sms * 32;
@@ -316,14 +352,21 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   const unsigned blocks = (unsigned)((warps + (kStreamThreads / 32) - 1) / (kStreamThreads / 32));
 #define AVQ_STREAM(T, D)                                                                            \
   aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, s.BH(), \
-                                                                   s.N, s.M0, s.C, kpw, log2C)
+                                                                   s.N, s.M0, s.C, kpw)
   if (dt == AVQ_F32) {
     if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
   } else {
     if (s.d == 64) AVQ_STREAM(bf16, 64); else AVQ_STREAM(bf16, 128);
   }
 #undef AVQ_STREAM
-  log.add("aggregate_stream");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (s.C > 0) {
+    const long long work = (long long)s.BH() * s.M0 * s.d;
+    const int pb = (int)std::min<long long>((work + 255) / 256, (long long)sms * 8);
+    aggregate_parents_kernel<<<pb, 256, 0, st>>>(vsum, s.BH(), s.M0, s.C, s.d);
+  }
+  log.add(s.C > 0 ? "aggregate_stream aggregate_parents" : "aggregate_stream");
   (void)err;
   return cudaGetLastError();
 }
