@@ -749,35 +749,38 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     __syncthreads();
 
     // ---- top-P over the importance (descending, ties to the lower index) ----
-    {
-      const int j = tid % M0, half = tid / M0;
-      if (tid < 2 * M0) {
-        const float wj = sW[j];
-        const int l0 = half * (M0 >> 1), l1 = half ? M0 : (M0 >> 1);
-        int rank = 0;
-        for (int l = l0; l < l1; ++l) {
-          const float wl = sW[l];
-          rank += (wl > wj) || (wl == wj && l < j);
-        }
-        sRK[half * 64 + j] = rank;
-      }
-      __syncthreads();
-      if (tid < M0) {
-        const int rank = sRK[tid] + sRK[64 + tid];
-        if (rank < P) sSEL[rank] = tid;
-        if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = sW[tid];
-      }
-      __syncthreads();
-      if (a.sel)
-        for (int rr = tid; rr < P; rr += 128) a.sel[((size_t)bh * a.nblk + blk) * P + rr] = sSEL[rr];
-    }
-    // the parents' value MMA must be done before its operands are reused; the
-    // CTA barrier after the first child copies orders everyone behind this
-    wait_bar(bar_x, ph_x);
+    // thread j < M0 ranks parent j against all M0 importances held in registers
     const int nch = (C > 0 && P > 0) ? (P + kChunkParents - 1) / kChunkParents : 0;
+    if (tid < M0) {
+      const float wj = sW[tid];
+      int rank = 0;
+#pragma unroll 1
+      for (int l0 = 0; l0 < M0; l0 += 16) {
+        float wv[16];
+#pragma unroll
+        for (int l = 0; l < 16; l += 4) {
+          const float4 w4 = reinterpret_cast<const float4*>(sW)[(l0 + l) >> 2];
+          wv[l] = w4.x;
+          wv[l + 1] = w4.y;
+          wv[l + 2] = w4.z;
+          wv[l + 3] = w4.w;
+        }
+#pragma unroll
+        for (int l = 0; l < 16; ++l) rank += (wv[l] > wj) || (wv[l] == wj && l0 + l < tid);
+      }
+      if (rank < P) {
+        sSEL[rank] = tid;
+        if (a.sel) a.sel[((size_t)bh * a.nblk + blk) * P + rank] = tid;
+      }
+      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = wj;
+    }
+    __syncthreads();
     if (tid == 0 && nch > 0) {
-      copy_cw(0);
+      copy_cw(0);  // the parent logit MMA has read the codewords
+      wait_bar(bar_x, ph_x);  // the parents' value MMA has read PR and VB
       copy_vb(0);
+    } else {
+      wait_bar(bar_x, ph_x);
     }
 
     // ---- child refinement in chunks of 8 selected parents ----
@@ -787,11 +790,11 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       const int np = chunk_np(q);
       const int slots = (np + 1) & ~1;
       const int n = slots * 8;
-      wait_bar(bar_cw, ph_cw);
       if (tid < 64) {
         const int rr = tid >> 3;
         nfc[tid] = rr < np ? (float)__ldg(cnt + M0 + sSEL[q * kChunkParents + rr] * 8 + (tid & 7)) : 0.f;
       }
+      wait_bar(bar_cw, ph_cw);
       tc::tc_fence_before();
       __syncthreads();
       if (*sAbort) goto done;
