@@ -547,6 +547,11 @@ struct FastSmem {
   static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
 };
 
+// The value MMAs are issued by a thread of the last warp, so that their issue
+// (about a hundred cycles per instruction) overlaps the logit MMAs, copies and
+// waits that thread 0 and warp 0 take care of.
+constexpr int kValueIssuer = 96;
+
 template <int D, int M0>
 __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap, const AttnArgs a) {
@@ -650,22 +655,25 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       if (tid == 0 && !tc::mbar_wait(bar, ph)) fail(a.err, sAbort);
       ph ^= 1;
     };
-    // child codewords / value sums of chunk q into the staging buffer (thread 0)
+    // child codewords / value sums of chunk q into the staging buffer: warp 0,
+    // one bulk copy per lane after lane 0 has announced the byte count
     auto chunk_np = [&](int q) { return min(kChunkParents, P - q * kChunkParents); };
     auto copy_cw = [&](int q) {
       const int np = chunk_np(q), slots = (np + 1) & ~1;
-      tc::mbar_arrive_expect_tx(bar_cw, (uint32_t)slots * AB);
-      for (int rr = 0; rr < slots; ++rr) {
-        const int p = sSEL[q * kChunkParents + min(rr, np - 1)];
-        tc::bulk_g2s(sCW + rr * AB, cw_h + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_cw);
+      if (lane == 0) tc::mbar_arrive_expect_tx(bar_cw, (uint32_t)slots * AB);
+      __syncwarp();
+      if (lane < slots) {
+        const int p = sSEL[q * kChunkParents + min(lane, np - 1)];
+        tc::bulk_g2s(sCW + lane * AB, cw_h + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_cw);
       }
     };
     auto copy_vb = [&](int q) {
       const int np = chunk_np(q);
-      tc::mbar_arrive_expect_tx(bar_vb, (uint32_t)np * AB);
-      for (int rr = 0; rr < np; ++rr) {
-        const int p = sSEL[q * kChunkParents + rr];
-        tc::bulk_g2s(sVB + rr * AB, vb_bh + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_vb);
+      if (lane == 0) tc::mbar_arrive_expect_tx(bar_vb, (uint32_t)np * AB);
+      __syncwarp();
+      if (lane < np) {
+        const int p = sSEL[q * kChunkParents + lane];
+        tc::bulk_g2s(sVB + lane * AB, vb_bh + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_vb);
       }
     };
 
@@ -742,11 +750,11 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     __syncthreads();
     if (*sAbort) goto done;
     if (tid < M0) sW[tid] = nfj * ((sWP[tid] + sWP[64 + tid]) + (sWP[128 + tid] + sWP[192 + tid]));
-    if (tid == 0) {
+    __syncthreads();
+    if (tid == kValueIssuer) {  // the parents' value MMA, issued while the others rank
       tc::tc_fence_after();
       issue_values(M0, false);
     }
-    __syncthreads();
 
     // ---- top-P over the importance (descending, ties to the lower index) ----
     // thread j < M0 ranks parent j against all M0 importances held in registers
@@ -775,12 +783,11 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = wj;
     }
     __syncthreads();
-    if (tid == 0 && nch > 0) {
-      copy_cw(0);  // the parent logit MMA has read the codewords
-      wait_bar(bar_x, ph_x);  // the parents' value MMA has read PR and VB
+    if (warp == 0 && nch > 0) copy_cw(0);  // the parent logit MMA has read the codewords
+    wait_bar(bar_x, ph_x);                 // the parents' value MMA has read PR and VB
+    if (warp == 0 && nch > 0) {
+      __syncwarp();
       copy_vb(0);
-    } else {
-      wait_bar(bar_x, ph_x);
     }
 
     // ---- child refinement in chunks of 8 selected parents ----
@@ -803,7 +810,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         issue_logits(n);
       }
       wait_bar(bar_mma, ph_mma);
-      if (tid == 0 && q + 1 < nch) copy_cw(q + 1);  // the logit MMA has read this chunk's codewords
+      if (warp == 0 && q + 1 < nch) {  // the logit MMA has read this chunk's codewords
+        __syncwarp();
+        copy_cw(q + 1);
+      }
       __syncthreads();
       tc::tc_fence_after();
       uint32_t r[64];
@@ -819,7 +829,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       const float cmax_any = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) * sl2;
       if (q > 0) wait_bar(bar_x, ph_x);  // previous chunk's value MMA: PR, VB and x are free
       const bool masked = __syncthreads_or(cmax_any > mref + kRescaleLog2) != 0;  // block-uniform, rare
-      if (tid == 0 && q > 0) copy_vb(q);
+      if (warp == 0 && q > 0) copy_vb(q);
       if (masked) {
         // masked maximum over non-empty children; rescale x and z if it is far above
         float cmm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
@@ -882,7 +892,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       tc::tc_fence_before();
       __syncthreads();
       if (*sAbort) goto done;
-      if (tid == 0) {
+      if (tid == kValueIssuer) {
         tc::tc_fence_after();
         issue_values(n, true);
       }
