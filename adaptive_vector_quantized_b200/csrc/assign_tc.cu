@@ -660,7 +660,6 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
           sMask[(slot ^ 1) * 2] = 0;
           sMask[(slot ^ 1) * 2 + 1] = 0;
         }
-        next_parents();
         const uint32_t m_lo = mk[0], m_hi = mk[1];
         const int n_lo = __popc(m_lo), np = n_lo + __popc(m_hi);
         const int myslot = par < 32 ? __popc(m_lo & ((1u << par) - 1u))
@@ -698,6 +697,9 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
               tc::mma_bf16(tP, ad, bd, idescC, k > 0);
             }
             tc::mma_commit(bar_c);
+            // the next tile's parent MMA queues behind this child MMA; its issue
+            // overlaps the child MMA instead of delaying the staging barrier
+            if (r0 == 0) next_parents();
             if (!tc::mbar_wait(bar_c, ph_c)) atomicOr(a.err, kErrTimeout);
             // last round: the K slot is read by nothing else now
             if (r0 + kStageAtoms >= np && t + 2 * nwg < s1) issue_k(t + 2 * nwg, slot);
