@@ -27,9 +27,10 @@ namespace {
 // added to its final code only (the child if it moved, else the parent):
 // every warp owns a contiguous range of keys of one head (so runs of equal
 // codes stay long), lanes cover the head dimension, a warp ballot per 32-key
-// group marks where runs start, the group's value rows are loaded up front
-// (one coalesced row per key) and the keys are walked in a fully unrolled
-// loop whose per-key work is a bit test and the adds.  A finished run is
+// group marks where runs start, and the keys are walked in sub-batches of
+// eight (one coalesced row load per key, the next sub-batch in flight while
+// the current one is added) whose per-key work is a bit test and the adds,
+// into two partial sums per run.  A finished run is
 // added to the global value sums (L2 resident) with one vector reduction per
 // lane.  Then each parent adds its children's sums to its own, which makes
 // it the sum over its whole cluster (Eq. 3).  Counts are produced by the
@@ -99,10 +100,21 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   const T* vb = V + (size_t)bh * N * D + lane * E;
   const int32_t* asg = assign + (size_t)bh * N;
 
-  float acc[E];
+  // two partial sums per run (even and odd keys of a group) halve the chain of
+  // dependent adds; they are combined when the run is flushed
+  float acc[2][E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int e = 0; e < E; ++e) acc[0][e] = acc[1][e] = 0.f;
   int cur = -1;
+  auto flush = [&]() {
+    float t[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      t[e] = acc[0][e] + acc[1][e];
+      acc[0][e] = acc[1][e] = 0.f;
+    }
+    flush_sum<E>(vs, cur, t, lane, D);
+  };
   int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
   for (int g = j0; g < j1; g += 32) {
     const int code = code_next;
@@ -111,31 +123,36 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     const int nlive = __popc(__ballot_sync(0xffffffffu, code >= 0));
     // run starts relative to the previous key (lane 0 compares with the open run)
     const unsigned newR = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? code != cur : prevc != code));
+    // keys in sub-batches of 8: the next sub-batch's rows are loaded while the
+    // current one is walked (16 rows in flight per warp, few registers)
+    typename F::R raw[8], nxt[8];
 #pragma unroll
-    for (int b0 = 0; b0 < 32; b0 += B) {
-      typename F::R raw[B];
+    for (int b = 0; b < 8; ++b)
+      if (b < nlive) raw[b] = F::load(vb + (size_t)(g + b) * D);
+#pragma unroll 1
+    for (int b0 = 0; b0 < nlive; b0 += 8) {
 #pragma unroll
-      for (int b = 0; b < B; ++b)
-        if (b0 + b < nlive) raw[b] = F::load(vb + (size_t)(g + b0 + b) * D);
+      for (int b = 0; b < 8; ++b)
+        if (b0 + 8 + b < nlive) nxt[b] = F::load(vb + (size_t)(g + b0 + 8 + b) * D);
 #pragma unroll
-      for (int b = 0; b < B; ++b) {
+      for (int b = 0; b < 8; ++b) {
         const int u = b0 + b;
         if (u < nlive) {
           float v[E];
           F::unpack(raw[b], v);
           if ((newR >> u) & 1u) {
-            if (cur >= 0) flush_sum<E>(vs, cur, acc, lane, D);
+            if (cur >= 0) flush();
             cur = __shfl_sync(0xffffffffu, code, u);
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] = 0.f;
           }
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] += v[e];
+          for (int e = 0; e < E; ++e) acc[b & 1][e] += v[e];
         }
       }
+#pragma unroll
+      for (int b = 0; b < 8; ++b) raw[b] = nxt[b];
     }
   }
-  if (cur >= 0) flush_sum<E>(vs, cur, acc, lane, D);
+  if (cur >= 0) flush();
 }
 
 // Parents hold their whole cluster: add the children's sums (keys that moved)
