@@ -371,6 +371,9 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
 // columns, B the bf16 triple (hi, mid, lo) whose sum is -|p|^2 / 2 to within
 // 2^-24 of it, so TMEM receives T directly.
 constexpr int kStageAtoms = 8;
+// Thread of each warpgroup that issues the parent MMAs (thread 0 issues the
+// child MMAs and the K copies), so that the two issue streams overlap.
+constexpr int kParentIssuer = 32;
 
 template <int D>
 struct WgSmem {
@@ -566,10 +569,13 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       if (*sAbort) break;
     }
     const int first = s0 + g;
-    // prologue: K of the first two tiles, parent MMA of the first
+    // prologue: K of the first two tiles (thread 0), parent MMA of the first
+    // (the parent issuer)
     if (wt == 0 && first < s1) {
       issue_k(first, it & 1);
       if (first + nwg < s1) issue_k(first + nwg, (it + 1) & 1);
+    }
+    if (wt == kParentIssuer && first < s1) {
       if (tc::mbar_wait(&bar_k[it & 1], (it >> 1) & 1)) {
         tc::tc_fence_after();
         issue_parents(it & 1);
@@ -581,7 +587,8 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       const int slot = it & 1;
       const uint32_t tP = tmem_g + (uint32_t)slot * 64u;  // parent, then child scores of this tile
       bool bad = false;
-      if (wt == 0) bad = kerr || !tc::mbar_wait(bar_p, ph_p);
+      if (wt == 0) bad = !tc::mbar_wait(bar_p, ph_p);
+      if (wt == kParentIssuer) bad = kerr;
       ph_p ^= 1;
       tc::tc_fence_before();
       if (wg_bar_or(barid, bad)) {  // parent scores of tile t in TMEM
@@ -593,7 +600,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       // next tile's parent MMA into the other half (its scores there were read
       // before the barrier above), so that it overlaps this tile's epilogue
       auto next_parents = [&]() {
-        if (wt == 0 && t + nwg < s1) {
+        if (wt == kParentIssuer && t + nwg < s1) {
           if (tc::mbar_wait(&bar_k[slot ^ 1], ((it + 1) >> 1) & 1)) {
             tc::tc_fence_after();
             issue_parents(slot ^ 1);
@@ -686,6 +693,9 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
           }
           tc::fence_proxy_async_smem();
           wg_bar(barid);  // staging written
+          // the next tile's parent MMA, issued by another thread while thread 0
+          // issues this round's child MMA
+          if (r0 == 0) next_parents();
           if (wt == 0) {
             tc::tc_fence_after();
             const uint32_t idescC = tc::idesc_bf16(kKeys, 8 * nat, 0, 0);
@@ -697,9 +707,6 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
               tc::mma_bf16(tP, ad, bd, idescC, k > 0);
             }
             tc::mma_commit(bar_c);
-            // the next tile's parent MMA queues behind this child MMA; its issue
-            // overlaps the child MMA instead of delaying the staging barrier
-            if (r0 == 0) next_parents();
             if (!tc::mbar_wait(bar_c, ph_c)) atomicOr(a.err, kErrTimeout);
             // last round: the K slot is read by nothing else now
             if (r0 + kStageAtoms >= np && t + 2 * nwg < s1) issue_k(t + 2 * nwg, slot);
