@@ -773,26 +773,33 @@ __global__ void __launch_bounds__(256) codebook_prep_kernel(const bf16* __restri
                                                             float* __restrict__ norms, int H, int M0,
                                                             int C) {
   constexpr int KH = D / 64;
+  constexpr int CH = D / 8;  // 16-byte chunks per code: one thread each
   const int Mt = M0 * (1 + C);
-  const long long total = (long long)H * Mt;
-  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+  const long long total = (long long)H * Mt * CH;
+  const long long span = (total + 31) / 32 * 32;  // whole warps, so the shuffles see every lane
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < span;
        u += (long long)gridDim.x * blockDim.x) {
-    const int code = (int)(u % Mt);
-    const long long h = u / Mt;
-    const bf16* src = code < M0 ? parents + ((size_t)h * M0 + code) * D
-                                : children + ((size_t)h * M0 * C + (code - M0)) * D;
-    float nrm = 0.f;
-    const int r = code & 7;
+    const bool live = u < total;
+    const int chunk = (int)(u % CH);
+    const long long hc = u / CH;  // h * Mt + code
+    const int code = (int)(hc % Mt);
+    const long long h = hc / Mt;
+    float v[8];
 #pragma unroll
-    for (int chunk = 0; chunk < D / 8; ++chunk) {
-      float v[8];
+    for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    if (live) {
+      const bf16* src = code < M0 ? parents + ((size_t)h * M0 + code) * D
+                                  : children + ((size_t)h * M0 * C + (code - M0)) * D;
       load8(src + chunk * 8, v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) nrm = fmaf(v[e], v[e], nrm);
-      const int kh = chunk >> 3, c = chunk & 7;
+      const int r = code & 7, kh = chunk >> 3, c = chunk & 7;
       store8(cw + (((size_t)h * (Mt / 8) + (code >> 3)) * KH + kh) * 512 + r * 64 + ((c ^ r) * 8), v);
     }
-    norms[u] = nrm;
+    float nrm = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) nrm = fmaf(v[e], v[e], nrm);
+#pragma unroll
+    for (int o = CH / 2; o >= 1; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
+    if (live && chunk == 0) norms[hc] = nrm;
   }
 }
 
@@ -865,8 +872,8 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
                              LaunchLog& log) {
   bf16* cw = static_cast<bf16*>(ws);
   float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
-  const long long work = (long long)s.H * s.Mt();
-  const int pblocks = (int)std::max<long long>(1, std::min<long long>((work + 255) / 256, num_sms() * 4));
+  const long long work = (long long)s.H * s.Mt() * (s.d / 8);
+  const int pblocks = (int)std::max<long long>(1, std::min<long long>((work + 255) / 256, num_sms() * 8));
   if (s.d == 64)
     codebook_prep_kernel<64><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
                                                       s.H, s.M0, s.C);
