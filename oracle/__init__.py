@@ -71,6 +71,8 @@ class Oracle:
         lib.avq_oracle_attention.argtypes = ([ctypes.c_int] * 8 + [ctypes.c_double, _D, _D, _D, _D, _D,
                                              _I32, _I32, ctypes.c_int, _D, _I32, _D])
         lib.avq_oracle_attention.restype = None
+        lib.avq_oracle_attention_tiled.argtypes = lib.avq_oracle_attention.argtypes + [ctypes.c_int]
+        lib.avq_oracle_attention_tiled.restype = None
         lib.avq_oracle_num_threads.restype = ctypes.c_int
         self.lib = lib
 
@@ -110,10 +112,12 @@ class Oracle:
 
     # ---- Algorithm 2 ---------------------------------------------------
     def attention(self, Q, parents, children, vsum, counts, P: int, block: int, scale: float,
-                  sel=None, blocks=None):
+                  sel=None, blocks=None, tile: int = 0):
         """Q [B,H,N,d]; vsum [B,H,Mt,d]; counts [B,H,Mt].  `sel` [B,H,nblk,P]
         overrides the top-P selection; `blocks` (list of (bh, block)) limits the
-        work to those query blocks (other rows of O stay NaN).
+        work to those query blocks (other rows of O stay NaN).  `tile` > 0 uses
+        the tiled importance with the count-extrapolated denominator (Sec. B,
+        Eqs. 13-14) over parent tiles of that many codes.
         Returns O [B,H,N,d], sel [B,H,nblk,P] int32, importance [B,H,nblk,M0]."""
         Q, parents, children, vsum = map(_f64, (Q, parents, children, vsum))
         counts = _f64(counts)
@@ -132,11 +136,11 @@ class Oracle:
         if blocks is not None:
             blk = np.ascontiguousarray(np.asarray(blocks, dtype=np.int32).reshape(-1, 2))
             nlist = blk.shape[0]
-        self.lib.avq_oracle_attention(B * H, H, N, d, M0, C, P, block, float(scale),
-                                      _p(Q, _D), _p(parents, _D), _p(children, _D),
-                                      _p(vsum, _D), _p(counts, _D), _p(sel_in, _I32),
-                                      _p(blk, _I32), nlist, _p(O, _D), _p(sel_out, _I32),
-                                      _p(imp, _D))
+        self.lib.avq_oracle_attention_tiled(B * H, H, N, d, M0, C, P, block, float(scale),
+                                            _p(Q, _D), _p(parents, _D), _p(children, _D),
+                                            _p(vsum, _D), _p(counts, _D), _p(sel_in, _I32),
+                                            _p(blk, _I32), nlist, _p(O, _D), _p(sel_out, _I32),
+                                            _p(imp, _D), int(tile))
         return O, sel_out, imp
 
 

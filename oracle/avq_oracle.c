@@ -207,7 +207,7 @@ static void attend_block(int d, int M0, int C, int P, double scale,
                          const double* par_h, const double* ch_h,
                          const double* vs, const double* ns,
                          const int32_t* sel_in, double* O, int32_t* sel_out,
-                         double* imp_out) {
+                         double* imp_out, int tile) {
   const int nI = i1 - i0;
   double* s = (double*)malloc(sizeof(double) * (size_t)nI * M0);
   double* A = (double*)malloc(sizeof(double) * (size_t)nI * M0);
@@ -238,10 +238,37 @@ static void attend_block(int d, int M0, int C, int P, double scale,
       z[r] += a * ns[j];
     }
   }
-  /* w_j = sum_i A_ij n_j / z_i  (Eq. 7) */
-  for (int j = 0; j < M0; ++j) {
-    w[j] = 0.0;
-    for (int r = 0; r < nI; ++r) w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];
+  if (tile <= 0 || tile >= M0) {
+    /* w_j = sum_i A_ij n_j / z_i  (Eq. 7) */
+    for (int j = 0; j < M0; ++j) {
+      w[j] = 0.0;
+      for (int r = 0; r < nI; ++r) w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];
+    }
+  } else {
+    /* Sec. B: the parents are visited in tiles of `tile` codes in index order;
+     * the importance of the codes in tile J uses the count-extrapolated
+     * denominator Z~_i(J) = (N / N_seen(J)) sum_{t <= J} Z_i(t)  (Eq. 13),
+     * w_j = sum_i A_ij n_j / Z~_i(J)  (Eq. 14).  N is the number of keys, the
+     * sum of the parents' counts; N_seen(J) the keys of parents in tiles <= J.
+     * A common reference max cancels in A / Z~. */
+    double ntot = 0.0;
+    for (int j = 0; j < M0; ++j) ntot += ns[j];
+    double* zpart = (double*)calloc((size_t)nI, sizeof(double));
+    double nseen = 0.0;
+    for (int j0 = 0; j0 < M0; j0 += tile) {
+      const int j1 = j0 + tile < M0 ? j0 + tile : M0;
+      for (int j = j0; j < j1; ++j) {
+        nseen += ns[j];
+        for (int r = 0; r < nI; ++r) zpart[r] += A[(size_t)r * M0 + j] * ns[j];
+      }
+      for (int j = j0; j < j1; ++j) {
+        w[j] = 0.0;
+        if (nseen <= 0.0) continue; /* every parent seen so far is empty: n_j = 0 */
+        for (int r = 0; r < nI; ++r)
+          if (zpart[r] > 0.0) w[j] += A[(size_t)r * M0 + j] * ns[j] / (ntot / nseen * zpart[r]);
+      }
+    }
+    free(zpart);
   }
   if (imp_out) memcpy(imp_out, w, sizeof(double) * (size_t)M0);
   /* S = top-P(w), or the caller's selection */
@@ -297,12 +324,17 @@ static void attend_block(int d, int M0, int C, int P, double scale,
  * are passed as doubles.  `sel_in` (nullable) overrides the top-P selection:
  * [BH][nblk][P].  O rows of unlisted blocks are left untouched.
  */
-void avq_oracle_attention(int BH, int H, int N, int d, int M0, int C, int P, int block,
-                          double scale, const double* Q,
-                          const double* parents, const double* children,
-                          const double* vsum, const double* counts,
-                          const int32_t* sel_in, const int32_t* blocks, int nlist,
-                          double* O, int32_t* sel_out, double* imp_out) {
+/*
+ * Stage 2 over all (or the listed) query blocks.  tile > 0 (and < M0) selects
+ * the tiled importance with the count-extrapolated denominator of Sec. B
+ * (Eqs. 13-14); everything else is unchanged by it.
+ */
+void avq_oracle_attention_tiled(int BH, int H, int N, int d, int M0, int C, int P, int block,
+                                double scale, const double* Q,
+                                const double* parents, const double* children,
+                                const double* vsum, const double* counts,
+                                const int32_t* sel_in, const int32_t* blocks, int nlist,
+                                double* O, int32_t* sel_out, double* imp_out, int tile) {
   const int Mt = M0 * (1 + C);
   const int nblk = (N + block - 1) / block;
   const int total = blocks ? nlist : BH * nblk;
@@ -318,8 +350,19 @@ void avq_oracle_attention(int BH, int H, int N, int d, int M0, int C, int P, int
                  parents + (size_t)h * M0 * d, children + (size_t)h * M0 * C * d,
                  vsum + (size_t)bh * Mt * d, counts + (size_t)bh * Mt,
                  sel_in ? sel_in + sb * P : NULL, O + (size_t)bh * N * d,
-                 sel_out ? sel_out + sb * P : NULL, imp_out ? imp_out + sb * M0 : NULL);
+                 sel_out ? sel_out + sb * P : NULL, imp_out ? imp_out + sb * M0 : NULL, tile);
   }
+}
+
+/* Stage 2 with the exact importance denominator (Eq. 7). */
+void avq_oracle_attention(int BH, int H, int N, int d, int M0, int C, int P, int block,
+                          double scale, const double* Q,
+                          const double* parents, const double* children,
+                          const double* vsum, const double* counts,
+                          const int32_t* sel_in, const int32_t* blocks, int nlist,
+                          double* O, int32_t* sel_out, double* imp_out) {
+  avq_oracle_attention_tiled(BH, H, N, d, M0, C, P, block, scale, Q, parents, children, vsum, counts,
+                             sel_in, blocks, nlist, O, sel_out, imp_out, 0);
 }
 
 int avq_oracle_num_threads(void) {

@@ -352,7 +352,44 @@ def pin_counting(orc):
     assert counts.shape[-1] == synth.m_total(inp["M0"], inp["C"])
 
 
+def pin_tiled_importance(orc):
+    """Tiled importance with the count-extrapolated denominator (Sec. B,
+    Eqs. 13-14), parents in tiles of `tile` codes:
+    - over the first tile Z~ = Z(0) N / N_seen(0), so that tile's importances
+      sum to |I| N_seen(0) / N whatever the logits;
+    - at the last tile N_seen = N and Z~ is the exact denominator, so the last
+      tile's importances equal Eq. 7's;
+    - with constant logits (Q = 0) every A is 1 and Z~ = N for every tile, so
+      all importances equal Eq. 7's;
+    - the selection is the top-P of the tiled importances."""
+    for mk, tile in ((case_regions, 8), (case_wide, 8), (case_wide, 16)):
+        inp = mk()
+        assign, vsum, counts, _ = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+        M0, P, blk, N = inp["M0"], inp["P"], inp["block"], inp["N"]
+        args = (inp["parents"], inp["children"], vsum, counts, P, blk, inp["scale"])
+        _, sel_t, imp_t = orc.attention(inp["Q"], *args, tile=tile)
+        _, _, imp_x = orc.attention(inp["Q"], *args)
+        nblk = imp_t.shape[2]
+        sizes = np.array([min(blk, N - b * blk) for b in range(nblk)], dtype=np.float64)
+        nseen0 = counts[..., :tile].sum(-1).astype(np.float64)     # [B,H]
+        ntot = counts[..., :M0].sum(-1).astype(np.float64)         # [B,H] == N
+        assert np.all(ntot == N)
+        want = sizes[None, None, :] * (nseen0 / ntot)[..., None]
+        assert np.allclose(imp_t[..., :tile].sum(-1), want, rtol=1e-11, atol=1e-300)
+        last = (M0 - 1) // tile * tile
+        assert _rel(imp_t[..., last:], imp_x[..., last:]) < 1e-12
+        for b in range(imp_t.shape[0]):
+            for h in range(imp_t.shape[1]):
+                for k in range(nblk):
+                    assert np.array_equal(sel_t[b, h, k], _topp_ref(imp_t[b, h, k], P))
+        Q0 = np.zeros(tuple(inp["Q"].shape), dtype=np.float64)
+        _, _, imp_t0 = orc.attention(Q0, *args, tile=tile)
+        _, _, imp_x0 = orc.attention(Q0, *args)
+        assert _rel(imp_t0, imp_x0) < 1e-12
+        assert not np.allclose(imp_t, imp_x, rtol=1e-6)  # the approximation is exercised
+
+
 ALL_PINS = [pin_hand_worked, pin_assign_brute, pin_aggregate, pin_representative,
             pin_rescale_exercised, pin_flat_p0, pin_exact_codebook, pin_importance, pin_topp,
             pin_relabel, pin_key_permutation, pin_keys_on_codewords, pin_strict_ties,
-            pin_masking, pin_counting]
+            pin_masking, pin_counting, pin_tiled_importance]

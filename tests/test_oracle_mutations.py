@@ -35,6 +35,12 @@ MUTANTS = [
     ("parent-mean-wrong-divisor", "sp /= C;", "sp /= (C + 1);"),
     ("z-missing-count", "z[r] += a * ns[j];", "z[r] += a;"),
     ("child-z-missing-count", "z[r] += dA * nc[c];", "z[r] += dA;"),
+    ("tiled-seen-codes-not-keys", "nseen += ns[j];", "nseen += 1.0;"),
+    ("tiled-extrapolation-inverted", "ns[j] / (ntot / nseen * zpart[r]);",
+     "ns[j] / (nseen / ntot * zpart[r]);"),
+    ("tiled-exact-denominator", "ns[j] / (ntot / nseen * zpart[r]);", "ns[j] / z[r];"),
+    ("tiled-partial-z-unweighted", "zpart[r] += A[(size_t)r * M0 + j] * ns[j];",
+     "zpart[r] += A[(size_t)r * M0 + j];"),
 ]
 
 
