@@ -28,6 +28,7 @@ AVQ_OK, AVQ_ERR_INVALID_ARG, AVQ_ERR_UNSUPPORTED, AVQ_ERR_CUDA = 0, 1, 2, 3
 AVQ_ERR_DEVICE, AVQ_ERR_TIMEOUT, AVQ_ERR_WORKSPACE = 4, 5, 6
 AVQ_F32, AVQ_BF16 = 0, 1
 AVQ_PATH_AUTO, AVQ_PATH_SIMT, AVQ_PATH_TC = 0, 1, 2
+AVQ_DENOM_AUTO, AVQ_DENOM_TWO_PASS, AVQ_DENOM_EXTRAPOLATED = 0, 1, 2
 
 
 class AVQError(RuntimeError):
@@ -147,7 +148,7 @@ def _dims(Q_like: torch.Tensor, parents: torch.Tensor, children) -> avq_dims:
 def avq_workspace_size(dims: avq_dims, dtype: int, deterministic=False, two_pass=False,
                        P: int = 0, block: int = 128) -> int:
     return int(lib().avq_workspace_size(ctypes.byref(dims), int(dtype), int(bool(deterministic)),
-                                        int(bool(two_pass)), int(P), int(block)))
+                                        int(two_pass), int(P), int(block)))
 
 
 def workspace(dims: avq_dims, dtype: int, device, deterministic=False, two_pass=False, P=0,
@@ -218,7 +219,8 @@ def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, 
                   two_pass=False, O=None, sel=None, importance=False, ws=None, stream=None):
     """Stage 2.  Returns (O [B,H,N,d], sel [B,H,nblk,P] int32, importance
     [B,H,nblk,M0] fp32 or None).  `importance=True` asks for the importance
-    output; a tensor is written in place."""
+    output; a tensor is written in place.  `two_pass`: AVQ_DENOM_AUTO (or
+    False), AVQ_DENOM_TWO_PASS (or True) or AVQ_DENOM_EXTRAPOLATED."""
     dims = _dims(Q, parents, children)
     dt = _dtype_code(Q)
     B, H, N, d = Q.shape
@@ -240,7 +242,7 @@ def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, 
     wp, wn = _ws_ptr(ws)
     _check(lib().avq_attention(ctypes.byref(dims), dt, _ptr(Q), _ptr(parents), _ptr(children),
                                _ptr(vsum), _ptr(counts), int(P), int(block), float(scale),
-                               int(bool(two_pass)), _ptr(O), _ptr(sel) if P > 0 else None,
+                               int(two_pass), _ptr(O), _ptr(sel) if P > 0 else None,
                                _ptr(imp), wp, wn, _stream(stream)))
     return O, sel, imp
 

@@ -219,7 +219,12 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
 
   float m = NEG_INF, z = 0.f;
   const int nT = (M0 + kTile - 1) / kTile;
-  const int sweeps = (a.two_pass || nT > 1) ? 2 : 1;
+  // two_pass == 2: one sweep over the parent tiles, the importance of each
+  // tile from the count-extrapolated denominator (Sec. B, Eqs. 13-14)
+  const bool extrap = a.two_pass == 2;
+  const int sweeps = extrap ? 1 : (a.two_pass || nT > 1) ? 2 : 1;
+  const float ntot = (float)a.N;  // keys of the head: the sum of the parents' counts
+  float nseen = 0.f;              // keys of the parents in the tiles swept so far
   bool x_started = false;
   bool q_ready = false;
 
@@ -284,7 +289,29 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
         const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
         if (!last || sweeps == 1) {
           const float mn = fmaxf(m, tmax);
-          if (mn != NEG_INF) {
+          if (extrap) {
+            // x holds the earlier tiles' A V-bar relative to the old max: rescale
+            // it (TMEM) to the new one; the previous value MMA has completed
+            const bool grow = x_started && mn != m;
+            if (__syncthreads_or(grow)) {
+              tc::tc_fence_after();
+              const float f = grow ? tc::ex2(m - mn) : 1.f;
+              for (int g = 0; g < D; g += 16) {
+                uint32_t xr[16];
+                tc::tmem_ld16(tX + lane_off + g, xr);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) xr[e] = __float_as_uint(__uint_as_float(xr[e]) * f);
+                tc::tmem_st16(tX + lane_off + g, xr);
+              }
+              tc::tmem_wait_st();
+            }
+            for (int j = 0; j < 64; ++j) nseen += sNF[j];
+          }
+          if (mn == NEG_INF) {  // every parent seen so far is empty: A = 0
+#pragma unroll
+            for (int e = 0; e < 64; ++e) r[e] = 0u;
+          } else {
             float zp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 64; e += 4) {
@@ -307,7 +334,8 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
         }
         if (last) {
           // probabilities as bf16, importance column sums of A / z in fp32
-          const float rz = valid ? 1.f / z : 0.f;
+          // (A / Z~ with Z~ = z N / N_seen when extrapolating)
+          const float rz = !valid || !(z > 0.f) ? 0.f : extrap ? nseen / (ntot * z) : 1.f / z;
 #pragma unroll
           for (int q = 0; q < 8; ++q) store_chunk8(sPR, tid, q * 8, reinterpret_cast<const float*>(r) + q * 8);
           float v[32];

@@ -251,6 +251,8 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, c
     return fail(AVQ_ERR_UNSUPPORTED, "block must be 64 or 128 (got %d)", block);
   if (!(scale > 0.f) || !isfinite(scale))
     return fail(AVQ_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (two_pass < 0 || two_pass > 2)
+    return fail(AVQ_ERR_INVALID_ARG, "two_pass must be 0, 1 or 2 (got %d)", two_pass);
   AVQ_REQUIRE_PTR(Q, "Q");
   AVQ_REQUIRE_PTR(parents, "parents");
   if (s.C > 0) AVQ_REQUIRE_PTR(children, "children");
@@ -264,6 +266,10 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, c
   if (t_path == AVQ_PATH_TC && !tc_ok)
     return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core attention kernel for this shape/dtype");
   const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
+  // the extrapolated denominator differs from the exact one only over several
+  // parent tiles, which only the tensor-core kernel sweeps
+  if (two_pass == 2 && s.M0 > 64 && !use_tc)
+    return fail(AVQ_ERR_UNSUPPORTED, "the extrapolated denominator needs the tensor-core kernel");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   LaunchLog log{};
   cudaError_t e;

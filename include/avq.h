@@ -71,6 +71,13 @@ typedef struct {
  * kernels and makes calls they do not cover return AVQ_ERR_UNSUPPORTED. */
 typedef enum { AVQ_PATH_AUTO = 0, AVQ_PATH_SIMT = 1, AVQ_PATH_TC = 2 } avq_path;
 
+/* Values of avq_attention's `two_pass` argument (importance denominator). */
+typedef enum {
+  AVQ_DENOM_AUTO = 0,
+  AVQ_DENOM_TWO_PASS = 1,
+  AVQ_DENOM_EXTRAPOLATED = 2
+} avq_denominator;
+
 /*
  * avq_quantize -- full-tree key quantisation and aggregation
  * (Sec. 4.2 "Vector Quantization for (A)VQ-Attention", Algorithm 1, Eq. 3).
@@ -153,10 +160,20 @@ avq_status avq_quantize_noalloc(const avq_dims* dims, avq_dtype dtype,
  * avq_quantize; vsum, counts as produced by avq_quantize.
  * P in [0, M0]; block in {64, 128}; scale > 0 (1/sqrt(d) for standard
  * attention; the paper omits it for clarity, Sec. 3.1).
- * two_pass != 0 selects the exact two-pass denominator: a first pass over
- * parent tiles finds the row max and z, a second recomputes the logits for
- * x and the importance.  Results equal the single-pass ones; it serves parent
- * codebooks too large to hold on chip.
+ * two_pass selects how the importance denominator is formed when the parents
+ * span several tiles of 64 codes (M0 > 64):
+ *   AVQ_DENOM_AUTO (0): exact; one pass when the parents fit one tile, else
+ *     the two-pass form below.
+ *   AVQ_DENOM_TWO_PASS (1): exact two-pass denominator: a first pass over
+ *     parent tiles finds the row max and z, a second recomputes the logits
+ *     for x and the importance.  Results equal the single-pass ones.
+ *   AVQ_DENOM_EXTRAPOLATED (2): one pass over the parent tiles in index order;
+ *     the importance of the parents of tile J uses the count-extrapolated
+ *     denominator Z~(J) = (N / N_seen(J)) * sum_{t <= J} Z(t) (Sec. B,
+ *     Eqs. 13-14), so the selection may differ from the exact one; x, z and
+ *     O are computed exactly for whatever is selected.  Needs the
+ *     tensor-core kernel when M0 > 64 (else AVQ_ERR_UNSUPPORTED).
+ * Any other value is AVQ_ERR_INVALID_ARG.
  * Outputs (device): O [B,H,N,d] of `dtype`; sel [B,H,nblk,P] int32, the
  * selected parents in descending importance (nblk = ceil(N/block)), may be
  * NULL when P == 0; importance [B,H,nblk,M0] fp32 or NULL.

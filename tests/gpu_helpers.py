@@ -44,9 +44,11 @@ def gpu_forward(inp, P=None, block=None, two_pass=None, path=avq.AVQ_PATH_AUTO,
                 O=O.cpu(), sel=sel.cpu().numpy(), imp=imp.cpu().numpy(), kernels=(k1 + " " + k2))
 
 
-def check_forward(inp, res, P=None, block=None, blocks=None):
+def check_forward(inp, res, P=None, block=None, blocks=None, tile=0):
     """Full parity of one forward against the oracle; `blocks` limits the
-    attention check to a list of (bh, block) pairs.  Returns diagnostics."""
+    attention check to a list of (bh, block) pairs; `tile` > 0 compares the
+    importance and selection with the oracle's tiled, count-extrapolated
+    importance over parent tiles of that size.  Returns diagnostics."""
     orc = oracle.default()
     P = inp["P"] if P is None else P
     block = inp["block"] if block is None else block
@@ -58,7 +60,7 @@ def check_forward(inp, res, P=None, block=None, blocks=None):
     parity.check_stats(res["vsum"], res["counts"], ref_vs, ref_n, abs_vs)
     # importance and selection against the oracle on the same statistics
     _, o_sel, o_imp = orc.attention(inp["Q"], inp["parents"], inp["children"], ref_vs, ref_n, P,
-                                    block, inp["scale"], blocks=blocks)
+                                    block, inp["scale"], blocks=blocks, tile=tile)
     B, H = inp["B"], inp["H"]
     nblk = res["sel"].shape[2]
     mask_blk = np.ones((B, H, nblk), dtype=bool)

@@ -56,10 +56,10 @@ def _q(dims, K=0x1000, V=0x2000, par=0x3000, ch=0x4000, a=0x5000, vs=0x6000, n=0
 
 
 def _a(dims, P=4, block=128, scale=0.125, Q=0x1000, par=0x3000, ch=0x4000, vs=0x6000, n=0x7000,
-       O=0x8000, sel=0x9000, imp=None, dt=avq.AVQ_BF16):
+       O=0x8000, sel=0x9000, imp=None, dt=avq.AVQ_BF16, two_pass=0):
     L = avq.lib()
-    return L.avq_attention(ctypes.byref(dims), dt, Q, par, ch, vs, n, P, block, scale, 0, O, sel,
-                           imp, None, 0, None)
+    return L.avq_attention(ctypes.byref(dims), dt, Q, par, ch, vs, n, P, block, scale, two_pass, O,
+                           sel, imp, None, 0, None)
 
 
 def test_host_validation_rejects_before_launch():
@@ -125,3 +125,18 @@ def test_noalloc_quantize_host_checks():
     st = L.avq_quantize_noalloc(None, avq.AVQ_BF16, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000,
                                 0x6000, 0x7000, None)
     assert st == 1
+
+
+def test_denominator_modes_host_checks():
+    """two_pass outside {0, 1, 2} is an argument error; the extrapolated
+    denominator over several parent tiles needs the tensor-core kernel."""
+    E = avq
+    big = avq.avq_dims(1, 2, 1024, 64, 128, 8)
+    assert _a(big, two_pass=3) == E.AVQ_ERR_INVALID_ARG
+    assert _a(big, two_pass=-1) == E.AVQ_ERR_INVALID_ARG
+    old = avq.avq_set_path(avq.AVQ_PATH_SIMT)
+    try:
+        assert _a(big, two_pass=E.AVQ_DENOM_EXTRAPOLATED) == E.AVQ_ERR_UNSUPPORTED
+        assert "tensor-core" in avq.last_error()
+    finally:
+        avq.avq_set_path(old)

@@ -155,6 +155,19 @@ def test_vit_p_and_block_variants(inputs, P, block):
         gh.check_forward(inp, res, P=P, block=block)
 
 
+def test_extrapolated_denominator(inputs):
+    """Sec. B, Eqs. 13-14 on the tensor-core kernel: importance and selection
+    against the oracle's tiled importance (tiles of 64 parents), O against the
+    oracle rerun on the GPU's selection; the selection differs from the exact
+    one somewhere, so the approximation is exercised."""
+    inp = inputs("largecb_small")
+    res = gh.gpu_forward(inp, two_pass=avq.AVQ_DENOM_EXTRAPOLATED, path=avq.AVQ_PATH_TC)
+    assert "attention_tc " in res["kernels"] + " "
+    gh.check_forward(inp, res, tile=64)
+    exact = gh.gpu_forward(inp, two_pass=avq.AVQ_DENOM_TWO_PASS, path=avq.AVQ_PATH_TC)
+    assert not np.array_equal(res["imp"], exact["imp"])
+
+
 def test_two_pass_equals_single_pass(inputs):
     inp = inputs("largecb_small")
     a = gh.gpu_forward(inp, two_pass=True)
