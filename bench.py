@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=None)
+    ap.add_argument("--denominator", default=None, choices=["auto", "two_pass", "extrapolated"],
+                    help="importance denominator for parent codebooks over several tiles "
+                         "(default: the workload's own setting)")
     ap.add_argument("--profile", action="store_true",
                     help="for profiler runs: no clock soak, no end-to-end leg, no CPU baseline")
     return ap.parse_args()
@@ -221,7 +224,7 @@ def workload_config(name, cfg):
     out = {"workload": name}
     out.update({k: cfg[k] for k in keys})
     out["order"] = cfg.get("order", "natural")
-    out["two_pass"] = bool(cfg.get("two_pass", False))
+    out["two_pass"] = int(cfg.get("two_pass", False))
     return out
 
 
@@ -243,7 +246,7 @@ def run_avq(args, cfg, inp):
     dev = torch.device("cuda", local)
     B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
     P, block = cfg["P"], cfg["block"]
-    two_pass = bool(cfg.get("two_pass", False))
+    two_pass = int(cfg.get("two_pass", False))
     Q, K, V = (inp[k].to(dev) for k in ("Q", "K", "V"))
     par = inp["parents"].to(dev)
     ch = inp["children"].to(dev) if cfg["C"] > 0 else None
@@ -391,6 +394,8 @@ def main():
     cfg = synth.get_config(args.config) if args.config in synth.CONFIGS else None
     if cfg is None:
         raise SystemExit(f"unknown config {args.config}")
+    if args.denominator is not None:
+        cfg["two_pass"] = {"auto": 0, "two_pass": 1, "extrapolated": 2}[args.denominator]
     rank = int(os.environ.get("RANK", "0"))
     seed = rank_seed(args.seed if args.seed is not None else synth.CONFIG_SEEDS.get(args.config, 1000), rank)
     if args.impl == "reference":

@@ -73,6 +73,8 @@ class Oracle:
         lib.avq_oracle_attention.restype = None
         lib.avq_oracle_attention_tiled.argtypes = lib.avq_oracle_attention.argtypes + [ctypes.c_int]
         lib.avq_oracle_attention_tiled.restype = None
+        lib.avq_oracle_codebook_update.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_D] * 8
+        lib.avq_oracle_codebook_update.restype = None
         lib.avq_oracle_num_threads.restype = ctypes.c_int
         self.lib = lib
 
@@ -142,6 +144,25 @@ class Oracle:
                                             _p(blk, _I32), nlist, _p(O, _D), _p(sel_out, _I32),
                                             _p(imp, _D), int(tile))
         return O, sel_out, imp
+
+
+    # ---- Sec. A: codebook update -----------------------------------------
+    def codebook_update(self, ksum, counts, S, Nst, parents, children, lam: float):
+        """ksum [B,H,Mt,d], counts [B,H,Mt]: Eq. 3 statistics of the keys;
+        S [H,Mt,d], Nst [H,Mt]: EMA state; parents [H,M0,d], children
+        [H,M0,C,d]: current codebook.  Returns (S', N', parents', children')."""
+        ksum, counts, parents, children = map(_f64, (ksum, counts, parents, children))
+        S = _f64(S).copy()
+        Nst = _f64(Nst).copy()
+        B, H, Mt, d = ksum.shape
+        M0 = parents.shape[1]
+        C = children.shape[2]
+        po = np.empty_like(parents)
+        co = np.empty_like(children)
+        self.lib.avq_oracle_codebook_update(B, H, d, M0, C, float(lam), _p(ksum, _D), _p(counts, _D),
+                                            _p(S, _D), _p(Nst, _D), _p(parents, _D),
+                                            _p(children, _D), _p(po, _D), _p(co, _D))
+        return S, Nst, po, co
 
 
 _default = None

@@ -373,3 +373,79 @@ int avq_oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Codebook update of Sec. A ("Codeword Clustering During Training").
+ * EMA statistics (Eq. 11), one set per head over the keys of every batch
+ * entry:  S_x <- lambda S_x + (1 - lambda) sum_k k,  N_x <- lambda N_x +
+ * (1 - lambda) |{k}|, over the keys quantised to code x, with the statistics
+ * of Eq. 3 (a parent counts its whole cluster, a child the keys that moved to
+ * it); ksum and counts are those statistics computed on the keys.
+ * Parents take their unconstrained means C_p = S_p / N_p.  Children take the
+ * mass-weighted projection of their means M_c = S_c / N_c onto the constraint
+ * sum_c C_pc = C C_p (Eq. 12):  delta = sum_c M_c - C C_p,
+ * sigma = sum_c 1 / N_c,  C_pc = M_c - delta / (N_c sigma).
+ * Readings where the pages are silent:
+ *   - a code with N_x = 0 after the update has no mean: it keeps its current
+ *     position (parents_in / children_in) in place of M_x;
+ *   - such massless children do not move; delta is spread over the children
+ *     with N_c > 0 only (sigma over those); if no child has mass, all C
+ *     children shift by -delta / C.
+ * Layouts: ksum [B][H][Mt][d], counts [B][H][Mt]; S [H][Mt][d], Nst [H][Mt]
+ * (updated in place); parents [H][M0][d], children [H][M0][C][d].
+ */
+void avq_oracle_codebook_update(int B, int H, int d, int M0, int C, double lambda,
+                                const double* ksum, const double* counts, double* S, double* Nst,
+                                const double* parents_in, const double* children_in,
+                                double* parents_out, double* children_out) {
+  const int Mt = M0 * (1 + C);
+  /* Eq. 11 */
+  for (int h = 0; h < H; ++h)
+    for (int x = 0; x < Mt; ++x) {
+      double n = 0.0;
+      for (int b = 0; b < B; ++b) n += counts[((size_t)b * H + h) * Mt + x];
+      Nst[(size_t)h * Mt + x] = lambda * Nst[(size_t)h * Mt + x] + (1.0 - lambda) * n;
+      for (int t = 0; t < d; ++t) {
+        double sk = 0.0;
+        for (int b = 0; b < B; ++b) sk += ksum[(((size_t)b * H + h) * Mt + x) * d + t];
+        double* sx = S + ((size_t)h * Mt + x) * d + t;
+        *sx = lambda * *sx + (1.0 - lambda) * sk;
+      }
+    }
+  double* Mc = (double*)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1) * d);
+  for (int h = 0; h < H; ++h)
+    for (int p = 0; p < M0; ++p) {
+      /* parent: unconstrained mean */
+      const double np = Nst[(size_t)h * Mt + p];
+      double* cp = parents_out + ((size_t)h * M0 + p) * d;
+      for (int t = 0; t < d; ++t)
+        cp[t] = np > 0.0 ? S[((size_t)h * Mt + p) * d + t] / np : parents_in[((size_t)h * M0 + p) * d + t];
+      if (C == 0) continue;
+      /* children: means, then the projection (Eq. 12) */
+      double sigma = 0.0;
+      int massive = 0;
+      for (int c = 0; c < C; ++c) {
+        const int x = M0 + p * C + c;
+        const double nc = Nst[(size_t)h * Mt + x];
+        for (int t = 0; t < d; ++t)
+          Mc[(size_t)c * d + t] = nc > 0.0 ? S[((size_t)h * Mt + x) * d + t] / nc
+                                           : children_in[(((size_t)h * M0 + p) * C + c) * d + t];
+        if (nc > 0.0) {
+          sigma += 1.0 / nc;
+          ++massive;
+        }
+      }
+      for (int t = 0; t < d; ++t) {
+        double delta = -C * cp[t];
+        for (int c = 0; c < C; ++c) delta += Mc[(size_t)c * d + t];
+        for (int c = 0; c < C; ++c) {
+          const double nc = Nst[(size_t)h * Mt + M0 + p * C + c];
+          double shift;
+          if (massive > 0) shift = nc > 0.0 ? delta / (nc * sigma) : 0.0;
+          else shift = delta / C;
+          children_out[(((size_t)h * M0 + p) * C + c) * d + t] = Mc[(size_t)c * d + t] - shift;
+        }
+      }
+    }
+  free(Mc);
+}

@@ -389,7 +389,90 @@ def pin_tiled_importance(orc):
         assert not np.allclose(imp_t, imp_x, rtol=1e-6)  # the approximation is exercised
 
 
+def _update_case(orc, lam, seed):
+    """Eq. 3 statistics of the keys of case_regions, a positive EMA prior."""
+    inp = case_regions()
+    assign, ksum, counts, _ = orc.quantize(inp["K"], inp["K"], inp["parents"], inp["children"])
+    rng = np.random.default_rng(seed)
+    H, M0, C, d = inp["H"], inp["M0"], inp["C"], inp["d"]
+    Mt = M0 * (1 + C)
+    S0 = rng.standard_normal((H, Mt, d))
+    N0 = rng.uniform(0.5, 4.0, (H, Mt))
+    out = orc.codebook_update(ksum, counts, S0, N0, inp["parents"], inp["children"], lam)
+    return inp, assign, ksum, counts, S0, N0, out
+
+
+def pin_codebook_update(orc):
+    """Sec. A: Eq. 11 EMA (lambda = 0 gives the step's own statistics, so the
+    parents are the plain means of their clusters, computed here from the keys
+    and codes; lambda = 1 keeps the state); Eq. 12 restores
+    sum_c C_pc = C C_p; and it is the minimiser of sum_c N_c |C_pc - M_c|^2
+    under that constraint (checked against a direct least-squares solve)."""
+    for lam in (0.0, 0.9, 1.0):
+        inp, assign, ksum, counts, S0, N0, (S1, N1, po, co) = _update_case(orc, lam, 21)
+        H, M0, C, d = inp["H"], inp["M0"], inp["C"], inp["d"]
+        # EMA
+        assert _rel(N1, lam * N0 + (1 - lam) * counts.sum(0)) < 1e-14
+        assert _rel(S1, lam * S0 + (1 - lam) * ksum.sum(0)) < 1e-14
+        if lam == 0.0:
+            K = np.asarray(inp["K"].float().numpy(), dtype=np.float64)
+            for h in range(H):
+                par = np.where(assign[0, h] < M0, assign[0, h], (assign[0, h] - M0) // C)
+                for p_ in range(M0):
+                    sel = par == p_
+                    if sel.any():
+                        assert _rel(po[h, p_], K[0, h][sel].mean(0)) < 1e-12
+        # constraint (Eq. 5 restored)
+        assert np.allclose(co.sum(2), C * po, rtol=0, atol=1e-10 * max(1.0, np.abs(po).max()))
+        # minimiser: eliminate the last child and solve the weighted least squares
+        for h in range(H):
+            for p_ in range(0, M0, 5):
+                xs = [M0 + p_ * C + c for c in range(C)]
+                n = N1[h, xs]
+                if not (n > 0).all():
+                    continue
+                M = S1[h, xs] / n[:, None]
+                # unknowns y_0..y_{C-2}; y_{C-1} = C C_p - sum y_c
+                A = np.zeros((C, C - 1))
+                bvec = np.zeros((C, d))
+                for c in range(C - 1):
+                    A[c, c] = math.sqrt(n[c])
+                    bvec[c] = math.sqrt(n[c]) * M[c]
+                A[C - 1, :] = -math.sqrt(n[C - 1])
+                bvec[C - 1] = math.sqrt(n[C - 1]) * (M[C - 1] - C * po[h, p_])
+                y, *_ = np.linalg.lstsq(A, bvec, rcond=None)
+                ref = np.vstack([y, C * po[h, p_] - y.sum(0)])
+                assert _rel(co[h, p_], ref) < 1e-9
+
+
+def pin_codebook_massless(orc):
+    """Readings for codes without mass: a massless child keeps its position
+    and the others absorb the displacement; with no massive child all C
+    children shift by the same amount; the constraint holds either way."""
+    rng = np.random.default_rng(22)
+    B, H, M0, C, d = 1, 1, 2, 4, 3
+    Mt = M0 * (1 + C)
+    par = rng.standard_normal((H, M0, d))
+    ch = rng.standard_normal((H, M0, C, d))
+    ksum = rng.standard_normal((B, H, Mt, d))
+    counts = np.zeros((B, H, Mt))
+    counts[0, 0, 0] = 5
+    counts[0, 0, M0 + 0] = 2
+    counts[0, 0, M0 + 1] = 3          # parent 0: children 2 and 3 massless
+    counts[0, 0, 1] = 4               # parent 1: no child has mass
+    for x in range(Mt):
+        if counts[0, 0, x] == 0:
+            ksum[0, 0, x] = 0.0
+    S1, N1, po, co = orc.codebook_update(ksum, counts, np.zeros((H, Mt, d)), np.zeros((H, Mt)), par, ch, 0.0)
+    assert np.allclose(co[0, 0, 2], ch[0, 0, 2]) and np.allclose(co[0, 0, 3], ch[0, 0, 3])
+    assert np.allclose(co.sum(2), C * po, atol=1e-12)
+    shift = ch[0, 1] - co[0, 1]
+    assert np.allclose(shift, shift[0][None, :], atol=1e-12)
+    assert np.allclose(po[0, 1], ksum[0, 0, 1] / 4)
+
+
 ALL_PINS = [pin_hand_worked, pin_assign_brute, pin_aggregate, pin_representative,
             pin_rescale_exercised, pin_flat_p0, pin_exact_codebook, pin_importance, pin_topp,
             pin_relabel, pin_key_permutation, pin_keys_on_codewords, pin_strict_ties,
-            pin_masking, pin_counting, pin_tiled_importance]
+            pin_masking, pin_counting, pin_tiled_importance, pin_codebook_update,
+            pin_codebook_massless]

@@ -41,6 +41,13 @@ MUTANTS = [
     ("tiled-exact-denominator", "ns[j] / (ntot / nseen * zpart[r]);", "ns[j] / z[r];"),
     ("tiled-partial-z-unweighted", "zpart[r] += A[(size_t)r * M0 + j] * ns[j];",
      "zpart[r] += A[(size_t)r * M0 + j];"),
+    ("ema-weights-swapped", "lambda * Nst[(size_t)h * Mt + x] + (1.0 - lambda) * n;",
+     "(1.0 - lambda) * Nst[(size_t)h * Mt + x] + lambda * n;"),
+    ("projection-not-mass-weighted", "shift = nc > 0.0 ? delta / (nc * sigma) : 0.0;",
+     "shift = nc > 0.0 ? delta / massive : 0.0;"),
+    ("projection-residual-sign", "double delta = -C * cp[t];", "double delta = C * cp[t];"),
+    ("massless-child-moves", "shift = nc > 0.0 ? delta / (nc * sigma) : 0.0;",
+     "shift = nc > 0.0 ? delta / (nc * sigma) : delta / C;"),
 ]
 
 
