@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
                 L.avq_attention.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                             _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+                L.avq_codebook_update.argtypes = [P(avq_dims), ctypes.c_int, ctypes.c_float, _vp, _vp,
+                                                  _vp, _vp, _vp, _vp, _vp]
                 L.avq_permute.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _vp]
                 L.avq_hilbert_order.argtypes = [ctypes.c_int, _vp]
@@ -80,7 +82,7 @@ def lib() -> ctypes.CDLL:
                 L.avq_status_string.argtypes = [ctypes.c_int]
                 L.avq_version.restype = ctypes.c_int
                 for name in ("avq_quantize", "avq_quantize_noalloc", "avq_attention", "avq_permute",
-                             "avq_hilbert_order", "avq_check_device"):
+                             "avq_hilbert_order", "avq_check_device", "avq_codebook_update"):
                     getattr(L, name).restype = ctypes.c_int
                 _lib = L
     return _lib
@@ -245,6 +247,29 @@ def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, 
                                int(two_pass), _ptr(O), _ptr(sel) if P > 0 else None,
                                _ptr(imp), wp, wn, _stream(stream)))
     return O, sel, imp
+
+
+def avq_codebook_update(ksum, counts, S, Nst, parents, children, lam: float, stream=None):
+    """Codebook update (EMA statistics and constraint projection).  ksum
+    [B,H,Mt,d] fp32 and counts [B,H,Mt] int32: avq_quantize's statistics of
+    the keys; S [H,Mt,d] and Nst [H,Mt] fp32: EMA state, updated in place;
+    parents [H,M0,d] and children [H,M0,C,d]: codebook, rewritten in place."""
+    B, H, Mt, d = ksum.shape
+    Hp, M0, dp = parents.shape
+    C = 0 if children is None else children.shape[2]
+    if Hp != H or dp != d or Mt != M0 * (1 + C):
+        raise ValueError("ksum must be [B, H, M0*(1+C), d] for parents [H, M0, d]")
+    if children is not None and tuple(children.shape) != (H, M0, C, d):
+        raise ValueError("children must be [H, M0, C, d]")
+    dims = avq_dims(B, H, 1, d, M0, C)
+    dt = _dtype_code(parents)
+    for t, want in ((ksum, torch.float32), (S, torch.float32), (Nst, torch.float32), (counts, torch.int32)):
+        if t.dtype != want:
+            raise TypeError(f"expected {want}, got {t.dtype}")
+    _check(lib().avq_codebook_update(ctypes.byref(dims), dt, float(lam), _ptr(ksum), _ptr(counts),
+                                     _ptr(S), _ptr(Nst), _ptr(parents), _ptr(children),
+                                     _stream(stream)))
+    return S, Nst, parents, children
 
 
 def avq_permute(X, idx, inverse=False, Y=None, stream=None):

@@ -289,6 +289,28 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, c
   return AVQ_OK;
 }
 
+avq_status avq_codebook_update(const avq_dims* dims, avq_dtype dtype, float lambda, const float* ksum,
+                               const int32_t* counts, float* S, float* Nst, void* parents, void* children,
+                               avq_stream_t stream) {
+  t_error[0] = 0;
+  avq_status st = check_dims(dims, dtype);
+  if (st != AVQ_OK) return st;
+  const Shape s = to_shape(dims);
+  if (!(lambda >= 0.f && lambda <= 1.f)) return fail(AVQ_ERR_INVALID_ARG, "lambda must be in [0, 1]");
+  AVQ_REQUIRE_PTR(ksum, "ksum");
+  AVQ_REQUIRE_PTR(counts, "counts");
+  AVQ_REQUIRE_PTR(S, "S");
+  AVQ_REQUIRE_PTR(Nst, "Nst");
+  AVQ_REQUIRE_PTR(parents, "parents");
+  if (s.C > 0) AVQ_REQUIRE_PTR(children, "children");
+  LaunchLog log{};
+  cudaError_t e = launch_codebook_update(s, dtype, lambda, ksum, counts, S, Nst, parents, children,
+                                         reinterpret_cast<cudaStream_t>(stream), log);
+  if (e != cudaSuccess) return cuda_fail(e, "codebook update launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}
+
 avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
                        int row_bytes, int inverse, avq_stream_t stream) {
   t_error[0] = 0;

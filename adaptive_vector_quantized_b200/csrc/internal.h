@@ -65,6 +65,12 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
                                 cudaStream_t st, LaunchLog& log);
 
 // ---- token permutation ----------------------------------------------------
+// Sec. A, Eqs. 11-12: EMA statistics S [H][Mt][d], Nst [H][Mt] updated in
+// place from the keys' Eq. 3 statistics ksum [BH][Mt][d], counts [BH][Mt];
+// parents [H][M0][d] and children [H][M0][C][d] rewritten in place.
+cudaError_t launch_codebook_update(const Shape& s, avq_dtype dt, float lambda, const float* ksum,
+                                   const int32_t* counts, float* S, float* Nst, void* parents,
+                                   void* children, cudaStream_t st, LaunchLog& log);
 cudaError_t launch_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
                            int row_bytes, int inverse, cudaStream_t st, LaunchLog& log);
 

@@ -187,6 +187,33 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q,
                          void* ws, size_t ws_bytes, avq_stream_t stream);
 
 /*
+ * avq_codebook_update -- codebook update for training (Sec. A "Codeword
+ * Clustering During Training", Eqs. 11-12).
+ *
+ * EMA statistics, per head over every batch entry (Eq. 11):
+ *   S_x <- lambda S_x + (1 - lambda) ksum_x,  N_x <- lambda N_x + (1 - lambda) counts_x,
+ * where ksum, counts are the Eq. 3 statistics of the keys, i.e. the vsum and
+ * counts outputs of avq_quantize called with the keys in place of the
+ * values (a parent counts its whole cluster, a child the keys that moved to
+ * it).  Then each parent becomes its mean S_p / N_p and its children the
+ * mass-weighted projection of their means M_c onto sum_c C_pc = C C_p
+ * (Eq. 12): C_pc = M_c - delta / (N_c sigma) with delta = sum_c M_c - C C_p
+ * and sigma = sum_c 1 / N_c, which restores Eq. 5.  A code whose updated N is
+ * 0 has no mean and keeps its current position; massless children do not
+ * move (the others absorb delta), and with no massive child all C children
+ * shift by delta / C.
+ * Arguments (device): ksum [B,H,Mt,d] fp32 and counts [B,H,Mt] int32 (read);
+ * S [H,Mt,d] fp32 and Nst [H,Mt] fp32, the EMA state (read and written);
+ * parents [H,M0,d] and children [H,M0,C,d] of `dtype`, the codebook (read
+ * and rewritten in place).  0 <= lambda <= 1.  dims->N is not used.
+ * Arithmetic is fp32; the bf16 codebook is rounded to nearest, so Eq. 5
+ * then holds to bf16 rounding.
+ */
+avq_status avq_codebook_update(const avq_dims* dims, avq_dtype dtype, float lambda,
+                               const float* ksum, const int32_t* counts, float* S, float* Nst,
+                               void* parents, void* children, avq_stream_t stream);
+
+/*
  * avq_permute -- token reordering gather/scatter (Sec. 4.2 and Fig. 3:
  * tokens reordered along a space-filling curve so that query tiles are
  * spatially compact).

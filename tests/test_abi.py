@@ -140,3 +140,15 @@ def test_denominator_modes_host_checks():
         assert "tensor-core" in avq.last_error()
     finally:
         avq.avq_set_path(old)
+
+
+def test_codebook_update_host_checks():
+    """lambda outside [0, 1] and missing buffers are rejected before launch."""
+    L = avq.lib()
+    d = avq.avq_dims(1, 2, 1, 64, 16, 8)
+    args = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None)
+    assert L.avq_codebook_update(ctypes.byref(d), avq.AVQ_BF16, 1.5, *args) == avq.AVQ_ERR_INVALID_ARG
+    assert L.avq_codebook_update(ctypes.byref(d), avq.AVQ_BF16, -0.1, *args) == avq.AVQ_ERR_INVALID_ARG
+    assert L.avq_codebook_update(ctypes.byref(d), avq.AVQ_BF16, 0.5, None, *args[1:]) == avq.AVQ_ERR_INVALID_ARG
+    assert "ksum" in avq.last_error()
+    assert L.avq_codebook_update(None, avq.AVQ_BF16, 0.5, *args) == avq.AVQ_ERR_INVALID_ARG
