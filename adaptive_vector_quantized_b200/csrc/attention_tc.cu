@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   int* sRK = reinterpret_cast<int*>(sm + S::kRK);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S::kMISC);
   int* sAbort = reinterpret_cast<int*>(sm + S::kMISC + 4);
+  float* sNtot = reinterpret_cast<float*>(sm + S::kMISC + 8);  // keys of the head (extrapolation)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int blk = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
     tc::mbar_init(bar_vb, 1);
     tc::fence_mbar_init();
     *sAbort = 0;
+    *sNtot = 0.f;
     tc::prefetch_tensormap(&qmap);
     tc::prefetch_tensormap(&omap);
   }
@@ -223,8 +225,13 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   // tile from the count-extrapolated denominator (Sec. B, Eqs. 13-14)
   const bool extrap = a.two_pass == 2;
   const int sweeps = extrap ? 1 : (a.two_pass || nT > 1) ? 2 : 1;
-  const float ntot = (float)a.N;  // keys of the head: the sum of the parents' counts
-  float nseen = 0.f;              // keys of the parents in the tiles swept so far
+  if (extrap) {  // N of Eq. 13: the keys of the head, the sum of the parents' counts
+    float c = 0.f;
+    for (int j = tid; j < M0; j += 128) c += (float)__ldg(cnt + j);
+    c = warp_sum(c);
+    if (lane == 0) atomicAdd(sNtot, c);  // read after the next CTA barrier
+  }
+  float nseen = 0.f;  // keys of the parents in the tiles swept so far
   bool x_started = false;
   bool q_ready = false;
 
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
         if (last) {
           // probabilities as bf16, importance column sums of A / z in fp32
           // (A / Z~ with Z~ = z N / N_seen when extrapolating)
-          const float rz = !valid || !(z > 0.f) ? 0.f : extrap ? nseen / (ntot * z) : 1.f / z;
+          const float rz = !valid || !(z > 0.f) ? 0.f : extrap ? nseen / (*sNtot * z) : 1.f / z;
 #pragma unroll
           for (int q = 0; q < 8; ++q) store_chunk8(sPR, tid, q * 8, reinterpret_cast<const float*>(r) + q * 8);
           float v[32];

@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=None)
+    ap.add_argument("--shard", default="batch", choices=["batch", "tokens"],
+                    help="batch: every rank runs its own batch (weak scaling); tokens: the ranks "
+                         "split one batch's tokens and sum the statistics (strong scaling)")
     ap.add_argument("--denominator", default=None, choices=["auto", "two_pass", "extrapolated"],
                     help="importance denominator for parent codebooks over several tiles "
                          "(default: the workload's own setting)")
@@ -229,11 +232,14 @@ def workload_config(name, cfg):
 
 
 # ---------------------------------------------------------------------------
-def run_avq(args, cfg, inp):
+def run_avq(args, cfg, inp, n_global=None):
+    """n_global: with --shard tokens, the tokens of all ranks (cfg and inp
+    then hold this rank's slice)."""
     import torch
     import torch.distributed as dist
 
     import adaptive_vector_quantized_b200 as avq
+    from adaptive_vector_quantized_b200.sharding import allreduce_stats
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -262,9 +268,13 @@ def run_avq(args, cfg, inp):
     O = torch.empty_like(Q)
     sel = torch.empty((B, H, nblk, max(P, 1)), dtype=torch.int32, device=dev)
 
+    exchange = n_global is not None and world > 1
+
     def step():
         avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
         k1 = avq.last_kernels()
+        if exchange:
+            allreduce_stats(vsum, counts)
         avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
                           ws=ws, stream=stream)
         return k1, avq.last_kernels()
@@ -292,6 +302,8 @@ def run_avq(args, cfg, inp):
         for s in range(args.steps):
             ev[s][0].record(stream)
             avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
+            if exchange:
+                allreduce_stats(vsum, counts)
             ev[s][1].record(stream)
             avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
                               ws=ws, stream=stream)
@@ -305,7 +317,7 @@ def run_avq(args, cfg, inp):
     t_s1 = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     t_s2 = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     ms_step = ms / args.steps
-    queries = B * H * N * world
+    queries = B * H * N * world if n_global is None else B * H * n_global
     value = queries / (ms_step * 1e-3)
 
     # end to end through the public API with host buffers
@@ -371,7 +383,8 @@ def run_avq(args, cfg, inp):
                    sample=f"{heads} head(s) x N={N} of the same workload, b=0: all keys quantised "
                           f"and all queries attended, float64, OpenMP")
     line = dict(metric=METRIC, value=value, unit="queries/s", n_gpus=world, steps=args.steps,
-                warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+                warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
+                scaling="weak" if n_global is None else "strong",
                 vs_baseline=None, dtype=cfg["dtype"], data="synthetic",
                 config=dict(workload_config(args.config, cfg),
                             l2="inputs larger than L2 (Q, K, V 134 MB each per step); no flush"
@@ -403,6 +416,19 @@ def main():
             return
         inp = synth.make_inputs(dict(cfg, B=1, H=1), seed)
         run_reference(args, cfg, inp)
+        return
+    if args.shard == "tokens":  # same inputs on every rank, each takes its slice of the tokens
+        from adaptive_vector_quantized_b200.sharding import shard_rows
+
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        base = args.seed if args.seed is not None else synth.CONFIG_SEEDS.get(args.config, 1000)
+        inp = synth.make_inputs(cfg, base)
+        n0, n1 = shard_rows(cfg["N"], cfg["block"], rank, world)
+        if n1 <= n0:
+            raise SystemExit("more ranks than query blocks")
+        for k in ("Q", "K", "V"):
+            inp[k] = inp[k][:, :, n0:n1].contiguous()
+        run_avq(args, dict(cfg, N=n1 - n0), inp, n_global=cfg["N"])
         return
     inp = synth.make_inputs(cfg, seed)
     run_avq(args, cfg, inp)
