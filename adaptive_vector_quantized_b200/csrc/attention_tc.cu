@@ -51,7 +51,7 @@ struct AttnArgs {
   int32_t* sel;     // [BH][nblk][P] or null
   float* importance;  // [BH][nblk][M0] or null
   unsigned int* err;
-  int H, N, M0, C, P, nblk, two_pass;
+  int H, N, M0, C, P, nblk, two_pass, BH;
   float scale_log2;  // scale * log2(e)
 };
 
@@ -563,20 +563,27 @@ done:
 //     a chunk) gets a zero value atom for the same reason;
 //   - the codewords of chunk q + 1 are copied as soon as the logit MMA of
 //     chunk q has read its own, the value sums as soon as its value MMA has;
-//   - the value MMAs are not waited for until their operands are reused.
+//   - the value MMAs are not waited for until their operands are reused;
+//   - the kernel is persistent: a CTA walks a contiguous range of (head,
+//     block) units and fetches the next unit's Q tile and parent codewords as
+//     soon as the current unit's last logit MMA has read its own, the parents'
+//     value sums as soon as its last value MMA has; the O tile is staged in
+//     the PR buffer and its TMA store is waited for only before PR is
+//     written again.
 template <int D>
 struct FastSmem {
   static constexpr int kAtomBytes = 1024 * (D / 64);       // one 8-code atom group
-  static constexpr int kQ = 0;                             // Q tile / O staging
+  static constexpr int kQ = 0;                             // Q tile
   static constexpr int kCW = kQ + kRows * D * 2;           // codewords: parents, then chunks
   static constexpr int kVB = kCW + 8 * kAtomBytes;         // value sums: parents, then chunks
-  static constexpr int kPR = kVB + 8 * kAtomBytes;         // probabilities / dA [128][64] bf16
-  static constexpr int kNF = kPR + kRows * 64 * 2;         // counts [2][64]: parents, current chunk
+  static constexpr int kPR = kVB + 8 * kAtomBytes;         // probabilities / dA [128][64] bf16; O staging
+  static constexpr int kNF = kPR + kRows * D * 2;          // counts [2][64]: parents, current chunk
   static constexpr int kW = kNF + 2 * 64 * 4;              // importance [64]
   static constexpr int kWP = kW + 64 * 4;                  // per-warp partial sums [4][64]
   static constexpr int kSEL = kWP + 4 * 64 * 4;            // selected parents [64]
   static constexpr int kRK = kSEL + 64 * 4;                // partial ranks [2][64]
-  static constexpr int kBAR = kRK + 2 * 64 * 4;            // 6 mbarriers
+  static constexpr int kCNT = kRK + 2 * 64 * 4;            // counts of the unit's head [Mt <= 576]
+  static constexpr int kBAR = kCNT + 576 * 4;              // 6 mbarriers
   static constexpr int kMISC = kBAR + 64;                  // tmem base, abort flag
   static constexpr int kTotal = kMISC + 32;
   static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
@@ -604,24 +611,43 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   float* sWP = reinterpret_cast<float*>(sm + S::kWP);
   int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
   int* sRK = reinterpret_cast<int*>(sm + S::kRK);
+  const int32_t* sCNT = reinterpret_cast<const int32_t*>(sm + S::kCNT);
   uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + S::kBAR);
-  uint64_t* bar_cw = bar_q + 1;   // codeword copies (parents, then one per chunk)
-  uint64_t* bar_vb = bar_q + 2;   // value-sum copies (parents, then one per chunk)
+  uint64_t* bar_cw = bar_q + 1;   // parents' codewords and the head's counts
+  uint64_t* bar_vb = bar_q + 2;   // parents' value sums
   uint64_t* bar_mma = bar_q + 3;  // logit MMAs
   uint64_t* bar_x = bar_q + 4;    // value MMAs
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S::kMISC);
   int* sAbort = reinterpret_cast<int*>(sm + S::kMISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int blk = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
-  const int row0 = blk * kRows;
-  const bool valid = row0 + tid < a.N;
   const int C = a.C, Mt = M0 * (1 + C), P = a.P;
-  const bf16* cw_h = a.cw + (size_t)h * (Mt / 8) * KH * 512;
-  const bf16* vb_bh = a.vb + (size_t)bh * (Mt / 8) * KH * 512;
-  const int32_t* cnt = a.counts + (size_t)bh * Mt;
   const float NEG_INF = __int_as_float(0xff800000);
   const float sl2 = a.scale_log2;
+  // this CTA's contiguous range of units u = bh * nblk + block
+  const int total = a.BH * a.nblk;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int u0 = blockIdx.x * per, u1 = min(total, u0 + per);
+  if (u0 >= u1) return;
+  const int nch = (C > 0 && P > 0) ? (P + kChunkParents - 1) / kChunkParents : 0;
+  auto unit_cw = [&](int u) { return a.cw + (size_t)((u / a.nblk) % a.H) * (Mt / 8) * KH * 512; };
+  auto unit_vb = [&](int u) { return a.vb + (size_t)(u / a.nblk) * (Mt / 8) * KH * 512; };
+  // the next unit's Q tile and parents' codewords / value sums (thread 0)
+  auto load_q = [&](int u) {
+    tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh)
+      tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, (u % a.nblk) * kRows, u / a.nblk, bar_q);
+  };
+  auto load_pcw = [&](int u) {
+    tc::mbar_arrive_expect_tx(bar_cw, M0 * D * 2 + Mt * 4);
+    tc::bulk_g2s(sCW, unit_cw(u), M0 * D * 2, bar_cw);
+    tc::bulk_g2s(sm + S::kCNT, a.counts + (size_t)(u / a.nblk) * Mt, Mt * 4, bar_cw);
+  };
+  auto load_pvb = [&](int u) {
+    tc::mbar_arrive_expect_tx(bar_vb, M0 * D * 2);
+    tc::bulk_g2s(sVB, unit_vb(u), M0 * D * 2, bar_vb);
+  };
 
   if (tid == 0) {
     for (int i = 0; i < 5; ++i) tc::mbar_init(bar_q + i, 1);
@@ -638,24 +664,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   if (tid == 0) {
     tc::prefetch_tensormap(&qmap);
     tc::prefetch_tensormap(&omap);
-    tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
-#pragma unroll
-    for (int kh = 0; kh < KH; ++kh) tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, row0, bh, bar_q);
-    tc::mbar_arrive_expect_tx(bar_cw, M0 * D * 2);
-    tc::bulk_g2s(sCW, cw_h, M0 * D * 2, bar_cw);
-    tc::mbar_arrive_expect_tx(bar_vb, M0 * D * 2);
-    tc::bulk_g2s(sVB, vb_bh, M0 * D * 2, bar_vb);
+    load_q(u0);
+    load_pcw(u0);
+    load_pvb(u0);
   }
-  float nfj = 0.f;
-  if (tid < M0) {
-    nfj = (float)__ldg(cnt + tid);
-    sNF[tid] = nfj;
-  }
-  if (tid == 0 && !(tc::mbar_wait(bar_q, 0) && tc::mbar_wait(bar_cw, 0))) fail(a.err, sAbort);
-  tc::tc_fence_before();
-  const bool any_empty = __syncthreads_or(tid < M0 && !(nfj > 0.f)) != 0;
-  tc::tc_fence_after();
-  if (*sAbort) goto done;
   {
     const uint32_t tmem = *sTmem;
     const uint32_t tS = tmem;          // logits
@@ -664,7 +676,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     const uint32_t sQa = tc::smem_u32(sQ), sCWa = tc::smem_u32(sCW), sVBa = tc::smem_u32(sVB),
                    sPRa = tc::smem_u32(sPR);
     const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
-    uint32_t ph_cw = 1, ph_vb = 0, ph_mma = 0, ph_x = 0;  // the parents' codeword phase is consumed
+    uint32_t ph_q = 0, ph_cw = 0, ph_vb = 0, ph_mma = 0, ph_x = 0;
 
     auto issue_logits = [&](int n) {  // S = Q * CW^T over n codes
       const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
@@ -690,27 +702,43 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       if (tid == 0 && !tc::mbar_wait(bar, ph)) fail(a.err, sAbort);
       ph ^= 1;
     };
-    // child codewords / value sums of chunk q into the staging buffer: warp 0,
-    // one bulk copy per lane after lane 0 has announced the byte count
+    // child atoms of chunk q (codewords or value sums) into the staging
+    // buffer: `slots` atoms, slot i from selected parent min(i, np - 1), as
+    // 16-byte cp.async pieces spread over all threads, one commit group
     auto chunk_np = [&](int q) { return min(kChunkParents, P - q * kChunkParents); };
-    auto copy_cw = [&](int q) {
-      const int np = chunk_np(q), slots = (np + 1) & ~1;
-      if (lane == 0) tc::mbar_arrive_expect_tx(bar_cw, (uint32_t)slots * AB);
-      __syncwarp();
-      if (lane < slots) {
-        const int p = sSEL[q * kChunkParents + min(lane, np - 1)];
-        tc::bulk_g2s(sCW + lane * AB, cw_h + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_cw);
-      }
-    };
-    auto copy_vb = [&](int q) {
+    auto copy_atoms = [&](uint8_t* dst, const bf16* src_h, int q, int slots) {
+      constexpr int kPieces = AB / 16;
       const int np = chunk_np(q);
-      if (lane == 0) tc::mbar_arrive_expect_tx(bar_vb, (uint32_t)np * AB);
-      __syncwarp();
-      if (lane < np) {
-        const int p = sSEL[q * kChunkParents + lane];
-        tc::bulk_g2s(sVB + lane * AB, vb_bh + (size_t)(M0 / 8 + p) * KH * 512, AB, bar_vb);
+      for (int i = tid; i < slots * kPieces; i += 128) {
+        const int sl = i / kPieces, off = i % kPieces;
+        const int p = sSEL[q * kChunkParents + min(sl, np - 1)];
+        tc::cp_async16(dst + sl * AB + off * 16,
+                       reinterpret_cast<const uint8_t*>(src_h + (size_t)(M0 / 8 + p) * KH * 512) + off * 16);
       }
+      tc::cp_async_commit();
     };
+    auto copy_cw = [&](int q, const bf16* cw_h) { copy_atoms(sCW, cw_h, q, (chunk_np(q) + 1) & ~1); };
+    auto copy_vb = [&](int q, const bf16* vb_bh) { copy_atoms(sVB, vb_bh, q, chunk_np(q)); };
+
+    for (int u = u0; u < u1; ++u) {
+    const int bh = u / a.nblk, blk = u % a.nblk;
+    const int row0 = blk * kRows;
+    const bool valid = row0 + tid < a.N;
+    const bf16* cw_h = unit_cw(u);
+    const bf16* vb_bh = unit_vb(u);
+    const bool has_next = u + 1 < u1;
+    wait_bar(bar_q, ph_q);
+    wait_bar(bar_cw, ph_cw);
+    __syncthreads();
+    float nfj = 0.f;
+    if (tid < M0) {
+      nfj = (float)sCNT[tid];
+      sNF[tid] = nfj;
+    }
+    tc::tc_fence_before();
+    const bool any_empty = __syncthreads_or(tid < M0 && !(nfj > 0.f)) != 0;
+    tc::tc_fence_after();
+    if (*sAbort) goto done;
 
     // ---- parents: logits, masked max, A = 2^(t - m), z, importance ----
     if (tid == 0) {
@@ -718,64 +746,88 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       issue_logits(M0);
     }
     wait_bar(bar_mma, ph_mma);
+    if (tid == 0) {
+      tc::bulk_wait_group_read0();  // the previous unit's O store has read its staging (PR)
+      if (nch == 0 && has_next) {   // Q and the parents' codewords are read: next unit's
+        load_q(u + 1);
+        load_pcw(u + 1);
+      }
+    }
     __syncthreads();
     tc::tc_fence_after();
     float m, z;
     {
-      uint32_t r[M0];
-#pragma unroll
-      for (int q = 0; q < M0 / 16; ++q) tc::tmem_ld16(tS + lane_off + q * 16, r + q * 16);
-      tc::tmem_wait_ld();
+      // the logits are read from TMEM in 16-column pieces: the maximum first,
+      // then A = 2^(t - m) (to PR in bf16, and back over the logits in fp32 for
+      // the importance, which needs 1 / z of the whole row)
       const float4* nf4 = reinterpret_cast<const float4*>(sNF);
       float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
-      if (!any_empty) {
 #pragma unroll
-        for (int e = 0; e < M0; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(r[e]));
-      } else {
+      for (int g = 0; g < M0 / 16; ++g) {
+        uint32_t r[16];
+        tc::tmem_ld16(tS + lane_off + g * 16, r);
+        tc::tmem_wait_ld();
+        if (!any_empty) {
 #pragma unroll
-        for (int e = 0; e < M0; e += 4) {
-          const float4 nf = nf4[e >> 2];
-          mx[0] = fmaxf(mx[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
-          mx[1] = fmaxf(mx[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
-          mx[2] = fmaxf(mx[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
-          mx[3] = fmaxf(mx[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
+          for (int e = 0; e < 16; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(r[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            const float4 nf = nf4[(g * 16 + e) >> 2];
+            mx[0] = fmaxf(mx[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
+            mx[1] = fmaxf(mx[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
+            mx[2] = fmaxf(mx[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
+            mx[3] = fmaxf(mx[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
+          }
         }
       }
       m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       const float nm = -m;
       float zp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < M0; e += 4) {
-        const float4 nf = nf4[e >> 2];
-        float a0 = tc::ex2(fmaf(__uint_as_float(r[e]), sl2, nm));
-        float a1 = tc::ex2(fmaf(__uint_as_float(r[e + 1]), sl2, nm));
-        float a2 = tc::ex2(fmaf(__uint_as_float(r[e + 2]), sl2, nm));
-        float a3 = tc::ex2(fmaf(__uint_as_float(r[e + 3]), sl2, nm));
-        if (any_empty) {
-          a0 = nf.x > 0.f ? a0 : 0.f;
-          a1 = nf.y > 0.f ? a1 : 0.f;
-          a2 = nf.z > 0.f ? a2 : 0.f;
-          a3 = nf.w > 0.f ? a3 : 0.f;
-        }
-        zp[0] = fmaf(a0, nf.x, zp[0]);
-        zp[1] = fmaf(a1, nf.y, zp[1]);
-        zp[2] = fmaf(a2, nf.z, zp[2]);
-        zp[3] = fmaf(a3, nf.w, zp[3]);
-        r[e] = __float_as_uint(a0);
-        r[e + 1] = __float_as_uint(a1);
-        r[e + 2] = __float_as_uint(a2);
-        r[e + 3] = __float_as_uint(a3);
-      }
-      z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+      for (int g = 0; g < M0 / 16; ++g) {
+        uint32_t r[16];
+        tc::tmem_ld16(tS + lane_off + g * 16, r);
+        tc::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < M0 / 8; ++c) store_chunk8(sPR, tid, c * 8, reinterpret_cast<const float*>(r) + c * 8);
+        for (int e = 0; e < 16; e += 4) {
+          const float4 nf = nf4[(g * 16 + e) >> 2];
+          float a0 = tc::ex2(fmaf(__uint_as_float(r[e]), sl2, nm));
+          float a1 = tc::ex2(fmaf(__uint_as_float(r[e + 1]), sl2, nm));
+          float a2 = tc::ex2(fmaf(__uint_as_float(r[e + 2]), sl2, nm));
+          float a3 = tc::ex2(fmaf(__uint_as_float(r[e + 3]), sl2, nm));
+          if (any_empty) {
+            a0 = nf.x > 0.f ? a0 : 0.f;
+            a1 = nf.y > 0.f ? a1 : 0.f;
+            a2 = nf.z > 0.f ? a2 : 0.f;
+            a3 = nf.w > 0.f ? a3 : 0.f;
+          }
+          zp[0] = fmaf(a0, nf.x, zp[0]);
+          zp[1] = fmaf(a1, nf.y, zp[1]);
+          zp[2] = fmaf(a2, nf.z, zp[2]);
+          zp[3] = fmaf(a3, nf.w, zp[3]);
+          r[e] = __float_as_uint(a0);
+          r[e + 1] = __float_as_uint(a1);
+          r[e + 2] = __float_as_uint(a2);
+          r[e + 3] = __float_as_uint(a3);
+        }
+        store_chunk8(sPR, tid, g * 16, reinterpret_cast<const float*>(r));
+        store_chunk8(sPR, tid, g * 16 + 8, reinterpret_cast<const float*>(r) + 8);
+        tc::tmem_st16(tS + lane_off + g * 16, r);
+      }
+      tc::tmem_wait_st();
+      z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
       // importance column sums of A / z (Eq. 7), fp32
       const float rz = valid ? 1.f / z : 0.f;
 #pragma unroll
       for (int g = 0; g < (M0 + 31) / 32; ++g) {
+        uint32_t r[32];
+        tc::tmem_ld16(tS + lane_off + g * 32, r);
+        if (g * 32 + 16 < M0) tc::tmem_ld16(tS + lane_off + g * 32 + 16, r + 16);
+        tc::tmem_wait_ld();
         float v[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = (g * 32 + e < M0) ? __uint_as_float(r[(g * 32 + e) % M0]) * rz : 0.f;
+        for (int e = 0; e < 32; ++e) v[e] = (g * 32 + e < M0) ? __uint_as_float(r[e]) * rz : 0.f;
         sWP[warp * 64 + g * 32 + lane] = reduce_scatter32(v, lane);
       }
     }
@@ -792,38 +844,38 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     }
 
     // ---- top-P over the importance (descending, ties to the lower index) ----
-    // thread j < M0 ranks parent j against all M0 importances held in registers
-    const int nch = (C > 0 && P > 0) ? (P + kChunkParents - 1) / kChunkParents : 0;
-    if (tid < M0) {
-      const float wj = sW[tid];
-      int rank = 0;
-#pragma unroll 1
-      for (int l0 = 0; l0 < M0; l0 += 16) {
-        float wv[16];
-#pragma unroll
-        for (int l = 0; l < 16; l += 4) {
-          const float4 w4 = reinterpret_cast<const float4*>(sW)[(l0 + l) >> 2];
-          wv[l] = w4.x;
-          wv[l + 1] = w4.y;
-          wv[l + 2] = w4.z;
-          wv[l + 3] = w4.w;
+    // thread t ranks parent t % 64 against half of the M0 importances; the
+    // two partial ranks are added by the first 64 threads
+    {
+      const int j = tid & 63, half = tid >> 6;
+      constexpr int kHalf = (M0 + 1) / 2;
+      if (j < M0) {
+        const float wj = sW[j];
+        int rank = 0;
+        const int l0 = half * kHalf, l1 = min(M0, l0 + kHalf);
+#pragma unroll 8
+        for (int l = l0; l < l1; ++l) {
+          const float wl = sW[l];
+          rank += (wl > wj) || (wl == wj && l < j);
         }
-#pragma unroll
-        for (int l = 0; l < 16; ++l) rank += (wv[l] > wj) || (wv[l] == wj && l0 + l < tid);
+        sRK[half * 64 + j] = rank;
       }
+    }
+    __syncthreads();
+    if (tid < M0) {
+      const int rank = sRK[tid] + sRK[64 + tid];
       if (rank < P) {
         sSEL[rank] = tid;
         if (a.sel) a.sel[((size_t)bh * a.nblk + blk) * P + rank] = tid;
       }
-      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = wj;
+      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = sW[tid];
     }
     __syncthreads();
-    if (warp == 0 && nch > 0) copy_cw(0);  // the parent logit MMA has read the codewords
-    wait_bar(bar_x, ph_x);                 // the parents' value MMA has read PR and VB
-    if (warp == 0 && nch > 0) {
-      __syncwarp();
-      copy_vb(0);
-    }
+    if (nch > 0) copy_cw(0, cw_h);  // the parent logit MMA has read the codewords
+    wait_bar(bar_x, ph_x);          // the parents' value MMA has read PR and VB
+    __syncthreads();
+    if (nch > 0) copy_vb(0, vb_bh);
+    if (tid == 0 && nch == 0 && has_next) load_pvb(u + 1);  // the parents' value MMA is done
 
     // ---- child refinement in chunks of 8 selected parents ----
     float mref = m;
@@ -834,9 +886,15 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       const int n = slots * 8;
       if (tid < 64) {
         const int rr = tid >> 3;
-        nfc[tid] = rr < np ? (float)__ldg(cnt + M0 + sSEL[q * kChunkParents + rr] * 8 + (tid & 7)) : 0.f;
+        nfc[tid] = rr < np ? (float)sCNT[M0 + sSEL[q * kChunkParents + rr] * 8 + (tid & 7)] : 0.f;
       }
-      wait_bar(bar_cw, ph_cw);
+      // this chunk's codewords: at q = 0 the value sums of chunk 0 were
+      // committed after them and may still be in flight
+      if (q == 0)
+        tc::cp_async_wait<1>();
+      else
+        tc::cp_async_wait<0>();
+      tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncthreads();
       if (*sAbort) goto done;
@@ -845,37 +903,42 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         issue_logits(n);
       }
       wait_bar(bar_mma, ph_mma);
-      if (warp == 0 && q + 1 < nch) {  // the logit MMA has read this chunk's codewords
-        __syncwarp();
-        copy_cw(q + 1);
+      if (tid == 0 && q + 1 == nch && has_next) {  // the last logit MMA: Q and CW are free
+        load_q(u + 1);
+        load_pcw(u + 1);
       }
       __syncthreads();
       tc::tc_fence_after();
-      uint32_t r[64];
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-        if (g * 16 < n) tc::tmem_ld16(tS + lane_off + g * 16, r + g * 16);
-      tc::tmem_wait_ld();
+      if (q + 1 < nch) copy_cw(q + 1, cw_h);  // the logit MMA has read this chunk's codewords
+      // the child logits are read from TMEM twice (maximum, then dA), 16
+      // columns (two slots) at a time, which keeps few of them in registers
       const float4* nf4 = reinterpret_cast<const float4*>(nfc);
       float cm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (e < n) cm[e & 3] = fmaxf(cm[e & 3], __uint_as_float(r[e]));
+      for (int g = 0; g < 4; ++g) {
+        if (g * 16 < n) {
+          uint32_t r[16];
+          tc::tmem_ld16(tS + lane_off + g * 16, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) cm[e & 3] = fmaxf(cm[e & 3], __uint_as_float(r[e]));
+        }
+      }
       const float cmax_any = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) * sl2;
       if (q > 0) wait_bar(bar_x, ph_x);  // previous chunk's value MMA: PR, VB and x are free
       const bool masked = __syncthreads_or(cmax_any > mref + kRescaleLog2) != 0;  // block-uniform, rare
-      if (warp == 0 && q > 0) copy_vb(q);
+      if (q > 0) copy_vb(q, vb_bh);
       if (masked) {
         // masked maximum over non-empty children; rescale x and z if it is far above
         float cmm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+        for (int g = 0; g < 4; ++g) {
+          if (g * 16 < n) {
+            uint32_t r[16];
+            tc::tmem_ld16(tS + lane_off + g * 16, r);
+            tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          if (e < n) {
-            const float4 nf = nf4[e >> 2];
-            cmm[0] = fmaxf(cmm[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
-            cmm[1] = fmaxf(cmm[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
-            cmm[2] = fmaxf(cmm[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
-            cmm[3] = fmaxf(cmm[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
+            for (int e = 0; e < 16; ++e)
+              cmm[e & 3] = fmaxf(cmm[e & 3], nfc[g * 16 + e] > 0.f ? __uint_as_float(r[e]) : NEG_INF);
           }
         }
         const float cmax = fmaxf(fmaxf(cmm[0], cmm[1]), fmaxf(cmm[2], cmm[3])) * sl2;
@@ -900,30 +963,42 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       const float nm = -mref, sl8 = sl2 * 0.125f;
       float zp[2] = {0.f, 0.f};
 #pragma unroll
-      for (int sl = 0; sl < 8; ++sl) {
-        if (sl < slots) {
-          float ssum = 0.f;
+      for (int g = 0; g < 4; ++g) {
+        if (g * 16 < n) {
+          uint32_t r[16];
+          tc::tmem_ld16(tS + lane_off + g * 16, r);
+          tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ssum += __uint_as_float(r[sl * 8 + e]);
-          const float ap = tc::ex2(fmaf(ssum, sl8, nm));
-          const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
-          const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
-          float da[8];
+          for (int hs = 0; hs < 2; ++hs) {
+            const int sl = 2 * g + hs;
+            float ssum = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            da[e] = tc::ex2(fmaf(__uint_as_float(r[sl * 8 + e]), sl2, nm)) - ap;
-            if (masked && !(nfv[e] > 0.f)) da[e] = 0.f;
-            zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
+            for (int e = 0; e < 8; ++e) ssum += __uint_as_float(r[hs * 8 + e]);
+            const float ap = tc::ex2(fmaf(ssum, sl8, nm));
+            const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
+            const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+            float da[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              da[e] = tc::ex2(fmaf(__uint_as_float(r[hs * 8 + e]), sl2, nm)) - ap;
+              if (masked && !(nfv[e] > 0.f)) da[e] = 0.f;
+              zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
+            }
+            store_chunk8(sPR, tid, sl * 8, da);
           }
-          store_chunk8(sPR, tid, sl * 8, da);
         }
       }
       z += zp[0] + zp[1];
       if (np & 1)  // padding slot: zero value sums, so it adds nothing
         for (int i = tid; i < AB / 16; i += 128)
           reinterpret_cast<uint4*>(sVB + np * AB)[i] = make_uint4(0, 0, 0, 0);
+      // this chunk's value sums: at q = 0 the codewords of chunk 1 were
+      // committed after them and may still be in flight
+      if (q == 0 && nch > 1)
+        tc::cp_async_wait<1>();
+      else
+        tc::cp_async_wait<0>();
       tc::fence_proxy_async_smem();
-      wait_bar(bar_vb, ph_vb);
       tc::tc_fence_before();
       __syncthreads();
       if (*sAbort) goto done;
@@ -933,10 +1008,12 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       }
     }
     if (nch > 0) wait_bar(bar_x, ph_x);  // the last value MMA
+    if (tid == 0 && nch > 0 && has_next) load_pvb(u + 1);
     __syncthreads();
     tc::tc_fence_after();
 
-    // ---- O = x / z -> bf16 -> shared (Q region) -> TMA store ----
+    // ---- O = x / z -> bf16 -> shared (PR region) -> TMA store (waited for
+    //      only before the staging is written again) ----
     {
       const float iz = 1.f / z;
       for (int g = 0; g < D; g += 16) {
@@ -946,20 +1023,23 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         float v[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(xr[e]) * iz;
-        store_chunk8(sQ, tid, g, v);
-        store_chunk8(sQ, tid, g + 8, v + 8);
+        store_chunk8(sPR, tid, g, v);
+        store_chunk8(sPR, tid, g + 8, v + 8);
       }
       tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
       __syncthreads();
       if (tid == 0) {
 #pragma unroll
-        for (int kh = 0; kh < KH; ++kh) tc::tma_store_3d(&omap, sQ + kh * kRows * 128, kh * 64, row0, bh);
+        for (int kh = 0; kh < KH; ++kh) tc::tma_store_3d(&omap, sPR + kh * kRows * 128, kh * 64, row0, bh);
         tc::bulk_commit_group();
-        tc::bulk_wait_group_read0();
       }
     }
+    }  // units
   }
 done:
+  tc::cp_async_wait<0>();
+  if (tid == 0) tc::bulk_wait_group_read0();  // the last O store has read the staging
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1014,6 +1094,12 @@ cudaError_t launch_fast_m(dim3 grid, const CUtensorMap& qmap, const CUtensorMap&
   cudaError_t e =
       cudaFuncSetAttribute(attention_fast_kernel<D, M0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // persistent: as many CTAs as fit at once (TMEM and registers allow four
+  // per SM at d = 64, two at d = 128), each walking a contiguous range of
+  // (head, block) units so that it can fetch the next unit's operands early
+  constexpr int kCtasPerSm = D == 64 ? 4 : 2;
+  const long long units = (long long)grid.x * grid.y;
+  grid = dim3((unsigned)std::max<long long>(1, std::min<long long>(units, (long long)num_sms() * kCtasPerSm)));
   attention_fast_kernel<D, M0><<<grid, 128, smem, st>>>(qmap, omap, a);
   return cudaGetLastError();
 }
@@ -1083,6 +1169,7 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
   a.C = s.C;
   a.P = P;
   a.nblk = (s.N + kRows - 1) / kRows;
+  a.BH = s.BH();
   a.two_pass = two_pass;
   a.scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(a.nblk, s.BH());

@@ -36,9 +36,9 @@ __device__ __forceinline__ void load8(const bf16* p, float* o) {
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
+  uint32_t r;  // one paired conversion, round to nearest even; `lo` in the low half
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // 8 fp32 -> 8 consecutive elements (16-byte aligned destination).
