@@ -30,6 +30,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -784,37 +785,34 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       const float nm = -m;
       float zp[4] = {0.f, 0.f, 0.f, 0.f};
+      auto a_pass = [&](auto masked_t) {
+        constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
-      for (int g = 0; g < M0 / 16; ++g) {
-        uint32_t r[16];
-        tc::tmem_ld16(tS + lane_off + g * 16, r);
-        tc::tmem_wait_ld();
+        for (int g = 0; g < M0 / 16; ++g) {
+          uint32_t r[16];
+          tc::tmem_ld16(tS + lane_off + g * 16, r);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 nf = nf4[(g * 16 + e) >> 2];
-          float a0 = tc::ex2(fmaf(__uint_as_float(r[e]), sl2, nm));
-          float a1 = tc::ex2(fmaf(__uint_as_float(r[e + 1]), sl2, nm));
-          float a2 = tc::ex2(fmaf(__uint_as_float(r[e + 2]), sl2, nm));
-          float a3 = tc::ex2(fmaf(__uint_as_float(r[e + 3]), sl2, nm));
-          if (any_empty) {
-            a0 = nf.x > 0.f ? a0 : 0.f;
-            a1 = nf.y > 0.f ? a1 : 0.f;
-            a2 = nf.z > 0.f ? a2 : 0.f;
-            a3 = nf.w > 0.f ? a3 : 0.f;
+          for (int e = 0; e < 16; e += 4) {
+            const float4 nf = nf4[(g * 16 + e) >> 2];
+            const float nfv[4] = {nf.x, nf.y, nf.z, nf.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              float av = tc::ex2(fmaf(__uint_as_float(r[e + k]), sl2, nm));
+              if (kMasked && !(nfv[k] > 0.f)) av = 0.f;
+              zp[k] = fmaf(av, nfv[k], zp[k]);
+              r[e + k] = __float_as_uint(av);
+            }
           }
-          zp[0] = fmaf(a0, nf.x, zp[0]);
-          zp[1] = fmaf(a1, nf.y, zp[1]);
-          zp[2] = fmaf(a2, nf.z, zp[2]);
-          zp[3] = fmaf(a3, nf.w, zp[3]);
-          r[e] = __float_as_uint(a0);
-          r[e + 1] = __float_as_uint(a1);
-          r[e + 2] = __float_as_uint(a2);
-          r[e + 3] = __float_as_uint(a3);
+          store_chunk8(sPR, tid, g * 16, reinterpret_cast<const float*>(r));
+          store_chunk8(sPR, tid, g * 16 + 8, reinterpret_cast<const float*>(r) + 8);
+          tc::tmem_st16(tS + lane_off + g * 16, r);
         }
-        store_chunk8(sPR, tid, g * 16, reinterpret_cast<const float*>(r));
-        store_chunk8(sPR, tid, g * 16 + 8, reinterpret_cast<const float*>(r) + 8);
-        tc::tmem_st16(tS + lane_off + g * 16, r);
-      }
+      };
+      if (any_empty)
+        a_pass(std::true_type{});
+      else
+        a_pass(std::false_type{});
       tc::tmem_wait_st();
       z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
       // importance column sums of A / z (Eq. 7), fp32
@@ -852,11 +850,13 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       if (j < M0) {
         const float wj = sW[j];
         int rank = 0;
-        const int l0 = half * kHalf, l1 = min(M0, l0 + kHalf);
-#pragma unroll 8
-        for (int l = l0; l < l1; ++l) {
-          const float wl = sW[l];
-          rank += (wl > wj) || (wl == wj && l < j);
+        const int l0 = half * kHalf;
+#pragma unroll
+        for (int l = 0; l < kHalf; l += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(sW + l0 + l);
+          const float wl[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) rank += (wl[k] > wj) || (wl[k] == wj && l0 + l + k < j);
         }
         sRK[half * 64 + j] = rank;
       }
@@ -959,35 +959,42 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
           if (need) mref = cmax;
         }
       }
-      // dA = 2^(t_c - m) - 2^(t_p - m), t_p the mean of the 8 child logits (Eq. 8)
+      // dA = 2^(t_c - m) - 2^(t_p - m), t_p the mean of the 8 child logits (Eq. 8);
+      // the masked variant (empty children give 0) only in the rare rescale case
       const float nm = -mref, sl8 = sl2 * 0.125f;
       float zp[2] = {0.f, 0.f};
+      auto da_pass = [&](auto masked_t) {
+        constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        if (g * 16 < n) {
-          uint32_t r[16];
-          tc::tmem_ld16(tS + lane_off + g * 16, r);
-          tc::tmem_wait_ld();
+        for (int g = 0; g < 4; ++g) {
+          if (g * 16 < n) {
+            uint32_t r[16];
+            tc::tmem_ld16(tS + lane_off + g * 16, r);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int hs = 0; hs < 2; ++hs) {
-            const int sl = 2 * g + hs;
-            float ssum = 0.f;
+            for (int hs = 0; hs < 2; ++hs) {
+              const int sl = 2 * g + hs;
+              const float* t = reinterpret_cast<const float*>(r) + hs * 8;
+              const float ssum = ((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7]));
+              const float ap = tc::ex2(fmaf(ssum, sl8, nm));
+              const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
+              const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+              float da[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ssum += __uint_as_float(r[hs * 8 + e]);
-            const float ap = tc::ex2(fmaf(ssum, sl8, nm));
-            const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
-            const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
-            float da[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              da[e] = tc::ex2(fmaf(__uint_as_float(r[hs * 8 + e]), sl2, nm)) - ap;
-              if (masked && !(nfv[e] > 0.f)) da[e] = 0.f;
-              zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
+              for (int e = 0; e < 8; ++e) {
+                da[e] = tc::ex2(fmaf(t[e], sl2, nm)) - ap;
+                if (kMasked && !(nfv[e] > 0.f)) da[e] = 0.f;
+                zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
+              }
+              store_chunk8(sPR, tid, sl * 8, da);
             }
-            store_chunk8(sPR, tid, sl * 8, da);
           }
         }
-      }
+      };
+      if (masked)
+        da_pass(std::true_type{});
+      else
+        da_pass(std::false_type{});
       z += zp[0] + zp[1];
       if (np & 1)  // padding slot: zero value sums, so it adds nothing
         for (int i = tid; i < AB / 16; i += 128)
