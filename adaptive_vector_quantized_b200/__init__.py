@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
                 L.avq_permute.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _vp]
                 L.avq_hilbert_order.argtypes = [ctypes.c_int, _vp]
+                L.avq_gilbert_order.argtypes = [ctypes.c_int, ctypes.c_int, _vp]
                 L.avq_workspace_size.argtypes = [P(avq_dims), ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int]
                 L.avq_workspace_size.restype = ctypes.c_size_t
@@ -82,7 +83,8 @@ def lib() -> ctypes.CDLL:
                 L.avq_status_string.argtypes = [ctypes.c_int]
                 L.avq_version.restype = ctypes.c_int
                 for name in ("avq_quantize", "avq_quantize_noalloc", "avq_attention", "avq_permute",
-                             "avq_hilbert_order", "avq_check_device", "avq_codebook_update"):
+                             "avq_hilbert_order", "avq_gilbert_order", "avq_check_device",
+                             "avq_codebook_update"):
                     getattr(L, name).restype = ctypes.c_int
                 _lib = L
     return _lib
@@ -291,6 +293,14 @@ def avq_hilbert_order(side: int) -> torch.Tensor:
     """Raster index of the t-th cell along a Hilbert curve (host tensor, int32)."""
     out = torch.empty(side * side, dtype=torch.int32)
     _check(lib().avq_hilbert_order(int(side), _vp(out.data_ptr())))
+    return out
+
+
+def avq_gilbert_order(width: int, height: int) -> torch.Tensor:
+    """Raster index (y*width + x) of the t-th cell along a generalised Hilbert
+    curve over a width x height grid (host tensor, int32)."""
+    out = torch.empty(max(1, int(width) * int(height)), dtype=torch.int32)  # sizes checked by the library
+    _check(lib().avq_gilbert_order(int(width), int(height), _vp(out.data_ptr())))
     return out
 
 

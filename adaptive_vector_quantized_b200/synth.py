@@ -41,8 +41,13 @@ CONFIGS = {
                  sigma_c=0.3, two_pass=False),
     "largecb": dict(dtype="bf16", B=1, H=8, N=16384, d=128, M0=256, C=8, P=32, block=128,
                     keys="tree", key_sigma=0.1, sigma_c=0.3, two_pass=True),
+    # the paper's 224 x 224 ViT shape: a 28 x 28 patch grid (N = 784, not a
+    # multiple of the query block) along the generalised Hilbert curve
+    "vit28": dict(dtype="bf16", B=2, H=12, N=784, d=64, M0=64, C=8, P=16, block=128,
+                  keys="regions", grid=(28, 28), key_sigma=0.1, noise=0.0, order="gilbert",
+                  sigma_c=0.3, two_pass=False),
 }
-CONFIG_SEEDS = {"tiny": 1000, "vit": 1001, "long": 1002, "largecb": 1003, "sweep": 1004}
+CONFIG_SEEDS = {"tiny": 1000, "vit": 1001, "long": 1002, "largecb": 1003, "sweep": 1004, "vit28": 1005}
 
 
 def sweep_config(P: int, N: int, order: str = "hilbert", flat192: bool = False) -> dict:
@@ -158,22 +163,32 @@ def _node_vectors(par_f, child_f, h, p, c):
     return out
 
 
-def _region_nodes(rng, side, n_seeds, M0, C, order):
-    """Tree node of every token: Voronoi regions of random seeds on the grid,
-    tokens taken along the requested order (hilbert, raster or random)."""
+def _region_nodes(rng, width, height, n_seeds, M0, C, order):
+    """Tree node of every token: Voronoi regions of random seeds on the
+    width x height grid, tokens taken along the requested order (hilbert
+    (2^k square grids), gilbert (any grid), raster or random)."""
     from scipy.spatial import cKDTree
 
-    seeds = rng.uniform(0.0, side, size=(n_seeds, 2))
+    if width == height:
+        seeds = rng.uniform(0.0, width, size=(n_seeds, 2))
+    else:
+        seeds = rng.uniform(0.0, 1.0, size=(n_seeds, 2)) * np.array([width, height])
     sp, sc = _pick_nodes(rng, n_seeds, M0, C)
-    yy, xx = np.divmod(np.arange(side * side), side)
+    yy, xx = np.divmod(np.arange(width * height), width)
     cells = np.stack([xx + 0.5, yy + 0.5], axis=1)
     _, nearest = cKDTree(seeds).query(cells)
     if order == "hilbert":
-        tok = hilbert_cells(side)
+        if width != height:
+            raise ValueError("the hilbert order needs a square 2^k grid; use gilbert")
+        tok = hilbert_cells(width)
+    elif order == "gilbert":
+        from .order import grid_order
+
+        tok = grid_order(width, height, "gilbert")
     elif order == "raster":
-        tok = np.arange(side * side)
+        tok = np.arange(width * height)
     elif order == "random":
-        tok = rng.permutation(side * side)
+        tok = rng.permutation(width * height)
     else:
         raise ValueError(order)
     return sp[nearest[tok]], sc[nearest[tok]]
@@ -197,17 +212,21 @@ def make_inputs(cfg: dict, seed: int) -> dict:
 
     K = np.empty((B, H, N, d), dtype=np.float32)
     sigma = cfg.get("key_sigma", 0.1)
+    q_gain = float(cfg.get("q_coherent", 0.0))
+    nodes = np.empty((B, H, N, d), dtype=np.float32) if q_gain > 0 else None
     for b in range(B):
         for h in range(H):
             if cfg["keys"] == "regions":
-                side = cfg["side"]
-                assert side * side == N
-                p, c = _region_nodes(rng_key, side, 4 * M0, M0, C, cfg.get("order", "hilbert"))
+                W, Hg = cfg["grid"] if "grid" in cfg else (cfg["side"], cfg["side"])
+                assert W * Hg == N
+                p, c = _region_nodes(rng_key, W, Hg, 4 * M0, M0, C, cfg.get("order", "hilbert"))
             elif cfg["keys"] == "tree":
                 p, c = _pick_nodes(rng_key, N, M0, C)
             else:
                 raise ValueError(cfg["keys"])
             base = _node_vectors(par_f, child_f, h, p, c)
+            if nodes is not None:
+                nodes[b, h] = base
             base += rng_key.standard_normal((N, d), dtype=np.float32) * np.float32(sigma)
             frac = cfg.get("noise", 0.0)
             if frac > 0:
@@ -215,6 +234,8 @@ def make_inputs(cfg: dict, seed: int) -> dict:
                 base[sel] = rng_key.uniform(-3.0, 3.0, size=(int(sel.sum()), d)).astype(np.float32)
             K[b, h] = base
     Q = rng_q.standard_normal((B, H, N, d), dtype=np.float32)
+    if nodes is not None:  # queries that look at their own region: q = g * node + N(0, 1)
+        Q += np.float32(q_gain) * nodes
     V = rng_v.standard_normal((B, H, N, d), dtype=np.float32)
 
     return dict(

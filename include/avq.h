@@ -235,6 +235,19 @@ avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, in
  */
 avq_status avq_hilbert_order(int side, int32_t* idx);
 
+/*
+ * avq_gilbert_order -- host helper: idx[t] = raster index (y*width + x) of the
+ * t-th cell of a generalised Hilbert ("Gilbert") curve over a width x height
+ * grid of any size (Sec. 4.2 and Fig. 3: tokens reordered so that tiles of
+ * consecutive tokens are compact 2-D regions, e.g. the 28 x 28 patch grid).
+ * The curve starts at cell (0, 0), moves one cell up, down, left or right at
+ * every step and visits every cell once; on a 2^k x 2^k grid it is the curve
+ * of avq_hilbert_order.  idx is host memory of width*height int32, the
+ * permutation to pass to avq_permute.  Returns AVQ_ERR_INVALID_ARG for a
+ * non-positive size, width*height > INT32_MAX or a NULL idx.
+ */
+avq_status avq_gilbert_order(int width, int height, int32_t* idx);
+
 /* Bytes of device workspace that avq_quantize and avq_attention need for
  * these arguments (the larger of the two).  0 means none. */
 size_t avq_workspace_size(const avq_dims* dims, avq_dtype dtype, int deterministic,

@@ -44,6 +44,11 @@ CASES = {
     "f32_d128": (_cfg(dtype="f32", N=1500, d=128, M0=24, C=4, P=6, block=64), 16),
     "sweep_p4_random": (synth.sweep_config(4, 4096, "random"), 1004),
     "sweep_p64_hilbert": (synth.sweep_config(64, 4096, "hilbert"), 1004),
+    # 28 x 28 patch grid along the generalised Hilbert curve (784 tokens: a
+    # ragged last query block); the second with queries that look at their
+    # own region, so that blocks select few, heavy parents
+    "vit28": (synth.get_config("vit28"), 1005),
+    "vit28_coherent_q": (synth.get_config("vit28", B=1, q_coherent=1.0), 1005),
 }
 
 
@@ -258,6 +263,13 @@ def test_permute_roundtrip_and_definition():
     X = torch.arange(side * side * 8, dtype=torch.float32).reshape(1, side * side, 8).cuda()
     Y = avq.avq_permute(X, order)
     assert torch.equal(Y.cpu()[0, :, 0] / 8, order.cpu().float())
+    # the 28 x 28 grid along the generalised Hilbert curve, and back
+    order = avq.avq_gilbert_order(28, 28).cuda()
+    X = torch.arange(784 * 8, dtype=torch.float32).reshape(1, 784, 8).cuda()
+    Y = avq.avq_permute(X, order)
+    Z = avq.avq_permute(Y, order, inverse=True)
+    assert torch.equal(Y.cpu()[0, :, 0] / 8, order.cpu().float())
+    assert torch.equal(Z.cpu(), X.cpu())
 
 
 def test_device_error_word_clean():
