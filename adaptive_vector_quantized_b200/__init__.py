@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
                                           ctypes.c_int, _vp]
                 L.avq_hilbert_order.argtypes = [ctypes.c_int, _vp]
                 L.avq_gilbert_order.argtypes = [ctypes.c_int, ctypes.c_int, _vp]
+                L.avq_selftest_wait.argtypes = [ctypes.c_int, _vp]
                 L.avq_workspace_size.argtypes = [P(avq_dims), ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int]
                 L.avq_workspace_size.restype = ctypes.c_size_t
@@ -84,7 +85,7 @@ def lib() -> ctypes.CDLL:
                 L.avq_version.restype = ctypes.c_int
                 for name in ("avq_quantize", "avq_quantize_noalloc", "avq_attention", "avq_permute",
                              "avq_hilbert_order", "avq_gilbert_order", "avq_check_device",
-                             "avq_codebook_update"):
+                             "avq_codebook_update", "avq_selftest_wait"):
                     getattr(L, name).restype = ctypes.c_int
                 _lib = L
     return _lib
@@ -302,6 +303,12 @@ def avq_gilbert_order(width: int, height: int) -> torch.Tensor:
     out = torch.empty(max(1, int(width) * int(height)), dtype=torch.int32)  # sizes checked by the library
     _check(lib().avq_gilbert_order(int(width), int(height), _vp(out.data_ptr())))
     return out
+
+
+def avq_selftest_wait(timeout_us: int = 2000, stream=None):
+    """Launch the bounded-wait self-test: the next avq_check_device raises
+    AVQError with status AVQ_ERR_TIMEOUT."""
+    _check(lib().avq_selftest_wait(int(timeout_us), _stream(stream)))
 
 
 def avq_check_device(stream=None):

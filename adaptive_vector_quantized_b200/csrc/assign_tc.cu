@@ -120,8 +120,17 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
   const uint32_t tmem = *sTmem;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
+  // per barrier, the parity of the phase that thread 0's last copy or MMA on
+  // it completes (bit b of `issued` once there was one): bits 0-1 the K ring
+  // slots, 2 the MMAs, 3 the codebook image; drained on the way out
+  uint32_t issued = 0, exp_par = 0;
+  auto note = [&](int b, uint32_t ph) {
+    issued |= 1u << b;
+    exp_par = (exp_par & ~(1u << b)) | ((ph & 1u) << b);
+  };
   auto issue_k = [&](int t, int slot) {
     const int bh = t / a.nblk, blk = t % a.nblk;
+    note(slot, (uint32_t)((t - t0) >> 1));  // waited at tile t - t0 with parity ((t - t0) >> 1) & 1
     tc::mbar_arrive_expect_tx(&bar_k[slot], kKeys * D * 2);
 #pragma unroll
     for (int kh = 0; kh < KH; ++kh)
@@ -146,6 +155,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     if (h != cur_h) {  // (re)load the head's codebook image and norms
       if (tid == 0) {
         const size_t bytes = S::parents_bytes(M0) + S::children_bytes(M0, C);
+        note(3, ph_cb);
         tc::mbar_arrive_expect_tx(bar_cb, (uint32_t)bytes);
         const bf16* src = a.cw + (size_t)h * Mt * D;
         // parents and (optionally) children are contiguous in the image
@@ -181,6 +191,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         const uint64_t bd = tc::sdesc_sw128(sParA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
         tc::mma_bf16(tmem, ad, bd, idesc, k > 0);
       }
+      note(2, ph_mma);
       tc::mma_commit(bar_mma);
     }
     if (!tc::mbar_wait(bar_mma, ph_mma)) atomicOr(a.err, kErrTimeout);
@@ -266,6 +277,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
                 ++idx;
               }
             }
+            note(2, ph_mma);
             tc::mma_commit(bar_mma);
           }
           if (!tc::mbar_wait(bar_mma, ph_mma)) atomicOr(a.err, kErrTimeout);
@@ -347,6 +359,15 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     if (tid == 0 && t + 2 < t1) issue_k(t + 2, slot);
   }
 
+  // nothing in flight before TMEM is freed (the waits return at once for
+  // completed operations; 1 ms limit)
+  if (issued) {
+    uint64_t* const bars[4] = {&bar_k[0], &bar_k[1], bar_mma, bar_cb};
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if ((issued >> b) & 1u)
+        if (!tc::mbar_wait(bars[b], (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
+  }
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -500,8 +521,19 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   const uint32_t lane_off = (uint32_t)(wwarp * 32) << 16;
   const int barid = 1 + g;
 
-  auto issue_k = [&](int t, int slot) {
-    const int bh = t / a.nblk, blk = t % a.nblk;
+  // per barrier, the parity of the phase that this thread's last copy or MMA
+  // on it completes (bit b of `issued` once there was one): bits 0-1 the K
+  // ring slots, 2 parent MMAs, 3 child MMAs, 4 the codebook image; drained
+  // on the way out
+  uint32_t issued = 0, exp_par = 0;
+  auto note = [&](int b, uint32_t ph) {
+    issued |= 1u << b;
+    exp_par = (exp_par & ~(1u << b)) | ((ph & 1u) << b);
+  };
+  // K tile t for the j-th tile of this warpgroup (ring slot j & 1)
+  auto issue_k = [&](int t, int j) {
+    const int bh = t / a.nblk, blk = t % a.nblk, slot = j & 1;
+    note(slot, (uint32_t)(j >> 1));
     tc::mbar_arrive_expect_tx(&bar_k[slot], (uint32_t)S::kTile);
 #pragma unroll
     for (int kh = 0; kh < KH; ++kh)
@@ -515,8 +547,10 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   uint32_t ph_cb = 0, ph_p = 0, ph_c = 0;
   int cur_h = -1, it = 0;
   bool aborted = false, kerr = false;
-  // parent scores of the K tile in `kslot` into TMEM half `kslot` (norm step last)
-  auto issue_parents = [&](int kslot) {
+  // parent scores of the K tile in `kslot` into TMEM half `kslot` (norm step
+  // last); the j-th tile's MMA completes the phase of parity j & 1
+  auto issue_parents = [&](int kslot, int j) {
+    note(2, (uint32_t)j);
     const uint32_t sKa = tc::smem_u32(sRing + kslot * S::kTile);
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
@@ -536,6 +570,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
     if (h != cur_h) {  // (re)load the head's codebook image and norms, CTA-wide
       if (tid == 0) {
         const size_t bytes = S::cb_bytes(M0, C);
+        note(4, ph_cb);
         tc::mbar_arrive_expect_tx(bar_cb, (uint32_t)bytes);
         const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cw + (size_t)h * Mt * D);
         for (size_t off = 0; off < bytes;) {
@@ -572,13 +607,13 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
     // prologue: K of the first two tiles (thread 0), parent MMA of the first
     // (the parent issuer)
     if (wt == 0 && first < s1) {
-      issue_k(first, it & 1);
-      if (first + nwg < s1) issue_k(first + nwg, (it + 1) & 1);
+      issue_k(first, it);
+      if (first + nwg < s1) issue_k(first + nwg, it + 1);
     }
     if (wt == kParentIssuer && first < s1) {
       if (tc::mbar_wait(&bar_k[it & 1], (it >> 1) & 1)) {
         tc::tc_fence_after();
-        issue_parents(it & 1);
+        issue_parents(it & 1, it);
       } else {
         kerr = true;
       }
@@ -603,7 +638,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
         if (wt == kParentIssuer && t + nwg < s1) {
           if (tc::mbar_wait(&bar_k[slot ^ 1], ((it + 1) >> 1) & 1)) {
             tc::tc_fence_after();
-            issue_parents(slot ^ 1);
+            issue_parents(slot ^ 1, it + 1);
           } else {
             kerr = true;
           }
@@ -611,7 +646,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       };
       if (C == 0) {
         next_parents();
-        if (wt == 0 && t + 2 * nwg < s1) issue_k(t + 2 * nwg, slot);  // K slot read by nothing else
+        if (wt == 0 && t + 2 * nwg < s1) issue_k(t + 2 * nwg, it + 2);  // K slot read by nothing else
       }
 
       // nearest parent = first maximum of T over the M0 parents: eight running
@@ -706,10 +741,11 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
               const uint64_t bd = tc::sdesc_sw128(sStA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
               tc::mma_bf16(tP, ad, bd, idescC, k > 0);
             }
+            note(3, ph_c);
             tc::mma_commit(bar_c);
             if (!tc::mbar_wait(bar_c, ph_c)) atomicOr(a.err, kErrTimeout);
             // last round: the K slot is read by nothing else now
-            if (r0 + kStageAtoms >= np && t + 2 * nwg < s1) issue_k(t + 2 * nwg, slot);
+            if (r0 + kStageAtoms >= np && t + 2 * nwg < s1) issue_k(t + 2 * nwg, it + 2);
           }
           ph_c ^= 1;
           wg_bar(barid);  // child scores in TMEM
@@ -756,6 +792,15 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
     s0 = s1;
   }
 
+  // nothing in flight before TMEM is freed (the waits return at once for
+  // completed operations; 1 ms limit)
+  if (issued) {
+    uint64_t* const bars[5] = {&bar_k[0], &bar_k[1], bar_p, bar_c, bar_cb};
+#pragma unroll
+    for (int b = 0; b < 5; ++b)
+      if ((issued >> b) & 1u)
+        if (!tc::mbar_wait(bars[b], (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
+  }
   tc::tc_fence_before();
   __syncthreads();
   if (tid < 32) {

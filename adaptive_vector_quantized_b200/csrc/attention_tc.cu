@@ -177,7 +177,15 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
   uint32_t ph_cp = 0, ph_mma = 0, ph_vb = 0;
+  // per barrier, the parity of the phase that thread 0's last copy or MMA on
+  // it completes (bit b of `issued` once there was one): drained on the way out
+  uint32_t issued = 0, exp_par = 0;
+  auto note = [&](int b, uint32_t ph) {
+    issued |= 1u << b;
+    exp_par = (exp_par & ~(1u << b)) | (ph << b);
+  };
   if (tid == 0) {
+    note(0, 0);
     tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
 #pragma unroll
     for (int kh = 0; kh < KH; ++kh) tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, row0, bh, bar_q);
@@ -188,6 +196,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
                  sPRa = tc::smem_u32(sPR);
   // S = Q * CW^T over n codes (n a multiple of 16, <= 64) -- one thread
   auto issue_logits = [&](int n) {
+    note(3, ph_mma);
     const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
@@ -199,6 +208,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   };
   // x += PR * VB over n codes -- one thread
   auto issue_values = [&](int n, bool acc) {
+    note(3, ph_mma);
     for (int k = 0; k < n / 16; ++k) {
       const uint64_t ad = tc::sdesc_sw128(sPRa + (k & 3) * 32, 16, 1024);
       const uint64_t bd = tc::sdesc_sw128(sVBa + k * 2 * (KH * 1024), 1024, KH * 1024);
@@ -245,9 +255,11 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       const int n = min(kTile, M0 - c0);
       if (tid == 0) {
         const uint32_t cwb = (uint32_t)n * D * 2;
+        note(1, ph_cp);
         tc::mbar_arrive_expect_tx(bar_cp, cwb);
         tc::bulk_g2s(sCW, cw_h + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
         if (last) {
+          note(2, ph_vb);
           tc::mbar_arrive_expect_tx(bar_vb, cwb);
           tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, cwb, bar_vb);
         }
@@ -426,6 +438,8 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
       const int slots = (np + 1) & ~1;
       const int n = slots * 8;
       if (tid == 0) {
+        note(1, ph_cp);
+        note(2, ph_vb);
         tc::mbar_arrive_expect_tx(bar_cp, 1u * slots * KH * 1024);
         tc::mbar_arrive_expect_tx(bar_vb, 1u * slots * KH * 1024);
         for (int r = 0; r < slots; ++r) {
@@ -541,6 +555,16 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   }
 
 done:
+  // nothing in flight before TMEM is freed (the waits return at once for
+  // completed operations; 1 ms limit)
+  if (issued) {
+    uint64_t* const bars[4] = {bar_q, bar_cp, bar_vb, bar_mma};
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if ((issued >> b) & 1u)
+        if (!tc::mbar_wait(bars[b], (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
+  }
+  if (tid == 0) tc::bulk_wait_group_read0();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -633,19 +657,33 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   const int nch = (C > 0 && P > 0) ? (P + kChunkParents - 1) / kChunkParents : 0;
   auto unit_cw = [&](int u) { return a.cw + (size_t)((u / a.nblk) % a.H) * (Mt / 8) * KH * 512; };
   auto unit_vb = [&](int u) { return a.vb + (size_t)(u / a.nblk) * (Mt / 8) * KH * 512; };
+  // mbarrier phases (the same in every thread), and per barrier the parity
+  // of the phase that the last operation issued by this thread completes
+  // (bit b of `issued` set once one was issued): on the way out the kernel
+  // waits, with a limit, for those, so no copy or MMA is in flight when it
+  // frees TMEM and returns, also after a timed-out wait
+  uint32_t ph_q = 0, ph_cw = 0, ph_vb = 0, ph_mma = 0, ph_x = 0;
+  uint32_t issued = 0, exp_par = 0;
+  auto note = [&](int b, uint32_t ph) {
+    issued |= 1u << b;
+    exp_par = (exp_par & ~(1u << b)) | (ph << b);
+  };
   // the next unit's Q tile and parents' codewords / value sums (thread 0)
   auto load_q = [&](int u) {
+    note(0, ph_q);
     tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
 #pragma unroll
     for (int kh = 0; kh < KH; ++kh)
       tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, (u % a.nblk) * kRows, u / a.nblk, bar_q);
   };
   auto load_pcw = [&](int u) {
+    note(1, ph_cw);
     tc::mbar_arrive_expect_tx(bar_cw, M0 * D * 2 + Mt * 4);
     tc::bulk_g2s(sCW, unit_cw(u), M0 * D * 2, bar_cw);
     tc::bulk_g2s(sm + S::kCNT, a.counts + (size_t)(u / a.nblk) * Mt, Mt * 4, bar_cw);
   };
   auto load_pvb = [&](int u) {
+    note(2, ph_vb);
     tc::mbar_arrive_expect_tx(bar_vb, M0 * D * 2);
     tc::bulk_g2s(sVB, unit_vb(u), M0 * D * 2, bar_vb);
   };
@@ -677,9 +715,9 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     const uint32_t sQa = tc::smem_u32(sQ), sCWa = tc::smem_u32(sCW), sVBa = tc::smem_u32(sVB),
                    sPRa = tc::smem_u32(sPR);
     const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
-    uint32_t ph_q = 0, ph_cw = 0, ph_vb = 0, ph_mma = 0, ph_x = 0;
 
     auto issue_logits = [&](int n) {  // S = Q * CW^T over n codes
+      note(3, ph_mma);
       const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
@@ -690,6 +728,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       tc::mma_commit(bar_mma);
     };
     auto issue_values = [&](int n, bool acc) {  // x (+)= PR * VB over n codes
+      note(4, ph_x);
       for (int k = 0; k < n / 16; ++k) {
         const uint64_t ad = tc::sdesc_sw128(sPRa + (k & 3) * 32, 16, 1024);
         const uint64_t bd = tc::sdesc_sw128(sVBa + k * 2 * AB, 1024, KH * 1024);
@@ -1045,6 +1084,15 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     }  // units
   }
 done:
+  // nothing of this CTA in flight before TMEM is freed: copies and MMAs this
+  // thread issued (the waits return at once for completed ones; 1 ms limit)
+  if (issued) {
+    uint64_t* const bars[5] = {bar_q, bar_cw, bar_vb, bar_mma, bar_x};
+#pragma unroll
+    for (int b = 0; b < 5; ++b)
+      if ((issued >> b) & 1u)
+        if (!tc::mbar_wait(bars[b], (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
+  }
   tc::cp_async_wait<0>();
   if (tid == 0) tc::bulk_wait_group_read0();  // the last O store has read the staging
   tc::tc_fence_before();

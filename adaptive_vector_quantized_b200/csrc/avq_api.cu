@@ -333,6 +333,19 @@ avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, in
   return AVQ_OK;
 }
 
+avq_status avq_selftest_wait(int timeout_us, avq_stream_t stream) {
+  t_error[0] = 0;
+  if (timeout_us < 1 || timeout_us > 1000000)
+    return fail(AVQ_ERR_INVALID_ARG, "timeout_us must be in [1, 1000000] (got %d)", timeout_us);
+  unsigned int* err = error_word();
+  if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+  const cudaError_t e =
+      launch_wait_probe(err, 1000ull * (unsigned long long)timeout_us, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", "wait_probe");
+  return AVQ_OK;
+}
+
 avq_status avq_check_device(avq_stream_t stream) {
   t_error[0] = 0;
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

@@ -248,6 +248,19 @@ avq_status avq_hilbert_order(int side, int32_t* idx);
  */
 avq_status avq_gilbert_order(int width, int height, int32_t* idx);
 
+/*
+ * avq_selftest_wait -- self-test of the failure path of the kernels' bounded
+ * waits: launches one thread that waits on an mbarrier nothing completes.
+ * The wait gives up after timeout_us microseconds (1 .. 1000000), sets the
+ * timeout bit of the device error word and the kernel ends; the next
+ * avq_check_device then returns AVQ_ERR_TIMEOUT and clears the word.  Every
+ * mbarrier wait in the library's kernels takes this path when a copy or MMA
+ * completion does not arrive in time (limit 2 s), and the kernels then finish
+ * without leaving copies or MMAs in flight.  Asynchronous on `stream`;
+ * AVQ_ERR_INVALID_ARG for an out-of-range timeout (before any launch).
+ */
+avq_status avq_selftest_wait(int timeout_us, avq_stream_t stream);
+
 /* Bytes of device workspace that avq_quantize and avq_attention need for
  * these arguments (the larger of the two).  0 means none. */
 size_t avq_workspace_size(const avq_dims* dims, avq_dtype dtype, int deterministic,

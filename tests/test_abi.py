@@ -152,3 +152,10 @@ def test_codebook_update_host_checks():
     assert L.avq_codebook_update(ctypes.byref(d), avq.AVQ_BF16, 0.5, None, *args[1:]) == avq.AVQ_ERR_INVALID_ARG
     assert "ksum" in avq.last_error()
     assert L.avq_codebook_update(None, avq.AVQ_BF16, 0.5, *args) == avq.AVQ_ERR_INVALID_ARG
+
+
+def test_wait_selftest_host_checks():
+    """The bounded-wait self-test rejects an out-of-range limit before any launch."""
+    L = avq.lib()
+    for bad in (0, -5, 1000001):
+        assert L.avq_selftest_wait(bad, None) == avq.AVQ_ERR_INVALID_ARG
