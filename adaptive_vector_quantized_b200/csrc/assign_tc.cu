@@ -412,9 +412,10 @@ struct WgSmem {
   __host__ __device__ static size_t misc_off(int M0, int C, int nwg) {
     return (norms_off(M0, C, nwg) + (size_t)M0 * (1 + C) * 4 + 15) & ~(size_t)15;
   }
-  // barriers: cb + 4 per warpgroup; masks: 4 words per warpgroup; tmem base, abort
+  // barriers: cb + 4 per warpgroup; parent masks: 8 words per warpgroup
+  // ([tile parity][present lo, hi, shared lo, hi]); tmem base, abort
   __host__ __device__ static size_t total(int M0, int C, int nwg) {
-    return misc_off(M0, C, nwg) + 8 * (1 + 4 * nwg) + 16 * nwg + 16;
+    return misc_off(M0, C, nwg) + 8 * (1 + 4 * nwg) + 32 * nwg + 16;
   }
 };
 
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nwg = blockDim.x >> 7;
   const int C = a.C, Mt = M0 * (1 + C);
-  const int tid = threadIdx.x, g = tid >> 7, wt = tid & 127, wwarp = wt >> 5;
+  const int tid = threadIdx.x, g = tid >> 7, wt = tid & 127, wwarp = wt >> 5, lane = tid & 31;
   uint8_t* sPar = sm;
   const uint8_t* sCh = sm + (size_t)M0 * D * 2;
   uint8_t* sRing = sm + S::wg_off(M0, C) + (size_t)g * S::kWg;
@@ -483,8 +484,8 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   uint64_t* bar_p = bar_k + 2;           // parent MMA done
   uint64_t* bar_c = bar_k + 3;           // child MMA done
   uint32_t* sMaskAll = reinterpret_cast<uint32_t*>(bar_cb + 1 + 4 * nwg);
-  uint32_t* sMask = sMaskAll + 4 * g;  // [tile parity][2 words]
-  uint32_t* sTmem = sMaskAll + 4 * nwg;
+  uint32_t* sMask = sMaskAll + 8 * g;  // [tile parity][present lo, hi, shared lo, hi]
+  uint32_t* sTmem = sMaskAll + 8 * nwg;
   int* sAbort = reinterpret_cast<int*>(sTmem + 1);
 
   const int t0 = blockIdx.x * a.tiles_per_cta;
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
     tc::mbar_init(bar_cb, 1);
     for (int w = 0; w < 4 * nwg; ++w) tc::mbar_init(bar_cb + 1 + w, 1);
     tc::fence_mbar_init();
-    for (int w = 0; w < 4 * nwg; ++w) sMaskAll[w] = 0;
+    for (int w = 0; w < 8 * nwg; ++w) sMaskAll[w] = 0;
     *sAbort = 0;
     tc::prefetch_tensormap(&kmap);
   }
@@ -689,26 +690,78 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       }
       int code = par;
       if (C > 0) {  // C == 8 on this path
-        uint32_t* mk = sMask + slot * 2;
+        // the tile's parents: present (some key chose it) and shared (a second
+        // warp of the tile, or a second key of this warp, chose it too)
+        uint32_t* mk = sMask + slot * 4;
+        const bool dup = __popc(__match_any_sync(0xffffffffu, par)) > 1;
         const uint32_t lo = __reduce_or_sync(0xffffffffu, par < 32 ? 1u << par : 0u);
         const uint32_t hi = __reduce_or_sync(0xffffffffu, par >= 32 ? 1u << (par - 32) : 0u);
+        const uint32_t dlo = __reduce_or_sync(0xffffffffu, dup && par < 32 ? 1u << par : 0u);
+        const uint32_t dhi = __reduce_or_sync(0xffffffffu, dup && par >= 32 ? 1u << (par - 32) : 0u);
         if ((wt & 31) == 0) {
-          if (lo) atomicOr(mk, lo);
-          if (hi) atomicOr(mk + 1, hi);
+          const uint32_t olo = lo ? atomicOr(mk, lo) : 0u;
+          const uint32_t ohi = hi ? atomicOr(mk + 1, hi) : 0u;
+          if ((lo & olo) | dlo) atomicOr(mk + 2, (lo & olo) | dlo);
+          if ((hi & ohi) | dhi) atomicOr(mk + 3, (hi & ohi) | dhi);
         }
         tc::tc_fence_before();
-        wg_bar(barid);  // parent set complete, parent scores read
-        if (wt == 0) {  // the other parity's set, for the next tile
-          sMask[(slot ^ 1) * 2] = 0;
-          sMask[(slot ^ 1) * 2 + 1] = 0;
+        wg_bar(barid);  // parent sets complete, parent scores read
+        if (wt == 0) {  // the other parity's sets, for the next tile
+#pragma unroll
+          for (int w = 0; w < 4; ++w) sMask[(slot ^ 1) * 4 + w] = 0;
         }
-        const uint32_t m_lo = mk[0], m_hi = mk[1];
+        // child scores on the tensor cores for every present parent when they
+        // fit one round, else for the shared parents only; the keys of the
+        // other parents (one key each) get theirs on the CUDA cores, while the
+        // child MMA runs
+        const uint32_t p_lo = mk[0], p_hi = mk[1];
+        const bool one_round = __popc(p_lo) + __popc(p_hi) <= kStageAtoms;
+        const uint32_t m_lo = one_round ? p_lo : mk[2], m_hi = one_round ? p_hi : mk[3];
         const int n_lo = __popc(m_lo), np = n_lo + __popc(m_hi);
-        const int myslot = par < 32 ? __popc(m_lo & ((1u << par) - 1u))
-                                    : n_lo + __popc(m_hi & ((1u << (par - 32)) - 1u));
+        const bool in_mma = par < 32 ? ((m_lo >> par) & 1u) != 0 : ((m_hi >> (par - 32)) & 1u) != 0;
+        const int myslot = !in_mma ? -1
+                           : par < 32 ? __popc(m_lo & ((1u << par) - 1u))
+                                      : n_lo + __popc(m_hi & ((1u << (par - 32)) - 1u));
         float vals[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) vals[c] = 0.f;
+        // one key at a time, the warp's 32 lanes take its 8 children x 4
+        // quarters of the dims (bf16 products, fp32 sums), read from the K tile
+        // and the children's atoms in shared memory (128-byte swizzle)
+        auto simt_children = [&]() {
+          unsigned todo = __ballot_sync(0xffffffffu, !in_mma);
+          const int c = lane >> 2, qd = lane & 3;
+          const uint8_t* kt = sRing + slot * S::kTile;
+          while (todo) {
+            const int kl = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const int kp = __shfl_sync(0xffffffffu, par, kl);
+            const int krow = wwarp * 32 + kl;
+            const uint8_t* ch = sCh + (size_t)kp * (KH * 1024);
+            float dot = 0.f;
+#pragma unroll
+            for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int chunk = qd * 2 + h2;
+                const uint4 kv = *reinterpret_cast<const uint4*>(kt + kh * (kKeys * 128) + krow * 128 +
+                                                                 ((chunk ^ (krow & 7)) << 4));
+                const uint4 cv = *reinterpret_cast<const uint4*>(ch + kh * 1024 + c * 128 + ((chunk ^ c) << 4));
+                dot = fma_bf16x2(kv.x, cv.x, dot);
+                dot = fma_bf16x2(kv.y, cv.y, dot);
+                dot = fma_bf16x2(kv.z, cv.z, dot);
+                dot = fma_bf16x2(kv.w, cv.w, dot);
+              }
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+              const float v = __shfl_sync(0xffffffffu, dot, cc * 4);
+              if (lane == kl) vals[cc] = v;
+            }
+          }
+        };
+        if (np == 0) next_parents();  // no child MMA for this tile
         for (int r0 = 0; r0 < np; r0 += kStageAtoms) {
           const int nr = min(kStageAtoms, np - r0);
           const int nat = (nr + 1) & ~1;
@@ -744,11 +797,10 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
             note(3, ph_c);
             tc::mma_commit(bar_c);
             if (!tc::mbar_wait(bar_c, ph_c)) atomicOr(a.err, kErrTimeout);
-            // last round: the K slot is read by nothing else now
-            if (r0 + kStageAtoms >= np && t + 2 * nwg < s1) issue_k(t + 2 * nwg, it + 2);
           }
+          if (r0 == 0) simt_children();
           ph_c ^= 1;
-          wg_bar(barid);  // child scores in TMEM
+          wg_bar(barid);  // child scores in TMEM; the CUDA-core children done
           tc::tc_fence_after();
           // one TMEM load per distinct staging slot among this warp's keys
           const int my = (myslot >= r0 && myslot < r0 + kStageAtoms) ? myslot - r0 : -1;
@@ -769,6 +821,11 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
             wg_bar(barid);  // staging and child columns free for the next round
           }
         }
+        if (np == 0) {
+          simt_children();
+          wg_bar(barid);  // the K tile is read by nothing else
+        }
+        if (wt == 0 && t + 2 * nwg < s1) issue_k(t + 2 * nwg, it + 2);  // K slot free
         float tchild = vals[0] + sNorm[M0 + par * 8];
         int cstar = 0;
 #pragma unroll
