@@ -2,6 +2,7 @@
 """Throughput of the AVQ-Attention forward hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config long] [--impl avq|reference]
+    (--config: a named workload, "sweep:P:N[:order]" or "flat192:N")
 
 One step = stage 1 (avq_quantize: full-tree key quantisation + aggregation)
 and stage 2 (avq_attention: parent attention, top-P per query block, child
@@ -280,6 +281,11 @@ def run_avq(args, cfg, inp, n_global=None):
         return k1, avq.last_kernels()
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # inputs that fit in L2 (126 MB on B200) would be timed warm: write a
+    # buffer of twice the L2 size between timed steps
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    in_bytes = 3 * B * H * N * d * Q.element_size()
+    fbuf = torch.empty(2 * l2_bytes // 4 + 1, dtype=torch.float32, device=dev) if in_bytes < 2 * l2_bytes else None
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
@@ -300,6 +306,8 @@ def run_avq(args, cfg, inp, n_global=None):
         torch.cuda.synchronize(dev)
         t0.record(stream)
         for s in range(args.steps):
+            if fbuf is not None:  # inputs fit in L2: evict them before every timed step
+                fbuf.zero_()
             ev[s][0].record(stream)
             avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
             if exchange:
@@ -313,9 +321,12 @@ def run_avq(args, cfg, inp, n_global=None):
         if world > 1:
             dist.barrier()
     avq.avq_check_device(stream)
-    ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
     t_s1 = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     t_s2 = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    if fbuf is None:
+        ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
+    else:  # the flushes are outside the steps' own events
+        ms = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev), dev, world)
     ms_step = ms / args.steps
     queries = B * H * N * world if n_global is None else B * H * n_global
     value = queries / (ms_step * 1e-3)
@@ -382,14 +393,16 @@ def run_avq(args, cfg, inp, n_global=None):
         cpu = dict(value=q / times[0], unit="queries/s", cores=cores, kind="oracle",
                    sample=f"{heads} head(s) x N={N} of the same workload, b=0: all keys quantised "
                           f"and all queries attended, float64, OpenMP")
+    l2_note = ("inputs larger than L2 (Q, K, V %.0f MB each per step); no flush" % (in_bytes / 3e6)
+               if fbuf is None else
+               "inputs smaller than 2x L2: a %.0f MB buffer written before every timed step, "
+               "outside the step's events" % (fbuf.numel() * 4 / 1e6))
     line = dict(metric=METRIC, value=value, unit="queries/s", n_gpus=world, steps=args.steps,
                 warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
                 scaling="weak" if n_global is None else "strong",
                 vs_baseline=None, dtype=cfg["dtype"], data="synthetic",
                 config=dict(workload_config(args.config, cfg),
-                            l2="inputs larger than L2 (Q, K, V 134 MB each per step); no flush"
-                            if cfg["N"] * cfg["H"] * cfg["B"] * cfg["d"] * 2 > 126e6 else
-                            "inputs smaller than L2; no flush"),
+                            l2=l2_note),
                 roofline=roofline, cpu_baseline=cpu, e2e=e2e,
                 gpu_launches=kernels_per_step * args.steps,
                 clocks=dict(clk.summary() or {}, window=f"sampled every 200 ms over warmup, "
@@ -400,17 +413,39 @@ def run_avq(args, cfg, inp, n_global=None):
     print(json.dumps(line), flush=True)
 
 
+def resolve_config(name):
+    """A named workload, or one point of the P x N sweep: "sweep:P:N[:order]"
+    (H=8, d=64, 64/P/8, order hilbert, raster or random) or the flat
+    192-codeword VQ "flat192:N"."""
+    from adaptive_vector_quantized_b200 import synth
+
+    if name in synth.CONFIGS:
+        return synth.get_config(name)
+    parts = name.split(":")
+    try:
+        if parts[0] == "sweep" and len(parts) in (3, 4):
+            return synth.sweep_config(int(parts[1]), int(parts[2]), parts[3] if len(parts) == 4 else "hilbert")
+        if parts[0] == "flat192" and len(parts) == 2:
+            return synth.sweep_config(0, int(parts[1]), flat192=True)
+    except ValueError as e:
+        raise SystemExit(f"bad config {name}: {e}")
+    raise SystemExit(f"unknown config {name}")
+
+
+def config_seed(name, synth):
+    base = name.split(":")[0]
+    return synth.CONFIG_SEEDS.get(name, synth.CONFIG_SEEDS.get("sweep" if base in ("sweep", "flat192") else base, 1000))
+
+
 def main():
     args = parse()
     from adaptive_vector_quantized_b200 import synth
 
-    cfg = synth.get_config(args.config) if args.config in synth.CONFIGS else None
-    if cfg is None:
-        raise SystemExit(f"unknown config {args.config}")
+    cfg = resolve_config(args.config)
     if args.denominator is not None:
         cfg["two_pass"] = {"auto": 0, "two_pass": 1, "extrapolated": 2}[args.denominator]
     rank = int(os.environ.get("RANK", "0"))
-    seed = rank_seed(args.seed if args.seed is not None else synth.CONFIG_SEEDS.get(args.config, 1000), rank)
+    seed = rank_seed(args.seed if args.seed is not None else config_seed(args.config, synth), rank)
     if args.impl == "reference":
         if rank != 0:
             return
@@ -421,7 +456,7 @@ def main():
         from adaptive_vector_quantized_b200.sharding import shard_rows
 
         world = int(os.environ.get("WORLD_SIZE", "1"))
-        base = args.seed if args.seed is not None else synth.CONFIG_SEEDS.get(args.config, 1000)
+        base = args.seed if args.seed is not None else config_seed(args.config, synth)
         inp = synth.make_inputs(cfg, base)
         n0, n1 = shard_rows(cfg["N"], cfg["block"], rank, world)
         if n1 <= n0:
