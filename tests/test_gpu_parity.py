@@ -49,6 +49,10 @@ CASES = {
     # own region, so that blocks select few, heavy parents
     "vit28": (synth.get_config("vit28"), 1005),
     "vit28_coherent_q": (synth.get_config("vit28", B=1, q_coherent=1.0), 1005),
+    # 80 heads x 8 blocks (the last one partial) = 640 units: more units than
+    # the persistent attention grid has CTAs, so CTAs walk two units each and
+    # some of them end on a partial block; P = 13 pads the second chunk
+    "multi_unit_ragged": (_cfg(H=80, N=1000, P=13), 17),
 }
 
 
