@@ -53,6 +53,11 @@ CASES = {
     # the persistent attention grid has CTAs, so CTAs walk two units each and
     # some of them end on a partial block; P = 13 pads the second chunk
     "multi_unit_ragged": (_cfg(H=80, N=1000, P=13), 17),
+    # d = 128 with one parent tile: the one-tile attention kernel's two
+    # 64-column halves (Q, O, codeword and value atoms), with the children in
+    # shared memory (M0 = 32) or read from L2 (M0 = 64) in the assignment
+    "d128_m64": (_cfg(H=3, N=1536, d=128, M0=64, P=16), 19),
+    "d128_m32_ragged": (_cfg(H=2, N=1000, d=128, M0=32, P=5), 20),
 }
 
 
