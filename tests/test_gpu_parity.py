@@ -58,6 +58,10 @@ CASES = {
     # shared memory (M0 = 32) or read from L2 (M0 = 64) in the assignment
     "d128_m64": (_cfg(H=3, N=1536, d=128, M0=64, P=16), 19),
     "d128_m32_ragged": (_cfg(H=2, N=1000, d=128, M0=32, P=5), 20),
+    "d128_m48": (_cfg(H=2, N=777, d=128, M0=48, P=7), 21),
+    "d128_m16": (_cfg(H=2, N=300, d=128, M0=16, P=3), 22),
+    # two parent tiles at d = 64: the general attention kernel's two sweeps
+    "m0_128_d64": (_cfg(H=2, N=1024, M0=128, P=16), 23),
 }
 
 
