@@ -354,9 +354,12 @@ size_t aggregate_det_workspace(const Shape& s) {
 
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log) {
-  cudaError_t e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * s.Mt() * s.d * sizeof(float), st);
-  if (e != cudaSuccess) return e;
+                             LaunchLog& log, bool vsum_zeroed) {
+  cudaError_t e = cudaSuccess;
+  if (!vsum_zeroed) {
+    e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * s.Mt() * s.d * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+  }
   (void)counts;
   const int sms = num_sms();
   // grid sized for about 32 resident warps per SM, each a contiguous multiple of 32 keys

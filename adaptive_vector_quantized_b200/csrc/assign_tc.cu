@@ -873,7 +873,9 @@ __global__ void __launch_bounds__(256) codebook_prep_kernel(const bf16* __restri
                                                             const bf16* __restrict__ children,
                                                             bf16* __restrict__ cw,
                                                             float* __restrict__ norms, int H, int M0,
-                                                            int C) {
+                                                            int C, uint4* __restrict__ zero_a,
+                                                            long long n_a, uint4* __restrict__ zero_b,
+                                                            long long n_b) {
   constexpr int KH = D / 64;
   constexpr int CH = D / 8;  // 16-byte chunks per code: one thread each
   const int Mt = M0 * (1 + C);
@@ -902,6 +904,16 @@ __global__ void __launch_bounds__(256) codebook_prep_kernel(const bf16* __restri
 #pragma unroll
     for (int o = CH / 2; o >= 1; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
     if (live && chunk == 0) norms[hc] = nrm;
+  }
+  // the stage's accumulators (counts, value sums) start at zero: cleared here
+  // instead of by separate memsets
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_a + n_b;
+       i += (long long)gridDim.x * blockDim.x) {
+    if (i < n_a)
+      zero_a[i] = z;
+    else
+      zero_b[i - n_a] = z;
   }
 }
 
@@ -971,17 +983,23 @@ size_t assign_tc_workspace(const Shape& s) {
 
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents, const void* children,
                              int32_t* assign, int32_t* counts, void* ws, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log) {
+                             LaunchLog& log, float* vsum_to_zero) {
   bf16* cw = static_cast<bf16*>(ws);
   float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
   const long long work = (long long)s.H * s.Mt() * (s.d / 8);
   const int pblocks = (int)std::max<long long>(1, std::min<long long>((work + 255) / 256, num_sms() * 8));
+  // counts (and the value sums when given) are zeroed by the same launch; both
+  // are 16-byte aligned and a whole number of 16-byte words (M0 % 16 == 0)
+  const long long n_counts = (long long)s.BH() * s.Mt() * 4 / 16;
+  const long long n_vsum = vsum_to_zero ? (long long)s.BH() * s.Mt() * s.d * 4 / 16 : 0;
+  uint4* zc = reinterpret_cast<uint4*>(counts);
+  uint4* zv = reinterpret_cast<uint4*>(vsum_to_zero);
   if (s.d == 64)
     codebook_prep_kernel<64><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
-                                                      s.H, s.M0, s.C);
+                                                      s.H, s.M0, s.C, zc, n_counts, zv, n_vsum);
   else
     codebook_prep_kernel<128><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
-                                                       s.H, s.M0, s.C);
+                                                       s.H, s.M0, s.C, zc, n_counts, zv, n_vsum);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   log.add("codebook_prep");

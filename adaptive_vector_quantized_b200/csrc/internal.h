@@ -35,7 +35,7 @@ cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, cons
 // vsum is zeroed inside; counts are left to the assignment kernels.
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log);
+                             LaunchLog& log, bool vsum_zeroed = false);
 // Deterministic aggregation (fixed-order sums, independent of the grid).
 size_t aggregate_det_workspace(const Shape& s);
 cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
@@ -46,9 +46,12 @@ cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
 // C in {0, 8}); needs assign_tc_workspace(s) bytes of workspace.
 bool assign_tc_supported(const Shape& s, avq_dtype dt);
 size_t assign_tc_workspace(const Shape& s);
+// Zeroes counts itself (and vsum when vsum_to_zero is given) before the
+// assignment adds into them.
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
                              const void* children, int32_t* assign, int32_t* counts, void* ws,
-                             unsigned int* err, cudaStream_t st, LaunchLog& log);
+                             unsigned int* err, cudaStream_t st, LaunchLog& log,
+                             float* vsum_to_zero = nullptr);
 
 // ---- stage 2 ------------------------------------------------------------
 cudaError_t launch_attention_simt(const Shape& s, avq_dtype dt, const void* Q, const void* parents,
