@@ -329,14 +329,27 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
       const uint8_t* atom = reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + par * 8) * D);
       float dchild = INF;
       int cstar = 0;
-      for (int c = 0; c < 8; ++c) {
-        float acc = 0.f;
+      // child c + 1's row is loaded while child c's dot product is summed
+      uint4 cb[2][KH][8];
+      auto load_child = [&](int c, uint4 (&dst)[KH][8]) {
 #pragma unroll
         for (int kh = 0; kh < KH; ++kh)
 #pragma unroll
           for (int s = 0; s < 8; ++s) {
             const int lc = (s + rot) & 7;
-            const uint4 cv = __ldg(reinterpret_cast<const uint4*>(atom + kh * 1024 + c * 128 + ((lc ^ c) << 4)));
+            dst[kh][s] = __ldg(reinterpret_cast<const uint4*>(atom + kh * 1024 + c * 128 + ((lc ^ c) << 4)));
+          }
+      };
+      load_child(0, cb[0]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c + 1 < 8) load_child(c + 1, cb[(c + 1) & 1]);
+        float acc = 0.f;
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint4 cv = cb[c & 1][kh][s];
             acc = fma_bf16x2(kq[kh][s].x, cv.x, acc);
             acc = fma_bf16x2(kq[kh][s].y, cv.y, acc);
             acc = fma_bf16x2(kq[kh][s].z, cv.z, acc);
