@@ -67,3 +67,24 @@ def test_reference_arm_rank0_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_config_names():
+    """Named workloads, sweep points and the flat 192-codeword VQ resolve to
+    the generator's configs; unknown or malformed names stop the bench."""
+    import pytest
+
+    import bench
+    from adaptive_vector_quantized_b200 import synth
+
+    assert bench.resolve_config("long") == synth.get_config("long")
+    c = bench.resolve_config("sweep:64:4096:random")
+    assert (c["P"], c["N"], c["order"], c["H"], c["M0"], c["C"]) == (64, 4096, "random", 8, 64, 8)
+    assert bench.resolve_config("sweep:4:16384")["order"] == "hilbert"
+    f = bench.resolve_config("flat192:65536")
+    assert (f["M0"], f["C"], f["P"]) == (192, 0, 0)
+    assert bench.config_seed("sweep:4:16384", synth) == synth.CONFIG_SEEDS["sweep"]
+    assert bench.config_seed("vit28", synth) == synth.CONFIG_SEEDS["vit28"]
+    for bad in ("nope", "sweep:4", "sweep:x:4096", "sweep:4:1000"):
+        with pytest.raises(SystemExit):
+            bench.resolve_config(bad)
