@@ -14,6 +14,7 @@
 // order by one warp, and parent totals are formed as stay + children in a
 // fixed order.  Nothing depends on the grid or the GPU's size.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -124,33 +125,45 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     // run starts relative to the previous key (lane 0 compares with the open run)
     const unsigned newR = __ballot_sync(0xffffffffu, code >= 0 && (lane == 0 ? code != cur : prevc != code));
     // keys in sub-batches of 8: the next sub-batch's rows are loaded while the
-    // current one is walked (16 rows in flight per warp, few registers)
-    typename F::R raw[8], nxt[8];
-#pragma unroll
-    for (int b = 0; b < 8; ++b)
-      if (b < nlive) raw[b] = F::load(vb + (size_t)(g + b) * D);
-#pragma unroll 1
-    for (int b0 = 0; b0 < nlive; b0 += 8) {
+    // current one is walked (16 rows in flight per warp, few registers); a
+    // full group of 32 keys takes a copy of the walk without per-key bounds
+    auto walk = [&](auto full_t) {
+      constexpr bool kFull = decltype(full_t)::value;
+      const int n = kFull ? 32 : nlive;
+      const T* rows = vb + (size_t)g * D;
+      typename F::R raw[8], nxt[8];
 #pragma unroll
       for (int b = 0; b < 8; ++b)
-        if (b0 + 8 + b < nlive) nxt[b] = F::load(vb + (size_t)(g + b0 + 8 + b) * D);
+        if (kFull || b < n) raw[b] = F::load(rows + (size_t)b * D);
+#pragma unroll 1
+      for (int b0 = 0; b0 < n; b0 += 8) {
+        const bool more = b0 + 8 < n;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        const int u = b0 + b;
-        if (u < nlive) {
-          float v[E];
-          F::unpack(raw[b], v);
-          if ((newR >> u) & 1u) {
-            if (cur >= 0) flush();
-            cur = __shfl_sync(0xffffffffu, code, u);
+        for (int b = 0; b < 8; ++b)
+          if (kFull ? more : b0 + 8 + b < n) nxt[b] = F::load(rows + (size_t)(b0 + 8 + b) * D);
+        const unsigned starts = (newR >> b0) & 0xffu;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          const int u = b0 + b;
+          if (kFull || u < n) {
+            float v[E];
+            F::unpack(raw[b], v);
+            if ((starts >> b) & 1u) {
+              if (cur >= 0) flush();
+              cur = __shfl_sync(0xffffffffu, code, u);
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[b & 1][e] += v[e];
           }
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[b & 1][e] += v[e];
         }
-      }
 #pragma unroll
-      for (int b = 0; b < 8; ++b) raw[b] = nxt[b];
-    }
+        for (int b = 0; b < 8; ++b) raw[b] = nxt[b];
+      }
+    };
+    if (nlive == 32)
+      walk(std::true_type{});
+    else
+      walk(std::false_type{});
   }
   if (cur >= 0) flush();
 }
