@@ -316,46 +316,65 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         if (tid < 4) sPairs[tid] = 0;  // for the next tile (read by everyone above)
       }
     } else if (C > 0) {  // C == 8; children from L2, dot products on the CUDA cores
-      // key row in registers, 16-byte chunks in rotated order
-      const int rot = tid & 7;
-      uint4 kq[KH][8];
+      // one key at a time, the warp's 32 lanes take its 8 children x 4 parts
+      // of the dims (so each child row is read by four neighbouring lanes,
+      // coalesced), the next key's child rows in flight meanwhile; the key's
+      // row comes from the K tile in shared memory (128-byte swizzle)
+      const int wl = tid & 31, cl = wl >> 2, ql = wl & 3;
+      const int warp_row0 = (tid >> 5) * 32;
+      auto child_row = [&](int pk) {
+        return reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + pk * 8) * D) + cl * 128;
+      };
+      uint4 cur[KH][2], nxt[KH][2];
+      auto load_rows = [&](const uint8_t* rowp, uint4 (&dst)[KH][2]) {
 #pragma unroll
-      for (int kh = 0; kh < KH; ++kh)
+        for (int kh = 0; kh < KH; ++kh)
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int lc = (s + rot) & 7;
-          kq[kh][s] = *reinterpret_cast<const uint4*>(sK + kh * (kKeys * 128) + tid * 128 + ((lc ^ rot) << 4));
+          for (int h2 = 0; h2 < 2; ++h2)
+            dst[kh][h2] = __ldg(reinterpret_cast<const uint4*>(rowp + kh * 1024 + (((2 * ql + h2) ^ cl) << 4)));
+      };
+      load_rows(child_row(__shfl_sync(0xffffffffu, par, 0)), cur);
+      float vals[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) vals[c] = 0.f;
+#pragma unroll 2
+      for (int k = 0; k < 32; ++k) {
+        const int pn = __shfl_sync(0xffffffffu, par, (k + 1) & 31);
+        if (k + 1 < 32) load_rows(child_row(pn), nxt);
+        const int krow = warp_row0 + k;
+        float dot = 0.f;
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const uint4 kv = *reinterpret_cast<const uint4*>(sK + kh * (kKeys * 128) + krow * 128 +
+                                                             (((2 * ql + h2) ^ (krow & 7)) << 4));
+            const uint4 cv = cur[kh][h2];
+            dot = fma_bf16x2(kv.x, cv.x, dot);
+            dot = fma_bf16x2(kv.y, cv.y, dot);
+            dot = fma_bf16x2(kv.z, cv.z, dot);
+            dot = fma_bf16x2(kv.w, cv.w, dot);
+          }
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const float v = __shfl_sync(0xffffffffu, dot, cc * 4);
+          if (wl == k) vals[cc] = v;
         }
-      const uint8_t* atom = reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + par * 8) * D);
+        if (k + 1 < 32) {
+#pragma unroll
+          for (int kh = 0; kh < KH; ++kh) {
+            cur[kh][0] = nxt[kh][0];
+            cur[kh][1] = nxt[kh][1];
+          }
+        }
+      }
       float dchild = INF;
       int cstar = 0;
-      // child c + 1's row is loaded while child c's dot product is summed
-      uint4 cb[2][KH][8];
-      auto load_child = [&](int c, uint4 (&dst)[KH][8]) {
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh)
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const int lc = (s + rot) & 7;
-            dst[kh][s] = __ldg(reinterpret_cast<const uint4*>(atom + kh * 1024 + c * 128 + ((lc ^ c) << 4)));
-          }
-      };
-      load_child(0, cb[0]);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        if (c + 1 < 8) load_child(c + 1, cb[(c + 1) & 1]);
-        float acc = 0.f;
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh)
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const uint4 cv = cb[c & 1][kh][s];
-            acc = fma_bf16x2(kq[kh][s].x, cv.x, acc);
-            acc = fma_bf16x2(kq[kh][s].y, cv.y, acc);
-            acc = fma_bf16x2(kq[kh][s].z, cv.z, acc);
-            acc = fma_bf16x2(kq[kh][s].w, cv.w, acc);
-          }
-        const float dc = fmaf(-2.f, acc, sNorm[M0 + par * 8 + c]);
+        const float dc = fmaf(-2.f, vals[c], sNorm[M0 + par * 8 + c]);
         if (dc < dchild) {
           dchild = dc;
           cstar = c;
