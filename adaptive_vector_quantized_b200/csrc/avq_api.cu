@@ -2,6 +2,7 @@
 // the host before anything is enqueued; a failed check launches nothing.
 #include <math.h>
 #include <stdarg.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -27,6 +28,19 @@ avq_status fail(avq_status s, const char* fmt, ...) {
   vsnprintf(t_error, sizeof(t_error), fmt, ap);
   va_end(ap);
   return s;
+}
+
+// Host-side fault injection for tests of the callers' error handling: when
+// the environment variable AVQ_FAULT names an entry point ("quantize",
+// "attention", "codebook_update", "permute") or is "all", that call returns
+// AVQ_ERR_CUDA after its argument checks and before anything reaches the GPU.
+bool injected(const char* entry) {
+  const char* v = getenv("AVQ_FAULT");
+  if (v == nullptr || *v == 0) return false;
+  return strcmp(v, "all") == 0 || strcmp(v, entry) == 0;
+}
+avq_status injected_fail(const char* entry) {
+  return fail(AVQ_ERR_CUDA, "injected failure before launch (AVQ_FAULT=%s, %s)", getenv("AVQ_FAULT"), entry);
 }
 
 avq_status cuda_fail(cudaError_t e, const char* where) {
@@ -216,6 +230,7 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
     if (st != AVQ_OK) return st;
   }
   void* ws_det_ptr = ws_det ? static_cast<char*>(ws) + ws_tc : nullptr;
+  if (injected("quantize")) return injected_fail("avq_quantize");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   LaunchLog log{};
   cudaError_t e;
@@ -273,6 +288,7 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, c
   // parent tiles, which only the tensor-core kernel sweeps
   if (two_pass == 2 && s.M0 > 64 && !use_tc)
     return fail(AVQ_ERR_UNSUPPORTED, "the extrapolated denominator needs the tensor-core kernel");
+  if (injected("attention")) return injected_fail("avq_attention");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   LaunchLog log{};
   cudaError_t e;
@@ -306,6 +322,7 @@ avq_status avq_codebook_update(const avq_dims* dims, avq_dtype dtype, float lamb
   AVQ_REQUIRE_PTR(Nst, "Nst");
   AVQ_REQUIRE_PTR(parents, "parents");
   if (s.C > 0) AVQ_REQUIRE_PTR(children, "children");
+  if (injected("codebook_update")) return injected_fail("avq_codebook_update");
   LaunchLog log{};
   cudaError_t e = launch_codebook_update(s, dtype, lambda, ksum, counts, S, Nst, parents, children,
                                          reinterpret_cast<cudaStream_t>(stream), log);
@@ -328,6 +345,7 @@ avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, in
   const char* x = static_cast<const char*>(X);
   const char* y = static_cast<const char*>(Y);
   if (x < y + bytes && y < x + bytes) return fail(AVQ_ERR_INVALID_ARG, "X and Y overlap");
+  if (injected("permute")) return injected_fail("avq_permute");
   LaunchLog log{};
   cudaError_t e = launch_permute(X, idx, Y, batch, rows, row_bytes, inverse,
                                  reinterpret_cast<cudaStream_t>(stream), log);
@@ -416,6 +434,7 @@ extern "C" avq_status avq_quantize_noalloc(const avq_dims* dims, avq_dtype dtype
   if (t_path == AVQ_PATH_TC && !tc_ok)
     return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core assignment kernel for this shape/dtype");
   const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
+  if (injected("quantize")) return injected_fail("avq_quantize_noalloc");
   void* scratch = nullptr;
   if (use_tc) {
     const size_t need = assign_tc_workspace(s);

@@ -23,6 +23,11 @@
  *     AVQ_ERR_CUDA means a launch was rejected by the CUDA runtime.  Faults
  *     detected inside kernels (a bounded wait that ran out) are recorded in
  *     the device error word and reported by avq_check_device.
+ *   - Fault injection for tests of a caller's error handling: if the
+ *     environment variable AVQ_FAULT is "quantize", "attention",
+ *     "codebook_update", "permute" or "all", the named entry points return
+ *     AVQ_ERR_CUDA after their argument checks, before any launch (nothing
+ *     reaches the GPU).  Unset or empty: no effect.
  *   - Layouts are dense row-major.  BH = B*H; tensor [B,H,N,d] puts head
  *     (b,h) at offset (b*H+h)*N*d.  Device pointers must be 16-byte aligned.
  *   - Codebook: one per head, shared by the batch (Algorithm 1 input

@@ -159,3 +159,33 @@ def test_wait_selftest_host_checks():
     L = avq.lib()
     for bad in (0, -5, 1000001):
         assert L.avq_selftest_wait(bad, None) == avq.AVQ_ERR_INVALID_ARG
+
+
+def test_fault_injection_before_launch(monkeypatch):
+    """AVQ_FAULT makes the named entry points fail after their argument checks
+    and before any launch (host only: nothing reaches a GPU)."""
+    import ctypes
+
+    L = avq.lib()
+    fake = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced
+    d = avq.avq_dims(1, 2, 256, 64, 16, 8)
+    calls = {
+        "quantize": lambda: L.avq_quantize(ctypes.byref(d), avq.AVQ_BF16, fake, fake, fake, fake, fake,
+                                           fake, fake, 0, fake, ctypes.c_size_t(1 << 40), None),
+        "attention": lambda: L.avq_attention(ctypes.byref(d), avq.AVQ_BF16, fake, fake, fake, fake, fake,
+                                             4, 128, ctypes.c_float(0.125), 0, fake, fake, None, fake,
+                                             ctypes.c_size_t(1 << 40), None),
+        "codebook_update": lambda: L.avq_codebook_update(ctypes.byref(d), avq.AVQ_BF16, ctypes.c_float(0.9),
+                                                         fake, fake, fake, fake, fake, fake, None),
+        "permute": lambda: L.avq_permute(fake, fake, ctypes.c_void_p(0x20000000), 1, 64, 128, 0, None),
+    }
+    for entry, call in calls.items():
+        monkeypatch.setenv("AVQ_FAULT", entry)
+        assert call() == avq.AVQ_ERR_CUDA, entry
+        assert "injected" in avq.last_error()
+    monkeypatch.setenv("AVQ_FAULT", "all")
+    for entry, call in calls.items():
+        assert call() == avq.AVQ_ERR_CUDA, entry
+    # argument checks still come first
+    monkeypatch.setenv("AVQ_FAULT", "all")
+    assert L.avq_permute(None, fake, fake, 1, 64, 128, 0, None) == avq.AVQ_ERR_INVALID_ARG

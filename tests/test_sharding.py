@@ -90,3 +90,46 @@ def test_sharded_statistics_and_output_two_ranks():
     for rank, ok_counts, err_vs, err_o, _ in res:
         assert ok_counts, f"rank {rank}: counts differ"
         assert err_vs < 1e-12 and err_o < 1e-12, (rank, err_vs, err_o)
+
+
+def _failing_worker(rank, world, port, q):
+    """Rank 1 leaves between steps (an exception before the statistics
+    exchange); rank 0 must learn of it from its collective, within the
+    process group's short timeout, instead of waiting for ever."""
+    import datetime
+
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    from adaptive_vector_quantized_b200.sharding import allreduce_stats
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        q.put((1, "left"))
+        raise SystemExit(3)  # no destroy_process_group: the rank is simply gone
+    vs = torch.ones(1, 2, 80, 64, dtype=torch.float64)
+    ns = torch.ones(1, 2, 80, dtype=torch.int64)
+    try:
+        allreduce_stats(vs, ns)
+        q.put((0, "no error"))
+    except Exception as e:  # the failure surfaces as an error of the collective
+        q.put((0, "error: " + type(e).__name__))
+
+
+def test_a_lost_rank_surfaces_as_an_error():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+            p.join(timeout=10)
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res[0]
+    assert procs[1].exitcode == 3
