@@ -346,8 +346,10 @@ avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, in
   const char* y = static_cast<const char*>(Y);
   if (x < y + bytes && y < x + bytes) return fail(AVQ_ERR_INVALID_ARG, "X and Y overlap");
   if (injected("permute")) return injected_fail("avq_permute");
+  unsigned int* err = error_word();
+  if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
   LaunchLog log{};
-  cudaError_t e = launch_permute(X, idx, Y, batch, rows, row_bytes, inverse,
+  cudaError_t e = launch_permute(X, idx, Y, batch, rows, row_bytes, inverse, err,
                                  reinterpret_cast<cudaStream_t>(stream), log);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);

@@ -74,8 +74,9 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
 cudaError_t launch_codebook_update(const Shape& s, avq_dtype dt, float lambda, const float* ksum,
                                    const int32_t* counts, float* S, float* Nst, void* parents,
                                    void* children, cudaStream_t st, LaunchLog& log);
+// Indices outside [0, rows) are skipped and set kErrBounds in err.
 cudaError_t launch_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
-                           int row_bytes, int inverse, cudaStream_t st, LaunchLog& log);
+                           int row_bytes, int inverse, unsigned int* err, cudaStream_t st, LaunchLog& log);
 
 // 3-D tiled TMA map over a bf16 tensor [batch][rows][inner] (inner contiguous),
 // box {box_inner, box_rows, 1}, 128-byte swizzle, zero fill out of bounds.

@@ -13,7 +13,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ 
                                                       const int32_t* __restrict__ idx,
                                                       uint4* __restrict__ Y, int rows,
                                                       int vec_per_row, int inverse,
-                                                      long long total) {
+                                                      long long total, unsigned int* err) {
   for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
        g += (long long)gridDim.x * blockDim.x) {
     const int v = (int)(g % vec_per_row);
@@ -21,6 +21,10 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ 
     const int i = (int)(br % rows);
     const long long b = br / rows;
     const int j = __ldg(idx + i);
+    if ((unsigned)j >= (unsigned)rows) {  // an index outside the rows: refused, reported
+      if (v == 0) atomicOr(err, kErrBounds);
+      continue;
+    }
     const long long src = inverse ? br : b * rows + j;
     const long long dst = inverse ? b * rows + j : br;
     Y[dst * vec_per_row + v] = __ldg(X + src * vec_per_row + v);
@@ -30,14 +34,14 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ 
 }  // namespace
 
 cudaError_t launch_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
-                           int row_bytes, int inverse, cudaStream_t st, LaunchLog& log) {
+                           int row_bytes, int inverse, unsigned int* err, cudaStream_t st, LaunchLog& log) {
   const int vpr = row_bytes / 16;
   const long long total = (long long)batch * rows * vpr;
   long long blocks = (total + 255) / 256;
   const long long cap = (long long)num_sms() * 8;
   if (blocks > cap) blocks = cap;
   permute_kernel<<<(unsigned)blocks, 256, 0, st>>>((const uint4*)X, idx, (uint4*)Y, rows, vpr,
-                                                   inverse, total);
+                                                   inverse, total, err);
   log.add("permute");
   return cudaGetLastError();
 }

@@ -227,7 +227,10 @@ avq_status avq_codebook_update(const avq_dims* dims, avq_dtype dtype, float lamb
  * inverse == 0: Y[b, i] = X[b, idx[i]]  (gather into curve order)
  * inverse != 0: Y[b, idx[i]] = X[b, i]  (scatter back)
  * row_bytes must be a positive multiple of 16; X and Y must not overlap.
- * idx is not checked for being a permutation on the device.
+ * On the device, an index outside [0, rows) is refused (that row is not
+ * copied) and sets the bounds bit of the device error word, which the next
+ * avq_check_device reports as AVQ_ERR_DEVICE; an in-range idx that is not a
+ * permutation is not detected.
  */
 avq_status avq_permute(const void* X, const int32_t* idx, void* Y, int batch, int rows,
                        int row_bytes, int inverse, avq_stream_t stream);
