@@ -16,10 +16,11 @@
 //               16 pairs); each thread then loads the 8 columns of its own
 //               parent (one TMEM load per distinct pair in its warp).  When
 //               the children do not fit in shared memory they are read from
-//               L2 and the dot products are bf16 x bf16 -> fp32 fused
-//               multiply-adds on the CUDA cores.  Either way the key moves
-//               to the first strictly smallest child only if it is strictly
-//               closer than the parent
+//               L2, one key at a time per warp (8 children x 4 parts of the
+//               dims over the lanes, coalesced, the next key's rows in
+//               flight), as bf16 x bf16 -> fp32 fused multiply-adds on the
+//               CUDA cores.  Either way the key moves to the first strictly
+//               smallest child only if it is strictly closer than the parent
 //   output      assign[key] = parent, or M0 + parent*C + child
 // Codewords are first converted into the swizzled-atom image shared with
 // the attention kernel (8 codes x 64 dims per 1024-byte atom) plus their
@@ -417,7 +418,10 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
 // Children of a tile: the child atoms of the parents that some key chose are
 // gathered (in index order, up to 8 per round) into a contiguous staging
 // operand, so one MMA chain of N = 8 x (atoms, rounded up to even) gives every
-// key its dot products with all those children.
+// key its dot products with all those children.  When those parents need more
+// than one round, only the parents that two or more of the tile's keys chose
+// are gathered, and the keys of the others get their 8 child dot products on
+// the CUDA cores (a warp per key) while the MMA runs.
 // Scores: T = k.c - |c|^2 / 2 orders the codewords of a key like the squared
 // distance |k|^2 - 2 T, reversed.  For the parents the -|p|^2 / 2 term is
 // folded into the MMA as one more K step: A holds 1, 1, 1 in its first three
