@@ -116,6 +116,46 @@ def pin_aggregate(orc):
             assert (counts[..., M0:].sum(-1) == moved.sum(-1)).all()
 
 
+def pin_aggregate_given_codes(orc):
+    """The aggregation of Algorithm 1 for codes made elsewhere (the checker of
+    GPU statistics, Eq. 3): a parent holds every key of its cluster, a child
+    only the keys that moved to it.
+    - hand-made code lists with the statistics written out by hand, one with
+      children (including a code of the last child) and one flat (C = 0);
+    - brute-force aggregation of the oracle's own codes on the seeded cases;
+    - Algorithm 1's own statistics when given Algorithm 1's codes."""
+    # M0 = 3, C = 2: children of parent m are codes 3 + 2m and 4 + 2m.
+    codes = np.array([0, 3, 4, 8, 2, 5, 1, 8, 7], dtype=np.int32)
+    N = codes.size
+    V = np.stack([2.0 ** np.arange(N), -np.arange(N, dtype=np.float64)], -1)[None, None]
+    vs, ns = orc.aggregate(codes[None, None], V, 3, 2)
+    # parents: 0 <- keys 0,1,2; 1 <- keys 5,6; 2 <- keys 3,4,7,8
+    # children: 3 <- key 1; 4 <- key 2; 5 <- key 5; 7 <- key 8; 8 <- keys 3,7
+    want_n = [3, 2, 4, 1, 1, 1, 0, 1, 2]
+    want_v = {0: [1 + 2 + 4, -(0 + 1 + 2)], 1: [32 + 64, -(5 + 6)],
+              2: [8 + 16 + 128 + 256, -(3 + 4 + 7 + 8)], 3: [2, -1], 4: [4, -2],
+              5: [32, -5], 6: [0, 0], 7: [256, -8], 8: [8 + 128, -(3 + 7)]}
+    assert ns[0, 0].tolist() == want_n, ns
+    for x, v in want_v.items():
+        assert vs[0, 0, x].tolist() == [float(t) for t in v], (x, vs[0, 0, x])
+    # flat codebook: M0 = 4, C = 0
+    flat = np.array([3, 0, 3, 1], dtype=np.int32)
+    Vf = np.arange(8, dtype=np.float64).reshape(1, 1, 4, 2)
+    vs, ns = orc.aggregate(flat[None, None], Vf, 4, 0)
+    assert ns[0, 0].tolist() == [1, 1, 0, 2]
+    assert vs[0, 0].tolist() == [[2, 3], [6, 7], [0, 0], [0 + 4, 1 + 5]]
+    for mk in CASES:
+        inp = mk()
+        M0, C = inp["M0"], inp["C"]
+        assign, vsum_q, counts_q, _ = orc.quantize(inp["K"], inp["V"], inp["parents"], inp["children"])
+        vs, ns = orc.aggregate(assign, inp["V"], M0, C)
+        vs_ref, ns_ref = brute.aggregate_brute(assign, inp["V"], M0, C)
+        assert (ns == ns_ref).all(), mk.__name__
+        assert _rel(vs, vs_ref) < 1e-12, mk.__name__
+        assert (ns == counts_q).all(), mk.__name__
+        assert _rel(vs, vsum_q) < 1e-12, mk.__name__
+
+
 def pin_representative(orc):
     """Sec. C identity: AVQ output equals exact softmax attention over the
     representative keys, for several P including P = M0."""
@@ -471,7 +511,8 @@ def pin_codebook_massless(orc):
     assert np.allclose(po[0, 1], ksum[0, 0, 1] / 4)
 
 
-ALL_PINS = [pin_hand_worked, pin_assign_brute, pin_aggregate, pin_representative,
+ALL_PINS = [pin_hand_worked, pin_assign_brute, pin_aggregate, pin_aggregate_given_codes,
+            pin_representative,
             pin_rescale_exercised, pin_flat_p0, pin_exact_codebook, pin_importance, pin_topp,
             pin_relabel, pin_key_permutation, pin_keys_on_codewords, pin_strict_ties,
             pin_masking, pin_counting, pin_tiled_importance, pin_codebook_update,

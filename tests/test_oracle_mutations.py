@@ -16,6 +16,14 @@ MUTANTS = [
     ("child-tie-to-last", "if (dc < d_child) { /* where", "if (dc <= d_child) { /* where"),
     ("parent-tie-to-last", "if (dm < d_best) {", "if (dm <= d_best) {"),
     ("child-count-dropped", "ns[code] += 1;\n      }\n      assign", "\n      }\n      assign"),
+    ("aggregate-child-count-dropped", "ns[code] += 1;\n      }\n    }\n  }\n}",
+     "\n      }\n    }\n  }\n}"),
+    ("aggregate-child-sum-to-parent",
+     "vs[(size_t)code * d + t] += v[t];\n        ns[code] += 1;\n      }\n    }\n  }\n}",
+     "vs[(size_t)a * d + t] += v[t];\n        ns[code] += 1;\n      }\n    }\n  }\n}"),
+    ("aggregate-parent-of-child-wrong",
+     "int32_t a = code < M0 ? code : (code - M0) / C;\n      const double* v",
+     "int32_t a = code < M0 ? code : (code - M0) % C;\n      const double* v"),
     ("child-index-transposed", "ch_h + ((size_t)a * C + c) * d", "ch_h + ((size_t)c * M0 + a) * d"),
     ("dA-sign", "exp(sc[c] - m[r]) - Ap", "Ap - exp(sc[c] - m[r])"),
     ("no-rescale", "double f = exp(m[r] - mp);", "double f = 1.0;"),
