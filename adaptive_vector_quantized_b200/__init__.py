@@ -139,6 +139,20 @@ def _stream(stream):
     return _vp(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _expect(t, name, shape, dtype, device):
+    """Raise unless `t` is a contiguous CUDA tensor of this shape, dtype and device."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} (all tensors on one GPU)")
+
+
 def _dims(Q_like: torch.Tensor, parents: torch.Tensor, children) -> avq_dims:
     B, H, N, d = Q_like.shape
     Hp, M0, dp = parents.shape
@@ -165,12 +179,27 @@ def workspace(dims: avq_dims, dtype: int, device, deterministic=False, two_pass=
     return torch.empty(n + 256, dtype=torch.uint8, device=device)
 
 
-def _ws_ptr(ws):
+def _ws_ptr(ws, device=None):
     if ws is None:
         return None, 0
+    if device is not None and ws.device != device:
+        raise ValueError(f"workspace is on {ws.device}, expected {device}")
     p = ws.data_ptr()
     off = (-p) % 256
     return _vp(p + off), ws.numel() - off
+
+
+def _check_stage1(K, V, parents, children, assign, vsum, counts, Mt):
+    """Shapes, dtypes and devices of stage 1's tensors: every tensor on K's
+    device, V like K, codebook in K's dtype, outputs of the stated layout."""
+    B, H, N, d = K.shape
+    dev = K.device
+    _expect(V, "V", K.shape, K.dtype, dev)
+    _expect(parents, "parents", parents.shape, K.dtype, dev)
+    _expect(children, "children", children.shape if children is not None else (), K.dtype, dev)
+    _expect(assign, "assign", (B, H, N), torch.int32, dev)
+    _expect(vsum, "vsum", (B, H, Mt, d), torch.float32, dev)
+    _expect(counts, "counts", (B, H, Mt), torch.int32, dev)
 
 
 def avq_quantize(K, V, parents, children, assign=None, vsum=None, counts=None,
@@ -183,6 +212,7 @@ def avq_quantize(K, V, parents, children, assign=None, vsum=None, counts=None,
     B, H, N, d = K.shape
     Mt = dims.M0 * (1 + dims.C)
     dev = K.device
+    _check_stage1(K, V, parents, children, assign, vsum, counts, Mt)
     if assign is None:
         assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
     if vsum is None:
@@ -191,10 +221,11 @@ def avq_quantize(K, V, parents, children, assign=None, vsum=None, counts=None,
         counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
     if ws is None:
         ws = workspace(dims, dt, dev, deterministic=deterministic)
-    wp, wn = _ws_ptr(ws)
-    _check(lib().avq_quantize(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
-                              _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
-                              int(bool(deterministic)), wp, wn, _stream(stream)))
+    wp, wn = _ws_ptr(ws, dev)
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(lib().avq_quantize(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
+                                  _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
+                                  int(bool(deterministic)), wp, wn, _stream(stream)))
     return assign, vsum, counts
 
 
@@ -208,15 +239,17 @@ def avq_quantize_noalloc(K, V, parents, children, assign=None, vsum=None, counts
     B, H, N, d = K.shape
     Mt = dims.M0 * (1 + dims.C)
     dev = K.device
+    _check_stage1(K, V, parents, children, assign, vsum, counts, Mt)
     if assign is None:
         assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
     if vsum is None:
         vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
     if counts is None:
         counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
-    _check(lib().avq_quantize_noalloc(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
-                                      _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
-                                      _stream(stream)))
+    with torch.cuda.device(dev):  # the scratch array and the launch are the current device's
+        _check(lib().avq_quantize_noalloc(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents),
+                                          _ptr(children), _ptr(assign), _ptr(vsum), _ptr(counts),
+                                          _stream(stream)))
     return assign, vsum, counts
 
 
@@ -233,6 +266,15 @@ def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, 
     dev = Q.device
     if scale is None:
         scale = d ** -0.5
+    Mt = dims.M0 * (1 + dims.C)
+    _expect(parents, "parents", parents.shape, Q.dtype, dev)
+    _expect(children, "children", children.shape if children is not None else (), Q.dtype, dev)
+    _expect(vsum, "vsum", (B, H, Mt, d), torch.float32, dev)
+    _expect(counts, "counts", (B, H, Mt), torch.int32, dev)
+    _expect(O, "O", Q.shape, Q.dtype, dev)
+    _expect(sel, "sel", (B, H, nblk, max(P, 0)), torch.int32, dev)
+    if isinstance(importance, torch.Tensor):
+        _expect(importance, "importance", (B, H, nblk, dims.M0), torch.float32, dev)
     if O is None:
         O = torch.empty_like(Q)
     if sel is None:
@@ -244,11 +286,12 @@ def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, 
         imp = torch.empty((B, H, nblk, dims.M0), dtype=torch.float32, device=dev)
     if ws is None:
         ws = workspace(dims, dt, dev, two_pass=two_pass, P=P, block=block)
-    wp, wn = _ws_ptr(ws)
-    _check(lib().avq_attention(ctypes.byref(dims), dt, _ptr(Q), _ptr(parents), _ptr(children),
-                               _ptr(vsum), _ptr(counts), int(P), int(block), float(scale),
-                               int(two_pass), _ptr(O), _ptr(sel) if P > 0 else None,
-                               _ptr(imp), wp, wn, _stream(stream)))
+    wp, wn = _ws_ptr(ws, dev)
+    with torch.cuda.device(dev):
+        _check(lib().avq_attention(ctypes.byref(dims), dt, _ptr(Q), _ptr(parents), _ptr(children),
+                                   _ptr(vsum), _ptr(counts), int(P), int(block), float(scale),
+                                   int(two_pass), _ptr(O), _ptr(sel) if P > 0 else None,
+                                   _ptr(imp), wp, wn, _stream(stream)))
     return O, sel, imp
 
 
@@ -266,12 +309,16 @@ def avq_codebook_update(ksum, counts, S, Nst, parents, children, lam: float, str
         raise ValueError("children must be [H, M0, C, d]")
     dims = avq_dims(B, H, 1, d, M0, C)
     dt = _dtype_code(parents)
-    for t, want in ((ksum, torch.float32), (S, torch.float32), (Nst, torch.float32), (counts, torch.int32)):
-        if t.dtype != want:
-            raise TypeError(f"expected {want}, got {t.dtype}")
-    _check(lib().avq_codebook_update(ctypes.byref(dims), dt, float(lam), _ptr(ksum), _ptr(counts),
-                                     _ptr(S), _ptr(Nst), _ptr(parents), _ptr(children),
-                                     _stream(stream)))
+    dev = parents.device
+    _expect(ksum, "ksum", (B, H, Mt, d), torch.float32, dev)
+    _expect(counts, "counts", (B, H, Mt), torch.int32, dev)
+    _expect(S, "S", (H, Mt, d), torch.float32, dev)
+    _expect(Nst, "Nst", (H, Mt), torch.float32, dev)
+    _expect(children, "children", (H, M0, C, d), parents.dtype, dev)
+    with torch.cuda.device(dev):
+        _check(lib().avq_codebook_update(ctypes.byref(dims), dt, float(lam), _ptr(ksum), _ptr(counts),
+                                         _ptr(S), _ptr(Nst), _ptr(parents), _ptr(children),
+                                         _stream(stream)))
     return S, Nst, parents, children
 
 
@@ -281,12 +328,13 @@ def avq_permute(X, idx, inverse=False, Y=None, stream=None):
     rows = X.shape[-2]
     batch = X.numel() // (rows * X.shape[-1])
     row_bytes = X.shape[-1] * X.element_size()
+    _expect(idx, "idx", (rows,), torch.int32, X.device)
+    _expect(Y, "Y", X.shape, X.dtype, X.device)
     if Y is None:
         Y = torch.empty_like(X)
-    if idx.dtype != torch.int32:
-        raise TypeError("idx must be int32")
-    _check(lib().avq_permute(_ptr(X), _ptr(idx), _ptr(Y), int(batch), int(rows), int(row_bytes),
-                             int(bool(inverse)), _stream(stream)))
+    with torch.cuda.device(X.device):
+        _check(lib().avq_permute(_ptr(X), _ptr(idx), _ptr(Y), int(batch), int(rows), int(row_bytes),
+                                 int(bool(inverse)), _stream(stream)))
     return Y
 
 

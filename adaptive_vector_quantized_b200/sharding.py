@@ -38,11 +38,12 @@ def allreduce_stats(vsum, counts, group=None):
 
 
 def sharded_forward(Q, K, V, parents, children, P: int, block: int = 128, scale=None,
-                    two_pass=0, group=None, stream=None):
+                    two_pass=0, group=None, stream=None, importance=False):
     """Both stages on this rank's slices Q, K, V [B,H,n_local,d] (cut by
     `shard_rows`), with the statistics summed over `group` in between.
     Returns (assign, vsum, counts, O, sel): local codes, global statistics,
-    local output and selections."""
+    local output and selections; with `importance` also the local blocks'
+    importances [B,H,nblk_local,M0] as a sixth item."""
     import torch
 
     import adaptive_vector_quantized_b200 as avq
@@ -56,9 +57,14 @@ def sharded_forward(Q, K, V, parents, children, P: int, block: int = 128, scale=
         counts = torch.zeros((B, H, Mt), dtype=torch.int32, device=K.device)
         allreduce_stats(vsum, counts, group)
         empty = torch.empty((B, H, 0), dtype=torch.int32, device=K.device)
-        return empty, vsum, counts, Q, torch.empty((B, H, 0, P), dtype=torch.int32, device=K.device)
+        out = (empty, vsum, counts, Q, torch.empty((B, H, 0, P), dtype=torch.int32, device=K.device))
+        if importance:
+            out += (torch.empty((B, H, 0, M0), dtype=torch.float32, device=K.device),)
+        return out
     assign, vsum, counts = avq.avq_quantize(K, V, parents, children, stream=stream)
     allreduce_stats(vsum, counts, group)
-    O, sel, _ = avq.avq_attention(Q, parents, children, vsum, counts, P, block, scale=scale,
-                                  two_pass=two_pass, stream=stream)
+    O, sel, imp = avq.avq_attention(Q, parents, children, vsum, counts, P, block, scale=scale,
+                                    two_pass=two_pass, stream=stream, importance=importance)
+    if importance:
+        return assign, vsum, counts, O, sel, imp
     return assign, vsum, counts, O, sel

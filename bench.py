@@ -12,7 +12,11 @@ Metric: queries/s = B*H*N per step / step time, whole job over all ranks
 collective on the data path).  Rank 0 prints one JSON line.
 
 `--impl reference` times the float64 CPU oracle instead, on a bounded sample
-of the same workload (rank 0 only).
+of the same workload (rank 0 only): min(H, host cores) heads of one batch.
+
+`--gpus N` with N > 1, run without a distributed launcher, starts N ranks
+itself (torch.distributed.run on 127.0.0.1); under a launcher the world size
+must equal N.
 """
 from __future__ import annotations
 
@@ -185,6 +189,9 @@ def cpu_oracle_sample(inp, heads, steps=1):
     import oracle
 
     orc = oracle.default()
+    # every host core (a distributed launcher sets OMP_NUM_THREADS=1 per rank;
+    # the oracle runs on rank 0 alone)
+    orc.set_threads(max(1, os.cpu_count() or 1))
     Kh = inp["K"][:1, :heads]
     Vh = inp["V"][:1, :heads]
     Qh = inp["Q"][:1, :heads]
@@ -207,16 +214,19 @@ def run_reference(args, cfg, inp):
         return
     import oracle  # noqa: F401  (the reference arm is the oracle)
 
-    heads = 1
+    heads = inp["H"]  # min(H, host cores): the oracle's stage 1 parallelises over heads
     queries, times, cores = cpu_oracle_sample(inp, heads, steps=args.warmup + args.steps)
     timed = times[args.warmup:]
     t = sum(timed)
     value = queries * len(timed) / t
-    sample = f"{heads} head(s) x N={inp['N']}: all keys quantised and all queries attended per step"
+    sample = (f"{heads} of the workload's {cfg['H']} heads x N={inp['N']} (b=0): all keys quantised "
+              f"and all queries attended per step, float64, OpenMP")
+    rcfg = dict(workload_config(args.config, cfg), B=1, H=heads, heads_of_workload=cfg["H"],
+                batches_of_workload=cfg["B"])
     line = dict(metric=METRIC, value=value, unit="queries/s", n_gpus=args.gpus, steps=args.steps,
                 warmup=args.warmup, ms_per_step=1e3 * t / len(timed), higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
-                config=workload_config(args.config, cfg),
+                config=rcfg,
                 cpu_baseline=dict(value=value, unit="queries/s", cores=cores, kind="oracle",
                                   sample=sample),
                 e2e=dict(value=value, unit="queries/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
@@ -437,8 +447,35 @@ def config_seed(name, synth):
     return synth.CONFIG_SEEDS.get(name, synth.CONFIG_SEEDS.get("sweep" if base in ("sweep", "flat192") else base, 1000))
 
 
+def launch_ranks(args):
+    """`--gpus N` with N > 1 outside a distributed launch: start N ranks (one
+    per GPU) with torch.distributed.run on this node and return its exit code."""
+    import socket
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__)] + sys.argv[1:]
+    try:
+        return subprocess.run(cmd, timeout=1800).returncode
+    except subprocess.TimeoutExpired:
+        print("bench: the ranks did not finish within 30 minutes", file=sys.stderr)
+        return 124
+
+
 def main():
     args = parse()
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        raise SystemExit(launch_ranks(args))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        print(f"bench: --gpus {args.gpus} but the launch has {world} rank(s)", file=sys.stderr)
+        raise SystemExit(2)
     from adaptive_vector_quantized_b200 import synth
 
     cfg = resolve_config(args.config)
@@ -449,7 +486,8 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        inp = synth.make_inputs(dict(cfg, B=1, H=1), seed)
+        heads = min(cfg["H"], max(1, os.cpu_count() or 1))
+        inp = synth.make_inputs(dict(cfg, B=1, H=heads), seed)
         run_reference(args, cfg, inp)
         return
     if args.shard == "tokens":  # same inputs on every rank, each takes its slice of the tokens

@@ -97,8 +97,10 @@ typedef enum {
  *   counts [B,H,Mt]   int32  key counts n with the same membership
  * Inputs (device): K, V [B,H,N,d]; parents [H,M0,d]; children [H,M0,C,d]
  * (may be NULL when C == 0), all of `dtype`.
- * deterministic != 0 makes vsum bitwise reproducible from run to run and
- * independent of the GPU's size (fixed-order reduction; needs workspace).
+ * deterministic != 0 makes vsum the sequential fp32 sum of each code's keys
+ * in key order (a parent: the keys that stayed, then its children in child
+ * order), which no launch shape enters: bitwise reproducible from run to run
+ * and independent of the GPU's size (needs workspace).
  * Workspace: `ws` (device, 256-byte aligned) of at least
  * avq_workspace_size(...) bytes; may be NULL when that size is 0.
  */

@@ -76,10 +76,16 @@ class Oracle:
         lib.avq_oracle_codebook_update.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_D] * 8
         lib.avq_oracle_codebook_update.restype = None
         lib.avq_oracle_num_threads.restype = ctypes.c_int
+        lib.avq_oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.avq_oracle_set_threads.restype = None
         self.lib = lib
 
     def num_threads(self) -> int:
         return int(self.lib.avq_oracle_num_threads())
+
+    def set_threads(self, n: int) -> None:
+        """Threads of the oracle's OpenMP loops (a launcher may have set 1)."""
+        self.lib.avq_oracle_set_threads(int(n))
 
     # ---- Algorithm 1 ---------------------------------------------------
     def quantize(self, K, V, parents, children):

@@ -374,6 +374,16 @@ int avq_oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the parallel loops above (host plumbing, no arithmetic). */
+void avq_oracle_set_threads(int n) {
+#ifdef _OPENMP
+  extern void omp_set_num_threads(int);
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /*
  * Codebook update of Sec. A ("Codeword Clustering During Training").
  * EMA statistics (Eq. 11), one set per head over the keys of every batch

@@ -153,3 +153,38 @@ def importance_brute(Q, parents, counts, block, scale):
             for blk in range(nblk):
                 W[b, h, blk] = mass[blk * block:(blk + 1) * block].sum(axis=0)
     return W
+
+
+def parent_attention_mass(Q, K, codes, M0, C, block, scale):
+    """True attention mass per parent and query block [B,H,nblk,M0]: the sum
+    over the block's queries i of the exact softmax weights (Eq. 1, scaled
+    logits, all N keys) of the keys whose parent is j.  Dividing the mass of
+    a set of parents by the block's row count gives the "capture" of the
+    pages' Table 5 (Sec. B) and Table 6: the fraction of true attention
+    weight that falls on keys assigned to the selected parents."""
+    Q, K = _f64(Q), _f64(K)
+    codes = np.asarray(codes)
+    B, H, N, d = Q.shape
+    nblk = (N + block - 1) // block
+    W = np.zeros((B, H, nblk, M0))
+    for b in range(B):
+        for h in range(H):
+            c = codes[b, h]
+            par = np.where(c < M0, c, (c - M0) // max(C, 1))
+            onehot = np.zeros((N, M0))
+            onehot[np.arange(N), par] = 1.0
+            for blk in range(nblk):
+                q = Q[b, h, blk * block:(blk + 1) * block]
+                p = _softmax_rows(scale * q @ K[b, h].T)  # [nI, N]
+                W[b, h, blk] = p.sum(axis=0) @ onehot
+    return W
+
+
+def top_p_capture(mass, sel, N, block):
+    """Mean over blocks of (sum of the selected parents' true mass) / |I|."""
+    mass = np.asarray(mass)
+    sel = np.asarray(sel)
+    nblk = mass.shape[-2]
+    sizes = np.array([min(block, N - k * block) for k in range(nblk)], dtype=np.float64)
+    got = np.take_along_axis(mass, sel.astype(np.int64), axis=-1).sum(-1)  # [B,H,nblk]
+    return float(np.mean(got / sizes))

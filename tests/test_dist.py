@@ -56,9 +56,14 @@ def test_max_over_ranks_gloo():
 def test_reference_arm_rank0_only():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--config", "tiny", "--steps", "1", "--warmup", "1"],
+                        "--config", "tiny", "--steps", "1", "--warmup", "1", "--gpus", "2"],
                        capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+    # a launch whose world size is not --gpus is refused
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--config", "tiny", "--steps", "1", "--warmup", "1", "--gpus", "4"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode != 0 and "rank" in r.stderr
     env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--config", "tiny", "--steps", "1", "--warmup", "1", "--gpus", "2"],
@@ -67,6 +72,20 @@ def test_reference_arm_rank0_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_spawns_its_own_ranks():
+    """`--gpus 2` without a launcher starts two ranks itself; the reference
+    arm then prints one line from rank 0 with n_gpus = 2."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--config", "tiny", "--steps", "1", "--warmup", "1", "--gpus", "2"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
 
 
 def test_bench_config_names():

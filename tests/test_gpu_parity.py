@@ -235,26 +235,35 @@ def test_deterministic_mode(inputs):
     assert "det_" in a["kernels"]
 
 
-def test_deterministic_matches_fixed_order_sum(inputs):
+@pytest.mark.parametrize("case", ["tiny", "multi_chunk"])
+def test_deterministic_matches_fixed_order_sum(inputs, case):
     """The deterministic value sums are the plain sequential fp32 sums of each
-    (parent, child) segment in key order, and parents add stay + children."""
-    inp = inputs("tiny")
+    (parent, child) segment in key order, and parents add stay + children.
+    That definition names no launch shape, so equality with it on a case of
+    several sort chunks, heads and batches (N = 5000, d = 128) is what makes
+    the result independent of the GPU's size."""
+    if case == "tiny":
+        inp = inputs("tiny")
+    else:
+        inp = synth.make_inputs(_cfg(B=2, H=2, N=5000, d=128, M0=32, P=8), 21)
     a = gh.gpu_forward(inp, deterministic=True)
-    V = inp["V"].numpy().astype(np.float32)
-    codes = a["assign"][0, 0]
+    V = inp["V"].float().numpy().astype(np.float32)
     M0, C = inp["M0"], inp["C"]
-    seg = {}
-    for j, code in enumerate(codes):
-        key = int(code)
-        acc = seg.get(key, np.zeros(V.shape[-1], dtype=np.float32))
-        seg[key] = np.float32(acc + V[0, 0, j])
-    for p in range(M0):
-        tot = seg.get(p, np.zeros(V.shape[-1], dtype=np.float32))
-        for c in range(C):
-            ch = seg.get(M0 + p * C + c, np.zeros(V.shape[-1], dtype=np.float32))
-            assert np.array_equal(a["vsum"][0, 0, M0 + p * C + c], ch)
-            tot = np.float32(tot + ch)
-        assert np.array_equal(a["vsum"][0, 0, p], tot)
+    zero = np.zeros(V.shape[-1], dtype=np.float32)
+    for b in range(inp["B"]):
+        for h in range(inp["H"]):
+            codes = a["assign"][b, h]
+            seg = {}
+            for j, code in enumerate(codes):
+                key = int(code)
+                seg[key] = np.float32(seg.get(key, zero) + V[b, h, j])
+            for p in range(M0):
+                tot = seg.get(p, zero)
+                for c in range(C):
+                    ch = seg.get(M0 + p * C + c, zero)
+                    assert np.array_equal(a["vsum"][b, h, M0 + p * C + c], ch)
+                    tot = np.float32(tot + ch)
+                assert np.array_equal(a["vsum"][b, h, p], tot)
 
 
 def test_permute_roundtrip_and_definition():
@@ -283,6 +292,46 @@ def test_permute_roundtrip_and_definition():
     Z = avq.avq_permute(Y, order, inverse=True)
     assert torch.equal(Y.cpu()[0, :, 0] / 8, order.cpu().float())
     assert torch.equal(Z.cpu(), X.cpu())
+
+
+def test_permute_refuses_out_of_range_indices():
+    """An index outside [0, rows) is not followed: its row is skipped and the
+    bounds bit of the device error word is set (reported as AVQ_ERR_DEVICE and
+    cleared by the check).  X and Y are views into larger buffers, so even a
+    check that failed to skip would only touch mapped memory."""
+    avq.avq_check_device()
+    rows, cols, batch = 300, 64, 2
+    big_x = torch.randn(batch, rows + 8, cols, dtype=torch.float32, device="cuda")
+    X = big_x[:, :rows].contiguous()
+    idx_h = torch.randperm(rows, dtype=torch.int64).to(torch.int32)
+    bad_at = (17, 203)
+    idx_h[bad_at[0]] = rows   # one past the end
+    idx_h[bad_at[1]] = -1     # negative
+    idx = idx_h.cuda()
+    sentinel = -12345.0
+    for inverse in (False, True):
+        Y = torch.full_like(X, sentinel)
+        avq.avq_permute(X, idx, inverse=inverse, Y=Y)
+        with pytest.raises(avq.AVQError) as ei:
+            avq.avq_check_device()
+        assert ei.value.status == avq.AVQ_ERR_DEVICE
+        avq.avq_check_device()  # the word was cleared
+        Xc, Yc = X.cpu(), Y.cpu()
+        ok = [i for i in range(rows) if i not in bad_at]
+        for b in range(batch):
+            for i in ok:
+                j = int(idx_h[i])
+                if inverse:
+                    assert torch.equal(Yc[b, j], Xc[b, i])
+                else:
+                    assert torch.equal(Yc[b, i], Xc[b, j])
+            if inverse:  # the destinations the bad entries would have named stay untouched
+                missing = sorted(set(range(rows)) - {int(idx_h[i]) for i in ok})
+                for j in missing:
+                    assert bool((Yc[b, j] == sentinel).all())
+            else:
+                for i in bad_at:
+                    assert bool((Yc[b, i] == sentinel).all())
 
 
 def test_device_error_word_clean():
