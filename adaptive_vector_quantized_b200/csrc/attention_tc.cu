@@ -35,6 +35,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_util.cuh"
+#include "fastmath.cuh"
 
 namespace avq {
 
@@ -619,6 +620,11 @@ struct FastSmem {
 // waits that thread 0 and warp 0 take care of.
 constexpr int kValueIssuer = 96;
 
+// Of each selected parent's 8 child exponentials, the first 2 * kPolyPairs
+// are evaluated on the FMA pipe (fm::exp2_poly2), the others on the
+// special-function unit, so that neither pipe alone bounds the child pass.
+constexpr int kPolyPairs = 1;
+
 template <int D, int M0>
 __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap, const AttnArgs a) {
@@ -632,7 +638,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   uint8_t* sVB = sm + S::kVB;
   uint8_t* sPR = sm + S::kPR;
   float* sNF = reinterpret_cast<float*>(sm + S::kNF);  // [0..63] parents, [64..127] current chunk
-  float* sW = reinterpret_cast<float*>(sm + S::kW);
+  uint32_t* sKEY = reinterpret_cast<uint32_t*>(sm + S::kW);  // importance ranking keys [64]
   float* sWP = reinterpret_cast<float*>(sm + S::kWP);
   int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
   int* sRK = reinterpret_cast<int*>(sm + S::kRK);
@@ -649,6 +655,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   const int C = a.C, Mt = M0 * (1 + C), P = a.P;
   const float NEG_INF = __int_as_float(0xff800000);
   const float sl2 = a.scale_log2;
+  const float2 sl2x2 = fm::f2(sl2, sl2);
   // this CTA's contiguous range of units u = bh * nblk + block
   const int total = a.BH * a.nblk;
   const int per = (total + gridDim.x - 1) / gridDim.x;
@@ -801,29 +808,31 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       // then A = 2^(t - m) (to PR in bf16, and back over the logits in fp32 for
       // the importance, which needs 1 / z of the whole row)
       const float4* nf4 = reinterpret_cast<const float4*>(sNF);
-      float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+      float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
       for (int g = 0; g < M0 / 16; ++g) {
         uint32_t r[16];
         tc::tmem_ld16(tS + lane_off + g * 16, r);
         tc::tmem_wait_ld();
+        const float* t = reinterpret_cast<const float*>(r);
         if (!any_empty) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(r[e]));
+          for (int e = 0; e < 16; e += 4) {
+            mx0 = fm::max3(mx0, t[e], t[e + 1]);
+            mx1 = fm::max3(mx1, t[e + 2], t[e + 3]);
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             const float4 nf = nf4[(g * 16 + e) >> 2];
-            mx[0] = fmaxf(mx[0], nf.x > 0.f ? __uint_as_float(r[e]) : NEG_INF);
-            mx[1] = fmaxf(mx[1], nf.y > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
-            mx[2] = fmaxf(mx[2], nf.z > 0.f ? __uint_as_float(r[e + 2]) : NEG_INF);
-            mx[3] = fmaxf(mx[3], nf.w > 0.f ? __uint_as_float(r[e + 3]) : NEG_INF);
+            mx0 = fm::max3(mx0, nf.x > 0.f ? t[e] : NEG_INF, nf.y > 0.f ? t[e + 1] : NEG_INF);
+            mx1 = fm::max3(mx1, nf.z > 0.f ? t[e + 2] : NEG_INF, nf.w > 0.f ? t[e + 3] : NEG_INF);
           }
         }
       }
-      m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
-      const float nm = -m;
-      float zp[4] = {0.f, 0.f, 0.f, 0.f};
+      m = fmaxf(mx0, mx1) * sl2;
+      const float2 nm2 = fm::f2(-m, -m);
+      float2 zp = fm::f2(0.f, 0.f);
       auto a_pass = [&](auto masked_t) {
         constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
@@ -834,14 +843,21 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             const float4 nf = nf4[(g * 16 + e) >> 2];
-            const float nfv[4] = {nf.x, nf.y, nf.z, nf.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              float av = tc::ex2(fmaf(__uint_as_float(r[e + k]), sl2, nm));
-              if (kMasked && !(nfv[k] > 0.f)) av = 0.f;
-              zp[k] = fmaf(av, nfv[k], zp[k]);
-              r[e + k] = __float_as_uint(av);
+            const float2 x01 = fm::fma2(fm::f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), sl2x2, nm2);
+            const float2 x23 = fm::fma2(fm::f2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), sl2x2, nm2);
+            float a0 = tc::ex2(x01.x), a1 = tc::ex2(x01.y), a2 = tc::ex2(x23.x), a3 = tc::ex2(x23.y);
+            if (kMasked) {
+              a0 = nf.x > 0.f ? a0 : 0.f;
+              a1 = nf.y > 0.f ? a1 : 0.f;
+              a2 = nf.z > 0.f ? a2 : 0.f;
+              a3 = nf.w > 0.f ? a3 : 0.f;
             }
+            zp = fm::fma2(fm::f2(a0, a1), fm::f2(nf.x, nf.y), zp);
+            zp = fm::fma2(fm::f2(a2, a3), fm::f2(nf.z, nf.w), zp);
+            r[e] = __float_as_uint(a0);
+            r[e + 1] = __float_as_uint(a1);
+            r[e + 2] = __float_as_uint(a2);
+            r[e + 3] = __float_as_uint(a3);
           }
           store_chunk8(sPR, tid, g * 16, reinterpret_cast<const float*>(r));
           store_chunk8(sPR, tid, g * 16 + 8, reinterpret_cast<const float*>(r) + 8);
@@ -853,27 +869,75 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       else
         a_pass(std::false_type{});
       tc::tmem_wait_st();
-      z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
-      // importance column sums of A / z (Eq. 7), fp32
+      z = zp.x + zp.y;
+      // importance column sums of A / z (Eq. 7), fp32.  The A values are read
+      // back in the 16x256b shape, in which each thread holds two adjacent
+      // columns of four rows of its warp (rows l/4, l/4 + 8 of each 16-lane
+      // half); the four rows' 1/z are scaled in, then a three-step butterfly
+      // reduce-scatter over the lanes that share l % 4 leaves lane l holding
+      // the warp's sums of columns 2l and 2l + 1.
       const float rz = valid ? 1.f / z : 0.f;
+      const int rl = lane >> 2;
+      const float z0 = __shfl_sync(0xffffffffu, rz, rl), z1 = __shfl_sync(0xffffffffu, rz, rl + 8),
+                  z2 = __shfl_sync(0xffffffffu, rz, rl + 16), z3 = __shfl_sync(0xffffffffu, rz, rl + 24);
+      float2 cs[8];
 #pragma unroll
-      for (int g = 0; g < (M0 + 31) / 32; ++g) {
-        uint32_t r[32];
-        tc::tmem_ld16(tS + lane_off + g * 32, r);
-        if (g * 32 + 16 < M0) tc::tmem_ld16(tS + lane_off + g * 32 + 16, r + 16);
-        tc::tmem_wait_ld();
-        float v[32];
+      for (int hcol = 0; hcol < 2; ++hcol) {
+        if (hcol * 32 < M0) {
+          uint32_t r[16];
+          fm::tmem_ld_16x256b_x4(tS + lane_off + hcol * 32, r);  // rows l/4, l/4 + 8
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = (g * 32 + e < M0) ? __uint_as_float(r[e]) * rz : 0.f;
-        sWP[warp * 64 + g * 32 + lane] = reduce_scatter32(v, lane);
+          for (int k = 0; k < 4; ++k) {
+            const int grp = hcol * 4 + k;
+            float2 s = fm::mul2(fm::f2(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1])), fm::f2(z0, z0));
+            cs[grp] = fm::fma2(fm::f2(__uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3])), fm::f2(z1, z1), s);
+          }
+          fm::tmem_ld_16x256b_x4(tS + lane_off + (16u << 16) + hcol * 32, r);  // rows 16 + l/4, 24 + l/4
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int grp = hcol * 4 + k;
+            float2 s = fm::fma2(fm::f2(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1])), fm::f2(z2, z2), cs[grp]);
+            s = fm::fma2(fm::f2(__uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3])), fm::f2(z3, z3), s);
+            cs[grp] = grp * 8 < M0 ? s : fm::f2(0.f, 0.f);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) cs[hcol * 4 + k] = fm::f2(0.f, 0.f);
+        }
       }
+      // reduce-scatter: lane bit 4 splits groups 0-3 / 4-7, bit 3 the pairs,
+      // bit 2 the last two; lane l ends with group l / 4
+#pragma unroll
+      for (int step = 0; step < 3; ++step) {
+        const int half = 4 >> step, bit = 16 >> step;
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float2 send = up ? cs[i] : cs[i + half];
+          const float2 keep = up ? cs[i + half] : cs[i];
+          const float rx = __shfl_xor_sync(0xffffffffu, send.x, bit);
+          const float ry = __shfl_xor_sync(0xffffffffu, send.y, bit);
+          cs[i] = fm::add2(keep, fm::f2(rx, ry));
+        }
+      }
+      *reinterpret_cast<float2*>(sWP + warp * 64 + 2 * lane) = cs[0];
     }
     tc::fence_proxy_async_smem();
     wait_bar(bar_vb, ph_vb);
     tc::tc_fence_before();
     __syncthreads();
     if (*sAbort) goto done;
-    if (tid < M0) sW[tid] = nfj * ((sWP[tid] + sWP[64 + tid]) + (sWP[128 + tid] + sWP[192 + tid]));
+    // ranking key of parent j: its importance with the 6 lowest mantissa bits
+    // replaced by 63 - j (importances are >= 0, so the unsigned order of the
+    // bits is the order of the values; equal values rank the lower index
+    // first).  The importance reported is the key's value part (relative
+    // change below 2^-17).
+    if (tid < M0) {
+      const float wj = nfj * ((sWP[tid] + sWP[64 + tid]) + (sWP[128 + tid] + sWP[192 + tid]));
+      sKEY[tid] = (__float_as_uint(wj) & ~63u) | (uint32_t)(63 - tid);
+    }
     __syncthreads();
     if (tid == kValueIssuer) {  // the parents' value MMA, issued while the others rank
       tc::tc_fence_after();
@@ -881,21 +945,19 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     }
 
     // ---- top-P over the importance (descending, ties to the lower index) ----
-    // thread t ranks parent t % 64 against half of the M0 importances; the
-    // two partial ranks are added by the first 64 threads
+    // thread t ranks parent t % 64 against half of the M0 keys; the two
+    // partial ranks are added by the first 64 threads
     {
       const int j = tid & 63, half = tid >> 6;
       constexpr int kHalf = (M0 + 1) / 2;
       if (j < M0) {
-        const float wj = sW[j];
+        const uint32_t kj = sKEY[j];
         int rank = 0;
         const int l0 = half * kHalf;
 #pragma unroll
         for (int l = 0; l < kHalf; l += 4) {
-          const float4 w4 = *reinterpret_cast<const float4*>(sW + l0 + l);
-          const float wl[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) rank += (wl[k] > wj) || (wl[k] == wj && l0 + l + k < j);
+          const uint4 k4 = *reinterpret_cast<const uint4*>(sKEY + l0 + l);
+          rank += (k4.x > kj) + (k4.y > kj) + (k4.z > kj) + (k4.w > kj);
         }
         sRK[half * 64 + j] = rank;
       }
@@ -907,7 +969,8 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         sSEL[rank] = tid;
         if (a.sel) a.sel[((size_t)bh * a.nblk + blk) * P + rank] = tid;
       }
-      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = sW[tid];
+      if (a.importance)
+        a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = __uint_as_float(sKEY[tid] & ~63u);
     }
     __syncthreads();
     if (nch > 0) copy_cw(0, cw_h);  // the parent logit MMA has read the codewords
@@ -942,6 +1005,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         issue_logits(n);
       }
       wait_bar(bar_mma, ph_mma);
+      if (q > 0) wait_bar(bar_x, ph_x);  // previous chunk's value MMA: PR, VB and x are free
       if (tid == 0 && q + 1 == nch && has_next) {  // the last logit MMA: Q and CW are free
         load_q(u + 1);
         load_pcw(u + 1);
@@ -949,38 +1013,100 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       __syncthreads();
       tc::tc_fence_after();
       if (q + 1 < nch) copy_cw(q + 1, cw_h);  // the logit MMA has read this chunk's codewords
-      // the child logits are read from TMEM twice (maximum, then dA), 16
-      // columns (two slots) at a time, which keeps few of them in registers
-      const float4* nf4 = reinterpret_cast<const float4*>(nfc);
-      float cm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        if (g * 16 < n) {
-          uint32_t r[16];
-          tc::tmem_ld16(tS + lane_off + g * 16, r);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) cm[e & 3] = fmaxf(cm[e & 3], __uint_as_float(r[e]));
-        }
-      }
-      const float cmax_any = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) * sl2;
-      if (q > 0) wait_bar(bar_x, ph_x);  // previous chunk's value MMA: PR, VB and x are free
-      const bool masked = __syncthreads_or(cmax_any > mref + kRescaleLog2) != 0;  // block-uniform, rare
       if (q > 0) copy_vb(q, vb_bh);
-      if (masked) {
-        // masked maximum over non-empty children; rescale x and z if it is far above
-        float cmm[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+      // dA = 2^(t_c - m) - 2^(t_p - m), t_p the mean of the 8 child logits
+      // (Eq. 8), with m the parents' maximum; the unmasked child maximum is
+      // taken on the way.  Empty children need no mask while every 2^(t - m)
+      // stays below 2^24: their value sums and counts are exactly zero.  The
+      // first kPolyPairs pairs of each parent's children take 2^x on the FMA
+      // pipe, the others on the special-function unit.
+      const float4* nf4 = reinterpret_cast<const float4*>(nfc);
+      float2 zc = fm::f2(0.f, 0.f);
+      float cm0 = NEG_INF, cm1 = NEG_INF;
+      auto da_pass = [&](auto masked_t, float mr) {
+        constexpr bool kMasked = decltype(masked_t)::value;
+        const float nm = -mr, sl8 = sl2 * 0.125f;
+        const float2 nm2 = fm::f2(nm, nm);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (g * 16 < n) {
+            uint32_t r[16];
+            tc::tmem_ld16(tS + lane_off + g * 16, r);
+            tc::tmem_wait_ld();
+            const float* t = reinterpret_cast<const float*>(r);
+            if (!kMasked) {
+#pragma unroll
+              for (int e = 0; e < 16; e += 4) {
+                cm0 = fm::max3(cm0, t[e], t[e + 1]);
+                cm1 = fm::max3(cm1, t[e + 2], t[e + 3]);
+              }
+            }
+#pragma unroll
+            for (int hs = 0; hs < 2; ++hs) {
+              const int sl = 2 * g + hs;
+              const float* tt = t + hs * 8;
+              const float2 s01 = fm::add2(fm::f2(tt[0], tt[1]), fm::f2(tt[2], tt[3]));
+              const float2 s45 = fm::add2(fm::f2(tt[4], tt[5]), fm::f2(tt[6], tt[7]));
+              const float2 s = fm::add2(s01, s45);
+              const float ap = tc::ex2(fmaf(s.x + s.y, sl8, nm));
+              const float2 nap = fm::f2(-ap, -ap);
+              const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
+              const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+              uint4 pk;
+              uint32_t* pkw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+              for (int e = 0; e < 8; e += 2) {
+                const float2 x = fm::fma2(fm::f2(tt[e], tt[e + 1]), sl2x2, nm2);
+                float2 ev;
+                if (e < 2 * kPolyPairs) {
+                  ev = fm::exp2_poly2(x);
+                } else {
+                  ev = fm::f2(tc::ex2(x.x), tc::ex2(x.y));
+                }
+                float2 da = fm::add2(ev, nap);
+                if (kMasked) {
+                  da.x = nfv[e] > 0.f ? da.x : 0.f;
+                  da.y = nfv[e + 1] > 0.f ? da.y : 0.f;
+                }
+                zc = fm::fma2(da, fm::f2(nfv[e], nfv[e + 1]), zc);
+                pkw[e >> 1] = pack_bf16x2(da.x, da.y);
+              }
+              *reinterpret_cast<uint4*>(sPR + tc::sw128_offset(tid, sl * 8)) = pk;
+            }
+          }
+        }
+      };
+      da_pass(std::false_type{}, mref);
+      if (np & 1)  // padding slot: zero value sums, so it adds nothing
+        for (int i = tid; i < AB / 16; i += 128)
+          reinterpret_cast<uint4*>(sVB + np * AB)[i] = make_uint4(0, 0, 0, 0);
+      // this chunk's value sums: at q = 0 the codewords of chunk 1 were
+      // committed after them and may still be in flight
+      if (q == 0 && nch > 1)
+        tc::cp_async_wait<1>();
+      else
+        tc::cp_async_wait<0>();
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      const float cmax_any = fmaxf(cm0, cm1) * sl2;
+      if (__syncthreads_or(cmax_any > mref + kRescaleLog2)) {  // block-uniform, rare
+        // masked maximum over non-empty children; rescale x and z if it is far
+        // above the reference, then dA again with the masks applied
+        tc::tc_fence_after();
+        float cmm0 = NEG_INF, cmm1 = NEG_INF;
         for (int g = 0; g < 4; ++g) {
           if (g * 16 < n) {
             uint32_t r[16];
             tc::tmem_ld16(tS + lane_off + g * 16, r);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              cmm[e & 3] = fmaxf(cmm[e & 3], nfc[g * 16 + e] > 0.f ? __uint_as_float(r[e]) : NEG_INF);
+            for (int e = 0; e < 16; e += 2) {
+              cmm0 = fmaxf(cmm0, nfc[g * 16 + e] > 0.f ? __uint_as_float(r[e]) : NEG_INF);
+              cmm1 = fmaxf(cmm1, nfc[g * 16 + e + 1] > 0.f ? __uint_as_float(r[e + 1]) : NEG_INF);
+            }
           }
         }
-        const float cmax = fmaxf(fmaxf(cmm[0], cmm[1]), fmaxf(cmm[2], cmm[3])) * sl2;
+        const float cmax = fmaxf(cmm0, cmm1) * sl2;
         const bool need = cmax > mref + kRescaleLog2;
         if (__syncthreads_or(need)) {
           tc::tc_fence_after();
@@ -997,56 +1123,13 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
           z *= f;
           if (need) mref = cmax;
         }
+        zc = fm::f2(0.f, 0.f);
+        da_pass(std::true_type{}, mref);
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
       }
-      // dA = 2^(t_c - m) - 2^(t_p - m), t_p the mean of the 8 child logits (Eq. 8);
-      // the masked variant (empty children give 0) only in the rare rescale case
-      const float nm = -mref, sl8 = sl2 * 0.125f;
-      float zp[2] = {0.f, 0.f};
-      auto da_pass = [&](auto masked_t) {
-        constexpr bool kMasked = decltype(masked_t)::value;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (g * 16 < n) {
-            uint32_t r[16];
-            tc::tmem_ld16(tS + lane_off + g * 16, r);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int hs = 0; hs < 2; ++hs) {
-              const int sl = 2 * g + hs;
-              const float* t = reinterpret_cast<const float*>(r) + hs * 8;
-              const float ssum = ((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7]));
-              const float ap = tc::ex2(fmaf(ssum, sl8, nm));
-              const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
-              const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
-              float da[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                da[e] = tc::ex2(fmaf(t[e], sl2, nm)) - ap;
-                if (kMasked && !(nfv[e] > 0.f)) da[e] = 0.f;
-                zp[e & 1] = fmaf(da[e], nfv[e], zp[e & 1]);
-              }
-              store_chunk8(sPR, tid, sl * 8, da);
-            }
-          }
-        }
-      };
-      if (masked)
-        da_pass(std::true_type{});
-      else
-        da_pass(std::false_type{});
-      z += zp[0] + zp[1];
-      if (np & 1)  // padding slot: zero value sums, so it adds nothing
-        for (int i = tid; i < AB / 16; i += 128)
-          reinterpret_cast<uint4*>(sVB + np * AB)[i] = make_uint4(0, 0, 0, 0);
-      // this chunk's value sums: at q = 0 the codewords of chunk 1 were
-      // committed after them and may still be in flight
-      if (q == 0 && nch > 1)
-        tc::cp_async_wait<1>();
-      else
-        tc::cp_async_wait<0>();
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      __syncthreads();
+      z += zc.x + zc.y;
       if (*sAbort) goto done;
       if (tid == kValueIssuer) {
         tc::tc_fence_after();
@@ -1062,13 +1145,18 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     //      only before the staging is written again) ----
     {
       const float iz = 1.f / z;
+      const float2 iz2 = fm::f2(iz, iz);
       for (int g = 0; g < D; g += 16) {
         uint32_t xr[16];
         tc::tmem_ld16(tX + lane_off + g, xr);
         tc::tmem_wait_ld();
         float v[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(xr[e]) * iz;
+        for (int e = 0; e < 16; e += 2) {
+          const float2 o = fm::mul2(fm::f2(__uint_as_float(xr[e]), __uint_as_float(xr[e + 1])), iz2);
+          v[e] = o.x;
+          v[e + 1] = o.y;
+        }
         store_chunk8(sPR, tid, g, v);
         store_chunk8(sPR, tid, g + 8, v + 8);
       }
