@@ -38,7 +38,6 @@
 #include "fastmath.cuh"
 
 namespace avq {
-
 namespace {
 
 constexpr int kRows = 128;          // queries per block (MMA M)
@@ -604,21 +603,19 @@ struct FastSmem {
   static constexpr int kVB = kCW + 8 * kAtomBytes;         // value sums: parents, then chunks
   static constexpr int kPR = kVB + 8 * kAtomBytes;         // probabilities / dA [128][64] bf16; O staging
   static constexpr int kNF = kPR + kRows * D * 2;          // counts [2][64]: parents, current chunk
-  static constexpr int kW = kNF + 2 * 64 * 4;              // importance [64]
+  static constexpr int kW = kNF + 2 * 64 * 4;              // ranking keys [64]
   static constexpr int kWP = kW + 64 * 4;                  // per-warp partial sums [4][64]
   static constexpr int kSEL = kWP + 4 * 64 * 4;            // selected parents [64]
-  static constexpr int kRK = kSEL + 64 * 4;                // partial ranks [2][64]
-  static constexpr int kCNT = kRK + 2 * 64 * 4;            // counts of the unit's head [Mt <= 576]
-  static constexpr int kBAR = kCNT + 576 * 4;              // 6 mbarriers
+  static constexpr int kCNT = kSEL + 64 * 4;               // counts of the unit's head [Mt <= 576]
+  static constexpr int kBAR = kCNT + 576 * 4;              // 5 mbarriers
   static constexpr int kMISC = kBAR + 64;                  // tmem base, abort flag
   static constexpr int kTotal = kMISC + 32;
   static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
 };
 
-// The value MMAs are issued by a thread of the last warp, so that their issue
-// (about a hundred cycles per instruction) overlaps the logit MMAs, copies and
-// waits that thread 0 and warp 0 take care of.
-constexpr int kValueIssuer = 96;
+// MMAs are issued by one elected lane of a warp (issuing takes 60-90 cycles
+// per instruction): the logit MMAs by warp 0, the value MMAs by warp 3, so
+// that the two overlap each other and the waits that thread 0 takes.
 
 // Of each selected parent's 8 child exponentials, the first 2 * kPolyPairs
 // are evaluated on the FMA pipe (fm::exp2_poly2), the others on the
@@ -641,7 +638,6 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   uint32_t* sKEY = reinterpret_cast<uint32_t*>(sm + S::kW);  // importance ranking keys [64]
   float* sWP = reinterpret_cast<float*>(sm + S::kWP);
   int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
-  int* sRK = reinterpret_cast<int*>(sm + S::kRK);
   const int32_t* sCNT = reinterpret_cast<const int32_t*>(sm + S::kCNT);
   uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + S::kBAR);
   uint64_t* bar_cw = bar_q + 1;   // parents' codewords and the head's counts
@@ -669,34 +665,35 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   // (bit b of `issued` set once one was issued): on the way out the kernel
   // waits, with a limit, for those, so no copy or MMA is in flight when it
   // frees TMEM and returns, also after a timed-out wait
-  uint32_t ph_q = 0, ph_cw = 0, ph_vb = 0, ph_mma = 0, ph_x = 0;
+  constexpr int kBars = 5;
+  uint32_t ph = 0;  // bit b: parity of barrier b's next phase
   uint32_t issued = 0, exp_par = 0;
-  auto note = [&](int b, uint32_t ph) {
+  auto note = [&](int b) {
     issued |= 1u << b;
-    exp_par = (exp_par & ~(1u << b)) | (ph << b);
+    exp_par = (exp_par & ~(1u << b)) | (ph & (1u << b));
   };
   // the next unit's Q tile and parents' codewords / value sums (thread 0)
   auto load_q = [&](int u) {
-    note(0, ph_q);
+    note(0);
     tc::mbar_arrive_expect_tx(bar_q, kRows * D * 2);
 #pragma unroll
     for (int kh = 0; kh < KH; ++kh)
       tc::tma_load_3d(sQ + kh * kRows * 128, &qmap, kh * 64, (u % a.nblk) * kRows, u / a.nblk, bar_q);
   };
   auto load_pcw = [&](int u) {
-    note(1, ph_cw);
+    note(1);
     tc::mbar_arrive_expect_tx(bar_cw, M0 * D * 2 + Mt * 4);
     tc::bulk_g2s(sCW, unit_cw(u), M0 * D * 2, bar_cw);
     tc::bulk_g2s(sm + S::kCNT, a.counts + (size_t)(u / a.nblk) * Mt, Mt * 4, bar_cw);
   };
   auto load_pvb = [&](int u) {
-    note(2, ph_vb);
+    note(2);
     tc::mbar_arrive_expect_tx(bar_vb, M0 * D * 2);
     tc::bulk_g2s(sVB, unit_vb(u), M0 * D * 2, bar_vb);
   };
 
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) tc::mbar_init(bar_q + i, 1);
+    for (int i = 0; i < kBars; ++i) tc::mbar_init(bar_q + i, 1);
     tc::fence_mbar_init();
     *sAbort = 0;
   }
@@ -724,7 +721,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
 
     auto issue_logits = [&](int n) {  // S = Q * CW^T over n codes
-      note(3, ph_mma);
+      note(3);
       const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
@@ -734,25 +731,29 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       }
       tc::mma_commit(bar_mma);
     };
-    auto issue_values = [&](int n, bool acc) {  // x (+)= PR * VB over n codes
-      note(4, ph_x);
-      for (int k = 0; k < n / 16; ++k) {
+    // x (+)= PR[:, 16 k0 ..] * VB over n codes (K steps k0 .. k0 + n/16)
+    auto issue_values = [&](int n, int k0, bool acc, uint64_t* bar, int b) {
+      note(b);
+      for (int k = k0; k < k0 + n / 16; ++k) {
         const uint64_t ad = tc::sdesc_sw128(sPRa + (k & 3) * 32, 16, 1024);
         const uint64_t bd = tc::sdesc_sw128(sVBa + k * 2 * AB, 1024, KH * 1024);
-        tc::mma_bf16(tX, ad, bd, idesc_x, (acc || k > 0) ? 1u : 0u);
+        tc::mma_bf16(tX, ad, bd, idesc_x, (acc || k > k0) ? 1u : 0u);
       }
-      tc::mma_commit(bar_x);
+      tc::mma_commit(bar);
     };
     // Waits are taken by thread 0 alone; the others meet it at the CTA barrier
     // that follows every wait, so no warp spins on the issue slots.
-    auto wait_bar = [&](uint64_t* bar, uint32_t& ph) {
-      if (tid == 0 && !tc::mbar_wait(bar, ph)) fail(a.err, sAbort);
-      ph ^= 1;
+    auto wait_bar = [&](int b) {
+      if (tid == 0 && !tc::mbar_wait(bar_q + b, (ph >> b) & 1u)) fail(a.err, sAbort);
+      ph ^= 1u << b;
     };
     // child atoms of chunk q (codewords or value sums) into the staging
     // buffer: `slots` atoms, slot i from selected parent min(i, np - 1), as
-    // 16-byte cp.async pieces spread over all threads, one commit group
+    // 16-byte cp.async pieces spread over all threads, one commit group.  An
+    // odd parent count is padded with a copy of the last parent's codewords
+    // (and zero value sums), so that the MMAs' N and K are multiples of 16.
     auto chunk_np = [&](int q) { return min(kChunkParents, P - q * kChunkParents); };
+    auto chunk_slots = [&](int q) { return (chunk_np(q) + 1) & ~1; };
     auto copy_atoms = [&](uint8_t* dst, const bf16* src_h, int q, int slots) {
       constexpr int kPieces = AB / 16;
       const int np = chunk_np(q);
@@ -764,7 +765,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       }
       tc::cp_async_commit();
     };
-    auto copy_cw = [&](int q, const bf16* cw_h) { copy_atoms(sCW, cw_h, q, (chunk_np(q) + 1) & ~1); };
+    auto copy_cw = [&](int q, const bf16* cw_h) { copy_atoms(sCW, cw_h, q, chunk_slots(q)); };
     auto copy_vb = [&](int q, const bf16* vb_bh) { copy_atoms(sVB, vb_bh, q, chunk_np(q)); };
 
     for (int u = u0; u < u1; ++u) {
@@ -774,8 +775,8 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     const bf16* cw_h = unit_cw(u);
     const bf16* vb_bh = unit_vb(u);
     const bool has_next = u + 1 < u1;
-    wait_bar(bar_q, ph_q);
-    wait_bar(bar_cw, ph_cw);
+    wait_bar(0);  // Q
+    wait_bar(1);  // parents' codewords and counts
     __syncthreads();
     float nfj = 0.f;
     if (tid < M0) {
@@ -788,11 +789,14 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     if (*sAbort) goto done;
 
     // ---- parents: logits, masked max, A = 2^(t - m), z, importance ----
-    if (tid == 0) {
-      tc::tc_fence_after();
-      issue_logits(M0);
+    if (warp == 0) {
+      if (tc::elect_one()) {
+        tc::tc_fence_after();
+        issue_logits(M0);
+      }
+      __syncwarp();
     }
-    wait_bar(bar_mma, ph_mma);
+    wait_bar(3);
     if (tid == 0) {
       tc::bulk_wait_group_read0();  // the previous unit's O store has read its staging (PR)
       if (nch == 0 && has_next) {   // Q and the parents' codewords are read: next unit's
@@ -804,27 +808,30 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     tc::tc_fence_after();
     float m, z;
     {
-      // the logits are read from TMEM in 16-column pieces: the maximum first,
-      // then A = 2^(t - m) (to PR in bf16, and back over the logits in fp32 for
-      // the importance, which needs 1 / z of the whole row)
+      // the row's logits are read from TMEM twice: all M0 at once (one wait)
+      // for the maximum, then 32 at a time for A = 2^(t - m) (to PR in bf16,
+      // and back over the logits in fp32 for the importance, which needs
+      // 1 / z of the whole row)
       const float4* nf4 = reinterpret_cast<const float4*>(sNF);
       float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-      for (int g = 0; g < M0 / 16; ++g) {
-        uint32_t r[16];
-        tc::tmem_ld16(tS + lane_off + g * 16, r);
+      for (int c0 = 0; c0 < M0; c0 += 32) {
+        constexpr int W = M0 < 32 ? M0 : 32;
+        uint32_t r[W];
+#pragma unroll
+        for (int g = 0; g < W / 16; ++g) tc::tmem_ld16(tS + lane_off + c0 + g * 16, r + g * 16);
         tc::tmem_wait_ld();
         const float* t = reinterpret_cast<const float*>(r);
         if (!any_empty) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
+          for (int e = 0; e < W; e += 4) {
             mx0 = fm::max3(mx0, t[e], t[e + 1]);
             mx1 = fm::max3(mx1, t[e + 2], t[e + 3]);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const float4 nf = nf4[(g * 16 + e) >> 2];
+          for (int e = 0; e < W; e += 4) {
+            const float4 nf = nf4[(c0 + e) >> 2];
             mx0 = fm::max3(mx0, nf.x > 0.f ? t[e] : NEG_INF, nf.y > 0.f ? t[e + 1] : NEG_INF);
             mx1 = fm::max3(mx1, nf.z > 0.f ? t[e + 2] : NEG_INF, nf.w > 0.f ? t[e + 3] : NEG_INF);
           }
@@ -836,32 +843,40 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       auto a_pass = [&](auto masked_t) {
         constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
-        for (int g = 0; g < M0 / 16; ++g) {
-          uint32_t r[16];
-          tc::tmem_ld16(tS + lane_off + g * 16, r);
+        for (int g2 = 0; g2 < M0 / 16; g2 += 2) {
+          uint32_t r[32];
+          tc::tmem_ld16(tS + lane_off + g2 * 16, r);
+          if (g2 + 1 < M0 / 16) tc::tmem_ld16(tS + lane_off + g2 * 16 + 16, r + 16);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const float4 nf = nf4[(g * 16 + e) >> 2];
-            const float2 x01 = fm::fma2(fm::f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), sl2x2, nm2);
-            const float2 x23 = fm::fma2(fm::f2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), sl2x2, nm2);
-            float a0 = tc::ex2(x01.x), a1 = tc::ex2(x01.y), a2 = tc::ex2(x23.x), a3 = tc::ex2(x23.y);
-            if (kMasked) {
-              a0 = nf.x > 0.f ? a0 : 0.f;
-              a1 = nf.y > 0.f ? a1 : 0.f;
-              a2 = nf.z > 0.f ? a2 : 0.f;
-              a3 = nf.w > 0.f ? a3 : 0.f;
+          for (int gg = 0; gg < 2; ++gg) {
+            const int g = g2 + gg;
+            if (g < M0 / 16) {
+              uint32_t* rg = r + gg * 16;
+#pragma unroll
+              for (int e = 0; e < 16; e += 4) {
+                const float4 nf = nf4[(g * 16 + e) >> 2];
+                const float2 x01 = fm::fma2(fm::f2(__uint_as_float(rg[e]), __uint_as_float(rg[e + 1])), sl2x2, nm2);
+                const float2 x23 = fm::fma2(fm::f2(__uint_as_float(rg[e + 2]), __uint_as_float(rg[e + 3])), sl2x2, nm2);
+                float a0 = tc::ex2(x01.x), a1 = tc::ex2(x01.y), a2 = tc::ex2(x23.x), a3 = tc::ex2(x23.y);
+                if (kMasked) {
+                  a0 = nf.x > 0.f ? a0 : 0.f;
+                  a1 = nf.y > 0.f ? a1 : 0.f;
+                  a2 = nf.z > 0.f ? a2 : 0.f;
+                  a3 = nf.w > 0.f ? a3 : 0.f;
+                }
+                zp = fm::fma2(fm::f2(a0, a1), fm::f2(nf.x, nf.y), zp);
+                zp = fm::fma2(fm::f2(a2, a3), fm::f2(nf.z, nf.w), zp);
+                rg[e] = __float_as_uint(a0);
+                rg[e + 1] = __float_as_uint(a1);
+                rg[e + 2] = __float_as_uint(a2);
+                rg[e + 3] = __float_as_uint(a3);
+              }
+              store_chunk8(sPR, tid, g * 16, reinterpret_cast<const float*>(rg));
+              store_chunk8(sPR, tid, g * 16 + 8, reinterpret_cast<const float*>(rg) + 8);
+              tc::tmem_st16(tS + lane_off + g * 16, rg);
             }
-            zp = fm::fma2(fm::f2(a0, a1), fm::f2(nf.x, nf.y), zp);
-            zp = fm::fma2(fm::f2(a2, a3), fm::f2(nf.z, nf.w), zp);
-            r[e] = __float_as_uint(a0);
-            r[e + 1] = __float_as_uint(a1);
-            r[e + 2] = __float_as_uint(a2);
-            r[e + 3] = __float_as_uint(a3);
           }
-          store_chunk8(sPR, tid, g * 16, reinterpret_cast<const float*>(r));
-          store_chunk8(sPR, tid, g * 16 + 8, reinterpret_cast<const float*>(r) + 8);
-          tc::tmem_st16(tS + lane_off + g * 16, r);
         }
       };
       if (any_empty)
@@ -882,29 +897,24 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
                   z2 = __shfl_sync(0xffffffffu, rz, rl + 16), z3 = __shfl_sync(0xffffffffu, rz, rl + 24);
       float2 cs[8];
 #pragma unroll
-      for (int hcol = 0; hcol < 2; ++hcol) {
-        if (hcol * 32 < M0) {
-          uint32_t r[16];
-          fm::tmem_ld_16x256b_x4(tS + lane_off + hcol * 32, r);  // rows l/4, l/4 + 8
+      for (int hc = 0; hc < 2; ++hc) {
+        if (hc * 32 < M0) {
+          uint32_t lo[16], hi[16];
+          fm::tmem_ld_16x256b_x4(tS + lane_off + hc * 32, lo);                // rows l/4, l/4 + 8
+          fm::tmem_ld_16x256b_x4(tS + lane_off + (16u << 16) + hc * 32, hi);  // rows 16 + l/4, 24 + l/4
           tc::tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int grp = hcol * 4 + k;
-            float2 s = fm::mul2(fm::f2(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1])), fm::f2(z0, z0));
-            cs[grp] = fm::fma2(fm::f2(__uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3])), fm::f2(z1, z1), s);
-          }
-          fm::tmem_ld_16x256b_x4(tS + lane_off + (16u << 16) + hcol * 32, r);  // rows 16 + l/4, 24 + l/4
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int grp = hcol * 4 + k;
-            float2 s = fm::fma2(fm::f2(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1])), fm::f2(z2, z2), cs[grp]);
-            s = fm::fma2(fm::f2(__uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3])), fm::f2(z3, z3), s);
+            const int grp = hc * 4 + k;
+            float2 s = fm::mul2(fm::f2(__uint_as_float(lo[4 * k]), __uint_as_float(lo[4 * k + 1])), fm::f2(z0, z0));
+            s = fm::fma2(fm::f2(__uint_as_float(lo[4 * k + 2]), __uint_as_float(lo[4 * k + 3])), fm::f2(z1, z1), s);
+            s = fm::fma2(fm::f2(__uint_as_float(hi[4 * k]), __uint_as_float(hi[4 * k + 1])), fm::f2(z2, z2), s);
+            s = fm::fma2(fm::f2(__uint_as_float(hi[4 * k + 2]), __uint_as_float(hi[4 * k + 3])), fm::f2(z3, z3), s);
             cs[grp] = grp * 8 < M0 ? s : fm::f2(0.f, 0.f);
           }
         } else {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) cs[hcol * 4 + k] = fm::f2(0.f, 0.f);
+          for (int k = 0; k < 4; ++k) cs[hc * 4 + k] = fm::f2(0.f, 0.f);
         }
       }
       // reduce-scatter: lane bit 4 splits groups 0-3 / 4-7, bit 3 the pairs,
@@ -925,7 +935,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       *reinterpret_cast<float2*>(sWP + warp * 64 + 2 * lane) = cs[0];
     }
     tc::fence_proxy_async_smem();
-    wait_bar(bar_vb, ph_vb);
+    wait_bar(2);  // parents' value sums
     tc::tc_fence_before();
     __syncthreads();
     if (*sAbort) goto done;
@@ -939,81 +949,73 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       sKEY[tid] = (__float_as_uint(wj) & ~63u) | (uint32_t)(63 - tid);
     }
     __syncthreads();
-    if (tid == kValueIssuer) {  // the parents' value MMA, issued while the others rank
-      tc::tc_fence_after();
-      issue_values(M0, false);
-    }
-
     // ---- top-P over the importance (descending, ties to the lower index) ----
-    // thread t ranks parent t % 64 against half of the M0 keys; the two
-    // partial ranks are added by the first 64 threads
-    {
-      const int j = tid & 63, half = tid >> 6;
-      constexpr int kHalf = (M0 + 1) / 2;
-      if (j < M0) {
-        const uint32_t kj = sKEY[j];
-        int rank = 0;
-        const int l0 = half * kHalf;
-#pragma unroll
-        for (int l = 0; l < kHalf; l += 4) {
-          const uint4 k4 = *reinterpret_cast<const uint4*>(sKEY + l0 + l);
-          rank += (k4.x > kj) + (k4.y > kj) + (k4.z > kj) + (k4.w > kj);
-        }
-        sRK[half * 64 + j] = rank;
-      }
-    }
-    __syncthreads();
+    // thread j < M0 of the first two warps ranks parent j against all keys,
+    // while the last warp issues the parents' value MMA
     if (tid < M0) {
-      const int rank = sRK[tid] + sRK[64 + tid];
+      const uint32_t kj = sKEY[tid];
+      int r0 = 0, r1 = 0;
+#pragma unroll
+      for (int l = 0; l < M0; l += 8) {
+        const uint4 ka = *reinterpret_cast<const uint4*>(sKEY + l);
+        const uint4 kb = *reinterpret_cast<const uint4*>(sKEY + l + 4);
+        r0 += (ka.x > kj) + (ka.y > kj) + (ka.z > kj) + (ka.w > kj);
+        r1 += (kb.x > kj) + (kb.y > kj) + (kb.z > kj) + (kb.w > kj);
+      }
+      const int rank = r0 + r1;
       if (rank < P) {
         sSEL[rank] = tid;
         if (a.sel) a.sel[((size_t)bh * a.nblk + blk) * P + rank] = tid;
       }
-      if (a.importance)
-        a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = __uint_as_float(sKEY[tid] & ~63u);
+      if (a.importance) a.importance[((size_t)bh * a.nblk + blk) * M0 + tid] = __uint_as_float(kj & ~63u);
+    }
+    if (warp == 3) {
+      if (tc::elect_one()) {
+        tc::tc_fence_after();
+        issue_values(M0, 0, false, bar_x, 4);
+      }
+      __syncwarp();
     }
     __syncthreads();
-    if (nch > 0) copy_cw(0, cw_h);  // the parent logit MMA has read the codewords
-    wait_bar(bar_x, ph_x);          // the parents' value MMA has read PR and VB
-    __syncthreads();
-    if (nch > 0) copy_vb(0, vb_bh);
-    if (tid == 0 && nch == 0 && has_next) load_pvb(u + 1);  // the parents' value MMA is done
 
     // ---- child refinement in chunks of 8 selected parents ----
+    // Chunk q: its codewords were copied during chunk q - 1 (chunk 0's right
+    // after the selection), its logit MMA issued as soon as they and the
+    // logit region were free; the chunk's value sums are copied, and the next
+    // chunk's codewords, while its dA pass runs.
     float mref = m;
-    float* nfc = sNF + 64;
+    if (nch > 0) {
+      copy_cw(0, cw_h);  // the parent logit MMA has read the parents' codewords
+      tc::cp_async_wait<0>();
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      if (warp == 0) {
+        if (tc::elect_one()) {
+          tc::tc_fence_after();
+          issue_logits(chunk_slots(0) * 8);
+        }
+        __syncwarp();
+      }
+    }
     for (int q = 0; q < nch; ++q) {
       const int np = chunk_np(q);
-      const int slots = (np + 1) & ~1;
-      const int n = slots * 8;
+      const int n = chunk_slots(q) * 8;
+      float* nfc = sNF + 64;
       if (tid < 64) {
         const int rr = tid >> 3;
         nfc[tid] = rr < np ? (float)sCNT[M0 + sSEL[q * kChunkParents + rr] * 8 + (tid & 7)] : 0.f;
       }
-      // this chunk's codewords: at q = 0 the value sums of chunk 0 were
-      // committed after them and may still be in flight
-      if (q == 0)
-        tc::cp_async_wait<1>();
-      else
-        tc::cp_async_wait<0>();
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      __syncthreads();
-      if (*sAbort) goto done;
-      if (tid == 0) {
-        tc::tc_fence_after();
-        issue_logits(n);
-      }
-      wait_bar(bar_mma, ph_mma);
-      if (q > 0) wait_bar(bar_x, ph_x);  // previous chunk's value MMA: PR, VB and x are free
+      wait_bar(3);  // this chunk's logits
+      wait_bar(4);  // the previous value MMA (the parents' at q = 0) has read PR and VB
       if (tid == 0 && q + 1 == nch && has_next) {  // the last logit MMA: Q and CW are free
         load_q(u + 1);
         load_pcw(u + 1);
       }
       __syncthreads();
       tc::tc_fence_after();
-      if (q + 1 < nch) copy_cw(q + 1, cw_h);  // the logit MMA has read this chunk's codewords
-      if (q > 0) copy_vb(q, vb_bh);
+      copy_vb(q, vb_bh);
+      if (q + 1 < nch) copy_cw(q + 1, cw_h);  // this chunk's logits are done
       // dA = 2^(t_c - m) - 2^(t_p - m), t_p the mean of the 8 child logits
       // (Eq. 8), with m the parents' maximum; the unmasked child maximum is
       // taken on the way.  Empty children need no mask while every 2^(t - m)
@@ -1028,50 +1030,51 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
         const float nm = -mr, sl8 = sl2 * 0.125f;
         const float2 nm2 = fm::f2(nm, nm);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (g * 16 < n) {
-            uint32_t r[16];
-            tc::tmem_ld16(tS + lane_off + g * 16, r);
+        for (int g2 = 0; g2 < 4; g2 += 2) {
+          if (g2 * 16 < n) {
+            uint32_t r[32];
+            tc::tmem_ld16(tS + lane_off + g2 * 16, r);
+            if (g2 * 16 + 16 < n) tc::tmem_ld16(tS + lane_off + g2 * 16 + 16, r + 16);
             tc::tmem_wait_ld();
-            const float* t = reinterpret_cast<const float*>(r);
-            if (!kMasked) {
 #pragma unroll
-              for (int e = 0; e < 16; e += 4) {
-                cm0 = fm::max3(cm0, t[e], t[e + 1]);
-                cm1 = fm::max3(cm1, t[e + 2], t[e + 3]);
-              }
-            }
-#pragma unroll
-            for (int hs = 0; hs < 2; ++hs) {
-              const int sl = 2 * g + hs;
-              const float* tt = t + hs * 8;
-              const float2 s01 = fm::add2(fm::f2(tt[0], tt[1]), fm::f2(tt[2], tt[3]));
-              const float2 s45 = fm::add2(fm::f2(tt[4], tt[5]), fm::f2(tt[6], tt[7]));
-              const float2 s = fm::add2(s01, s45);
-              const float ap = tc::ex2(fmaf(s.x + s.y, sl8, nm));
-              const float2 nap = fm::f2(-ap, -ap);
-              const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
-              const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
-              uint4 pk;
-              uint32_t* pkw = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                const float2 x = fm::fma2(fm::f2(tt[e], tt[e + 1]), sl2x2, nm2);
-                float2 ev;
-                if (e < 2 * kPolyPairs) {
-                  ev = fm::exp2_poly2(x);
-                } else {
-                  ev = fm::f2(tc::ex2(x.x), tc::ex2(x.y));
+            for (int s4 = 0; s4 < 4; ++s4) {
+              const int sl = 2 * g2 + s4;  // parent slot
+              if (sl * 8 < n) {
+                const float* tt = reinterpret_cast<const float*>(r) + s4 * 8;
+                if (!kMasked) {
+                  cm0 = fm::max3(cm0, tt[0], tt[1]);
+                  cm1 = fm::max3(cm1, tt[2], tt[3]);
+                  cm0 = fm::max3(cm0, tt[4], tt[5]);
+                  cm1 = fm::max3(cm1, tt[6], tt[7]);
                 }
-                float2 da = fm::add2(ev, nap);
-                if (kMasked) {
-                  da.x = nfv[e] > 0.f ? da.x : 0.f;
-                  da.y = nfv[e + 1] > 0.f ? da.y : 0.f;
+                const float2 s01 = fm::add2(fm::f2(tt[0], tt[1]), fm::f2(tt[2], tt[3]));
+                const float2 s45 = fm::add2(fm::f2(tt[4], tt[5]), fm::f2(tt[6], tt[7]));
+                const float2 sm2 = fm::add2(s01, s45);
+                const float ap = tc::ex2(fmaf(sm2.x + sm2.y, sl8, nm));
+                const float2 nap = fm::f2(-ap, -ap);
+                const float4 na = nf4[sl * 2], nb = nf4[sl * 2 + 1];
+                const float nfv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+                uint4 pk;
+                uint32_t* pkw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  const float2 x = fm::fma2(fm::f2(tt[e], tt[e + 1]), sl2x2, nm2);
+                  float2 ev;
+                  if (e < 2 * kPolyPairs) {
+                    ev = fm::exp2_poly2(x);
+                  } else {
+                    ev = fm::f2(tc::ex2(x.x), tc::ex2(x.y));
+                  }
+                  float2 da = fm::add2(ev, nap);
+                  if (kMasked) {
+                    da.x = nfv[e] > 0.f ? da.x : 0.f;
+                    da.y = nfv[e + 1] > 0.f ? da.y : 0.f;
+                  }
+                  zc = fm::fma2(da, fm::f2(nfv[e], nfv[e + 1]), zc);
+                  pkw[e >> 1] = pack_bf16x2(da.x, da.y);
                 }
-                zc = fm::fma2(da, fm::f2(nfv[e], nfv[e + 1]), zc);
-                pkw[e >> 1] = pack_bf16x2(da.x, da.y);
+                *reinterpret_cast<uint4*>(sPR + tc::sw128_offset(tid, sl * 8)) = pk;
               }
-              *reinterpret_cast<uint4*>(sPR + tc::sw128_offset(tid, sl * 8)) = pk;
             }
           }
         }
@@ -1080,12 +1083,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       if (np & 1)  // padding slot: zero value sums, so it adds nothing
         for (int i = tid; i < AB / 16; i += 128)
           reinterpret_cast<uint4*>(sVB + np * AB)[i] = make_uint4(0, 0, 0, 0);
-      // this chunk's value sums: at q = 0 the codewords of chunk 1 were
-      // committed after them and may still be in flight
-      if (q == 0 && nch > 1)
-        tc::cp_async_wait<1>();
-      else
-        tc::cp_async_wait<0>();
+      tc::cp_async_wait<0>();  // this chunk's value sums and the next chunk's codewords
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       const float cmax_any = fmaxf(cm0, cm1) * sl2;
@@ -1131,13 +1129,22 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       }
       z += zc.x + zc.y;
       if (*sAbort) goto done;
-      if (tid == kValueIssuer) {
-        tc::tc_fence_after();
-        issue_values(n, true);
+      if (warp == 3) {  // this chunk's value MMA
+        if (tc::elect_one()) {
+          tc::tc_fence_after();
+          issue_values(n, 0, true, bar_x, 4);
+        }
+        __syncwarp();
+      } else if (warp == 0 && q + 1 < nch) {  // the next chunk's logits (its codewords are in)
+        if (tc::elect_one()) {
+          tc::tc_fence_after();
+          issue_logits(chunk_slots(q + 1) * 8);
+        }
+        __syncwarp();
       }
     }
-    if (nch > 0) wait_bar(bar_x, ph_x);  // the last value MMA
-    if (tid == 0 && nch > 0 && has_next) load_pvb(u + 1);
+    wait_bar(4);  // the last value MMA (the parents' when there are no chunks)
+    if (tid == 0 && has_next) load_pvb(u + 1);
     __syncthreads();
     tc::tc_fence_after();
 
@@ -1175,11 +1182,10 @@ done:
   // nothing of this CTA in flight before TMEM is freed: copies and MMAs this
   // thread issued (the waits return at once for completed ones; 1 ms limit)
   if (issued) {
-    uint64_t* const bars[5] = {bar_q, bar_cw, bar_vb, bar_mma, bar_x};
 #pragma unroll
-    for (int b = 0; b < 5; ++b)
+    for (int b = 0; b < kBars; ++b)
       if ((issued >> b) & 1u)
-        if (!tc::mbar_wait(bars[b], (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
+        if (!tc::mbar_wait(bar_q + b, (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
   }
   tc::cp_async_wait<0>();
   if (tid == 0) tc::bulk_wait_group_read0();  // the last O store has read the staging
@@ -1190,6 +1196,7 @@ done:
     tc::tmem_dealloc(*sTmem, S::kTmemCols);
   }
 }
+
 
 // Codewords and value sums -> bf16 images of swizzled atoms.  Code a of a head
 // (parents first, then child c of parent p at M0 + p*C + c) lands in atom
@@ -1337,3 +1344,4 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
 }
 
 }  // namespace avq
+
