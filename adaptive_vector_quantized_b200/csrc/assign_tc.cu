@@ -486,12 +486,6 @@ __device__ __forceinline__ int nth_set(uint32_t m, int n) {
   }
   return pos;
 }
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                 "=r"(r[7])
-               : "r"(taddr));
-}
 
 // bf16 bits of x, round to nearest even.
 __device__ __forceinline__ uint32_t bf16_bits(float x) {
@@ -838,19 +832,23 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
           ph_c ^= 1;
           wg_bar(barid);  // child scores in TMEM; the CUDA-core children done
           tc::tc_fence_after();
-          // one TMEM load per distinct staging slot among this warp's keys
+          // the round's child columns in two 32-column loads (only the halves
+          // that some key of the warp needs), each key taking its slot's 8
           const int my = (myslot >= r0 && myslot < r0 + kStageAtoms) ? myslot - r0 : -1;
-          unsigned pending = __ballot_sync(0xffffffffu, my >= 0);
-          while (pending) {
-            const int sl = __shfl_sync(0xffffffffu, my, __ffs(pending) - 1);
-            uint32_t rr[8];
-            tmem_ld8(tP + lane_off + sl * 8, rr);
-            tc::tmem_wait_ld();
-            if (my == sl) {
 #pragma unroll
-              for (int c = 0; c < 8; ++c) vals[c] = __uint_as_float(rr[c]);
+          for (int hh = 0; hh < kStageAtoms / 4; ++hh) {
+            if (__any_sync(0xffffffffu, my >= 4 * hh && my < 4 * hh + 4)) {
+              uint32_t rr[32];
+              tc::tmem_ld16(tP + lane_off + hh * 32, rr);
+              tc::tmem_ld16(tP + lane_off + hh * 32 + 16, rr + 16);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int s4 = 0; s4 < 4; ++s4)
+                if (my == 4 * hh + s4) {
+#pragma unroll
+                  for (int c = 0; c < 8; ++c) vals[c] = __uint_as_float(rr[8 * s4 + c]);
+                }
             }
-            pending &= ~__ballot_sync(0xffffffffu, my == sl);
           }
           if (r0 + kStageAtoms < np) {
             tc::tc_fence_before();
