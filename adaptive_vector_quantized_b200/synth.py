@@ -46,8 +46,13 @@ CONFIGS = {
     "vit28": dict(dtype="bf16", B=2, H=12, N=784, d=64, M0=64, C=8, P=16, block=128,
                   keys="regions", grid=(28, 28), key_sigma=0.1, noise=0.0, order="gilbert",
                   sigma_c=0.3, two_pass=False),
+    # depth-3 tree (the conclusion's "deeper hierarchies"): 64 parents, 512
+    # children, 4096 grandchildren; P parents refined, then P of their children
+    "deep3": dict(dtype="bf16", B=1, H=8, N=16384, d=64, M0=64, C=8, P=16, P2=16, block=128,
+                  keys="tree3", key_sigma=0.03, sigma_c=0.3, sigma_g=0.1, noise=0.0, depth=3),
 }
-CONFIG_SEEDS = {"tiny": 1000, "vit": 1001, "long": 1002, "largecb": 1003, "sweep": 1004, "vit28": 1005}
+CONFIG_SEEDS = {"tiny": 1000, "vit": 1001, "long": 1002, "largecb": 1003, "sweep": 1004, "vit28": 1005,
+                "deep3": 1006}
 
 
 def sweep_config(P: int, N: int, order: str = "hilbert", flat192: bool = False) -> dict:
@@ -112,6 +117,18 @@ def _round_dtype(a: np.ndarray, dtype: str) -> torch.Tensor:
     raise ValueError(dtype)
 
 
+def _centred_offsets(rng, C: int, d: int, sigma: float):
+    """C offsets [C, d] in grid units, N(0, sigma^2) draws rounded to the
+    grid and shifted (in whole units) so that they sum to exactly zero."""
+    off = np.rint(rng.standard_normal((C, d)) * sigma * GRID_UNITS).astype(np.int64)
+    tot = off.sum(axis=0)
+    q = np.floor_divide(tot, C)
+    r = tot - q * C  # 0 <= r < C
+    off -= q[None, :]
+    off -= (np.arange(C)[:, None] < r[None, :]).astype(np.int64)
+    return off
+
+
 def make_codebook(rng: np.random.Generator, H: int, M0: int, C: int, d: int,
                   sigma_c: float = 0.3):
     """Parents [H,M0,d] and children [H,M0,C,d] in grid units (int64) with
@@ -124,21 +141,78 @@ def make_codebook(rng: np.random.Generator, H: int, M0: int, C: int, d: int,
     for h in range(H):
         for m in range(M0):
             for _ in range(1000):
-                off = np.rint(rng.standard_normal((C, d)) * sigma_c * GRID_UNITS).astype(np.int64)
-                tot = off.sum(axis=0)
-                q = np.floor_divide(tot, C)
-                r = tot - q * C  # 0 <= r < C
-                off -= q[None, :]
-                # remove the remainder one unit at a time from the first r offsets
-                idx = np.arange(C)[:, None] < r[None, :]
-                off -= idx.astype(np.int64)
-                ch = par[h, m][None, :] + off
+                ch = par[h, m][None, :] + _centred_offsets(rng, C, d, sigma_c)
                 if np.abs(ch).max() <= GRID_LIMIT:
                     break
             else:  # pragma: no cover - astronomically unlikely
                 raise RuntimeError("could not draw children inside the grid limit")
             child[h, m] = ch
     return par, child
+
+
+def make_codebook3(rng: np.random.Generator, H: int, M0: int, C: int, d: int,
+                   sigma_c: float = 0.3, sigma_g: float = 0.1):
+    """A depth-3 tree in grid units: parents [H,M0,d], children [H,M0,C,d],
+    grandchildren [H,M0,C,C,d]; every child is exactly the mean of its
+    grandchildren and every parent of its children (centred integer offsets),
+    all values at most 8 significant bits (exact in bf16)."""
+    par, child = make_codebook(rng, H, M0, C, d, sigma_c)
+    gc = np.empty((H, M0, C, C, d), dtype=np.int64)
+    for h in range(H):
+        for m in range(M0):
+            for c in range(C):
+                for _ in range(1000):
+                    g = child[h, m, c][None, :] + _centred_offsets(rng, C, d, sigma_g)
+                    if np.abs(g).max() <= GRID_LIMIT:
+                        break
+                else:  # pragma: no cover - astronomically unlikely
+                    raise RuntimeError("could not draw grandchildren inside the grid limit")
+                gc[h, m, c] = g
+    return par, child, gc
+
+
+def m_total3(M0: int, C: int) -> int:
+    """Codewords of the depth-3 tree: M0 parents, M0*C children, M0*C*C grandchildren."""
+    return M0 + M0 * C + M0 * C * C
+
+
+def make_inputs3(cfg: dict, seed: int) -> dict:
+    """Inputs of a depth-3 forward: as make_inputs, plus grandchildren
+    [H,M0,C,C,d].  Keys: a uniform parent, then a uniform level (parent,
+    child or grandchild) and a uniform node of that level below the parent,
+    plus N(0, key_sigma^2) noise; a fraction `noise` of keys ~U(-3,3)^d."""
+    B, H, N, d, M0, C = (cfg[k] for k in ("B", "H", "N", "d", "M0", "C"))
+    dtype = cfg["dtype"]
+    s_code, s_key, s_q, s_v = np.random.SeedSequence(seed).spawn(4)
+    rng_key = np.random.default_rng(s_key)
+    par_i, ch_i, gc_i = make_codebook3(np.random.default_rng(s_code), H, M0, C, d,
+                                       cfg.get("sigma_c", 0.3), cfg.get("sigma_g", 0.1))
+    par_f, ch_f, gc_f = (x.astype(np.float64) / GRID_UNITS for x in (par_i, ch_i, gc_i))
+    K = np.empty((B, H, N, d), dtype=np.float32)
+    sigma = cfg.get("key_sigma", 0.03)
+    for b in range(B):
+        for h in range(H):
+            p = rng_key.integers(0, M0, N)
+            lvl = rng_key.integers(0, 3, N)
+            c = rng_key.integers(0, C, N)
+            g = rng_key.integers(0, C, N)
+            base = np.where((lvl == 0)[:, None], par_f[h][p],
+                            np.where((lvl == 1)[:, None], ch_f[h][p, c], gc_f[h][p, c, g]))
+            base = base + rng_key.standard_normal((N, d)) * sigma
+            frac = cfg.get("noise", 0.0)
+            if frac > 0:
+                sel = rng_key.random(N) < frac
+                base[sel] = rng_key.uniform(-3.0, 3.0, size=(int(sel.sum()), d))
+            K[b, h] = base.astype(np.float32)
+    Q = np.random.default_rng(s_q).standard_normal((B, H, N, d), dtype=np.float32)
+    V = np.random.default_rng(s_v).standard_normal((B, H, N, d), dtype=np.float32)
+    return dict(
+        Q=_round_dtype(Q, dtype), K=_round_dtype(K, dtype), V=_round_dtype(V, dtype),
+        parents=_round_dtype(par_f, dtype), children=_round_dtype(ch_f, dtype),
+        grandchildren=_round_dtype(gc_f, dtype),
+        B=B, H=H, N=N, d=d, M0=M0, C=C, P=cfg["P"], P2=cfg.get("P2", cfg["P"]), block=cfg["block"],
+        scale=1.0 / math.sqrt(d), dtype=dtype, depth=3,
+    )
 
 
 def _tree_nodes(M0: int, C: int):

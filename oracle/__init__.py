@@ -75,6 +75,11 @@ class Oracle:
         lib.avq_oracle_attention_tiled.restype = None
         lib.avq_oracle_codebook_update.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_D] * 8
         lib.avq_oracle_codebook_update.restype = None
+        lib.avq_oracle_quantize3.argtypes = [ctypes.c_int] * 6 + [_D] * 5 + [_I32, _D, _I64, _D]
+        lib.avq_oracle_quantize3.restype = None
+        lib.avq_oracle_attention3.argtypes = ([ctypes.c_int] * 9 + [ctypes.c_double] + [_D] * 6
+                                              + [_I32, _I32, _D, _I32, _I32, _D, _D])
+        lib.avq_oracle_attention3.restype = None
         lib.avq_oracle_num_threads.restype = ctypes.c_int
         lib.avq_oracle_set_threads.argtypes = [ctypes.c_int]
         lib.avq_oracle_set_threads.restype = None
@@ -151,6 +156,50 @@ class Oracle:
                                             _p(imp, _D), int(tile))
         return O, sel_out, imp
 
+
+    # ---- depth-3 tree (Sec. 6, "deeper hierarchies") ------------------------
+    def quantize3(self, K, V, parents, children, grandchildren):
+        """Algorithm 1 one level deeper.  grandchildren [H,M0,C,C,d].  Returns
+        assign [B,H,N] (codes: parents, then M0*C children, then M0*C*C
+        grandchildren), vsum [B,H,Mt3,d], counts [B,H,Mt3], dec [B,H,N,6]."""
+        K, V, parents, children, grandchildren = map(_f64, (K, V, parents, children, grandchildren))
+        B, H, N, d = K.shape
+        M0 = parents.shape[1]
+        C = children.shape[2]
+        Mt = M0 + M0 * C + M0 * C * C
+        assign = np.empty((B, H, N), dtype=np.int32)
+        vsum = np.empty((B, H, Mt, d), dtype=np.float64)
+        counts = np.empty((B, H, Mt), dtype=np.int64)
+        dec = np.empty((B, H, N, 6), dtype=np.float64)
+        self.lib.avq_oracle_quantize3(B * H, H, N, d, M0, C, _p(K, _D), _p(V, _D), _p(parents, _D),
+                                      _p(children, _D), _p(grandchildren, _D), _p(assign, _I32),
+                                      _p(vsum, _D), _p(counts, _I64), _p(dec, _D))
+        return assign, vsum, counts, dec
+
+    def attention3(self, Q, parents, children, grandchildren, vsum, counts, P: int, P2: int,
+                   block: int, scale: float, sel=None, sel2=None):
+        """Algorithm 2 one level deeper.  Returns O [B,H,N,d], sel [B,H,nblk,P]
+        (parents), sel2 [B,H,nblk,P2] (child codes), importance [B,H,nblk,M0],
+        child importance [B,H,nblk,P*C] (candidates in the order of sel)."""
+        Q, parents, children, grandchildren, vsum = map(_f64, (Q, parents, children, grandchildren, vsum))
+        counts = _f64(counts)
+        B, H, N, d = Q.shape
+        M0 = parents.shape[1]
+        C = children.shape[2]
+        nblk = (N + block - 1) // block
+        O = np.full((B, H, N, d), np.nan)
+        sel_out = np.full((B, H, nblk, max(P, 0)), -1, dtype=np.int32)
+        sel2_out = np.full((B, H, nblk, max(P2, 0)), -1, dtype=np.int32)
+        imp = np.full((B, H, nblk, M0), np.nan)
+        imp2 = np.full((B, H, nblk, max(P * C, 0)), np.nan)
+        si = None if sel is None else np.ascontiguousarray(np.asarray(sel), dtype=np.int32)
+        si2 = None if sel2 is None else np.ascontiguousarray(np.asarray(sel2), dtype=np.int32)
+        self.lib.avq_oracle_attention3(B * H, H, N, d, M0, C, P, P2, block, float(scale), _p(Q, _D),
+                                       _p(parents, _D), _p(children, _D), _p(grandchildren, _D),
+                                       _p(vsum, _D), _p(counts, _D), _p(si, _I32), _p(si2, _I32),
+                                       _p(O, _D), _p(sel_out, _I32), _p(sel2_out, _I32), _p(imp, _D),
+                                       _p(imp2, _D))
+        return O, sel_out, sel2_out, imp, imp2
 
     # ---- Sec. A: codebook update -----------------------------------------
     def codebook_update(self, ksum, counts, S, Nst, parents, children, lam: float):

@@ -459,3 +459,273 @@ void avq_oracle_codebook_update(int B, int H, int d, int M0, int C, double lambd
     }
   free(Mc);
 }
+
+/* ------------------------------------------------------------------------
+ * Depth-3 tree: the "deeper hierarchies" named as the next step in the
+ * conclusion (Sec. 6).  Every child has C grandchildren and equals their
+ * mean, as every parent equals the mean of its children (Eq. 5).  Code
+ * layout per head: parents [0, M0), child (m, c) at M0 + m*C + c, grandchild
+ * (m, c, g) at M0 + M0*C + (m*C + c)*C + g.
+ *
+ * Readings (the pages name the extension but give no algorithm; these are
+ * Algorithms 1 and 2 applied once more, one level down):
+ *   - Algorithm 1 descends one more level: a key that moved to child c*
+ *     moves on to c*'s nearest grandchild (first strict minimum) only if that
+ *     grandchild is strictly closer than c*.  Statistics (Eq. 3): a key counts
+ *     at its parent, at its child if it moved, and at its grandchild if it
+ *     moved twice.
+ *   - Algorithm 2: after the child refinement of the top-P parents, each of
+ *     the P*C refined children gets an importance like Eq. 7, using the
+ *     logits and denominator of the attention after that refinement:
+ *     w_c(I) = sum_{i in I} exp(s_ic - m_i) n_c / z_i; the top-P2 of them
+ *     (descending, ties to the lower child code) are refined with their
+ *     grandchildren exactly as parents are with their children: the child's
+ *     logit is recovered as the mean of its grandchildren's (Eq. 8) and
+ *     dA = exp(s_ig) - exp(s_ic) (Eq. 9), zero for empty grandchildren.
+ * ---------------------------------------------------------------------- */
+
+/* Algorithm 1, depth 3, for one key: `dec` (nullable) receives 6 decision
+ * distances: the 4 of assign_one, then the best and second-best grandchild
+ * distance (INFINITY when the key did not move to a child). */
+static int32_t assign_one3(const double* k, const double* par_h, const double* ch_h,
+                           const double* gc_h, int d, int M0, int C, double* dec) {
+  int32_t code = assign_one(k, par_h, ch_h, d, M0, C, dec);
+  if (dec) { dec[4] = INFINITY; dec[5] = INFINITY; }
+  if (code < M0) return code;
+  /* the key sits at child c = code - M0 (c = m*C + c'): scan its grandchildren */
+  const int32_t c = code - M0;
+  const double d_child = sqdist(k, ch_h + (size_t)c * d, d);
+  double d_g = INFINITY, d_g2 = INFINITY;
+  int32_t g_star = 0;
+  for (int g = 0; g < C; ++g) {
+    double dg = sqdist(k, gc_h + ((size_t)c * C + g) * d, d);
+    if (dg < d_g) { /* first strict minimum */
+      d_g2 = d_g;
+      d_g = dg;
+      g_star = g;
+    } else if (dg < d_g2) {
+      d_g2 = dg;
+    }
+  }
+  if (dec) { dec[4] = d_g; dec[5] = d_g2; }
+  /* moves to the grandchild only when strictly closer than the child */
+  if (d_g < d_child) return M0 + M0 * C + c * C + g_star;
+  return code;
+}
+
+void avq_oracle_quantize3(int BH, int H, int N, int d, int M0, int C,
+                          const double* K, const double* V, const double* parents,
+                          const double* children, const double* grandchildren,
+                          int32_t* assign, double* vsum, int64_t* counts, double* dec) {
+  const int M1 = M0 * C, Mt = M0 + M1 + M1 * C;
+#pragma omp parallel for schedule(dynamic)
+  for (int bh = 0; bh < BH; ++bh) {
+    const int h = bh % H;
+    const double* par_h = parents + (size_t)h * M0 * d;
+    const double* ch_h = children + (size_t)h * M1 * d;
+    const double* gc_h = grandchildren + (size_t)h * M1 * C * d;
+    double* vs = vsum + (size_t)bh * Mt * d;
+    int64_t* ns = counts + (size_t)bh * Mt;
+    memset(vs, 0, sizeof(double) * (size_t)Mt * d);
+    memset(ns, 0, sizeof(int64_t) * (size_t)Mt);
+    for (int j = 0; j < N; ++j) {
+      const double* k = K + ((size_t)bh * N + j) * d;
+      const double* v = V + ((size_t)bh * N + j) * d;
+      double* dj = dec ? dec + ((size_t)bh * N + j) * 6 : NULL;
+      const int32_t code = assign_one3(k, par_h, ch_h, gc_h, d, M0, C, dj);
+      /* the key's parent, and its child when it moved at least once */
+      int32_t child = -1, a;
+      if (code < M0) a = code;
+      else if (code < M0 + M1) { child = code; a = (code - M0) / C; }
+      else { child = M0 + (code - M0 - M1) / C; a = (child - M0) / C; }
+      for (int t = 0; t < d; ++t) vs[(size_t)a * d + t] += v[t];
+      ns[a] += 1;
+      if (child >= 0) {
+        for (int t = 0; t < d; ++t) vs[(size_t)child * d + t] += v[t];
+        ns[child] += 1;
+      }
+      if (code >= M0 + M1) {
+        for (int t = 0; t < d; ++t) vs[(size_t)code * d + t] += v[t];
+        ns[code] += 1;
+      }
+      assign[(size_t)bh * N + j] = code;
+    }
+  }
+}
+
+/* top-P2 of the candidate children: descending importance, ties to the lower
+ * child code */
+static void top_p_codes(const double* w, const int32_t* code, int n, int P2, int32_t* out) {
+  char* taken = (char*)calloc((size_t)(n > 0 ? n : 1), 1);
+  for (int r = 0; r < P2; ++r) {
+    int best = -1;
+    for (int j = 0; j < n; ++j) {
+      if (taken[j]) continue;
+      if (best < 0 || w[j] > w[best] || (w[j] == w[best] && code[j] < code[best])) best = j;
+    }
+    taken[best] = 1;
+    out[r] = best;
+  }
+  free(taken);
+}
+
+/* Algorithm 2, depth 3, for one query block of one head. */
+static void attend_block3(int d, int M0, int C, int P, int P2, double scale,
+                          const double* Q, int i0, int i1, const double* par_h,
+                          const double* ch_h, const double* gc_h, const double* vs,
+                          const double* ns, const int32_t* sel_in, const int32_t* sel2_in,
+                          double* O, int32_t* sel_out, int32_t* sel2_out, double* imp_out,
+                          double* imp2_out) {
+  const int M1 = M0 * C;
+  const int nI = i1 - i0, nc = P * C;
+  double* s = (double*)malloc(sizeof(double) * (size_t)nI * M0);
+  double* A = (double*)malloc(sizeof(double) * (size_t)nI * M0);
+  double* m = (double*)malloc(sizeof(double) * (size_t)nI);
+  double* x = (double*)malloc(sizeof(double) * (size_t)nI * d);
+  double* z = (double*)malloc(sizeof(double) * (size_t)nI);
+  double* w = (double*)malloc(sizeof(double) * (size_t)M0);
+  int32_t* S = (int32_t*)malloc(sizeof(int32_t) * (size_t)(P > 0 ? P : 1));
+  double* sc = (double*)malloc(sizeof(double) * (size_t)nI * (nc > 0 ? nc : 1));
+  int32_t* ccode = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nc > 0 ? nc : 1));
+  double* w2 = (double*)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
+  int32_t* S2 = (int32_t*)malloc(sizeof(int32_t) * (size_t)(P2 > 0 ? P2 : 1));
+  double* sg = (double*)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1));
+
+  /* coarse pass over the parents, as in attend_block */
+  for (int r = 0; r < nI; ++r) {
+    const double* q = Q + (size_t)(i0 + r) * d;
+    for (int j = 0; j < M0; ++j) s[(size_t)r * M0 + j] = scale * dot(q, par_h + (size_t)j * d, d);
+    m[r] = -INFINITY;
+    for (int j = 0; j < M0; ++j)
+      if (ns[j] > 0 && s[(size_t)r * M0 + j] > m[r]) m[r] = s[(size_t)r * M0 + j];
+    for (int j = 0; j < M0; ++j)
+      A[(size_t)r * M0 + j] = ns[j] > 0 ? exp(s[(size_t)r * M0 + j] - m[r]) : 0.0;
+    for (int t = 0; t < d; ++t) x[(size_t)r * d + t] = 0.0;
+    z[r] = 0.0;
+    for (int j = 0; j < M0; ++j) {
+      double a = A[(size_t)r * M0 + j];
+      for (int t = 0; t < d; ++t) x[(size_t)r * d + t] += a * vs[(size_t)j * d + t];
+      z[r] += a * ns[j];
+    }
+  }
+  /* parents' importance (Eq. 7) and top-P */
+  for (int j = 0; j < M0; ++j) {
+    w[j] = 0.0;
+    for (int r = 0; r < nI; ++r) w[j] += A[(size_t)r * M0 + j] * ns[j] / z[r];
+  }
+  if (imp_out) memcpy(imp_out, w, sizeof(double) * (size_t)M0);
+  if (P > 0) {
+    if (sel_in) memcpy(S, sel_in, sizeof(int32_t) * (size_t)P);
+    else top_p(w, M0, P, S);
+    if (sel_out) memcpy(sel_out, S, sizeof(int32_t) * (size_t)P);
+  }
+  /* child refinement of the selected parents (online max merge, Eqs. 8-9) */
+  for (int k = 0; k < P; ++k)
+    for (int c = 0; c < C; ++c) ccode[k * C + c] = M0 + S[k] * C + c;
+  for (int r = 0; r < nI; ++r) {
+    const double* q = Q + (size_t)(i0 + r) * d;
+    for (int k = 0; k < P; ++k) {
+      const int p = S[k];
+      double* scr = sc + (size_t)r * nc + (size_t)k * C;
+      for (int c = 0; c < C; ++c) scr[c] = scale * dot(q, ch_h + ((size_t)p * C + c) * d, d);
+      double mp = m[r];
+      for (int c = 0; c < C; ++c)
+        if (ns[M0 + p * C + c] > 0 && scr[c] > mp) mp = scr[c];
+      double f = exp(m[r] - mp);
+      for (int t = 0; t < d; ++t) x[(size_t)r * d + t] *= f;
+      z[r] *= f;
+      m[r] = mp;
+      double sp = 0.0;
+      for (int c = 0; c < C; ++c) sp += scr[c];
+      sp /= C;
+      double Ap = exp(sp - m[r]);
+      for (int c = 0; c < C; ++c) {
+        const int x_c = M0 + p * C + c;
+        double dA = ns[x_c] > 0 ? exp(scr[c] - m[r]) - Ap : 0.0;
+        for (int t = 0; t < d; ++t) x[(size_t)r * d + t] += dA * vs[(size_t)x_c * d + t];
+        z[r] += dA * ns[x_c];
+      }
+    }
+  }
+  /* the refined children's importance, with the logits and denominator of
+   * the attention after the child refinement, and their top-P2 */
+  for (int u = 0; u < nc; ++u) {
+    w2[u] = 0.0;
+    const double n_u = ns[ccode[u]];
+    if (!(n_u > 0)) continue;
+    for (int r = 0; r < nI; ++r) w2[u] += exp(sc[(size_t)r * nc + u] - m[r]) * n_u / z[r];
+  }
+  if (imp2_out) memcpy(imp2_out, w2, sizeof(double) * (size_t)nc);
+  if (P2 > 0) {
+    if (sel2_in) {
+      /* caller's child codes -> candidate slots */
+      for (int k = 0; k < P2; ++k) {
+        S2[k] = 0;
+        for (int u = 0; u < nc; ++u)
+          if (ccode[u] == sel2_in[k]) S2[k] = u;
+      }
+    } else {
+      top_p_codes(w2, ccode, nc, P2, S2);
+    }
+    if (sel2_out)
+      for (int k = 0; k < P2; ++k) sel2_out[k] = ccode[S2[k]];
+  }
+  /* grandchild refinement of the selected children */
+  for (int r = 0; r < nI; ++r) {
+    const double* q = Q + (size_t)(i0 + r) * d;
+    for (int k = 0; k < P2; ++k) {
+      const int cc = ccode[S2[k]] - M0; /* child index m*C + c */
+      for (int g = 0; g < C; ++g) sg[g] = scale * dot(q, gc_h + ((size_t)cc * C + g) * d, d);
+      double mp = m[r];
+      for (int g = 0; g < C; ++g)
+        if (ns[M0 + M1 + cc * C + g] > 0 && sg[g] > mp) mp = sg[g];
+      double f = exp(m[r] - mp);
+      for (int t = 0; t < d; ++t) x[(size_t)r * d + t] *= f;
+      z[r] *= f;
+      m[r] = mp;
+      /* the child's logit as the mean of its grandchildren's (Eq. 8) */
+      double scm = 0.0;
+      for (int g = 0; g < C; ++g) scm += sg[g];
+      scm /= C;
+      double Ac = exp(scm - m[r]);
+      for (int g = 0; g < C; ++g) {
+        const int x_g = M0 + M1 + cc * C + g;
+        double dA = ns[x_g] > 0 ? exp(sg[g] - m[r]) - Ac : 0.0;
+        for (int t = 0; t < d; ++t) x[(size_t)r * d + t] += dA * vs[(size_t)x_g * d + t];
+        z[r] += dA * ns[x_g];
+      }
+    }
+  }
+  for (int r = 0; r < nI; ++r)
+    for (int t = 0; t < d; ++t) O[(size_t)(i0 + r) * d + t] = x[(size_t)r * d + t] / z[r];
+
+  free(s); free(A); free(m); free(x); free(z); free(w); free(S); free(sc); free(ccode);
+  free(w2); free(S2); free(sg);
+}
+
+/* Stage 2, depth 3, over every (bh, query block).  sel [BH][nblk][P] parents,
+ * sel2 [BH][nblk][P2] child codes, imp [BH][nblk][M0], imp2 [BH][nblk][P*C]
+ * (candidate children in the order of sel, C each); sel_in / sel2_in
+ * (nullable) override the two selections. */
+void avq_oracle_attention3(int BH, int H, int N, int d, int M0, int C, int P, int P2, int block,
+                           double scale, const double* Q, const double* parents,
+                           const double* children, const double* grandchildren,
+                           const double* vsum, const double* counts, const int32_t* sel_in,
+                           const int32_t* sel2_in, double* O, int32_t* sel_out,
+                           int32_t* sel2_out, double* imp_out, double* imp2_out) {
+  const int M1 = M0 * C, Mt = M0 + M1 + M1 * C;
+  const int nblk = (N + block - 1) / block;
+#pragma omp parallel for schedule(dynamic)
+  for (int u = 0; u < BH * nblk; ++u) {
+    const int bh = u / nblk, b = u % nblk, h = bh % H;
+    const int i0 = b * block, i1 = i0 + block < N ? i0 + block : N;
+    const size_t sb = (size_t)bh * nblk + b;
+    attend_block3(d, M0, C, P, P2, scale, Q + (size_t)bh * N * d, i0, i1,
+                  parents + (size_t)h * M0 * d, children + (size_t)h * M1 * d,
+                  grandchildren + (size_t)h * M1 * C * d, vsum + (size_t)bh * Mt * d,
+                  counts + (size_t)bh * Mt, sel_in ? sel_in + sb * P : NULL,
+                  sel2_in ? sel2_in + sb * P2 : NULL, O + (size_t)bh * N * d,
+                  sel_out ? sel_out + sb * P : NULL, sel2_out ? sel2_out + sb * P2 : NULL,
+                  imp_out ? imp_out + sb * M0 : NULL, imp2_out ? imp2_out + sb * P * C : NULL);
+  }
+}

@@ -188,3 +188,124 @@ def top_p_capture(mass, sel, N, block):
     sizes = np.array([min(block, N - k * block) for k in range(nblk)], dtype=np.float64)
     got = np.take_along_axis(mass, sel.astype(np.int64), axis=-1).sum(-1)  # [B,H,nblk]
     return float(np.mean(got / sizes))
+
+
+# ---- depth-3 tree --------------------------------------------------------
+def assign_brute3(K, parents, children, grandchildren):
+    """Final codes [B,H,N] of the depth-3 descent by full distance tables:
+    nearest parent; nearest child of it, taken when strictly closer; then
+    nearest grandchild of that child, taken when strictly closer than it."""
+    K, parents, children, grandchildren = map(_f64, (K, parents, children, grandchildren))
+    codes2 = assign_brute(K, parents, children)
+    B, H, N, d = K.shape
+    M0, C = parents.shape[1], children.shape[2]
+    M1 = M0 * C
+    codes = codes2.copy()
+    for b in range(B):
+        for h in range(H):
+            k = K[b, h]
+            c2 = codes2[b, h]
+            moved = np.nonzero(c2 >= M0)[0]
+            if moved.size == 0:
+                continue
+            cidx = c2[moved] - M0
+            ch = children[h].reshape(M1, d)[cidx]                      # [n, d]
+            gc = grandchildren[h].reshape(M1, C, d)[cidx]              # [n, C, d]
+            dch = ((k[moved] - ch) ** 2).sum(-1)
+            dg = ((k[moved][:, None, :] - gc) ** 2).sum(-1)            # [n, C]
+            g = dg.argmin(axis=1)
+            go = dg[np.arange(moved.size), g] < dch
+            codes[b, h, moved[go]] = M0 + M1 + cidx[go] * C + g[go]
+    return codes
+
+
+def _lineage3(codes, M0, C):
+    """(parent, child or -1, grandchild or -1) code arrays of depth-3 codes."""
+    codes = np.asarray(codes)
+    M1 = M0 * C
+    is_g = codes >= M0 + M1
+    is_c = (codes >= M0) & ~is_g
+    child = np.where(is_c, codes, np.where(is_g, M0 + (codes - M0 - M1) // C, -1))
+    parent = np.where(codes < M0, codes, (child - M0) // C)
+    grand = np.where(is_g, codes, -1)
+    return parent, child, grand
+
+
+def aggregate_brute3(codes, V, M0, C):
+    """Eq. 3 statistics of the depth-3 tree: a key counts at its parent, its
+    child (if it moved) and its grandchild (if it moved twice)."""
+    V = _f64(V)
+    B, H, N, d = V.shape
+    Mt = M0 + M0 * C + M0 * C * C
+    vs = np.zeros((B, H, Mt, d))
+    ns = np.zeros((B, H, Mt), dtype=np.int64)
+    parent, child, grand = _lineage3(codes, M0, C)
+    for b in range(B):
+        for h in range(H):
+            for lvl in (parent[b, h], child[b, h], grand[b, h]):
+                ok = lvl >= 0
+                np.add.at(vs[b, h], lvl[ok], V[b, h][ok])
+                np.add.at(ns[b, h], lvl[ok], 1)
+    return vs, ns
+
+
+def representative_attention3(Q, codes, V, parents, children, grandchildren, sel, sel2, block,
+                              scale, depth2_only=False):
+    """Exact softmax attention over representative keys of the depth-3 tree:
+    a key is represented by its grandchild if its child is among the block's
+    selected children, else by its child if its parent is among the block's
+    selected parents, else by its parent.  With `depth2_only` the grandchild
+    level is ignored (the representatives after the child refinement)."""
+    Q, V, parents, children, grandchildren = map(_f64, (Q, V, parents, children, grandchildren))
+    B, H, N, d = Q.shape
+    M0, C = parents.shape[1], children.shape[2]
+    M1 = M0 * C
+    parent, child, grand = _lineage3(codes, M0, C)
+    sel, sel2 = np.asarray(sel), np.asarray(sel2)
+    nblk = (N + block - 1) // block
+    Y = np.empty_like(Q)
+    for b in range(B):
+        for h in range(H):
+            pv = parents[h][parent[b, h]]
+            cv = children[h].reshape(M1, d)[np.clip(child[b, h] - M0, 0, M1 - 1)]
+            gv = grandchildren[h].reshape(M1 * C, d)[np.clip(grand[b, h] - M0 - M1, 0, M1 * C - 1)]
+            for blk in range(nblk):
+                i0, i1 = blk * block, min(N, (blk + 1) * block)
+                rep = pv.copy()
+                if sel.shape[-1] > 0:
+                    use_c = (child[b, h] >= 0) & np.isin(parent[b, h], sel[b, h, blk])
+                    rep[use_c] = cv[use_c]
+                    if not depth2_only and sel2.shape[-1] > 0:
+                        use_g = (grand[b, h] >= 0) & use_c & np.isin(child[b, h], sel2[b, h, blk])
+                        rep[use_g] = gv[use_g]
+                Y[b, h, i0:i1] = _softmax_rows(scale * Q[b, h, i0:i1] @ rep.T) @ V[b, h]
+    return Y
+
+
+def child_mass3(Q, codes, parents, children, grandchildren, sel, block, scale):
+    """Importance of the refined children written as a block sum of softmax
+    mass: for each block and each child of its selected parents (in the order
+    of sel, C each), the mass that exact softmax attention over the depth-2
+    representatives (after the child refinement) puts on the keys counted at
+    that child.  [B,H,nblk,P*C]"""
+    Q = _f64(Q)
+    B, H, N, d = Q.shape
+    M0, C = parents.shape[1], children.shape[2]
+    parent, child, _ = _lineage3(codes, M0, C)
+    parents_f, children_f = _f64(parents), _f64(children)
+    sel = np.asarray(sel)
+    P = sel.shape[-1]
+    nblk = (N + block - 1) // block
+    W = np.zeros((B, H, nblk, P * C))
+    for b in range(B):
+        for h in range(H):
+            for blk in range(nblk):
+                i0, i1 = blk * block, min(N, (blk + 1) * block)
+                use_c = (child[b, h] >= 0) & np.isin(parent[b, h], sel[b, h, blk])
+                rep = parents_f[h][parent[b, h]].copy()
+                rep[use_c] = children_f[h].reshape(M0 * C, d)[child[b, h][use_c] - M0]
+                mass = _softmax_rows(scale * Q[b, h, i0:i1] @ rep.T).sum(axis=0)  # [N]
+                for k, p in enumerate(sel[b, h, blk]):
+                    for c in range(C):
+                        W[b, h, blk, k * C + c] = mass[child[b, h] == M0 + p * C + c].sum()
+    return W

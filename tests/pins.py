@@ -511,9 +511,190 @@ def pin_codebook_massless(orc):
     assert np.allclose(po[0, 1], ksum[0, 0, 1] / 4)
 
 
+# ---- depth-3 tree (Sec. 6, "deeper hierarchies") ----------------------------
+def case3_small():
+    cfg = dict(dtype="bf16", B=1, H=2, N=600, d=32, M0=8, C=4, P=3, P2=4, block=128,
+               key_sigma=0.03)
+    return synth.make_inputs3(cfg, 14)
+
+
+def case3_wide():
+    cfg = dict(dtype="f32", B=1, H=1, N=700, d=64, M0=16, C=8, P=4, P2=6, block=64,
+               key_sigma=0.03, noise=0.05)
+    return synth.make_inputs3(cfg, 15)
+
+
+CASES3 = (case3_small, case3_wide)
+
+
+def _run3(orc, inp, P=None, P2=None, sel=None, sel2=None):
+    P = inp["P"] if P is None else P
+    P2 = inp["P2"] if P2 is None else P2
+    a, vs, ns, _ = orc.quantize3(inp["K"], inp["V"], inp["parents"], inp["children"], inp["grandchildren"])
+    O, s1, s2, w1, w2 = orc.attention3(inp["Q"], inp["parents"], inp["children"], inp["grandchildren"],
+                                        vs, ns, P, P2, inp["block"], inp["scale"], sel=sel, sel2=sel2)
+    return a, vs, ns, O, s1, s2, w1, w2
+
+
+def pin3_assign_brute(orc):
+    """Depth-3 codes equal the full distance-table descent (Alg. 1, one level deeper)."""
+    for mk in CASES3:
+        inp = mk()
+        a, _, _, _ = orc.quantize3(inp["K"], inp["V"], inp["parents"], inp["children"], inp["grandchildren"])
+        ref = brute.assign_brute3(inp["K"], inp["parents"], inp["children"], inp["grandchildren"])
+        assert (a == ref).all(), (mk.__name__, int((a != ref).sum()))
+        M0, C = inp["M0"], inp["C"]
+        assert (a >= M0 + M0 * C).any() and ((a >= M0) & (a < M0 + M0 * C)).any() and (a < M0).any()
+
+
+def pin3_strict_ties(orc):
+    """Depth-3 ties by hand (d = 2, one parent, C = 3): a key equally far from
+    two grandchildren takes the first; a key whose best grandchild is exactly
+    as far as its child stays at the child (the strict comparisons of
+    Algorithm 1, one level down)."""
+    par = np.array([[[0.0, 0.0]]])
+    ch = np.array([[[[2.0, 0.0], [-2.0, 0.0], [0.0, 0.0]]]])
+    gc = np.array([[[[[3.0, 1.0], [3.0, -1.0], [0.0, 0.0]],
+                     [[-3.0, 1.0], [-3.0, -1.0], [0.0, 0.0]],
+                     [[1.0, 0.0], [-1.0, 0.0], [0.0, 0.0]]]]])
+    assert np.array_equal(gc.mean(3), ch) and np.array_equal(ch.mean(2), par)
+    K = np.array([[3.2, 0.0],    # child 0 (1.44 < 10.24); grandchildren 0 and 1 tie at 1.04 -> g0
+                  [3.0, 0.0],    # child 0 at 1; best grandchild also at 1: stays at child 0
+                  [-3.2, 0.0],   # child 1, its grandchild 0
+                  [0.0, 0.0],    # on the parent: no child strictly closer
+                  [0.9, 0.0]])   # child 2 coincides with the parent, equally far: stays at the parent
+    a, _, _, _ = orc.quantize3(K[None, None], np.ones((1, 1, 5, 2)), par, ch, gc)
+    # codes: parent 0; children 1..3; grandchild (c, g) at 4 + 3 c + g
+    assert a[0, 0].tolist() == [4, 1, 7, 0, 0], a
+
+
+def pin3_aggregate(orc):
+    """Depth-3 statistics (Eq. 3 at three levels) and their invariants."""
+    for mk in CASES3:
+        inp = mk()
+        M0, C, N = inp["M0"], inp["C"], inp["N"]
+        M1 = M0 * C
+        a, vs, ns, _ = orc.quantize3(inp["K"], inp["V"], inp["parents"], inp["children"], inp["grandchildren"])
+        vs_ref, ns_ref = brute.aggregate_brute3(a, inp["V"], M0, C)
+        assert (ns == ns_ref).all()
+        assert _rel(vs, vs_ref) < 1e-12
+        assert (ns[..., :M0].sum(-1) == N).all()
+        ch = ns[..., M0:M0 + M1].reshape(*ns.shape[:-1], M0, C).sum(-1)
+        gc = ns[..., M0 + M1:].reshape(*ns.shape[:-1], M1, C).sum(-1)
+        assert (ch <= ns[..., :M0]).all() and (gc <= ns[..., M0:M0 + M1]).all()
+        assert (gc.sum(-1) == (a >= M0 + M1).sum(-1)).all()
+
+
+def pin3_representative(orc):
+    """Depth-3 output equals exact softmax attention over representative keys
+    (the Sec. C identity applied at both levels), for several (P, P2)."""
+    for mk in CASES3:
+        inp = mk()
+        M0, C = inp["M0"], inp["C"]
+        for P, P2 in ((1, 1), (inp["P"], inp["P2"]), (M0, M0 * C), (inp["P"], 0)):
+            a, vs, ns, O, s1, s2, _, _ = _run3(orc, inp, P=P, P2=P2)
+            Y = brute.representative_attention3(inp["Q"], a, inp["V"], inp["parents"], inp["children"],
+                                                inp["grandchildren"], s1, s2, inp["block"], inp["scale"])
+            assert _rel(O, Y) < 1e-10, (mk.__name__, P, P2, _rel(O, Y))
+
+
+def pin3_limits(orc):
+    """P = 0 is flat VQ attention over the parents (Eq. 4); P2 = 0 is the
+    depth-2 method on the same parent and child statistics."""
+    inp = case3_small()
+    M0, C = inp["M0"], inp["C"]
+    a, vs, ns, O, _, _, _, _ = _run3(orc, inp, P=0, P2=0)
+    Y = brute.flat_vq_attention(inp["Q"], inp["parents"], vs[..., :M0, :], ns[..., :M0], inp["scale"])
+    assert _rel(O, Y) < 1e-10
+    a, vs, ns, O, s1, _, _, _ = _run3(orc, inp, P2=0)
+    k2 = M0 + M0 * C
+    O2, s2d, _ = orc.attention(inp["Q"], inp["parents"], inp["children"], vs[..., :k2, :], ns[..., :k2],
+                               inp["P"], inp["block"], inp["scale"])
+    assert (s2d == s1).all()
+    assert _rel(O, O2) < 1e-12
+
+
+def pin3_exact_codebook(orc):
+    """Keys placed on the grandchildren, every parent and every child refined:
+    exact attention (Eq. 1).  Keys on the children with every parent refined:
+    exact attention for any P2."""
+    rng = np.random.default_rng(33)
+    H, M0, C, d, N = 1, 6, 3, 8, 200
+    par, ch, gc = synth.make_codebook3(rng, H, M0, C, d, sigma_c=0.4, sigma_g=0.1)
+    par, ch, gc = par / 64.0, ch / 64.0, gc / 64.0
+    Q = rng.standard_normal((1, H, N, d))
+    V = rng.standard_normal((1, H, N, d))
+    pick = rng.integers(0, M0 * C * C, N)
+    K = gc[0].reshape(M0 * C * C, d)[pick][None, None]
+    a, vs, ns, _ = orc.quantize3(K, V, par, ch, gc)
+    assert (a >= M0 + M0 * C).all()
+    O, _, _, _, _ = orc.attention3(Q, par, ch, gc, vs, ns, M0, M0 * C, 64, 0.5)
+    assert _rel(O, brute.exact_attention(Q, K, V, 0.5)) < 1e-10
+    K = ch[0].reshape(M0 * C, d)[rng.integers(0, M0 * C, N)][None, None]
+    a, vs, ns, _ = orc.quantize3(K, V, par, ch, gc)
+    assert ((a >= M0) & (a < M0 + M0 * C)).all()
+    for P2 in (0, 2, M0 * C):
+        O, _, _, _, _ = orc.attention3(Q, par, ch, gc, vs, ns, M0, P2, 64, 0.5)
+        assert _rel(O, brute.exact_attention(Q, K, V, 0.5)) < 1e-10
+
+
+def pin3_child_importance(orc):
+    """The refined children's importance is the block sum of the softmax mass
+    that attention over the depth-2 representatives puts on each child's
+    keys; it never exceeds the block's rows; the second selection is the
+    top-P2 of it, ties to the lower child code."""
+    for mk in CASES3:
+        inp = mk()
+        a, vs, ns, O, s1, s2, w1, w2 = _run3(orc, inp)
+        W = brute.child_mass3(inp["Q"], a, inp["parents"], inp["children"], inp["grandchildren"], s1,
+                              inp["block"], inp["scale"])
+        assert _rel(w2, W) < 1e-10
+        N, blk = inp["N"], inp["block"]
+        sizes = np.array([min(blk, N - k * blk) for k in range(w2.shape[2])], dtype=np.float64)
+        assert (w2.sum(-1) <= sizes[None, None, :] * (1 + 1e-12)).all()
+        C, M0 = inp["C"], inp["M0"]
+        for idx in np.ndindex(*s2.shape[:3]):
+            codes = (M0 + s1[idx][:, None] * C + np.arange(C)[None, :]).reshape(-1)
+            order = np.lexsort((codes, -w2[idx]))[: inp["P2"]]
+            assert s2[idx].tolist() == codes[order].tolist()
+    # exact ties: zero queries, one key on every grandchild (equal counts per level)
+    rng = np.random.default_rng(44)
+    M0, C, d = 4, 3, 8
+    par, ch, gc = synth.make_codebook3(rng, 1, M0, C, d, sigma_c=0.2, sigma_g=0.05)
+    # parents pushed apart (offsets kept, so the means still hold exactly)
+    big = 8 * par
+    ch, gc = ch - par[:, :, None] + big[:, :, None], gc - par[:, :, None, None] + big[:, :, None, None]
+    par, ch, gc = big / 64.0, ch / 64.0, gc / 64.0
+    K = gc[0].reshape(M0 * C * C, d)[None, None]
+    V = rng.standard_normal(K.shape)
+    Q = np.zeros_like(K)
+    a, vs, ns, _ = orc.quantize3(K, V, par, ch, gc)
+    assert (a[0, 0] == M0 + M0 * C + np.arange(M0 * C * C)).all()  # every key on its grandchild
+    _, s1, s2, _, w2 = orc.attention3(Q, par, ch, gc, vs, ns, 2, 3, 64, 1.0)
+    assert s1[0, 0, 0].tolist() == [0, 1]
+    assert np.all(w2[0, 0, 0] == w2[0, 0, 0, 0])
+    assert s2[0, 0, 0].tolist() == [M0, M0 + 1, M0 + 2]
+
+
+def pin3_zero_offsets(orc):
+    """Grandchildren equal to their child: no key moves to a grandchild (the
+    move needs a strictly smaller distance), and refining children changes
+    nothing."""
+    inp = dict(case3_small())
+    gc = inp["grandchildren"].clone()
+    gc[:] = inp["children"][..., None, :]
+    inp["grandchildren"] = gc
+    a, vs, ns, O, _, _, _, _ = _run3(orc, inp)
+    M0, C = inp["M0"], inp["C"]
+    assert (a < M0 + M0 * C).all() and (ns[..., M0 + M0 * C:] == 0).all()
+    _, _, _, O0, _, _, _, _ = _run3(orc, inp, P2=0)
+    assert _rel(O, O0) < 1e-12
+
+
 ALL_PINS = [pin_hand_worked, pin_assign_brute, pin_aggregate, pin_aggregate_given_codes,
             pin_representative,
             pin_rescale_exercised, pin_flat_p0, pin_exact_codebook, pin_importance, pin_topp,
             pin_relabel, pin_key_permutation, pin_keys_on_codewords, pin_strict_ties,
             pin_masking, pin_counting, pin_tiled_importance, pin_codebook_update,
-            pin_codebook_massless]
+            pin_codebook_massless, pin3_assign_brute, pin3_strict_ties, pin3_aggregate, pin3_representative,
+            pin3_limits, pin3_exact_codebook, pin3_child_importance, pin3_zero_offsets]
