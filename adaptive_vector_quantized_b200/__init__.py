@@ -66,6 +66,10 @@ def lib() -> ctypes.CDLL:
                 L.avq_attention.argtypes = [P(avq_dims), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                             _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+                L.avq_quantize3.argtypes = [P(avq_dims), ctypes.c_int] + [_vp] * 8 + [_vp]
+                L.avq_attention3.argtypes = ([P(avq_dims), ctypes.c_int] + [_vp] * 6
+                                             + [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float]
+                                             + [_vp] * 5 + [_vp])
                 L.avq_codebook_update.argtypes = [P(avq_dims), ctypes.c_int, ctypes.c_float, _vp, _vp,
                                                   _vp, _vp, _vp, _vp, _vp]
                 L.avq_permute.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -84,6 +88,7 @@ def lib() -> ctypes.CDLL:
                 L.avq_status_string.argtypes = [ctypes.c_int]
                 L.avq_version.restype = ctypes.c_int
                 for name in ("avq_quantize", "avq_quantize_noalloc", "avq_attention", "avq_permute",
+                             "avq_quantize3", "avq_attention3",
                              "avq_hilbert_order", "avq_gilbert_order", "avq_check_device",
                              "avq_codebook_update", "avq_selftest_wait"):
                     getattr(L, name).restype = ctypes.c_int
@@ -293,6 +298,88 @@ def avq_attention(Q, parents, children, vsum, counts, P: int, block: int = 128, 
                                    int(two_pass), _ptr(O), _ptr(sel) if P > 0 else None,
                                    _ptr(imp), wp, wn, _stream(stream)))
     return O, sel, imp
+
+
+def m_total3(M0: int, C: int) -> int:
+    """Codes of a depth-3 tree: M0 parents, M0*C children, M0*C*C grandchildren."""
+    return M0 + M0 * C + M0 * C * C
+
+
+def _dims3(X, parents, children, grandchildren):
+    B, H, N, d = X.shape
+    Hp, M0, dp = parents.shape
+    if Hp != H or dp != d:
+        raise ValueError("parents must be [H, M0, d]")
+    C = children.shape[2]
+    if tuple(children.shape) != (H, M0, C, d):
+        raise ValueError("children must be [H, M0, C, d]")
+    if tuple(grandchildren.shape) != (H, M0, C, C, d):
+        raise ValueError("grandchildren must be [H, M0, C, C, d]")
+    return avq_dims(B, H, N, d, M0, C)
+
+
+def avq_quantize3(K, V, parents, children, grandchildren, assign=None, vsum=None, counts=None,
+                  stream=None):
+    """Stage 1 over a depth-3 tree.  K, V [B,H,N,d]; parents [H,M0,d];
+    children [H,M0,C,d]; grandchildren [H,M0,C,C,d].  Returns (assign [B,H,N]
+    int32, vsum [B,H,Mt3,d] fp32, counts [B,H,Mt3] int32), Mt3 = m_total3."""
+    dims = _dims3(K, parents, children, grandchildren)
+    dt = _dtype_code(K)
+    B, H, N, d = K.shape
+    Mt = m_total3(dims.M0, dims.C)
+    dev = K.device
+    _expect(V, "V", K.shape, K.dtype, dev)
+    for t, nm in ((parents, "parents"), (children, "children"), (grandchildren, "grandchildren")):
+        _expect(t, nm, t.shape, K.dtype, dev)
+    _expect(assign, "assign", (B, H, N), torch.int32, dev)
+    _expect(vsum, "vsum", (B, H, Mt, d), torch.float32, dev)
+    _expect(counts, "counts", (B, H, Mt), torch.int32, dev)
+    if assign is None:
+        assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    if vsum is None:
+        vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
+    if counts is None:
+        counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().avq_quantize3(ctypes.byref(dims), dt, _ptr(K), _ptr(V), _ptr(parents), _ptr(children),
+                                   _ptr(grandchildren), _ptr(assign), _ptr(vsum), _ptr(counts),
+                                   _stream(stream)))
+    return assign, vsum, counts
+
+
+def avq_attention3(Q, parents, children, grandchildren, vsum, counts, P: int, P2: int, block: int = 128,
+                   scale=None, O=None, importance=False, stream=None):
+    """Stage 2 over a depth-3 tree.  Returns (O [B,H,N,d], sel [B,H,nblk,P]
+    parents, sel2 [B,H,nblk,P2] child codes, importance [B,H,nblk,M0] or None,
+    importance2 [B,H,nblk,P*C] or None)."""
+    dims = _dims3(Q, parents, children, grandchildren)
+    dt = _dtype_code(Q)
+    B, H, N, d = Q.shape
+    M0, C = dims.M0, dims.C
+    Mt = m_total3(M0, C)
+    nblk = (N + block - 1) // block
+    dev = Q.device
+    if scale is None:
+        scale = d ** -0.5
+    for t, nm in ((parents, "parents"), (children, "children"), (grandchildren, "grandchildren")):
+        _expect(t, nm, t.shape, Q.dtype, dev)
+    _expect(vsum, "vsum", (B, H, Mt, d), torch.float32, dev)
+    _expect(counts, "counts", (B, H, Mt), torch.int32, dev)
+    _expect(O, "O", Q.shape, Q.dtype, dev)
+    if O is None:
+        O = torch.empty_like(Q)
+    sel = torch.empty((B, H, nblk, max(P, 0)), dtype=torch.int32, device=dev)
+    sel2 = torch.empty((B, H, nblk, max(P2, 0)), dtype=torch.int32, device=dev)
+    imp = imp2 = None
+    if importance:
+        imp = torch.empty((B, H, nblk, M0), dtype=torch.float32, device=dev)
+        imp2 = torch.empty((B, H, nblk, max(P * C, 1)), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().avq_attention3(ctypes.byref(dims), dt, _ptr(Q), _ptr(parents), _ptr(children),
+                                    _ptr(grandchildren), _ptr(vsum), _ptr(counts), int(P), int(P2),
+                                    int(block), float(scale), _ptr(O), _ptr(sel) if P > 0 else None,
+                                    _ptr(sel2) if P2 > 0 else None, _ptr(imp), _ptr(imp2), _stream(stream)))
+    return O, sel, sel2, imp, imp2
 
 
 def avq_codebook_update(ksum, counts, S, Nst, parents, children, lam: float, stream=None):

@@ -85,7 +85,7 @@ __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* ac
 template <typename T, int D>
 __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum, int BH, int N,
-    int M0, int C, int keys_per_warp) {
+    int Mt, int keys_per_warp) {
   constexpr int E = D / 32;
   using F = Frag<T, E>;
   constexpr int B = F::kBatch;  // keys loaded at once (32 / B batches per group)
@@ -96,7 +96,6 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   const int j0 = (gw % warps_per_head) * keys_per_warp;
   const int j1 = min(N, j0 + keys_per_warp);
   if (bh >= BH || j0 >= j1) return;
-  const int Mt = M0 * (1 + C);
   float* vs = vsum + (size_t)bh * Mt * D;
   const T* vb = V + (size_t)bh * N * D + lane * E;
   const int32_t* asg = assign + (size_t)bh * N;
@@ -168,21 +167,23 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   if (cur >= 0) flush();
 }
 
-// Parents hold their whole cluster: add the children's sums (keys that moved)
-// to the parent's own (keys that stayed), children in index order.
-__global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restrict__ vsum, int BH, int M0, int C,
-                                                               int D) {
-  const int Mt = M0 * (1 + C);
-  const long long total = (long long)BH * M0 * D;
+// Nodes hold their whole subtree: add the sums of the n nodes' children
+// (keys that moved on) to each node's own (keys that stopped there), children
+// in index order.  Node i of the level starting at code `lo` has its C
+// children at codes lo2 + i*C .. lo2 + i*C + C - 1 (for a two-level tree:
+// lo = 0, n = M0, lo2 = M0).
+__global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restrict__ vsum, int BH, int Mt, int lo,
+                                                               int n, int lo2, int C, int D) {
+  const long long total = (long long)BH * n * D;
   for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
        u += (long long)gridDim.x * blockDim.x) {
     const int t = (int)(u % D);
     const long long bp = u / D;
-    const int p = (int)(bp % M0);
-    float* vs = vsum + (bp / M0) * (long long)Mt * D;
-    float s = vs[(size_t)p * D + t];
-    for (int c = 0; c < C; ++c) s += vs[(size_t)(M0 + p * C + c) * D + t];
-    vs[(size_t)p * D + t] = s;
+    const int p = (int)(bp % n);
+    float* vs = vsum + (bp / n) * (long long)Mt * D;
+    float s = vs[(size_t)(lo + p) * D + t];
+    for (int c = 0; c < C; ++c) s += vs[(size_t)(lo2 + p * C + c) * D + t];
+    vs[(size_t)(lo + p) * D + t] = s;
   }
 }
 
@@ -367,10 +368,11 @@ size_t aggregate_det_workspace(const Shape& s) {
 
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log, bool vsum_zeroed) {
+                             LaunchLog& log, bool vsum_zeroed, bool depth3) {
   cudaError_t e = cudaSuccess;
+  const int Mt = depth3 ? s.M0 + s.M0 * s.C + s.M0 * s.C * s.C : s.Mt();
   if (!vsum_zeroed) {
-    e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * s.Mt() * s.d * sizeof(float), st);
+    e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * Mt * s.d * sizeof(float), st);
     if (e != cudaSuccess) return e;
   }
   (void)counts;
@@ -385,7 +387,7 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   const unsigned blocks = (unsigned)((warps + (kStreamThreads / 32) - 1) / (kStreamThreads / 32));
 #define AVQ_STREAM(T, D)                                                                            \
   aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, s.BH(), \
-                                                                   s.N, s.M0, s.C, kpw)
+                                                                   s.N, Mt, kpw)
   if (dt == AVQ_F32) {
     if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
   } else {
@@ -397,7 +399,13 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   if (s.C > 0) {
     const long long work = (long long)s.BH() * s.M0 * s.d;
     const int pb = (int)std::min<long long>((work + 255) / 256, (long long)sms * 8);
-    aggregate_parents_kernel<<<pb, 256, 0, st>>>(vsum, s.BH(), s.M0, s.C, s.d);
+    if (depth3) {  // children first take their grandchildren's sums
+      const long long work3 = (long long)s.BH() * s.M0 * s.C * s.d;
+      const int pb3 = (int)std::min<long long>((work3 + 255) / 256, (long long)sms * 8);
+      aggregate_parents_kernel<<<pb3, 256, 0, st>>>(vsum, s.BH(), Mt, s.M0, s.M0 * s.C, s.M0 + s.M0 * s.C,
+                                                    s.C, s.d);
+    }
+    aggregate_parents_kernel<<<pb, 256, 0, st>>>(vsum, s.BH(), Mt, 0, s.M0, s.M0, s.C, s.d);
   }
   log.add(s.C > 0 ? "aggregate_stream aggregate_parents" : "aggregate_stream");
   (void)err;

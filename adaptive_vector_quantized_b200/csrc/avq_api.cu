@@ -308,6 +308,79 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, c
   return AVQ_OK;
 }
 
+avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, const void* V,
+                         const void* parents, const void* children, const void* grandchildren,
+                         int32_t* assign, float* vsum, int32_t* counts, avq_stream_t stream) {
+  t_error[0] = 0;
+  avq_status st = check_dims(dims, dtype);
+  if (st != AVQ_OK) return st;
+  const Shape s = to_shape(dims);
+  if (s.C < 1) return fail(AVQ_ERR_INVALID_ARG, "a depth-3 tree needs C >= 1 (got %d)", s.C);
+  AVQ_REQUIRE_PTR(K, "K");
+  AVQ_REQUIRE_PTR(V, "V");
+  AVQ_REQUIRE_PTR(parents, "parents");
+  AVQ_REQUIRE_PTR(children, "children");
+  AVQ_REQUIRE_PTR(grandchildren, "grandchildren");
+  AVQ_REQUIRE_PTR(assign, "assign");
+  AVQ_REQUIRE_PTR(vsum, "vsum");
+  AVQ_REQUIRE_PTR(counts, "counts");
+  if (t_path == AVQ_PATH_TC) return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core kernel for a depth-3 tree");
+  if (injected("quantize3")) return injected_fail("avq_quantize3");
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const size_t mt3 = (size_t)s.M0 + (size_t)s.M0 * s.C + (size_t)s.M0 * s.C * s.C;
+  LaunchLog log{};
+  unsigned int* err = error_word();
+  if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+  cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * mt3 * sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "zero counts");
+  e = launch_assign3_simt(s, dtype, K, parents, children, grandchildren, assign, counts, cs, log);
+  if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
+  e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, false, true);
+  if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}
+
+avq_status avq_attention3(const avq_dims* dims, avq_dtype dtype, const void* Q, const void* parents,
+                          const void* children, const void* grandchildren, const float* vsum,
+                          const int32_t* counts, int P, int P2, int block, float scale, void* O,
+                          int32_t* sel, int32_t* sel2, float* importance, float* importance2,
+                          avq_stream_t stream) {
+  t_error[0] = 0;
+  avq_status st = check_dims(dims, dtype);
+  if (st != AVQ_OK) return st;
+  const Shape s = to_shape(dims);
+  if (s.C < 1) return fail(AVQ_ERR_INVALID_ARG, "a depth-3 tree needs C >= 1 (got %d)", s.C);
+  if (P < 0 || P > s.M0) return fail(AVQ_ERR_INVALID_ARG, "P must be in [0, M0] (got %d)", P);
+  if (P2 < 0 || P2 > P * s.C)
+    return fail(AVQ_ERR_INVALID_ARG, "P2 must be in [0, P*C] (got %d with P*C = %d)", P2, P * s.C);
+  if (block != 64 && block != 128)
+    return fail(AVQ_ERR_UNSUPPORTED, "block must be 64 or 128 (got %d)", block);
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(AVQ_ERR_INVALID_ARG, "scale must be finite and > 0");
+  AVQ_REQUIRE_PTR(Q, "Q");
+  AVQ_REQUIRE_PTR(parents, "parents");
+  AVQ_REQUIRE_PTR(children, "children");
+  AVQ_REQUIRE_PTR(grandchildren, "grandchildren");
+  AVQ_REQUIRE_PTR(vsum, "vsum");
+  AVQ_REQUIRE_PTR(counts, "counts");
+  AVQ_REQUIRE_PTR(O, "O");
+  if (P > 0) AVQ_REQUIRE_PTR(sel, "sel");
+  if (P2 > 0) AVQ_REQUIRE_PTR(sel2, "sel2");
+  if (importance != nullptr && !aligned(importance, 16))
+    return fail(AVQ_ERR_INVALID_ARG, "importance is not 16-byte aligned");
+  if (importance2 != nullptr && !aligned(importance2, 16))
+    return fail(AVQ_ERR_INVALID_ARG, "importance2 is not 16-byte aligned");
+  if (t_path == AVQ_PATH_TC) return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core kernel for a depth-3 tree");
+  if (injected("attention3")) return injected_fail("avq_attention3");
+  LaunchLog log{};
+  cudaError_t e = launch_attention3_simt(s, dtype, Q, parents, children, grandchildren, vsum, counts, P, P2,
+                                         block, scale, O, sel, sel2, importance, importance2,
+                                         reinterpret_cast<cudaStream_t>(stream), log);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
+  return AVQ_OK;
+}
+
 avq_status avq_codebook_update(const avq_dims* dims, avq_dtype dtype, float lambda, const float* ksum,
                                const int32_t* counts, float* S, float* Nst, void* parents, void* children,
                                avq_stream_t stream) {

@@ -32,10 +32,24 @@ cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, cons
                                const void* children, int32_t* assign, int32_t* counts,
                                cudaStream_t st, LaunchLog& log);
 // Algorithm 1, value sums for given codes, streaming variant.
-// vsum is zeroed inside; counts are left to the assignment kernels.
+// vsum is zeroed inside; counts are left to the assignment kernels.  depth3:
+// codes of a three-level tree (parents, M0*C children, M0*C*C grandchildren).
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log, bool vsum_zeroed = false);
+                             LaunchLog& log, bool vsum_zeroed = false, bool depth3 = false);
+// Depth-3 tree (three levels, codes parents | M0*C children | M0*C*C
+// grandchildren): assignment one level deeper on the CUDA cores; counts are
+// added into counts[BH][Mt3], which the caller zeroes first.
+cudaError_t launch_assign3_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
+                                const void* children, const void* grandchildren, int32_t* assign,
+                                int32_t* counts, cudaStream_t st, LaunchLog& log);
+// Depth-3 attention on the CUDA cores: parents, the top-P parents' children,
+// the top-P2 refined children's grandchildren.
+cudaError_t launch_attention3_simt(const Shape& s, avq_dtype dt, const void* Q, const void* parents,
+                                   const void* children, const void* grandchildren, const float* vsum,
+                                   const int32_t* counts, int P, int P2, int block, float scale, void* O,
+                                   int32_t* sel, int32_t* sel2, float* importance, float* importance2,
+                                   cudaStream_t st, LaunchLog& log);
 // Deterministic aggregation (fixed-order sums, independent of the grid).
 size_t aggregate_det_workspace(const Shape& s);
 cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,

@@ -68,6 +68,24 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+def algorithmic3(cfg):
+    """Bytes and tensor-free FLOPs of a depth-3 step (parents, M0*C children,
+    M0*C*C grandchildren; P parents and P2 children refined per block)."""
+    B, H, N, d, M0, C, P, blk = (cfg[k] for k in ("B", "H", "N", "d", "M0", "C", "P", "block"))
+    P2 = cfg.get("P2", P)
+    s = 2 if cfg["dtype"] == "bf16" else 4
+    BH = B * H
+    Mt = M0 + M0 * C + M0 * C * C
+    nblk = -(-N // blk)
+    stats = BH * Mt * (4 * d + 4)
+    code = H * Mt * d * s
+    s1_bytes = 2 * BH * N * d * s + code + stats + 4 * BH * N
+    s1_flops = 2 * BH * N * (M0 + 2 * C) * d
+    s2_bytes = BH * N * d * 2 * s + stats + code + 4 * BH * nblk * (P + P2)
+    s2_flops = 4 * BH * N * (M0 + P * C + P2 * C) * d + 2 * BH * N * P * C * d
+    return dict(s1_bytes=s1_bytes, s1_flops=s1_flops, s2_bytes=s2_bytes, s2_flops=s2_flops)
+
+
 def algorithmic(cfg):
     """Bytes and tensor FLOPs the method must move/compute per step, per stage.
 
@@ -237,6 +255,8 @@ def workload_config(name, cfg):
     keys = ("B", "H", "N", "d", "M0", "C", "P", "block")
     out = {"workload": name}
     out.update({k: cfg[k] for k in keys})
+    if cfg.get("depth", 2) == 3:
+        out.update(depth=3, P2=cfg.get("P2", cfg["P"]))
     out["order"] = cfg.get("order", "natural")
     out["two_pass"] = int(cfg.get("two_pass", False))
     return out
@@ -270,24 +290,39 @@ def run_avq(args, cfg, inp, n_global=None):
     stream = torch.cuda.current_stream(dev)
     dims = avq.avq_dims(B, H, N, d, cfg["M0"], cfg["C"])
     dt = avq.AVQ_BF16 if cfg["dtype"] == "bf16" else avq.AVQ_F32
-    ws = avq.workspace(dims, dt, dev, two_pass=two_pass, P=P, block=block)
-    Mt = cfg["M0"] * (1 + cfg["C"])
+    depth3 = cfg.get("depth", 2) == 3
+    ws = None if depth3 else avq.workspace(dims, dt, dev, two_pass=two_pass, P=P, block=block)
+    Mt = avq.m_total3(cfg["M0"], cfg["C"]) if depth3 else cfg["M0"] * (1 + cfg["C"])
     nblk = -(-N // block)
     assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
     vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
     counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
     sel = torch.empty((B, H, nblk, max(P, 1)), dtype=torch.int32, device=dev)
+    gch = inp["grandchildren"].to(dev) if depth3 else None
 
     exchange = n_global is not None and world > 1
 
+    def quantize():
+        if depth3:
+            avq.avq_quantize3(K, V, par, ch, gch, assign, vsum, counts, stream=stream)
+        else:
+            avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
+
+    def attend():
+        if depth3:
+            avq.avq_attention3(Q, par, ch, gch, vsum, counts, P, cfg.get("P2", P), block, inp["scale"], O=O,
+                               stream=stream)
+        else:
+            avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
+                              ws=ws, stream=stream)
+
     def step():
-        avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
+        quantize()
         k1 = avq.last_kernels()
         if exchange:
             allreduce_stats(vsum, counts)
-        avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
-                          ws=ws, stream=stream)
+        attend()
         return k1, avq.last_kernels()
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -319,12 +354,11 @@ def run_avq(args, cfg, inp, n_global=None):
             if fbuf is not None:  # inputs fit in L2: evict them before every timed step
                 fbuf.zero_()
             ev[s][0].record(stream)
-            avq.avq_quantize(K, V, par, ch, assign, vsum, counts, ws=ws, stream=stream)
+            quantize()
             if exchange:
                 allreduce_stats(vsum, counts)
             ev[s][1].record(stream)
-            avq.avq_attention(Q, par, ch, vsum, counts, P, block, inp["scale"], two_pass, O, sel,
-                              ws=ws, stream=stream)
+            attend()
             ev[s][2].record(stream)
         t1.record(stream)
         torch.cuda.synchronize(dev)
@@ -382,7 +416,7 @@ def run_avq(args, cfg, inp, n_global=None):
         return
 
     peaks = load_peaks()
-    alg = algorithmic(cfg)
+    alg = algorithmic3(cfg) if depth3 else algorithmic(cfg)
     s1_gbs = alg["s1_bytes"] / (t_s1 * 1e-3) / 1e9
     s2_gbs = alg["s2_bytes"] / (t_s2 * 1e-3) / 1e9
     s2_tfs = alg["s2_flops"] / (t_s2 * 1e-3) / 1e12
@@ -397,7 +431,7 @@ def run_avq(args, cfg, inp, n_global=None):
                     kernel="attention_tc", peak_source=peaks["source"],
                     step_roofline_us=t_roof * 1e6, step_frac=t_roof * 1e3 / ms_step)
     cpu = None
-    if not args.no_cpu_baseline and not args.profile and world == 1:  # rank 0 at N=1 only
+    if not args.no_cpu_baseline and not args.profile and world == 1 and not depth3:  # rank 0 at N=1 only
         heads = min(cfg["H"], max(1, os.cpu_count() or 1))
         q, times, cores = cpu_oracle_sample(inp, heads, steps=1)
         cpu = dict(value=q / times[0], unit="queries/s", cores=cores, kind="oracle",
@@ -503,7 +537,7 @@ def main():
             inp[k] = inp[k][:, :, n0:n1].contiguous()
         run_avq(args, dict(cfg, N=n1 - n0), inp, n_global=cfg["N"])
         return
-    inp = synth.make_inputs(cfg, seed)
+    inp = synth.make_inputs3(cfg, seed) if cfg.get("depth", 2) == 3 else synth.make_inputs(cfg, seed)
     run_avq(args, cfg, inp)
 
 

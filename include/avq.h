@@ -194,6 +194,56 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q,
                          void* ws, size_t ws_bytes, avq_stream_t stream);
 
 /*
+ * avq_quantize3 -- a depth-3 tree: Algorithm 1 (Sec. 4.2) one level further
+ * down, the "deeper hierarchies" named as the next step in the conclusion
+ * (Sec. 6).  Every child has C grandchildren and should be their mean, as
+ * every parent the mean of its children (Eq. 5).
+ *
+ * Every key goes to its nearest parent a (ties to the lower index), then to
+ * the nearest child c* of a (first strict minimum) if strictly closer than a,
+ * then to the nearest grandchild g* of c* if strictly closer than c*.
+ * Codes per head (Mt3 = M0 + M0*C + M0*C*C):
+ *   parents [0, M0); child (m, c) at M0 + m*C + c; grandchild (m, c, g) at
+ *   M0 + M0*C + (m*C + c)*C + g.
+ * Outputs (device, written in full; the call zeroes them first):
+ *   assign [B,H,N]      int32  final code
+ *   vsum   [B,H,Mt3,d]  fp32   value sums (Eq. 3): every node holds the keys of
+ *                              its subtree that reached it
+ *   counts [B,H,Mt3]    int32  key counts with the same membership
+ * Inputs (device): K, V [B,H,N,d]; parents [H,M0,d]; children [H,M0,C,d];
+ * grandchildren [H,M0,C,C,d], all of `dtype`; 1 <= C <= 8.  CUDA-core kernels
+ * (AVQ_ERR_UNSUPPORTED under AVQ_PATH_TC); no workspace.
+ */
+avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, const void* V,
+                         const void* parents, const void* children, const void* grandchildren,
+                         int32_t* assign, float* vsum, int32_t* counts, avq_stream_t stream);
+
+/*
+ * avq_attention3 -- Algorithm 2 (Sec. 4.3) over a depth-3 tree.
+ *
+ * Per query block: the parents' pass and the child refinement of the top-P
+ * parents as in avq_attention; then each of the P*C refined children gets
+ * an importance in the sense of Eq. 7 with the logits, maximum and
+ * denominator of the attention after that refinement,
+ *   w_c(I) = sum_{i in I} exp(s_ic - m_i) n_c / z_i,
+ * the top-P2 of them (descending, ties to the lower child code) are refined
+ * with their grandchildren: the child's logit is the mean of its
+ * grandchildren's (Eq. 8), dA = exp(s_ig) - exp(s_ic) (Eq. 9), zero for
+ * empty grandchildren, merged with the online maximum.  Y = x / z.
+ * Outputs (device): O [B,H,N,d] (dtype); sel [B,H,nblk,P] parents in
+ * descending importance; sel2 [B,H,nblk,P2] child codes (M0 + m*C + c) in
+ * descending child importance; importance [B,H,nblk,M0] (nullable);
+ * importance2 [B,H,nblk,P*C] (nullable), the refined children in the order of
+ * sel, C each.  0 <= P <= M0, 0 <= P2 <= P*C, block 64 or 128; vsum and
+ * counts as avq_quantize3 writes them.  CUDA-core kernel; no workspace.
+ */
+avq_status avq_attention3(const avq_dims* dims, avq_dtype dtype, const void* Q, const void* parents,
+                          const void* children, const void* grandchildren, const float* vsum,
+                          const int32_t* counts, int P, int P2, int block, float scale, void* O,
+                          int32_t* sel, int32_t* sel2, float* importance, float* importance2,
+                          avq_stream_t stream);
+
+/*
  * avq_codebook_update -- codebook update for training (Sec. A "Codeword
  * Clustering During Training", Eqs. 11-12).
  *

@@ -137,3 +137,52 @@ def check_output(gpu_O, ref_O, V, dtype, rows=None):
     assert np.isfinite(g).all(), "non-finite output"
     assert err <= O_TOL[dtype] * vmax, f"O error {err} > {O_TOL[dtype]} * {vmax}"
     return err / vmax
+
+
+def acceptable_code3(k, parents_h, children_h, gc_h, g, M0, C, band=ASSIGN_BAND):
+    """Is depth-3 code g acceptable for key k within the near-tie band, at each
+    of the descent's decisions (parent choice, child vs parent, grandchild vs
+    child)?  children_h [M0,C,d], gc_h [M0*C,C,d]."""
+    M1 = M0 * C
+    if g < M0:
+        pg, cg, gg = g, -1, -1
+    elif g < M0 + M1:
+        pg, cg, gg = (g - M0) // C, g - M0, -1
+    else:
+        cg = (g - M0 - M1) // C
+        pg, gg = cg // C, (g - M0 - M1) % C
+    dp = ((parents_h - k[None]) ** 2).sum(-1)
+    if dp[pg] > dp.min() + band * (k @ k + parents_h[pg] @ parents_h[pg]):
+        return False
+    dc = ((children_h[pg] - k[None]) ** 2).sum(-1)
+    if cg < 0:
+        cb = int(dc.argmin())
+        return dc.min() >= dp[pg] - band * (k @ k + children_h[pg][cb] @ children_h[pg][cb])
+    c = cg - pg * C
+    tol_c = band * (k @ k + children_h[pg][c] @ children_h[pg][c])
+    if not (dc[c] <= dc.min() + tol_c and dc[c] <= dp[pg] + tol_c):
+        return False
+    dg = ((gc_h[cg] - k[None]) ** 2).sum(-1)
+    if gg < 0:
+        gb = int(dg.argmin())
+        return dg.min() >= dc[c] - band * (k @ k + gc_h[cg][gb] @ gc_h[cg][gb])
+    tol_g = band * (k @ k + gc_h[cg][gg] @ gc_h[cg][gg])
+    return dg[gg] <= dg.min() + tol_g and dg[gg] <= dc[c] + tol_g
+
+
+def check_assign3(gpu_assign, oracle_assign, K, parents, children, grandchildren):
+    """Depth-3 codes: bit-exact outside the near-tie band."""
+    gpu_assign = np.asarray(gpu_assign)
+    bad = np.argwhere(gpu_assign != np.asarray(oracle_assign))
+    if len(bad) == 0:
+        return 0
+    K, par, ch, gc = _f64(K), _f64(parents), _f64(children), _f64(grandchildren)
+    M0, C = par.shape[1], ch.shape[2]
+    Mt = M0 + M0 * C + M0 * C * C
+    assert ((gpu_assign >= 0) & (gpu_assign < Mt)).all(), "code out of range"
+    for b, h, j in bad:
+        g = int(gpu_assign[b, h, j])
+        ok = acceptable_code3(K[b, h, j], par[h], ch[h], gc[h].reshape(M0 * C, C, -1), g, M0, C)
+        assert ok, f"key {(int(b), int(h), int(j))}: GPU code {g}, oracle {int(oracle_assign[b, h, j])}"
+    assert len(bad) <= max(8, gpu_assign.size // 1000), f"{len(bad)} near-tie disagreements"
+    return len(bad)

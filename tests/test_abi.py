@@ -178,6 +178,11 @@ def test_fault_injection_before_launch(monkeypatch):
         "codebook_update": lambda: L.avq_codebook_update(ctypes.byref(d), avq.AVQ_BF16, ctypes.c_float(0.9),
                                                          fake, fake, fake, fake, fake, fake, None),
         "permute": lambda: L.avq_permute(fake, fake, ctypes.c_void_p(0x20000000), 1, 64, 128, 0, None),
+        "quantize3": lambda: L.avq_quantize3(ctypes.byref(d), avq.AVQ_BF16, fake, fake, fake, fake, fake,
+                                             fake, fake, fake, None),
+        "attention3": lambda: L.avq_attention3(ctypes.byref(d), avq.AVQ_BF16, fake, fake, fake, fake, fake,
+                                               fake, 4, 8, 128, ctypes.c_float(0.125), fake, fake, fake,
+                                               None, None, None),
     }
     for entry, call in calls.items():
         monkeypatch.setenv("AVQ_FAULT", entry)
@@ -189,3 +194,30 @@ def test_fault_injection_before_launch(monkeypatch):
     # argument checks still come first
     monkeypatch.setenv("AVQ_FAULT", "all")
     assert L.avq_permute(None, fake, fake, 1, 64, 128, 0, None) == avq.AVQ_ERR_INVALID_ARG
+
+
+def test_depth3_host_checks():
+    """The depth-3 entry points reject bad arguments before any launch."""
+    L = avq.lib()
+    fake = ctypes.c_void_p(0x10000)
+    d = avq.avq_dims(1, 2, 256, 64, 16, 8)
+    d0 = avq.avq_dims(1, 2, 256, 64, 16, 0)
+    q3 = lambda dims, gc=fake: L.avq_quantize3(ctypes.byref(dims), avq.AVQ_BF16, fake, fake, fake, fake, gc,  # noqa: E731
+                                                fake, fake, fake, None)
+    assert q3(d0) == avq.AVQ_ERR_INVALID_ARG and "C >= 1" in avq.last_error()
+    assert q3(d, None) == avq.AVQ_ERR_INVALID_ARG and "grandchildren" in avq.last_error()
+    assert q3(d, ctypes.c_void_p(0x10004)) == avq.AVQ_ERR_INVALID_ARG
+
+    def a3(P, P2, block=128, sel2=fake):
+        return L.avq_attention3(ctypes.byref(d), avq.AVQ_BF16, fake, fake, fake, fake, fake, fake, P, P2,
+                                block, ctypes.c_float(0.125), fake, fake, sel2, None, None, None)
+    assert a3(17, 0) == avq.AVQ_ERR_INVALID_ARG            # P > M0
+    assert a3(4, 33) == avq.AVQ_ERR_INVALID_ARG            # P2 > P*C
+    assert a3(4, -1) == avq.AVQ_ERR_INVALID_ARG
+    assert a3(4, 4, block=96) == avq.AVQ_ERR_UNSUPPORTED
+    assert a3(4, 4, sel2=None) == avq.AVQ_ERR_INVALID_ARG and "sel2" in avq.last_error()
+    old = avq.avq_set_path(avq.AVQ_PATH_TC)
+    try:
+        assert a3(4, 4) == avq.AVQ_ERR_UNSUPPORTED and q3(d) == avq.AVQ_ERR_UNSUPPORTED
+    finally:
+        avq.avq_set_path(old)

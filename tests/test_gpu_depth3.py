@@ -1,0 +1,152 @@
+"""The depth-3 tree on the GPU against the float64 oracle, through the C ABI
+(needs a B200).  Same rules as the two-level parity tests: codes bit-exact
+outside the near-tie band (at each of the three decisions), counts
+bit-exact, value sums within the summed-magnitude bound, both selections
+exact outside the importance tie band (the second one judged on the oracle
+rerun with the GPU's parent selection), O within the dtype's tolerance of the
+oracle rerun on the GPU's two selections."""
+import numpy as np
+import pytest
+import torch
+
+import adaptive_vector_quantized_b200 as avq
+import oracle
+from adaptive_vector_quantized_b200 import synth
+from oracle import brute
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(**kw):
+    base = dict(dtype="bf16", B=1, H=2, N=1000, d=64, M0=16, C=8, P=4, P2=6, block=128,
+                key_sigma=0.03, sigma_c=0.3, sigma_g=0.1)
+    base.update(kw)
+    return base
+
+
+CASES = {
+    "bf16_ragged": (_cfg(), 61),
+    "f32_d128_b64": (_cfg(dtype="f32", N=700, d=128, M0=8, C=4, P=3, P2=5, block=64), 62),
+    "bf16_noise": (_cfg(N=1536, noise=0.1, P=5, P2=3), 63),
+    "p2_zero": (_cfg(N=512, P2=0), 64),
+    "p_zero": (_cfg(N=512, P=0, P2=0), 65),
+    "c1": (_cfg(N=300, C=1, P=4, P2=2), 66),
+    "all_children": (_cfg(N=400, M0=4, C=3, P=4, P2=12), 67),
+}
+
+
+def run_gpu3(inp, P=None, P2=None):
+    P = inp["P"] if P is None else P
+    P2 = inp["P2"] if P2 is None else P2
+    d = {k: inp[k].cuda().contiguous() for k in ("Q", "K", "V", "parents", "children", "grandchildren")}
+    assign, vsum, counts = avq.avq_quantize3(d["K"], d["V"], d["parents"], d["children"], d["grandchildren"])
+    k1 = avq.last_kernels()
+    O, sel, sel2, imp, imp2 = avq.avq_attention3(d["Q"], d["parents"], d["children"], d["grandchildren"],
+                                                 vsum, counts, P, P2, inp["block"], inp["scale"],
+                                                 importance=True)
+    k2 = avq.last_kernels()
+    avq.avq_check_device()
+    torch.cuda.synchronize()
+    return dict(assign=assign.cpu().numpy(), vsum=vsum.cpu().numpy(), counts=counts.cpu().numpy(),
+                O=O.cpu(), sel=sel.cpu().numpy(), sel2=sel2.cpu().numpy(), imp=imp.cpu().numpy(),
+                imp2=imp2.cpu().numpy(), kernels=k1 + " " + k2)
+
+
+def check3(inp, res, P=None, P2=None):
+    orc = oracle.default()
+    P = inp["P"] if P is None else P
+    P2 = inp["P2"] if P2 is None else P2
+    M0, C = inp["M0"], inp["C"]
+    args = (inp["parents"], inp["children"], inp["grandchildren"])
+    o_assign, _, _, _ = orc.quantize3(inp["K"], inp["V"], *args)
+    ties = parity.check_assign3(res["assign"], o_assign, inp["K"], *args)
+    ref_vs, ref_n = brute.aggregate_brute3(res["assign"], inp["V"], M0, C)
+    abs_vs, _ = brute.aggregate_brute3(res["assign"], inp["V"].abs(), M0, C)
+    parity.check_stats(res["vsum"], res["counts"], ref_vs, ref_n, abs_vs)
+    # parents' importance and selection on the GPU's statistics
+    _, _, _, o_imp, _ = orc.attention3(inp["Q"], *args, ref_vs, ref_n, P, P2, inp["block"], inp["scale"])
+    rel = np.abs(res["imp"] - o_imp) / (np.abs(o_imp) + 1e-6)
+    assert rel.max() <= 1e-4, rel.max()
+    parity.check_sel(res["sel"], o_imp, P)
+    # children's importance and the second selection on the GPU's parent selection
+    _, _, _, _, o_imp2 = orc.attention3(inp["Q"], *args, ref_vs, ref_n, P, P2, inp["block"], inp["scale"],
+                                        sel=res["sel"])
+    if P * C > 0:
+        g2 = res["imp2"][..., :P * C]
+        rel2 = np.abs(g2 - o_imp2) / (np.abs(o_imp2) + 1e-6)
+        assert rel2.max() <= 1e-4, rel2.max()
+    if P2 > 0:
+        # child codes -> candidate slots (the order of sel, C each)
+        cand = M0 + res["sel"][..., :, None] * C + np.arange(C)
+        cand = cand.reshape(*res["sel"].shape[:-1], P * C)
+        slots = np.empty_like(res["sel2"])
+        for idx in np.ndindex(*res["sel2"].shape[:-1]):
+            lut = {int(c): u for u, c in enumerate(cand[idx])}
+            slots[idx] = [lut[int(c)] for c in res["sel2"][idx]]
+        parity.check_sel(slots, o_imp2, P2)
+    O_ref, _, _, _, _ = orc.attention3(inp["Q"], *args, ref_vs, ref_n, P, P2, inp["block"], inp["scale"],
+                                       sel=res["sel"] if P > 0 else None,
+                                       sel2=res["sel2"] if P2 > 0 else None)
+    err = parity.check_output(res["O"], O_ref, inp["V"], inp["dtype"])
+    return dict(near_tie_keys=ties, O_rel_err=err)
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_depth3_parity(case):
+    cfg, seed = CASES[case]
+    inp = synth.make_inputs3(cfg, seed)
+    res = run_gpu3(inp)
+    assert "assign3_simt" in res["kernels"] and "attention3_simt" in res["kernels"]
+    M0, C = inp["M0"], inp["C"]
+    a = res["assign"]
+    if case != "c1":
+        assert (a >= M0 + M0 * C).any() and (a < M0).any()  # every level is reached
+    print(case, res["kernels"], check3(inp, res))
+
+
+def test_depth3_workload_sampled_invariants():
+    """The bench's depth-3 workload (B=1, H=8, N=16384, 64/16/16, C=8): full
+    parity on two heads, invariants on all."""
+    cfg = synth.get_config("deep3")
+    inp = synth.make_inputs3(cfg, synth.CONFIG_SEEDS["deep3"])
+    res = run_gpu3(inp)
+    N, M0, C = inp["N"], inp["M0"], inp["C"]
+    M1 = M0 * C
+    n = res["counts"]
+    assert (n[..., :M0].sum(-1) == N).all()
+    assert (n[..., M0:M0 + M1].sum(-1) == (res["assign"] >= M0).sum(-1)).all()
+    assert (n[..., M0 + M1:].sum(-1) == (res["assign"] >= M0 + M1).sum(-1)).all()
+    sizes = np.minimum(inp["block"], N - np.arange(res["imp"].shape[2]) * inp["block"])
+    assert np.allclose(res["imp"].sum(-1), sizes[None, None, :], rtol=1e-4)
+    sub = dict(inp)
+    for k in ("Q", "K", "V"):
+        sub[k] = inp[k][:, :2].contiguous()
+    sub["parents"], sub["children"], sub["grandchildren"] = (inp[k][:2] for k in ("parents", "children",
+                                                                                   "grandchildren"))
+    sub["H"] = 2
+    res2 = {k: (v[:, :2] if isinstance(v, np.ndarray) else v) for k, v in res.items()}
+    res2["O"] = res["O"][:, :2]
+    print("deep3", res["kernels"], check3(sub, res2))
+
+
+def test_depth3_equals_depth2_when_p2_is_zero():
+    """With P2 = 0 the depth-3 output equals the two-level output on the same
+    parents, children and (parent and child) statistics, on the GPU."""
+    cfg, seed = CASES["bf16_ragged"]
+    inp = synth.make_inputs3(cfg, seed)
+    res = run_gpu3(inp, P2=0)
+    M0, C = inp["M0"], inp["C"]
+    k2 = M0 + M0 * C
+    vs = torch.from_numpy(np.ascontiguousarray(res["vsum"][:, :, :k2])).cuda()
+    ns = torch.from_numpy(np.ascontiguousarray(res["counts"][:, :, :k2])).cuda()
+    old = avq.avq_set_path(avq.AVQ_PATH_SIMT)
+    try:
+        O2, sel2d, _ = avq.avq_attention(inp["Q"].cuda(), inp["parents"].cuda(), inp["children"].cuda(), vs, ns,
+                                         inp["P"], inp["block"], inp["scale"])
+    finally:
+        avq.avq_set_path(old)
+    torch.cuda.synchronize()
+    assert np.array_equal(sel2d.cpu().numpy(), res["sel"])
+    diff = (O2.cpu().float() - res["O"].float()).abs().max().item()
+    assert diff <= 2e-2 * float(inp["V"].float().abs().max())
