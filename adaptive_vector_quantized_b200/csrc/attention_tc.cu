@@ -754,14 +754,20 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     // (and zero value sums), so that the MMAs' N and K are multiples of 16.
     auto chunk_np = [&](int q) { return min(kChunkParents, P - q * kChunkParents); };
     auto chunk_slots = [&](int q) { return (chunk_np(q) + 1) & ~1; };
+    // thread t copies the 16-byte pieces t, t + 128, ... : always the same
+    // piece offset of every (128 / kPieces)-th atom
+    constexpr int kPieces = AB / 16;               // 64 (d = 64) or 128 (d = 128)
+    constexpr int kAtomStep = 128 / kPieces;       // atoms advanced per round of 128 pieces
+    const int my_off = (tid % kPieces) * 16, my_sl0 = tid / kPieces;
     auto copy_atoms = [&](uint8_t* dst, const bf16* src_h, int q, int slots) {
-      constexpr int kPieces = AB / 16;
       const int np = chunk_np(q);
-      for (int i = tid; i < slots * kPieces; i += 128) {
-        const int sl = i / kPieces, off = i % kPieces;
-        const int p = sSEL[q * kChunkParents + min(sl, np - 1)];
-        tc::cp_async16(dst + sl * AB + off * 16,
-                       reinterpret_cast<const uint8_t*>(src_h + (size_t)(M0 / 8 + p) * KH * 512) + off * 16);
+      const int* selq = sSEL + q * kChunkParents;
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(src_h) + (size_t)(M0 / 8) * AB + my_off;
+      uint8_t* d0 = dst + my_off;
+#pragma unroll
+      for (int r = 0; r < kChunkParents / kAtomStep; ++r) {
+        const int sl = my_sl0 + r * kAtomStep;
+        if (sl < slots) tc::cp_async16(d0 + sl * AB, src + (size_t)selq[min(sl, np - 1)] * AB);
       }
       tc::cp_async_commit();
     };
@@ -1153,6 +1159,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
     {
       const float iz = 1.f / z;
       const float2 iz2 = fm::f2(iz, iz);
+#pragma unroll
       for (int g = 0; g < D; g += 16) {
         uint32_t xr[16];
         tc::tmem_ld16(tX + lane_off + g, xr);
