@@ -428,9 +428,10 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
 // columns, B the bf16 triple (hi, mid, lo) whose sum is -|p|^2 / 2 to within
 // 2^-24 of it, so TMEM receives T directly.
 constexpr int kStageAtoms = 8;
-// Thread of each warpgroup that issues the parent MMAs (thread 0 issues the
-// child MMAs and the K copies), so that the two issue streams overlap.
-constexpr int kParentIssuer = 32;
+// Thread 0 of each warpgroup issues the K copies and every MMA: a tile's
+// child MMA goes in ahead of the next tile's parent MMA, and one issuer per
+// barrier keeps the drain on the way out exact (it waits for the phase of
+// the issuer's last operation).
 
 template <int D>
 struct WgSmem {
@@ -635,13 +636,12 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       if (*sAbort) break;
     }
     const int first = s0 + g;
-    // prologue: K of the first two tiles (thread 0), parent MMA of the first
-    // (the parent issuer)
+    // prologue (thread 0): K of the first two tiles, parent MMA of the first
     if (wt == 0 && first < s1) {
       issue_k(first, it);
       if (first + nwg < s1) issue_k(first + nwg, it + 1);
     }
-    if (wt == kParentIssuer && first < s1) {
+    if (wt == 0 && first < s1) {
       if (tc::mbar_wait(&bar_k[it & 1], (it >> 1) & 1)) {
         tc::tc_fence_after();
         issue_parents(it & 1, it);
@@ -654,7 +654,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       const uint32_t tP = tmem_g + (uint32_t)slot * 64u;  // parent, then child scores of this tile
       bool bad = false;
       if (wt == 0) bad = !tc::mbar_wait(bar_p, ph_p);
-      if (wt == kParentIssuer) bad = kerr;
+      if (wt == 0) bad = bad || kerr;
       ph_p ^= 1;
       tc::tc_fence_before();
       if (wg_bar_or(barid, bad)) {  // parent scores of tile t in TMEM
@@ -665,8 +665,8 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       tc::tc_fence_after();
       // next tile's parent MMA into the other half (its scores there were read
       // before the barrier above), so that it overlaps this tile's epilogue
-      auto next_parents = [&]() {
-        if (wt == kParentIssuer && t + nwg < s1) {
+      auto next_parents = [&](int issuer) {
+        if (wt == issuer && t + nwg < s1) {
           if (tc::mbar_wait(&bar_k[slot ^ 1], ((it + 1) >> 1) & 1)) {
             tc::tc_fence_after();
             issue_parents(slot ^ 1, it + 1);
@@ -676,7 +676,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
         }
       };
       if (C == 0) {
-        next_parents();
+        next_parents(0);
         if (wt == 0 && t + 2 * nwg < s1) issue_k(t + 2 * nwg, it + 2);  // K slot read by nothing else
       }
 
@@ -791,7 +791,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
             }
           }
         };
-        if (np == 0) next_parents();  // no child MMA for this tile
+        if (np == 0) next_parents(0);  // no child MMA for this tile
         for (int r0 = 0; r0 < np; r0 += kStageAtoms) {
           const int nr = min(kStageAtoms, np - r0);
           const int nat = (nr + 1) & ~1;
@@ -811,9 +811,9 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
           }
           tc::fence_proxy_async_smem();
           wg_bar(barid);  // staging written
-          // the next tile's parent MMA, issued by another thread while thread 0
-          // issues this round's child MMA
-          if (r0 == 0) next_parents();
+          // this round's child MMA, then (first round) the next tile's parent
+          // MMA behind it, both from thread 0, so that the child scores the
+          // tile waits for are not queued behind the next tile's parents
           if (wt == 0) {
             tc::tc_fence_after();
             const uint32_t idescC = tc::idesc_bf16(kKeys, 8 * nat, 0, 0);
@@ -826,6 +826,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
             }
             note(3, ph_c);
             tc::mma_commit(bar_c);
+            if (r0 == 0) next_parents(0);
             if (!tc::mbar_wait(bar_c, ph_c)) atomicOr(a.err, kErrTimeout);
           }
           if (r0 == 0) simt_children();
@@ -874,7 +875,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       }
       const int row = (t - bh * a.nblk) * kKeys + wt;
       if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
-      count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
+      count_codes_par(a.counts + (size_t)bh * Mt, par, code, row < a.N, M0);
     }
     if (aborted) *sAbort = 1;
     tc::tc_fence_before();

@@ -99,6 +99,18 @@ __device__ __forceinline__ void count_codes(int32_t* counts, int code, bool vali
   if (moved && lane == __ffs(peers_c) - 1) atomicAdd(counts + code, __popc(peers_c));
 }
 
+// The same for a caller that already knows the key's parent `par`.
+__device__ __forceinline__ void count_codes_par(int32_t* counts, int par, int code, bool valid, int M0) {
+  const int lane = threadIdx.x & 31;
+  const int pkey = valid ? par : -1 - lane;
+  const unsigned peers_p = __match_any_sync(0xffffffffu, pkey);
+  if (valid && lane == __ffs(peers_p) - 1) atomicAdd(counts + par, __popc(peers_p));
+  const bool moved = valid && code >= M0;
+  const int ckey = moved ? code : -1 - lane;
+  const unsigned peers_c = __match_any_sync(0xffffffffu, ckey);
+  if (moved && lane == __ffs(peers_c) - 1) atomicAdd(counts + code, __popc(peers_c));
+}
+
 // Vector reduction into global memory (sm_90+): four fp32 adds in one op.
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
