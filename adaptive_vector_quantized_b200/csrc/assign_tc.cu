@@ -4,10 +4,12 @@
 // Persistent CTAs walk contiguous ranges of 128-key tiles.  Per tile:
 //   K tile      TMA (128B swizzle) into a two-slot ring, the next tile in
 //               flight while the current one is processed
-//   parents     D = K P^T on tcgen05 into TMEM (M = 128 keys, N = M0);
-//               thread r owns key r = TMEM lane r and takes the first
-//               minimum of |p|^2 - 2 k.p over the parents (|k|^2 is the same
-//               for every codeword of a key and is dropped)
+//   parents     T = K P^T - |p|^2 / 2 on tcgen05 into TMEM (M = 128 keys,
+//               N = M0; the norm term is one more K step, ones times the
+//               bf16 triple hi + mid + lo of -|p|^2 / 2); thread r owns key
+//               r = TMEM lane r and takes the first maximum of T over the
+//               parents, i.e. the first minimum of |p|^2 - 2 k.p (|k|^2 is
+//               the same for every codeword of a key and is dropped)
 //   children    the C = 8 children of every parent are in shared memory as
 //               one swizzled atom each, so the children of two adjacent
 //               parents form an N = 16 operand tile: one MMA per parent pair
@@ -15,12 +17,14 @@
 //               its dot products with those 16 children (TMEM, in rounds of
 //               16 pairs); each thread then loads the 8 columns of its own
 //               parent (one TMEM load per distinct pair in its warp).  When
-//               the children do not fit in shared memory they are read from
-//               L2, one key at a time per warp (8 children x 4 parts of the
-//               dims over the lanes, coalesced, the next key's rows in
-//               flight), as bf16 x bf16 -> fp32 fused multiply-adds on the
-//               CUDA cores.  Either way the key moves to the first strictly
-//               smallest child only if it is strictly closer than the parent
+//               the children do not fit in shared memory, this kernel writes
+//               the parents only and a second launch (assign_children_kernel)
+//               refines every key on the CUDA cores: 8 lanes per key, each
+//               lane a slice of the dims of the key, its parent and the 8
+//               children (coalesced 16-byte loads from L2), the partial dot
+//               products summed over the 8 lanes.  Either way the key moves
+//               to the first strictly smallest child only if it is strictly
+//               closer than the parent
 //   output      assign[key] = parent, or M0 + parent*C + child
 // Codewords are first converted into the swizzled-atom image shared with
 // the attention kernel (8 codes x 64 dims per 1024-byte atom) plus their
@@ -46,6 +50,8 @@ struct AssignArgs {
   int32_t* counts;     // [BH][Mt], accumulated (zeroed by the caller)
   unsigned int* err;
   int H, N, M0, C, nblk, ntiles, tiles_per_cta;
+  int parents_only;  // general kernel with C > 0 and the children not in shared memory:
+                     // parents only, no counts (assign_children_kernel follows)
 };
 
 // bf16 pair x bf16 pair accumulated into fp32 (two exact products, two roundings).
@@ -61,14 +67,22 @@ __device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
   return d;
 }
 
+// bf16 bits of x, round to nearest even.
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
 template <int D, bool CH_SMEM>
 struct AssignSmem {
   static constexpr int KH = D / 64;
-  // parents image | children image (optional) | K ring [2] | norms | pair bits | barriers
+  // parents image | children image (optional) | K ring [2] | A and B of the
+  // norm step | norms | pair bits | barriers
   __host__ __device__ static size_t parents_bytes(int M0) { return (size_t)M0 * D * 2; }
   __host__ __device__ static size_t children_bytes(int M0, int C) { return CH_SMEM ? (size_t)M0 * C * D * 2 : 0; }
   __host__ __device__ static size_t ring_off(int M0, int C) { return parents_bytes(M0) + children_bytes(M0, C); }
-  __host__ __device__ static size_t norms_off(int M0, int C) { return ring_off(M0, C) + 2 * kKeys * D * 2; }
+  __host__ __device__ static size_t ones_off(int M0, int C) { return ring_off(M0, C) + 2 * kKeys * D * 2; }
+  __host__ __device__ static size_t bnorm_off(int M0, int C) { return ones_off(M0, C) + kKeys * 128; }
+  __host__ __device__ static size_t norms_off(int M0, int C) { return bnorm_off(M0, C) + (size_t)M0 * 128; }
   __host__ __device__ static size_t pairs_off(int M0, int C) {
     return (norms_off(M0, C) + (size_t)M0 * (1 + C) * 4 + 15) & ~(size_t)15;
   }
@@ -87,6 +101,8 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
   uint8_t* sPar = sm;
   uint8_t* sCh = sm + S::parents_bytes(M0);
   uint8_t* sRing = sm + S::ring_off(M0, C);
+  uint8_t* sOnes = sm + S::ones_off(M0, C);
+  uint8_t* sBn = sm + S::bnorm_off(M0, C);
   float* sNorm = reinterpret_cast<float*>(sm + S::norms_off(M0, C));
   uint32_t* sPairs = reinterpret_cast<uint32_t*>(sm + S::pairs_off(M0, C));  // 128-bit set of parent pairs
   uint64_t* bar_k = reinterpret_cast<uint64_t*>(sm + S::bar_off(M0, C));  // [2]
@@ -111,6 +127,13 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     sPairs[0] = sPairs[1] = sPairs[2] = sPairs[3] = 0;
     tc::prefetch_tensormap(&kmap);
   }
+  // A of the norm step: row r = (1, 1, 1, 0, ...) in logical 16-byte chunk 0
+  for (int i = tid; i < kKeys * 8; i += 128) {
+    const int r = i >> 3, pos = i & 7;
+    reinterpret_cast<uint4*>(sOnes)[i] =
+        pos == (r & 7) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0, 0, 0, 0);
+  }
+  tc::fence_proxy_async_smem();
   if (warp == 0) {
     tc::tmem_alloc(sTmem, ncols);
     tc::tmem_relinquish();
@@ -168,6 +191,20 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         }
       }
       for (int j = tid; j < Mt; j += 128) sNorm[j] = __ldg(a.norms + (size_t)h * Mt + j);
+      for (int i = tid; i < M0 * 8; i += 128) {  // B of the norm step: -|p|^2 / 2 as a bf16 triple
+        const int m = i >> 3, pos = i & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (pos == (m & 7)) {
+          const float n = -0.5f * __ldg(a.norms + (size_t)h * Mt + m);
+          const uint32_t hi = bf16_bits(n);
+          const float r1 = n - __uint_as_float(hi << 16);
+          const uint32_t mid = bf16_bits(r1);
+          const uint32_t lo = bf16_bits(r1 - __uint_as_float(mid << 16));
+          v = make_uint4(hi | (mid << 16), lo, 0u, 0u);
+        }
+        reinterpret_cast<uint4*>(sBn)[i] = v;
+      }
+      tc::fence_proxy_async_smem();
       if (!tc::mbar_wait(bar_cb, ph_cb)) {
         atomicOr(a.err, kErrTimeout);
         *sAbort = 1;
@@ -192,6 +229,8 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         const uint64_t bd = tc::sdesc_sw128(sParA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
         tc::mma_bf16(tmem, ad, bd, idesc, k > 0);
       }
+      tc::mma_bf16(tmem, tc::sdesc_sw128(tc::smem_u32(sOnes), 16, 1024), tc::sdesc_sw128(tc::smem_u32(sBn), 16, 1024),
+                   idesc, 1);
       note(2, ph_mma);
       tc::mma_commit(bar_mma);
     }
@@ -199,9 +238,10 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     ph_mma ^= 1;
     tc::tc_fence_after();
 
-    // nearest parent: first minimum of |p|^2 - 2 k.p; four independent running
-    // minima over interleaved 16-column groups, merged in index order
-    float best = INF;
+    // nearest parent: first maximum of T = k.p - |p|^2 / 2 (the MMA's norm
+    // step added the second term); four independent running maxima over
+    // interleaved 16-column groups, merged in index order
+    float bestT = -INF;
     int par = 0;
     for (int g0 = 0; g0 < M0; g0 += 64) {
       uint32_t r[64];
@@ -213,7 +253,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
       int iq[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        bq[q] = INF;
+        bq[q] = -INF;
         iq[q] = 0;
       }
 #pragma unroll
@@ -222,20 +262,21 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         for (int q = 0; q < 4; ++q) {
           const int m = g0 + q * 16 + e;
           if (m < M0) {
-            const float dm = fmaf(-2.f, __uint_as_float(r[q * 16 + e]), sNorm[m]);
-            if (dm < bq[q]) {
-              bq[q] = dm;
+            const float v = __uint_as_float(r[q * 16 + e]);
+            if (v > bq[q]) {
+              bq[q] = v;
               iq[q] = m;
             }
           }
         }
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (bq[q] < best) {
-          best = bq[q];
+        if (bq[q] > bestT) {
+          bestT = bq[q];
           par = iq[q];
         }
     }
+    const float best = -2.f * bestT;  // the parent's |p|^2 - 2 k.p, for the child test
     int code = par;
     if constexpr (CH_SMEM) {
       if (C > 0) {  // C == 8 on this path
@@ -316,76 +357,10 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
         if (dchild < best) code = M0 + par * 8 + cstar;
         if (tid < 4) sPairs[tid] = 0;  // for the next tile (read by everyone above)
       }
-    } else if (C > 0) {  // C == 8; children from L2, dot products on the CUDA cores
-      // one key at a time, the warp's 32 lanes take its 8 children x 4 parts
-      // of the dims (so each child row is read by four neighbouring lanes,
-      // coalesced), the next key's child rows in flight meanwhile; the key's
-      // row comes from the K tile in shared memory (128-byte swizzle)
-      const int wl = tid & 31, cl = wl >> 2, ql = wl & 3;
-      const int warp_row0 = (tid >> 5) * 32;
-      auto child_row = [&](int pk) {
-        return reinterpret_cast<const uint8_t*>(a.cw + ((size_t)h * Mt + M0 + pk * 8) * D) + cl * 128;
-      };
-      uint4 cur[KH][2], nxt[KH][2];
-      auto load_rows = [&](const uint8_t* rowp, uint4 (&dst)[KH][2]) {
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh)
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2)
-            dst[kh][h2] = __ldg(reinterpret_cast<const uint4*>(rowp + kh * 1024 + (((2 * ql + h2) ^ cl) << 4)));
-      };
-      load_rows(child_row(__shfl_sync(0xffffffffu, par, 0)), cur);
-      float vals[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) vals[c] = 0.f;
-#pragma unroll 2
-      for (int k = 0; k < 32; ++k) {
-        const int pn = __shfl_sync(0xffffffffu, par, (k + 1) & 31);
-        if (k + 1 < 32) load_rows(child_row(pn), nxt);
-        const int krow = warp_row0 + k;
-        float dot = 0.f;
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh)
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const uint4 kv = *reinterpret_cast<const uint4*>(sK + kh * (kKeys * 128) + krow * 128 +
-                                                             (((2 * ql + h2) ^ (krow & 7)) << 4));
-            const uint4 cv = cur[kh][h2];
-            dot = fma_bf16x2(kv.x, cv.x, dot);
-            dot = fma_bf16x2(kv.y, cv.y, dot);
-            dot = fma_bf16x2(kv.z, cv.z, dot);
-            dot = fma_bf16x2(kv.w, cv.w, dot);
-          }
-        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-        dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const float v = __shfl_sync(0xffffffffu, dot, cc * 4);
-          if (wl == k) vals[cc] = v;
-        }
-        if (k + 1 < 32) {
-#pragma unroll
-          for (int kh = 0; kh < KH; ++kh) {
-            cur[kh][0] = nxt[kh][0];
-            cur[kh][1] = nxt[kh][1];
-          }
-        }
-      }
-      float dchild = INF;
-      int cstar = 0;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float dc = fmaf(-2.f, vals[c], sNorm[M0 + par * 8 + c]);
-        if (dc < dchild) {
-          dchild = dc;
-          cstar = c;
-        }
-      }
-      if (dchild < best) code = M0 + par * 8 + cstar;
     }
     const int row = blk * kKeys + tid;
     if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
-    count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
+    if (!a.parents_only) count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
 
     tc::tc_fence_before();
     __syncthreads();  // K slot and TMEM free
@@ -488,10 +463,6 @@ __device__ __forceinline__ int nth_set(uint32_t m, int n) {
   return pos;
 }
 
-// bf16 bits of x, round to nearest even.
-__device__ __forceinline__ uint32_t bf16_bits(float x) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
-}
 
 template <int D, int M0>
 __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -901,6 +872,86 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   }
 }
 
+// Child refinement for keys whose parent is already in `assign` (C = 8):
+// 8 lanes per key, 4 keys per warp.  Lane s of a key holds dims
+// [s D/8, (s+1) D/8) of the key, its parent and its 8 children (16-byte
+// loads; the 8 lanes of a key read each 128- or 256-byte row once,
+// coalesced), accumulates the 9 partial dot products in fp32 (bf16 x bf16
+// products) and sums them over the 8 lanes.  Distances |c|^2 - 2 k.c with the
+// fp32 squared norms; the key moves to the first strictly smallest child only
+// if it is strictly closer than its parent.  Counts: the parent for every
+// key, the child for keys that moved.
+template <int D>
+__global__ void __launch_bounds__(256) assign_children_kernel(const bf16* __restrict__ K,
+                                                              const bf16* __restrict__ parents,
+                                                              const bf16* __restrict__ children,
+                                                              const float* __restrict__ norms,
+                                                              int32_t* __restrict__ assign,
+                                                              int32_t* __restrict__ counts, int BH, int H,
+                                                              int N, int M0) {
+  constexpr int C = 8;
+  constexpr int DL = D / 8;      // dims per lane
+  constexpr int CHK = DL / 8;    // 16-byte chunks per lane and row
+  const int Mt = M0 * (1 + C);
+  const int lane = threadIdx.x & 31, sub = lane & 7, kq = lane >> 3;
+  const long long total = (long long)BH * N;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long k0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4; k0 < total;
+       k0 += warps * 4) {  // warp-uniform loop
+    const long long key = k0 + kq;
+    const bool live = key < total;
+    const long long bh = live ? key / N : 0;
+    const int h = (int)(bh % H);
+    const int p = live ? __ldg(assign + key) : 0;
+    const bf16* kr = K + (size_t)(live ? key : 0) * D + sub * DL;
+    const bf16* pr = parents + ((size_t)h * M0 + p) * D + sub * DL;
+    const bf16* cr = children + ((size_t)h * M0 + p) * C * D + sub * DL;
+    float acc[1 + C];
+#pragma unroll
+    for (int j = 0; j <= C; ++j) acc[j] = 0.f;
+#pragma unroll
+    for (int q = 0; q < CHK; ++q) {
+      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + q * 8));
+      uint4 cv[1 + C];
+      cv[0] = __ldg(reinterpret_cast<const uint4*>(pr + q * 8));
+#pragma unroll
+      for (int c = 0; c < C; ++c) cv[1 + c] = __ldg(reinterpret_cast<const uint4*>(cr + (size_t)c * D + q * 8));
+#pragma unroll
+      for (int j = 0; j <= C; ++j) {
+        acc[j] = fma_bf16x2(kv.x, cv[j].x, acc[j]);
+        acc[j] = fma_bf16x2(kv.y, cv[j].y, acc[j]);
+        acc[j] = fma_bf16x2(kv.z, cv[j].z, acc[j]);
+        acc[j] = fma_bf16x2(kv.w, cv[j].w, acc[j]);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+      for (int j = 0; j <= C; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+    if (live && sub == 0) {
+      const float* nh = norms + (size_t)h * Mt;
+      const float dp = fmaf(-2.f, acc[0], nh[p]);
+      float dc = fmaf(-2.f, acc[1], nh[M0 + p * C]);
+      int cstar = 0;
+#pragma unroll
+      for (int c = 1; c < C; ++c) {
+        const float d = fmaf(-2.f, acc[1 + c], nh[M0 + p * C + c]);
+        if (d < dc) {
+          dc = d;
+          cstar = c;
+        }
+      }
+      int32_t* cnt = counts + (size_t)bh * Mt;
+      atomicAdd(cnt + p, 1);
+      if (dc < dp) {
+        const int code = M0 + p * C + cstar;
+        assign[key] = code;
+        atomicAdd(cnt + code, 1);
+      }
+    }
+  }
+}
+
 // Codewords -> swizzled-atom image (code a in atom a/8, row a%8) and fp32
 // squared norms.  Children of parent p are codes M0 + p*C + c.
 template <int D>
@@ -1055,6 +1106,7 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
   a.nblk = (s.N + kKeys - 1) / kKeys;
   a.ntiles = a.nblk * s.BH();
   a.tiles_per_cta = 1;
+  a.parents_only = 0;
   const size_t ch_bytes = (size_t)s.M0 * s.C * s.d * 2;
   if (s.M0 <= 64) {  // warpgroup-pipelined kernel when the whole image fits
     const int nwg = s.d == 64 ? wg_count<64>(s) : wg_count<128>(s);
@@ -1065,11 +1117,30 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
     }
   }
   const bool ch_smem = ch_bytes <= 96 * 1024;
+  // children too large for shared memory: parents here, children refined by
+  // a second, CUDA-core launch with many warps per SM
+  const bool split = !ch_smem && s.C > 0;
+  a.parents_only = split ? 1 : 0;
   if (s.d == 64)
     e = ch_smem ? launch_impl<64, true>(s, kmap, a, st) : launch_impl<64, false>(s, kmap, a, st);
   else
     e = ch_smem ? launch_impl<128, true>(s, kmap, a, st) : launch_impl<128, false>(s, kmap, a, st);
-  log.add(ch_smem ? "assign_tc" : "assign_tc_l2children");
+  if (e != cudaSuccess) return e;
+  log.add(ch_smem || s.C == 0 ? "assign_tc" : "assign_tc_parents");
+  if (split) {
+    const long long groups = ((long long)s.BH() * s.N + 3) / 4;  // 4 keys per warp
+    const int blocks = (int)std::max<long long>(1, std::min<long long>((groups + 7) / 8, (long long)num_sms() * 16));
+    if (s.d == 64)
+      assign_children_kernel<64><<<blocks, 256, 0, st>>>((const bf16*)K, (const bf16*)parents,
+                                                         (const bf16*)children, norms, assign, counts, s.BH(),
+                                                         s.H, s.N, s.M0);
+    else
+      assign_children_kernel<128><<<blocks, 256, 0, st>>>((const bf16*)K, (const bf16*)parents,
+                                                          (const bf16*)children, norms, assign, counts, s.BH(),
+                                                          s.H, s.N, s.M0);
+    e = cudaGetLastError();
+    log.add("assign_children");
+  }
   return e;
 }
 
