@@ -50,8 +50,6 @@ struct AssignArgs {
   int32_t* counts;     // [BH][Mt], accumulated (zeroed by the caller)
   unsigned int* err;
   int H, N, M0, C, nblk, ntiles, tiles_per_cta;
-  int parents_only;  // general kernel with C > 0 and the children not in shared memory:
-                     // parents only, no counts (assign_children_kernel follows)
 };
 
 // bf16 pair x bf16 pair accumulated into fp32 (two exact products, two roundings).
@@ -360,7 +358,7 @@ __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ 
     }
     const int row = blk * kKeys + tid;
     if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
-    if (!a.parents_only) count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
+    count_codes(a.counts + (size_t)bh * Mt, code, row < a.N, M0, C);
 
     tc::tc_fence_before();
     __syncthreads();  // K slot and TMEM free
@@ -872,6 +870,235 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   }
 }
 
+// Parents only, for codebooks whose children do not fit in shared memory (or
+// C = 0): persistent CTAs over contiguous 128-key tiles; the parents' image of
+// the head and the norm step's operands stay in shared memory, K tiles come
+// through a two-slot TMA ring, and TMEM holds two score slots, so the next
+// tile's MMA runs while this tile's first maximum of T is taken.  With
+// children, assign_children_kernel then refines every key (and counts);
+// without, this kernel counts.
+template <int D>
+struct ParentsSmem {
+  // parents image | K ring [2] | A and B of the norm step | barriers | tmem, abort
+  __host__ __device__ static size_t ring_off(int M0) { return (size_t)M0 * D * 2; }
+  __host__ __device__ static size_t ones_off(int M0) { return ring_off(M0) + 2 * kKeys * D * 2; }
+  __host__ __device__ static size_t bnorm_off(int M0) { return ones_off(M0) + kKeys * 128; }
+  __host__ __device__ static size_t bar_off(int M0) { return bnorm_off(M0) + (size_t)M0 * 128; }
+  __host__ __device__ static size_t total(int M0) { return bar_off(M0) + 64; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                             const AssignArgs a) {
+  using S = ParentsSmem<D>;
+  constexpr int KH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int M0 = a.M0, C = a.C, Mt = M0 * (1 + C);
+  uint8_t* sPar = sm;
+  uint8_t* sRing = sm + S::ring_off(M0);
+  uint8_t* sOnes = sm + S::ones_off(M0);
+  uint8_t* sBn = sm + S::bnorm_off(M0);
+  uint64_t* bar_k = reinterpret_cast<uint64_t*>(sm + S::bar_off(M0));  // [2]
+  uint64_t* bar_cb = bar_k + 2;
+  uint64_t* bar_mma = bar_k + 3;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar_k + 4);
+  int* sAbort = reinterpret_cast<int*>(bar_k + 4) + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int t0 = blockIdx.x * a.tiles_per_cta;
+  const int t1 = min(a.ntiles, t0 + a.tiles_per_cta);
+  if (t0 >= t1) return;
+  const uint32_t slot_cols = M0 <= 32 ? 32u : M0 <= 64 ? 64u : M0 <= 128 ? 128u : 256u;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) tc::mbar_init(bar_k + i, 1);
+    tc::fence_mbar_init();
+    *sAbort = 0;
+    tc::prefetch_tensormap(&kmap);
+  }
+  // A of the norm step: row r = (1, 1, 1, 0, ...) in logical 16-byte chunk 0
+  for (int i = tid; i < kKeys * 8; i += 128) {
+    const int r = i >> 3, pos = i & 7;
+    reinterpret_cast<uint4*>(sOnes)[i] =
+        pos == (r & 7) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0, 0, 0, 0);
+  }
+  tc::fence_proxy_async_smem();
+  if (warp == 0) {
+    tc::tmem_alloc(sTmem, 2 * slot_cols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+  // per barrier, the parity of the phase that thread 0's last copy or MMA on
+  // it completes (bit b of `issued` once there was one): bits 0-1 the K ring
+  // slots, 2 the parents' image, 3 the MMAs (the order of the barriers
+  // bar_k[0..3]); drained on the way out
+  uint32_t issued = 0, exp_par = 0;
+  auto note = [&](int b, uint32_t ph) {
+    issued |= 1u << b;
+    exp_par = (exp_par & ~(1u << b)) | ((ph & 1u) << b);
+  };
+  auto issue_k = [&](int t) {  // tile t into ring slot (t - t0) & 1
+    const int it = t - t0, slot = it & 1, bh = t / a.nblk, blk = t % a.nblk;
+    note(slot, (uint32_t)(it >> 1));
+    tc::mbar_arrive_expect_tx(&bar_k[slot], kKeys * D * 2);
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh)
+      tc::tma_load_3d(sRing + slot * (kKeys * D * 2) + kh * (kKeys * 128), &kmap, kh * 64, blk * kKeys, bh,
+                      &bar_k[slot]);
+  };
+  uint32_t ph_cb = 0, ph_mma = 0;
+  // the head's parents' image and the norm step's B (CTA-wide)
+  auto load_head = [&](int h) {
+    if (tid == 0) {
+      const uint32_t bytes = (uint32_t)(M0 * D * 2);
+      note(2, ph_cb);
+      tc::mbar_arrive_expect_tx(bar_cb, bytes);
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cw + (size_t)h * Mt * D);
+      for (uint32_t off = 0; off < bytes; off += 65536)
+        tc::bulk_g2s(sPar + off, src + off, min(bytes - off, 65536u), bar_cb);
+    }
+    for (int i = tid; i < M0 * 8; i += 128) {  // -|p|^2 / 2 as a bf16 triple
+      const int m = i >> 3, pos = i & 7;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (pos == (m & 7)) {
+        const float n = -0.5f * __ldg(a.norms + (size_t)h * Mt + m);
+        const uint32_t hi = bf16_bits(n);
+        const float r1 = n - __uint_as_float(hi << 16);
+        const uint32_t mid = bf16_bits(r1);
+        const uint32_t lo = bf16_bits(r1 - __uint_as_float(mid << 16));
+        v = make_uint4(hi | (mid << 16), lo, 0u, 0u);
+      }
+      reinterpret_cast<uint4*>(sBn)[i] = v;
+    }
+    tc::fence_proxy_async_smem();
+    if (!tc::mbar_wait(bar_cb, ph_cb)) {
+      atomicOr(a.err, kErrTimeout);
+      *sAbort = 1;
+    }
+    ph_cb ^= 1;
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+  };
+  const uint32_t idesc = tc::idesc_bf16(kKeys, M0, 0, 0);
+  // thread 0: wait for tile t's K, then T = K P^T - |p|^2 / 2 into its TMEM slot
+  auto issue_mma = [&](int t) {
+    const int it = t - t0, slot = it & 1;
+    if (!tc::mbar_wait(&bar_k[slot], (uint32_t)(it >> 1) & 1u)) {
+      atomicOr(a.err, kErrTimeout);
+      *sAbort = 1;
+      return;
+    }
+    tc::tc_fence_after();
+    const uint32_t sKa = tc::smem_u32(sRing + slot * (kKeys * D * 2)), sParA = tc::smem_u32(sPar);
+    const uint32_t d = tmem + (uint32_t)slot * slot_cols;
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+      const uint64_t ad = tc::sdesc_sw128(sKa + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024);
+      const uint64_t bd = tc::sdesc_sw128(sParA + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+      tc::mma_bf16(d, ad, bd, idesc, k > 0);
+    }
+    tc::mma_bf16(d, tc::sdesc_sw128(tc::smem_u32(sOnes), 16, 1024), tc::sdesc_sw128(tc::smem_u32(sBn), 16, 1024),
+                 idesc, 1);
+    note(3, (uint32_t)it);  // the it-th commit completes phase it
+    tc::mma_commit(bar_mma);
+  };
+
+  int cur_h = (t0 / a.nblk) % a.H;
+  if (tid == 0) {
+    issue_k(t0);
+    if (t0 + 1 < t1) issue_k(t0 + 1);
+  }
+  load_head(cur_h);
+  if (tid == 0 && !*sAbort) issue_mma(t0);
+  __syncthreads();  // the abort flag is the same for every thread below
+  const float NEG_INF = __int_as_float(0xff800000);
+  for (int t = t0; t < t1; ++t) {
+    const int it = t - t0, slot = it & 1;
+    const int bh = t / a.nblk, blk = t % a.nblk;
+    if (*sAbort) break;  // uniform: read after the barrier that ended the previous tile
+    if (!tc::mbar_wait(bar_mma, ph_mma)) {
+      atomicOr(a.err, kErrTimeout);
+      *sAbort = 1;
+    }
+    ph_mma ^= 1;
+    tc::tc_fence_after();
+    if (tid == 0 && t + 2 < t1) issue_k(t + 2);  // this tile's K slot is read
+    if (t + 1 < t1) {  // the next tile's MMA into the other slot, behind a head change if any
+      const int hn = ((t + 1) / a.nblk) % a.H;
+      if (hn != cur_h) {
+        load_head(hn);
+        cur_h = hn;
+      }
+      if (tid == 0 && !*sAbort) issue_mma(t + 1);
+    }
+    // first maximum of T: four independent running maxima over interleaved
+    // 16-column groups, merged in index order
+    const uint32_t ts = tmem + (uint32_t)slot * slot_cols + lane_off;
+    float bestT = NEG_INF;
+    int par = 0;
+    for (int g0 = 0; g0 < M0; g0 += 64) {
+      uint32_t r[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (g0 + q * 16 < M0) tc::tmem_ld16(ts + g0 + q * 16, r + q * 16);
+      tc::tmem_wait_ld();
+      float bq[4];
+      int iq[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        bq[q] = NEG_INF;
+        iq[q] = 0;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int m = g0 + q * 16 + e;
+          if (m < M0) {
+            const float v = __uint_as_float(r[q * 16 + e]);
+            if (v > bq[q]) {
+              bq[q] = v;
+              iq[q] = m;
+            }
+          }
+        }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (bq[q] > bestT) {
+          bestT = bq[q];
+          par = iq[q];
+        }
+    }
+    const int row = blk * kKeys + tid;
+    if (row < a.N) a.assign[(size_t)bh * a.N + row] = par;
+    if (C == 0) count_codes(a.counts + (size_t)bh * Mt, par, row < a.N, M0, C);
+    tc::tc_fence_before();
+    __syncthreads();  // this TMEM slot is read: the MMA two tiles on may overwrite it
+  }
+
+  // nothing in flight before TMEM is freed (the waits return at once for
+  // completed operations; 1 ms limit)
+  if (issued) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if ((issued >> b) & 1u)
+        if (!tc::mbar_wait(bar_k + b, (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 2 * slot_cols);
+  }
+}
+
 // Child refinement for keys whose parent is already in `assign` (C = 8):
 // 8 lanes per key, 4 keys per warp.  Lane s of a key holds dims
 // [s D/8, (s+1) D/8) of the key, its parent and its 8 children (16-byte
@@ -1022,6 +1249,23 @@ cudaError_t launch_impl(const Shape& s, const CUtensorMap& kmap, AssignArgs a, c
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
+template <int D>
+cudaError_t launch_parents(const Shape& s, const CUtensorMap& kmap, AssignArgs a, cudaStream_t st) {
+  const size_t smem = ParentsSmem<D>::total(s.M0) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(assign_parents_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  // CTAs per SM: shared memory (228 KB per SM, 1 KB reserved per CTA) and
+  // TMEM (512 columns; two score slots per CTA)
+  const int slot = s.M0 <= 32 ? 32 : s.M0 <= 64 ? 64 : s.M0 <= 128 ? 128 : 256;
+  const int per_sm = std::max(1, std::min((int)((228 * 1024) / (smem + 1024)), 512 / (2 * slot)));
+  const int ctas = std::min(a.ntiles, num_sms() * per_sm);
+  a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
+  const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+  assign_parents_kernel<D><<<grid, 128, smem, st>>>(kmap, a);
+  return cudaGetLastError();
+}
+
 // Warpgroups per CTA for the pipelined kernel (0: the image does not fit).
 template <int D>
 int wg_count(const Shape& s) {
@@ -1106,7 +1350,6 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
   a.nblk = (s.N + kKeys - 1) / kKeys;
   a.ntiles = a.nblk * s.BH();
   a.tiles_per_cta = 1;
-  a.parents_only = 0;
   const size_t ch_bytes = (size_t)s.M0 * s.C * s.d * 2;
   if (s.M0 <= 64) {  // warpgroup-pipelined kernel when the whole image fits
     const int nwg = s.d == 64 ? wg_count<64>(s) : wg_count<128>(s);
@@ -1116,18 +1359,18 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
       return e;
     }
   }
-  const bool ch_smem = ch_bytes <= 96 * 1024;
-  // children too large for shared memory: parents here, children refined by
-  // a second, CUDA-core launch with many warps per SM
-  const bool split = !ch_smem && s.C > 0;
-  a.parents_only = split ? 1 : 0;
-  if (s.d == 64)
-    e = ch_smem ? launch_impl<64, true>(s, kmap, a, st) : launch_impl<64, false>(s, kmap, a, st);
-  else
-    e = ch_smem ? launch_impl<128, true>(s, kmap, a, st) : launch_impl<128, false>(s, kmap, a, st);
+  const bool ch_smem = s.C > 0 && ch_bytes <= 96 * 1024;
+  if (ch_smem) {
+    e = s.d == 64 ? launch_impl<64, true>(s, kmap, a, st) : launch_impl<128, true>(s, kmap, a, st);
+    log.add("assign_tc");
+    return e;
+  }
+  // children too large for shared memory (or none): parents on the tensor
+  // cores, then the children refined by a CUDA-core launch with many warps
+  e = s.d == 64 ? launch_parents<64>(s, kmap, a, st) : launch_parents<128>(s, kmap, a, st);
   if (e != cudaSuccess) return e;
-  log.add(ch_smem || s.C == 0 ? "assign_tc" : "assign_tc_parents");
-  if (split) {
+  log.add("assign_tc_parents");
+  if (s.C > 0) {
     const long long groups = ((long long)s.BH() * s.N + 3) / 4;  // 4 keys per warp
     const int blocks = (int)std::max<long long>(1, std::min<long long>((groups + 7) / 8, (long long)num_sms() * 16));
     if (s.d == 64)
