@@ -3,8 +3,10 @@
 //
 // Given every key's final code, each key adds its value to its parent, and to
 // its child when it moved to one.  Parents therefore hold their whole
-// cluster, children only the keys closer to them than to the parent.  (The
-// key counts n of Eq. 3 are produced by the assignment kernels.)
+// cluster, children only the keys closer to them than to the parent.  The
+// key counts n of Eq. 3 come either from the assignment kernels or, for the
+// warpgroup tensor-core assignment, from the same streaming pass (each run
+// adds its length to its code) followed by the same upward pass as the sums.
 //
 // Streaming variant: runs of equal codes are summed in registers and added to
 // the statistics with global vector reductions; see aggregate_stream_kernel.
@@ -33,9 +35,9 @@ namespace {
 // the current one is added) whose per-key work is a bit test and the adds,
 // into two partial sums per run.  A finished run is
 // added to the global value sums (L2 resident) with one vector reduction per
-// lane.  Then each parent adds its children's sums to its own, which makes
-// it the sum over its whole cluster (Eq. 3).  Counts are produced by the
-// assignment kernels.
+// lane (and, when `counts` is given, lane 0 adds the run's length to its
+// code's count).  Then each parent adds its children's sums (and counts) to
+// its own, which makes it the sum over its whole cluster (Eq. 3).
 constexpr int kStreamThreads = 256;
 
 // One lane's E consecutive elements of a value row, as loaded.
@@ -84,8 +86,8 @@ __device__ __forceinline__ void flush_sum(float* vsum, int code, const float* ac
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
-    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum, int BH, int N,
-    int Mt, int keys_per_warp) {
+    const T* __restrict__ V, const int32_t* __restrict__ assign, float* __restrict__ vsum,
+    int32_t* __restrict__ counts, int BH, int N, int Mt, int keys_per_warp) {
   constexpr int E = D / 32;
   using F = Frag<T, E>;
   constexpr int B = F::kBatch;  // keys loaded at once (32 / B batches per group)
@@ -99,14 +101,15 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
   float* vs = vsum + (size_t)bh * Mt * D;
   const T* vb = V + (size_t)bh * N * D + lane * E;
   const int32_t* asg = assign + (size_t)bh * N;
+  int32_t* cn = counts ? counts + (size_t)bh * Mt : nullptr;
 
   // two partial sums per run (even and odd keys of a group) halve the chain of
   // dependent adds; they are combined when the run is flushed
   float acc[2][E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[0][e] = acc[1][e] = 0.f;
-  int cur = -1;
-  auto flush = [&]() {
+  int cur = -1, run0 = j0;  // the open run's code and first key
+  auto flush = [&](int end) {  // the open run ends before key `end`
     float t[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -114,6 +117,7 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
       acc[0][e] = acc[1][e] = 0.f;
     }
     flush_sum<E>(vs, cur, t, lane, D);
+    if (cn && lane == 0) atomicAdd(cn + cur, end - run0);
   };
   int code_next = j0 + lane < j1 ? __ldg(asg + j0 + lane) : -1;
   for (int g = j0; g < j1; g += 32) {
@@ -148,8 +152,9 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
             float v[E];
             F::unpack(raw[b], v);
             if ((starts >> b) & 1u) {
-              if (cur >= 0) flush();
+              if (cur >= 0) flush(g + u);
               cur = __shfl_sync(0xffffffffu, code, u);
+              run0 = g + u;
             }
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[b & 1][e] += v[e];
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     else
       walk(std::false_type{});
   }
-  if (cur >= 0) flush();
+  if (cur >= 0) flush(j1);
 }
 
 // Nodes hold their whole subtree: add the sums of the n nodes' children
@@ -172,8 +177,9 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
 // in index order.  Node i of the level starting at code `lo` has its C
 // children at codes lo2 + i*C .. lo2 + i*C + C - 1 (for a two-level tree:
 // lo = 0, n = M0, lo2 = M0).
-__global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restrict__ vsum, int BH, int Mt, int lo,
-                                                               int n, int lo2, int C, int D) {
+__global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restrict__ vsum,
+                                                               int32_t* __restrict__ counts, int BH, int Mt,
+                                                               int lo, int n, int lo2, int C, int D) {
   const long long total = (long long)BH * n * D;
   for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
        u += (long long)gridDim.x * blockDim.x) {
@@ -184,6 +190,12 @@ __global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restric
     float s = vs[(size_t)(lo + p) * D + t];
     for (int c = 0; c < C; ++c) s += vs[(size_t)(lo2 + p * C + c) * D + t];
     vs[(size_t)(lo + p) * D + t] = s;
+    if (counts && t == 0) {
+      int32_t* ns = counts + (bp / n) * (long long)Mt;
+      int k = ns[lo + p];
+      for (int c = 0; c < C; ++c) k += ns[lo2 + p * C + c];
+      ns[lo + p] = k;
+    }
   }
 }
 
@@ -368,14 +380,14 @@ size_t aggregate_det_workspace(const Shape& s) {
 
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log, bool vsum_zeroed, bool depth3) {
+                             LaunchLog& log, bool vsum_zeroed, bool depth3, bool count) {
   cudaError_t e = cudaSuccess;
   const int Mt = depth3 ? s.M0 + s.M0 * s.C + s.M0 * s.C * s.C : s.Mt();
   if (!vsum_zeroed) {
     e = cudaMemsetAsync(vsum, 0, (size_t)s.BH() * Mt * s.d * sizeof(float), st);
     if (e != cudaSuccess) return e;
   }
-  (void)counts;
+  int32_t* cnt = count ? counts : nullptr;  // counts left to this pass (zeroed by the caller)
   const int sms = num_sms();
   // grid sized for about 32 resident warps per SM, each a contiguous multiple of 32 keys
   const long long total_keys = (long long)s.BH() * s.N;
@@ -386,7 +398,7 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
   const unsigned blocks = (unsigned)((warps + (kStreamThreads / 32) - 1) / (kStreamThreads / 32));
 #define AVQ_STREAM(T, D)                                                                            \
-  aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, s.BH(), \
+  aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, cnt, s.BH(), \
                                                                    s.N, Mt, kpw)
   if (dt == AVQ_F32) {
     if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
@@ -402,10 +414,10 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
     if (depth3) {  // children first take their grandchildren's sums
       const long long work3 = (long long)s.BH() * s.M0 * s.C * s.d;
       const int pb3 = (int)std::min<long long>((work3 + 255) / 256, (long long)sms * 8);
-      aggregate_parents_kernel<<<pb3, 256, 0, st>>>(vsum, s.BH(), Mt, s.M0, s.M0 * s.C, s.M0 + s.M0 * s.C,
-                                                    s.C, s.d);
+      aggregate_parents_kernel<<<pb3, 256, 0, st>>>(vsum, cnt, s.BH(), Mt, s.M0, s.M0 * s.C,
+                                                    s.M0 + s.M0 * s.C, s.C, s.d);
     }
-    aggregate_parents_kernel<<<pb, 256, 0, st>>>(vsum, s.BH(), Mt, 0, s.M0, s.M0, s.C, s.d);
+    aggregate_parents_kernel<<<pb, 256, 0, st>>>(vsum, cnt, s.BH(), Mt, 0, s.M0, s.M0, s.C, s.d);
   }
   log.add(s.C > 0 ? "aggregate_stream aggregate_parents" : "aggregate_stream");
   (void)err;

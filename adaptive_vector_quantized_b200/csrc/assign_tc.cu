@@ -50,6 +50,7 @@ struct AssignArgs {
   int32_t* counts;     // [BH][Mt], accumulated (zeroed by the caller)
   unsigned int* err;
   int H, N, M0, C, nblk, ntiles, tiles_per_cta;
+  int count;  // warpgroup kernel: 0 leaves the counts to the streaming value sums
 };
 
 // bf16 pair x bf16 pair accumulated into fp32 (two exact products, two roundings).
@@ -844,7 +845,7 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
       }
       const int row = (t - bh * a.nblk) * kKeys + wt;
       if (row < a.N) a.assign[(size_t)bh * a.N + row] = code;
-      count_codes_par(a.counts + (size_t)bh * Mt, par, code, row < a.N, M0);
+      if (a.count) count_codes_par(a.counts + (size_t)bh * Mt, par, code, row < a.N, M0);
     }
     if (aborted) *sAbort = 1;
     tc::tc_fence_before();
@@ -1313,7 +1314,8 @@ size_t assign_tc_workspace(const Shape& s) {
 
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents, const void* children,
                              int32_t* assign, int32_t* counts, void* ws, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log, float* vsum_to_zero) {
+                             LaunchLog& log, float* vsum_to_zero, bool* counts_left) {
+  if (counts_left) *counts_left = false;
   bf16* cw = static_cast<bf16*>(ws);
   float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
   const long long work = (long long)s.H * s.Mt() * (s.d / 8);
@@ -1350,11 +1352,16 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
   a.nblk = (s.N + kKeys - 1) / kKeys;
   a.ntiles = a.nblk * s.BH();
   a.tiles_per_cta = 1;
+  a.count = 1;
   const size_t ch_bytes = (size_t)s.M0 * s.C * s.d * 2;
   if (s.M0 <= 64) {  // warpgroup-pipelined kernel when the whole image fits
     const int nwg = s.d == 64 ? wg_count<64>(s) : wg_count<128>(s);
     if (nwg > 0) {
+      // the streaming value sums count runs of equal codes far more cheaply
+      // than the tile's warp-aggregated atomics on the assignment's chain
+      if (counts_left) a.count = 0;
       e = s.d == 64 ? launch_wg<64>(s, kmap, a, nwg, st) : launch_wg<128>(s, kmap, a, nwg, st);
+      if (e == cudaSuccess && counts_left) *counts_left = true;
       log.add("assign_tc_wg");
       return e;
     }

@@ -238,9 +238,10 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
   if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
   // the tensor-core path zeroes counts (and, for the atomic-order value sums,
   // vsum) in its codebook preparation launch
+  bool counts_left = false;  // counts left by the assignment to the streaming sums
   if (use_tc) {
     e = launch_assign_tc(s, K, parents, children, assign, counts, ws, err, cs, log,
-                         deterministic ? nullptr : vsum);
+                         deterministic ? nullptr : vsum, deterministic ? nullptr : &counts_left);
   } else {
     e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), cs);
     if (e != cudaSuccess) return cuda_fail(e, "zero counts");
@@ -250,7 +251,7 @@ avq_status avq_quantize(const avq_dims* dims, avq_dtype dtype, const void* K, co
   if (deterministic)
     e = launch_aggregate_det(s, dtype, V, assign, vsum, counts, ws_det_ptr, cs, log);
   else
-    e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, use_tc);
+    e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, use_tc, false, counts_left);
   if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
   snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
   return AVQ_OK;
@@ -529,15 +530,16 @@ extern "C" avq_status avq_quantize_noalloc(const avq_dims* dims, avq_dtype dtype
   // The scratch needs no clearing: the codebook image is rewritten in full
   // by every call before the assignment reads it.
   cudaError_t e;
+  bool counts_left = false;  // counts left by the assignment to the streaming sums
   if (use_tc) {  // counts and vsum zeroed by the codebook preparation launch
-    e = launch_assign_tc(s, K, parents, children, assign, counts, scratch, err, cs, log, vsum);
+    e = launch_assign_tc(s, K, parents, children, assign, counts, scratch, err, cs, log, vsum, &counts_left);
   } else {
     e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * s.Mt() * sizeof(int32_t), cs);
     if (e != cudaSuccess) return cuda_fail(e, "zero counts");
     e = launch_assign_simt(s, dtype, K, parents, children, assign, counts, cs, log);
   }
   if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
-  e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, use_tc);
+  e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, use_tc, false, counts_left);
   if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
   snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
   return AVQ_OK;

@@ -32,11 +32,14 @@ cudaError_t launch_assign_simt(const Shape& s, avq_dtype dt, const void* K, cons
                                const void* children, int32_t* assign, int32_t* counts,
                                cudaStream_t st, LaunchLog& log);
 // Algorithm 1, value sums for given codes, streaming variant.
-// vsum is zeroed inside; counts are left to the assignment kernels.  depth3:
-// codes of a three-level tree (parents, M0*C children, M0*C*C grandchildren).
+// vsum is zeroed inside unless vsum_zeroed; counts are added here only when
+// `count` is set (then zeroed by the caller and left out by the assignment),
+// else the assignment kernels produce them.  depth3: codes of a three-level
+// tree (parents, M0*C children, M0*C*C grandchildren).
 cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const int32_t* assign,
                              float* vsum, int32_t* counts, unsigned int* err, cudaStream_t st,
-                             LaunchLog& log, bool vsum_zeroed = false, bool depth3 = false);
+                             LaunchLog& log, bool vsum_zeroed = false, bool depth3 = false,
+                             bool count = false);
 // Depth-3 tree (three levels, codes parents | M0*C children | M0*C*C
 // grandchildren): assignment one level deeper on the CUDA cores; counts are
 // added into counts[BH][Mt3], which the caller zeroes first.
@@ -61,11 +64,13 @@ cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
 bool assign_tc_supported(const Shape& s, avq_dtype dt);
 size_t assign_tc_workspace(const Shape& s);
 // Zeroes counts itself (and vsum when vsum_to_zero is given) before the
-// assignment adds into them.
+// assignment adds into them.  With counts_left given, the warpgroup kernel
+// may leave the counts to the streaming value sums: *counts_left tells the
+// caller whether it did.
 cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
                              const void* children, int32_t* assign, int32_t* counts, void* ws,
                              unsigned int* err, cudaStream_t st, LaunchLog& log,
-                             float* vsum_to_zero = nullptr);
+                             float* vsum_to_zero = nullptr, bool* counts_left = nullptr);
 
 // ---- stage 2 ------------------------------------------------------------
 cudaError_t launch_attention_simt(const Shape& s, avq_dtype dt, const void* Q, const void* parents,
