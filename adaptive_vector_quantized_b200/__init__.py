@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
                 L.avq_hilbert_order.argtypes = [ctypes.c_int, _vp]
                 L.avq_gilbert_order.argtypes = [ctypes.c_int, ctypes.c_int, _vp]
                 L.avq_selftest_wait.argtypes = [ctypes.c_int, _vp]
+                L.avq_selftest_exp2.argtypes = [_vp, _vp, ctypes.c_int64, _vp]
                 L.avq_workspace_size.argtypes = [P(avq_dims), ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int]
                 L.avq_workspace_size.restype = ctypes.c_size_t
@@ -90,7 +91,7 @@ def lib() -> ctypes.CDLL:
                 for name in ("avq_quantize", "avq_quantize_noalloc", "avq_attention", "avq_permute",
                              "avq_quantize3", "avq_attention3",
                              "avq_hilbert_order", "avq_gilbert_order", "avq_check_device",
-                             "avq_codebook_update", "avq_selftest_wait"):
+                             "avq_codebook_update", "avq_selftest_wait", "avq_selftest_exp2"):
                     getattr(L, name).restype = ctypes.c_int
                 _lib = L
     return _lib
@@ -444,6 +445,19 @@ def avq_selftest_wait(timeout_us: int = 2000, stream=None):
     """Launch the bounded-wait self-test: the next avq_check_device raises
     AVQError with status AVQ_ERR_TIMEOUT."""
     _check(lib().avq_selftest_wait(int(timeout_us), _stream(stream)))
+
+
+def avq_selftest_exp2(x, y=None, stream=None):
+    """The FMA-pipe 2^x of the attention kernel on a contiguous fp32 CUDA
+    tensor with an even number of elements; returns y (allocated if None)."""
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.float32):
+        raise TypeError("x must be a float32 CUDA tensor")
+    if y is None:
+        y = torch.empty_like(x)
+    _expect(y, "y", x.shape, torch.float32, x.device)
+    with torch.cuda.device(x.device):
+        _check(lib().avq_selftest_exp2(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
+    return y
 
 
 def avq_check_device(stream=None):

@@ -443,6 +443,20 @@ avq_status avq_selftest_wait(int timeout_us, avq_stream_t stream) {
   return AVQ_OK;
 }
 
+avq_status avq_selftest_exp2(const float* x, float* y, int64_t n, avq_stream_t stream) {
+  t_error[0] = 0;
+  AVQ_REQUIRE_PTR(x, "x");
+  AVQ_REQUIRE_PTR(y, "y");
+  if (n < 0 || n > (int64_t(1) << 30) || (n & 1))
+    return fail(AVQ_ERR_INVALID_ARG, "n must be even and in [0, 2^30] (got %lld)", (long long)n);
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 7u)
+    return fail(AVQ_ERR_INVALID_ARG, "x and y must be 8-byte aligned");
+  const cudaError_t e = launch_exp2_probe(x, y, (long long)n, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 self-test launch");
+  snprintf(t_kernels, sizeof(t_kernels), "%s", "exp2_probe");
+  return AVQ_OK;
+}
+
 avq_status avq_check_device(avq_stream_t stream) {
   t_error[0] = 0;
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

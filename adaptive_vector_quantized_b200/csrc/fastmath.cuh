@@ -29,12 +29,14 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // minimise the largest relative error on [-1/2, 1/2] (Lawson's iteratively
 // reweighted least squares): 7.5e-5.  2^j is then added to the exponent
 // field as an integer, j * 2^23 (the rounding constant's own high bits fall
-// off the top of the 32-bit word).  Inputs below -127 are clamped there
-// (result 0 or a tiny denormal); inputs must stay below 128.
+// off the top of the 32-bit word).  Inputs below -126 are clamped there, so
+// that the exponent field of the result never goes below zero (j >= -126 and
+// 2^f >= 2^-1/2 keep it at 0 or above: a non-negative number below 2^-125);
+// inputs must stay below 127.5.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -127.0f);
-  x.y = fmaxf(x.y, -127.0f);
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
   const float2 j = add2(x, f2(kRound, kRound));
   const float2 jf = add2(j, f2(-kRound, -kRound));
   const float2 f = add2(x, f2(-jf.x, -jf.y));

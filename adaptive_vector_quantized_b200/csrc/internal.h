@@ -106,6 +106,7 @@ cudaError_t make_tmap_3d_bf16(CUtensorMap* map, const void* base, int inner, int
 unsigned int* error_word();
 // One thread waits, with the given limit, on an mbarrier that nothing
 // completes (self-test of the bounded waits; sets kErrTimeout in err).
+cudaError_t launch_exp2_probe(const float* x, float* y, long long n, cudaStream_t st);
 cudaError_t launch_wait_probe(unsigned int* err, unsigned long long timeout_ns, cudaStream_t st);
 
 int num_sms();

@@ -321,6 +321,19 @@ avq_status avq_gilbert_order(int width, int height, int32_t* idx);
  */
 avq_status avq_selftest_wait(int timeout_us, avq_stream_t stream);
 
+/*
+ * avq_selftest_exp2 -- evaluates the FMA-pipe 2^x that the one-tile attention
+ * kernel uses for a quarter of its child exponentials (Cody-Waite reduction
+ * to x = j + f, |f| <= 1/2, and a fitted cubic for 2^f; relative error at
+ * most 7.5e-5 for normal results), so that tests can hold it to that bound.
+ * x, y: device fp32 arrays of n elements (n even, 0 <= n <= 2^30; 8-byte
+ * aligned); y[i] = 2^x[i] for -127 <= x[i] < 128 (inputs below -127 are
+ * clamped there).  Asynchronous on `stream`; AVQ_ERR_INVALID_ARG for a null
+ * pointer, an odd or out-of-range n or a misaligned pointer (before any
+ * launch).
+ */
+avq_status avq_selftest_exp2(const float* x, float* y, int64_t n, avq_stream_t stream);
+
 /* Bytes of device workspace that avq_quantize and avq_attention need for
  * these arguments (the larger of the two).  0 means none. */
 size_t avq_workspace_size(const avq_dims* dims, avq_dtype dtype, int deterministic,

@@ -161,6 +161,18 @@ def test_wait_selftest_host_checks():
         assert L.avq_selftest_wait(bad, None) == avq.AVQ_ERR_INVALID_ARG
 
 
+def test_exp2_selftest_host_checks():
+    """The exp2 self-test rejects null pointers, odd or out-of-range lengths and
+    misaligned pointers before any launch (no pointer is dereferenced)."""
+    L = avq.lib()
+    ok = ctypes.c_void_p(0x10000)
+    assert L.avq_selftest_exp2(None, ok, 2, None) == avq.AVQ_ERR_INVALID_ARG
+    assert L.avq_selftest_exp2(ok, None, 2, None) == avq.AVQ_ERR_INVALID_ARG
+    for bad_n in (3, -2, (1 << 30) + 2):
+        assert L.avq_selftest_exp2(ok, ok, bad_n, None) == avq.AVQ_ERR_INVALID_ARG
+    assert L.avq_selftest_exp2(ctypes.c_void_p(0x10004), ok, 2, None) == avq.AVQ_ERR_INVALID_ARG
+
+
 def test_fault_injection_before_launch(monkeypatch):
     """AVQ_FAULT makes the named entry points fail after their argument checks
     and before any launch (host only: nothing reaches a GPU)."""

@@ -146,6 +146,34 @@ def test_tc_attention_rescale_path():
     print("rescale", res["kernels"], diag)
 
 
+def test_tc_attention_far_below_children():
+    """Non-empty children whose logits lie far below the maximum (2^x with x
+    below -126 after the rescale, where the exponential evaluated on the FMA
+    pipe is clamped), next to children far above it (the rescale branch): no
+    NaN, and the oracle's output."""
+    H, M0, C, d, N = 1, 16, 8, 64, 512
+    rng = np.random.default_rng(6)
+    par = np.zeros((H, M0, d), dtype=np.float32)
+    par[0, :, 1:] = np.rint(rng.standard_normal((M0, d - 1)) * 8) / 8
+    off = np.zeros((C, d), dtype=np.float32)
+    off[:, 0] = [-6, -6, 2, 2, 2, 2, 2, 2]  # children 0 and 1 take the FMA-pipe exponential
+    ch = par[:, :, None, :] + off[None, None]
+    assert np.array_equal(ch.mean(2), par)
+    pick_p = rng.integers(0, M0, N)
+    pick_c = rng.integers(0, 2, N) * 2  # children 0 (far below) or 2 (far above)
+    K = ch[0][pick_p, pick_c][None, None]
+    Q = np.zeros((1, H, N, d), dtype=np.float32)
+    Q[..., 0] = 16.0
+    Q[..., 1:] = np.rint(rng.standard_normal((N, d - 1)) * 4) / 16
+    V = rng.standard_normal((1, H, N, d)).astype(np.float32)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)  # noqa: E731
+    inp = dict(Q=t(Q), K=t(K), V=t(V), parents=t(par), children=t(ch), B=1, H=H, N=N, d=d,
+               M0=M0, C=C, P=M0, block=128, scale=1.0, dtype="bf16", two_pass=False)
+    res = _forward_tc_attention(inp)
+    assert not torch.isnan(res["O"]).any()
+    gh.check_forward(inp, res)
+
+
 @pytest.mark.parametrize("P", [3, 13, 24, 40, 64])
 def test_tc_attention_chunking(inputs, P):
     """Tensor-core attention with P not a multiple of 8 (a padded child slot)
