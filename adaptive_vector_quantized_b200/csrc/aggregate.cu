@@ -394,7 +394,7 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   const long long want_warps = (long long)sms * 32;
   int kpw = (int)((total_keys + want_warps - 1) / want_warps);
   kpw = ((kpw + 31) / 32) * 32;
-  if (kpw < 64) kpw = 64;
+  if (kpw < 32) kpw = 32;
   const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
   const unsigned blocks = (unsigned)((warps + (kStreamThreads / 32) - 1) / (kStreamThreads / 32));
 #define AVQ_STREAM(T, D)                                                                            \
