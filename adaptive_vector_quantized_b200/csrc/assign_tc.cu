@@ -875,21 +875,25 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
 // C = 0): persistent CTAs over contiguous 128-key tiles; the parents' image of
 // the head and the norm step's operands stay in shared memory, K tiles come
 // through a two-slot TMA ring, and TMEM holds two score slots, so the next
-// tile's MMA runs while this tile's first maximum of T is taken.  With
-// children, assign_children_kernel then refines every key (and counts);
-// without, this kernel counts.
+// tile's MMA runs while this tile's first maximum of T is taken.  Two
+// warpgroups take the maximum, each over alternate 64-column groups of the
+// same TMEM lanes (its own keys' rows), and the first merges the second's
+// result in index order.  With children, assign_children_kernel then refines
+// every key (and counts); without, this kernel counts.
 template <int D>
 struct ParentsSmem {
-  // parents image | K ring [2] | A and B of the norm step | barriers | tmem, abort
+  // parents image | K ring [2] | A and B of the norm step | second warpgroup's
+  // maxima [128] and their parents [128] | barriers | tmem, abort
   __host__ __device__ static size_t ring_off(int M0) { return (size_t)M0 * D * 2; }
   __host__ __device__ static size_t ones_off(int M0) { return ring_off(M0) + 2 * kKeys * D * 2; }
   __host__ __device__ static size_t bnorm_off(int M0) { return ones_off(M0) + kKeys * 128; }
-  __host__ __device__ static size_t bar_off(int M0) { return bnorm_off(M0) + (size_t)M0 * 128; }
+  __host__ __device__ static size_t xchg_off(int M0) { return bnorm_off(M0) + (size_t)M0 * 128; }
+  __host__ __device__ static size_t bar_off(int M0) { return xchg_off(M0) + 2 * kKeys * 4; }
   __host__ __device__ static size_t total(int M0) { return bar_off(M0) + 64; }
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(256) assign_parents_kernel(const __grid_constant__ CUtensorMap kmap,
                                                              const AssignArgs a) {
   using S = ParentsSmem<D>;
   constexpr int KH = D / 64;
@@ -900,13 +904,16 @@ __global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_consta
   uint8_t* sRing = sm + S::ring_off(M0);
   uint8_t* sOnes = sm + S::ones_off(M0);
   uint8_t* sBn = sm + S::bnorm_off(M0);
+  float* sXT = reinterpret_cast<float*>(sm + S::xchg_off(M0));  // [kKeys]
+  int* sXP = reinterpret_cast<int*>(sXT + kKeys);               // [kKeys]
   uint64_t* bar_k = reinterpret_cast<uint64_t*>(sm + S::bar_off(M0));  // [2]
   uint64_t* bar_cb = bar_k + 2;
   uint64_t* bar_mma = bar_k + 3;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar_k + 4);
   int* sAbort = reinterpret_cast<int*>(bar_k + 4) + 1;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, wt = tid & 127;
+  const int nthr = blockDim.x;
   const int t0 = blockIdx.x * a.tiles_per_cta;
   const int t1 = min(a.ntiles, t0 + a.tiles_per_cta);
   if (t0 >= t1) return;
@@ -919,7 +926,7 @@ __global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_consta
     tc::prefetch_tensormap(&kmap);
   }
   // A of the norm step: row r = (1, 1, 1, 0, ...) in logical 16-byte chunk 0
-  for (int i = tid; i < kKeys * 8; i += 128) {
+  for (int i = tid; i < kKeys * 8; i += nthr) {
     const int r = i >> 3, pos = i & 7;
     reinterpret_cast<uint4*>(sOnes)[i] =
         pos == (r & 7) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0, 0, 0, 0);
@@ -933,7 +940,7 @@ __global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_consta
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *sTmem;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 
   // per barrier, the parity of the phase that thread 0's last copy or MMA on
   // it completes (bit b of `issued` once there was one): bits 0-1 the K ring
@@ -964,7 +971,7 @@ __global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_consta
       for (uint32_t off = 0; off < bytes; off += 65536)
         tc::bulk_g2s(sPar + off, src + off, min(bytes - off, 65536u), bar_cb);
     }
-    for (int i = tid; i < M0 * 8; i += 128) {  // -|p|^2 / 2 as a bf16 triple
+    for (int i = tid; i < M0 * 8; i += nthr) {  // -|p|^2 / 2 as a bf16 triple
       const int m = i >> 3, pos = i & 7;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (pos == (m & 7)) {
@@ -1039,12 +1046,13 @@ __global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_consta
       }
       if (tid == 0 && !*sAbort) issue_mma(t + 1);
     }
-    // first maximum of T: four independent running maxima over interleaved
-    // 16-column groups, merged in index order
+    // first maximum of T: this warpgroup's 64-column groups (wg, wg + 2, ...),
+    // four independent running maxima over interleaved 16-column groups in
+    // each, merged in index order
     const uint32_t ts = tmem + (uint32_t)slot * slot_cols + lane_off;
     float bestT = NEG_INF;
-    int par = 0;
-    for (int g0 = 0; g0 < M0; g0 += 64) {
+    int par = wg == 0 ? 0 : M0;  // the merge keeps an in-range parent whatever the scores
+    for (int g0 = wg * 64; g0 < M0; g0 += 128) {
       uint32_t r[64];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -1077,9 +1085,22 @@ __global__ void __launch_bounds__(128) assign_parents_kernel(const __grid_consta
           par = iq[q];
         }
     }
-    const int row = blk * kKeys + tid;
-    if (row < a.N) a.assign[(size_t)bh * a.N + row] = par;
-    if (C == 0) count_codes(a.counts + (size_t)bh * Mt, par, row < a.N, M0, C);
+    if (wg == 1) {
+      sXT[wt] = bestT;
+      sXP[wt] = par;
+    }
+    __syncthreads();  // the second warpgroup's maxima are in
+    if (wg == 0) {  // merge: the larger T, equal T to the lower parent index
+      const float ot = sXT[wt];
+      const int op = sXP[wt];
+      if (ot > bestT || (ot == bestT && op < par)) {
+        bestT = ot;
+        par = op;
+      }
+      const int row = blk * kKeys + wt;
+      if (row < a.N) a.assign[(size_t)bh * a.N + row] = par;
+      if (C == 0) count_codes(a.counts + (size_t)bh * Mt, par, row < a.N, M0, C);
+    }
     tc::tc_fence_before();
     __syncthreads();  // this TMEM slot is read: the MMA two tiles on may overwrite it
   }
@@ -1263,7 +1284,7 @@ cudaError_t launch_parents(const Shape& s, const CUtensorMap& kmap, AssignArgs a
   const int ctas = std::min(a.ntiles, num_sms() * per_sm);
   a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
   const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
-  assign_parents_kernel<D><<<grid, 128, smem, st>>>(kmap, a);
+  assign_parents_kernel<D><<<grid, 256, smem, st>>>(kmap, a);
   return cudaGetLastError();
 }
 
