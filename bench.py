@@ -298,7 +298,7 @@ def run_avq(args, cfg, inp, n_global=None):
     vsum = torch.empty((B, H, Mt, d), dtype=torch.float32, device=dev)
     counts = torch.empty((B, H, Mt), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
-    sel = torch.empty((B, H, nblk, max(P, 1)), dtype=torch.int32, device=dev)
+    sel = torch.empty((B, H, nblk, P), dtype=torch.int32, device=dev)
     gch = inp["grandchildren"].to(dev) if depth3 else None
 
     exchange = n_global is not None and world > 1
