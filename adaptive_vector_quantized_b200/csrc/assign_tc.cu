@@ -53,18 +53,6 @@ struct AssignArgs {
   int count;  // warpgroup kernel: 0 leaves the counts to the streaming value sums
 };
 
-// bf16 pair x bf16 pair accumulated into fp32 (two exact products, two roundings).
-__device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
-  float d;
-  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t.reg .f32 t;\n\t"
-      "mov.b32 {a0, a1}, %1;\n\t"
-      "mov.b32 {b0, b1}, %2;\n\t"
-      "fma.rn.f32.bf16 t, a0, b0, %3;\n\t"
-      "fma.rn.f32.bf16 %0, a1, b1, t;\n\t}"
-      : "=f"(d)
-      : "r"(a), "r"(b), "f"(c));
-  return d;
-}
 
 // bf16 bits of x, round to nearest even.
 __device__ __forceinline__ uint32_t bf16_bits(float x) {

@@ -20,6 +20,21 @@ enum : unsigned int {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// bf16 pair x bf16 pair accumulated into fp32, the low halves first: the
+// products of two bf16 values are exact in fp32, so this equals two fmaf on
+// the values converted to fp32 (two roundings).
+__device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 t, a0, b0, %3;\n\t"
+      "fma.rn.f32.bf16 %0, a1, b1, t;\n\t}"
+      : "=f"(d)
+      : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+
 // 8 consecutive elements -> fp32 (p must be 16-byte aligned).
 __device__ __forceinline__ void load8(const float* p, float* o) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(p));

@@ -21,6 +21,8 @@
 // are refined with their grandchildren: the child's logit is the mean of its
 // grandchildren's (Eq. 8), dA = exp(s_g - m) - exp(s_c - m) (Eq. 9), zero for
 // empty grandchildren, merged with the online maximum.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -163,6 +165,38 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
   __syncthreads();
 
   const float* qr = qs + (size_t)(tid < block ? tid : 0) * (D + 1);
+  // bf16: the row's query as bf16 pairs in registers, multiplied with the
+  // codewords by fma.rn.f32.bf16 in the same order as dot3 (the bf16 products
+  // are exact in fp32, so the sums are the same); fp32: the row in shared memory
+  constexpr bool kBf16 = std::is_same<T, bf16>::value;
+  uint32_t qv[kBf16 ? D / 2 : 1];
+  if constexpr (kBf16) {
+    const uint4* qp = reinterpret_cast<const uint4*>(Q + ((size_t)bh * N + (valid ? i : blk * block)) * D);
+#pragma unroll
+    for (int t = 0; t < D / 8; ++t) {
+      const uint4 u = __ldg(qp + t);
+      qv[4 * t] = u.x;
+      qv[4 * t + 1] = u.y;
+      qv[4 * t + 2] = u.z;
+      qv[4 * t + 3] = u.w;
+    }
+  }
+  auto qdot = [&](const T* c) -> float {
+    if constexpr (kBf16) {
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < D; t += 8) {
+        const uint4 cv = __ldg(reinterpret_cast<const uint4*>(c + t));
+        acc = fma_bf16x2(qv[t / 2], cv.x, acc);
+        acc = fma_bf16x2(qv[t / 2 + 1], cv.y, acc);
+        acc = fma_bf16x2(qv[t / 2 + 2], cv.z, acc);
+        acc = fma_bf16x2(qv[t / 2 + 3], cv.w, acc);
+      }
+      return acc;
+    } else {
+      return dot3<T, D>(qr, c);
+    }
+  };
   const T* par = parents + (size_t)h * M0 * D;
   const T* chd = children + (size_t)h * M1 * D;
   const T* gcd = grandchildren + (size_t)h * M1 * C * D;
@@ -187,7 +221,7 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
   for (int j = 0; j < M0; ++j) {
     const float nj = nf[j];
     if (nj > 0.f) {
-      const float s = scale * dot3<T, D>(qr, par + (size_t)j * D);
+      const float s = scale * qdot(par + (size_t)j * D);
       if (s > m) {
         z = z * expf(m - s) + nj;
         m = s;
@@ -202,7 +236,7 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
       const float nj = nf[j];
       float a = 0.f;
       if (nj > 0.f) {
-        a = expf(scale * dot3<T, D>(qr, par + (size_t)j * D) - m);
+        a = expf(scale * qdot(par + (size_t)j * D) - m);
         add_row(a, vs + (size_t)j * D);
       }
       const float col = warp_sum(valid ? a * nj * rz : 0.f);
@@ -236,7 +270,7 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       if (c < C) {
-        sc[c] = scale * dot3<T, D>(qr, sub + (size_t)c * D);
+        sc[c] = scale * qdot(sub + (size_t)c * D);
         sp += sc[c];
         if (nf[code0 + c] > 0.f && sc[c] > mp) mp = sc[c];
       }
@@ -273,7 +307,7 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
       const int code = M0 + ssel[u / C] * C + (u % C);
       const float nc = nf[code];
       float a = 0.f;
-      if (nc > 0.f) a = expf(scale * dot3<T, D>(qr, chd + (size_t)(code - M0) * D) - m);
+      if (nc > 0.f) a = expf(scale * qdot(chd + (size_t)(code - M0) * D) - m);
       const float col = warp_sum(a * nc * rz);
       if (lane == 0 && col != 0.f) atomicAdd(w2 + u, col);
     }
