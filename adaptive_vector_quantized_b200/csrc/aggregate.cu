@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
     int32_t* __restrict__ counts, int BH, int N, int Mt, int keys_per_warp) {
   constexpr int E = D / 32;
   using F = Frag<T, E>;
-  constexpr int B = F::kBatch;  // keys loaded at once (32 / B batches per group)
+  grid_dependency_wait();  // codes (and zeroed sums) of the launches before
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kStreamThreads / 32) + (threadIdx.x >> 5);
   const int warps_per_head = (N + keys_per_warp - 1) / keys_per_warp;
@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(kStreamThreads) aggregate_stream_kernel(
 __global__ void __launch_bounds__(256) aggregate_parents_kernel(float* __restrict__ vsum,
                                                                int32_t* __restrict__ counts, int BH, int Mt,
                                                                int lo, int n, int lo2, int C, int D) {
+  grid_dependency_wait();  // the streamed sums and counts
   const long long total = (long long)BH * n * D;
   for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
        u += (long long)gridDim.x * blockDim.x) {
@@ -397,15 +398,16 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
   if (kpw < 32) kpw = 32;
   const long long warps = (long long)s.BH() * ((s.N + kpw - 1) / kpw);
   const unsigned blocks = (unsigned)((warps + (kStreamThreads / 32) - 1) / (kStreamThreads / 32));
-#define AVQ_STREAM(T, D)                                                                            \
-  aggregate_stream_kernel<T, D><<<blocks, kStreamThreads, 0, st>>>((const T*)V, assign, vsum, cnt, s.BH(), \
-                                                                   s.N, Mt, kpw)
+#define AVQ_STREAM(T, D)                                                                          \
+  e = launch_after(aggregate_stream_kernel<T, D>, dim3(blocks), dim3(kStreamThreads), 0, st, (const T*)V, \
+                   assign, vsum, cnt, s.BH(), s.N, Mt, kpw)
   if (dt == AVQ_F32) {
     if (s.d == 64) AVQ_STREAM(float, 64); else AVQ_STREAM(float, 128);
   } else {
     if (s.d == 64) AVQ_STREAM(bf16, 64); else AVQ_STREAM(bf16, 128);
   }
 #undef AVQ_STREAM
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (s.C > 0) {
@@ -414,10 +416,13 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
     if (depth3) {  // children first take their grandchildren's sums
       const long long work3 = (long long)s.BH() * s.M0 * s.C * s.d;
       const int pb3 = (int)std::min<long long>((work3 + 255) / 256, (long long)sms * 8);
-      aggregate_parents_kernel<<<pb3, 256, 0, st>>>(vsum, cnt, s.BH(), Mt, s.M0, s.M0 * s.C,
-                                                    s.M0 + s.M0 * s.C, s.C, s.d);
+      e = launch_after(aggregate_parents_kernel, dim3(pb3), dim3(256), 0, st, vsum, cnt, s.BH(), Mt, s.M0,
+                       s.M0 * s.C, s.M0 + s.M0 * s.C, s.C, s.d);
+      if (e != cudaSuccess) return e;
     }
-    aggregate_parents_kernel<<<pb, 256, 0, st>>>(vsum, cnt, s.BH(), Mt, 0, s.M0, s.M0, s.C, s.d);
+    e = launch_after(aggregate_parents_kernel, dim3(pb), dim3(256), 0, st, vsum, cnt, s.BH(), Mt, 0, s.M0, s.M0,
+                     s.C, s.d);
+    if (e != cudaSuccess) return e;
   }
   log.add(s.C > 0 ? "aggregate_stream aggregate_parents" : "aggregate_stream");
   (void)err;

@@ -510,6 +510,9 @@ __global__ void __launch_bounds__(384, 1) assign_wg_kernel(const __grid_constant
   const uint32_t tmem_g = *sTmem + (uint32_t)g * 128u;
   const uint32_t lane_off = (uint32_t)(wwarp * 32) << 16;
   const int barid = 1 + g;
+  // the set-up above may overlap the codebook preparation; its image, norms
+  // and zeroed statistics are read below
+  grid_dependency_wait();
 
   // per barrier, the parity of the phase that this thread's last copy or MMA
   // on it completes (bit b of `issued` once there was one): bits 0-1 the K
@@ -1201,6 +1204,7 @@ __global__ void __launch_bounds__(256) codebook_prep_kernel(const bf16* __restri
                                                             long long n_b) {
   constexpr int KH = D / 64;
   constexpr int CH = D / 8;  // 16-byte chunks per code: one thread each
+  allow_dependents();  // the assignment's set-up may overlap this launch
   const int Mt = M0 * (1 + C);
   const long long total = (long long)H * Mt * CH;
   const long long span = (total + 31) / 32 * 32;  // whole warps, so the shuffles see every lane
@@ -1293,8 +1297,7 @@ cudaError_t launch_wg_m(const Shape& s, const CUtensorMap& kmap, AssignArgs a, i
   const int ctas = std::min(a.ntiles, num_sms());
   a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
   const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
-  assign_wg_kernel<D, M0><<<grid, 128 * nwg, smem, st>>>(kmap, a);
-  return cudaGetLastError();
+  return launch_after(assign_wg_kernel<D, M0>, dim3(grid), dim3(128 * nwg), smem, st, kmap, a);
 }
 
 template <int D>

@@ -707,7 +707,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   if (tid == 0) {
     tc::prefetch_tensormap(&qmap);
     tc::prefetch_tensormap(&omap);
-    load_q(u0);
+    load_q(u0);  // Q is an input: before the wait for the image preparation
+  }
+  grid_dependency_wait();  // codeword and value-sum images, counts
+  if (tid == 0) {
     load_pcw(u0);
     load_pvb(u0);
   }
@@ -1215,6 +1218,7 @@ __global__ void __launch_bounds__(256) attention_prep_kernel(const bf16* __restr
                                                              bf16* __restrict__ cw, bf16* __restrict__ vb,
                                                              int H, int BH, int M0, int C) {
   constexpr int KH = D / 64;
+  allow_dependents();  // the attention's set-up and first Q tile may overlap this launch
   const int Mt = M0 * (1 + C);
   const int chunks_per_code = D / 8;
   const long long n_cw = (long long)H * Mt * chunks_per_code;
@@ -1257,7 +1261,8 @@ cudaError_t launch_fast_m(dim3 grid, const CUtensorMap& qmap, const CUtensorMap&
   constexpr int kCtasPerSm = D == 64 ? 4 : 2;
   const long long units = (long long)grid.x * grid.y;
   grid = dim3((unsigned)std::max<long long>(1, std::min<long long>(units, (long long)num_sms() * kCtasPerSm)));
-  attention_fast_kernel<D, M0><<<grid, 128, smem, st>>>(qmap, omap, a);
+  e = launch_after(attention_fast_kernel<D, M0>, dim3(grid), dim3(128), smem, st, qmap, omap, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
