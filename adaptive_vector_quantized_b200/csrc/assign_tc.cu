@@ -81,6 +81,7 @@ template <int D, bool CH_SMEM>
 __global__ void __launch_bounds__(128) assign_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                                         const AssignArgs a) {
   using S = AssignSmem<D, CH_SMEM>;
+  grid_dependency_wait();  // the codebook image, norms and zeroed statistics
   constexpr int KH = D / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -887,6 +888,7 @@ template <int D>
 __global__ void __launch_bounds__(256) assign_parents_kernel(const __grid_constant__ CUtensorMap kmap,
                                                              const AssignArgs a) {
   using S = ParentsSmem<D>;
+  grid_dependency_wait();  // the codebook image, norms and zeroed statistics
   constexpr int KH = D / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1129,6 +1131,7 @@ __global__ void __launch_bounds__(256) assign_children_kernel(const bf16* __rest
                                                               int32_t* __restrict__ assign,
                                                               int32_t* __restrict__ counts, int BH, int H,
                                                               int N, int M0) {
+  grid_dependency_wait();  // the parents of the pass before
   constexpr int C = 8;
   constexpr int DL = D / 8;      // dims per lane
   constexpr int CHK = DL / 8;    // 16-byte chunks per lane and row
@@ -1205,6 +1208,7 @@ __global__ void __launch_bounds__(256) codebook_prep_kernel(const bf16* __restri
   constexpr int KH = D / 64;
   constexpr int CH = D / 8;  // 16-byte chunks per code: one thread each
   allow_dependents();  // the assignment's set-up may overlap this launch
+  grid_dependency_wait();  // the workspace image may still be read by the launch before
   const int Mt = M0 * (1 + C);
   const long long total = (long long)H * Mt * CH;
   const long long span = (total + 31) / 32 * 32;  // whole warps, so the shuffles see every lane
@@ -1257,8 +1261,7 @@ cudaError_t launch_impl(const Shape& s, const CUtensorMap& kmap, AssignArgs a, c
   const int ctas = std::min(a.ntiles, num_sms() * per_sm);
   a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
   const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
-  assign_tc_kernel<D, CH><<<grid, 128, smem, st>>>(kmap, a);
-  return cudaGetLastError();
+  return launch_after(assign_tc_kernel<D, CH>, dim3(grid), dim3(128), smem, st, kmap, a);
 }
 
 constexpr size_t kMaxSmem = 227 * 1024;
@@ -1276,8 +1279,7 @@ cudaError_t launch_parents(const Shape& s, const CUtensorMap& kmap, AssignArgs a
   const int ctas = std::min(a.ntiles, num_sms() * per_sm);
   a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
   const int grid = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
-  assign_parents_kernel<D><<<grid, 256, smem, st>>>(kmap, a);
-  return cudaGetLastError();
+  return launch_after(assign_parents_kernel<D>, dim3(grid), dim3(256), smem, st, kmap, a);
 }
 
 // Warpgroups per CTA for the pipelined kernel (0: the image does not fit).
@@ -1338,13 +1340,15 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
   const long long n_vsum = vsum_to_zero ? (long long)s.BH() * s.Mt() * s.d * 4 / 16 : 0;
   uint4* zc = reinterpret_cast<uint4*>(counts);
   uint4* zv = reinterpret_cast<uint4*>(vsum_to_zero);
+  cudaError_t e;
   if (s.d == 64)
-    codebook_prep_kernel<64><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
-                                                      s.H, s.M0, s.C, zc, n_counts, zv, n_vsum);
+    e = launch_after(codebook_prep_kernel<64>, dim3(pblocks), dim3(256), 0, st, (const bf16*)parents,
+                     (const bf16*)children, cw, norms, s.H, s.M0, s.C, zc, n_counts, zv, n_vsum);
   else
-    codebook_prep_kernel<128><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, cw, norms,
-                                                       s.H, s.M0, s.C, zc, n_counts, zv, n_vsum);
-  cudaError_t e = cudaGetLastError();
+    e = launch_after(codebook_prep_kernel<128>, dim3(pblocks), dim3(256), 0, st, (const bf16*)parents,
+                     (const bf16*)children, cw, norms, s.H, s.M0, s.C, zc, n_counts, zv, n_vsum);
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   log.add("codebook_prep");
 
@@ -1393,13 +1397,14 @@ cudaError_t launch_assign_tc(const Shape& s, const void* K, const void* parents,
     const long long groups = ((long long)s.BH() * s.N + 3) / 4;  // 4 keys per warp
     const int blocks = (int)std::max<long long>(1, std::min<long long>((groups + 7) / 8, (long long)num_sms() * 16));
     if (s.d == 64)
-      assign_children_kernel<64><<<blocks, 256, 0, st>>>((const bf16*)K, (const bf16*)parents,
-                                                         (const bf16*)children, norms, assign, counts, s.BH(),
-                                                         s.H, s.N, s.M0);
+      e = launch_after(assign_children_kernel<64>, dim3(blocks), dim3(256), 0, st, (const bf16*)K,
+                       (const bf16*)parents, (const bf16*)children, (const float*)norms, assign, counts, s.BH(),
+                       s.H, s.N, s.M0);
     else
-      assign_children_kernel<128><<<blocks, 256, 0, st>>>((const bf16*)K, (const bf16*)parents,
-                                                          (const bf16*)children, norms, assign, counts, s.BH(),
-                                                          s.H, s.N, s.M0);
+      e = launch_after(assign_children_kernel<128>, dim3(blocks), dim3(256), 0, st, (const bf16*)K,
+                       (const bf16*)parents, (const bf16*)children, (const float*)norms, assign, counts, s.BH(),
+                       s.H, s.N, s.M0);
+    if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     log.add("assign_children");
   }

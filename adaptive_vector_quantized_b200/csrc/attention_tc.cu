@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
                                                            const __grid_constant__ CUtensorMap omap,
                                                            const AttnArgs a) {
   using S = Smem<D>;
+  grid_dependency_wait();  // the image preparation before
   constexpr int KH = D / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -707,10 +708,12 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
   if (tid == 0) {
     tc::prefetch_tensormap(&qmap);
     tc::prefetch_tensormap(&omap);
-    load_q(u0);  // Q is an input: before the wait for the image preparation
   }
-  grid_dependency_wait();  // codeword and value-sum images, counts
+  // images and counts of the preparation before; Q too, since the launch
+  // that wrote it may have ended only just before that preparation began
+  grid_dependency_wait();
   if (tid == 0) {
+    load_q(u0);
     load_pcw(u0);
     load_pvb(u0);
   }
@@ -1219,6 +1222,7 @@ __global__ void __launch_bounds__(256) attention_prep_kernel(const bf16* __restr
                                                              int H, int BH, int M0, int C) {
   constexpr int KH = D / 64;
   allow_dependents();  // the attention's set-up and first Q tile may overlap this launch
+  grid_dependency_wait();  // the statistics of the launches before; the images may still be read
   const int Mt = M0 * (1 + C);
   const int chunks_per_code = D / 8;
   const long long n_cw = (long long)H * Mt * chunks_per_code;
@@ -1302,13 +1306,15 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
   bf16* vb = reinterpret_cast<bf16*>(static_cast<char*>(ws) + align256((size_t)s.H * s.Mt() * s.d * 2));
   const long long work = (long long)(s.H + s.BH()) * s.Mt() * (s.d / 8);
   const int pblocks = (int)std::min<long long>((work + 255) / 256, (long long)num_sms() * 8);
+  cudaError_t e;
   if (s.d == 64)
-    attention_prep_kernel<64><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, vsum,
-                                                       cw, vb, s.H, s.BH(), s.M0, s.C);
+    e = launch_after(attention_prep_kernel<64>, dim3(pblocks), dim3(256), 0, st, (const bf16*)parents,
+                     (const bf16*)children, vsum, cw, vb, s.H, s.BH(), s.M0, s.C);
   else
-    attention_prep_kernel<128><<<pblocks, 256, 0, st>>>((const bf16*)parents, (const bf16*)children, vsum,
-                                                        cw, vb, s.H, s.BH(), s.M0, s.C);
-  cudaError_t e = cudaGetLastError();
+    e = launch_after(attention_prep_kernel<128>, dim3(pblocks), dim3(256), 0, st, (const bf16*)parents,
+                     (const bf16*)children, vsum, cw, vb, s.H, s.BH(), s.M0, s.C);
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   log.add("attention_prep");
 
@@ -1344,12 +1350,14 @@ cudaError_t launch_attention_tc(const Shape& s, const void* Q, const void* paren
     const int smem = Smem<64>::kTotal + 1024;
     e = cudaFuncSetAttribute(attention_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attention_tc_kernel<64><<<grid, 128, smem, st>>>(qmap, omap, a);
+    e = launch_after(attention_tc_kernel<64>, grid, dim3(128), smem, st, qmap, omap, a);
+    if (e != cudaSuccess) return e;
   } else {
     const int smem = Smem<128>::kTotal + 1024;
     e = cudaFuncSetAttribute(attention_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attention_tc_kernel<128><<<grid, 128, smem, st>>>(qmap, omap, a);
+    e = launch_after(attention_tc_kernel<128>, grid, dim3(128), smem, st, qmap, omap, a);
+    if (e != cudaSuccess) return e;
   }
   log.add("attention_tc");
   return cudaGetLastError();
