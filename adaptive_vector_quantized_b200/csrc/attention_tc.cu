@@ -59,9 +59,13 @@ struct AttnArgs {
 // shared memory plan (bytes); every operand region 1024-aligned
 template <int D>
 struct Smem {
+  // codeword tile buffers: at d = 128 two, so that the next tile's codewords
+  // arrive while this tile is processed (two CTAs per SM still fit); at d = 64
+  // one (four CTAs per SM)
+  static constexpr int kNB = D == 128 ? 2 : 1;
   static constexpr int kQ = 0;                              // Q tile / O staging
-  static constexpr int kCW = kQ + kRows * D * 2;            // codeword tile (64 codes)
-  static constexpr int kVB = kCW + kTile * D * 2;           // value-sum tile (64 codes)
+  static constexpr int kCW = kQ + kRows * D * 2;            // codeword tile(s) (64 codes each)
+  static constexpr int kVB = kCW + kNB * kTile * D * 2;     // value-sum tile (64 codes)
   static constexpr int kPR = kVB + kTile * D * 2;           // probabilities [128][64] bf16
   static constexpr int kNF = kPR + kRows * kTile * 2;       // counts of the tile (float)
   static constexpr int kBI = kNF + kTile * 4;               // mask bias of the tile (0 / -inf)
@@ -69,8 +73,9 @@ struct Smem {
   static constexpr int kWP = kW + 256 * 4;                  // per-warp partial sums [4][kTile]
   static constexpr int kSEL = kWP + 4 * kTile * 4;          // selected parents [256]
   static constexpr int kRK = kSEL + 256 * 4;                // partial ranks [2][128]
-  static constexpr int kBAR = kRK + 256 * 4;                // 4 mbarriers
-  static constexpr int kMISC = kBAR + 32;                   // tmem base, abort flag
+  static constexpr int kCNTP = kRK + 256 * 4;               // the parents' counts (float) [256]
+  static constexpr int kBAR = kCNTP + 256 * 4;              // 5 mbarriers
+  static constexpr int kMISC = kBAR + 40;                   // tmem base, abort flag
   static constexpr int kTotal = kMISC + 32;
   static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;  // logits [64] + output [D]
 };
@@ -133,10 +138,12 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   float* sWP = reinterpret_cast<float*>(sm + S::kWP);
   int* sSEL = reinterpret_cast<int*>(sm + S::kSEL);
   uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + S::kBAR);
-  uint64_t* bar_cp = bar_q + 1;   // codeword tiles
+  uint64_t* bar_cp = bar_q + 1;   // codeword tiles in buffer 0
   uint64_t* bar_mma = bar_q + 2;
   uint64_t* bar_vb = bar_q + 3;   // value-sum tiles (waited on only before the value MMA)
+  uint64_t* bar_cp1 = bar_q + 4;  // codeword tiles in buffer 1 (d = 128)
   int* sRK = reinterpret_cast<int*>(sm + S::kRK);
+  float* sCNTP = reinterpret_cast<float*>(sm + S::kCNTP);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S::kMISC);
   int* sAbort = reinterpret_cast<int*>(sm + S::kMISC + 4);
   float* sNtot = reinterpret_cast<float*>(sm + S::kMISC + 8);  // keys of the head (extrapolation)
@@ -158,6 +165,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
     tc::mbar_init(bar_cp, 1);
     tc::mbar_init(bar_mma, 1);
     tc::mbar_init(bar_vb, 1);
+    tc::mbar_init(bar_cp1, 1);
     tc::fence_mbar_init();
     *sAbort = 0;
     *sNtot = 0.f;
@@ -168,7 +176,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
     tc::tmem_alloc(sTmem, S::kTmemCols);
     tc::tmem_relinquish();
   }
-  for (int j = tid; j < M0; j += 128) sW[j] = 0.f;
+  for (int j = tid; j < M0; j += 128) {
+    sW[j] = 0.f;
+    sCNTP[j] = (float)__ldg(cnt + j);
+  }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -177,7 +188,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   const uint32_t tX = tmem + kTile;  // output accumulator, D columns
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-  uint32_t ph_cp = 0, ph_mma = 0, ph_vb = 0;
+  uint32_t ph_cp = 0, ph_mma = 0, ph_vb = 0, ph_cp1 = 0;
   // per barrier, the parity of the phase that thread 0's last copy or MMA on
   // it completes (bit b of `issued` once there was one): drained on the way out
   uint32_t issued = 0, exp_par = 0;
@@ -195,14 +206,16 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
   const uint32_t idesc_x = tc::idesc_bf16(kRows, D, 0, 1);
   const uint32_t sQa = tc::smem_u32(sQ), sCWa = tc::smem_u32(sCW), sVBa = tc::smem_u32(sVB),
                  sPRa = tc::smem_u32(sPR);
-  // S = Q * CW^T over n codes (n a multiple of 16, <= 64) -- one thread
-  auto issue_logits = [&](int n) {
+  // S = Q * CW^T over n codes (n a multiple of 16, <= 64) from codeword
+  // buffer `b` -- one thread
+  auto issue_logits = [&](int n, int b) {
     note(3, ph_mma);
     const uint32_t idesc = tc::idesc_bf16(kRows, n, 0, 0);
+    const uint32_t cwa = sCWa + (uint32_t)(b * kTile * D * 2);
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
       const uint64_t ad = tc::sdesc_sw128(sQa + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16, 1024);
-      const uint64_t bd = tc::sdesc_sw128(sCWa + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
+      const uint64_t bd = tc::sdesc_sw128(cwa + (k >> 2) * 1024 + (k & 3) * 32, 16, KH * 1024);
       tc::mma_bf16(tS, ad, bd, idesc, k > 0);
     }
     tc::mma_commit(bar_mma);
@@ -222,9 +235,23 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
     ph_mma ^= 1;
     tc::tc_fence_after();
   };
-  auto wait_cp = [&]() {
-    if (!tc::mbar_wait(bar_cp, ph_cp)) fail(a.err, sAbort);
-    ph_cp ^= 1;
+  auto wait_cp = [&](int b) {
+    if (b == 0) {
+      if (!tc::mbar_wait(bar_cp, ph_cp)) fail(a.err, sAbort);
+      ph_cp ^= 1;
+    } else {
+      if (!tc::mbar_wait(bar_cp1, ph_cp1)) fail(a.err, sAbort);
+      ph_cp1 ^= 1;
+    }
+  };
+  // parent tile t's codewords into buffer b (thread 0)
+  auto copy_tile = [&](int t, int b) {
+    const int n = min(kTile, M0 - t * kTile);
+    const uint32_t cwb = (uint32_t)n * D * 2;
+    uint64_t* bar = b == 0 ? bar_cp : bar_cp1;
+    if (b == 0) note(1, ph_cp); else note(4, ph_cp1);
+    tc::mbar_arrive_expect_tx(bar, cwb);
+    tc::bulk_g2s(sCW + b * kTile * D * 2, cw_h + (size_t)(t * kTile / 8) * KH * 512, cwb, bar);
   };
   auto wait_vb = [&]() {
     if (!tc::mbar_wait(bar_vb, ph_vb)) fail(a.err, sAbort);
@@ -249,31 +276,35 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
 
   // ---- parents: one sweep (all parents in one tile) or two (running max and
   //      denominator first, then probabilities, values and importance) ----
+  // The g-th tile of the sweeps uses codeword buffer g % kNB; with two
+  // buffers, tile g + 1's copy is issued as soon as tile g's logit MMA is
+  // (buffer (g + 1) % 2 was last read by tile g - 1's MMA, which completed).
+  constexpr int kNB = S::kNB;
+  if (kNB == 2 && tid == 0) copy_tile(0, 0);
   for (int sweep = 0; sweep < sweeps; ++sweep) {
     const bool last = sweep == sweeps - 1;
     for (int t = 0; t < nT; ++t) {
       const int c0 = t * kTile;
       const int n = min(kTile, M0 - c0);
+      const int g = sweep * nT + t, b = g % kNB;
+      uint8_t* cwbuf = sCW + b * kTile * D * 2;
       if (tid == 0) {
-        const uint32_t cwb = (uint32_t)n * D * 2;
-        note(1, ph_cp);
-        tc::mbar_arrive_expect_tx(bar_cp, cwb);
-        tc::bulk_g2s(sCW, cw_h + (size_t)(c0 / 8) * KH * 512, cwb, bar_cp);
+        if (kNB == 1) copy_tile(t, 0);
         if (last) {
           note(2, ph_vb);
-          tc::mbar_arrive_expect_tx(bar_vb, cwb);
-          tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, cwb, bar_vb);
+          tc::mbar_arrive_expect_tx(bar_vb, (uint32_t)n * D * 2);
+          tc::bulk_g2s(sVB, vb_bh + (size_t)(c0 / 8) * KH * 512, (uint32_t)n * D * 2, bar_vb);
         }
       }
       // a partial tile: zero the unused codeword rows so that the logits MMA can
       // always run over 64 columns with finite results
       for (int i = tid; i < (kTile - n) * KH * 8; i += 128) {
         const int row = n + i / (KH * 8), rest = i % (KH * 8);
-        *reinterpret_cast<uint4*>(sCW + (row >> 3) * (KH * 1024) + (rest >> 3) * 1024 + (row & 7) * 128 +
+        *reinterpret_cast<uint4*>(cwbuf + (row >> 3) * (KH * 1024) + (rest >> 3) * 1024 + (row & 7) * 128 +
                                   (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
       }
       for (int j = tid; j < kTile; j += 128) {
-        const float nf = j < n ? (float)__ldg(cnt + c0 + j) : 0.f;
+        const float nf = j < n ? sCNTP[c0 + j] : 0.f;
         sNF[j] = nf;
         sBI[j] = nf > 0.f ? 0.f : NEG_INF;
       }
@@ -282,12 +313,13 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
         if (!tc::mbar_wait(bar_q, 0)) fail(a.err, sAbort);
         q_ready = true;
       }
-      wait_cp();
+      wait_cp(b);
       __syncthreads();
       if (*sAbort) goto done;
       if (tid == 0) {
         tc::tc_fence_after();
-        issue_logits(kTile);
+        issue_logits(kTile, b);
+        if (kNB == 2 && g + 1 < sweeps * nT) copy_tile((g + 1) % nT, b ^ 1);
       }
       wait_mma();
       {
@@ -458,12 +490,12 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_tc_kernel(cons
         const int r = j >> 3;
         sNF[j] = r < np ? (float)__ldg(cnt + M0 + sSEL[q * kChunkParents + r] * 8 + (j & 7)) : 0.f;
       }
-      wait_cp();
+      wait_cp(0);
       __syncthreads();
       if (*sAbort) goto done;
       if (tid == 0) {
         tc::tc_fence_after();
-        issue_logits(n);
+        issue_logits(n, 0);
       }
       wait_mma();
       uint32_t r[64];
@@ -559,9 +591,9 @@ done:
   // nothing in flight before TMEM is freed (the waits return at once for
   // completed operations; 1 ms limit)
   if (issued) {
-    uint64_t* const bars[4] = {bar_q, bar_cp, bar_vb, bar_mma};
+    uint64_t* const bars[5] = {bar_q, bar_cp, bar_vb, bar_mma, bar_cp1};
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
+    for (int b = 0; b < 5; ++b)
       if ((issued >> b) & 1u)
         if (!tc::mbar_wait(bars[b], (exp_par >> b) & 1u, 1000000ull)) atomicOr(a.err, kErrTimeout);
   }
