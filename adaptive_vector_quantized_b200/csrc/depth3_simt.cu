@@ -166,8 +166,8 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
 
   const float* qr = qs + (size_t)(tid < block ? tid : 0) * (D + 1);
   // bf16: the row's query as bf16 pairs in registers, multiplied with the
-  // codewords by fma.rn.f32.bf16 in the same order as dot3 (the bf16 products
-  // are exact in fp32, so the sums are the same); fp32: the row in shared memory
+  // codewords by fma.rn.f32.bf16 (the bf16 products are exact in fp32); fp32:
+  // the row in shared memory
   constexpr bool kBf16 = std::is_same<T, bf16>::value;
   uint32_t qv[kBf16 ? D / 2 : 1];
   if constexpr (kBf16) {
@@ -183,16 +183,18 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
   }
   auto qdot = [&](const T* c) -> float {
     if constexpr (kBf16) {
-      float acc = 0.f;
+      // four partial sums (dims t, t+1 mod 8 in one, ...) shorten the chain of
+      // dependent adds; combined in a fixed order
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int t = 0; t < D; t += 8) {
         const uint4 cv = __ldg(reinterpret_cast<const uint4*>(c + t));
-        acc = fma_bf16x2(qv[t / 2], cv.x, acc);
-        acc = fma_bf16x2(qv[t / 2 + 1], cv.y, acc);
-        acc = fma_bf16x2(qv[t / 2 + 2], cv.z, acc);
-        acc = fma_bf16x2(qv[t / 2 + 3], cv.w, acc);
+        acc[0] = fma_bf16x2(qv[t / 2], cv.x, acc[0]);
+        acc[1] = fma_bf16x2(qv[t / 2 + 1], cv.y, acc[1]);
+        acc[2] = fma_bf16x2(qv[t / 2 + 2], cv.z, acc[2]);
+        acc[3] = fma_bf16x2(qv[t / 2 + 3], cv.w, acc[3]);
       }
-      return acc;
+      return (acc[0] + acc[1]) + (acc[2] + acc[3]);
     } else {
       return dot3<T, D>(qr, c);
     }
