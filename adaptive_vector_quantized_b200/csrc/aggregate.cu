@@ -46,14 +46,12 @@ struct Frag;
 template <>
 struct Frag<bf16, 2> {
   using R = uint32_t;
-  static constexpr int kBatch = 32;
   __device__ __forceinline__ static R load(const bf16* p) { return __ldg(reinterpret_cast<const unsigned*>(p)); }
   __device__ __forceinline__ static void unpack(R r, float* o) { o[0] = bf16_lo(r); o[1] = bf16_hi(r); }
 };
 template <>
 struct Frag<bf16, 4> {
   using R = uint2;
-  static constexpr int kBatch = 32;
   __device__ __forceinline__ static R load(const bf16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
   __device__ __forceinline__ static void unpack(R r, float* o) {
     o[0] = bf16_lo(r.x); o[1] = bf16_hi(r.x); o[2] = bf16_lo(r.y); o[3] = bf16_hi(r.y);
@@ -62,14 +60,12 @@ struct Frag<bf16, 4> {
 template <>
 struct Frag<float, 2> {
   using R = float2;
-  static constexpr int kBatch = 32;
   __device__ __forceinline__ static R load(const float* p) { return __ldg(reinterpret_cast<const float2*>(p)); }
   __device__ __forceinline__ static void unpack(R r, float* o) { o[0] = r.x; o[1] = r.y; }
 };
 template <>
 struct Frag<float, 4> {
   using R = float4;
-  static constexpr int kBatch = 16;
   __device__ __forceinline__ static R load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
   __device__ __forceinline__ static void unpack(R r, float* o) { o[0] = r.x; o[1] = r.y; o[2] = r.z; o[3] = r.w; }
 };

@@ -61,7 +61,6 @@ __device__ __forceinline__ uint32_t bf16_bits(float x) {
 
 template <int D, bool CH_SMEM>
 struct AssignSmem {
-  static constexpr int KH = D / 64;
   // parents image | children image (optional) | K ring [2] | A and B of the
   // norm step | norms | pair bits | barriers
   __host__ __device__ static size_t parents_bytes(int M0) { return (size_t)M0 * D * 2; }
