@@ -1321,6 +1321,10 @@ bool assign_tc_supported(const Shape& s, avq_dtype dt) {
   return true;
 }
 
+bool assign_tc_uses_warpgroups(const Shape& s) {
+  return s.M0 <= 64 && (s.d == 64 ? wg_count<64>(s) : wg_count<128>(s)) > 0;
+}
+
 size_t assign_tc_workspace(const Shape& s) {
   return align256((size_t)s.H * s.Mt() * s.d * 2) + align256((size_t)s.H * s.Mt() * 4);
 }

@@ -18,6 +18,7 @@ namespace avq {
 __device__ unsigned int g_avq_error_word;
 
 namespace {
+avq_status noalloc_scratch(void** out);  // the static scratch of this device (defined below)
 thread_local char t_error[512];
 thread_local char t_kernels[512];
 thread_local int t_path = AVQ_PATH_AUTO;
@@ -325,8 +326,20 @@ avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, c
   AVQ_REQUIRE_PTR(assign, "assign");
   AVQ_REQUIRE_PTR(vsum, "vsum");
   AVQ_REQUIRE_PTR(counts, "counts");
-  if (t_path == AVQ_PATH_TC) return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core kernel for a depth-3 tree");
+  // tensor-core path: the two-level warpgroup assignment (its codebook image
+  // in the library's static scratch), then the grandchild refinement on the
+  // CUDA cores; the counts of all three levels from the value-sum passes
+  const bool tc_ok = s.C == 8 && assign_tc_supported(s, dtype) && assign_tc_uses_warpgroups(s) &&
+                     assign_tc_workspace(s) <= AVQ_NOALLOC_SCRATCH_BYTES;
+  if (t_path == AVQ_PATH_TC && !tc_ok)
+    return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core assignment for this depth-3 shape/dtype");
+  const bool use_tc = tc_ok && t_path != AVQ_PATH_SIMT;
   if (injected("quantize3")) return injected_fail("avq_quantize3");
+  void* scratch = nullptr;
+  if (use_tc) {
+    st = noalloc_scratch(&scratch);
+    if (st != AVQ_OK) return st;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const size_t mt3 = (size_t)s.M0 + (size_t)s.M0 * s.C + (size_t)s.M0 * s.C * s.C;
   LaunchLog log{};
@@ -334,9 +347,17 @@ avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, c
   if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
   cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)s.BH() * mt3 * sizeof(int32_t), cs);
   if (e != cudaSuccess) return cuda_fail(e, "zero counts");
-  e = launch_assign3_simt(s, dtype, K, parents, children, grandchildren, assign, counts, cs, log);
+  bool count_in_sums = false;
+  if (use_tc) {
+    e = launch_assign_tc(s, K, parents, children, assign, counts, scratch, err, cs, log, nullptr,
+                         &count_in_sums);
+    if (e == cudaSuccess && !count_in_sums) e = cudaErrorInvalidValue;  // the warpgroup kernel must leave the counts
+    if (e == cudaSuccess) e = launch_assign3_grandchildren(s, K, children, grandchildren, assign, cs, log);
+  } else {
+    e = launch_assign3_simt(s, dtype, K, parents, children, grandchildren, assign, counts, cs, log);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "assignment launch");
-  e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, false, true);
+  e = launch_aggregate(s, dtype, V, assign, vsum, counts, err, cs, log, false, true, count_in_sums);
   if (e != cudaSuccess) return cuda_fail(e, "aggregation launch");
   snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
   return AVQ_OK;

@@ -21,6 +21,7 @@
 // are refined with their grandchildren: the child's logit is the mean of its
 // grandchildren's (Eq. 8), dA = exp(s_g - m) - exp(s_c - m) (Eq. 9), zero for
 // empty grandchildren, merged with the online maximum.
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -351,7 +352,105 @@ __global__ void __launch_bounds__(128) attention3_simt_kernel(
   }
 }
 
+// Stage 1 of a depth-3 tree after the two-level tensor-core assignment:
+// every key whose code is a child moves to that child's nearest grandchild
+// when it is strictly closer (Algorithm 1, one level down; C = 8).  8 lanes
+// per key, 4 keys per warp: lane s holds 16-byte chunks of the key, its child
+// and the child's grandchildren (dims [s D/8, (s+1) D/8)), accumulates the 9
+// partial dot products and squared norms in fp32 (bf16 x bf16 products) and
+// sums them over the 8 lanes; distances |r|^2 - 2 k.r (|k|^2 is common), the
+// first strict minimum among the grandchildren, moved only if strictly
+// closer than the child.  Keys at a parent are left as they are.
+template <int D>
+__global__ void __launch_bounds__(256) assign3_grandchildren_kernel(const bf16* __restrict__ K,
+                                                                    const bf16* __restrict__ children,
+                                                                    const bf16* __restrict__ grandchildren,
+                                                                    int32_t* __restrict__ assign, int BH,
+                                                                    int H, int N, int M0) {
+  constexpr int C = 8;
+  constexpr int DL = D / 8;    // dims per lane
+  constexpr int CHK = DL / 8;  // 16-byte chunks per lane and row
+  const int M1 = M0 * C;
+  const int lane = threadIdx.x & 31, sub = lane & 7, kq = lane >> 3;
+  const long long total = (long long)BH * N;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long k0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4; k0 < total;
+       k0 += warps * 4) {  // warp-uniform loop
+    const long long key = k0 + kq;
+    const int code = key < total ? assign[key] : -1;
+    const bool moved = code >= M0 && code < M0 + M1;
+    if (!__any_sync(0xffffffffu, moved)) continue;
+    const int cl = moved ? code - M0 : 0;  // the child's index among the head's M0*C children
+    const int h = (int)((moved ? key / N : 0) % H);
+    const bf16* kr = K + (size_t)(moved ? key : 0) * D + sub * DL;
+    const bf16* cr = children + ((size_t)h * M1 + cl) * D + sub * DL;
+    const bf16* gr = grandchildren + ((size_t)h * M1 + cl) * C * D + sub * DL;
+    float acc[1 + C], nrm[1 + C];
+#pragma unroll
+    for (int j = 0; j <= C; ++j) acc[j] = nrm[j] = 0.f;
+    if (moved) {
+#pragma unroll
+      for (int q = 0; q < CHK; ++q) {
+        const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + q * 8));
+        uint4 cv[1 + C];
+        cv[0] = __ldg(reinterpret_cast<const uint4*>(cr + q * 8));
+#pragma unroll
+        for (int g = 0; g < C; ++g) cv[1 + g] = __ldg(reinterpret_cast<const uint4*>(gr + (size_t)g * D + q * 8));
+#pragma unroll
+        for (int j = 0; j <= C; ++j) {
+          acc[j] = fma_bf16x2(kv.x, cv[j].x, acc[j]);
+          acc[j] = fma_bf16x2(kv.y, cv[j].y, acc[j]);
+          acc[j] = fma_bf16x2(kv.z, cv[j].z, acc[j]);
+          acc[j] = fma_bf16x2(kv.w, cv[j].w, acc[j]);
+          nrm[j] = fma_bf16x2(cv[j].x, cv[j].x, nrm[j]);
+          nrm[j] = fma_bf16x2(cv[j].y, cv[j].y, nrm[j]);
+          nrm[j] = fma_bf16x2(cv[j].z, cv[j].z, nrm[j]);
+          nrm[j] = fma_bf16x2(cv[j].w, cv[j].w, nrm[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+      for (int j = 0; j <= C; ++j) {
+        acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        nrm[j] += __shfl_xor_sync(0xffffffffu, nrm[j], o);
+      }
+    if (moved && sub == 0) {
+      const float dc = fmaf(-2.f, acc[0], nrm[0]);
+      float dg = fmaf(-2.f, acc[1], nrm[1]);
+      int gstar = 0;
+#pragma unroll
+      for (int g = 1; g < C; ++g) {
+        const float d = fmaf(-2.f, acc[1 + g], nrm[1 + g]);
+        if (d < dg) {
+          dg = d;
+          gstar = g;
+        }
+      }
+      if (dg < dc) assign[key] = M0 + M1 + cl * C + gstar;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_assign3_grandchildren(const Shape& s, const void* K, const void* children,
+                                         const void* grandchildren, int32_t* assign, cudaStream_t st,
+                                         LaunchLog& log) {
+  const long long groups = ((long long)s.BH() * s.N + 3) / 4;  // 4 keys per warp
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((groups + 7) / 8, (long long)num_sms() * 16));
+  if (s.d == 64)
+    assign3_grandchildren_kernel<64><<<blocks, 256, 0, st>>>((const bf16*)K, (const bf16*)children,
+                                                             (const bf16*)grandchildren, assign, s.BH(), s.H,
+                                                             s.N, s.M0);
+  else
+    assign3_grandchildren_kernel<128><<<blocks, 256, 0, st>>>((const bf16*)K, (const bf16*)children,
+                                                              (const bf16*)grandchildren, assign, s.BH(), s.H,
+                                                              s.N, s.M0);
+  log.add("assign3_grandchildren");
+  return cudaGetLastError();
+}
 
 cudaError_t launch_assign3_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
                                 const void* children, const void* grandchildren, int32_t* assign,

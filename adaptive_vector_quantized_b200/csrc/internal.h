@@ -43,6 +43,12 @@ cudaError_t launch_aggregate(const Shape& s, avq_dtype dt, const void* V, const 
 // Depth-3 tree (three levels, codes parents | M0*C children | M0*C*C
 // grandchildren): assignment one level deeper on the CUDA cores; counts are
 // added into counts[BH][Mt3], which the caller zeroes first.
+// Depth-3 stage 1 after the two-level tensor-core assignment (bf16, C = 8,
+// d in {64, 128}): keys at a child move to its nearest grandchild when
+// strictly closer; assign[] is rewritten in place (no counts).
+cudaError_t launch_assign3_grandchildren(const Shape& s, const void* K, const void* children,
+                                         const void* grandchildren, int32_t* assign, cudaStream_t st,
+                                         LaunchLog& log);
 cudaError_t launch_assign3_simt(const Shape& s, avq_dtype dt, const void* K, const void* parents,
                                 const void* children, const void* grandchildren, int32_t* assign,
                                 int32_t* counts, cudaStream_t st, LaunchLog& log);
@@ -63,6 +69,9 @@ cudaError_t launch_aggregate_det(const Shape& s, avq_dtype dt, const void* V,
 // C in {0, 8}); needs assign_tc_workspace(s) bytes of workspace.
 bool assign_tc_supported(const Shape& s, avq_dtype dt);
 size_t assign_tc_workspace(const Shape& s);
+// True when launch_assign_tc takes the warpgroup kernel for this shape (the
+// whole two-level codebook image in shared memory).
+bool assign_tc_uses_warpgroups(const Shape& s);
 // Zeroes counts itself (and vsum when vsum_to_zero is given) before the
 // assignment adds into them.  With counts_left given, the warpgroup kernel
 // may leave the counts to the streaming value sums: *counts_left tells the

@@ -211,8 +211,15 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q,
  *                              its subtree that reached it
  *   counts [B,H,Mt3]    int32  key counts with the same membership
  * Inputs (device): K, V [B,H,N,d]; parents [H,M0,d]; children [H,M0,C,d];
- * grandchildren [H,M0,C,C,d], all of `dtype`; 1 <= C <= 8.  CUDA-core kernels
- * (AVQ_ERR_UNSUPPORTED under AVQ_PATH_TC); no workspace.
+ * grandchildren [H,M0,C,C,d], all of `dtype`; 1 <= C <= 8.  No workspace.
+ * Kernels: for bf16 with C == 8 and a two-level codebook image that fits one
+ * CTA's shared memory (M0 <= 64), the parent and child decisions run on the
+ * tensor cores as in avq_quantize, their codebook image in the static scratch
+ * array of avq_quantize_noalloc (same set-up and race rules: calls whose
+ * executions may overlap on one device must not share it), and a CUDA-core
+ * pass refines the keys at a child with its grandchildren; otherwise (and
+ * under AVQ_PATH_SIMT) one CUDA-core kernel takes all three decisions.
+ * AVQ_PATH_TC on a shape without the tensor-core route: AVQ_ERR_UNSUPPORTED.
  */
 avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, const void* V,
                          const void* parents, const void* children, const void* grandchildren,

@@ -36,11 +36,22 @@ CASES = {
 }
 
 
-def run_gpu3(inp, P=None, P2=None):
+def tc_route(inp):
+    """Shapes whose stage 1 takes the tensor-core route by default: bf16,
+    C = 8, the two-level codebook image within one CTA's shared memory."""
+    return inp["dtype"] == "bf16" and inp["C"] == 8 and inp["M0"] <= 64
+
+
+def run_gpu3(inp, P=None, P2=None, path=None):
     P = inp["P"] if P is None else P
     P2 = inp["P2"] if P2 is None else P2
     d = {k: inp[k].cuda().contiguous() for k in ("Q", "K", "V", "parents", "children", "grandchildren")}
-    assign, vsum, counts = avq.avq_quantize3(d["K"], d["V"], d["parents"], d["children"], d["grandchildren"])
+    old = avq.avq_set_path(avq.AVQ_PATH_AUTO if path is None else path)
+    try:
+        assign, vsum, counts = avq.avq_quantize3(d["K"], d["V"], d["parents"], d["children"],
+                                                 d["grandchildren"])
+    finally:
+        avq.avq_set_path(old)
     k1 = avq.last_kernels()
     O, sel, sel2, imp, imp2 = avq.avq_attention3(d["Q"], d["parents"], d["children"], d["grandchildren"],
                                                  vsum, counts, P, P2, inp["block"], inp["scale"],
@@ -92,12 +103,21 @@ def check3(inp, res, P=None, P2=None):
     return dict(near_tie_keys=ties, O_rel_err=err)
 
 
+@pytest.mark.parametrize("route", ["auto", "simt"])
 @pytest.mark.parametrize("case", list(CASES))
-def test_depth3_parity(case):
+def test_depth3_parity(case, route):
     cfg, seed = CASES[case]
     inp = synth.make_inputs3(cfg, seed)
-    res = run_gpu3(inp)
-    assert "assign3_simt" in res["kernels"] and "attention3_simt" in res["kernels"]
+    if route == "simt":
+        res = run_gpu3(inp, path=avq.AVQ_PATH_SIMT)
+        assert "assign3_simt" in res["kernels"]
+    else:
+        res = run_gpu3(inp)
+        if tc_route(inp):
+            assert "assign_tc_wg" in res["kernels"] and "assign3_grandchildren" in res["kernels"]
+        else:
+            assert "assign3_simt" in res["kernels"]
+    assert "attention3_simt" in res["kernels"]
     M0, C = inp["M0"], inp["C"]
     a = res["assign"]
     if case != "c1":
@@ -105,12 +125,15 @@ def test_depth3_parity(case):
     print(case, res["kernels"], check3(inp, res))
 
 
-def test_depth3_workload_sampled_invariants():
+@pytest.mark.parametrize("route", ["auto", "simt"])
+def test_depth3_workload_sampled_invariants(route):
     """The bench's depth-3 workload (B=1, H=8, N=16384, 64/16/16, C=8): full
-    parity on two heads, invariants on all."""
+    parity on two heads, invariants on all; the default (tensor-core) stage 1
+    and the CUDA-core one."""
     cfg = synth.get_config("deep3")
     inp = synth.make_inputs3(cfg, synth.CONFIG_SEEDS["deep3"])
-    res = run_gpu3(inp)
+    res = run_gpu3(inp, path=avq.AVQ_PATH_SIMT if route == "simt" else None)
+    assert ("assign_tc_wg" in res["kernels"]) == (route == "auto")
     N, M0, C = inp["N"], inp["M0"], inp["C"]
     M1 = M0 * C
     n = res["counts"]
@@ -150,3 +173,19 @@ def test_depth3_equals_depth2_when_p2_is_zero():
     assert np.array_equal(sel2d.cpu().numpy(), res["sel"])
     diff = (O2.cpu().float() - res["O"].float()).abs().max().item()
     assert diff <= 2e-2 * float(inp["V"].float().abs().max())
+
+
+def test_depth3_tc_route_refusals():
+    """Forcing the tensor-core route on a depth-3 shape it does not cover
+    (f32, or C != 8) is refused before any launch."""
+    for name in ("f32_d128_b64", "all_children"):
+        cfg, seed = CASES[name]
+        inp = synth.make_inputs3(cfg, seed)
+        d = {k: inp[k].cuda().contiguous() for k in ("K", "V", "parents", "children", "grandchildren")}
+        old = avq.avq_set_path(avq.AVQ_PATH_TC)
+        try:
+            with pytest.raises(RuntimeError):
+                avq.avq_quantize3(d["K"], d["V"], d["parents"], d["children"], d["grandchildren"])
+        finally:
+            avq.avq_set_path(old)
+    avq.avq_check_device()
