@@ -859,22 +859,25 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attention_fast_kernel(
       const float4* nf4 = reinterpret_cast<const float4*>(sNF);
       float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-      for (int c0 = 0; c0 < M0; c0 += 32) {
+      for (int c0 = 0; c0 < M0; c0 += 32) {  // columns c0 .. min(c0 + 32, M0) - 1
         constexpr int W = M0 < 32 ? M0 : 32;
         uint32_t r[W];
 #pragma unroll
-        for (int g = 0; g < W / 16; ++g) tc::tmem_ld16(tS + lane_off + c0 + g * 16, r + g * 16);
+        for (int g = 0; g < W / 16; ++g)
+          if (c0 + g * 16 < M0) tc::tmem_ld16(tS + lane_off + c0 + g * 16, r + g * 16);
         tc::tmem_wait_ld();
         const float* t = reinterpret_cast<const float*>(r);
         if (!any_empty) {
 #pragma unroll
           for (int e = 0; e < W; e += 4) {
+            if (c0 + e >= M0) break;
             mx0 = fm::max3(mx0, t[e], t[e + 1]);
             mx1 = fm::max3(mx1, t[e + 2], t[e + 3]);
           }
         } else {
 #pragma unroll
           for (int e = 0; e < W; e += 4) {
+            if (c0 + e >= M0) break;
             const float4 nf = nf4[(c0 + e) >> 2];
             mx0 = fm::max3(mx0, nf.x > 0.f ? t[e] : NEG_INF, nf.y > 0.f ? t[e + 1] : NEG_INF);
             mx1 = fm::max3(mx1, nf.z > 0.f ? t[e + 2] : NEG_INF, nf.w > 0.f ? t[e + 3] : NEG_INF);

@@ -392,12 +392,22 @@ avq_status avq_attention3(const avq_dims* dims, avq_dtype dtype, const void* Q, 
     return fail(AVQ_ERR_INVALID_ARG, "importance is not 16-byte aligned");
   if (importance2 != nullptr && !aligned(importance2, 16))
     return fail(AVQ_ERR_INVALID_ARG, "importance2 is not 16-byte aligned");
-  if (t_path == AVQ_PATH_TC) return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core kernel for a depth-3 tree");
+  const bool tc_ok = attention3_tc_supported(s, dtype, P, P2, block);
+  if (t_path == AVQ_PATH_TC && !tc_ok)
+    return fail(AVQ_ERR_UNSUPPORTED, "no tensor-core depth-3 attention for this shape/dtype/P/P2/block");
   if (injected("attention3")) return injected_fail("avq_attention3");
   LaunchLog log{};
-  cudaError_t e = launch_attention3_simt(s, dtype, Q, parents, children, grandchildren, vsum, counts, P, P2,
-                                         block, scale, O, sel, sel2, importance, importance2,
-                                         reinterpret_cast<cudaStream_t>(stream), log);
+  cudaError_t e;
+  if (tc_ok && t_path != AVQ_PATH_SIMT) {
+    unsigned int* err = error_word();
+    if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
+    e = launch_attention3_tc(s, Q, parents, children, grandchildren, vsum, counts, P, P2, scale, O, sel, sel2,
+                             importance, importance2, err, reinterpret_cast<cudaStream_t>(stream), log);
+  } else {
+    e = launch_attention3_simt(s, dtype, Q, parents, children, grandchildren, vsum, counts, P, P2, block,
+                               scale, O, sel, sel2, importance, importance2,
+                               reinterpret_cast<cudaStream_t>(stream), log);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   snprintf(t_kernels, sizeof(t_kernels), "%s", log.text);
   return AVQ_OK;

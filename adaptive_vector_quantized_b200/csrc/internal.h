@@ -54,6 +54,13 @@ cudaError_t launch_assign3_simt(const Shape& s, avq_dtype dt, const void* K, con
                                 int32_t* counts, cudaStream_t st, LaunchLog& log);
 // Depth-3 attention on the CUDA cores: parents, the top-P parents' children,
 // the top-P2 refined children's grandchildren.
+// Depth-3 attention on the tensor cores: bf16, block 128, d 64 or 128, C 8,
+// M0 in {16, 32, 48, 64}, P and P2 at most 16.
+bool attention3_tc_supported(const Shape& s, avq_dtype dt, int P, int P2, int block);
+cudaError_t launch_attention3_tc(const Shape& s, const void* Q, const void* parents, const void* children,
+                                 const void* grandchildren, const float* vsum, const int32_t* counts, int P,
+                                 int P2, float scale, void* O, int32_t* sel, int32_t* sel2, float* importance,
+                                 float* importance2, unsigned int* err, cudaStream_t st, LaunchLog& log);
 cudaError_t launch_attention3_simt(const Shape& s, avq_dtype dt, const void* Q, const void* parents,
                                    const void* children, const void* grandchildren, const float* vsum,
                                    const int32_t* counts, int P, int P2, int block, float scale, void* O,

@@ -230,9 +230,10 @@ def test_depth3_host_checks():
     assert a3(4, 4, sel2=None) == avq.AVQ_ERR_INVALID_ARG and "sel2" in avq.last_error()
     old = avq.avq_set_path(avq.AVQ_PATH_TC)
     try:
-        # no tensor-core attention over a depth-3 tree; the tensor-core
-        # assignment only with C == 8 (and bf16)
-        assert a3(4, 4) == avq.AVQ_ERR_UNSUPPORTED
+        # the tensor-core kernels: attention with block 128 and P, P2 <= 16;
+        # the assignment with C == 8 and bf16
+        assert a3(4, 4, block=64) == avq.AVQ_ERR_UNSUPPORTED
+        assert a3(4, 20) == avq.AVQ_ERR_UNSUPPORTED
         assert q3(avq.avq_dims(1, 2, 256, 64, 16, 4)) == avq.AVQ_ERR_UNSUPPORTED
         assert L.avq_quantize3(ctypes.byref(d), avq.AVQ_F32, fake, fake, fake, fake, fake, fake, fake, fake,
                                None) == avq.AVQ_ERR_UNSUPPORTED

@@ -33,6 +33,10 @@ CASES = {
     "p_zero": (_cfg(N=512, P=0, P2=0), 65),
     "c1": (_cfg(N=300, C=1, P=4, P2=2), 66),
     "all_children": (_cfg(N=400, M0=4, C=3, P=4, P2=12), 67),
+    "bf16_d128": (_cfg(N=900, d=128, M0=32, P=6, P2=7), 68),
+    "bf16_m48_full": (_cfg(N=700, M0=48, P=16, P2=16), 69),
+    "bf16_p20": (_cfg(N=600, M0=32, P=20, P2=4), 70),
+    "bf16_b64": (_cfg(N=500, block=64), 71),
 }
 
 
@@ -40,6 +44,12 @@ def tc_route(inp):
     """Shapes whose stage 1 takes the tensor-core route by default: bf16,
     C = 8, the two-level codebook image within one CTA's shared memory."""
     return inp["dtype"] == "bf16" and inp["C"] == 8 and inp["M0"] <= 64
+
+
+def tc_route2(inp, P, P2):
+    """Shapes whose depth-3 attention takes the tensor-core kernel by default."""
+    return (inp["dtype"] == "bf16" and inp["C"] == 8 and inp["block"] == 128 and inp["M0"] % 16 == 0
+            and inp["M0"] <= 64 and P <= 16 and P2 <= 16)
 
 
 def run_gpu3(inp, P=None, P2=None, path=None):
@@ -50,13 +60,13 @@ def run_gpu3(inp, P=None, P2=None, path=None):
     try:
         assign, vsum, counts = avq.avq_quantize3(d["K"], d["V"], d["parents"], d["children"],
                                                  d["grandchildren"])
+        k1 = avq.last_kernels()
+        O, sel, sel2, imp, imp2 = avq.avq_attention3(d["Q"], d["parents"], d["children"], d["grandchildren"],
+                                                     vsum, counts, P, P2, inp["block"], inp["scale"],
+                                                     importance=True)
+        k2 = avq.last_kernels()
     finally:
         avq.avq_set_path(old)
-    k1 = avq.last_kernels()
-    O, sel, sel2, imp, imp2 = avq.avq_attention3(d["Q"], d["parents"], d["children"], d["grandchildren"],
-                                                 vsum, counts, P, P2, inp["block"], inp["scale"],
-                                                 importance=True)
-    k2 = avq.last_kernels()
     avq.avq_check_device()
     torch.cuda.synchronize()
     return dict(assign=assign.cpu().numpy(), vsum=vsum.cpu().numpy(), counts=counts.cpu().numpy(),
@@ -110,14 +120,15 @@ def test_depth3_parity(case, route):
     inp = synth.make_inputs3(cfg, seed)
     if route == "simt":
         res = run_gpu3(inp, path=avq.AVQ_PATH_SIMT)
-        assert "assign3_simt" in res["kernels"]
+        assert "assign3_simt" in res["kernels"] and "attention3_simt" in res["kernels"]
     else:
         res = run_gpu3(inp)
         if tc_route(inp):
             assert "assign_tc_wg" in res["kernels"] and "assign3_grandchildren" in res["kernels"]
         else:
             assert "assign3_simt" in res["kernels"]
-    assert "attention3_simt" in res["kernels"]
+        want = "attention3_tc" if tc_route2(inp, inp["P"], inp["P2"]) else "attention3_simt"
+        assert want in res["kernels"], res["kernels"]
     M0, C = inp["M0"], inp["C"]
     a = res["assign"]
     if case != "c1":
@@ -134,6 +145,7 @@ def test_depth3_workload_sampled_invariants(route):
     inp = synth.make_inputs3(cfg, synth.CONFIG_SEEDS["deep3"])
     res = run_gpu3(inp, path=avq.AVQ_PATH_SIMT if route == "simt" else None)
     assert ("assign_tc_wg" in res["kernels"]) == (route == "auto")
+    assert ("attention3_tc" in res["kernels"]) == (route == "auto")
     N, M0, C = inp["N"], inp["M0"], inp["C"]
     M1 = M0 * C
     n = res["counts"]
