@@ -426,9 +426,10 @@ def run_avq(args, cfg, inp, n_global=None):
     # kernel of the step in the ncu launch list (the stage-2 time also holds its
     # 1% image-preparation kernel).  Stage 1 is reported under "stages".
     achieved = alg["s2_bytes"] / (t_s2 * 1e-3) / 1e9
+    att = "attention3_tc" if depth3 else "attention_tc"
     roofline = dict(bound="hbm", achieved=achieved, peak=peaks["hbm"], unit="GB/s",
-                    frac=achieved / peaks["hbm"], traffic=traffic_for("attention_tc.cu", args.config),
-                    kernel="attention_tc", peak_source=peaks["source"],
+                    frac=achieved / peaks["hbm"], traffic=traffic_for(att + ".cu", args.config),
+                    kernel=att, peak_source=peaks["source"],
                     step_roofline_us=t_roof * 1e6, step_frac=t_roof * 1e3 / ms_step)
     cpu = None
     if not args.no_cpu_baseline and not args.profile and world == 1 and not depth3:  # rank 0 at N=1 only
