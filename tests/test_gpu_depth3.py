@@ -37,6 +37,10 @@ CASES = {
     "bf16_m48_full": (_cfg(N=700, M0=48, P=16, P2=16), 69),
     "bf16_p20": (_cfg(N=600, M0=32, P=20, P2=4), 70),
     "bf16_b64": (_cfg(N=500, block=64), 71),
+    "bf16_b2": (_cfg(B=2, N=300, M0=32, P=5, P2=9), 72),
+    "bf16_p1": (_cfg(N=400, P=1, P2=1), 73),
+    "bf16_p2_all": (_cfg(N=500, M0=16, P=2, P2=16), 74),
+    "bf16_sparse": (_cfg(N=40, M0=64, P=16, P2=16), 75),
 }
 
 
@@ -131,8 +135,10 @@ def test_depth3_parity(case, route):
         assert want in res["kernels"], res["kernels"]
     M0, C = inp["M0"], inp["C"]
     a = res["assign"]
-    if case != "c1":
+    if case not in ("c1", "bf16_sparse"):
         assert (a >= M0 + M0 * C).any() and (a < M0).any()  # every level is reached
+    if case == "bf16_sparse":  # most parents and children hold no key
+        assert (res["counts"][..., :M0] == 0).sum() > M0 // 2
     print(case, res["kernels"], check3(inp, res))
 
 
