@@ -242,7 +242,13 @@ avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, c
  * descending child importance; importance [B,H,nblk,M0] (nullable);
  * importance2 [B,H,nblk,P*C] (nullable), the refined children in the order of
  * sel, C each.  0 <= P <= M0, 0 <= P2 <= P*C, block 64 or 128; vsum and
- * counts as avq_quantize3 writes them.  CUDA-core kernel; no workspace.
+ * counts as avq_quantize3 writes them.  No workspace.
+ * Kernels: for bf16, block 128, C == 8, M0 in {16, 32, 48, 64}, d 64 or 128
+ * and P, P2 <= 16, one tensor-core kernel (a CTA per query block; the
+ * codeword rows and the value sums, rounded to bf16, are read straight from
+ * the arguments, so nothing is prepared); otherwise (and under
+ * AVQ_PATH_SIMT) a CUDA-core kernel.  AVQ_PATH_TC on another shape:
+ * AVQ_ERR_UNSUPPORTED.
  */
 avq_status avq_attention3(const avq_dims* dims, avq_dtype dtype, const void* Q, const void* parents,
                           const void* children, const void* grandchildren, const float* vsum,
