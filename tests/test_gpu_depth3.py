@@ -207,3 +207,38 @@ def test_depth3_tc_route_refusals():
         finally:
             avq.avq_set_path(old)
     avq.avq_check_device()
+
+
+def test_depth3_tc_rescale_paths():
+    """Children far above the parents' maximum and grandchildren far above the
+    children's (logit gaps up to 64 against the reference-maximum margin of
+    2^24): the tensor-core kernel's rescale branch at both levels, against
+    the oracle."""
+    H, M0, C, d, N = 1, 16, 8, 64, 512
+    rng = np.random.default_rng(7)
+    par = np.zeros((H, M0, d), dtype=np.float32)
+    par[0, :, 2:] = np.rint(rng.standard_normal((M0, d - 2)) * 8) / 8
+    steps = [4, -4, 3, -3, 2, -2, 1, -1]
+    offc = np.zeros((C, d), dtype=np.float32)
+    offc[:, 0] = steps
+    ch = par[:, :, None, :] + offc[None, None]
+    offg = np.zeros((C, d), dtype=np.float32)
+    offg[:, 1] = steps
+    gc = ch[:, :, :, None, :] + offg[None, None, None]
+    assert np.array_equal(ch.mean(2), par) and np.array_equal(gc.mean(3), ch)
+    pick_p = rng.integers(0, M0, N)
+    pick_c = rng.integers(0, 2, N) * 2  # children 0 or 2: far along +e0
+    pick_g = rng.integers(0, 2, N) * 2  # grandchildren 0 or 2: far along +e1
+    K = gc[0][pick_p, pick_c, pick_g][None, None]
+    Q = np.zeros((1, H, N, d), dtype=np.float32)
+    Q[..., 0] = 16.0
+    Q[..., 1] = 16.0
+    Q[..., 2:] = np.rint(rng.standard_normal((N, d - 2)) * 4) / 16
+    V = rng.standard_normal((1, H, N, d)).astype(np.float32)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)  # noqa: E731
+    inp = dict(Q=t(Q), K=t(K), V=t(V), parents=t(par), children=t(ch), grandchildren=t(gc), B=1, H=H, N=N,
+               d=d, M0=M0, C=C, P=4, P2=6, block=128, scale=1.0, dtype="bf16", depth=3)
+    res = run_gpu3(inp)
+    assert "attention3_tc" in res["kernels"]
+    assert (res["assign"] >= M0 + M0 * C).all()  # every key at a grandchild
+    print("rescale3", res["kernels"], check3(inp, res))
