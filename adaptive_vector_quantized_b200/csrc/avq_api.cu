@@ -70,8 +70,10 @@ avq_status check_dims(const avq_dims* d, avq_dtype dt) {
   if (d->M0 < 1 || d->M0 > 256) return fail(AVQ_ERR_UNSUPPORTED, "M0 must be in [1, 256] (got %d)", d->M0);
   if (d->C < 0 || d->C > 8) return fail(AVQ_ERR_UNSUPPORTED, "C must be in [0, 8] (got %d)", d->C);
   const long long rows = (long long)d->B * d->H * d->N;
-  if (rows > (1ll << 31) - 1 || (long long)d->B * d->H > 65535 * 64)
+  if (rows > (1ll << 31) - 1)
     return fail(AVQ_ERR_UNSUPPORTED, "B*H*N = %lld exceeds the supported range", rows);
+  if ((long long)d->B * d->H > 65535)  // several kernels take one grid row per (batch, head)
+    return fail(AVQ_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", (long long)d->B * d->H);
   return AVQ_OK;
 }
 

@@ -65,7 +65,8 @@ typedef enum {
 typedef enum { AVQ_F32 = 0, AVQ_BF16 = 1 } avq_dtype;
 
 /* Problem shape of one attention layer.  Supported: B, H >= 1; N >= 1;
- * d in {64, 128}; 1 <= M0 <= 256; 0 <= C <= 8. */
+ * d in {64, 128}; 1 <= M0 <= 256; 0 <= C <= 8; B*H <= 65535 (one grid row
+ * per head) and B*H*N < 2^31.  Outside: AVQ_ERR_UNSUPPORTED. */
 typedef struct {
   int B, H, N, d, M0, C;
 } avq_dims;

@@ -71,6 +71,9 @@ def test_host_validation_rejects_before_launch():
     assert _q(avq.avq_dims(1, 2, 64, 96, 16, 4)) == E.AVQ_ERR_UNSUPPORTED
     assert _q(avq.avq_dims(1, 2, 64, 64, 300, 4)) == E.AVQ_ERR_UNSUPPORTED
     assert _q(avq.avq_dims(1, 2, 64, 64, 16, 9)) == E.AVQ_ERR_UNSUPPORTED
+    assert _q(avq.avq_dims(2, 32768, 1, 64, 16, 4)) == E.AVQ_ERR_UNSUPPORTED  # B*H above 65535
+    assert "65535" in avq.last_error()
+    assert _q(avq.avq_dims(1, 1024, 1 << 21, 64, 16, 4)) == E.AVQ_ERR_UNSUPPORTED  # B*H*N >= 2^31
     assert _q(ok, K=None) == E.AVQ_ERR_INVALID_ARG
     assert "K is NULL" in avq.last_error()
     assert _q(ok, V=0x2004) == E.AVQ_ERR_INVALID_ARG
