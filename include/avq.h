@@ -218,8 +218,9 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q,
  * tensor cores as in avq_quantize, their codebook image in the static scratch
  * array of avq_quantize_noalloc (same set-up and race rules: calls whose
  * executions may overlap on one device must not share it), and a CUDA-core
- * pass refines the keys at a child with its grandchildren; otherwise (and
- * under AVQ_PATH_SIMT) one CUDA-core kernel takes all three decisions.
+ * pass refines the keys at a child with its grandchildren; otherwise (also
+ * when the image does not fit that array, and under AVQ_PATH_SIMT) one
+ * CUDA-core kernel takes all three decisions.
  * AVQ_PATH_TC on a shape without the tensor-core route: AVQ_ERR_UNSUPPORTED.
  */
 avq_status avq_quantize3(const avq_dims* dims, avq_dtype dtype, const void* K, const void* V,
