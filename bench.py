@@ -56,6 +56,9 @@ def parse():
                          "(default: the workload's own setting)")
     ap.add_argument("--profile", action="store_true",
                     help="for profiler runs: no clock soak, no end-to-end leg, no CPU baseline")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture each stage's library call once as a CUDA graph and replay the graphs "
+                         "in the timed steps (the same kernels without the host's per-call launch work)")
     return ap.parse_args()
 
 
@@ -303,19 +306,19 @@ def run_avq(args, cfg, inp, n_global=None):
 
     exchange = n_global is not None and world > 1
 
-    def quantize(Kb, Vb):
+    def quantize(Kb, Vb, st=stream):
         if depth3:
-            avq.avq_quantize3(Kb, Vb, par, ch, gch, assign, vsum, counts, stream=stream)
+            avq.avq_quantize3(Kb, Vb, par, ch, gch, assign, vsum, counts, stream=st)
         else:
-            avq.avq_quantize(Kb, Vb, par, ch, assign, vsum, counts, ws=ws, stream=stream)
+            avq.avq_quantize(Kb, Vb, par, ch, assign, vsum, counts, ws=ws, stream=st)
 
-    def attend(Qb, Ob, selb):
+    def attend(Qb, Ob, selb, st=stream):
         """Stage 2; returns the parent selection it wrote."""
         if depth3:
             return avq.avq_attention3(Qb, par, ch, gch, vsum, counts, P, cfg.get("P2", P), block, inp["scale"],
-                                      O=Ob, stream=stream)[1]
+                                      O=Ob, stream=st)[1]
         avq.avq_attention(Qb, par, ch, vsum, counts, P, block, inp["scale"], two_pass, Ob, selb,
-                          ws=ws, stream=stream)
+                          ws=ws, stream=st)
         return selb
 
     last_sel = [sel]
@@ -350,6 +353,24 @@ def run_avq(args, cfg, inp, n_global=None):
             soak += 1
             if soak % 32 == 0:
                 torch.cuda.synchronize(dev)
+        # --graph: each stage's call captured once (on a side stream, as graph
+        # capture requires) and replayed on the timing stream
+        gq = ga = None
+        if args.graph:
+            if exchange:
+                raise SystemExit("--graph is not offered with the token-sharded statistics exchange")
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(stream)
+            gq, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gq, stream=cap, capture_error_mode="relaxed"):
+                quantize(K, V, st=cap)
+            with torch.cuda.graph(ga, stream=cap, capture_error_mode="relaxed"):
+                attend(Q, O, sel, st=cap)
+            stream.wait_stream(cap)
+            for _ in range(3):
+                gq.replay()
+                ga.replay()
+            avq.avq_check_device(stream)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
@@ -358,11 +379,17 @@ def run_avq(args, cfg, inp, n_global=None):
             if fbuf is not None:  # inputs fit in L2: evict them before every timed step
                 fbuf.zero_()
             ev[s][0].record(stream)
-            quantize(K, V)
+            if gq is not None:
+                gq.replay()
+            else:
+                quantize(K, V)
             if exchange:
                 allreduce_stats(vsum, counts)
             ev[s][1].record(stream)
-            attend(Q, O, sel)
+            if ga is not None:
+                ga.replay()
+            else:
+                attend(Q, O, sel)
             ev[s][2].record(stream)
         t1.record(stream)
         torch.cuda.synchronize(dev)
@@ -479,7 +506,8 @@ def run_avq(args, cfg, inp, n_global=None):
                 scaling="weak" if n_global is None else "strong",
                 vs_baseline=None, dtype=cfg["dtype"], data="synthetic",
                 config=dict(workload_config(args.config, cfg),
-                            l2=l2_note),
+                            l2=l2_note, **({"launch": "CUDA graph replay of each stage's call"}
+                                           if args.graph else {})),
                 roofline=roofline, cpu_baseline=cpu, e2e=e2e,
                 gpu_launches=kernels_per_step * args.steps,
                 clocks=dict(clk.summary() or {}, window=f"sampled every 200 ms over warmup, "
