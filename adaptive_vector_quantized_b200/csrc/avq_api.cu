@@ -301,7 +301,12 @@ avq_status avq_attention(const avq_dims* dims, avq_dtype dtype, const void* Q, c
     if (st != AVQ_OK) return st;
     unsigned int* err = error_word();
     if (err == nullptr) return fail(AVQ_ERR_CUDA, "cannot resolve the device error word");
-    e = launch_attention_tc(s, Q, parents, children, vsum, counts, P, block, scale, two_pass, O,
+    // with no selection and no importance output nothing depends on the
+    // importance denominator: one sweep over several parent tiles (online
+    // maximum); a single tile keeps the one-tile kernel
+    const bool one_sweep = two_pass == AVQ_DENOM_AUTO && P == 0 && importance == nullptr && s.M0 > 64;
+    const int sweep_mode = one_sweep ? AVQ_DENOM_EXTRAPOLATED : two_pass;
+    e = launch_attention_tc(s, Q, parents, children, vsum, counts, P, block, scale, sweep_mode, O,
                             sel, importance, ws, err, cs, log);
   } else {
     e = launch_attention_simt(s, dtype, Q, parents, children, vsum, counts, P, block, scale, O,

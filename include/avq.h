@@ -171,7 +171,9 @@ avq_status avq_quantize_noalloc(const avq_dims* dims, avq_dtype dtype,
  * two_pass selects how the importance denominator is formed when the parents
  * span several tiles of 64 codes (M0 > 64):
  *   AVQ_DENOM_AUTO (0): exact; one pass when the parents fit one tile, else
- *     the two-pass form below.
+ *     the two-pass form below; with P == 0 and importance == NULL (nothing
+ *     then depends on the denominator) one pass over the tiles with a
+ *     running maximum, whatever M0.
  *   AVQ_DENOM_TWO_PASS (1): exact two-pass denominator: a first pass over
  *     parent tiles finds the row max and z, a second recomputes the logits
  *     for x and the importance.  Results equal the single-pass ones.

@@ -364,3 +364,27 @@ def test_permute_refuses_out_of_range_indices():
 
 def test_device_error_word_clean():
     avq.avq_check_device()
+
+
+@pytest.mark.parametrize("M0,C", [(192, 0), (128, 8)])
+def test_p0_without_importance_one_sweep(M0, C):
+    """P = 0 and no importance output over several parent tiles: nothing
+    depends on the importance denominator, so the kernel takes one sweep with
+    a running maximum; O equals the oracle's (Eq. 4) and the two-sweep run's."""
+    inp = synth.make_inputs(_cfg(N=1000, M0=M0, C=C, P=0), 31)
+    d = gh.to_dev(inp)
+    ch = d["children"] if C > 0 else None
+    assign, vsum, counts = avq.avq_quantize(d["K"], d["V"], d["parents"], ch)
+    O1, _, _ = avq.avq_attention(d["Q"], d["parents"], ch, vsum, counts, 0, inp["block"], inp["scale"])
+    k = avq.last_kernels()
+    O2, _, _ = avq.avq_attention(d["Q"], d["parents"], ch, vsum, counts, 0, inp["block"], inp["scale"],
+                                 importance=True)
+    avq.avq_check_device()
+    torch.cuda.synchronize()
+    assert "attention_tc" in k
+    orc = oracle.default()
+    ref_vs, ref_n = orc.aggregate(assign.cpu().numpy(), inp["V"], M0, C)
+    O_ref, _, _ = orc.attention(inp["Q"], inp["parents"], inp["children"], ref_vs, ref_n, 0, inp["block"],
+                                inp["scale"])
+    parity.check_output(O1.cpu(), O_ref, inp["V"], inp["dtype"])
+    parity.check_output(O2.cpu(), O_ref, inp["V"], inp["dtype"])
